@@ -1,0 +1,264 @@
+"""Python binding of libgpt_b200.so (ctypes; argument marshalling only).
+
+Every function below forwards to the C entry point of the same name declared
+in include/gpt.h; every step of the training path runs in the library's CUDA
+kernels.  PyTorch is used only to own device memory (the model arena) and to
+name CUDA streams.  Importing this package raises if the compiled library is
+missing: there is no fallback path.
+"""
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgpt_b200.so")
+
+GPT_OK, GPT_ERR_ARG, GPT_ERR_CONFIG, GPT_ERR_WORKSPACE, GPT_ERR_STATE = 0, 1, 2, 3, 4
+GPT_ERR_INPUT, GPT_ERR_NONFINITE, GPT_ERR_CUDA, GPT_ERR_TIMEOUT = 5, 6, 7, 8
+DTYPE_F32, DTYPE_BF16, DTYPE_I32 = 0, 1, 2
+KIND_PARAM, KIND_GRAD, KIND_ADAM_M, KIND_ADAM_V, KIND_ROW_STATE, KIND_PARAM_LP, KIND_ACT = range(7)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python gpt_pretraining_step_decoder_b200/build.py` "
+        "(there is no CPU fallback)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+
+class GptConfig(ctypes.Structure):
+    _fields_ = [
+        ("n_layer", ctypes.c_int), ("d_model", ctypes.c_int), ("n_head", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("n_kv_head", ctypes.c_int), ("d_ff", ctypes.c_int),
+        ("vocab", ctypes.c_int), ("seq_len", ctypes.c_int), ("micro_batch", ctypes.c_int),
+        ("grad_accum", ctypes.c_int), ("dtype", ctypes.c_int), ("tie_embeddings", ctypes.c_int),
+        ("qk_norm", ctypes.c_int), ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float),
+        ("softcap", ctypes.c_float), ("init_std", ctypes.c_float), ("adam_b1", ctypes.c_float),
+        ("adam_b2", ctypes.c_float), ("adam_eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
+        ("grad_clip", ctypes.c_float), ("lr_mult_embed", ctypes.c_float),
+        ("lr_mult_head", ctypes.c_float), ("lr_mult_matrix", ctypes.c_float),
+        ("lr_mult_table", ctypes.c_float), ("x0_rows", ctypes.c_longlong),
+        ("v_rows", ctypes.c_longlong), ("table_beta", ctypes.c_float),
+        ("table_eps", ctypes.c_float), ("hash_p1", ctypes.c_ulonglong),
+        ("hash_p2", ctypes.c_ulonglong), ("lm_chunk_rows", ctypes.c_int),
+    ]
+
+
+_P, _I, _LL, _SZ, _F, _ULL = (ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t,
+                              ctypes.c_float, ctypes.c_ulonglong)
+_SIGS = {
+    "gpt_default_config": [ctypes.POINTER(GptConfig)],
+    "gpt_workspace_bytes": [ctypes.POINTER(GptConfig), ctypes.POINTER(_SZ)],
+    "gpt_create": [ctypes.POINTER(GptConfig), _ULL, _P, _SZ, _P, ctypes.POINTER(_P)],
+    "gpt_destroy": [_P],
+    "gpt_set_stream": [_P, _P],
+    "gpt_forward_loss": [_P, _P, _P, _P],
+    "gpt_backward_step": [_P, _F],
+    "gpt_num_params": [_P, ctypes.POINTER(_LL), ctypes.POINTER(_LL)],
+    "gpt_flops_per_token": [ctypes.POINTER(GptConfig), ctypes.POINTER(_LL), ctypes.POINTER(_LL)],
+    "gpt_tensor": [_P, ctypes.c_char_p, _I, ctypes.POINTER(_P), ctypes.POINTER(_I), _LL * 4],
+    "gpt_params_changed": [_P],
+    "gpt_sync_status": [_P],
+    "ngram_hash": [_P, _I, _I, _I, _ULL, _ULL, _LL, _P, _P],
+    "ngram_gather": [_P, _I, _P, _LL, _I, _I, _P, _I, _P],
+    "ngram_sparse_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
+    "ngram_sparse_update": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P, _SZ, _P],
+    "ngram_sync_status": [_P],
+    "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _SZ, _P],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_int
+_lib.gpt_last_error.argtypes = []
+_lib.gpt_last_error.restype = ctypes.c_char_p
+
+
+class GptError(RuntimeError):
+    def __init__(self, code, fn):
+        self.code = code
+        msg = _lib.gpt_last_error().decode(errors="replace")
+        super().__init__(f"{fn} returned {code}: {msg}")
+
+
+def _check(code, fn):
+    if code != GPT_OK:
+        raise GptError(code, fn)
+    return code
+
+
+def _ptr(x):
+    """Device/host address of a torch tensor, an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ------------------------------------------------------------------ raw entry points
+def gpt_last_error():
+    return _lib.gpt_last_error().decode(errors="replace")
+
+
+def make_config(**fields):
+    """GptConfig from gpt_default_config() plus keyword overrides (dtype may be 'f32'/'bf16')."""
+    c = GptConfig()
+    _check(_lib.gpt_default_config(ctypes.byref(c)), "gpt_default_config")
+    for k, v in fields.items():
+        if k == "dtype" and isinstance(v, str):
+            v = DTYPE_BF16 if v == "bf16" else DTYPE_F32
+        if any(k == f[0] for f in GptConfig._fields_):
+            setattr(c, k, v)
+    if c.n_kv_head == 0 or "n_kv_head" not in fields:
+        c.n_kv_head = c.n_head
+    return c
+
+
+def gpt_workspace_bytes(cfg):
+    n = ctypes.c_size_t()
+    _check(_lib.gpt_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)), "gpt_workspace_bytes")
+    return n.value
+
+
+def gpt_flops_per_token(cfg):
+    f, fc = ctypes.c_longlong(), ctypes.c_longlong()
+    _check(_lib.gpt_flops_per_token(ctypes.byref(cfg), ctypes.byref(f), ctypes.byref(fc)),
+           "gpt_flops_per_token")
+    return f.value, fc.value
+
+
+def gpt_create(cfg, seed, arena, arena_bytes, stream=None):
+    h = ctypes.c_void_p()
+    _check(_lib.gpt_create(ctypes.byref(cfg), seed, _ptr(arena), arena_bytes, _stream(stream),
+                           ctypes.byref(h)), "gpt_create")
+    return h.value
+
+
+def gpt_destroy(h):
+    return _check(_lib.gpt_destroy(h), "gpt_destroy")
+
+
+def gpt_set_stream(h, stream):
+    return _check(_lib.gpt_set_stream(h, _stream(stream)), "gpt_set_stream")
+
+
+def gpt_forward_loss(h, tokens, targets, loss):
+    return _check(_lib.gpt_forward_loss(h, _ptr(tokens), _ptr(targets), _ptr(loss)), "gpt_forward_loss")
+
+
+def gpt_backward_step(h, lr):
+    return _check(_lib.gpt_backward_step(h, float(lr)), "gpt_backward_step")
+
+
+def gpt_num_params(h):
+    d, t = ctypes.c_longlong(), ctypes.c_longlong()
+    _check(_lib.gpt_num_params(h, ctypes.byref(d), ctypes.byref(t)), "gpt_num_params")
+    return d.value, t.value
+
+
+def gpt_tensor(h, name, kind):
+    p, dt, shape = ctypes.c_void_p(), ctypes.c_int(), (ctypes.c_longlong * 4)()
+    _check(_lib.gpt_tensor(h, name.encode(), kind, ctypes.byref(p), ctypes.byref(dt), shape),
+           "gpt_tensor")
+    return p.value, dt.value, tuple(shape)
+
+
+def gpt_params_changed(h):
+    return _check(_lib.gpt_params_changed(h), "gpt_params_changed")
+
+
+def gpt_sync_status(h):
+    """Returns the status code (does not raise): GPT_OK or a device-reported error."""
+    return _lib.gpt_sync_status(h)
+
+
+def ngram_hash(tokens, B, T, vocab, p1, p2, rows, rows_out, stream=None):
+    return _check(_lib.ngram_hash(_ptr(tokens), B, T, vocab, p1, p2, rows, _ptr(rows_out),
+                                  _stream(stream)), "ngram_hash")
+
+
+def ngram_gather(rows, n, table, n_rows, d, dtype, out, accumulate, stream=None):
+    return _check(_lib.ngram_gather(_ptr(rows), n, _ptr(table), n_rows, d, dtype, _ptr(out),
+                                    accumulate, _stream(stream)), "ngram_gather")
+
+
+def ngram_sparse_update_workspace_bytes(n, d):
+    b = ctypes.c_size_t()
+    _check(_lib.ngram_sparse_update_workspace_bytes(n, d, ctypes.byref(b)),
+           "ngram_sparse_update_workspace_bytes")
+    return b.value
+
+
+def ngram_sparse_update(table, row_state, n_rows, d, dtype, rows, grad, n, lr, beta, eps,
+                        updated_rows_out, n_updated_out, workspace, ws_bytes, stream=None):
+    return _check(_lib.ngram_sparse_update(
+        _ptr(table), _ptr(row_state), n_rows, d, dtype, _ptr(rows), _ptr(grad), n, lr, beta, eps,
+        _ptr(updated_rows_out), _ptr(n_updated_out), _ptr(workspace), ws_bytes, _stream(stream)),
+        "ngram_sparse_update")
+
+
+def ngram_sync_status(stream=None):
+    return _lib.ngram_sync_status(_stream(stream))
+
+
+def gptx_gemm_bf16(M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, C, ldc, beta, splits, workspace,
+                   ws_bytes, stream=None):
+    return _check(_lib.gptx_gemm_bf16(M, N, K, _ptr(A), lda, a_kmajor, _ptr(B), ldb, b_kmajor,
+                                      _ptr(C), ldc, beta, splits, _ptr(workspace), ws_bytes,
+                                      _stream(stream)), "gptx_gemm_bf16")
+
+
+# ------------------------------------------------------------------ convenience
+class Model:
+    """A model whose arena is a torch uint8 CUDA tensor (memory ownership only)."""
+
+    def __init__(self, cfg, seed=0, device="cuda", stream=None):
+        import torch
+        self.torch = torch
+        self.cfg = cfg
+        self.bytes = gpt_workspace_bytes(cfg)
+        self.arena = torch.empty(self.bytes + 256, dtype=torch.uint8, device=device)
+        base = self.arena.data_ptr()
+        self.base = (base + 255) & ~255
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.h = gpt_create(cfg, seed, self.base, self.bytes, self.stream)
+        self.loss = torch.zeros(1, dtype=torch.float32, device=device)
+
+    def tensor(self, name, kind=KIND_PARAM):
+        """torch view of a named tensor inside the arena (no copy)."""
+        torch = self.torch
+        p, dt, shape = gpt_tensor(self.h, name, kind)
+        tdt = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16, DTYPE_I32: torch.int32}[dt]
+        esz = 2 if dt == DTYPE_BF16 else 4
+        rows, cols = shape[0], shape[1]
+        off = p - self.arena.data_ptr()
+        return self.arena[off:off + rows * cols * esz].view(tdt).view(rows, cols)
+
+    def forward_loss(self, tokens, targets):
+        gpt_forward_loss(self.h, tokens, targets, self.loss)
+        return self.loss
+
+    def backward_step(self, lr):
+        gpt_backward_step(self.h, lr)
+
+    def sync_status(self):
+        return gpt_sync_status(self.h)
+
+    def close(self):
+        if self.h:
+            gpt_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,73 @@
+// gemm_common.cuh -- operand and epilogue description shared by the GEMMs.
+//
+// Every dense contraction of the step is C[m, n] = sum_k A[m, k] * B[n, k]
+// followed by an epilogue.  Operands are row-major buffers read either
+// K-major (element [r, k] at ptr[r * ld + k]) or MN-major (element [r, k] at
+// ptr[k * ld + r]); this covers forward (x W^T), data-gradient (dY W) and
+// weight-gradient (dY^T X) products without any transposed copies.
+#pragma once
+#include "common.cuh"
+
+struct GemmOperand {
+  const void* ptr;
+  long long ld;   // elements between consecutive rows of the stored buffer
+  int kmajor;     // 1: [rows, K] storage; 0: [K, rows] storage
+};
+
+enum EpiMode {
+  EPI_STORE = 0,      // C(act) = alpha * acc
+  EPI_STORE_F32 = 1,  // C(f32) = alpha * acc
+  EPI_ACCUM_F32 = 2,  // C(f32) = (beta ? C : 0) + alpha * acc
+  EPI_RELU2 = 3,      // r = relu(acc): C(act) = r, C2(act) = r * r
+  EPI_DRELU2 = 4,     // C(act) = 2 * aux(act) * acc   (ReLU^2 backward)
+};
+
+struct GemmEpilogue {
+  int mode;
+  void* C;          // output [M, ldc]
+  long long ldc;
+  void* C2;         // second output (EPI_RELU2), same ld as C
+  const void* aux;  // EPI_DRELU2 input, same ld as C
+  float alpha;
+  int beta;
+};
+
+template <typename act_t>
+__device__ __forceinline__ void epi_apply_one(const GemmEpilogue& e, long long m, long long n,
+                                              float acc) {
+  const long long off = m * e.ldc + n;
+  acc *= e.alpha;
+  switch (e.mode) {
+    case EPI_STORE: reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(acc); break;
+    case EPI_STORE_F32: reinterpret_cast<float*>(e.C)[off] = acc; break;
+    case EPI_ACCUM_F32: {
+      float* c = reinterpret_cast<float*>(e.C);
+      c[off] = (e.beta ? c[off] : 0.f) + acc;
+      break;
+    }
+    case EPI_RELU2: {
+      float r = fmaxf(acc, 0.f);
+      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(r);
+      reinterpret_cast<act_t*>(e.C2)[off] = from_f<act_t>(r * r);
+      break;
+    }
+    case EPI_DRELU2: {
+      float r = to_f(reinterpret_cast<const act_t*>(e.aux)[off]);
+      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(2.f * r * acc);
+      break;
+    }
+  }
+}
+
+// Sum split-K partials [S, M, N] (fp32, in split order) into the epilogue.
+template <typename act_t>
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N,
+                                     GemmEpilogue e) {
+  const long long total = (long long)M * N;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part[(long long)s * total + i];
+    epi_apply_one<act_t>(e, i / N, i % N, acc);
+  }
+}

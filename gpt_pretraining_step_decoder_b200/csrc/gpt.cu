@@ -1,0 +1,991 @@
+// gpt.cu -- C ABI of libgpt_b200.so and the host-side step orchestration.
+//
+// All device memory comes from the caller's arena; this file carves it,
+// enqueues every kernel of a forward / backward / optimizer step on one CUDA
+// stream, and maps the device error word to status codes.  The meaning of
+// each entry point is documented in include/gpt.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdarg>
+#include <cstring>
+#include <type_traits>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/gpt.h"
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "layers.cuh"
+#include "ngram.cuh"
+#include "optim.cuh"
+
+// ======================================================================== errors
+static thread_local std::string g_last_error;
+
+static int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                    \
+  do {                                                                                    \
+    cudaError_t e_ = (expr);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return fail(GPT_ERR_CUDA, "%s failed: %s (%s:%d)", #expr, cudaGetErrorString(e_),   \
+                  __FILE__, __LINE__);                                                    \
+  } while (0)
+
+#define LAUNCH_CHECK() CUDA_TRY(cudaGetLastError())
+
+#define TRY(expr)            \
+  do {                       \
+    int s_ = (expr);         \
+    if (s_ != GPT_OK) return s_; \
+  } while (0)
+
+extern "C" const char* gpt_last_error(void) { return g_last_error.c_str(); }
+
+// ======================================================================== device props
+static int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+// standalone operations' error word (one per device that loads the library)
+__device__ unsigned g_ngram_err;
+
+// ======================================================================== TMA maps
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+static int get_encode() {
+  if (g_encode) return GPT_OK;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  CUDA_TRY(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+  if (!fn || q != cudaDriverEntryPointSuccess) return fail(GPT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return GPT_OK;
+}
+
+// 2-D bf16 map over a row-major [outer, inner] buffer with row pitch `ld`
+// elements, 128-byte swizzle, zero fill outside the tensor.
+static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_inner, uint32_t box_outer) {
+  TRY(get_encode());
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((ld * 2) & 15))
+    return fail(GPT_ERR_ARG, "TMA operand not 16-byte aligned (ptr %p, ld %llu)", ptr,
+                (unsigned long long)ld);
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GPT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return GPT_OK;
+}
+
+// ======================================================================== GEMM dispatch
+template <int BN>
+static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
+                          int splits, float* partial, unsigned* err, cudaStream_t st) {
+  using C = tc::Cfg<BN>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    CUDA_TRY(cudaFuncSetAttribute(tc::gemm_tc_kernel<BN, bf16>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    attr_done = true;
+  }
+  CUtensorMap ta, tb;
+  if (A.kmajor) TRY(make_tmap(&ta, A.ptr, K, M, A.ld, tc::BK, tc::BM));
+  else TRY(make_tmap(&ta, A.ptr, M, K, A.ld, 64, tc::BK));
+  if (B.kmajor) TRY(make_tmap(&tb, B.ptr, K, N, B.ld, tc::BK, BN));
+  else TRY(make_tmap(&tb, B.ptr, N, K, B.ld, 64, tc::BK));
+  tc::Params p;
+  p.M = M; p.N = N; p.K = K;
+  p.a_kmajor = A.kmajor; p.b_kmajor = B.kmajor;
+  p.m_tiles = cdiv(M, tc::BM);
+  p.n_tiles = cdiv(N, BN);
+  p.kb_total = cdiv(K, tc::BK);
+  if (splits < 1) splits = 1;
+  if (splits > p.kb_total) splits = p.kb_total;
+  p.kb_per_split = cdiv(p.kb_total, splits);
+  p.splits = cdiv(p.kb_total, p.kb_per_split);
+  p.epi = e;
+  p.partial = partial;
+  p.err = err;
+  const int tiles = p.m_tiles * p.n_tiles * p.splits;
+  const int grid = tiles < device_sms() ? tiles : device_sms();
+  tc::gemm_tc_kernel<BN, bf16><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
+  LAUNCH_CHECK();
+  if (p.splits > 1) {
+    const long long total = (long long)M * N;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 4 * device_sms()) blocks = 4 * device_sms();
+    splitk_reduce_kernel<bf16><<<blocks, 256, 0, st>>>(partial, p.splits, M, N, e);
+    LAUNCH_CHECK();
+  }
+  return GPT_OK;
+}
+
+// Choose split-K so a small-output, long-K product still fills the GPU.
+static int pick_splits(int M, int N, int K, int BN) {
+  const int tiles = cdiv(M, 128) * cdiv(N, BN);
+  const int kb = cdiv(K, 64);
+  const int sms = device_sms();
+  int s = 1;
+  while (tiles * s < sms && kb / (s * 2) >= 8) s *= 2;
+  while (tiles * (s + 1) <= sms + sms / 8 && kb / (s + 1) >= 8) ++s;
+  return s;
+}
+
+struct GemmCtx {
+  bool bf16;
+  float* splitk;          // fp32 scratch for split-K partials
+  long long splitk_elems;
+  unsigned* err;
+  cudaStream_t st;
+};
+
+static int gemm(const GemmCtx& g, int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
+                bool allow_split = false) {
+  if (M <= 0 || N <= 0 || K <= 0) return GPT_OK;
+  if (!g.bf16) {
+    gemm_simt<float, float>(M, N, K, A, B, e, g.st);
+    LAUNCH_CHECK();
+    return GPT_OK;
+  }
+  const int BN = (N >= 256) ? 256 : 128;
+  int splits = 1;
+  if (allow_split && (e.mode == EPI_ACCUM_F32 || e.mode == EPI_STORE_F32)) {
+    splits = pick_splits(M, N, K, BN);
+    while (splits > 1 && (long long)splits * M * N > g.splitk_elems) --splits;
+  }
+  if (BN == 256) return gemm_tc_launch<256>(M, N, K, A, B, e, splits, g.splitk, g.err, g.st);
+  return gemm_tc_launch<128>(M, N, K, A, B, e, splits, g.splitk, g.err, g.st);
+}
+
+static GemmOperand op_k(const void* p, long long ld) { return GemmOperand{p, ld, 1}; }
+static GemmOperand op_mn(const void* p, long long ld) { return GemmOperand{p, ld, 0}; }
+static GemmEpilogue epi(int mode, void* C, long long ldc, int beta = 0, void* C2 = nullptr,
+                        const void* aux = nullptr, float alpha = 1.f) {
+  GemmEpilogue e;
+  e.mode = mode; e.C = C; e.ldc = ldc; e.C2 = C2; e.aux = aux; e.alpha = alpha; e.beta = beta;
+  return e;
+}
+
+// ======================================================================== arena plan
+struct Carver {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    off = (off + 255) & ~size_t(255);
+    size_t r = off;
+    off += bytes;
+    return r;
+  }
+};
+
+struct DenseTensor {
+  std::string name;
+  long long off;  // element offset in the flat dense buffers
+  long long rows, cols;
+};
+
+struct LayerActs {
+  size_t u, rstd1, qkv, rstd_q, rstd_k, o, lse, u2, rstd2, r, g;
+};
+
+struct Plan {
+  // dense flat buffers
+  std::vector<DenseTensor> dense;
+  long long dense_n = 0, e_end = 0, h_end = 0;
+  size_t P, G, M, V, Plp;
+  size_t hx = 0, hv = 0, hx_state = 0, hv_state = 0;
+  size_t x, emb_rstd, xf, rstd_f, tok_copy, rows_x, rows_v;
+  std::vector<LayerActs> layers;
+  size_t dx, dx_lp, du, dqkv, da, dout, Dattn, gv, dxf, pending;
+  size_t logits, dz, tok_loss, ce_scale, ce_count, loss_scratch;
+  size_t sort_keys_a, sort_keys_b, sort_vals_a, sort_vals_b, sort_counts;
+  size_t seg_start, pstart, plen, pseg, pslot, lfirst, lnslots, lseg, counters, seg_partial;
+  size_t splitk; long long splitk_elems;
+  size_t norm_part, clip_coef, grad_norm, rope_cs, err;
+  int chunk;
+  size_t total;
+};
+
+static bool cfg_bf16(const gpt_config& c) { return c.dtype == GPT_DTYPE_BF16; }
+
+static int validate(const gpt_config* c) {
+  if (!c) return fail(GPT_ERR_ARG, "null config");
+  if (c->n_layer < 1 || c->d_model < 1 || c->n_head < 1 || c->head_dim < 2 || c->d_ff < 1 ||
+      c->vocab < 2 || c->seq_len < 1 || c->micro_batch < 1 || c->grad_accum < 1)
+    return fail(GPT_ERR_CONFIG, "non-positive dimension in config");
+  if (c->dtype != GPT_DTYPE_F32 && c->dtype != GPT_DTYPE_BF16)
+    return fail(GPT_ERR_CONFIG, "dtype must be GPT_DTYPE_F32 or GPT_DTYPE_BF16");
+  if (c->d_model != c->n_head * c->head_dim)
+    return fail(GPT_ERR_CONFIG, "d_model (%d) != n_head * head_dim (%d)", c->d_model, c->n_head * c->head_dim);
+  if (c->n_kv_head != 0 && c->n_kv_head != c->n_head)
+    return fail(GPT_ERR_CONFIG, "grouped KV heads are not supported (n_kv_head must equal n_head)");
+  if (c->head_dim % 2 || c->head_dim > 128) return fail(GPT_ERR_CONFIG, "head_dim must be even and <= 128");
+  if (c->d_model % 4 || c->d_model > 2048 || c->d_ff % 4)
+    return fail(GPT_ERR_CONFIG, "d_model must be a multiple of 4 and <= 2048; d_ff a multiple of 4");
+  if (cfg_bf16(*c)) {
+    if (c->head_dim != 128) return fail(GPT_ERR_CONFIG, "bf16 mode needs head_dim == 128");
+    if (c->d_model % 64 || c->d_ff % 64 || c->vocab % 64)
+      return fail(GPT_ERR_CONFIG, "bf16 mode needs d_model, d_ff, vocab multiples of 64");
+  }
+  if (c->x0_rows < 0 || c->v_rows < 0 || c->x0_rows > 0x7fffffffLL || c->v_rows > 0x7fffffffLL)
+    return fail(GPT_ERR_CONFIG, "table rows out of range");
+  const long long N = (long long)c->micro_batch * c->seq_len;
+  if (N > (1LL << 24)) return fail(GPT_ERR_CONFIG, "too many tokens per micro-batch");
+  if (c->norm_eps <= 0.f || c->rope_base <= 1.f) return fail(GPT_ERR_CONFIG, "bad norm_eps or rope_base");
+  return GPT_OK;
+}
+
+static void make_plan(const gpt_config& c, Plan& p) {
+  const bool b16 = cfg_bf16(c);
+  const size_t es = b16 ? 2 : 4;  // activation element size
+  const long long N = (long long)c.micro_batch * c.seq_len;
+  const long long d = c.d_model, a = (long long)c.n_head * c.head_dim, F = c.d_ff, V = c.vocab;
+  const long long BH = (long long)c.micro_batch * c.n_head;
+  // ---- dense flat layout: [wte][lm_head][layers...], each padded to 64 elements
+  long long off = 0;
+  auto add = [&](const std::string& nm, long long r, long long k) {
+    p.dense.push_back({nm, off, r, k});
+    off += ((r * k + 63) / 64) * 64;
+  };
+  add("wte", V, d);
+  p.e_end = off;
+  if (!c.tie_embeddings) add("lm_head", V, d);
+  p.h_end = off;
+  for (int l = 0; l < c.n_layer; ++l) {
+    add("h" + std::to_string(l) + ".wqkv", 3 * a, d);
+    add("h" + std::to_string(l) + ".wo", d, a);
+    add("h" + std::to_string(l) + ".w1", F, d);
+    add("h" + std::to_string(l) + ".w2", d, F);
+  }
+  p.dense_n = off;
+  Carver cv;
+  p.P = cv.take(off * 4);
+  p.G = cv.take(off * 4);
+  p.M = cv.take(off * 4);
+  p.V = cv.take(off * 4);
+  p.Plp = b16 ? cv.take(off * 2) : 0;
+  const size_t tes = b16 ? 2 : 4;
+  if (c.x0_rows) { p.hx = cv.take(c.x0_rows * d * tes); p.hx_state = cv.take(c.x0_rows * 4); }
+  if (c.v_rows) { p.hv = cv.take(c.v_rows * a * tes); p.hv_state = cv.take(c.v_rows * 4); }
+  // ---- activations
+  p.x = cv.take(N * d * 4);
+  p.emb_rstd = cv.take(N * 4);
+  p.tok_copy = cv.take(N * 4);
+  p.rows_x = cv.take(N * 4);
+  p.rows_v = cv.take(N * 4);
+  p.layers.resize(c.n_layer);
+  for (int l = 0; l < c.n_layer; ++l) {
+    LayerActs& L = p.layers[l];
+    L.u = cv.take(N * d * es);
+    L.rstd1 = cv.take(N * 4);
+    L.qkv = cv.take(N * 3 * a * es);
+    L.rstd_q = cv.take(N * c.n_head * 4);
+    L.rstd_k = cv.take(N * c.n_head * 4);
+    L.o = cv.take(N * a * es);
+    L.lse = cv.take(BH * c.seq_len * 4);
+    L.u2 = cv.take(N * d * es);
+    L.rstd2 = cv.take(N * 4);
+    L.r = cv.take(N * F * es);
+    L.g = cv.take(N * F * es);
+  }
+  p.xf = cv.take(N * d * es);
+  p.rstd_f = cv.take(N * 4);
+  // ---- backward work
+  p.dx = cv.take(N * d * 4);
+  p.dx_lp = cv.take(N * d * es);
+  p.du = cv.take(N * d * 4);
+  p.dqkv = cv.take(N * 3 * a * es);
+  p.da = cv.take(N * F * es);
+  p.dout = cv.take(N * a * es);
+  p.Dattn = cv.take(BH * c.seq_len * 4);
+  p.gv = c.v_rows ? cv.take(N * a * 4) : 0;
+  p.dxf = cv.take(N * d * 4);
+  p.pending = cv.take(V * d * 4);
+  // ---- LM head chunk
+  long long chunk = c.lm_chunk_rows > 0 ? c.lm_chunk_rows : 8192;
+  if (chunk > N) chunk = N;
+  p.chunk = (int)chunk;
+  p.logits = cv.take(chunk * V * 4);
+  p.dz = cv.take(chunk * V * es);
+  p.tok_loss = cv.take(N * 4);
+  p.ce_scale = cv.take(4);
+  p.ce_count = cv.take(4);
+  p.loss_scratch = cv.take(4);
+  // ---- bucketing workspace (positions by row / by token)
+  const long long nblk = (N + RADIX_TILE - 1) / RADIX_TILE;
+  p.sort_keys_a = cv.take(N * 4);
+  p.sort_keys_b = cv.take(N * 4);
+  p.sort_vals_a = cv.take(N * 4);
+  p.sort_vals_b = cv.take(N * 4);
+  p.sort_counts = cv.take(256 * nblk * 4);
+  const long long maxp = N + N / PIECE + 2, maxl = N / PIECE + 2, maxslots = 2 * (N / PIECE) + 4;
+  p.seg_start = cv.take((N + 1) * 4);
+  p.pstart = cv.take(maxp * 4);
+  p.plen = cv.take(maxp * 4);
+  p.pseg = cv.take(maxp * 4);
+  p.pslot = cv.take(maxp * 4);
+  p.lfirst = cv.take(maxl * 4);
+  p.lnslots = cv.take(maxl * 4);
+  p.lseg = cv.take(maxl * 4);
+  p.counters = cv.take(16);
+  p.seg_partial = cv.take(maxslots * (d > a ? d : a) * 4);
+  // ---- split-K partials: the largest weight gradient x 8 splits
+  long long mx = 3 * a * d;
+  if (F * d > mx) mx = F * d;
+  p.splitk_elems = b16 ? 8 * mx : 0;
+  p.splitk = b16 ? cv.take(p.splitk_elems * 4) : 0;
+  p.norm_part = cv.take(NORM_BLOCKS * 8);
+  p.clip_coef = cv.take(4);
+  p.grad_norm = cv.take(4);
+  p.rope_cs = cv.take((long long)c.seq_len * c.head_dim * 4);
+  p.err = cv.take(16);
+  p.total = cv.take(0) + 256;
+}
+
+// ======================================================================== model
+struct gpt_model {
+  gpt_config cfg;
+  Plan plan;
+  uint8_t* base;
+  size_t bytes;
+  cudaStream_t st;
+  int micro = 0;
+  long long step_t = 0;
+  bool have_fwd = false;
+  template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+  unsigned* err() const { return at<unsigned>(plan.err); }
+};
+
+static const DenseTensor* find_dense(const gpt_model* m, const std::string& name) {
+  for (const auto& t : m->plan.dense)
+    if (t.name == name) return &t;
+  return nullptr;
+}
+
+extern "C" int gpt_default_config(gpt_config* c) {
+  if (!c) return fail(GPT_ERR_ARG, "null config");
+  memset(c, 0, sizeof(*c));
+  c->n_layer = 2; c->d_model = 128; c->n_head = 4; c->head_dim = 32; c->n_kv_head = 4;
+  c->d_ff = 512; c->vocab = 512; c->seq_len = 64; c->micro_batch = 4; c->grad_accum = 1;
+  c->dtype = GPT_DTYPE_F32; c->tie_embeddings = 1; c->qk_norm = 1;
+  c->rope_base = 10000.f; c->norm_eps = 1.1920929e-07f; c->softcap = 0.f; c->init_std = 0.02f;
+  c->adam_b1 = 0.8f; c->adam_b2 = 0.95f; c->adam_eps = 1e-10f; c->weight_decay = 0.f;
+  c->grad_clip = 0.f;
+  c->lr_mult_embed = c->lr_mult_head = c->lr_mult_matrix = c->lr_mult_table = 1.f;
+  c->x0_rows = 0; c->v_rows = 0; c->table_beta = 0.95f; c->table_eps = 1e-10f;
+  c->hash_p1 = 2654435761ull; c->hash_p2 = 2246822519ull;
+  c->lm_chunk_rows = 0;
+  return GPT_OK;
+}
+
+extern "C" int gpt_workspace_bytes(const gpt_config* cfg, size_t* bytes) {
+  if (!bytes) return fail(GPT_ERR_ARG, "null bytes");
+  TRY(validate(cfg));
+  Plan p;
+  make_plan(*cfg, p);
+  *bytes = p.total;
+  return GPT_OK;
+}
+
+extern "C" int gpt_flops_per_token(const gpt_config* c, long long* flops, long long* flops_causal) {
+  TRY(validate(c));
+  const long long d = c->d_model, a = (long long)c->n_head * c->head_dim, F = c->d_ff, V = c->vocab;
+  const long long mat = (long long)c->n_layer * (3 * a * d + d * a + F * d + d * F) + V * d;
+  const long long attn = 12LL * c->n_layer * c->n_head * c->head_dim * c->seq_len;
+  if (flops) *flops = 6 * mat + attn;
+  if (flops_causal) *flops_causal = 6 * mat + attn / 2;
+  return GPT_OK;
+}
+
+static int grid_for(long long n, int per_block) {
+  long long b = (n + per_block - 1) / per_block;
+  return (int)(b < 1 ? 1 : b);
+}
+
+static int refresh_lp(gpt_model* m) {
+  if (!cfg_bf16(m->cfg)) return GPT_OK;
+  const Plan& p = m->plan;
+  to_bf16_kernel<<<4 * device_sms(), 256, 0, m->st>>>(m->at<float>(p.P), m->at<bf16>(p.Plp), p.dense_n);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+extern "C" int gpt_create(const gpt_config* cfg, unsigned long long seed, void* arena, size_t arena_bytes,
+                          void* cuda_stream, gpt_model** out) {
+  if (!out || !arena) return fail(GPT_ERR_ARG, "null arena or out");
+  *out = nullptr;
+  TRY(validate(cfg));
+  if (reinterpret_cast<uintptr_t>(arena) & 255) return fail(GPT_ERR_ARG, "arena not 256-byte aligned");
+  gpt_model* m = new gpt_model();
+  m->cfg = *cfg;
+  make_plan(m->cfg, m->plan);
+  if (arena_bytes < m->plan.total) {
+    size_t need = m->plan.total;
+    delete m;
+    return fail(GPT_ERR_WORKSPACE, "arena too small: %zu < %zu bytes", arena_bytes, need);
+  }
+  m->base = static_cast<uint8_t*>(arena);
+  m->bytes = arena_bytes;
+  m->st = static_cast<cudaStream_t>(cuda_stream);
+  const Plan& p = m->plan;
+  const gpt_config& c = m->cfg;
+  cudaError_t e = cudaMemsetAsync(arena, 0, p.total, m->st);
+  if (e != cudaSuccess) { delete m; return fail(GPT_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e)); }
+  const int blocks = 8 * device_sms();
+  uint32_t stream_id = 1;
+  for (const auto& t : p.dense) {
+    init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.P) + t.off, t.rows * t.cols,
+                                                        c.init_std, seed, stream_id++);
+  }
+  const long long a = (long long)c.n_head * c.head_dim;
+  if (c.x0_rows) {
+    if (cfg_bf16(c))
+      init_normal_kernel<bf16><<<blocks, 256, 0, m->st>>>(m->at<bf16>(p.hx), c.x0_rows * c.d_model, c.init_std, seed, 0x10000u);
+    else
+      init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.hx), c.x0_rows * c.d_model, c.init_std, seed, 0x10000u);
+  }
+  if (c.v_rows) {
+    if (cfg_bf16(c))
+      init_normal_kernel<bf16><<<blocks, 256, 0, m->st>>>(m->at<bf16>(p.hv), c.v_rows * a, c.init_std, seed, 0x10001u);
+    else
+      init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.hv), c.v_rows * a, c.init_std, seed, 0x10001u);
+  }
+  rope_table_kernel<<<grid_for((long long)c.seq_len * c.head_dim / 2, 256), 256, 0, m->st>>>(
+      m->at<float>(p.rope_cs), c.seq_len, c.head_dim, (double)c.rope_base);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) { delete m; return fail(GPT_ERR_CUDA, "init launch: %s", cudaGetErrorString(e)); }
+  int s = refresh_lp(m);
+  if (s != GPT_OK) { delete m; return s; }
+  *out = m;
+  return GPT_OK;
+}
+
+extern "C" int gpt_destroy(gpt_model* m) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  cudaStreamSynchronize(m->st);
+  delete m;
+  return GPT_OK;
+}
+
+extern "C" int gpt_set_stream(gpt_model* m, void* s) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  m->st = static_cast<cudaStream_t>(s);
+  return GPT_OK;
+}
+
+extern "C" int gpt_num_params(const gpt_model* m, long long* dense, long long* table) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  long long dn = 0;
+  for (const auto& t : m->plan.dense) dn += t.rows * t.cols;
+  if (dense) *dense = dn;
+  if (table) *table = m->cfg.x0_rows * m->cfg.d_model + m->cfg.v_rows * (long long)m->cfg.n_head * m->cfg.head_dim;
+  return GPT_OK;
+}
+
+extern "C" int gpt_params_changed(gpt_model* m) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  return refresh_lp(m);
+}
+
+extern "C" int gpt_sync_status(gpt_model* m) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  CUDA_TRY(cudaStreamSynchronize(m->st));
+  unsigned w = 0;
+  CUDA_TRY(cudaMemcpy(&w, m->err(), 4, cudaMemcpyDeviceToHost));
+  if (w) CUDA_TRY(cudaMemset(m->err(), 0, 4));
+  if (w & GPT_EBIT_TIMEOUT) return fail(GPT_ERR_TIMEOUT, "a kernel's bounded wait gave up");
+  if (w & GPT_EBIT_INPUT) return fail(GPT_ERR_INPUT, "token, target or row id out of range");
+  if (w & GPT_EBIT_NONFINITE) return fail(GPT_ERR_NONFINITE, "non-finite loss or gradient norm");
+  return GPT_OK;
+}
+
+extern "C" int gpt_tensor(gpt_model* m, const char* name, int kind, void** ptr, int* dtype,
+                          long long shape[4]) {
+  if (!m || !name || !ptr) return fail(GPT_ERR_ARG, "null argument");
+  const Plan& p = m->plan;
+  const gpt_config& c = m->cfg;
+  const bool b16 = cfg_bf16(c);
+  long long sh[4] = {1, 1, 1, 1};
+  int dt = GPT_DTYPE_F32;
+  void* ptr_out = nullptr;
+  const std::string nm(name);
+  const long long N = (long long)c.micro_batch * c.seq_len;
+  const long long a = (long long)c.n_head * c.head_dim;
+  if (kind == GPT_KIND_ACT) {
+    if (nm == "per_token_loss") { ptr_out = m->at<float>(p.tok_loss); sh[0] = c.micro_batch; sh[1] = c.seq_len; }
+    else if (nm == "rows_x" && c.x0_rows) { ptr_out = m->at<int32_t>(p.rows_x); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
+    else if (nm == "rows_v" && c.v_rows) { ptr_out = m->at<int32_t>(p.rows_v); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
+    else if (nm == "grad_norm") { ptr_out = m->at<float>(p.grad_norm); }
+    else return fail(GPT_ERR_ARG, "unknown activation '%s'", name);
+    (void)N;
+  } else if (nm == "hx" || nm == "hv") {
+    const bool isx = nm == "hx";
+    const long long rows = isx ? c.x0_rows : c.v_rows;
+    if (!rows) return fail(GPT_ERR_ARG, "table '%s' absent", name);
+    sh[0] = rows; sh[1] = isx ? c.d_model : a;
+    if (kind == GPT_KIND_PARAM) { ptr_out = m->base + (isx ? p.hx : p.hv); dt = b16 ? GPT_DTYPE_BF16 : GPT_DTYPE_F32; }
+    else if (kind == GPT_KIND_ROW_STATE) { ptr_out = m->base + (isx ? p.hx_state : p.hv_state); sh[1] = 1; }
+    else return fail(GPT_ERR_ARG, "tables have kinds PARAM and ROW_STATE only");
+  } else {
+    const DenseTensor* t = find_dense(m, nm);
+    if (!t) return fail(GPT_ERR_ARG, "unknown tensor '%s'", name);
+    sh[0] = t->rows; sh[1] = t->cols;
+    switch (kind) {
+      case GPT_KIND_PARAM: ptr_out = m->at<float>(p.P) + t->off; break;
+      case GPT_KIND_GRAD: ptr_out = m->at<float>(p.G) + t->off; break;
+      case GPT_KIND_ADAM_M: ptr_out = m->at<float>(p.M) + t->off; break;
+      case GPT_KIND_ADAM_V: ptr_out = m->at<float>(p.V) + t->off; break;
+      case GPT_KIND_PARAM_LP:
+        if (!b16) return fail(GPT_ERR_ARG, "no bf16 copy in fp32 mode");
+        ptr_out = m->at<bf16>(p.Plp) + t->off; dt = GPT_DTYPE_BF16; break;
+      default: return fail(GPT_ERR_ARG, "bad kind %d for '%s'", kind, name);
+    }
+  }
+  *ptr = ptr_out;
+  if (dtype) *dtype = dt;
+  if (shape) for (int i = 0; i < 4; ++i) shape[i] = sh[i];
+  return GPT_OK;
+}
+
+// ======================================================================== bucketing
+struct SortWs {
+  uint32_t *ka, *kb, *counts;
+  int32_t *va, *vb;
+  int32_t *seg_start, *pstart, *plen, *pseg, *pslot, *lfirst, *lnslots, *lseg, *counters;
+  float* partial;
+};
+
+static SortWs sort_ws(const gpt_model* m) {
+  const Plan& p = m->plan;
+  SortWs w;
+  w.ka = m->at<uint32_t>(p.sort_keys_a); w.kb = m->at<uint32_t>(p.sort_keys_b);
+  w.va = m->at<int32_t>(p.sort_vals_a); w.vb = m->at<int32_t>(p.sort_vals_b);
+  w.counts = m->at<uint32_t>(p.sort_counts);
+  w.seg_start = m->at<int32_t>(p.seg_start); w.pstart = m->at<int32_t>(p.pstart);
+  w.plen = m->at<int32_t>(p.plen); w.pseg = m->at<int32_t>(p.pseg); w.pslot = m->at<int32_t>(p.pslot);
+  w.lfirst = m->at<int32_t>(p.lfirst); w.lnslots = m->at<int32_t>(p.lnslots); w.lseg = m->at<int32_t>(p.lseg);
+  w.counters = m->at<int32_t>(p.counters); w.partial = m->at<float>(p.seg_partial);
+  return w;
+}
+
+// Stable sort of (key, position) by key, then segments and pieces.  Leaves
+// sorted keys in *keys_out and positions in *perm_out.
+static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long key_range,
+                         const uint32_t** keys_out, const int32_t** perm_out, int32_t* uniq_out,
+                         int* n_uniq_out, unsigned* err, cudaStream_t st) {
+  iota_kernel<<<grid_for(n, 256), 256, 0, st>>>(keys, w.ka, w.va, n, key_range, err);
+  LAUNCH_CHECK();
+  int bits = 1;
+  while (bits < 32 && (1LL << bits) < key_range) ++bits;
+  const int passes = (bits + 7) / 8;
+  const int nblk = (n + RADIX_TILE - 1) / RADIX_TILE;
+  uint32_t *kin = w.ka, *kout = w.kb;
+  int32_t *vin = w.va, *vout = w.vb;
+  for (int ps = 0; ps < passes; ++ps) {
+    radix_hist_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, n, 8 * ps, w.counts);
+    exclusive_scan_kernel<<<1, 1024, 0, st>>>(w.counts, 256 * nblk);
+    radix_scatter_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, vin, n, 8 * ps, w.counts, kout, vout);
+    LAUNCH_CHECK();
+    std::swap(kin, kout);
+    std::swap(vin, vout);
+  }
+  segments_kernel<<<1, 1024, 0, st>>>(kin, n, w.seg_start, w.pstart, w.plen, w.pseg, w.pslot, w.lfirst,
+                                      w.lnslots, w.lseg, w.counters, uniq_out, n_uniq_out);
+  LAUNCH_CHECK();
+  *keys_out = kin;
+  *perm_out = vin;
+  return GPT_OK;
+}
+
+template <typename tab_t>
+static int table_update(const SortWs& w, tab_t* table, float* state, long long n_rows, int d,
+                        const int32_t* rows, const float* grad, int n, float lr, float beta, float eps,
+                        int32_t* uniq_out, int* n_uniq_out, unsigned* err, cudaStream_t st) {
+  const uint32_t* skeys;
+  const int32_t* perm;
+  TRY(bucket_by_key(w, rows, n, n_rows, &skeys, &perm, uniq_out, n_uniq_out, err, st));
+  const long long maxp = (long long)n + n / PIECE + 2, maxl = n / PIECE + 2;
+  table_piece_kernel<tab_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
+      table, state, d, grad, skeys, perm, w.pstart, w.plen, w.pslot, w.counters, w.partial, lr, beta, eps);
+  table_long_kernel<tab_t><<<grid_for(maxl * 32, 256), 256, 0, st>>>(
+      table, state, d, skeys, w.seg_start, w.lfirst, w.lnslots, w.lseg, w.counters, w.partial, lr, beta, eps);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+// ======================================================================== forward
+template <typename act_t>
+static int attention_fwd(const gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
+  const gpt_config& c = m->cfg;
+  dim3 grid(cdiv(c.seq_len, 4), c.micro_batch * c.n_head);
+  attn_fwd_simt_kernel<act_t><<<grid, 128, 4 * c.head_dim * 4, m->st>>>(qkv, o, lse, c.micro_batch, c.seq_len,
+                                                                        c.n_head, c.head_dim);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+template <typename act_t>
+static int attention_bwd(const gpt_model* m, const act_t* qkv, const act_t* o, const act_t* dout,
+                         const float* lse, float* Dv, act_t* dqkv) {
+  const gpt_config& c = m->cfg;
+  const long long N = (long long)c.micro_batch * c.seq_len;
+  attn_bwd_pre_kernel<act_t><<<grid_for(N * c.n_head * 32, 256), 256, 0, m->st>>>(
+      o, dout, Dv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
+  LAUNCH_CHECK();
+  dim3 grid(cdiv(c.seq_len, 4), c.micro_batch * c.n_head);
+  attn_bwd_dq_simt_kernel<act_t><<<grid, 128, 4 * 2 * c.head_dim * 4, m->st>>>(
+      qkv, dout, lse, Dv, dqkv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
+  attn_bwd_dkdv_simt_kernel<act_t><<<grid, 128, 4 * 2 * c.head_dim * 4, m->st>>>(
+      qkv, dout, lse, Dv, dqkv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+template <typename act_t>
+static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targets, float* loss_dev) {
+  const gpt_config& c = m->cfg;
+  const Plan& p = m->plan;
+  const bool b16 = cfg_bf16(c);
+  cudaStream_t st = m->st;
+  const int N = c.micro_batch * c.seq_len;
+  const int d = c.d_model, H = c.n_head, hd = c.head_dim, a = H * hd, F = c.d_ff, V = c.vocab;
+  unsigned* err = m->err();
+  GemmCtx g{b16, m->at<float>(p.splitk), p.splitk_elems, err, st};
+  // weights read by the GEMMs: the bf16 copy in bf16 mode, the master in fp32 mode
+  auto W = [&](const std::string& nm) -> const act_t* {
+    const DenseTensor* t = find_dense(m, nm);
+    return b16 ? reinterpret_cast<const act_t*>(m->at<bf16>(p.Plp) + t->off)
+               : reinterpret_cast<const act_t*>(m->at<float>(p.P) + t->off);
+  };
+  CUDA_TRY(cudaMemcpyAsync(m->at<int32_t>(p.tok_copy), tokens, (size_t)N * 4, cudaMemcpyDeviceToDevice, st));
+  if (c.x0_rows || c.v_rows) {
+    ngram_hash_kernel<<<grid_for(N, 256), 256, 0, st>>>(
+        tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.x0_rows ? c.x0_rows : 1,
+        c.x0_rows ? m->at<int32_t>(p.rows_x) : nullptr, c.v_rows ? c.v_rows : 1,
+        c.v_rows ? m->at<int32_t>(p.rows_v) : nullptr, err);
+    LAUNCH_CHECK();
+  }
+  float* x = m->at<float>(p.x);
+  embed_fwd_kernel<act_t, act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+      tokens, W("wte"), c.x0_rows ? reinterpret_cast<const act_t*>(m->base + p.hx) : nullptr,
+      m->at<int32_t>(p.rows_x), x, m->at<float>(p.emb_rstd), N, d, V, c.norm_eps, err);
+  LAUNCH_CHECK();
+  const int rows_blocks = grid_for((long long)N * 32, 256);
+  for (int l = 0; l < c.n_layer; ++l) {
+    const LayerActs& L = p.layers[l];
+    const std::string pre = "h" + std::to_string(l) + ".";
+    act_t* u = m->at<act_t>(L.u);
+    act_t* qkv = m->at<act_t>(L.qkv);
+    act_t* o = m->at<act_t>(L.o);
+    act_t* u2 = m->at<act_t>(L.u2);
+    rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps);
+    LAUNCH_CHECK();
+    TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a)));
+    rope_qknorm_fwd_kernel<act_t, act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+        qkv, m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
+        c.v_rows ? reinterpret_cast<const act_t*>(m->base + p.hv) : nullptr, m->at<int32_t>(p.rows_v), N,
+        c.seq_len, H, hd, c.qk_norm, c.norm_eps);
+    LAUNCH_CHECK();
+    TRY(attention_fwd<act_t>(m, qkv, o, m->at<float>(L.lse)));
+    TRY(gemm(g, N, d, a, op_k(o, a), op_k(W(pre + "wo"), a), epi(EPI_ACCUM_F32, x, d, 1)));
+    rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps);
+    LAUNCH_CHECK();
+    TRY(gemm(g, N, F, d, op_k(u2, d), op_k(W(pre + "w1"), d),
+             epi(EPI_RELU2, m->at<act_t>(L.r), F, 0, m->at<act_t>(L.g))));
+    TRY(gemm(g, N, d, F, op_k(m->at<act_t>(L.g), F), op_k(W(pre + "w2"), F), epi(EPI_ACCUM_F32, x, d, 1)));
+  }
+  act_t* xf = m->at<act_t>(p.xf);
+  rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps);
+  ce_prepare_kernel<<<1, 1024, 0, st>>>(targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
+  LAUNCH_CHECK();
+  // chunked LM head + cross-entropy; the head's gradient pieces are formed
+  // here while each logits chunk is live: dxf (fp32) and the pending head
+  // weight gradient, which backward adds into the dense gradient.
+  const act_t* Wlm = W(c.tie_embeddings ? "wte" : "lm_head");
+  float* logits = m->at<float>(p.logits);
+  act_t* dz = m->at<act_t>(p.dz);
+  for (int r0 = 0, ci = 0; r0 < N; r0 += p.chunk, ++ci) {
+    const int rows = (N - r0 < p.chunk) ? (N - r0) : p.chunk;
+    TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), epi(EPI_STORE_F32, logits, V)));
+    ce_chunk_kernel<act_t><<<rows, 512, 0, st>>>(logits, dz, targets + r0, m->at<float>(p.tok_loss) + r0, V,
+                                                 c.softcap, m->at<float>(p.ce_scale), err);
+    LAUNCH_CHECK();
+    TRY(gemm(g, rows, d, V, op_k(dz, V), op_mn(Wlm, d), epi(EPI_STORE_F32, m->at<float>(p.dxf) + (long long)r0 * d, d)));
+    TRY(gemm(g, V, d, rows, op_mn(dz, V), op_mn(xf + (long long)r0 * d, d),
+             epi(EPI_ACCUM_F32, m->at<float>(p.pending), d, ci > 0), true));
+  }
+  loss_reduce_kernel<<<1, 1024, 0, st>>>(m->at<float>(p.tok_loss), N, m->at<int>(p.ce_count), loss_dev, err);
+  LAUNCH_CHECK();
+  m->have_fwd = true;
+  return GPT_OK;
+}
+
+// ======================================================================== backward
+template <typename act_t>
+static int backward_impl(gpt_model* m, float lr) {
+  const gpt_config& c = m->cfg;
+  const Plan& p = m->plan;
+  const bool b16 = cfg_bf16(c);
+  cudaStream_t st = m->st;
+  const int N = c.micro_batch * c.seq_len;
+  const int d = c.d_model, H = c.n_head, hd = c.head_dim, a = H * hd, F = c.d_ff, V = c.vocab;
+  unsigned* err = m->err();
+  GemmCtx g{b16, m->at<float>(p.splitk), p.splitk_elems, err, st};
+  auto W = [&](const std::string& nm) -> const act_t* {
+    const DenseTensor* t = find_dense(m, nm);
+    return b16 ? reinterpret_cast<const act_t*>(m->at<bf16>(p.Plp) + t->off)
+               : reinterpret_cast<const act_t*>(m->at<float>(p.P) + t->off);
+  };
+  auto Gp = [&](const std::string& nm) -> float* { return m->at<float>(p.G) + find_dense(m, nm)->off; };
+  const int beta = m->micro > 0;
+  const int rows_blocks = grid_for((long long)N * 32, 256);
+  // LM-head weight gradient staged by the forward pass
+  float* g_head = Gp(c.tie_embeddings ? "wte" : "lm_head");
+  accumulate_kernel<<<4 * device_sms(), 256, 0, st>>>(g_head, m->at<float>(p.pending), (long long)V * d, beta);
+  if (!c.tie_embeddings && !beta) CUDA_TRY(cudaMemsetAsync(Gp("wte"), 0, (size_t)V * d * 4, st));
+  float* dx = m->at<float>(p.dx);
+  act_t* dx_lp = m->at<act_t>(p.dx_lp);
+  float* du = m->at<float>(p.du);
+  act_t* dqkv = m->at<act_t>(p.dqkv);
+  act_t* da = m->at<act_t>(p.da);
+  act_t* dout = m->at<act_t>(p.dout);
+  rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(m->at<float>(p.dxf), m->at<act_t>(p.xf),
+                                                        m->at<float>(p.rstd_f), dx, dx_lp, N, d, 0);
+  LAUNCH_CHECK();
+  for (int l = c.n_layer - 1; l >= 0; --l) {
+    const LayerActs& L = p.layers[l];
+    const std::string pre = "h" + std::to_string(l) + ".";
+    // ---- MLP: x += relu(u2 W1^T)^2 W2^T
+    TRY(gemm(g, d, F, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.g), F), epi(EPI_ACCUM_F32, Gp(pre + "w2"), F, beta), true));
+    TRY(gemm(g, N, F, d, op_k(dx_lp, d), op_mn(W(pre + "w2"), F), epi(EPI_DRELU2, da, F, 0, nullptr, m->at<act_t>(L.r))));
+    TRY(gemm(g, F, d, N, op_mn(da, F), op_mn(m->at<act_t>(L.u2), d), epi(EPI_ACCUM_F32, Gp(pre + "w1"), d, beta), true));
+    TRY(gemm(g, N, d, F, op_k(da, F), op_mn(W(pre + "w1"), d), epi(EPI_STORE_F32, du, d)));
+    rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1);
+    LAUNCH_CHECK();
+    // ---- attention: x += o Wo^T
+    TRY(gemm(g, d, a, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.o), a), epi(EPI_ACCUM_F32, Gp(pre + "wo"), a, beta), true));
+    TRY(gemm(g, N, a, d, op_k(dx_lp, d), op_mn(W(pre + "wo"), a), epi(EPI_STORE, dout, a)));
+    TRY(attention_bwd<act_t>(m, m->at<act_t>(L.qkv), m->at<act_t>(L.o), dout, m->at<float>(L.lse),
+                             m->at<float>(p.Dattn), dqkv));
+    rope_qknorm_bwd_kernel<act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+        dqkv, m->at<act_t>(L.qkv), m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
+        c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
+    LAUNCH_CHECK();
+    TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true));
+    TRY(gemm(g, N, d, 3 * a, op_k(dqkv, 3 * a), op_mn(W(pre + "wqkv"), d), epi(EPI_STORE_F32, du, d)));
+    rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1);
+    LAUNCH_CHECK();
+  }
+  // dx now holds dL/dx0 per position.
+  const SortWs w = sort_ws(m);
+  {
+    // token embedding gradient, bucketed by token id
+    const uint32_t* skeys;
+    const int32_t* perm;
+    TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
+    const long long maxp = (long long)N + N / PIECE + 2, maxl = N / PIECE + 2;
+    emb_piece_kernel<act_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
+        Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, w.pstart, w.plen, w.pslot,
+        w.counters, w.partial);
+    emb_long_kernel<<<grid_for(maxl * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, w.seg_start, w.lfirst,
+                                                             w.lnslots, w.lseg, w.counters, w.partial);
+    LAUNCH_CHECK();
+  }
+  const float lr_t = lr * c.lr_mult_table;
+  if (c.v_rows)
+    TRY(table_update<act_t>(w, reinterpret_cast<act_t*>(m->base + p.hv), m->at<float>(p.hv_state), c.v_rows, a,
+                            m->at<int32_t>(p.rows_v), m->at<float>(p.gv), N, lr_t, c.table_beta, c.table_eps,
+                            nullptr, nullptr, err, st));
+  if (c.x0_rows)
+    TRY(table_update<act_t>(w, reinterpret_cast<act_t*>(m->base + p.hx), m->at<float>(p.hx_state), c.x0_rows, d,
+                            m->at<int32_t>(p.rows_x), dx, N, lr_t, c.table_beta, c.table_eps, nullptr, nullptr, err, st));
+  // ---- dense step every grad_accum calls
+  m->micro += 1;
+  if (m->micro == c.grad_accum) {
+    m->micro = 0;
+    m->step_t += 1;
+    float* coef = nullptr;
+    if (c.grad_clip > 0.f) {
+      sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, st>>>(m->at<float>(p.G), p.dense_n, m->at<double>(p.norm_part));
+      clip_coef_kernel<<<1, 256, 0, st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, c.grad_clip,
+                                         m->at<float>(p.clip_coef), m->at<float>(p.grad_norm), err);
+      LAUNCH_CHECK();
+      coef = m->at<float>(p.clip_coef);
+    }
+    AdamArgs aa;
+    aa.p = m->at<float>(p.P); aa.g = m->at<float>(p.G); aa.m = m->at<float>(p.M); aa.v = m->at<float>(p.V);
+    aa.p_lp = b16 ? m->at<bf16>(p.Plp) : nullptr;
+    aa.n = p.dense_n; aa.e_end = p.e_end; aa.h_end = p.h_end;
+    aa.lr_e = lr * c.lr_mult_embed; aa.lr_h = lr * c.lr_mult_head; aa.lr_m = lr * c.lr_mult_matrix;
+    aa.b1 = c.adam_b1; aa.b2 = c.adam_b2; aa.eps = c.adam_eps; aa.wd = c.weight_decay;
+    aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
+    aa.bc2 = (float)(1.0 - pow((double)c.adam_b2, (double)m->step_t));
+    aa.clip = coef;
+    adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
+    LAUNCH_CHECK();
+  }
+  m->have_fwd = false;
+  return GPT_OK;
+}
+
+extern "C" int gpt_forward_loss(gpt_model* m, const int32_t* tokens, const int32_t* targets, float* loss_dev) {
+  if (!m || !tokens || !targets || !loss_dev) return fail(GPT_ERR_ARG, "null argument");
+  if (cfg_bf16(m->cfg)) return forward_impl<bf16>(m, tokens, targets, loss_dev);
+  return forward_impl<float>(m, tokens, targets, loss_dev);
+}
+
+extern "C" int gpt_backward_step(gpt_model* m, float lr) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  if (!m->have_fwd) return fail(GPT_ERR_STATE, "gpt_backward_step needs a preceding gpt_forward_loss");
+  if (!std::isfinite(lr)) return fail(GPT_ERR_ARG, "learning rate not finite");
+  if (cfg_bf16(m->cfg)) return backward_impl<bf16>(m, lr);
+  return backward_impl<float>(m, lr);
+}
+
+// ======================================================================== standalone ngram
+extern "C" int ngram_hash(const int32_t* tokens, int B, int T, int vocab, unsigned long long p1,
+                          unsigned long long p2, long long rows, int32_t* rows_out, void* stream) {
+  if (!tokens || !rows_out || B < 0 || T < 0 || vocab < 1 || rows < 1 || rows > 0x7fffffffLL)
+    return fail(GPT_ERR_ARG, "ngram_hash: bad argument");
+  if ((long long)B * T == 0) return GPT_OK;
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  ngram_hash_kernel<<<grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream>>>(
+      tokens, B, T, vocab, p1, p2, rows, rows_out, 1, nullptr, err);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+extern "C" int ngram_gather(const int32_t* rows, int n, const void* table, long long n_rows, int d, int dtype,
+                            void* out, int accumulate, void* stream) {
+  if (!rows || !table || !out || n < 0 || n_rows < 1 || d < 4 || d % 4 || d > 2048)
+    return fail(GPT_ERR_ARG, "ngram_gather: bad argument (d must be a multiple of 4, <= 2048)");
+  if (n == 0) return GPT_OK;
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  const int grid = grid_for((long long)n * 32, 256);
+  if (dtype == GPT_DTYPE_BF16)
+    ngram_gather_kernel<bf16><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows, d,
+                                                                      (bf16*)out, accumulate, err);
+  else if (dtype == GPT_DTYPE_F32)
+    ngram_gather_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const float*)table, n_rows, d,
+                                                                       (float*)out, accumulate, err);
+  else
+    return fail(GPT_ERR_ARG, "ngram_gather: dtype must be F32 or BF16");
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+struct NgramWsPlan {
+  size_t ka, kb, va, vb, counts, seg_start, pstart, plen, pseg, pslot, lfirst, lnslots, lseg, counters, partial, total;
+};
+
+static NgramWsPlan ngram_ws_plan(int n, int d) {
+  NgramWsPlan w;
+  Carver cv;
+  const long long nblk = (n + RADIX_TILE - 1) / RADIX_TILE;
+  const long long maxp = (long long)n + n / PIECE + 2, maxl = n / PIECE + 2, maxslots = 2 * (n / PIECE) + 4;
+  w.ka = cv.take((size_t)n * 4); w.kb = cv.take((size_t)n * 4);
+  w.va = cv.take((size_t)n * 4); w.vb = cv.take((size_t)n * 4);
+  w.counts = cv.take(256 * nblk * 4);
+  w.seg_start = cv.take(((size_t)n + 1) * 4);
+  w.pstart = cv.take(maxp * 4); w.plen = cv.take(maxp * 4); w.pseg = cv.take(maxp * 4); w.pslot = cv.take(maxp * 4);
+  w.lfirst = cv.take(maxl * 4); w.lnslots = cv.take(maxl * 4); w.lseg = cv.take(maxl * 4);
+  w.counters = cv.take(16);
+  w.partial = cv.take(maxslots * (size_t)d * 4);
+  w.total = cv.take(0);
+  return w;
+}
+
+extern "C" int ngram_sparse_update_workspace_bytes(int n, int d, size_t* bytes) {
+  if (!bytes || n < 0 || d < 4) return fail(GPT_ERR_ARG, "ngram_sparse_update_workspace_bytes: bad argument");
+  *bytes = ngram_ws_plan(n, d).total;
+  return GPT_OK;
+}
+
+extern "C" int ngram_sparse_update(void* table, float* row_state, long long n_rows, int d, int dtype,
+                                   const int32_t* rows, const float* grad, int n, float lr, float beta, float eps,
+                                   int32_t* updated_rows_out, int* n_updated_out_dev, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  if (!table || !row_state || !rows || !grad || n < 0 || n_rows < 1 || n_rows > 0x7fffffffLL || d < 4 ||
+      d % 4 || d > 2048)
+    return fail(GPT_ERR_ARG, "ngram_sparse_update: bad argument (d must be a multiple of 4, <= 2048)");
+  if (dtype != GPT_DTYPE_F32 && dtype != GPT_DTYPE_BF16) return fail(GPT_ERR_ARG, "ngram_sparse_update: bad dtype");
+  if (n == 0) {
+    if (n_updated_out_dev) CUDA_TRY(cudaMemsetAsync(n_updated_out_dev, 0, 4, (cudaStream_t)stream));
+    return GPT_OK;
+  }
+  const NgramWsPlan pl = ngram_ws_plan(n, d);
+  if (!workspace || ws_bytes < pl.total)
+    return fail(GPT_ERR_WORKSPACE, "ngram_sparse_update: workspace %zu < %zu bytes", ws_bytes, pl.total);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(GPT_ERR_ARG, "workspace not 256-byte aligned");
+  uint8_t* b = static_cast<uint8_t*>(workspace);
+  SortWs w;
+  w.ka = (uint32_t*)(b + pl.ka); w.kb = (uint32_t*)(b + pl.kb);
+  w.va = (int32_t*)(b + pl.va); w.vb = (int32_t*)(b + pl.vb);
+  w.counts = (uint32_t*)(b + pl.counts);
+  w.seg_start = (int32_t*)(b + pl.seg_start); w.pstart = (int32_t*)(b + pl.pstart);
+  w.plen = (int32_t*)(b + pl.plen); w.pseg = (int32_t*)(b + pl.pseg); w.pslot = (int32_t*)(b + pl.pslot);
+  w.lfirst = (int32_t*)(b + pl.lfirst); w.lnslots = (int32_t*)(b + pl.lnslots); w.lseg = (int32_t*)(b + pl.lseg);
+  w.counters = (int32_t*)(b + pl.counters); w.partial = (float*)(b + pl.partial);
+  cudaStream_t st = (cudaStream_t)stream;
+  // rows outside the table are rejected on the device before bucketing
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  if (dtype == GPT_DTYPE_BF16)
+    return table_update<bf16>(w, (bf16*)table, row_state, n_rows, d, rows, grad, n, lr, beta, eps,
+                              updated_rows_out, n_updated_out_dev, err, st);
+  return table_update<float>(w, (float*)table, row_state, n_rows, d, rows, grad, n, lr, beta, eps,
+                             updated_rows_out, n_updated_out_dev, err, st);
+}
+
+extern "C" int ngram_sync_status(void* stream) {
+  CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned w = 0;
+  CUDA_TRY(cudaMemcpyFromSymbol(&w, g_ngram_err, 4));
+  if (w) {
+    unsigned z = 0;
+    CUDA_TRY(cudaMemcpyToSymbol(g_ngram_err, &z, 4));
+  }
+  if (w & GPT_EBIT_INPUT) return fail(GPT_ERR_INPUT, "row or token id out of range");
+  if (w & GPT_EBIT_TIMEOUT) return fail(GPT_ERR_TIMEOUT, "a kernel's bounded wait gave up");
+  return GPT_OK;
+}
+
+// ======================================================================== kernel-level test entry
+extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmajor, const void* B,
+                              long long ldb, int b_kmajor, float* C, long long ldc, int beta, int splits,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || ldc < N)
+    return fail(GPT_ERR_ARG, "gptx_gemm_bf16: bad argument");
+  if (splits < 1) splits = 1;
+  if (splits > 1 && (!workspace || ws_bytes < (size_t)splits * M * N * 4))
+    return fail(GPT_ERR_WORKSPACE, "gptx_gemm_bf16: split-K needs splits*M*N*4 bytes of workspace");
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  GemmEpilogue e = epi(EPI_ACCUM_F32, C, ldc, beta);
+  GemmOperand a{A, lda, a_kmajor ? 1 : 0}, b{B, ldb, b_kmajor ? 1 : 0};
+  if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, (cudaStream_t)stream);
+  return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, (cudaStream_t)stream);
+}

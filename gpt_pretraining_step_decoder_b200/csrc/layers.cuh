@@ -1,0 +1,526 @@
+// layers.cuh -- memory-bound layer kernels of the decoder step.
+//
+// One warp per row (token) for the row-wise normalisations; 128-bit (fp32) or
+// 64-bit (bf16) vector accesses along the row; reductions with warp shuffles.
+// act_t is the activation type (float in the fp32 mode, bf16 otherwise); the
+// residual stream and its gradient stay fp32 in both modes.
+#pragma once
+#include "common.cuh"
+
+constexpr int MAXV = 16;  // vec4 chunks per lane: rows up to 32 * 4 * 16 = 2048 wide
+
+// --------------------------------------------------------------------------
+// Token embedding + parameter-free RMSNorm + optional x0 bigram row
+// ("$1000 tier nanochat run", `GPT.forward`: x = norm(wte(idx)); decoder-rtx
+// posts: a 2M-row bigram table "added to x0").
+//   x[t] = wte[tok_t] * rstd_t + Hx[rx_t],   rstd_t = 1/sqrt(mean(wte[tok_t]^2) + eps)
+template <typename w_t, typename tab_t>
+__global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __restrict__ wte,
+                                 const tab_t* __restrict__ hx, const int32_t* __restrict__ rx,
+                                 float* __restrict__ x, float* __restrict__ rstd_out, int N, int d,
+                                 int V, float eps, unsigned* err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= N) return;
+  int id = tok[warp];
+  if (id < 0 || id >= V) {
+    if (lane == 0) set_error(err, GPT_EBIT_INPUT);
+    id = 0;
+  }
+  float v[MAXV][4];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) {
+      load4(wte + (long long)id * d + c, v[j]);
+      ss += v[j][0] * v[j][0] + v[j][1] * v[j][1] + v[j][2] * v[j][2] + v[j][3] * v[j][3];
+    }
+  }
+  ss = warp_sum(ss);
+  const float rstd = rsqrtf(ss / d + eps);
+  if (lane == 0) rstd_out[warp] = rstd;
+  const long long row = hx ? (long long)rx[warp] : 0;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) {
+      float o[4] = {v[j][0] * rstd, v[j][1] * rstd, v[j][2] * rstd, v[j][3] * rstd};
+      if (hx) {
+        float h[4];
+        load4(hx + row * d + c, h);
+        o[0] += h[0]; o[1] += h[1]; o[2] += h[2]; o[3] += h[3];
+      }
+      store4(x + (long long)warp * d + c, o);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// RMSNorm forward ("$1000 tier nanochat run", `norm`: F.rms_norm without
+// affine parameters): u = x * rstd, rstd = 1/sqrt(mean(x^2) + eps).
+template <typename act_t>
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, act_t* __restrict__ u,
+                                   float* __restrict__ rstd_out, int N, int d, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= N) return;
+  const float* xr = x + (long long)warp * d;
+  float v[MAXV][4];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) {
+      load4(xr + c, v[j]);
+      ss += v[j][0] * v[j][0] + v[j][1] * v[j][1] + v[j][2] * v[j][2] + v[j][3] * v[j][3];
+    }
+  }
+  ss = warp_sum(ss);
+  const float rstd = rsqrtf(ss / d + eps);
+  if (lane == 0) rstd_out[warp] = rstd;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) {
+      float o[4] = {v[j][0] * rstd, v[j][1] * rstd, v[j][2] * rstd, v[j][3] * rstd};
+      store4(u + (long long)warp * d + c, o);
+    }
+  }
+}
+
+// RMSNorm backward: dx (+)= rstd * (du - u * mean(du * u)); also writes the
+// activation-typed copy of dx that the next GEMMs read.
+template <typename act_t>
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __restrict__ u,
+                                   const float* __restrict__ rstd, float* __restrict__ dx,
+                                   act_t* __restrict__ dx_lp, int N, int d, int accumulate) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= N) return;
+  const long long base = (long long)warp * d;
+  float g[MAXV][4], y[MAXV][4];
+  float dot = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) {
+      load4(du + base + c, g[j]);
+      load4(u + base + c, y[j]);
+      dot += g[j][0] * y[j][0] + g[j][1] * y[j][1] + g[j][2] * y[j][2] + g[j][3] * y[j][3];
+    }
+  }
+  dot = warp_sum(dot) / d;
+  const float r = rstd[warp];
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) {
+      float o[4];
+      if (accumulate) load4(dx + base + c, o);
+      else o[0] = o[1] = o[2] = o[3] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] += r * (g[j][i] - y[j][i] * dot);
+      store4(dx + base + c, o);
+      store4(dx_lp + base + c, o);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// RoPE cos/sin table: theta[t, i] = t * base^(-2i/hd) for i < hd/2
+// ("$1000 tier nanochat run", `_precompute_rotary_embeddings`), evaluated in
+// double precision and stored fp32 (the pages keep a bf16 table).
+__global__ void rope_table_kernel(float* __restrict__ cs, int T, int hd, double base) {
+  const int h = hd / 2;
+  const long long total = (long long)T * h;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / h), j = (int)(i % h);
+    const double inv_freq = 1.0 / pow(base, (2.0 * j) / hd);
+    const double th = t * inv_freq;
+    cs[2 * i] = (float)cos(th);
+    cs[2 * i + 1] = (float)sin(th);
+  }
+}
+
+// Per (position, head): rotate q and k ("$1000 tier nanochat run",
+// `apply_rotary_emb`: y1 = x1 cos + x2 sin, y2 = -x1 sin + x2 cos), then
+// RMSNorm each head (QK-norm, `q, k = norm(q), norm(k)` after RoPE), and add
+// the value-table row to v (decoder-rtx posts: 1M-row table "added to
+// values").  In place on qkv [N, 3a]; rstd_q/rstd_k [N, H].
+template <typename act_t, typename tab_t>
+__global__ void rope_qknorm_fwd_kernel(act_t* __restrict__ qkv, const float* __restrict__ cs,
+                                       float* __restrict__ rstd_q, float* __restrict__ rstd_k,
+                                       const tab_t* __restrict__ hv, const int32_t* __restrict__ rv,
+                                       int N, int T, int H, int hd, int qk_norm, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= N * H) return;
+  const int n = warp / H, h = warp % H, t = n % T;
+  const int a = H * hd, half = hd / 2;
+  act_t* row = qkv + (long long)n * 3 * a;
+  for (int which = 0; which < 2; ++which) {
+    act_t* x = row + which * a + h * hd;
+    float y1[2], y2[2];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = lane + 32 * k;
+      y1[k] = y2[k] = 0.f;
+      if (i < half) {
+        const float c = cs[2 * ((long long)t * half + i)], s = cs[2 * ((long long)t * half + i) + 1];
+        const float x1 = to_f(x[i]), x2 = to_f(x[i + half]);
+        y1[k] = x1 * c + x2 * s;
+        y2[k] = -x1 * s + x2 * c;
+        ss += y1[k] * y1[k] + y2[k] * y2[k];
+      }
+    }
+    float r = 1.f;
+    if (qk_norm) {
+      ss = warp_sum(ss);
+      r = rsqrtf(ss / hd + eps);
+      if (lane == 0) (which == 0 ? rstd_q : rstd_k)[(long long)n * H + h] = r;
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = lane + 32 * k;
+      if (i < half) {
+        x[i] = from_f<act_t>(y1[k] * r);
+        x[i + half] = from_f<act_t>(y2[k] * r);
+      }
+    }
+  }
+  if (hv) {
+    act_t* v = row + 2 * a + h * hd;
+    const tab_t* src = hv + (long long)rv[n] * a + h * hd;
+    for (int i = lane; i < hd; i += 32) v[i] = from_f<act_t>(to_f(v[i]) + to_f(src[i]));
+  }
+}
+
+// Backward of the above, in place on dqkv: QK-norm backward with the saved
+// normalised q/k and rstd, then the inverse rotation (rotation by -theta).
+// The v part is summed over layers into gv (fp32 [N, a]) for the value table.
+template <typename act_t>
+__global__ void rope_qknorm_bwd_kernel(act_t* __restrict__ dqkv, const act_t* __restrict__ qkv,
+                                       const float* __restrict__ cs, const float* __restrict__ rstd_q,
+                                       const float* __restrict__ rstd_k, float* __restrict__ gv,
+                                       int gv_accumulate, int N, int T, int H, int hd, int qk_norm) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= N * H) return;
+  const int n = warp / H, h = warp % H, t = n % T;
+  const int a = H * hd, half = hd / 2;
+  for (int which = 0; which < 2; ++which) {
+    act_t* g = dqkv + (long long)n * 3 * a + which * a + h * hd;
+    const act_t* y = qkv + (long long)n * 3 * a + which * a + h * hd;
+    float g1[2], g2[2], y1[2], y2[2];
+    float dot = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = lane + 32 * k;
+      g1[k] = g2[k] = y1[k] = y2[k] = 0.f;
+      if (i < half) {
+        g1[k] = to_f(g[i]); g2[k] = to_f(g[i + half]);
+        y1[k] = to_f(y[i]); y2[k] = to_f(y[i + half]);
+        dot += g1[k] * y1[k] + g2[k] * y2[k];
+      }
+    }
+    float r = 1.f;
+    if (qk_norm) {
+      dot = warp_sum(dot) / hd;
+      r = (which == 0 ? rstd_q : rstd_k)[(long long)n * H + h];
+    } else {
+      dot = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = lane + 32 * k;
+      if (i < half) {
+        const float d1 = r * (g1[k] - y1[k] * dot), d2 = r * (g2[k] - y2[k] * dot);
+        const float c = cs[2 * ((long long)t * half + i)], s = cs[2 * ((long long)t * half + i) + 1];
+        g[i] = from_f<act_t>(d1 * c - d2 * s);
+        g[i + half] = from_f<act_t>(d1 * s + d2 * c);
+      }
+    }
+  }
+  if (gv) {
+    const act_t* dv = dqkv + (long long)n * 3 * a + 2 * a + h * hd;
+    float* dst = gv + (long long)n * a + h * hd;
+    for (int i = lane; i < hd; i += 32) dst[i] = (gv_accumulate ? dst[i] : 0.f) + to_f(dv[i]);
+  }
+}
+
+// --------------------------------------------------------------------------
+// Cross-entropy over one chunk of rows of fp32 logits [rows, V], fused
+// forward and backward ("$1000 tier nanochat run", `GPT.forward`: optional
+// softcap c*tanh(z/c), logits in fp32, F.cross_entropy(ignore_index=-1)).
+//   loss_t = logsumexp(z_t) - z_t[y_t]           (0 for ignored targets)
+//   dlogits = (softmax(z_t) - onehot(y_t)) * scale * dz/dlogit
+// scale = 1 / (n_valid * grad_accum) is read from the device.
+template <typename act_t>
+__global__ void __launch_bounds__(512) ce_chunk_kernel(float* __restrict__ logits,
+                                                       act_t* __restrict__ dz,
+                                                       const int32_t* __restrict__ targets,
+                                                       float* __restrict__ tok_loss, int V,
+                                                       float softcap, const float* __restrict__ scale_dev,
+                                                       unsigned* err) {
+  __shared__ float sh[32];
+  const long long row = blockIdx.x;
+  float* z = logits + row * V;
+  act_t* g = dz + row * V;
+  int y = targets[row];
+  if (y < -1 || y >= V) {
+    if (threadIdx.x == 0) set_error(err, GPT_EBIT_INPUT);
+    y = -1;
+  }
+  float mx = -INFINITY;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) {
+    float v = z[i];
+    if (softcap > 0.f) { v = softcap * tanhf(v / softcap); z[i] = v; }
+    mx = fmaxf(mx, v);
+  }
+  mx = block_max(mx, sh);
+  float se = 0.f;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) se += expf(z[i] - mx);
+  se = block_sum(se, sh);
+  const float lse = mx + logf(se);
+  if (threadIdx.x == 0) {
+    const float l = (y >= 0) ? (lse - z[y]) : 0.f;
+    tok_loss[row] = l;
+    if (y >= 0 && !isfinite(l)) set_error(err, GPT_EBIT_NONFINITE);
+  }
+  const float sc = (y >= 0) ? *scale_dev : 0.f;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) {
+    const float zi = z[i];
+    float gi = (expf(zi - lse) - (i == y ? 1.f : 0.f)) * sc;
+    if (softcap > 0.f) { const float tt = zi / softcap; gi *= (1.f - tt * tt); }
+    g[i] = from_f<act_t>(gi);
+  }
+}
+
+// Counts non-ignored targets and sets scale = 1/(count * A) (single block).
+__global__ void ce_prepare_kernel(const int32_t* __restrict__ targets, int N, int A,
+                                  float* __restrict__ scale_out, int* __restrict__ count_out) {
+  __shared__ float sh[32];
+  float c = 0.f;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) c += (targets[i] >= 0) ? 1.f : 0.f;
+  c = block_sum(c, sh);
+  if (threadIdx.x == 0) {
+    const int n = (int)(c + 0.5f);
+    *count_out = n;
+    *scale_out = n > 0 ? 1.f / ((float)n * (float)A) : 0.f;
+  }
+}
+
+// loss = sum(tok_loss) / count, summed in a fixed order (single block, fp64).
+__global__ void loss_reduce_kernel(const float* __restrict__ tok_loss, int N,
+                                   const int* __restrict__ count, float* __restrict__ loss_out,
+                                   unsigned* err) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) s += tok_loss[i];
+  s = warp_sum_d(s);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) sh[wid] = s;
+  __syncthreads();
+  if (wid == 0) {
+    double r = (lane < (int)(blockDim.x >> 5)) ? sh[lane] : 0.0;
+    r = warp_sum_d(r);
+    if (lane == 0) {
+      const float l = *count > 0 ? (float)(r / *count) : 0.f;
+      *loss_out = l;
+      if (!isfinite(l)) set_error(err, GPT_EBIT_NONFINITE);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// Causal softmax attention, SIMT reference kernels (any head_dim <= 128, any
+// T; fp32 accumulation).  The fp32 mode's attention.  q, k, v are read from
+// qkv [N, 3a]; o is [N, a]; lse [B*H, T] is the log-sum-exp of the scaled
+// scores.  One warp per query row (forward, dq) or key row (dk, dv).
+template <typename act_t>
+__global__ void attn_fwd_simt_kernel(const act_t* __restrict__ qkv, act_t* __restrict__ o,
+                                     float* __restrict__ lse_out, int B, int T, int H, int hd) {
+  extern __shared__ float qs[];  // [warps][hd]
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + wib;
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  if (i >= T) return;
+  const int a = H * hd;
+  const float scale = rsqrtf((float)hd);
+  float* q = qs + wib * hd;
+  const act_t* qrow = qkv + ((long long)b * T + i) * 3 * a + h * hd;
+  for (int c = lane; c < hd; c += 32) q[c] = to_f(qrow[c]);
+  __syncwarp();
+  float m = -INFINITY, l = 0.f;
+  for (int j = lane; j <= i; j += 32) {
+    const act_t* krow = qkv + ((long long)b * T + j) * 3 * a + a + h * hd;
+    float s = 0.f;
+    for (int c = 0; c < hd; ++c) s = fmaf(q[c], to_f(krow[c]), s);
+    s *= scale;
+    const float mn = fmaxf(m, s);
+    l = l * expf(m - mn) + expf(s - mn);
+    m = mn;
+  }
+  const float M = warp_max(m);
+  l = (m == -INFINITY) ? 0.f : l * expf(m - M);
+  l = warp_sum(l);
+  const float lse = M + logf(l);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int j0 = 0; j0 <= i; j0 += 32) {
+    const int j = j0 + lane;
+    float p = 0.f;
+    if (j <= i) {
+      const act_t* krow = qkv + ((long long)b * T + j) * 3 * a + a + h * hd;
+      float s = 0.f;
+      for (int c = 0; c < hd; ++c) s = fmaf(q[c], to_f(krow[c]), s);
+      p = expf(s * scale - lse);
+    }
+    const int cnt = min(32, i - j0 + 1);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+      const act_t* vrow = qkv + ((long long)b * T + j0 + jj) * 3 * a + 2 * a + h * hd;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = lane + 32 * k;
+        if (c < hd) acc[k] = fmaf(pj, to_f(vrow[c]), acc[k]);
+      }
+    }
+  }
+  act_t* orow = o + ((long long)b * T + i) * a + h * hd;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = lane + 32 * k;
+    if (c < hd) orow[c] = from_f<act_t>(acc[k]);
+  }
+  if (lane == 0) lse_out[(long long)bh * T + i] = lse;
+}
+
+// D[bh, i] = sum_c dO[i, c] * O[i, c]  (softmax-backward row term)
+template <typename act_t>
+__global__ void attn_bwd_pre_kernel(const act_t* __restrict__ o, const act_t* __restrict__ dout,
+                                    float* __restrict__ Dout, int B, int T, int H, int hd) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= B * T * H) return;
+  const int n = warp / H, h = warp % H, b = n / T, t = n % T;
+  const int a = H * hd;
+  float s = 0.f;
+  for (int c = lane; c < hd; c += 32)
+    s += to_f(o[(long long)n * a + h * hd + c]) * to_f(dout[(long long)n * a + h * hd + c]);
+  s = warp_sum(s);
+  if (lane == 0) Dout[((long long)b * H + h) * T + t] = s;
+}
+
+// dq for one query row per warp: dq = scale * sum_j P_ij (dP_ij - D_i) k_j
+template <typename act_t>
+__global__ void attn_bwd_dq_simt_kernel(const act_t* __restrict__ qkv, const act_t* __restrict__ dout,
+                                        const float* __restrict__ lse, const float* __restrict__ Dv,
+                                        act_t* __restrict__ dqkv, int B, int T, int H, int hd) {
+  extern __shared__ float sm[];  // [warps][2*hd]
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + wib;
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  if (i >= T) return;
+  const int a = H * hd;
+  const float scale = rsqrtf((float)hd);
+  float* q = sm + wib * 2 * hd;
+  float* go = q + hd;
+  const long long n = (long long)b * T + i;
+  for (int c = lane; c < hd; c += 32) {
+    q[c] = to_f(qkv[n * 3 * a + h * hd + c]);
+    go[c] = to_f(dout[n * a + h * hd + c]);
+  }
+  __syncwarp();
+  const float L = lse[(long long)bh * T + i], Di = Dv[(long long)bh * T + i];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int j0 = 0; j0 <= i; j0 += 32) {
+    const int j = j0 + lane;
+    float ds = 0.f;
+    if (j <= i) {
+      const act_t* krow = qkv + ((long long)b * T + j) * 3 * a + a + h * hd;
+      const act_t* vrow = krow + a;
+      float s = 0.f, dp = 0.f;
+      for (int c = 0; c < hd; ++c) {
+        s = fmaf(q[c], to_f(krow[c]), s);
+        dp = fmaf(go[c], to_f(vrow[c]), dp);
+      }
+      const float p = expf(s * scale - L);
+      ds = p * (dp - Di);
+    }
+    const int cnt = min(32, i - j0 + 1);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float d = __shfl_sync(0xffffffffu, ds, jj);
+      const act_t* krow = qkv + ((long long)b * T + j0 + jj) * 3 * a + a + h * hd;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = lane + 32 * k;
+        if (c < hd) acc[k] = fmaf(d, to_f(krow[c]), acc[k]);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = lane + 32 * k;
+    if (c < hd) dqkv[n * 3 * a + h * hd + c] = from_f<act_t>(acc[k] * scale);
+  }
+}
+
+// dk, dv for one key row per warp: dv = sum_i P_ij dO_i, dk = scale * sum_i dS_ij q_i
+template <typename act_t>
+__global__ void attn_bwd_dkdv_simt_kernel(const act_t* __restrict__ qkv, const act_t* __restrict__ dout,
+                                          const float* __restrict__ lse, const float* __restrict__ Dv,
+                                          act_t* __restrict__ dqkv, int B, int T, int H, int hd) {
+  extern __shared__ float sm[];  // [warps][2*hd]
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * (blockDim.x >> 5) + wib;
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  if (j >= T) return;
+  const int a = H * hd;
+  const float scale = rsqrtf((float)hd);
+  float* kk = sm + wib * 2 * hd;
+  float* vv = kk + hd;
+  const long long nj = (long long)b * T + j;
+  for (int c = lane; c < hd; c += 32) {
+    kk[c] = to_f(qkv[nj * 3 * a + a + h * hd + c]);
+    vv[c] = to_f(qkv[nj * 3 * a + 2 * a + h * hd + c]);
+  }
+  __syncwarp();
+  float dk[4] = {0.f, 0.f, 0.f, 0.f}, dv[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i0 = j; i0 < T; i0 += 32) {
+    const int i = i0 + lane;
+    float p = 0.f, ds = 0.f;
+    if (i < T) {
+      const long long ni = (long long)b * T + i;
+      const act_t* qrow = qkv + ni * 3 * a + h * hd;
+      const act_t* grow = dout + ni * a + h * hd;
+      float s = 0.f, dp = 0.f;
+      for (int c = 0; c < hd; ++c) {
+        s = fmaf(to_f(qrow[c]), kk[c], s);
+        dp = fmaf(to_f(grow[c]), vv[c], dp);
+      }
+      p = expf(s * scale - lse[(long long)bh * T + i]);
+      ds = p * (dp - Dv[(long long)bh * T + i]);
+    }
+    const int cnt = min(32, T - i0);
+    for (int ii = 0; ii < cnt; ++ii) {
+      const float pi = __shfl_sync(0xffffffffu, p, ii);
+      const float di = __shfl_sync(0xffffffffu, ds, ii);
+      const long long ni = (long long)b * T + i0 + ii;
+      const act_t* qrow = qkv + ni * 3 * a + h * hd;
+      const act_t* grow = dout + ni * a + h * hd;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = lane + 32 * k;
+        if (c < hd) {
+          dv[k] = fmaf(pi, to_f(grow[c]), dv[k]);
+          dk[k] = fmaf(di, to_f(qrow[c]), dk[k]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = lane + 32 * k;
+    if (c < hd) {
+      dqkv[nj * 3 * a + a + h * hd + c] = from_f<act_t>(dk[k] * scale);
+      dqkv[nj * 3 * a + 2 * a + h * hd + c] = from_f<act_t>(dv[k]);
+    }
+  }
+}

@@ -1,0 +1,249 @@
+/*
+ * gpt.h -- C ABI of libgpt_b200.so: one training step of a modernised
+ * GPT-2-style decoder with hashed bigram tables, on one B200 (sm_100a).
+ *
+ * What the step computes (each call below names its source passage):
+ *   - forward: token embedding + parameter-free RMSNorm, optional x0 bigram
+ *     table, per layer pre-norm attention (RoPE, QK-norm, causal softmax,
+ *     optional value bigram table) and a ReLU^2 MLP, final RMSNorm, LM head
+ *     (tied or untied, optional logit soft-cap), mean cross-entropy
+ *     ("$1000 tier nanochat run", karpathy/nanochat discussion #8, pasted GPT
+ *     module `GPT.forward`, `Block.forward`, `CausalSelfAttention.forward`;
+ *     modded-nanogpt README, "rotary embeddings, RMSNorm, ReLU^2");
+ *   - a hand-written backward (decoder-rtx posts, "speedrun the backward
+ *     pass"), with the bigram tables' sparse per-row-magnitude optimizer
+ *     applied inside backward so that no table gradient buffer exists
+ *     (decoder-rtx posts: "Dropped .grad buffers from the hash tables and
+ *     inlined the optimizer in their backward math"; "sparse, no first
+ *     moment, and only per-row magnitude");
+ *   - AdamW on the dense weights every `grad_accum` backward calls
+ *     (nanochat `setup_optimizers`: betas (0.8, 0.95), eps 1e-10).
+ *
+ * Conventions shared by every entry point:
+ *   - Memory: the caller allocates all device memory.  A model lives in one
+ *     caller-owned device arena of gpt_workspace_bytes() bytes, which the
+ *     library carves and never frees; the library itself calls no cudaMalloc.
+ *     Host-side handles are owned by the library and freed by gpt_destroy().
+ *   - Streams: every call enqueues work on the model's CUDA stream (or the
+ *     stream argument) and returns without synchronising, unless noted.
+ *   - Errors: every function returns an int status, GPT_OK (0) on success.
+ *     Argument and configuration errors are detected on the host before any
+ *     work is enqueued.  Faults found by kernels (token id out of range,
+ *     non-finite loss, a bounded wait that gave up) set a device error word
+ *     instead of trapping; it is reported by the next gpt_sync_status() /
+ *     ngram_sync_status().  gpt_last_error() gives a thread-local message.
+ *   - Layouts: row-major; token ids and targets are int32 [B, T]; a target of
+ *     -1 is ignored by the loss.  Linear weights are (out, in): y = x W^T.
+ */
+#ifndef GPT_B200_H
+#define GPT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define GPT_OK             0
+#define GPT_ERR_ARG        1  /* null pointer, bad size, unknown name        */
+#define GPT_ERR_CONFIG     2  /* unsupported or inconsistent configuration   */
+#define GPT_ERR_WORKSPACE  3  /* arena or workspace smaller than required    */
+#define GPT_ERR_STATE      4  /* call out of order (backward without forward) */
+#define GPT_ERR_INPUT      5  /* token/target/row id out of range (device)   */
+#define GPT_ERR_NONFINITE  6  /* loss or gradient norm not finite (device)   */
+#define GPT_ERR_CUDA       7  /* a CUDA runtime call failed                  */
+#define GPT_ERR_TIMEOUT    8  /* a kernel's bounded wait gave up (device)    */
+
+/* ---- element types --------------------------------------------------- */
+#define GPT_DTYPE_F32   0   /* fp32 everywhere, SIMT FFMA, no TF32 (tight parity mode) */
+#define GPT_DTYPE_BF16  1   /* bf16 activations and GEMM operands, fp32 accumulate,
+                               fp32 master weights and optimizer state            */
+#define GPT_DTYPE_I32   2
+
+/* ---- tensor kinds for gpt_tensor() ----------------------------------- */
+#define GPT_KIND_PARAM      0  /* master value (fp32 dense; tables in the model dtype) */
+#define GPT_KIND_GRAD       1  /* fp32 accumulated dense gradient of the last step     */
+#define GPT_KIND_ADAM_M     2  /* fp32 AdamW first moment                               */
+#define GPT_KIND_ADAM_V     3  /* fp32 AdamW second moment                              */
+#define GPT_KIND_ROW_STATE  4  /* fp32 per-row second moment of a bigram table          */
+#define GPT_KIND_PARAM_LP   5  /* bf16 copy read by the GEMMs (bf16 mode only)          */
+#define GPT_KIND_ACT        6  /* named activation buffers of the last forward          */
+
+/*
+ * Model configuration (plain old data).  Fields the pages do not fix carry
+ * this library's reading: norm_eps = 1.1920929e-7 (fp32 machine epsilon,
+ * PyTorch's default for F.rms_norm without eps), bigram hash constants
+ * p1 = 2654435761, p2 = 2246822519, table beta 0.95 / eps 1e-10.
+ * Constraints: d_model == n_head * head_dim, n_kv_head == n_head (or 0),
+ * head_dim even; in bf16 mode head_dim == 128 and d_model, d_ff, vocab are
+ * multiples of 64; x0_rows / v_rows are 0 (table absent) or >= 1.
+ */
+typedef struct gpt_config {
+  int n_layer, d_model, n_head, head_dim, n_kv_head, d_ff, vocab, seq_len, micro_batch;
+  int grad_accum;         /* A >= 1 backward calls per AdamW step                */
+  int dtype;              /* GPT_DTYPE_F32 or GPT_DTYPE_BF16                      */
+  int tie_embeddings;     /* 1: LM head shares the token embedding                */
+  int qk_norm;            /* 1: RMSNorm each q/k head after RoPE                  */
+  float rope_base;        /* 10000                                                */
+  float norm_eps;         /* RMSNorm epsilon                                      */
+  float softcap;          /* 0 = off; c > 0: z = c * tanh(z / c)                  */
+  float init_std;         /* N(0, init_std) initialisation of every weight        */
+  float adam_b1, adam_b2, adam_eps, weight_decay;
+  float grad_clip;        /* 0 = off; else global L2 clip of the dense gradient   */
+  float lr_mult_embed, lr_mult_head, lr_mult_matrix, lr_mult_table;
+  long long x0_rows;      /* rows of the table added to x0 (0 = none)             */
+  long long v_rows;       /* rows of the table added to the values (0 = none)     */
+  float table_beta, table_eps;
+  unsigned long long hash_p1, hash_p2;
+  int lm_chunk_rows;      /* rows per LM-head/cross-entropy chunk; 0 = default    */
+} gpt_config;
+
+typedef struct gpt_model gpt_model;
+
+/* Fill *cfg with the defaults above (tiny fp32 decoder shape).  Host only. */
+int gpt_default_config(gpt_config* cfg);
+
+/* Bytes of device arena gpt_create() needs for cfg.  Host only. */
+int gpt_workspace_bytes(const gpt_config* cfg, size_t* bytes);
+
+/*
+ * Create a model inside `arena` (device pointer, 256-byte aligned, at least
+ * gpt_workspace_bytes() bytes, owned by the caller and kept alive until
+ * gpt_destroy).  Weights and tables are initialised on the device to
+ * N(0, init_std) from a counter-based generator (Philox-4x32-10) keyed by
+ * `seed`; optimizer and row states start at zero.  `cuda_stream` is a
+ * cudaStream_t (NULL = legacy default stream).  Enqueues the initialisation
+ * and returns; *out receives the host handle.
+ */
+int gpt_create(const gpt_config* cfg, unsigned long long seed, void* arena,
+               size_t arena_bytes, void* cuda_stream, gpt_model** out);
+
+/* Release the host handle (the arena stays the caller's).  Synchronises the stream. */
+int gpt_destroy(gpt_model* m);
+
+/* Change the stream later calls enqueue on. */
+int gpt_set_stream(gpt_model* m, void* cuda_stream);
+
+/*
+ * Forward pass and loss of one micro-batch ("$1000 tier nanochat run",
+ * `GPT.forward` with targets).  tokens_dev, targets_dev: device int32
+ * [micro_batch, seq_len]; targets may be -1 (ignored).  loss_dev: device
+ * float, receives the mean cross-entropy over non-ignored targets (0 when
+ * there are none).  Activations for the backward pass are kept in the arena.
+ * Out-of-range ids set GPT_ERR_INPUT on the device error word.
+ */
+int gpt_forward_loss(gpt_model* m, const int32_t* tokens_dev, const int32_t* targets_dev,
+                     float* loss_dev);
+
+/*
+ * Backward pass of the last forward, scaled by 1/grad_accum (nanochat training
+ * loop: loss / gradient_accumulation_steps).  Dense gradients accumulate in
+ * fp32 (the first backward of a step overwrites).  Both bigram tables are
+ * updated in place from this micro-batch's gradient before the call returns
+ * (x0 table from dL/dx0 per position, value table from the sum over layers of
+ * dL/dv), with learning rate lr * lr_mult_table.  On every grad_accum-th call
+ * the optional global-norm clip and AdamW (learning rate lr * the group's
+ * multiplier) are applied to the dense weights; the gradient buffers keep
+ * that step's accumulated gradient until the next step starts.
+ * Returns GPT_ERR_STATE when no forward precedes it.
+ */
+int gpt_backward_step(gpt_model* m, float lr);
+
+/* Dense (matmul + embedding) and table parameter counts.  Host only. */
+int gpt_num_params(const gpt_model* m, long long* dense, long long* table);
+
+/* Training FLOPs per token, 6 * matmul params + 12 * L * H * hd * T (nanochat
+ * `estimate_flops`, PaLM form; the LM-head matrix counted once).  Host only. */
+int gpt_flops_per_token(const gpt_config* cfg, long long* flops, long long* flops_causal);
+
+/*
+ * Look up a named tensor inside the arena for export / import.  Names:
+ * "wte", "lm_head" (untied only), "h<l>.wqkv" [3*H*hd, d] (rows q|k|v),
+ * "h<l>.wo" [d, H*hd], "h<l>.w1" [d_ff, d], "h<l>.w2" [d, d_ff], "hx", "hv";
+ * kind GPT_KIND_ACT: "per_token_loss" [B, T] fp32, "rows_x" / "rows_v" [B, T]
+ * int32.  Writes the device pointer, its element type and up to four dims
+ * (unused dims are 1).  Host only, no synchronisation.  After writing
+ * PARAM tensors from outside, call gpt_params_changed().
+ */
+int gpt_tensor(gpt_model* m, const char* name, int kind, void** dev_ptr, int* dtype,
+               long long shape[4]);
+
+/* Re-derive the bf16 GEMM copies from the fp32 master weights (enqueued). */
+int gpt_params_changed(gpt_model* m);
+
+/* Synchronise the model's stream, read and clear the device error word. */
+int gpt_sync_status(gpt_model* m);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* gpt_last_error(void);
+
+/* ---- standalone bigram-table operations (also used inside the step) ---- */
+
+/*
+ * Bigram hash rows (decoder-rtx posts, "bi-gram hash tables"): for each
+ * position, a = tokens[b, t-1] (a = vocab at t = 0), c = tokens[b, t],
+ * key = (a*p1 mod 2^64) XOR (c*p2 mod 2^64), rows_out[b, t] = key mod rows.
+ * tokens / rows_out: device int32 [B, T].  Ids outside [0, vocab) set the
+ * device error word (ngram_sync_status) and give row 0.  rows <= 2^31-1.
+ */
+int ngram_hash(const int32_t* tokens, int B, int T, int vocab, unsigned long long p1,
+               unsigned long long p2, long long rows, int32_t* rows_out, void* stream);
+
+/*
+ * Row gather: out[i, :] (+)= table[rows[i], :] for i < n (decoder-rtx posts:
+ * table rows "added to x0" / "added to values").  table: device [n_rows, d]
+ * of `dtype` (GPT_DTYPE_F32 or GPT_DTYPE_BF16); out: device [n, d] of the same
+ * dtype, overwritten (accumulate = 0) or added to (accumulate = 1).
+ * Rows outside [0, n_rows) set the device error word and leave out[i] as is.
+ */
+int ngram_gather(const int32_t* rows, int n, const void* table, long long n_rows, int d,
+                 int dtype, void* out, int accumulate, void* stream);
+
+/* Device workspace bytes ngram_sparse_update() needs for n positions of width d. */
+int ngram_sparse_update_workspace_bytes(int n, int d, size_t* bytes);
+
+/*
+ * Sparse per-row-magnitude table update, applied in place (decoder-rtx
+ * posts: "sparse, no first moment, and only per-row magnitude", inlined
+ * into backward).  For every distinct row r among rows[0..n):
+ *   G = sum of grad[i, :] over i with rows[i] == r   (summed in order of i)
+ *   s_r = beta * s_r + (1 - beta) * mean_j G[j]^2
+ *   table[r, :] -= lr * G / (sqrt(s_r) + eps)
+ * Other rows and states are untouched.  Positions are bucketed by row with
+ * a stable radix sort (no atomics), so the result is deterministic.
+ * table: device [n_rows, d] of `dtype` (bf16 rows are rounded to nearest
+ * even); row_state: device fp32 [n_rows]; grad: device fp32 [n, d].
+ * updated_rows_out (nullable): device int32 [n], receives the distinct
+ * rows in ascending order; n_updated_out_dev (nullable): device int32, their
+ * count.  workspace: device, ws_bytes >= ngram_sparse_update_workspace_bytes.
+ */
+int ngram_sparse_update(void* table, float* row_state, long long n_rows, int d, int dtype,
+                        const int32_t* rows, const float* grad, int n, float lr, float beta,
+                        float eps, int32_t* updated_rows_out, int* n_updated_out_dev,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream` and read + clear the standalone operations' device
+ * error word (GPT_ERR_INPUT for out-of-range ids). */
+int ngram_sync_status(void* stream);
+
+/* ---- kernel-level test entry point ------------------------------------- */
+
+/*
+ * C[m, n] (+)= sum_k A[m, k] B[n, k] on the tcgen05 tensor-core GEMM that the
+ * step uses for every dense contraction (bf16 operands, fp32 accumulation).
+ * A is read K-major (a_kmajor = 1: element [m, k] at A[m*lda + k]) or M-major
+ * (a_kmajor = 0: at A[k*lda + m]); B likewise with N.  C: device fp32 [M, ldc],
+ * overwritten (beta = 0) or added to (beta = 1).  splits > 1 splits K and
+ * needs workspace of splits*M*N*4 bytes (partials summed in split order).
+ * Operands must be 16-byte aligned with lda*2, ldb*2 multiples of 16.
+ */
+int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmajor, const void* B,
+                   long long ldb, int b_kmajor, float* C, long long ldc, int beta, int splits,
+                   void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT_B200_H */

@@ -1,0 +1,166 @@
+"""Kernel-level parity on the GPU, through the C ABI: the tcgen05 GEMM in every
+operand layout, and the bigram-table hash / gather / sparse update against the
+fp64 oracle (bit-exact on row ids and updated-row sets)."""
+
+import numpy as np
+import pytest
+
+from oracle import hashing, optim
+from synthetic import round_to_bf16, zipf_stream
+from tests.helpers import device_ints, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    import torch
+    import gpt_pretraining_step_decoder_b200 as g
+    assert torch.cuda.is_available()
+    return g
+
+
+def _bf16_dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 384, 160), (776, 264, 520), (256, 768, 768)])
+@pytest.mark.parametrize("a_k,b_k", [(1, 1), (1, 0), (0, 0), (0, 1)])
+def test_gemm_layouts_match_fp64(g, M, N, K, a_k, b_k):
+    import torch
+    rng = np.random.default_rng(M * 7 + N * 3 + K + 11 * a_k + 5 * b_k)
+    A = round_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    B = round_to_bf16(rng.standard_normal((N, K)).astype(np.float32))
+    ref = A.astype(np.float64) @ B.astype(np.float64).T
+    Ad = _bf16_dev(A if a_k else A.T)
+    Bd = _bf16_dev(B if b_k else B.T)
+    C = torch.full((M, N), 7.0, dtype=torch.float32, device="cuda")
+    g.gptx_gemm_bf16(M, N, K, Ad, K if a_k else M, a_k, Bd, K if b_k else N, b_k, C, N, 0, 1, None, 0)
+    torch.cuda.synchronize()
+    assert g.ngram_sync_status() == g.GPT_OK
+    err = rel_l2(C.cpu().numpy(), ref)
+    assert err < 1e-5, err
+    # beta = 1 accumulates
+    g.gptx_gemm_bf16(M, N, K, Ad, K if a_k else M, a_k, Bd, K if b_k else N, b_k, C, N, 1, 1, None, 0)
+    torch.cuda.synchronize()
+    assert rel_l2(C.cpu().numpy(), 2 * ref) < 1e-5
+
+
+def test_gemm_split_k_is_deterministic_and_exact(g):
+    import torch
+    M, N, K = 768, 768, 4096
+    rng = np.random.default_rng(5)
+    A = round_to_bf16(rng.standard_normal((K, M)).astype(np.float32))   # stored [K, M]
+    B = round_to_bf16(rng.standard_normal((K, N)).astype(np.float32))   # stored [K, N]
+    ref = A.astype(np.float64).T @ B.astype(np.float64)
+    ws = torch.empty(8 * M * N * 4, dtype=torch.uint8, device="cuda")
+    outs = []
+    for splits in (1, 4, 4):
+        C = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+        g.gptx_gemm_bf16(M, N, K, _bf16_dev(A), M, 0, _bf16_dev(B), N, 0, C, N, 0, splits, ws, ws.numel())
+        torch.cuda.synchronize()
+        outs.append(C.cpu().numpy())
+    assert rel_l2(outs[0], ref) < 1e-5 and rel_l2(outs[1], ref) < 1e-5
+    np.testing.assert_array_equal(outs[1], outs[2])
+
+
+def test_ngram_hash_bit_exact(g):
+    import torch
+    B, T, V = 4, 333, 50304
+    tok = zipf_stream(B * T, V, 3).reshape(B, T)
+    for rows in (2097152, 1048576, 1000003):
+        out = torch.empty((B, T), dtype=torch.int32, device="cuda")
+        g.ngram_hash(device_ints(tok), B, T, V, 2654435761, 2246822519, rows, out)
+        torch.cuda.synchronize()
+        ref = hashing.bigram_rows(tok, V, 2654435761, 2246822519, rows)
+        np.testing.assert_array_equal(out.cpu().numpy(), ref)
+    assert g.ngram_sync_status() == g.GPT_OK
+
+
+def test_ngram_hash_rejects_bad_tokens(g):
+    import torch
+    tok = np.array([[1, 2, 70000, 3]])
+    out = torch.empty((1, 4), dtype=torch.int32, device="cuda")
+    g.ngram_hash(device_ints(tok), 1, 4, 50304, 2654435761, 2246822519, 1024, out)
+    assert g.ngram_sync_status() == g.GPT_ERR_INPUT
+    assert g.ngram_sync_status() == g.GPT_OK   # cleared
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ngram_gather(g, dtype):
+    import torch
+    rng = np.random.default_rng(2)
+    R, d, n = 5000, 768, 1000
+    tab = rng.standard_normal((R, d)).astype(np.float32)
+    if dtype == "bf16":
+        tab = round_to_bf16(tab)
+    rows = rng.integers(0, R, n)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    dt = g.DTYPE_BF16 if dtype == "bf16" else g.DTYPE_F32
+    T = torch.from_numpy(tab).to(tdt).cuda()
+    out = torch.ones((n, d), dtype=tdt, device="cuda")
+    g.ngram_gather(device_ints(rows), n, T, R, d, dt, out, 0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.float().cpu().numpy(), tab[rows])
+    g.ngram_gather(device_ints(rows), n, T, R, d, dt, out, 1)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(out.float().cpu().numpy(), 2 * tab[rows], rtol=1e-2 if dtype == "bf16" else 0)
+
+
+@pytest.mark.parametrize("dtype,R,n,d", [("f32", 1000, 3000, 128), ("bf16", 2048, 6000, 768),
+                                         ("bf16", 2097152, 32768, 768)])
+def test_ngram_sparse_update_matches_oracle(g, dtype, R, n, d):
+    """Zipf-skewed bigram rows: long segments, singletons, ragged piece tails."""
+    import torch
+    rng = np.random.default_rng(R + n)
+    tok = zipf_stream(n + 1, 50304, R).reshape(1, n + 1)[:, :n]
+    rows = hashing.bigram_rows(tok, 50304, 2654435761, 2246822519, R).reshape(-1)
+    grad = rng.standard_normal((n, d)).astype(np.float32)
+    touched = np.unique(rows)
+    # build only the touched rows on the host; the table is initialised on the device
+    tab0 = rng.standard_normal((len(touched), d)).astype(np.float32) * 0.02
+    if dtype == "bf16":
+        tab0 = round_to_bf16(tab0)
+    s0 = np.abs(rng.standard_normal(len(touched))) * 0.1
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    T = torch.zeros((R, d), dtype=tdt, device="cuda")
+    S = torch.zeros(R, dtype=torch.float32, device="cuda")
+    idx = torch.from_numpy(touched).cuda()
+    T[idx] = torch.from_numpy(tab0).to(tdt).cuda()
+    S[idx] = torch.from_numpy(s0.astype(np.float32)).cuda()
+    ws_bytes = g.ngram_sparse_update_workspace_bytes(n, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    upd = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    nupd = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lr, beta, eps = 0.01, 0.95, 1e-10
+    g.ngram_sparse_update(T, S, R, d, g.DTYPE_BF16 if dtype == "bf16" else g.DTYPE_F32,
+                          device_ints(rows), torch.from_numpy(grad).cuda(), n, lr, beta, eps,
+                          upd, nupd, ws, ws_bytes)
+    assert g.ngram_sync_status() == g.GPT_OK
+    k = int(nupd.item())
+    np.testing.assert_array_equal(upd[:k].cpu().numpy(), touched)
+    # oracle on the touched rows only (compact index space); at full size a
+    # sample of rows (the most frequent ones plus random ones), since each
+    # row's update depends only on its own positions
+    sel = np.arange(len(touched))
+    if n > 8000:
+        counts = np.bincount(np.searchsorted(touched, rows), minlength=len(touched))
+        sel = np.unique(np.concatenate([np.argsort(-counts)[:40],
+                                        rng.choice(len(touched), 200, replace=False)]))
+    keep = np.isin(rows, touched[sel])
+    remap = {r: i for i, r in enumerate(touched[sel])}
+    crow = np.array([remap[r] for r in rows[keep]])
+    W1, s1, u = optim.table_update(tab0[sel].astype(np.float64),
+                                   s0[sel].astype(np.float32).astype(np.float64),
+                                   crow, grad[keep].astype(np.float64), lr, beta, eps)
+    tab0 = tab0[sel]
+    Wg = T[idx[torch.from_numpy(sel).cuda()]].float().cpu().numpy()
+    Sg = S[idx[torch.from_numpy(sel).cuda()]].cpu().numpy()
+    tol = 2e-2 if dtype == "bf16" else 1e-4
+    assert rel_l2(Wg - tab0, W1 - tab0) < tol
+    assert rel_l2(Sg, s1) < tol
+    # untouched rows stay zero
+    mask = torch.ones(R, dtype=torch.bool, device="cuda")
+    mask[idx] = False
+    assert int((T[mask] != 0).sum()) == 0 and int((S[mask] != 0).sum()) == 0
