@@ -1,0 +1,377 @@
+"""Training-step throughput of the decoder on B200s (tokens/s and MFU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1, NCCL).  A step is grad_accum x
+(forward + backward) micro-batches plus the optimizer step, over the
+workload's synthetic Zipf(1.1) token stream, with random-init weights.
+Default workload: the 12-layer d=768 bf16 decoder, 32 x 1024 = 32K tokens per
+step, tied vocab 50304.
+
+Rank 0 prints one JSON line.  `value` is whole-job tokens/s with the inputs
+already in HBM (CUDA events on the model's stream, barrier + synchronize on
+both sides, max over ranks).  `e2e` repeats the measurement through the same
+public calls with pinned host buffers, copying each step's tokens/targets in
+and its loss out inside the timed region.  `roofline` is the dominant kernel
+class (by time) from CUDA events bracketing every kernel in a second timed
+pass of the same steps.  `cpu_baseline` times the fp64 oracle on a bounded
+sample on the host cores.  `--impl reference` times that oracle as the
+reference arm on the same metric.
+"""
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import tokens_and_targets, workload  # noqa: E402
+
+SPEC_BF16_FLOPS = 2.25e15           # B200 dense bf16 spec (the metric's denominator)
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "training tokens/sec and MFU (% of B200 dense BF16 peak) at 1 GPU"
+L2_NOTE = "no L2 flush: a step's working set (weights, activations, logits chunk) is > 10 GB, far above the 126 MB L2"
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(w, seed):
+    """fp64 oracle: one full step on one sequence at the workload's length."""
+    from oracle.step import OracleTrainer
+    from synthetic import init_params
+    ws = dict(w, micro_batch=1, grad_accum=1)
+    if ws["x0_rows"] or ws["v_rows"]:
+        ws["x0_rows"] = min(ws["x0_rows"], 1 << 16)
+        ws["v_rows"] = min(ws["v_rows"], 1 << 15)
+    params = init_params(ws, seed=seed)
+    tr = OracleTrainer(ws, params)
+    tok, tgt = tokens_and_targets(1, ws["seq_len"], ws["vocab"], seed)
+    return tr, tok, tgt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, seconds=20.0):
+    tr, tok, tgt = oracle_sample(w, w["seed"])
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        tr.forward_loss(tok, tgt)
+        tr.backward_step(1e-3)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el > seconds or steps >= 3:
+            break
+    return {"value": steps * w["seq_len"] / el, "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, {steps} full step(s) (forward, backward, updates) on one "
+                      f"{w['seq_len']}-token sequence of the same workload, tables (if any) cut to "
+                      f"64K/32K rows; {el:.1f} s of host time"}
+
+
+def run_reference(args, w, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    tr, tok, tgt = oracle_sample(w, w["seed"])
+    for _ in range(args.warmup):
+        tr.forward_loss(tok, tgt)
+        tr.backward_step(1e-3)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        tr.forward_loss(tok, tgt)
+        tr.backward_step(1e-3)
+    el = time.perf_counter() - t0
+    value = args.steps * w["seq_len"] / el
+    sample = (f"fp64 NumPy oracle, one {w['seq_len']}-token sequence per step (forward, backward, "
+              f"AdamW), warmup {args.warmup}, timed {args.steps}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_json(w, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": blas_threads(),
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_json(w, world):
+    return {"workload": f"{w['name']}: {w['n_layer']} layers, d {w['d_model']}, {w['n_head']}x{w['head_dim']} heads, "
+                        f"ReLU^2 MLP {w['d_ff']}, vocab {w['vocab']} ({'tied' if w['tie_embeddings'] else 'untied'}), "
+                        f"bigram tables {w['x0_rows']}/{w['v_rows']} rows",
+            "tokens_per_step": w["micro_batch"] * w["seq_len"] * w["grad_accum"] * world,
+            "seq_len": w["seq_len"], "micro_batch": w["micro_batch"], "grad_accum": w["grad_accum"],
+            "parallelism": f"dp{world}", "l2": L2_NOTE}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w, rank, world, dist):
+    import torch
+    import gpt_pretraining_step_decoder_b200 as g
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = g.make_config(**w)
+    model = g.Model(cfg, seed=w["seed"] + 17 * rank)
+    A, B, T, V = w["grad_accum"], w["micro_batch"], w["seq_len"], w["vocab"]
+    n_micro = A * (args.warmup + args.steps)
+    host_tok, host_tgt = [], []
+    for i in range(n_micro):
+        tok, tgt = tokens_and_targets(B, T, V, w["seed"] + 1000 * rank, w["zipf_s"], w["repeat_frac"], micro=i)
+        host_tok.append(torch.from_numpy(tok).pin_memory())
+        host_tgt.append(torch.from_numpy(tgt).pin_memory())
+    dev_tok = [t.to(dev) for t in host_tok]
+    dev_tgt = [t.to(dev) for t in host_tgt]
+    stream = model.stream
+    flat_grad = None
+    if world > 1:
+        p, _, shape = g.gpt_tensor(model.h, "*", g.KIND_GRAD)
+        off = p - model.arena.data_ptr()
+        flat_grad = model.arena[off:off + shape[0] * 4].view(torch.float32)
+    lr = args.lr
+
+    def step(i, tok_src, tgt_src, loss_host=None):
+        for a in range(A):
+            j = i * A + a
+            model.forward_loss(tok_src[j], tgt_src[j])
+            if world > 1:
+                g.gpt_backward(model.h, lr)
+            else:
+                model.backward_step(lr)
+            if loss_host is not None:
+                loss_host.copy_(model.loss, non_blocking=True)
+        if world > 1:
+            dist.all_reduce(flat_grad)
+            flat_grad.mul_(1.0 / world)
+            g.gpt_optimizer_step(model.h, lr)
+
+    def timed(fn_step, first, count):
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for i in range(first, first + count):
+            fn_step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        ms = ev0.elapsed_time(ev1)
+        if dist is not None:
+            t = torch.tensor([ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    # warm-up
+    for i in range(args.warmup):
+        step(i, dev_tok, dev_tgt)
+    torch.cuda.synchronize()
+    st = model.sync_status()
+    if st != g.GPT_OK:
+        raise RuntimeError(f"device error after warm-up: {st} {g.gpt_last_error()}")
+
+    # timed region: inputs resident in HBM
+    l0 = g.gpt_launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = timed(lambda i: step(i, dev_tok, dev_tgt), args.warmup, args.steps)
+    launches = g.gpt_launch_count() - l0
+    clocks = clk.summary()
+    tokens_per_step = A * B * T * world
+    value = tokens_per_step * args.steps / (ms / 1e3)
+    loss = float(model.loss.item())
+
+    # second timed pass with every kernel bracketed by CUDA events (roofline)
+    g.gpt_profile_enable(model.h, 1)
+    ms_prof = timed(lambda i: step(i, dev_tok, dev_tgt), args.warmup, args.steps)
+    prof = g.gpt_profile_read(model.h)
+    g.gpt_profile_enable(model.h, 0)
+
+    # end-to-end through the public calls with pinned host buffers
+    in_tok = torch.empty_like(dev_tok[0])
+    in_tgt = torch.empty_like(dev_tgt[0])
+    loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
+
+    def e2e_step(i):
+        for a in range(A):
+            j = i * A + a
+            in_tok.copy_(host_tok[j], non_blocking=True)
+            in_tgt.copy_(host_tgt[j], non_blocking=True)
+            model.forward_loss(in_tok, in_tgt)
+            if world > 1:
+                g.gpt_backward(model.h, lr)
+            else:
+                model.backward_step(lr)
+            loss_host.copy_(model.loss, non_blocking=True)
+        if world > 1:
+            dist.all_reduce(flat_grad)
+            flat_grad.mul_(1.0 / world)
+            g.gpt_optimizer_step(model.h, lr)
+
+    ms_e2e = timed(e2e_step, args.warmup, args.steps)
+    st = model.sync_status()
+    if st != g.GPT_OK:
+        raise RuntimeError(f"device error in timed steps: {st} {g.gpt_last_error()}")
+
+    if rank != 0:
+        return
+    f_tok, f_tok_causal = g.gpt_flops_per_token(cfg)
+    peaks, peak_src = measured_peaks()
+    tok_s_gpu = value / world
+    mfu_spec = tok_s_gpu * f_tok / SPEC_BF16_FLOPS
+    mfu_meas = tok_s_gpu * f_tok / (peaks["bf16_tflops_sustained"] * 1e12)
+    total_ms = sum(v["ms"] for v in prof.values())
+    dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    if dom["flops"] > 0:
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "peak_source": f"{peak_src} bf16 sustained (cuBLAS loop under the power cap)"}
+    else:
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_src} HBM copy"}
+    roof["launches_per_step"] = dom["launches"] / args.steps
+    roof["share_of_step"] = dom["ms"] / total_ms if total_ms else None
+    roof["per_launch"] = ("gemm: algorithmic 2*M*N*K FLOPs of every contraction in the step, "
+                          "summed, over the summed CUDA-event time of those launches")
+    breakdown = {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
+                     "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["flops"] and v["ms"] else None,
+                     "gbs": (v["bytes"] / (v["ms"] / 1e3) / 1e9) if v["bytes"] and v["ms"] else None}
+                 for k, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"])}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w["dtype"] == "bf16" else "f32",
+        "data": "synthetic (Zipf(1.1) token stream, random-init weights)",
+        "config": config_json(w, world),
+        "mfu": {"formula": mfu_spec, "causal": tok_s_gpu * f_tok_causal / SPEC_BF16_FLOPS,
+                "of_measured_sustained": mfu_meas, "flops_per_token": f_tok,
+                "flops_per_token_causal": f_tok_causal, "peak_spec_flops": SPEC_BF16_FLOPS},
+        "loss_last": loss,
+        "roofline": roof,
+        "breakdown": breakdown,
+        "profiled_ms_per_step": ms_prof / args.steps,
+        "e2e": {"value": tokens_per_step * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(A * (host_tok[0].numel() + host_tgt[0].numel()) * 4),
+                "d2h_bytes_per_step": int(A * 4)},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="gpt2s_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--lr", type=float, default=1e-4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = workload(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    try:
+        run_ours(args, w, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -43,6 +43,12 @@ class GptConfig(ctypes.Structure):
     ]
 
 
+class GptProfEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("scopes", ctypes.c_longlong),
+                ("launches", ctypes.c_longlong), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 _P, _I, _LL, _SZ, _F, _ULL = (ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t,
                               ctypes.c_float, ctypes.c_ulonglong)
 _SIGS = {
@@ -53,6 +59,11 @@ _SIGS = {
     "gpt_set_stream": [_P, _P],
     "gpt_forward_loss": [_P, _P, _P, _P],
     "gpt_backward_step": [_P, _F],
+    "gpt_backward": [_P, _F],
+    "gpt_optimizer_step": [_P, _F],
+    "gpt_launch_count": [ctypes.POINTER(_LL)],
+    "gpt_profile_enable": [_P, _I],
+    "gpt_profile_read": [_P, ctypes.POINTER(GptProfEntry), _I, ctypes.POINTER(_I)],
     "gpt_num_params": [_P, ctypes.POINTER(_LL), ctypes.POINTER(_LL)],
     "gpt_flops_per_token": [ctypes.POINTER(GptConfig), ctypes.POINTER(_LL), ctypes.POINTER(_LL)],
     "gpt_tensor": [_P, ctypes.c_char_p, _I, ctypes.POINTER(_P), ctypes.POINTER(_I), _LL * 4],
@@ -156,6 +167,34 @@ def gpt_forward_loss(h, tokens, targets, loss):
 
 def gpt_backward_step(h, lr):
     return _check(_lib.gpt_backward_step(h, float(lr)), "gpt_backward_step")
+
+
+def gpt_backward(h, lr):
+    return _check(_lib.gpt_backward(h, float(lr)), "gpt_backward")
+
+
+def gpt_optimizer_step(h, lr):
+    return _check(_lib.gpt_optimizer_step(h, float(lr)), "gpt_optimizer_step")
+
+
+def gpt_launch_count():
+    n = ctypes.c_longlong()
+    _check(_lib.gpt_launch_count(ctypes.byref(n)), "gpt_launch_count")
+    return n.value
+
+
+def gpt_profile_enable(h, on):
+    return _check(_lib.gpt_profile_enable(h, int(on)), "gpt_profile_enable")
+
+
+def gpt_profile_read(h, cap=64):
+    """{class name: dict(scopes, launches, ms, flops, bytes)} since the last read."""
+    arr = (GptProfEntry * cap)()
+    n = ctypes.c_int()
+    _check(_lib.gpt_profile_read(h, arr, cap, ctypes.byref(n)), "gpt_profile_read")
+    return {arr[i].name.decode(): dict(scopes=arr[i].scopes, launches=arr[i].launches,
+                                       ms=arr[i].ms, flops=arr[i].flops, bytes=arr[i].bytes)
+            for i in range(min(n.value, cap))}
 
 
 def gpt_num_params(h):

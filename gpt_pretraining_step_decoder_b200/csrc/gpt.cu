@@ -13,6 +13,7 @@
 #include <cstdarg>
 #include <cstring>
 #include <type_traits>
+#include <atomic>
 #include <map>
 #include <string>
 #include <vector>
@@ -22,6 +23,7 @@
 #include "gemm_common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "attention_fa.cuh"
 #include "layers.cuh"
 #include "ngram.cuh"
 #include "optim.cuh"
@@ -56,6 +58,9 @@ static int fail(int code, const char* fmt, ...) {
   } while (0)
 
 extern "C" const char* gpt_last_error(void) { return g_last_error.c_str(); }
+
+// Kernels this library has launched in this process (read by gpt_launch_count).
+static std::atomic<long long> g_launches{0};
 
 // ======================================================================== device props
 static int device_sms() {
@@ -130,13 +135,13 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   p.err = err;
   const int tiles = p.m_tiles * p.n_tiles * p.splits;
   const int grid = tiles < device_sms() ? tiles : device_sms();
-  tc::gemm_tc_kernel<BN, bf16><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
+  ++g_launches; tc::gemm_tc_kernel<BN, bf16><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
   LAUNCH_CHECK();
   if (p.splits > 1) {
     const long long total = (long long)M * N;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * device_sms()) blocks = 4 * device_sms();
-    splitk_reduce_kernel<bf16><<<blocks, 256, 0, st>>>(partial, p.splits, M, N, e);
+    ++g_launches; splitk_reduce_kernel<bf16><<<blocks, 256, 0, st>>>(partial, p.splits, M, N, e);
     LAUNCH_CHECK();
   }
   return GPT_OK;
@@ -153,17 +158,64 @@ static int pick_splits(int M, int N, int K, int BN) {
   return s;
 }
 
+// ======================================================================== live timing
+// Optional per-kernel-class timing with CUDA events recorded on the model's
+// stream around each kernel (or small group of kernels) while enabled.
+struct ProfRec {
+  const char* cls;
+  cudaEvent_t a, b;
+  double flops, bytes;
+  long long launches;
+};
+struct Prof {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  cudaEvent_t get() {
+    if (used == pool.size()) {
+      cudaEvent_t e = nullptr;
+      cudaEventCreate(&e);
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+};
+struct ProfScope {
+  Prof* p = nullptr;
+  cudaStream_t st = nullptr;
+  long idx = -1;
+  long long l0 = 0;
+  ProfScope(Prof* prof, cudaStream_t s, const char* cls, double flops, double bytes) : p(prof), st(s) {
+    if (!p || !p->on) return;
+    ProfRec r;
+    r.cls = cls; r.a = p->get(); r.b = p->get(); r.flops = flops; r.bytes = bytes; r.launches = 0;
+    l0 = g_launches.load();
+    cudaEventRecord(r.a, st);
+    p->recs.push_back(r);
+    idx = (long)p->recs.size() - 1;
+  }
+  ~ProfScope() {
+    if (idx < 0) return;
+    ProfRec& r = p->recs[idx];
+    r.launches = g_launches.load() - l0;
+    cudaEventRecord(r.b, st);
+  }
+};
+
 struct GemmCtx {
   bool bf16;
   float* splitk;          // fp32 scratch for split-K partials
   long long splitk_elems;
   unsigned* err;
   cudaStream_t st;
+  Prof* prof;
 };
 
 static int gemm(const GemmCtx& g, int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
                 bool allow_split = false) {
   if (M <= 0 || N <= 0 || K <= 0) return GPT_OK;
+  ProfScope ps(g.prof, g.st, "gemm", 2.0 * M * N * K, 0.0);
   if (!g.bf16) {
     gemm_simt<float, float>(M, N, K, A, B, e, g.st);
     LAUNCH_CHECK();
@@ -373,6 +425,7 @@ struct gpt_model {
   int micro = 0;
   long long step_t = 0;
   bool have_fwd = false;
+  Prof prof;
   template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
   unsigned* err() const { return at<unsigned>(plan.err); }
 };
@@ -426,7 +479,7 @@ static int grid_for(long long n, int per_block) {
 static int refresh_lp(gpt_model* m) {
   if (!cfg_bf16(m->cfg)) return GPT_OK;
   const Plan& p = m->plan;
-  to_bf16_kernel<<<4 * device_sms(), 256, 0, m->st>>>(m->at<float>(p.P), m->at<bf16>(p.Plp), p.dense_n);
+  ++g_launches; to_bf16_kernel<<<4 * device_sms(), 256, 0, m->st>>>(m->at<float>(p.P), m->at<bf16>(p.Plp), p.dense_n);
   LAUNCH_CHECK();
   return GPT_OK;
 }
@@ -455,23 +508,25 @@ extern "C" int gpt_create(const gpt_config* cfg, unsigned long long seed, void* 
   const int blocks = 8 * device_sms();
   uint32_t stream_id = 1;
   for (const auto& t : p.dense) {
-    init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.P) + t.off, t.rows * t.cols,
+    ++g_launches; init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.P) + t.off, t.rows * t.cols,
                                                         c.init_std, seed, stream_id++);
   }
   const long long a = (long long)c.n_head * c.head_dim;
   if (c.x0_rows) {
-    if (cfg_bf16(c))
-      init_normal_kernel<bf16><<<blocks, 256, 0, m->st>>>(m->at<bf16>(p.hx), c.x0_rows * c.d_model, c.init_std, seed, 0x10000u);
-    else
-      init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.hx), c.x0_rows * c.d_model, c.init_std, seed, 0x10000u);
+    if (cfg_bf16(c)) {
+      ++g_launches; init_normal_kernel<bf16><<<blocks, 256, 0, m->st>>>(m->at<bf16>(p.hx), c.x0_rows * c.d_model, c.init_std, seed, 0x10000u);
+    } else {
+      ++g_launches; init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.hx), c.x0_rows * c.d_model, c.init_std, seed, 0x10000u);
+    }
   }
   if (c.v_rows) {
-    if (cfg_bf16(c))
-      init_normal_kernel<bf16><<<blocks, 256, 0, m->st>>>(m->at<bf16>(p.hv), c.v_rows * a, c.init_std, seed, 0x10001u);
-    else
-      init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.hv), c.v_rows * a, c.init_std, seed, 0x10001u);
+    if (cfg_bf16(c)) {
+      ++g_launches; init_normal_kernel<bf16><<<blocks, 256, 0, m->st>>>(m->at<bf16>(p.hv), c.v_rows * a, c.init_std, seed, 0x10001u);
+    } else {
+      ++g_launches; init_normal_kernel<float><<<blocks, 256, 0, m->st>>>(m->at<float>(p.hv), c.v_rows * a, c.init_std, seed, 0x10001u);
+    }
   }
-  rope_table_kernel<<<grid_for((long long)c.seq_len * c.head_dim / 2, 256), 256, 0, m->st>>>(
+  ++g_launches; rope_table_kernel<<<grid_for((long long)c.seq_len * c.head_dim / 2, 256), 256, 0, m->st>>>(
       m->at<float>(p.rope_cs), c.seq_len, c.head_dim, (double)c.rope_base);
   e = cudaGetLastError();
   if (e != cudaSuccess) { delete m; return fail(GPT_ERR_CUDA, "init launch: %s", cudaGetErrorString(e)); }
@@ -484,6 +539,7 @@ extern "C" int gpt_create(const gpt_config* cfg, unsigned long long seed, void* 
 extern "C" int gpt_destroy(gpt_model* m) {
   if (!m) return fail(GPT_ERR_ARG, "null model");
   cudaStreamSynchronize(m->st);
+  for (cudaEvent_t e : m->prof.pool) cudaEventDestroy(e);
   delete m;
   return GPT_OK;
 }
@@ -539,6 +595,16 @@ extern "C" int gpt_tensor(gpt_model* m, const char* name, int kind, void** ptr, 
     else if (nm == "grad_norm") { ptr_out = m->at<float>(p.grad_norm); }
     else return fail(GPT_ERR_ARG, "unknown activation '%s'", name);
     (void)N;
+  } else if (nm == "*") {
+    // the whole flat dense buffer of this kind (tensors padded to 64 elements)
+    sh[0] = p.dense_n;
+    switch (kind) {
+      case GPT_KIND_PARAM: ptr_out = m->at<float>(p.P); break;
+      case GPT_KIND_GRAD: ptr_out = m->at<float>(p.G); break;
+      case GPT_KIND_ADAM_M: ptr_out = m->at<float>(p.M); break;
+      case GPT_KIND_ADAM_V: ptr_out = m->at<float>(p.V); break;
+      default: return fail(GPT_ERR_ARG, "flat buffer '*' has kinds PARAM, GRAD, ADAM_M, ADAM_V");
+    }
   } else if (nm == "hx" || nm == "hv") {
     const bool isx = nm == "hx";
     const long long rows = isx ? c.x0_rows : c.v_rows;
@@ -594,7 +660,7 @@ static SortWs sort_ws(const gpt_model* m) {
 static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long key_range,
                          const uint32_t** keys_out, const int32_t** perm_out, int32_t* uniq_out,
                          int* n_uniq_out, unsigned* err, cudaStream_t st) {
-  iota_kernel<<<grid_for(n, 256), 256, 0, st>>>(keys, w.ka, w.va, n, key_range, err);
+  ++g_launches; iota_kernel<<<grid_for(n, 256), 256, 0, st>>>(keys, w.ka, w.va, n, key_range, err);
   LAUNCH_CHECK();
   int bits = 1;
   while (bits < 32 && (1LL << bits) < key_range) ++bits;
@@ -603,14 +669,14 @@ static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long 
   uint32_t *kin = w.ka, *kout = w.kb;
   int32_t *vin = w.va, *vout = w.vb;
   for (int ps = 0; ps < passes; ++ps) {
-    radix_hist_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, n, 8 * ps, w.counts);
-    exclusive_scan_kernel<<<1, 1024, 0, st>>>(w.counts, 256 * nblk);
-    radix_scatter_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, vin, n, 8 * ps, w.counts, kout, vout);
+    ++g_launches; radix_hist_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, n, 8 * ps, w.counts);
+    ++g_launches; exclusive_scan_kernel<<<1, 1024, 0, st>>>(w.counts, 256 * nblk);
+    ++g_launches; radix_scatter_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, vin, n, 8 * ps, w.counts, kout, vout);
     LAUNCH_CHECK();
     std::swap(kin, kout);
     std::swap(vin, vout);
   }
-  segments_kernel<<<1, 1024, 0, st>>>(kin, n, w.seg_start, w.pstart, w.plen, w.pseg, w.pslot, w.lfirst,
+  ++g_launches; segments_kernel<<<1, 1024, 0, st>>>(kin, n, w.seg_start, w.pstart, w.plen, w.pseg, w.pslot, w.lfirst,
                                       w.lnslots, w.lseg, w.counters, uniq_out, n_uniq_out);
   LAUNCH_CHECK();
   *keys_out = kin;
@@ -626,9 +692,9 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const int32_t* perm;
   TRY(bucket_by_key(w, rows, n, n_rows, &skeys, &perm, uniq_out, n_uniq_out, err, st));
   const long long maxp = (long long)n + n / PIECE + 2, maxl = n / PIECE + 2;
-  table_piece_kernel<tab_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
+  ++g_launches; table_piece_kernel<tab_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
       table, state, d, grad, skeys, perm, w.pstart, w.plen, w.pslot, w.counters, w.partial, lr, beta, eps);
-  table_long_kernel<tab_t><<<grid_for(maxl * 32, 256), 256, 0, st>>>(
+  ++g_launches; table_long_kernel<tab_t><<<grid_for(maxl * 32, 256), 256, 0, st>>>(
       table, state, d, skeys, w.seg_start, w.lfirst, w.lnslots, w.lseg, w.counters, w.partial, lr, beta, eps);
   LAUNCH_CHECK();
   return GPT_OK;
@@ -636,27 +702,60 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
 
 // ======================================================================== forward
 template <typename act_t>
-static int attention_fwd(const gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
+static int attention_fwd(gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
   const gpt_config& c = m->cfg;
+  ProfScope ps(&m->prof, m->st, "attention_fwd",
+               2.0 * c.micro_batch * c.n_head * (double)c.seq_len * c.seq_len * c.head_dim, 0.0);
+  if (std::is_same<act_t, bf16>::value) {
+    static bool attr = false;
+    if (!attr) {
+      CUDA_TRY(cudaFuncSetAttribute(fa::fa_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::F_SMEM));
+      attr = true;
+    }
+    dim3 g(cdiv(c.seq_len, fa::F_BQ), c.micro_batch * c.n_head);
+    ++g_launches; fa::fa_fwd_kernel<<<g, fa::F_THREADS, fa::F_SMEM, m->st>>>(
+        reinterpret_cast<const bf16*>(qkv), reinterpret_cast<bf16*>(o), lse, c.seq_len, c.n_head);
+    LAUNCH_CHECK();
+    return GPT_OK;
+  }
   dim3 grid(cdiv(c.seq_len, 4), c.micro_batch * c.n_head);
-  attn_fwd_simt_kernel<act_t><<<grid, 128, 4 * c.head_dim * 4, m->st>>>(qkv, o, lse, c.micro_batch, c.seq_len,
+  ++g_launches; attn_fwd_simt_kernel<act_t><<<grid, 128, 4 * c.head_dim * 4, m->st>>>(qkv, o, lse, c.micro_batch, c.seq_len,
                                                                         c.n_head, c.head_dim);
   LAUNCH_CHECK();
   return GPT_OK;
 }
 
 template <typename act_t>
-static int attention_bwd(const gpt_model* m, const act_t* qkv, const act_t* o, const act_t* dout,
+static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const act_t* dout,
                          const float* lse, float* Dv, act_t* dqkv) {
   const gpt_config& c = m->cfg;
+  ProfScope ps(&m->prof, m->st, "attention_bwd",
+               5.0 * c.micro_batch * c.n_head * (double)c.seq_len * c.seq_len * c.head_dim, 0.0);
   const long long N = (long long)c.micro_batch * c.seq_len;
-  attn_bwd_pre_kernel<act_t><<<grid_for(N * c.n_head * 32, 256), 256, 0, m->st>>>(
+  ++g_launches; attn_bwd_pre_kernel<act_t><<<grid_for(N * c.n_head * 32, 256), 256, 0, m->st>>>(
       o, dout, Dv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
   LAUNCH_CHECK();
+  if (std::is_same<act_t, bf16>::value) {
+    static bool attr = false;
+    if (!attr) {
+      CUDA_TRY(cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::B_SMEM));
+      CUDA_TRY(cudaFuncSetAttribute(fa::fa_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Q_SMEM));
+      attr = true;
+    }
+    dim3 gk(cdiv(c.seq_len, fa::B_BK), c.micro_batch * c.n_head);
+    dim3 gq(cdiv(c.seq_len, fa::B_BQ), c.micro_batch * c.n_head);
+    const bf16* q16 = reinterpret_cast<const bf16*>(qkv);
+    const bf16* d16 = reinterpret_cast<const bf16*>(dout);
+    bf16* g16 = reinterpret_cast<bf16*>(dqkv);
+    ++g_launches; fa::fa_bwd_dkdv_kernel<<<gk, fa::B_THREADS, fa::B_SMEM, m->st>>>(q16, d16, lse, Dv, g16, c.seq_len, c.n_head);
+    ++g_launches; fa::fa_bwd_dq_kernel<<<gq, fa::B_THREADS, fa::Q_SMEM, m->st>>>(q16, d16, lse, Dv, g16, c.seq_len, c.n_head);
+    LAUNCH_CHECK();
+    return GPT_OK;
+  }
   dim3 grid(cdiv(c.seq_len, 4), c.micro_batch * c.n_head);
-  attn_bwd_dq_simt_kernel<act_t><<<grid, 128, 4 * 2 * c.head_dim * 4, m->st>>>(
+  ++g_launches; attn_bwd_dq_simt_kernel<act_t><<<grid, 128, 4 * 2 * c.head_dim * 4, m->st>>>(
       qkv, dout, lse, Dv, dqkv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
-  attn_bwd_dkdv_simt_kernel<act_t><<<grid, 128, 4 * 2 * c.head_dim * 4, m->st>>>(
+  ++g_launches; attn_bwd_dkdv_simt_kernel<act_t><<<grid, 128, 4 * 2 * c.head_dim * 4, m->st>>>(
       qkv, dout, lse, Dv, dqkv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
   LAUNCH_CHECK();
   return GPT_OK;
@@ -671,26 +770,33 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   const int N = c.micro_batch * c.seq_len;
   const int d = c.d_model, H = c.n_head, hd = c.head_dim, a = H * hd, F = c.d_ff, V = c.vocab;
   unsigned* err = m->err();
-  GemmCtx g{b16, m->at<float>(p.splitk), p.splitk_elems, err, st};
+  GemmCtx g{b16, m->at<float>(p.splitk), p.splitk_elems, err, st, &m->prof};
   // weights read by the GEMMs: the bf16 copy in bf16 mode, the master in fp32 mode
   auto W = [&](const std::string& nm) -> const act_t* {
     const DenseTensor* t = find_dense(m, nm);
     return b16 ? reinterpret_cast<const act_t*>(m->at<bf16>(p.Plp) + t->off)
                : reinterpret_cast<const act_t*>(m->at<float>(p.P) + t->off);
   };
+  const size_t es = sizeof(act_t);
+  Prof* pf = &m->prof;
   CUDA_TRY(cudaMemcpyAsync(m->at<int32_t>(p.tok_copy), tokens, (size_t)N * 4, cudaMemcpyDeviceToDevice, st));
   if (c.x0_rows || c.v_rows) {
-    ngram_hash_kernel<<<grid_for(N, 256), 256, 0, st>>>(
+    ProfScope ps(pf, st, "ngram_hash", 0.0, (double)N * 12);
+    ++g_launches; ngram_hash_kernel<<<grid_for(N, 256), 256, 0, st>>>(
         tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.x0_rows ? c.x0_rows : 1,
         c.x0_rows ? m->at<int32_t>(p.rows_x) : nullptr, c.v_rows ? c.v_rows : 1,
         c.v_rows ? m->at<int32_t>(p.rows_v) : nullptr, err);
     LAUNCH_CHECK();
   }
   float* x = m->at<float>(p.x);
-  embed_fwd_kernel<act_t, act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+  {
+  ProfScope ps(pf, st, "embed", 0.0, (double)N * d * (es + 4 + (c.x0_rows ? es : 0)));
+  ++g_launches; embed_fwd_kernel<act_t, act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
       tokens, W("wte"), c.x0_rows ? reinterpret_cast<const act_t*>(m->base + p.hx) : nullptr,
       m->at<int32_t>(p.rows_x), x, m->at<float>(p.emb_rstd), N, d, V, c.norm_eps, err);
   LAUNCH_CHECK();
+  }
+  const double norm_bytes = (double)N * d * (4 + es) + 4.0 * N;
   const int rows_blocks = grid_for((long long)N * 32, 256);
   for (int l = 0; l < c.n_layer; ++l) {
     const LayerActs& L = p.layers[l];
@@ -699,25 +805,37 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     act_t* qkv = m->at<act_t>(L.qkv);
     act_t* o = m->at<act_t>(L.o);
     act_t* u2 = m->at<act_t>(L.u2);
-    rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps);
-    LAUNCH_CHECK();
+    {
+      ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
+      ++g_launches; rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps);
+      LAUNCH_CHECK();
+    }
     TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a)));
-    rope_qknorm_fwd_kernel<act_t, act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
-        qkv, m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
-        c.v_rows ? reinterpret_cast<const act_t*>(m->base + p.hv) : nullptr, m->at<int32_t>(p.rows_v), N,
-        c.seq_len, H, hd, c.qk_norm, c.norm_eps);
-    LAUNCH_CHECK();
+    {
+      ProfScope ps(pf, st, "rope_qknorm_fwd", 0.0, (double)N * a * es * (4 + (c.v_rows ? 3 : 0)));
+      ++g_launches; rope_qknorm_fwd_kernel<act_t, act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+          qkv, m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
+          c.v_rows ? reinterpret_cast<const act_t*>(m->base + p.hv) : nullptr, m->at<int32_t>(p.rows_v), N,
+          c.seq_len, H, hd, c.qk_norm, c.norm_eps);
+      LAUNCH_CHECK();
+    }
     TRY(attention_fwd<act_t>(m, qkv, o, m->at<float>(L.lse)));
     TRY(gemm(g, N, d, a, op_k(o, a), op_k(W(pre + "wo"), a), epi(EPI_ACCUM_F32, x, d, 1)));
-    rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps);
-    LAUNCH_CHECK();
+    {
+      ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
+      ++g_launches; rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps);
+      LAUNCH_CHECK();
+    }
     TRY(gemm(g, N, F, d, op_k(u2, d), op_k(W(pre + "w1"), d),
              epi(EPI_RELU2, m->at<act_t>(L.r), F, 0, m->at<act_t>(L.g))));
     TRY(gemm(g, N, d, F, op_k(m->at<act_t>(L.g), F), op_k(W(pre + "w2"), F), epi(EPI_ACCUM_F32, x, d, 1)));
   }
   act_t* xf = m->at<act_t>(p.xf);
-  rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps);
-  ce_prepare_kernel<<<1, 1024, 0, st>>>(targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
+  {
+    ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
+    ++g_launches; rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps);
+  }
+  ++g_launches; ce_prepare_kernel<<<1, 1024, 0, st>>>(targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
   LAUNCH_CHECK();
   // chunked LM head + cross-entropy; the head's gradient pieces are formed
   // here while each logits chunk is live: dxf (fp32) and the pending head
@@ -728,22 +846,27 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   for (int r0 = 0, ci = 0; r0 < N; r0 += p.chunk, ++ci) {
     const int rows = (N - r0 < p.chunk) ? (N - r0) : p.chunk;
     TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), epi(EPI_STORE_F32, logits, V)));
-    ce_chunk_kernel<act_t><<<rows, 512, 0, st>>>(logits, dz, targets + r0, m->at<float>(p.tok_loss) + r0, V,
-                                                 c.softcap, m->at<float>(p.ce_scale), err);
-    LAUNCH_CHECK();
+    {
+      ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * (4 + es));
+      ++g_launches; ce_chunk_kernel<act_t><<<rows, 512, 0, st>>>(logits, dz, targets + r0, m->at<float>(p.tok_loss) + r0, V,
+                                                   c.softcap, m->at<float>(p.ce_scale), err);
+      LAUNCH_CHECK();
+    }
     TRY(gemm(g, rows, d, V, op_k(dz, V), op_mn(Wlm, d), epi(EPI_STORE_F32, m->at<float>(p.dxf) + (long long)r0 * d, d)));
     TRY(gemm(g, V, d, rows, op_mn(dz, V), op_mn(xf + (long long)r0 * d, d),
              epi(EPI_ACCUM_F32, m->at<float>(p.pending), d, ci > 0), true));
   }
-  loss_reduce_kernel<<<1, 1024, 0, st>>>(m->at<float>(p.tok_loss), N, m->at<int>(p.ce_count), loss_dev, err);
+  ++g_launches; loss_reduce_kernel<<<1, 1024, 0, st>>>(m->at<float>(p.tok_loss), N, m->at<int>(p.ce_count), loss_dev, err);
   LAUNCH_CHECK();
   m->have_fwd = true;
   return GPT_OK;
 }
 
 // ======================================================================== backward
+static int optimizer_step_impl(gpt_model* m, float lr);
+
 template <typename act_t>
-static int backward_impl(gpt_model* m, float lr) {
+static int backward_impl(gpt_model* m, float lr, bool do_step) {
   const gpt_config& c = m->cfg;
   const Plan& p = m->plan;
   const bool b16 = cfg_bf16(c);
@@ -751,7 +874,7 @@ static int backward_impl(gpt_model* m, float lr) {
   const int N = c.micro_batch * c.seq_len;
   const int d = c.d_model, H = c.n_head, hd = c.head_dim, a = H * hd, F = c.d_ff, V = c.vocab;
   unsigned* err = m->err();
-  GemmCtx g{b16, m->at<float>(p.splitk), p.splitk_elems, err, st};
+  GemmCtx g{b16, m->at<float>(p.splitk), p.splitk_elems, err, st, &m->prof};
   auto W = [&](const std::string& nm) -> const act_t* {
     const DenseTensor* t = find_dense(m, nm);
     return b16 ? reinterpret_cast<const act_t*>(m->at<bf16>(p.Plp) + t->off)
@@ -760,19 +883,25 @@ static int backward_impl(gpt_model* m, float lr) {
   auto Gp = [&](const std::string& nm) -> float* { return m->at<float>(p.G) + find_dense(m, nm)->off; };
   const int beta = m->micro > 0;
   const int rows_blocks = grid_for((long long)N * 32, 256);
+  const size_t es = sizeof(act_t);
+  Prof* pf = &m->prof;
+  const double nb_bytes = (double)N * d * (4 + es + 4 + es) + 4.0 * N + (double)N * d * 4;
   // LM-head weight gradient staged by the forward pass
   float* g_head = Gp(c.tie_embeddings ? "wte" : "lm_head");
-  accumulate_kernel<<<4 * device_sms(), 256, 0, st>>>(g_head, m->at<float>(p.pending), (long long)V * d, beta);
-  if (!c.tie_embeddings && !beta) CUDA_TRY(cudaMemsetAsync(Gp("wte"), 0, (size_t)V * d * 4, st));
+  {
+    ProfScope ps(pf, st, "head_grad_accumulate", 0.0, (double)V * d * 12);
+    ++g_launches; accumulate_kernel<<<4 * device_sms(), 256, 0, st>>>(g_head, m->at<float>(p.pending), (long long)V * d, beta);
+    if (!c.tie_embeddings && !beta) CUDA_TRY(cudaMemsetAsync(Gp("wte"), 0, (size_t)V * d * 4, st));
+  }
   float* dx = m->at<float>(p.dx);
   act_t* dx_lp = m->at<act_t>(p.dx_lp);
   float* du = m->at<float>(p.du);
   act_t* dqkv = m->at<act_t>(p.dqkv);
   act_t* da = m->at<act_t>(p.da);
   act_t* dout = m->at<act_t>(p.dout);
-  rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(m->at<float>(p.dxf), m->at<act_t>(p.xf),
+  { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); ++g_launches; rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(m->at<float>(p.dxf), m->at<act_t>(p.xf),
                                                         m->at<float>(p.rstd_f), dx, dx_lp, N, d, 0);
-  LAUNCH_CHECK();
+  LAUNCH_CHECK(); }
   for (int l = c.n_layer - 1; l >= 0; --l) {
     const LayerActs& L = p.layers[l];
     const std::string pre = "h" + std::to_string(l) + ".";
@@ -781,54 +910,74 @@ static int backward_impl(gpt_model* m, float lr) {
     TRY(gemm(g, N, F, d, op_k(dx_lp, d), op_mn(W(pre + "w2"), F), epi(EPI_DRELU2, da, F, 0, nullptr, m->at<act_t>(L.r))));
     TRY(gemm(g, F, d, N, op_mn(da, F), op_mn(m->at<act_t>(L.u2), d), epi(EPI_ACCUM_F32, Gp(pre + "w1"), d, beta), true));
     TRY(gemm(g, N, d, F, op_k(da, F), op_mn(W(pre + "w1"), d), epi(EPI_STORE_F32, du, d)));
-    rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1);
-    LAUNCH_CHECK();
+    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); ++g_launches; rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1);
+    LAUNCH_CHECK(); }
     // ---- attention: x += o Wo^T
     TRY(gemm(g, d, a, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.o), a), epi(EPI_ACCUM_F32, Gp(pre + "wo"), a, beta), true));
     TRY(gemm(g, N, a, d, op_k(dx_lp, d), op_mn(W(pre + "wo"), a), epi(EPI_STORE, dout, a)));
     TRY(attention_bwd<act_t>(m, m->at<act_t>(L.qkv), m->at<act_t>(L.o), dout, m->at<float>(L.lse),
                              m->at<float>(p.Dattn), dqkv));
-    rope_qknorm_bwd_kernel<act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
-        dqkv, m->at<act_t>(L.qkv), m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
-        c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
-    LAUNCH_CHECK();
+    {
+      ProfScope ps(pf, st, "rope_qknorm_bwd", 0.0, (double)N * a * es * 6 + (c.v_rows ? (double)N * a * (es + 8) : 0.0));
+      ++g_launches; rope_qknorm_bwd_kernel<act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+          dqkv, m->at<act_t>(L.qkv), m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
+          c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
+      LAUNCH_CHECK();
+    }
     TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true));
     TRY(gemm(g, N, d, 3 * a, op_k(dqkv, 3 * a), op_mn(W(pre + "wqkv"), d), epi(EPI_STORE_F32, du, d)));
-    rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1);
-    LAUNCH_CHECK();
+    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); ++g_launches; rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1);
+    LAUNCH_CHECK(); }
   }
   // dx now holds dL/dx0 per position.
   const SortWs w = sort_ws(m);
   {
     // token embedding gradient, bucketed by token id
+    ProfScope ps(pf, st, "embedding_grad", 0.0, (double)N * d * 4);
     const uint32_t* skeys;
     const int32_t* perm;
     TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
     const long long maxp = (long long)N + N / PIECE + 2, maxl = N / PIECE + 2;
-    emb_piece_kernel<act_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
+    ++g_launches; emb_piece_kernel<act_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
         Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, w.pstart, w.plen, w.pslot,
         w.counters, w.partial);
-    emb_long_kernel<<<grid_for(maxl * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, w.seg_start, w.lfirst,
+    ++g_launches; emb_long_kernel<<<grid_for(maxl * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, w.seg_start, w.lfirst,
                                                              w.lnslots, w.lseg, w.counters, w.partial);
     LAUNCH_CHECK();
   }
   const float lr_t = lr * c.lr_mult_table;
-  if (c.v_rows)
+  if (c.v_rows) {
+    ProfScope ps(pf, st, "table_update", 0.0, (double)N * a * 4);
     TRY(table_update<act_t>(w, reinterpret_cast<act_t*>(m->base + p.hv), m->at<float>(p.hv_state), c.v_rows, a,
                             m->at<int32_t>(p.rows_v), m->at<float>(p.gv), N, lr_t, c.table_beta, c.table_eps,
                             nullptr, nullptr, err, st));
-  if (c.x0_rows)
+  }
+  if (c.x0_rows) {
+    ProfScope ps(pf, st, "table_update", 0.0, (double)N * d * 4);
     TRY(table_update<act_t>(w, reinterpret_cast<act_t*>(m->base + p.hx), m->at<float>(p.hx_state), c.x0_rows, d,
                             m->at<int32_t>(p.rows_x), dx, N, lr_t, c.table_beta, c.table_eps, nullptr, nullptr, err, st));
-  // ---- dense step every grad_accum calls
+  }
   m->micro += 1;
-  if (m->micro == c.grad_accum) {
+  m->have_fwd = false;
+  if (do_step && m->micro == c.grad_accum) return optimizer_step_impl(m, lr);
+  return GPT_OK;
+}
+
+// Global-norm clip (optional) and AdamW over the accumulated dense gradient.
+static int optimizer_step_impl(gpt_model* m, float lr) {
+  const gpt_config& c = m->cfg;
+  const Plan& p = m->plan;
+  const bool b16 = cfg_bf16(c);
+  cudaStream_t st = m->st;
+  unsigned* err = m->err();
+  ProfScope ps(&m->prof, st, "adamw", 0.0, (double)p.dense_n * (b16 ? 30 : 28));
+  {
     m->micro = 0;
     m->step_t += 1;
     float* coef = nullptr;
     if (c.grad_clip > 0.f) {
-      sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, st>>>(m->at<float>(p.G), p.dense_n, m->at<double>(p.norm_part));
-      clip_coef_kernel<<<1, 256, 0, st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, c.grad_clip,
+      ++g_launches; sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, st>>>(m->at<float>(p.G), p.dense_n, m->at<double>(p.norm_part));
+      ++g_launches; clip_coef_kernel<<<1, 256, 0, st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, c.grad_clip,
                                          m->at<float>(p.clip_coef), m->at<float>(p.grad_norm), err);
       LAUNCH_CHECK();
       coef = m->at<float>(p.clip_coef);
@@ -842,10 +991,9 @@ static int backward_impl(gpt_model* m, float lr) {
     aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
     aa.bc2 = (float)(1.0 - pow((double)c.adam_b2, (double)m->step_t));
     aa.clip = coef;
-    adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
+    ++g_launches; adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
     LAUNCH_CHECK();
   }
-  m->have_fwd = false;
   return GPT_OK;
 }
 
@@ -859,8 +1007,69 @@ extern "C" int gpt_backward_step(gpt_model* m, float lr) {
   if (!m) return fail(GPT_ERR_ARG, "null model");
   if (!m->have_fwd) return fail(GPT_ERR_STATE, "gpt_backward_step needs a preceding gpt_forward_loss");
   if (!std::isfinite(lr)) return fail(GPT_ERR_ARG, "learning rate not finite");
-  if (cfg_bf16(m->cfg)) return backward_impl<bf16>(m, lr);
-  return backward_impl<float>(m, lr);
+  if (cfg_bf16(m->cfg)) return backward_impl<bf16>(m, lr, true);
+  return backward_impl<float>(m, lr, true);
+}
+
+extern "C" int gpt_backward(gpt_model* m, float lr) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  if (!m->have_fwd) return fail(GPT_ERR_STATE, "gpt_backward needs a preceding gpt_forward_loss");
+  if (!std::isfinite(lr)) return fail(GPT_ERR_ARG, "learning rate not finite");
+  if (cfg_bf16(m->cfg)) return backward_impl<bf16>(m, lr, false);
+  return backward_impl<float>(m, lr, false);
+}
+
+extern "C" int gpt_optimizer_step(gpt_model* m, float lr) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  if (m->micro == 0) return fail(GPT_ERR_STATE, "gpt_optimizer_step needs at least one gpt_backward");
+  if (!std::isfinite(lr)) return fail(GPT_ERR_ARG, "learning rate not finite");
+  return optimizer_step_impl(m, lr);
+}
+
+extern "C" int gpt_launch_count(long long* n) {
+  if (!n) return fail(GPT_ERR_ARG, "null pointer");
+  *n = g_launches.load();
+  return GPT_OK;
+}
+
+extern "C" int gpt_profile_enable(gpt_model* m, int on) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  if (on) {
+    m->prof.recs.clear();
+    m->prof.used = 0;
+  }
+  m->prof.on = on != 0;
+  return GPT_OK;
+}
+
+extern "C" int gpt_profile_read(gpt_model* m, gpt_prof_entry* out, int cap, int* n) {
+  if (!m || !n || (cap > 0 && !out)) return fail(GPT_ERR_ARG, "null argument");
+  CUDA_TRY(cudaStreamSynchronize(m->st));
+  std::vector<gpt_prof_entry> agg;
+  for (const ProfRec& r : m->prof.recs) {
+    float ms = 0.f;
+    CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    gpt_prof_entry* e = nullptr;
+    for (auto& x : agg)
+      if (strncmp(x.name, r.cls, sizeof(x.name)) == 0) e = &x;
+    if (!e) {
+      gpt_prof_entry z;
+      memset(&z, 0, sizeof(z));
+      strncpy(z.name, r.cls, sizeof(z.name) - 1);
+      agg.push_back(z);
+      e = &agg.back();
+    }
+    e->scopes += 1;
+    e->launches += r.launches;
+    e->ms += ms;
+    e->flops += r.flops;
+    e->bytes += r.bytes;
+  }
+  *n = (int)agg.size();
+  for (int i = 0; i < (int)agg.size() && i < cap; ++i) out[i] = agg[i];
+  m->prof.recs.clear();
+  m->prof.used = 0;
+  return GPT_OK;
 }
 
 // ======================================================================== standalone ngram
@@ -871,7 +1080,7 @@ extern "C" int ngram_hash(const int32_t* tokens, int B, int T, int vocab, unsign
   if ((long long)B * T == 0) return GPT_OK;
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
-  ngram_hash_kernel<<<grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream>>>(
+  ++g_launches; ngram_hash_kernel<<<grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream>>>(
       tokens, B, T, vocab, p1, p2, rows, rows_out, 1, nullptr, err);
   LAUNCH_CHECK();
   return GPT_OK;
@@ -885,14 +1094,15 @@ extern "C" int ngram_gather(const int32_t* rows, int n, const void* table, long 
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
   const int grid = grid_for((long long)n * 32, 256);
-  if (dtype == GPT_DTYPE_BF16)
-    ngram_gather_kernel<bf16><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows, d,
+  if (dtype == GPT_DTYPE_BF16) {
+    ++g_launches; ngram_gather_kernel<bf16><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows, d,
                                                                       (bf16*)out, accumulate, err);
-  else if (dtype == GPT_DTYPE_F32)
-    ngram_gather_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const float*)table, n_rows, d,
+  } else if (dtype == GPT_DTYPE_F32) {
+    ++g_launches; ngram_gather_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const float*)table, n_rows, d,
                                                                        (float*)out, accumulate, err);
-  else
+  } else {
     return fail(GPT_ERR_ARG, "ngram_gather: dtype must be F32 or BF16");
+  }
   LAUNCH_CHECK();
   return GPT_OK;
 }

@@ -151,6 +151,18 @@ int gpt_forward_loss(gpt_model* m, const int32_t* tokens_dev, const int32_t* tar
  */
 int gpt_backward_step(gpt_model* m, float lr);
 
+/*
+ * The two halves of gpt_backward_step, for callers that exchange gradients
+ * between them (data-parallel training): gpt_backward() runs the backward pass
+ * and the table updates and accumulates the dense gradient without stepping;
+ * gpt_optimizer_step() applies the clip and AdamW to whatever gradient has
+ * accumulated (at least one gpt_backward since the last step), then starts a
+ * new accumulation.  gpt_backward_step(m, lr) equals gpt_backward(m, lr)
+ * followed, on every grad_accum-th call, by gpt_optimizer_step(m, lr).
+ */
+int gpt_backward(gpt_model* m, float lr);
+int gpt_optimizer_step(gpt_model* m, float lr);
+
 /* Dense (matmul + embedding) and table parameter counts.  Host only. */
 int gpt_num_params(const gpt_model* m, long long* dense, long long* table);
 
@@ -163,7 +175,11 @@ int gpt_flops_per_token(const gpt_config* cfg, long long* flops, long long* flop
  * "wte", "lm_head" (untied only), "h<l>.wqkv" [3*H*hd, d] (rows q|k|v),
  * "h<l>.wo" [d, H*hd], "h<l>.w1" [d_ff, d], "h<l>.w2" [d, d_ff], "hx", "hv";
  * kind GPT_KIND_ACT: "per_token_loss" [B, T] fp32, "rows_x" / "rows_v" [B, T]
- * int32.  Writes the device pointer, its element type and up to four dims
+ * int32, "grad_norm" (fp32 scalar, set when grad_clip > 0).  The name "*"
+ * with kind PARAM / GRAD / ADAM_M / ADAM_V is the whole flat fp32 dense
+ * buffer [n] (each tensor padded to a multiple of 64 elements, pads zero),
+ * e.g. for an all-reduce of the gradient between gpt_backward and
+ * gpt_optimizer_step.  Writes the device pointer, its element type and up to four dims
  * (unused dims are 1).  Host only, no synchronisation.  After writing
  * PARAM tensors from outside, call gpt_params_changed().
  */
@@ -172,6 +188,28 @@ int gpt_tensor(gpt_model* m, const char* name, int kind, void** dev_ptr, int* dt
 
 /* Re-derive the bf16 GEMM copies from the fp32 master weights (enqueued). */
 int gpt_params_changed(gpt_model* m);
+
+/*
+ * Live timing: while enabled, every kernel (or fixed group of kernels) the
+ * model enqueues is bracketed by CUDA events on the model's stream.
+ * gpt_profile_read() synchronises, sums elapsed time, launches and the
+ * algorithmic FLOPs / bytes per kernel class ("gemm", "attention_fwd",
+ * "rmsnorm_fwd", "table_update", "adamw", ...) into out[0..cap), sets *n to
+ * the number of classes, and clears the records.  Enabling (on = 1) clears.
+ */
+typedef struct gpt_prof_entry {
+  char name[32];
+  long long scopes;    /* bracketed groups */
+  long long launches;  /* kernels launched inside them */
+  double ms;           /* summed CUDA-event time */
+  double flops;        /* algorithmic FLOPs (contractions) */
+  double bytes;        /* algorithmic bytes (memory-bound kernels) */
+} gpt_prof_entry;
+int gpt_profile_enable(gpt_model* m, int on);
+int gpt_profile_read(gpt_model* m, gpt_prof_entry* out, int cap, int* n);
+
+/* Number of CUDA kernels this library has launched in this process.  Host only. */
+int gpt_launch_count(long long* n);
 
 /* Synchronise the model's stream, read and clear the device error word. */
 int gpt_sync_status(gpt_model* m);

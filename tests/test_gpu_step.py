@@ -124,3 +124,10 @@ def test_out_of_range_token_reports_input_error(g):
     model.forward_loss(device_ints(tok), device_ints(tgt))
     assert model.sync_status() == g.GPT_ERR_INPUT
     assert model.sync_status() == g.GPT_OK
+
+
+def test_bf16_long_ragged_sequence(g):
+    # T = 520: several 128-row query tiles and 64-key tiles with a ragged tail
+    w = small_case("gpt2s_bf16", n_layer=1, seq_len=520, micro_batch=1, vocab=1024, grad_accum=2)
+    model, orc, losses, _ = run_pair(g, w, steps=2)
+    check(g, w, model, orc, losses, 1e-2, 2e-2)
