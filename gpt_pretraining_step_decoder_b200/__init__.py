@@ -74,7 +74,7 @@ _SIGS = {
     "ngram_sparse_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
     "ngram_sparse_update": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P, _SZ, _P],
     "ngram_sync_status": [_P],
-    "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _SZ, _P],
+    "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -248,10 +248,13 @@ def ngram_sync_status(stream=None):
     return _lib.ngram_sync_status(_stream(stream))
 
 
-def gptx_gemm_bf16(M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, C, ldc, beta, splits, workspace,
-                   ws_bytes, stream=None):
-    return _check(_lib.gptx_gemm_bf16(M, N, K, _ptr(A), lda, a_kmajor, _ptr(B), ldb, b_kmajor,
-                                      _ptr(C), ldc, beta, splits, _ptr(workspace), ws_bytes,
+EPI_STORE, EPI_STORE_F32, EPI_ACCUM_F32, EPI_RELU2, EPI_DRELU2, EPI_LOGITS = range(6)
+
+
+def gptx_gemm_bf16(M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, C, ldc, beta=0, splits=1,
+                   workspace=None, ws_bytes=0, stream=None, mode=EPI_ACCUM_F32, aux=None):
+    return _check(_lib.gptx_gemm_bf16(M, N, K, _ptr(A), lda, a_kmajor, _ptr(B), ldb, b_kmajor, mode,
+                                      _ptr(C), ldc, _ptr(aux), beta, splits, _ptr(workspace), ws_bytes,
                                       _stream(stream)), "gptx_gemm_bf16")
 
 

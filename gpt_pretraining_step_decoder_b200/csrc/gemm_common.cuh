@@ -18,18 +18,23 @@ enum EpiMode {
   EPI_STORE = 0,      // C(act) = alpha * acc
   EPI_STORE_F32 = 1,  // C(f32) = alpha * acc
   EPI_ACCUM_F32 = 2,  // C(f32) = (beta ? C : 0) + alpha * acc
-  EPI_RELU2 = 3,      // r = relu(acc): C(act) = r, C2(act) = r * r
-  EPI_DRELU2 = 4,     // C(act) = 2 * aux(act) * acc   (ReLU^2 backward)
+  EPI_RELU2 = 3,      // C(act) = relu(acc)^2                        (ReLU^2 forward)
+  EPI_DRELU2 = 4,     // C(act) = 2 * sqrt(aux(act)) * acc, aux = relu(a)^2  (ReLU^2 backward:
+                      // d relu(a)^2 / da = 2 relu(a) = 2 sqrt(relu(a)^2))
+  EPI_LOGITS = 5,     // z = softcap(acc): C(f32) = z, and per (row, column tile) the
+                      // running max and sum of exp(z - max) into stats (tensor-core path)
 };
 
 struct GemmEpilogue {
   int mode;
   void* C;          // output [M, ldc]
   long long ldc;
-  void* C2;         // second output (EPI_RELU2), same ld as C
-  const void* aux;  // EPI_DRELU2 input, same ld as C
+  void* C2;         // unused second output
+  const void* aux;  // EPI_DRELU2 input relu(a)^2, same ld as C
   float alpha;
   int beta;
+  float softcap;    // EPI_LOGITS: 0 = off, else z = softcap * tanh(acc / softcap)
+  float2* stats;    // EPI_LOGITS: [M, n_tiles] (max, sum of exp(z - max))
 };
 
 template <typename act_t>
@@ -46,16 +51,18 @@ __device__ __forceinline__ void epi_apply_one(const GemmEpilogue& e, long long m
       break;
     }
     case EPI_RELU2: {
-      float r = fmaxf(acc, 0.f);
-      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(r);
-      reinterpret_cast<act_t*>(e.C2)[off] = from_f<act_t>(r * r);
+      const float r = fmaxf(acc, 0.f);
+      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(r * r);
       break;
     }
     case EPI_DRELU2: {
-      float r = to_f(reinterpret_cast<const act_t*>(e.aux)[off]);
-      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(2.f * r * acc);
+      const float g = to_f(reinterpret_cast<const act_t*>(e.aux)[off]);
+      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(2.f * sqrtf(g) * acc);
       break;
     }
+    case EPI_LOGITS:
+      reinterpret_cast<float*>(e.C)[off] = acc;
+      break;
   }
 }
 

@@ -11,7 +11,9 @@
 //               TMEM accumulators, committing to mbarriers;
 //   warps 2..5  the epilogue: tcgen05.ld of the finished accumulator (one
 //               TMEM lane = one output row per thread), apply the epilogue,
-//               store to global, release the accumulator.
+//               stage 128-byte rows in shared memory and write them with
+//               asynchronous TMA stores (TMA reduce-add for fp32
+//               accumulation), then release the accumulator.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i + 1.  K-major and MN-major operands are both read straight from their
 // row-major buffers (the UMMA descriptor's major-ness bit), so forward,
@@ -30,13 +32,31 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // bf16 elements per 128-byte swizzle row
 constexpr int NUM_THREADS = 192;
 
-template <int BN> struct Cfg {
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+// Epilogue kind of one kernel instantiation (compile time, so each kernel
+// carries only its own epilogue code).
+enum KMode {
+  K_STORE = 0,    // bf16 output
+  K_STORE_F32,    // fp32 output (also accumulate with beta = 0)
+  K_REDUCE_F32,   // fp32 C += acc by TMA reduce-add (accumulate with beta = 1)
+  K_PARTIAL,      // split-K fp32 partials [splits, M, N]
+  K_RELU2,        // bf16 relu(acc)^2
+  K_DRELU2,       // bf16 2 sqrt(aux) acc
+  K_LOGITS,       // fp32 softcap(acc) + per-tile row statistics
+};
+
+// HEAVY = 1: the epilogue-heavy variant (logits, ReLU^2 backward) trades one
+// pipeline stage for double-buffered staging and a whole-tile activation buffer.
+template <int BN, int HEAVY> struct Cfg {
+  static constexpr int STAGES = (BN == 256) ? (HEAVY ? 3 : 4) : (HEAVY ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators (power of two >= 32)
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int NSTG = HEAVY ? 2 : 1;          // staging buffers per epilogue warp
+  static constexpr int NAUX = HEAVY ? 2 : 1;          // activation blocks in flight per epilogue warp
+  static constexpr int AUX = NAUX * 32 * 128;         // activation bytes per epilogue warp
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * NSTG * 32 * 128 + 4 * AUX + 1024 /*align*/ +
+                                    256 /*barriers*/;
 };
 
 struct Params {
@@ -159,104 +179,79 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kmajor, int 
   return smem_desc(base + k * 16 * 128, 64 * BK * 2, 1024);
 }
 
-template <typename act_t>
-__device__ __forceinline__ void epilogue_row32(const Params& p, long long m, int n0,
-                                               const uint32_t (&r)[32], int split) {
-  const GemmEpilogue& e = p.epi;
-  float v[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  if (m >= p.M) return;
-  if (p.splits > 1) {
-    float* dst = p.partial + ((long long)split * p.M + m) * p.N + n0;
-    if (n0 + 32 <= p.N) {
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) store4(dst + i, &v[i]);
-    } else {
-      for (int i = 0; i < 32 && n0 + i < p.N; ++i) dst[i] = v[i];
-    }
-    return;
-  }
-  if (n0 + 32 > p.N) {
-    for (int i = 0; i < 32 && n0 + i < p.N; ++i) epi_apply_one<act_t>(e, m, n0 + i, v[i]);
-    return;
-  }
-  const long long off = m * e.ldc + n0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] *= e.alpha;
-  switch (e.mode) {
-    case EPI_STORE: {
-      act_t* c = reinterpret_cast<act_t*>(e.C) + off;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) store4(c + i, &v[i]);
-      break;
-    }
-    case EPI_STORE_F32: {
-      float* c = reinterpret_cast<float*>(e.C) + off;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) store4(c + i, &v[i]);
-      break;
-    }
-    case EPI_ACCUM_F32: {
-      float* c = reinterpret_cast<float*>(e.C) + off;
-      if (e.beta) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float o[4];
-          load4(c + i, o);
-          o[0] += v[i]; o[1] += v[i + 1]; o[2] += v[i + 2]; o[3] += v[i + 3];
-          store4(c + i, o);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) store4(c + i, &v[i]);
-      }
-      break;
-    }
-    case EPI_RELU2: {
-      act_t* c = reinterpret_cast<act_t*>(e.C) + off;
-      act_t* c2 = reinterpret_cast<act_t*>(e.C2) + off;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        float rr[4], gg[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) { rr[j] = fmaxf(v[i + j], 0.f); gg[j] = rr[j] * rr[j]; }
-        store4(c + i, rr);
-        store4(c2 + i, gg);
-      }
-      break;
-    }
-    case EPI_DRELU2: {
-      act_t* c = reinterpret_cast<act_t*>(e.C) + off;
-      const act_t* a = reinterpret_cast<const act_t*>(e.aux) + off;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        float rr[4], o[4];
-        load4(a + i, rr);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = 2.f * rr[j] * v[i + j];
-        store4(c + i, o);
-      }
-      break;
-    }
-  }
-}
+// ------------------------------------------------------------------ epilogue
+// Each epilogue warp owns 32 output rows (its TMEM lane quarter) and walks the
+// tile in column blocks of 32 fp32 (fp32 outputs) or 64 bf16 (bf16 outputs),
+// i.e. 128-byte rows.  TMEM -> registers (one row per lane; row-local work such
+// as the cross-entropy statistics happens here) -> a 32 x 128-byte staging
+// block in shared memory written in the TMA 128-byte swizzle (conflict-free)
+// -> one asynchronous TMA store, or a TMA reduce-add when the product is
+// accumulated into an fp32 buffer (residual stream, weight gradients).  The
+// ReLU^2 backward's second input is brought in by TMA one block ahead.
+constexpr int STG_BYTES = 32 * 128;  // per epilogue warp
+constexpr int AUX_BYTES = 32 * 128;
 
-template <int BN, typename act_t>
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// byte offset of 16-byte chunk j of row r in a 128-byte-swizzled block
+__device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
+
+template <int BN, int KM, typename act_t>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmAux,
                    const Params p) {
-  using C = Cfg<BN>;
+  constexpr int HEAVY = (KM == K_DRELU2 || KM == K_LOGITS) ? 1 : 0;
+  using C = Cfg<BN, HEAVY>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* stg_all = smem + C::STAGES * C::STAGE_BYTES;
+  uint8_t* aux_all = stg_all + 4 * C::NSTG * STG_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(aux_all + 4 * C::AUX);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* auxbar = tempty + 2;  // NAUX per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -265,6 +260,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 128); }
+    for (int s = 0; s < 8; ++s) mbar_init(&auxbar[s], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -353,25 +349,157 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp - 2;
+    uint8_t* stg_base = stg_all + ew * C::NSTG * STG_BYTES;
+    uint8_t* auxs = aux_all + ew * C::AUX;
+    int sbuf = 0;
+    uint64_t* abar = &auxbar[ew * 2];   // abar[b] guards activation buffer b
+    uint32_t aux_phase = 0;             // bit b: parity of the next wait on abar[b]
+    uint32_t aux_pending = 0;           // bit b: a load into buffer b is in flight
+    const GemmEpilogue& e = p.epi;
+    constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL || KM == K_LOGITS;
+    constexpr bool has_aux = KM == K_DRELU2;
+    constexpr int CW = f32out ? 32 : 64;  // columns per 128-byte staging row
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int split = t % p.splits;
       const int mn = t / p.splits;
-      const long long m0 = (long long)(mn / p.n_tiles) * BM;
+      const int m0 = (mn / p.n_tiles) * BM;
       const int n0 = (mn % p.n_tiles) * BN;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) break;
-      tc_fence_after();
-      const long long m = m0 + q * 32 + lane;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
-        if (n0 + c * 32 < p.N) epilogue_row32<act_t>(p, m, n0 + c * 32, r, split);
+      const int mrow0 = m0 + q * 32;
+      const long long m = (long long)mrow0 + lane;
+      const int nblk = min(BN / CW, (p.N - n0 + CW - 1) / CW);
+      if (has_aux) {  // the tile's first ReLU^2 activation blocks, ahead of the accumulator
+        for (int b = 0; b < C::NAUX && b < nblk; ++b) {
+          if (lane == 0) {
+            mbar_expect_tx(&abar[b], AUX_BYTES);
+            tma_load_2d(auxs + b * AUX_BYTES, &tmAux, &abar[b], n0 + b * 64, mrow0);
+          }
+          aux_pending |= 1u << b;
+        }
       }
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) { ok = false; break; }
+      tc_fence_after();
+      float rmax = -INFINITY, rsum = 0.f;
+      const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < nblk; ++c) {
+        const int nc = n0 + c * CW;
+        float v[64];
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_nowait(trow + c * CW, r0);
+          if (CW == 64) tmem_ld32_nowait(trow + c * CW + 32, r1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r0[i]) * e.alpha;
+          if (CW == 64) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[32 + i] = __uint_as_float(r1[i]) * e.alpha;
+          }
+        }
+        if constexpr (KM == K_LOGITS) {
+          const int nv = min(32, p.N - nc);
+          if (e.softcap > 0.f) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = e.softcap * tanhf(v[i] / e.softcap);
+          }
+          float cmax = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) cmax = fmaxf(cmax, v[i]);
+          const float nm = fmaxf(rmax, cmax);
+          float s = (rmax == -INFINITY) ? 0.f : rsum * __expf(rmax - nm);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) s += __expf(v[i] - nm);
+          rmax = nm;
+          rsum = s;
+        } else if constexpr (KM == K_RELU2) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) { const float r = fmaxf(v[i], 0.f); v[i] = r * r; }
+        } else if constexpr (KM == K_DRELU2) {
+          const int b = c % C::NAUX;
+          if (!mbar_wait(&abar[b], (aux_phase >> b) & 1u, abort_flag, p.err)) { ok = false; break; }
+          aux_phase ^= 1u << b;
+          aux_pending &= ~(1u << b);
+          const uint8_t* ab = auxs + b * AUX_BYTES;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(ab + swz128(lane, j));
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              // d relu(a)^2 / da = 2 relu(a) = 2 g rsqrt(g) for g = relu(a)^2 > 0
+              const float2 gg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+              v[j * 8 + 2 * h] *= gg.x > 0.f ? 2.f * gg.x * rsqrtf(gg.x) : 0.f;
+              v[j * 8 + 2 * h + 1] *= gg.y > 0.f ? 2.f * gg.y * rsqrtf(gg.y) : 0.f;
+            }
+          }
+          __syncwarp();
+          if (c + C::NAUX < nblk) {  // refill this buffer NAUX blocks ahead
+            if (lane == 0) {
+              mbar_expect_tx(&abar[b], AUX_BYTES);
+              tma_load_2d(auxs + b * AUX_BYTES, &tmAux, &abar[b], nc + C::NAUX * 64, mrow0);
+            }
+            aux_pending |= 1u << b;
+          }
+        }
+        // the TMA store that last used this staging block must have read it
+        uint8_t* stg = stg_base + sbuf * STG_BYTES;
+        if (lane == 0) {
+          if (C::NSTG == 2) bulk_wait_read1();
+          else bulk_wait_read0();
+        }
+        __syncwarp();
+        if (f32out) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(stg + swz128(lane, j)) =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4 o;
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * j], v[8 * j + 1]);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * j + 2], v[8 * j + 3]);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * j + 4], v[8 * j + 5]);
+            __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * j + 6], v[8 * j + 7]);
+            o.x = *reinterpret_cast<uint32_t*>(&b0);
+            o.y = *reinterpret_cast<uint32_t*>(&b1);
+            o.z = *reinterpret_cast<uint32_t*>(&b2);
+            o.w = *reinterpret_cast<uint32_t*>(&b3);
+            *reinterpret_cast<uint4*>(stg + swz128(lane, j)) = o;
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (KM == K_PARTIAL) tma_store_3d(&tmC, stg, nc, mrow0, split);
+          else if constexpr (KM == K_REDUCE_F32) tma_reduce_add_2d(&tmC, stg, nc, mrow0);
+          else tma_store_2d(&tmC, stg, nc, mrow0);
+          bulk_commit();
+        }
+        sbuf = (sbuf + 1) % C::NSTG;
+      }
+      if (!ok) break;
+      if (KM == K_LOGITS && m < p.M) e.stats[m * p.n_tiles + (mn % p.n_tiles)] = make_float2(rmax, rsum);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (lane == 0) bulk_wait0();  // all of this warp's stores are complete
+    if (has_aux && lane == 0) {
+      // an aborted tile may leave activation loads in flight: let them land
+      for (int b = 0; b < C::NAUX; ++b) {
+        if (!((aux_pending >> b) & 1u)) continue;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&abar[b], (aux_phase >> b) & 1u)) {
+          if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
+        }
+      }
     }
   }
   tc_fence_before();

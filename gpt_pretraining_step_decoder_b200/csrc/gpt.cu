@@ -28,6 +28,21 @@
 #include "ngram.cuh"
 #include "optim.cuh"
 
+// Run the statements with NV = d / 128 (vec4 chunks per lane of a row kernel)
+// as a compile-time constant; rows that are not a multiple of 128 use MAXV.
+#define WITH_NV(d, ...);                                      \
+  do {                                                       \
+    switch (((d) % 128 == 0) ? (d) / 128 : 0) {              \
+      case 1: { constexpr int NV = 1; __VA_ARGS__; } break;  \
+      case 2: { constexpr int NV = 2; __VA_ARGS__; } break;  \
+      case 4: { constexpr int NV = 4; __VA_ARGS__; } break;  \
+      case 6: { constexpr int NV = 6; __VA_ARGS__; } break;  \
+      case 8: { constexpr int NV = 8; __VA_ARGS__; } break;  \
+      case 16: { constexpr int NV = 16; __VA_ARGS__; } break; \
+      default: { constexpr int NV = MAXV; __VA_ARGS__; } break; \
+    }                                                        \
+  } while (0)
+
 // ======================================================================== errors
 static thread_local std::string g_last_error;
 
@@ -85,37 +100,57 @@ static int get_encode() {
   return GPT_OK;
 }
 
-// 2-D bf16 map over a row-major [outer, inner] buffer with row pitch `ld`
-// elements, 128-byte swizzle, zero fill outside the tensor.
-static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
-                     uint32_t box_inner, uint32_t box_outer) {
+// Tensor map of `rank` dims (innermost first) with byte strides for dims 1..,
+// 128-byte swizzle, zero fill outside the tensor.
+static int make_tmap_gen(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
+                         const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   TRY(get_encode());
-  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((ld * 2) & 15))
-    return fail(GPT_ERR_ARG, "TMA operand not 16-byte aligned (ptr %p, ld %llu)", ptr,
-                (unsigned long long)ld);
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (reinterpret_cast<uintptr_t>(ptr) & 15) return fail(GPT_ERR_ARG, "TMA operand %p not 16-byte aligned", ptr);
+  for (int i = 0; i + 1 < rank; ++i)
+    if (strides_bytes[i] & 15) return fail(GPT_ERR_ARG, "TMA row pitch %llu not a multiple of 16 bytes",
+                                           (unsigned long long)strides_bytes[i]);
+  cuuint64_t d[3], s[2];
+  cuuint32_t b[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  CUresult r = g_encode(m, dt, rank, const_cast<void*>(ptr), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(GPT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return GPT_OK;
 }
 
+// 2-D bf16 map over a row-major [outer, inner] buffer with row pitch `ld` elements.
+static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_inner, uint32_t box_outer) {
+  const uint64_t dims[2] = {inner, outer}, str[1] = {ld * 2};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return make_tmap_gen(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, str, box);
+}
+
 // ======================================================================== GEMM dispatch
-template <int BN>
-static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
-                          int splits, float* partial, unsigned* err, cudaStream_t st) {
-  using C = tc::Cfg<BN>;
+template <int BN, int KM>
+static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tcm,
+                            const CUtensorMap& taux, const tc::Params& p, cudaStream_t st) {
+  using C = tc::Cfg<BN, (KM == tc::K_DRELU2 || KM == tc::K_LOGITS) ? 1 : 0>;
+  static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
   static bool attr_done = false;
   if (!attr_done) {
-    CUDA_TRY(cudaFuncSetAttribute(tc::gemm_tc_kernel<BN, bf16>,
+    CUDA_TRY(cudaFuncSetAttribute(tc::gemm_tc_kernel<BN, KM, bf16>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     attr_done = true;
   }
-  CUtensorMap ta, tb;
+  const int tiles = p.m_tiles * p.n_tiles * p.splits;
+  const int grid = tiles < device_sms() ? tiles : device_sms();
+  ++g_launches; tc::gemm_tc_kernel<BN, KM, bf16><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, tcm, taux, p);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+template <int BN>
+static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
+                          int splits, float* partial, unsigned* err, cudaStream_t st) {
+  CUtensorMap ta, tb, tcm, taux;
   if (A.kmajor) TRY(make_tmap(&ta, A.ptr, K, M, A.ld, tc::BK, tc::BM));
   else TRY(make_tmap(&ta, A.ptr, M, K, A.ld, 64, tc::BK));
   if (B.kmajor) TRY(make_tmap(&tb, B.ptr, K, N, B.ld, tc::BK, BN));
@@ -133,10 +168,39 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   p.epi = e;
   p.partial = partial;
   p.err = err;
-  const int tiles = p.m_tiles * p.n_tiles * p.splits;
-  const int grid = tiles < device_sms() ? tiles : device_sms();
-  ++g_launches; tc::gemm_tc_kernel<BN, bf16><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
-  LAUNCH_CHECK();
+  // output map: split-K partials [splits, M, N] fp32 (3-D so each split clips at M),
+  // fp32 outputs in 32-column boxes, bf16 outputs in 64-column boxes (128-byte rows)
+  if (p.splits > 1) {
+    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)M, (uint64_t)p.splits};
+    const uint64_t str[2] = {(uint64_t)N * 4, (uint64_t)M * N * 4};
+    const uint32_t box[3] = {32, 32, 1};
+    TRY(make_tmap_gen(&tcm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, partial, dims, str, box));
+  } else if (e.mode == EPI_STORE_F32 || e.mode == EPI_ACCUM_F32 || e.mode == EPI_LOGITS) {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M}, str[1] = {(uint64_t)e.ldc * 4};
+    const uint32_t box[2] = {32, 32};
+    TRY(make_tmap_gen(&tcm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, e.C, dims, str, box));
+  } else {
+    TRY(make_tmap(&tcm, e.C, N, M, e.ldc, 64, 32));
+  }
+  if (p.splits == 1 && e.mode == EPI_DRELU2) TRY(make_tmap(&taux, e.aux, N, M, e.ldc, 64, 32));
+  else taux = tcm;
+  int km;
+  if (p.splits > 1) km = tc::K_PARTIAL;
+  else if (e.mode == EPI_STORE) km = tc::K_STORE;
+  else if (e.mode == EPI_STORE_F32 || (e.mode == EPI_ACCUM_F32 && !e.beta)) km = tc::K_STORE_F32;
+  else if (e.mode == EPI_ACCUM_F32) km = tc::K_REDUCE_F32;
+  else if (e.mode == EPI_RELU2) km = tc::K_RELU2;
+  else if (e.mode == EPI_DRELU2) km = tc::K_DRELU2;
+  else km = tc::K_LOGITS;
+  switch (km) {
+    case tc::K_STORE: TRY((gemm_tc_launch_k<BN, tc::K_STORE>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_REDUCE_F32: TRY((gemm_tc_launch_k<BN, tc::K_REDUCE_F32>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_RELU2: TRY((gemm_tc_launch_k<BN, tc::K_RELU2>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_DRELU2: TRY((gemm_tc_launch_k<BN, tc::K_DRELU2>(ta, tb, tcm, taux, p, st))); break;
+    default: TRY((gemm_tc_launch_k<BN, tc::K_LOGITS>(ta, tb, tcm, taux, p, st))); break;
+  }
   if (p.splits > 1) {
     const long long total = (long long)M * N;
     int blocks = (int)((total + 255) / 256);
@@ -213,9 +277,9 @@ struct GemmCtx {
 };
 
 static int gemm(const GemmCtx& g, int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
-                bool allow_split = false) {
+                bool allow_split = false, const char* label = "gemm") {
   if (M <= 0 || N <= 0 || K <= 0) return GPT_OK;
-  ProfScope ps(g.prof, g.st, "gemm", 2.0 * M * N * K, 0.0);
+  ProfScope ps(g.prof, g.st, label, 2.0 * M * N * K, 0.0);
   if (!g.bf16) {
     gemm_simt<float, float>(M, N, K, A, B, e, g.st);
     LAUNCH_CHECK();
@@ -237,6 +301,7 @@ static GemmEpilogue epi(int mode, void* C, long long ldc, int beta = 0, void* C2
                         const void* aux = nullptr, float alpha = 1.f) {
   GemmEpilogue e;
   e.mode = mode; e.C = C; e.ldc = ldc; e.C2 = C2; e.aux = aux; e.alpha = alpha; e.beta = beta;
+  e.softcap = 0.f; e.stats = nullptr;
   return e;
 }
 
@@ -258,7 +323,7 @@ struct DenseTensor {
 };
 
 struct LayerActs {
-  size_t u, rstd1, qkv, rstd_q, rstd_k, o, lse, u2, rstd2, r, g;
+  size_t u, rstd1, qkv, rstd_q, rstd_k, o, lse, u2, rstd2, g;
 };
 
 struct Plan {
@@ -270,7 +335,7 @@ struct Plan {
   size_t x, emb_rstd, xf, rstd_f, tok_copy, rows_x, rows_v;
   std::vector<LayerActs> layers;
   size_t dx, dx_lp, du, dqkv, da, dout, Dattn, gv, dxf, pending;
-  size_t logits, dz, tok_loss, ce_scale, ce_count, loss_scratch;
+  size_t logits, dz, ce_stats, tok_loss, ce_scale, ce_count, loss_scratch;
   size_t sort_keys_a, sort_keys_b, sort_vals_a, sort_vals_b, sort_counts;
   size_t seg_start, pstart, plen, pseg, pslot, lfirst, lnslots, lseg, counters, seg_partial;
   size_t splitk; long long splitk_elems;
@@ -358,7 +423,6 @@ static void make_plan(const gpt_config& c, Plan& p) {
     L.lse = cv.take(BH * c.seq_len * 4);
     L.u2 = cv.take(N * d * es);
     L.rstd2 = cv.take(N * 4);
-    L.r = cv.take(N * F * es);
     L.g = cv.take(N * F * es);
   }
   p.xf = cv.take(N * d * es);
@@ -380,6 +444,7 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.chunk = (int)chunk;
   p.logits = cv.take(chunk * V * 4);
   p.dz = cv.take(chunk * V * es);
+  p.ce_stats = cv.take(chunk * ((V + 127) / 128) * 8);
   p.tok_loss = cv.take(N * 4);
   p.ce_scale = cv.take(4);
   p.ce_count = cv.take(4);
@@ -692,10 +757,10 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const int32_t* perm;
   TRY(bucket_by_key(w, rows, n, n_rows, &skeys, &perm, uniq_out, n_uniq_out, err, st));
   const long long maxp = (long long)n + n / PIECE + 2, maxl = n / PIECE + 2;
-  ++g_launches; table_piece_kernel<tab_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
-      table, state, d, grad, skeys, perm, w.pstart, w.plen, w.pslot, w.counters, w.partial, lr, beta, eps);
-  ++g_launches; table_long_kernel<tab_t><<<grid_for(maxl * 32, 256), 256, 0, st>>>(
-      table, state, d, skeys, w.seg_start, w.lfirst, w.lnslots, w.lseg, w.counters, w.partial, lr, beta, eps);
+  WITH_NV(d, ++g_launches; table_piece_kernel<NV, tab_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
+      table, state, d, grad, skeys, perm, w.pstart, w.plen, w.pslot, w.counters, w.partial, lr, beta, eps););
+  WITH_NV(d, ++g_launches; table_long_kernel<NV, tab_t><<<grid_for(maxl * 32, 256), 256, 0, st>>>(
+      table, state, d, skeys, w.seg_start, w.lfirst, w.lnslots, w.lseg, w.counters, w.partial, lr, beta, eps););
   LAUNCH_CHECK();
   return GPT_OK;
 }
@@ -791,9 +856,9 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   float* x = m->at<float>(p.x);
   {
   ProfScope ps(pf, st, "embed", 0.0, (double)N * d * (es + 4 + (c.x0_rows ? es : 0)));
-  ++g_launches; embed_fwd_kernel<act_t, act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+  WITH_NV(d, ++g_launches; embed_fwd_kernel<NV, act_t, act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
       tokens, W("wte"), c.x0_rows ? reinterpret_cast<const act_t*>(m->base + p.hx) : nullptr,
-      m->at<int32_t>(p.rows_x), x, m->at<float>(p.emb_rstd), N, d, V, c.norm_eps, err);
+      m->at<int32_t>(p.rows_x), x, m->at<float>(p.emb_rstd), N, d, V, c.norm_eps, err););
   LAUNCH_CHECK();
   }
   const double norm_bytes = (double)N * d * (4 + es) + 4.0 * N;
@@ -807,10 +872,10 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     act_t* u2 = m->at<act_t>(L.u2);
     {
       ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
-      ++g_launches; rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps);
+      WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps););
       LAUNCH_CHECK();
     }
-    TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a)));
+    TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a), false, "gemm.qkv_fwd"));
     {
       ProfScope ps(pf, st, "rope_qknorm_fwd", 0.0, (double)N * a * es * (4 + (c.v_rows ? 3 : 0)));
       ++g_launches; rope_qknorm_fwd_kernel<act_t, act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
@@ -820,20 +885,20 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       LAUNCH_CHECK();
     }
     TRY(attention_fwd<act_t>(m, qkv, o, m->at<float>(L.lse)));
-    TRY(gemm(g, N, d, a, op_k(o, a), op_k(W(pre + "wo"), a), epi(EPI_ACCUM_F32, x, d, 1)));
+    TRY(gemm(g, N, d, a, op_k(o, a), op_k(W(pre + "wo"), a), epi(EPI_ACCUM_F32, x, d, 1), false, "gemm.o_fwd"));
     {
       ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
-      ++g_launches; rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps);
+      WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps););
       LAUNCH_CHECK();
     }
     TRY(gemm(g, N, F, d, op_k(u2, d), op_k(W(pre + "w1"), d),
-             epi(EPI_RELU2, m->at<act_t>(L.r), F, 0, m->at<act_t>(L.g))));
-    TRY(gemm(g, N, d, F, op_k(m->at<act_t>(L.g), F), op_k(W(pre + "w2"), F), epi(EPI_ACCUM_F32, x, d, 1)));
+             epi(EPI_RELU2, m->at<act_t>(L.g), F), false, "gemm.up_fwd"));
+    TRY(gemm(g, N, d, F, op_k(m->at<act_t>(L.g), F), op_k(W(pre + "w2"), F), epi(EPI_ACCUM_F32, x, d, 1), false, "gemm.down_fwd"));
   }
   act_t* xf = m->at<act_t>(p.xf);
   {
     ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
-    ++g_launches; rmsnorm_fwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps);
+    WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps););
   }
   ++g_launches; ce_prepare_kernel<<<1, 1024, 0, st>>>(targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
   LAUNCH_CHECK();
@@ -845,16 +910,28 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   act_t* dz = m->at<act_t>(p.dz);
   for (int r0 = 0, ci = 0; r0 < N; r0 += p.chunk, ++ci) {
     const int rows = (N - r0 < p.chunk) ? (N - r0) : p.chunk;
-    TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), epi(EPI_STORE_F32, logits, V)));
-    {
+    if (b16) {
+      GemmEpilogue el = epi(EPI_LOGITS, logits, V);
+      el.softcap = c.softcap;
+      el.stats = m->at<float2>(p.ce_stats);
+      TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), el, false, "gemm.lm_fwd"));
+      ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * (4 + es));
+      ++g_launches; ce_stats_kernel<act_t><<<rows, 256, 0, st>>>(logits, m->at<float2>(p.ce_stats), cdiv(V, V >= 256 ? 256 : 128), dz,
+                                                   targets + r0, m->at<float>(p.tok_loss) + r0, V, c.softcap,
+                                                   m->at<float>(p.ce_scale), err);
+      LAUNCH_CHECK();
+    } else {
+      TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), epi(EPI_STORE_F32, logits, V), false,
+               "gemm.lm_fwd"));
       ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * (4 + es));
       ++g_launches; ce_chunk_kernel<act_t><<<rows, 512, 0, st>>>(logits, dz, targets + r0, m->at<float>(p.tok_loss) + r0, V,
                                                    c.softcap, m->at<float>(p.ce_scale), err);
       LAUNCH_CHECK();
     }
-    TRY(gemm(g, rows, d, V, op_k(dz, V), op_mn(Wlm, d), epi(EPI_STORE_F32, m->at<float>(p.dxf) + (long long)r0 * d, d)));
+    TRY(gemm(g, rows, d, V, op_k(dz, V), op_mn(Wlm, d), epi(EPI_STORE_F32, m->at<float>(p.dxf) + (long long)r0 * d, d), false,
+             "gemm.lm_dgrad"));
     TRY(gemm(g, V, d, rows, op_mn(dz, V), op_mn(xf + (long long)r0 * d, d),
-             epi(EPI_ACCUM_F32, m->at<float>(p.pending), d, ci > 0), true));
+             epi(EPI_ACCUM_F32, m->at<float>(p.pending), d, ci > 0), true, "gemm.lm_wgrad"));
   }
   ++g_launches; loss_reduce_kernel<<<1, 1024, 0, st>>>(m->at<float>(p.tok_loss), N, m->at<int>(p.ce_count), loss_dev, err);
   LAUNCH_CHECK();
@@ -899,22 +976,22 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
   act_t* dqkv = m->at<act_t>(p.dqkv);
   act_t* da = m->at<act_t>(p.da);
   act_t* dout = m->at<act_t>(p.dout);
-  { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); ++g_launches; rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(m->at<float>(p.dxf), m->at<act_t>(p.xf),
-                                                        m->at<float>(p.rstd_f), dx, dx_lp, N, d, 0);
+  { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; rmsnorm_bwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(m->at<float>(p.dxf), m->at<act_t>(p.xf),
+                                                        m->at<float>(p.rstd_f), dx, dx_lp, N, d, 0););
   LAUNCH_CHECK(); }
   for (int l = c.n_layer - 1; l >= 0; --l) {
     const LayerActs& L = p.layers[l];
     const std::string pre = "h" + std::to_string(l) + ".";
     // ---- MLP: x += relu(u2 W1^T)^2 W2^T
-    TRY(gemm(g, d, F, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.g), F), epi(EPI_ACCUM_F32, Gp(pre + "w2"), F, beta), true));
-    TRY(gemm(g, N, F, d, op_k(dx_lp, d), op_mn(W(pre + "w2"), F), epi(EPI_DRELU2, da, F, 0, nullptr, m->at<act_t>(L.r))));
-    TRY(gemm(g, F, d, N, op_mn(da, F), op_mn(m->at<act_t>(L.u2), d), epi(EPI_ACCUM_F32, Gp(pre + "w1"), d, beta), true));
-    TRY(gemm(g, N, d, F, op_k(da, F), op_mn(W(pre + "w1"), d), epi(EPI_STORE_F32, du, d)));
-    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); ++g_launches; rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1);
+    TRY(gemm(g, d, F, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.g), F), epi(EPI_ACCUM_F32, Gp(pre + "w2"), F, beta), true, "gemm.down_wgrad"));
+    TRY(gemm(g, N, F, d, op_k(dx_lp, d), op_mn(W(pre + "w2"), F), epi(EPI_DRELU2, da, F, 0, nullptr, m->at<act_t>(L.g)), false, "gemm.down_dgrad"));
+    TRY(gemm(g, F, d, N, op_mn(da, F), op_mn(m->at<act_t>(L.u2), d), epi(EPI_ACCUM_F32, Gp(pre + "w1"), d, beta), true, "gemm.up_wgrad"));
+    TRY(gemm(g, N, d, F, op_k(da, F), op_mn(W(pre + "w1"), d), epi(EPI_STORE_F32, du, d), false, "gemm.up_dgrad"));
+    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; rmsnorm_bwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1););
     LAUNCH_CHECK(); }
     // ---- attention: x += o Wo^T
-    TRY(gemm(g, d, a, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.o), a), epi(EPI_ACCUM_F32, Gp(pre + "wo"), a, beta), true));
-    TRY(gemm(g, N, a, d, op_k(dx_lp, d), op_mn(W(pre + "wo"), a), epi(EPI_STORE, dout, a)));
+    TRY(gemm(g, d, a, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.o), a), epi(EPI_ACCUM_F32, Gp(pre + "wo"), a, beta), true, "gemm.o_wgrad"));
+    TRY(gemm(g, N, a, d, op_k(dx_lp, d), op_mn(W(pre + "wo"), a), epi(EPI_STORE, dout, a), false, "gemm.o_dgrad"));
     TRY(attention_bwd<act_t>(m, m->at<act_t>(L.qkv), m->at<act_t>(L.o), dout, m->at<float>(L.lse),
                              m->at<float>(p.Dattn), dqkv));
     {
@@ -924,9 +1001,9 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
           c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
       LAUNCH_CHECK();
     }
-    TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true));
-    TRY(gemm(g, N, d, 3 * a, op_k(dqkv, 3 * a), op_mn(W(pre + "wqkv"), d), epi(EPI_STORE_F32, du, d)));
-    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); ++g_launches; rmsnorm_bwd_kernel<act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1);
+    TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true, "gemm.qkv_wgrad"));
+    TRY(gemm(g, N, d, 3 * a, op_k(dqkv, 3 * a), op_mn(W(pre + "wqkv"), d), epi(EPI_STORE_F32, du, d), false, "gemm.qkv_dgrad"));
+    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; rmsnorm_bwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1););
     LAUNCH_CHECK(); }
   }
   // dx now holds dL/dx0 per position.
@@ -938,9 +1015,9 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const int32_t* perm;
     TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
     const long long maxp = (long long)N + N / PIECE + 2, maxl = N / PIECE + 2;
-    ++g_launches; emb_piece_kernel<act_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
+    WITH_NV(d, ++g_launches; emb_piece_kernel<NV, act_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
         Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, w.pstart, w.plen, w.pslot,
-        w.counters, w.partial);
+        w.counters, w.partial););
     ++g_launches; emb_long_kernel<<<grid_for(maxl * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, w.seg_start, w.lfirst,
                                                              w.lnslots, w.lseg, w.counters, w.partial);
     LAUNCH_CHECK();
@@ -1185,17 +1262,24 @@ extern "C" int ngram_sync_status(void* stream) {
 
 // ======================================================================== kernel-level test entry
 extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmajor, const void* B,
-                              long long ldb, int b_kmajor, float* C, long long ldc, int beta, int splits,
-                              void* workspace, size_t ws_bytes, void* stream) {
-  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || ldc < N)
+                              long long ldb, int b_kmajor, int mode, void* C, long long ldc, const void* aux,
+                              int beta, int splits, void* workspace, size_t ws_bytes, void* stream) {
+  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || ldc < N || mode < EPI_STORE || mode > EPI_LOGITS)
     return fail(GPT_ERR_ARG, "gptx_gemm_bf16: bad argument");
+  if (mode == EPI_DRELU2 && !aux) return fail(GPT_ERR_ARG, "gptx_gemm_bf16: ReLU^2 backward needs aux");
   if (splits < 1) splits = 1;
+  if (splits > 1 && (mode != EPI_ACCUM_F32 && mode != EPI_STORE_F32))
+    return fail(GPT_ERR_ARG, "gptx_gemm_bf16: split-K only for fp32 outputs");
   if (splits > 1 && (!workspace || ws_bytes < (size_t)splits * M * N * 4))
     return fail(GPT_ERR_WORKSPACE, "gptx_gemm_bf16: split-K needs splits*M*N*4 bytes of workspace");
+  if (mode == EPI_LOGITS && (!workspace || ws_bytes < (size_t)M * cdiv(N, N >= 256 ? 256 : 128) * 8))
+    return fail(GPT_ERR_WORKSPACE, "gptx_gemm_bf16: logits need M*n_tiles*8 bytes of workspace for statistics");
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
-  GemmEpilogue e = epi(EPI_ACCUM_F32, C, ldc, beta);
+  GemmEpilogue e = epi(mode, C, ldc, beta, nullptr, aux);
+  if (mode == EPI_LOGITS) e.stats = (float2*)workspace;
   GemmOperand a{A, lda, a_kmajor ? 1 : 0}, b{B, ldb, b_kmajor ? 1 : 0};
-  if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, (cudaStream_t)stream);
-  return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, (cudaStream_t)stream);
+  GemmCtx g{true, (float*)workspace, (long long)(ws_bytes / 4), err, (cudaStream_t)stream, nullptr};
+  if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
+  return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
 }

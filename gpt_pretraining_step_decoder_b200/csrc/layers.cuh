@@ -8,13 +8,16 @@
 #include "common.cuh"
 
 constexpr int MAXV = 16;  // vec4 chunks per lane: rows up to 32 * 4 * 16 = 2048 wide
+// Row kernels take NV = vec4 chunks per lane as a template parameter so their
+// per-row register arrays are exactly as large as the row (d = 128 * NV when
+// d is a multiple of 128, else NV = MAXV with predication).
 
 // --------------------------------------------------------------------------
 // Token embedding + parameter-free RMSNorm + optional x0 bigram row
 // ("$1000 tier nanochat run", `GPT.forward`: x = norm(wte(idx)); decoder-rtx
 // posts: a 2M-row bigram table "added to x0").
 //   x[t] = wte[tok_t] * rstd_t + Hx[rx_t],   rstd_t = 1/sqrt(mean(wte[tok_t]^2) + eps)
-template <typename w_t, typename tab_t>
+template <int NV, typename w_t, typename tab_t>
 __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __restrict__ wte,
                                  const tab_t* __restrict__ hx, const int32_t* __restrict__ rx,
                                  float* __restrict__ x, float* __restrict__ rstd_out, int N, int d,
@@ -26,10 +29,10 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __r
     if (lane == 0) set_error(err, GPT_EBIT_INPUT);
     id = 0;
   }
-  float v[MAXV][4];
+  float v[NV][4];
   float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       load4(wte + (long long)id * d + c, v[j]);
@@ -41,7 +44,7 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __r
   if (lane == 0) rstd_out[warp] = rstd;
   const long long row = hx ? (long long)rx[warp] : 0;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       float o[4] = {v[j][0] * rstd, v[j][1] * rstd, v[j][2] * rstd, v[j][3] * rstd};
@@ -58,16 +61,16 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __r
 // --------------------------------------------------------------------------
 // RMSNorm forward ("$1000 tier nanochat run", `norm`: F.rms_norm without
 // affine parameters): u = x * rstd, rstd = 1/sqrt(mean(x^2) + eps).
-template <typename act_t>
+template <int NV, typename act_t>
 __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, act_t* __restrict__ u,
                                    float* __restrict__ rstd_out, int N, int d, float eps) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N) return;
   const float* xr = x + (long long)warp * d;
-  float v[MAXV][4];
+  float v[NV][4];
   float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       load4(xr + c, v[j]);
@@ -78,7 +81,7 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, act_t* __restric
   const float rstd = rsqrtf(ss / d + eps);
   if (lane == 0) rstd_out[warp] = rstd;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       float o[4] = {v[j][0] * rstd, v[j][1] * rstd, v[j][2] * rstd, v[j][3] * rstd};
@@ -89,17 +92,17 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, act_t* __restric
 
 // RMSNorm backward: dx (+)= rstd * (du - u * mean(du * u)); also writes the
 // activation-typed copy of dx that the next GEMMs read.
-template <typename act_t>
+template <int NV, typename act_t>
 __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __restrict__ u,
                                    const float* __restrict__ rstd, float* __restrict__ dx,
                                    act_t* __restrict__ dx_lp, int N, int d, int accumulate) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N) return;
   const long long base = (long long)warp * d;
-  float g[MAXV][4], y[MAXV][4];
+  float g[NV][4], y[NV][4];
   float dot = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       load4(du + base + c, g[j]);
@@ -110,7 +113,7 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __
   dot = warp_sum(dot) / d;
   const float r = rstd[warp];
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       float o[4];
@@ -291,6 +294,53 @@ __global__ void __launch_bounds__(512) ce_chunk_kernel(float* __restrict__ logit
     float gi = (expf(zi - lse) - (i == y ? 1.f : 0.f)) * sc;
     if (softcap > 0.f) { const float tt = zi / softcap; gi *= (1.f - tt * tt); }
     g[i] = from_f<act_t>(gi);
+  }
+}
+
+// The same loss and logit gradient for one row of a chunk whose GEMM epilogue
+// already folded each 256-column tile into (max, sum of exp(z - max)):
+// lse = M + log sum_j s_j exp(m_j - M) over the tiles, then one pass over the
+// row writes dz.  One block per row; V a multiple of 4.
+template <typename act_t>
+__global__ void __launch_bounds__(256) ce_stats_kernel(const float* __restrict__ logits,
+                                                       const float2* __restrict__ stats, int n_tiles,
+                                                       act_t* __restrict__ dz,
+                                                       const int32_t* __restrict__ targets,
+                                                       float* __restrict__ tok_loss, int V, float softcap,
+                                                       const float* __restrict__ scale_dev, unsigned* err) {
+  __shared__ float sh[32];
+  const long long row = blockIdx.x;
+  const float* z = logits + row * V;
+  act_t* g = dz + row * V;
+  int y = targets[row];
+  if (y < -1 || y >= V) {
+    if (threadIdx.x == 0) set_error(err, GPT_EBIT_INPUT);
+    y = -1;
+  }
+  const float2* st = stats + row * n_tiles;
+  float mx = -INFINITY;
+  for (int j = threadIdx.x; j < n_tiles; j += blockDim.x) mx = fmaxf(mx, st[j].x);
+  mx = block_max(mx, sh);
+  float se = 0.f;
+  for (int j = threadIdx.x; j < n_tiles; j += blockDim.x) se += st[j].y * __expf(st[j].x - mx);
+  se = block_sum(se, sh);
+  const float lse = mx + logf(se);
+  if (threadIdx.x == 0) {
+    const float l = (y >= 0) ? (lse - z[y]) : 0.f;
+    tok_loss[row] = l;
+    if (y >= 0 && !isfinite(l)) set_error(err, GPT_EBIT_NONFINITE);
+  }
+  const float sc = (y >= 0) ? *scale_dev : 0.f;
+  for (int i = threadIdx.x * 4; i < V; i += blockDim.x * 4) {
+    float v[4], o[4];
+    load4(z + i, v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float gi = (__expf(v[k] - lse) - (i + k == y ? 1.f : 0.f)) * sc;
+      if (softcap > 0.f) { const float tt = v[k] / softcap; gi *= (1.f - tt * tt); }
+      o[k] = gi;
+    }
+    store4(g + i, o);
   }
 }
 

@@ -288,14 +288,14 @@ __global__ void __launch_bounds__(1024) segments_kernel(
 // ---------------------------------------------------------------- row update
 // Apply the per-row-magnitude step to one row with its summed gradient G
 // (held by the warp, 4 values per lane per chunk).
-template <typename tab_t>
+template <int NV, typename tab_t>
 __device__ __forceinline__ void table_row_update(tab_t* __restrict__ table, float* __restrict__ state,
-                                                 long long r, int d, const float (&G)[MAXV][4],
+                                                 long long r, int d, const float (&G)[NV][4],
                                                  float lr, float beta, float eps) {
   const int lane = threadIdx.x & 31;
   float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) ss += G[j][0] * G[j][0] + G[j][1] * G[j][1] + G[j][2] * G[j][2] + G[j][3] * G[j][3];
   }
@@ -303,7 +303,7 @@ __device__ __forceinline__ void table_row_update(tab_t* __restrict__ table, floa
   const float s_new = beta * state[r] + (1.f - beta) * (ss / d);
   const float step = lr / (sqrtf(s_new) + eps);
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       float w[4];
@@ -318,16 +318,17 @@ __device__ __forceinline__ void table_row_update(tab_t* __restrict__ table, floa
 }
 
 // Sum the gradient rows of one piece (in sorted = position order).
+template <int NV>
 __device__ __forceinline__ void piece_sum(const float* __restrict__ grad, const int32_t* __restrict__ perm,
-                                          int st, int len, int d, float (&G)[MAXV][4]) {
+                                          int st, int len, int d, float (&G)[NV][4]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
+  for (int j = 0; j < NV; ++j) G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
   for (int q = 0; q < len; ++q) {
     const long long pos = perm[st + q];
     if (pos < 0) continue;
 #pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c = (j * 32 + lane) * 4;
       if (c < d) {
         float g[4];
@@ -340,7 +341,7 @@ __device__ __forceinline__ void piece_sum(const float* __restrict__ grad, const 
 
 // One warp per piece: whole segments are updated directly; pieces of long
 // segments store their partial sums.
-template <typename tab_t>
+template <int NV, typename tab_t>
 __global__ void table_piece_kernel(tab_t* __restrict__ table, float* __restrict__ state, int d,
                                    const float* __restrict__ grad, const uint32_t* __restrict__ skeys,
                                    const int32_t* __restrict__ perm, const int32_t* __restrict__ pstart,
@@ -350,13 +351,13 @@ __global__ void table_piece_kernel(tab_t* __restrict__ table, float* __restrict_
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= counters[0]) return;
   const int st = pstart[warp], len = plen[warp], slot = pslot[warp];
-  float G[MAXV][4];
-  piece_sum(grad, perm, st, len, d, G);
+  float G[NV][4];
+  piece_sum<NV>(grad, perm, st, len, d, G);
   if (slot < 0) {
-    table_row_update(table, state, (long long)skeys[st], d, G, lr, beta, eps);
+    table_row_update<NV>(table, state, (long long)skeys[st], d, G, lr, beta, eps);
   } else {
 #pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c = (j * 32 + lane) * 4;
       if (c < d) store4(partial + (long long)slot * d + c, G[j]);
     }
@@ -364,7 +365,7 @@ __global__ void table_piece_kernel(tab_t* __restrict__ table, float* __restrict_
 }
 
 // One warp per long segment: add its partial sums in piece order, update.
-template <typename tab_t>
+template <int NV, typename tab_t>
 __global__ void table_long_kernel(tab_t* __restrict__ table, float* __restrict__ state, int d,
                                   const uint32_t* __restrict__ skeys, const int32_t* __restrict__ seg_start,
                                   const int32_t* __restrict__ lseg_first_slot,
@@ -375,12 +376,12 @@ __global__ void table_long_kernel(tab_t* __restrict__ table, float* __restrict__
   if (warp >= counters[1]) return;
   const int first = lseg_first_slot[warp], k = lseg_nslots[warp];
   const long long r = skeys[seg_start[lseg_seg[warp]]];
-  float G[MAXV][4];
+  float G[NV][4];
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
+  for (int j = 0; j < NV; ++j) G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
   for (int q = 0; q < k; ++q) {
 #pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c = (j * 32 + lane) * 4;
       if (c < d) {
         float g[4];
@@ -389,7 +390,7 @@ __global__ void table_long_kernel(tab_t* __restrict__ table, float* __restrict__
       }
     }
   }
-  table_row_update(table, state, r, d, G, lr, beta, eps);
+  table_row_update<NV>(table, state, r, d, G, lr, beta, eps);
 }
 
 // ---------------------------------------------------------------- embedding grad
@@ -397,14 +398,14 @@ __global__ void table_long_kernel(tab_t* __restrict__ table, float* __restrict__
 // (dx0_t - h_t * mean(dx0_t * h_t)) with h_t = wte[tok_t] * rstd_t, summed per
 // token id over its positions (same bucketing as the tables) and added to
 // the fp32 gradient dwte.
-template <typename w_t>
+template <int NV, typename w_t>
 __device__ __forceinline__ void emb_piece_sum(const float* __restrict__ dx0, const w_t* __restrict__ wte,
                                               const float* __restrict__ rstd, const int32_t* __restrict__ perm,
-                                              long long row, int st, int len, int d, float (&G)[MAXV][4]) {
+                                              long long row, int st, int len, int d, float (&G)[NV][4]) {
   const int lane = threadIdx.x & 31;
-  float e[MAXV][4];
+  float e[NV][4];
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
     const int c = (j * 32 + lane) * 4;
     if (c < d) load4(wte + row * d + c, e[j]);
@@ -413,10 +414,10 @@ __device__ __forceinline__ void emb_piece_sum(const float* __restrict__ dx0, con
     const long long pos = perm[st + q];
     if (pos < 0) continue;
     const float r = rstd[pos];
-    float g[MAXV][4];
+    float g[NV][4];
     float dot = 0.f;
 #pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c = (j * 32 + lane) * 4;
       if (c < d) {
         load4(dx0 + pos * d + c, g[j]);
@@ -425,7 +426,7 @@ __device__ __forceinline__ void emb_piece_sum(const float* __restrict__ dx0, con
     }
     dot = warp_sum(dot) * r / d;  // mean(dx0 * h)
 #pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c = (j * 32 + lane) * 4;
       if (c < d)
 #pragma unroll
@@ -434,7 +435,7 @@ __device__ __forceinline__ void emb_piece_sum(const float* __restrict__ dx0, con
   }
 }
 
-template <typename w_t>
+template <int NV, typename w_t>
 __global__ void emb_piece_kernel(float* __restrict__ dwte, const w_t* __restrict__ wte, int d,
                                  const float* __restrict__ dx0, const float* __restrict__ rstd,
                                  const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm,
@@ -445,11 +446,11 @@ __global__ void emb_piece_kernel(float* __restrict__ dwte, const w_t* __restrict
   if (warp >= counters[0]) return;
   const int st = pstart[warp], len = plen[warp], slot = pslot[warp];
   const long long row = skeys[st];
-  float G[MAXV][4];
-  emb_piece_sum(dx0, wte, rstd, perm, row, st, len, d, G);
+  float G[NV][4];
+  emb_piece_sum<NV>(dx0, wte, rstd, perm, row, st, len, d, G);
   float* dst = (slot < 0) ? dwte + row * d : partial + (long long)slot * d;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
+  for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       float o[4];

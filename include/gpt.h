@@ -269,18 +269,24 @@ int ngram_sync_status(void* stream);
 /* ---- kernel-level test entry point ------------------------------------- */
 
 /*
- * C[m, n] (+)= sum_k A[m, k] B[n, k] on the tcgen05 tensor-core GEMM that the
- * step uses for every dense contraction (bf16 operands, fp32 accumulation).
+ * One dense contraction on the tcgen05 tensor-core GEMM that the step uses
+ * for every product: acc[m, n] = sum_k A[m, k] B[n, k], bf16 operands, fp32
+ * accumulation, then the epilogue `mode`:
+ *   0 store      C (bf16) = acc                 3 ReLU^2     C (bf16) = relu(acc)^2
+ *   1 store fp32 C (fp32) = acc                 4 ReLU^2 bwd C (bf16) = 2 sqrt(aux) acc
+ *   2 accumulate C (fp32) = (beta ? C : 0) + acc   (aux: bf16 relu(a)^2, same ld as C)
+ *   5 logits     C (fp32) = acc, and per (row, 256-column tile) the running max
+ *                and sum of exp(acc - max) written as float pairs to `workspace`
+ *                ([M, ceil(N/256)]; 128-column tiles when N < 256)
  * A is read K-major (a_kmajor = 1: element [m, k] at A[m*lda + k]) or M-major
- * (a_kmajor = 0: at A[k*lda + m]); B likewise with N.  C: device fp32 [M, ldc],
- * overwritten (beta = 0) or added to (beta = 1).  splits > 1 splits K and
- * needs workspace of splits*M*N*4 bytes (partials summed in split order).
- * Operands must be 16-byte aligned with lda*2, ldb*2 multiples of 16.
+ * (a_kmajor = 0: at A[k*lda + m]); B likewise with N.  splits > 1 (modes 1 and
+ * 2 only) splits K and needs workspace of splits*M*N*4 bytes, the partials
+ * being summed in split order.  Operands, C and aux must be 16-byte aligned
+ * with row pitches that are multiples of 16 bytes.  Asynchronous on `stream`.
  */
 int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmajor, const void* B,
-                   long long ldb, int b_kmajor, float* C, long long ldc, int beta, int splits,
-                   void* workspace, size_t ws_bytes, void* stream);
-
+                   long long ldb, int b_kmajor, int mode, void* C, long long ldc, const void* aux,
+                   int beta, int splits, void* workspace, size_t ws_bytes, void* stream);
 #ifdef __cplusplus
 }
 #endif

@@ -164,3 +164,46 @@ def test_ngram_sparse_update_matches_oracle(g, dtype, R, n, d):
     mask = torch.ones(R, dtype=torch.bool, device="cuda")
     mask[idx] = False
     assert int((T[mask] != 0).sum()) == 0 and int((S[mask] != 0).sum()) == 0
+
+
+@pytest.mark.parametrize("b_k", [1, 0])
+def test_gemm_epilogue_modes_match_fp64(g, b_k):
+    """Every epilogue of the tensor-core GEMM against its definition on the fp64 product."""
+    import torch
+    M, N, K = 200, 640, 192
+    rng = np.random.default_rng(17 + b_k)
+    A = round_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    B = round_to_bf16(rng.standard_normal((N, K)).astype(np.float32))
+    acc = A.astype(np.float64) @ B.astype(np.float64).T
+    Ad, Bd = _bf16_dev(A), _bf16_dev(B if b_k else B.T)
+    ldb = K if b_k else N
+    aux = round_to_bf16(np.maximum(rng.standard_normal((M, N)), 0).astype(np.float32) ** 2)
+    auxd = _bf16_dev(aux)
+    ws = torch.zeros(M * 3 * 8, dtype=torch.uint8, device="cuda")
+    cases = {
+        g.EPI_STORE: (torch.bfloat16, acc, 4e-3),
+        g.EPI_STORE_F32: (torch.float32, acc, 1e-5),
+        g.EPI_RELU2: (torch.bfloat16, np.maximum(acc, 0) ** 2, 4e-3),
+        g.EPI_DRELU2: (torch.bfloat16, 2 * np.sqrt(aux.astype(np.float64)) * acc, 4e-3),
+        g.EPI_LOGITS: (torch.float32, acc, 1e-5),
+    }
+    for mode, (dt, ref, tol) in cases.items():
+        C = torch.full((M, N), 3.0, dtype=dt, device="cuda")
+        g.gptx_gemm_bf16(M, N, K, Ad, K, 1, Bd, ldb, b_k, C, N, 0, 1, ws, ws.numel(), mode=mode,
+                         aux=auxd if mode == g.EPI_DRELU2 else None)
+        torch.cuda.synchronize()
+        assert g.ngram_sync_status() == g.GPT_OK
+        assert rel_l2(C.float().cpu().numpy(), ref) < tol, mode
+    # logits statistics: per (row, 256-column tile) max and sum of exp(z - max)
+    st = ws[:M * 3 * 8].view(torch.float32).view(M, 3, 2).cpu().numpy().astype(np.float64)
+    for j in range(3):
+        z = acc[:, 256 * j:256 * (j + 1)]
+        mx = z.max(axis=1)
+        np.testing.assert_allclose(st[:, j, 0], mx, rtol=1e-5, atol=1e-4)
+        np.testing.assert_allclose(st[:, j, 1], np.exp(z - mx[:, None]).sum(axis=1), rtol=1e-4)
+    # accumulate with beta = 1 adds into C (TMA reduce-add)
+    C = torch.from_numpy(rng.standard_normal((M, N)).astype(np.float32)).cuda()
+    C0 = C.cpu().numpy().astype(np.float64)
+    g.gptx_gemm_bf16(M, N, K, Ad, K, 1, Bd, ldb, b_k, C, N, 1, 1, None, 0, mode=g.EPI_ACCUM_F32)
+    torch.cuda.synchronize()
+    assert rel_l2(C.cpu().numpy(), C0 + acc) < 1e-5
