@@ -74,6 +74,7 @@ _SIGS = {
     "ngram_sparse_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
     "ngram_sparse_update": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P, _SZ, _P],
     "ngram_sync_status": [_P],
+    "ngram_sparse_update_noalloc": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P],
     "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
 }
 for _name, _args in _SIGS.items():
@@ -242,6 +243,14 @@ def ngram_sparse_update(table, row_state, n_rows, d, dtype, rows, grad, n, lr, b
         _ptr(table), _ptr(row_state), n_rows, d, dtype, _ptr(rows), _ptr(grad), n, lr, beta, eps,
         _ptr(updated_rows_out), _ptr(n_updated_out), _ptr(workspace), ws_bytes, _stream(stream)),
         "ngram_sparse_update")
+
+
+def ngram_sparse_update_noalloc(table, row_state, n_rows, d, dtype, rows, grad, n, lr, beta, eps,
+                                updated_rows_out, n_updated_out, stream=None):
+    """ngram_sparse_update with the library's built-in scratch (no device allocation)."""
+    return _check(_lib.ngram_sparse_update_noalloc(
+        _ptr(table), _ptr(row_state), n_rows, d, dtype, _ptr(rows), _ptr(grad), n, lr, beta, eps,
+        _ptr(updated_rows_out), _ptr(n_updated_out), _stream(stream)), "ngram_sparse_update_noalloc")
 
 
 def ngram_sync_status(stream=None):

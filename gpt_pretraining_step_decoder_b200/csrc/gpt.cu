@@ -1283,3 +1283,40 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
   if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
 }
+
+// ======================================================================== allocation-free table update
+// Scratch for ngram_sparse_update_noalloc: a fixed array in the library's own
+// device image, so the entry point never asks for device memory.  Every GPU
+// that loads the library holds these bytes until the process exits.  All
+// calls share it; each call writes every scratch byte it later reads, so
+// nothing has to start at zero.
+#define GPT_NOALLOC_SCRATCH_BYTES (16u << 20)
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GPT_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device.  In host code the symbol
+// itself is only a host-side stand-in, so the address is looked up with the
+// device current, once, the first time the device is used.
+static std::atomic<void*> g_noalloc_addr[128];
+
+extern "C" int ngram_sparse_update_noalloc(void* table, float* row_state, long long n_rows, int d, int dtype,
+                                           const int32_t* rows, const float* grad, int n, float lr, float beta,
+                                           float eps, int32_t* updated_rows_out, int* n_updated_out_dev,
+                                           void* stream) {
+  if (n < 0 || d < 4) return fail(GPT_ERR_ARG, "ngram_sparse_update_noalloc: bad argument");
+  const size_t need = ngram_ws_plan(n, d).total;
+  if (need > GPT_NOALLOC_SCRATCH_BYTES)
+    return fail(GPT_ERR_WORKSPACE,
+                "ngram_sparse_update_noalloc: n = %d positions of width d = %d need %zu bytes of scratch, "
+                "more than the %u-byte built-in buffer; use ngram_sparse_update with a workspace",
+                n, d, need, (unsigned)GPT_NOALLOC_SCRATCH_BYTES);
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 128) return fail(GPT_ERR_ARG, "ngram_sparse_update_noalloc: device index %d out of range", dev);
+  void* scratch = g_noalloc_addr[dev].load();
+  if (!scratch) {
+    CUDA_TRY(cudaGetSymbolAddress(&scratch, g_noalloc_scratch));
+    g_noalloc_addr[dev].store(scratch);
+  }
+  return ngram_sparse_update(table, row_state, n_rows, d, dtype, rows, grad, n, lr, beta, eps, updated_rows_out,
+                             n_updated_out_dev, scratch, GPT_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -266,6 +266,32 @@ int ngram_sparse_update(void* table, float* row_state, long long n_rows, int d, 
  * error word (GPT_ERR_INPUT for out-of-range ids). */
 int ngram_sync_status(void* stream);
 
+/*
+ * ngram_sparse_update without a caller workspace.  Same arguments, result and
+ * error reporting as ngram_sparse_update, minus `workspace` / `ws_bytes`: the
+ * scratch comes from a 16 MiB buffer compiled into the library, so this call
+ * never allocates device memory (no cudaMalloc, no cudaFree, no allocating
+ * library routine).  It is meant for callers that have no way to hand over
+ * scratch memory: a host runtime that owns every byte of device memory through
+ * its own pool and forbids allocations on the side, a plugin that is given
+ * tensors but no allocator, or a loop that cannot afford cudaMalloc's implicit
+ * synchronisation.  The pages have no counterpart of this entry point.
+ *
+ * Limit: the scratch of ngram_sparse_update_workspace_bytes(n, d) must fit in
+ * 16 MiB (e.g. n <= 32768 positions at d <= 1024, or n <= 65536 at d = 768);
+ * larger calls return GPT_ERR_WORKSPACE before any work is enqueued.
+ * The first call on a device looks up the buffer's device address (with that
+ * device current) and should come before any stream capture.  All calls share
+ * the one buffer: calls whose execution overlaps on the GPU (different
+ * streams, or the same buffer used from two host threads' streams) race on it
+ * and must be ordered by the caller.  Every GPU that loads the library keeps
+ * the 16 MiB until the process exits.
+ */
+int ngram_sparse_update_noalloc(void* table, float* row_state, long long n_rows, int d, int dtype,
+                                const int32_t* rows, const float* grad, int n, float lr, float beta,
+                                float eps, int32_t* updated_rows_out, int* n_updated_out_dev,
+                                void* stream);
+
 /* ---- kernel-level test entry point ------------------------------------- */
 
 /*
