@@ -113,6 +113,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
   }
 }
+// The same wait made warp-uniform: every lane waits, and the warp proceeds only
+// if all lanes succeeded.  Used wherever the warp next executes .sync.aligned
+// tcgen05 instructions, which must never be reached by a partial warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned* err) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, err);
+  return __all_sync(0xffffffffu, ok);
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y) {
   asm volatile(
@@ -380,7 +388,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           aux_pending |= 1u << b;
         }
       }
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err)) { ok = false; break; }
+      if (!warp_wait(&tfull[acc], acc_phase, abort_flag, p.err)) { ok = false; break; }
       tc_fence_after();
       float rmax = -INFINITY, rsum = 0.f;
       const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
@@ -422,7 +430,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 64; ++i) { const float r = fmaxf(v[i], 0.f); v[i] = r * r; }
         } else if constexpr (KM == K_DRELU2) {
           const int b = c % C::NAUX;
-          if (!mbar_wait(&abar[b], (aux_phase >> b) & 1u, abort_flag, p.err)) { ok = false; break; }
+          if (!warp_wait(&abar[b], (aux_phase >> b) & 1u, abort_flag, p.err)) { ok = false; break; }
           aux_phase ^= 1u << b;
           aux_pending &= ~(1u << b);
           const uint8_t* ab = auxs + b * AUX_BYTES;

@@ -24,6 +24,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "attention_fa.cuh"
+#include "attention_tc.cuh"
 #include "layers.cuh"
 #include "ngram.cuh"
 #include "optim.cuh"
@@ -774,12 +775,17 @@ static int attention_fwd(gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
   if (std::is_same<act_t, bf16>::value) {
     static bool attr = false;
     if (!attr) {
-      CUDA_TRY(cudaFuncSetAttribute(fa::fa_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::F_SMEM));
+      CUDA_TRY(cudaFuncSetAttribute(fatc::fa_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fatc::SMEM_BYTES));
       attr = true;
     }
-    dim3 g(cdiv(c.seq_len, fa::F_BQ), c.micro_batch * c.n_head);
-    ++g_launches; fa::fa_fwd_kernel<<<g, fa::F_THREADS, fa::F_SMEM, m->st>>>(
-        reinterpret_cast<const bf16*>(qkv), reinterpret_cast<bf16*>(o), lse, c.seq_len, c.n_head);
+    const long long a = (long long)c.n_head * c.head_dim, ntok = (long long)c.micro_batch * c.seq_len;
+    CUtensorMap tqk, tv;
+    TRY(make_tmap(&tqk, qkv, 3 * a, ntok, 3 * a, 64, 128));
+    TRY(make_tmap(&tv, qkv, 3 * a, ntok, 3 * a, 64, 64));
+    dim3 g(cdiv(c.seq_len, fatc::BQ), c.micro_batch * c.n_head);
+    ++g_launches; fatc::fa_tc_fwd_kernel<<<g, fatc::THREADS, fatc::SMEM_BYTES, m->st>>>(
+        tqk, tv, reinterpret_cast<bf16*>(o), lse, c.seq_len, c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
   }
