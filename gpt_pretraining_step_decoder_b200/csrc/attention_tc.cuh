@@ -332,3 +332,454 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 }  // namespace fatc
+
+// ============================================================================
+// Backward on tcgen05 (same operation as fa::fa_bwd_dkdv_kernel /
+// fa::fa_bwd_dq_kernel): with P = exp(s/sqrt(hd) - lse) recomputed from the
+// forward's log-sum-exp and D_q = rowsum(dO_q * O_q),
+//   dV = P^T dO,  dS = P (dP - D) with dP = dO V^T,  dK = dS^T Q / sqrt(hd),
+//   dQ = dS K / sqrt(hd).
+// Two kernels so every output element has one writer (no atomics): one CTA
+// per 128-key tile computes dK, dV over the query tiles (64 queries) from the
+// diagonal on; one CTA per 128-query tile computes dQ over the key tiles (64
+// keys) up to the diagonal.
+//
+// A K-major 128-byte-swizzled tile [rows x 128 hd] (two 64-column halves) is
+// also, byte for byte, the MN-major layout of the same matrix read as
+// [N = hd, K = rows]: the halves are the two 64-wide N chunks (LBO = half
+// size) and 8-row groups are 1 KB apart.  So Q, K and dO are loaded once and
+// read through both descriptors.
+namespace fatcb {
+
+using fatc::LOG2E;
+constexpr int THREADS = 192;
+
+// K-major [rows x 128] tile, MMA k-step k over the 128 columns
+__device__ __forceinline__ uint64_t kdesc128(uint32_t base, int half_bytes, int k) {
+  return tc::smem_desc(base + (k >> 2) * half_bytes + (k & 3) * 32, 16, 1024);
+}
+// K-major [rows x 64] tile (one swizzle atom wide), k-step k over the 64 columns
+__device__ __forceinline__ uint64_t kdesc64(uint32_t base, int k) {
+  return tc::smem_desc(base + k * 32, 16, 1024);
+}
+// the same [rows x 128] tile read MN-major as [N = 128 (two halves), K = rows]
+__device__ __forceinline__ uint64_t mndesc(uint32_t base, int half_bytes, int k) {
+  return tc::smem_desc(base + k * 2048, half_bytes, 1024);
+}
+__device__ __forceinline__ uint32_t idesc(int n, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r0[32], r1[32];
+  tc::tmem_ld32_nowait(taddr, r0);
+  tc::tmem_ld32_nowait(taddr + 32, r1);
+  tc::tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) { v[i] = __uint_as_float(r0[i]); v[32 + i] = __uint_as_float(r1[i]); }
+}
+// one row of 64 bf16 (128 bytes) into a K-major swizzled [rows x 64] tile
+__device__ __forceinline__ void st_row64(uint8_t* tile, int r, const float (&v)[64]) {
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    uint4 w;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * jj], v[8 * jj + 1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * jj + 2], v[8 * jj + 3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * jj + 4], v[8 * jj + 5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * jj + 6], v[8 * jj + 7]);
+    w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
+    w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((jj ^ (r & 7)) << 4)) = w;
+  }
+}
+// one 128-column fp32 TMEM row, scaled, as bf16 to global (256 bytes)
+__device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t o[32];
+    tc::tmem_ld32_nowait(taddr + cc * 32, o);
+    tc::tmem_wait_ld();
+    if (valid) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        uint4 w;
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * scale, __uint_as_float(o[i + 1]) * scale);
+        __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * scale, __uint_as_float(o[i + 3]) * scale);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * scale, __uint_as_float(o[i + 5]) * scale);
+        __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * scale, __uint_as_float(o[i + 7]) * scale);
+        w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
+        w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
+        *reinterpret_cast<uint4*>(dst + cc * 32 + i) = w;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+// smem: K, V [128 x 128] (32 KB each); per stage Q_i, dO_i [64 x 128] (16 KB
+// each); per buffer P^T, dS^T [128 keys x 64 queries] (16 KB each).
+constexpr int KV_T = 32768, QT64 = 16384, PT = 16384;
+constexpr int DKDV_SMEM = 2 * KV_T + 2 * 2 * QT64 + 2 * 2 * PT + 1024 + 256;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    fa_tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
+                          const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
+                          const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+  using namespace tc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + KV_T;
+  uint8_t* sQ = sV + KV_T;           // [2 stages]
+  uint8_t* sO = sQ + 2 * QT64;       // dO [2 stages]
+  uint8_t* sP = sO + 2 * QT64;       // P^T [2]
+  uint8_t* sS = sP + 2 * PT;         // dS^T [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + 2 * PT);
+  uint64_t* kv_full = bars;          // 1
+  uint64_t* q_full = bars + 1;       // 2
+  uint64_t* q_empty = bars + 3;      // 2
+  uint64_t* s_full = bars + 5;       // 2
+  uint64_t* s_empty = bars + 7;      // 2
+  uint64_t* p_full = bars + 9;       // 2
+  uint64_t* p_free = bars + 11;      // 2
+  uint64_t* o_full = bars + 13;      // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x;  // key tiles near the start have the most query tiles: launched first
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int a = H * 128;
+  const int k0 = kt * 128;
+  const int row_base = b * T;
+  const int qi0 = k0 / 64, nq = (T + 63) / 64;
+  const int n_it = nq - qi0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 128);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&p_free[s], 1);
+    }
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // S^T: 0, 64; dP^T: 128, 192; dV: 256; dK: 384
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA
+      bool ok = true;
+      mbar_expect_tx(kv_full, 2 * KV_T);
+      tma_load_2d(sK, &tm128, kv_full, a + h * 128, row_base + k0);
+      tma_load_2d(sK + KV_T / 2, &tm128, kv_full, a + h * 128 + 64, row_base + k0);
+      tma_load_2d(sV, &tm128, kv_full, 2 * a + h * 128, row_base + k0);
+      tma_load_2d(sV + KV_T / 2, &tm128, kv_full, 2 * a + h * 128 + 64, row_base + k0);
+      int issued = 0;
+      for (int i = 0; i < n_it && ok; ++i) {
+        const int s = i & 1;
+        if (!mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+        mbar_expect_tx(&q_full[s], 2 * QT64);
+        const int qr = row_base + (qi0 + i) * 64;
+        uint8_t* q = sQ + s * QT64;
+        uint8_t* o = sO + s * QT64;
+        tma_load_2d(q, &tm64, &q_full[s], h * 128, qr);
+        tma_load_2d(q + QT64 / 2, &tm64, &q_full[s], h * 128 + 64, qr);
+        tma_load_2d(o, &tmDO, &q_full[s], h * 128, qr);
+        tma_load_2d(o + QT64 / 2, &tmDO, &q_full[s], h * 128 + 64, qr);
+        ++issued;
+      }
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(kv_full, 0)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
+      for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) {
+        const uint64_t t1 = globaltimer_ns();
+        while (!mbar_try_wait(&q_full[i & 1], (i >> 1) & 1)) if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA
+      const uint32_t id_s = idesc(64, false);   // S^T = K Q^T, dP^T = V dO^T (N = 64 queries)
+      const uint32_t id_g = idesc(128, true);   // dV += P^T dO, dK += dS^T Q (N = 128, B MN-major)
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+      bool ok = mbar_wait(kv_full, 0, abort_flag, err);
+      for (int i = 0; i <= n_it && ok; ++i) {
+        if (i < n_it) {
+          const int s = i & 1;
+          if (!mbar_wait(&q_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[s], ((i >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t aQ = smem_u32(sQ + s * QT64), aO = smem_u32(sO + s * QT64);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc_mma(tmem + s * 64, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc_mma(tmem + 128 + s * 64, kdesc128(aV, KV_T / 2, k), kdesc128(aO, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+          tc_commit(&s_full[s]);
+        }
+        if (i >= 1) {
+          const int ip = i - 1, s = ip & 1;
+          if (!mbar_wait(&p_full[s], (ip >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t aP = smem_u32(sP + s * PT), aS = smem_u32(sS + s * PT);
+          const uint32_t aQ = smem_u32(sQ + s * QT64), aO = smem_u32(sO + s * QT64);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma(tmem + 256, kdesc64(aP, k), mndesc(aO, QT64 / 2, k), id_g, (ip > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma(tmem + 384, kdesc64(aS, k), mndesc(aQ, QT64 / 2, k), id_g, (ip > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&p_free[s]);
+          tc_commit(&q_empty[s]);
+          if (ip == n_it - 1) tc_commit(o_full);
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- P^T, dS^T
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float c = rsqrtf(128.f) * LOG2E;
+    const float* lse_bh = lse + (long long)bh * T;
+    const float* D_bh = Dv + (long long)bh * T;
+    bool ok = true;
+    for (int i = 0; i < n_it; ++i) {
+      const int s = i & 1;
+      const int qbase = (qi0 + i) * 64;
+      if (!warp_wait(&s_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      float sv[64], dp[64];
+      ld64(tmem + lane_off + s * 64, sv);
+      ld64(tmem + lane_off + 128 + s * 64, dp);
+      tc_fence_before();
+      mbar_arrive(&s_empty[s]);
+      // P^T[key, q] = exp2(s c - lse_q log2e) for key <= q < T; dS^T = P^T (dP^T - D_q)
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const int qq = qbase + e;
+        const bool live = (key <= qq) && (qq < T);
+        const float L = live ? lse_bh[qq] * LOG2E : 0.f;
+        const float Dq = live ? D_bh[qq] : 0.f;
+        const float p = live ? exp2f(fmaf(sv[e], c, -L)) : 0.f;
+        sv[e] = p;
+        dp[e] = p * (dp[e] - Dq);
+      }
+      if (i >= 2 && !warp_wait(&p_free[s], ((i - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      st_row64(sP + s * PT, r, sv);
+      st_row64(sS + s * PT, r, dp);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(&p_full[s]);
+    }
+    if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
+      tc_fence_after();
+      const bool valid = key < T;
+      bf16* krow = dqkv + ((long long)row_base + (valid ? key : 0)) * 3 * a + a + h * 128;
+      row128_out(tmem + lane_off + 256, 1.f, krow + a, valid);             // dV
+      row128_out(tmem + lane_off + 384, rsqrtf(128.f), krow, valid);       // dK
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+// smem: Q, dO [128 x 128] (32 KB each); per stage K_j, V_j [64 x 128] (16 KB
+// each, 3 stages); per buffer dS [128 queries x 64 keys] (16 KB, 2 buffers).
+constexpr int DQ_STAGES = 3;
+constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 2 * PT + 1024 + 256;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    fa_tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
+                        const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
+                        const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+  using namespace tc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sO = sQ + KV_T;
+  uint8_t* sK = sO + KV_T;                   // [stages]
+  uint8_t* sV = sK + DQ_STAGES * QT64;       // [stages]
+  uint8_t* sS = sV + DQ_STAGES * QT64;       // dS [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + 2 * PT);
+  uint64_t* q_full = bars;                   // 1
+  uint64_t* kv_full = bars + 1;              // 3
+  uint64_t* kv_empty = bars + 4;             // 3
+  uint64_t* s_full = bars + 7;               // 2
+  uint64_t* s_empty = bars + 9;              // 2
+  uint64_t* p_full = bars + 11;              // 2
+  uint64_t* p_free = bars + 13;              // 2
+  uint64_t* o_full = bars + 15;              // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = gridDim.x - 1 - blockIdx.x;  // latest query tiles (most key tiles) first
+  const int bh = blockIdx.y, b = bh / H, h = bh % H;
+  const int a = H * 128;
+  const int q0 = qt * 128;
+  const int row_base = b * T;
+  const int n_it = min((q0 + 128) / 64, (T + 63) / 64);  // key tiles of 64 up to the diagonal
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 128);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&p_free[s], 1);
+    }
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // S: 0, 64; dP: 128, 192; dQ: 256
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA
+      bool ok = true;
+      mbar_expect_tx(q_full, 2 * KV_T);
+      tma_load_2d(sQ, &tm128, q_full, h * 128, row_base + q0);
+      tma_load_2d(sQ + KV_T / 2, &tm128, q_full, h * 128 + 64, row_base + q0);
+      // dO [128 x 128] through the 64-row map: half hf (64 columns) x row block rb
+      for (int hf = 0; hf < 2; ++hf)
+        for (int rb = 0; rb < 2; ++rb)
+          tma_load_2d(sO + hf * (KV_T / 2) + rb * 8192, &tmDO, q_full, h * 128 + 64 * hf, row_base + q0 + 64 * rb);
+      int issued = 0;
+      for (int j = 0; j < n_it && ok; ++j) {
+        const int s = j % DQ_STAGES;
+        if (!mbar_wait(&kv_empty[s], ((j / DQ_STAGES) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+        mbar_expect_tx(&kv_full[s], 2 * QT64);
+        const int kr = row_base + j * 64;
+        uint8_t* k = sK + s * QT64;
+        uint8_t* v = sV + s * QT64;
+        tma_load_2d(k, &tm64, &kv_full[s], a + h * 128, kr);
+        tma_load_2d(k + QT64 / 2, &tm64, &kv_full[s], a + h * 128 + 64, kr);
+        tma_load_2d(v, &tm64, &kv_full[s], 2 * a + h * 128, kr);
+        tma_load_2d(v + QT64 / 2, &tm64, &kv_full[s], 2 * a + h * 128 + 64, kr);
+        ++issued;
+      }
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(q_full, 0)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
+      for (int j = (issued > DQ_STAGES ? issued - DQ_STAGES : 0); j < issued; ++j) {
+        const uint64_t t1 = globaltimer_ns();
+        while (!mbar_try_wait(&kv_full[j % DQ_STAGES], (j / DQ_STAGES) & 1))
+          if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA
+      const uint32_t id_s = idesc(64, false);   // S = Q K^T, dP = dO V^T (N = 64 keys)
+      const uint32_t id_g = idesc(128, true);   // dQ += dS K (N = 128, B MN-major)
+      const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
+      bool ok = mbar_wait(q_full, 0, abort_flag, err);
+      for (int j = 0; j <= n_it && ok; ++j) {
+        if (j < n_it) {
+          const int st = j % DQ_STAGES, s = j & 1;
+          if (!mbar_wait(&kv_full[st], (j / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc_mma(tmem + s * 64, kdesc128(aQ, KV_T / 2, k), kdesc128(aK, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc_mma(tmem + 128 + s * 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+          tc_commit(&s_full[s]);
+        }
+        if (j >= 1) {
+          const int jp = j - 1, s = jp & 1, st = jp % DQ_STAGES;
+          if (!mbar_wait(&p_full[s], (jp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t aS = smem_u32(sS + s * PT), aK = smem_u32(sK + st * QT64);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma(tmem + 256, kdesc64(aS, k), mndesc(aK, QT64 / 2, k), id_g, (jp > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&p_free[s]);
+          tc_commit(&kv_empty[st]);
+          if (jp == n_it - 1) tc_commit(o_full);
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- dS
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int qpos = q0 + r;
+    const bool valid = qpos < T;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float c = rsqrtf(128.f) * LOG2E;
+    const float L = valid ? lse[(long long)bh * T + qpos] * LOG2E : 0.f;
+    const float Dq = valid ? Dv[(long long)bh * T + qpos] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_it; ++j) {
+      const int s = j & 1;
+      if (!warp_wait(&s_full[s], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      float sv[64], dp[64];
+      ld64(tmem + lane_off + s * 64, sv);
+      ld64(tmem + lane_off + 128 + s * 64, dp);
+      tc_fence_before();
+      mbar_arrive(&s_empty[s]);
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const int kk = j * 64 + e;
+        const bool live = valid && (kk <= qpos);
+        const float p = live ? exp2f(fmaf(sv[e], c, -L)) : 0.f;
+        dp[e] = p * (dp[e] - Dq);
+      }
+      if (j >= 2 && !warp_wait(&p_free[s], ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      st_row64(sS + s * PT, r, dp);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(&p_full[s]);
+    }
+    if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
+      tc_fence_after();
+      bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128;
+      row128_out(tmem + lane_off + 256, rsqrtf(128.f), qrow, valid);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+}  // namespace fatcb

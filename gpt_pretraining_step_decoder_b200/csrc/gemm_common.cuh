@@ -23,6 +23,9 @@ enum EpiMode {
                       // d relu(a)^2 / da = 2 relu(a) = 2 sqrt(relu(a)^2))
   EPI_LOGITS = 5,     // z = softcap(acc): C(f32) = z, and per (row, column tile) the
                       // running max and sum of exp(z - max) into stats (tensor-core path)
+  EPI_QKV = 6,        // fused q|k|v projection output (tensor-core path, 128-wide heads):
+                      // q, k heads rotated (RoPE) and RMS-normalised per head, v heads plus
+                      // the value-table row; C(act) = result
 };
 
 struct GemmEpilogue {
@@ -35,6 +38,15 @@ struct GemmEpilogue {
   int beta;
   float softcap;    // EPI_LOGITS: 0 = off, else z = softcap * tanh(acc / softcap)
   float2* stats;    // EPI_LOGITS: [M, n_tiles] (max, sum of exp(z - max))
+  // EPI_QKV: rope table [T, 64, (cos, sin)], per-(row, head) rstd outputs,
+  // optional value table [rows, H*128] (bf16) and its row per position
+  const float* rope;
+  float* rstd_q;
+  float* rstd_k;
+  const void* hv;
+  const int32_t* rv;
+  int T, H, qk_norm;
+  float eps;
 };
 
 template <typename act_t>

@@ -42,6 +42,7 @@ enum KMode {
   K_RELU2,        // bf16 relu(acc)^2
   K_DRELU2,       // bf16 2 sqrt(aux) acc
   K_LOGITS,       // fp32 softcap(acc) + per-tile row statistics
+  K_QKV,          // bf16 q|k|v with RoPE + QK-norm (+ value-table row) per 128-wide head
 };
 
 // HEAVY = 1: the epilogue-heavy variant (logits, ReLU^2 backward) trades one
@@ -392,8 +393,96 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       float rmax = -INFINITY, rsum = 0.f;
       const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if constexpr (KM == K_QKV) {
+        // one 128-wide head per iteration; this lane owns row m of it
+        const bool row_ok = m < p.M;
+        const int tpos = row_ok ? (int)(m % e.T) : 0;
 #pragma unroll 1
-      for (int c = 0; c < nblk; ++c) {
+        for (int hh = 0; hh < BN / 128; ++hh) {
+          const int nc = n0 + hh * 128;
+          if (nc >= p.N) break;  // warp-uniform
+          const int head = nc / 128, sec = head / e.H, hi = head % e.H;
+          float v[128];
+          {
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld32_nowait(trow + hh * 128, r0);
+            tmem_ld32_nowait(trow + hh * 128 + 32, r1);
+            tmem_ld32_nowait(trow + hh * 128 + 64, r2);
+            tmem_ld32_nowait(trow + hh * 128 + 96, r3);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              v[i] = __uint_as_float(r0[i]);
+              v[32 + i] = __uint_as_float(r1[i]);
+              v[64 + i] = __uint_as_float(r2[i]);
+              v[96 + i] = __uint_as_float(r3[i]);
+            }
+          }
+          if (sec < 2) {
+            // RoPE ("$1000 tier nanochat run", apply_rotary_emb): y1 = x1 cos + x2 sin,
+            // y2 = -x1 sin + x2 cos over the two halves of the head, then QK-norm
+            const float2* cs = reinterpret_cast<const float2*>(e.rope) + (long long)tpos * 64;
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              const float2 w = cs[i];
+              const float x1 = v[i], x2 = v[i + 64];
+              v[i] = x1 * w.x + x2 * w.y;
+              v[i + 64] = -x1 * w.y + x2 * w.x;
+              ss += v[i] * v[i] + v[i + 64] * v[i + 64];
+            }
+            if (e.qk_norm) {
+              const float rs = rsqrtf(ss / 128.f + e.eps);
+#pragma unroll
+              for (int i = 0; i < 128; ++i) v[i] *= rs;
+              if (row_ok) (sec == 0 ? e.rstd_q : e.rstd_k)[m * e.H + hi] = rs;
+            }
+          } else if (e.hv && row_ok) {
+            // the value-table row of this position (decoder-rtx posts: table "added to values")
+            const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const act_t*>(e.hv) +
+                                                              (long long)e.rv[m] * (e.H * 128) + hi * 128);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const uint4 raw = src[j];
+              const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+              for (int hq = 0; hq < 4; ++hq) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[hq]));
+                v[j * 8 + 2 * hq] += f.x;
+                v[j * 8 + 2 * hq + 1] += f.y;
+              }
+            }
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint8_t* stg = stg_base + sbuf * STG_BYTES;
+            if (lane == 0) {
+              if (C::NSTG == 2) bulk_wait_read1();
+              else bulk_wait_read0();
+            }
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float* x = &v[half * 64 + 8 * j];
+              uint4 o;
+              __nv_bfloat162 b0 = __floats2bfloat162_rn(x[0], x[1]), b1 = __floats2bfloat162_rn(x[2], x[3]);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(x[4], x[5]), b3 = __floats2bfloat162_rn(x[6], x[7]);
+              o.x = *reinterpret_cast<uint32_t*>(&b0); o.y = *reinterpret_cast<uint32_t*>(&b1);
+              o.z = *reinterpret_cast<uint32_t*>(&b2); o.w = *reinterpret_cast<uint32_t*>(&b3);
+              *reinterpret_cast<uint4*>(stg + swz128(lane, j)) = o;
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmC, stg, nc + half * 64, mrow0);
+              bulk_commit();
+            }
+            sbuf = (sbuf + 1) % C::NSTG;
+          }
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < (KM == K_QKV ? 0 : nblk); ++c) {
         const int nc = n0 + c * CW;
         float v[64];
         {

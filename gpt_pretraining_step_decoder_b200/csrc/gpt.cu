@@ -192,6 +192,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   else if (e.mode == EPI_ACCUM_F32) km = tc::K_REDUCE_F32;
   else if (e.mode == EPI_RELU2) km = tc::K_RELU2;
   else if (e.mode == EPI_DRELU2) km = tc::K_DRELU2;
+  else if (e.mode == EPI_QKV) km = tc::K_QKV;
   else km = tc::K_LOGITS;
   switch (km) {
     case tc::K_STORE: TRY((gemm_tc_launch_k<BN, tc::K_STORE>(ta, tb, tcm, taux, p, st))); break;
@@ -200,6 +201,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
     case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_RELU2: TRY((gemm_tc_launch_k<BN, tc::K_RELU2>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_DRELU2: TRY((gemm_tc_launch_k<BN, tc::K_DRELU2>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_QKV: TRY((gemm_tc_launch_k<BN, tc::K_QKV>(ta, tb, tcm, taux, p, st))); break;
     default: TRY((gemm_tc_launch_k<BN, tc::K_LOGITS>(ta, tb, tcm, taux, p, st))); break;
   }
   if (p.splits > 1) {
@@ -303,6 +305,8 @@ static GemmEpilogue epi(int mode, void* C, long long ldc, int beta = 0, void* C2
   GemmEpilogue e;
   e.mode = mode; e.C = C; e.ldc = ldc; e.C2 = C2; e.aux = aux; e.alpha = alpha; e.beta = beta;
   e.softcap = 0.f; e.stats = nullptr;
+  e.rope = nullptr; e.rstd_q = e.rstd_k = nullptr; e.hv = nullptr; e.rv = nullptr;
+  e.T = e.H = e.qk_norm = 0; e.eps = 0.f;
   return e;
 }
 
@@ -800,26 +804,33 @@ template <typename act_t>
 static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const act_t* dout,
                          const float* lse, float* Dv, act_t* dqkv) {
   const gpt_config& c = m->cfg;
+  const long long N = (long long)c.micro_batch * c.seq_len;
   ProfScope ps(&m->prof, m->st, "attention_bwd",
                5.0 * c.micro_batch * c.n_head * (double)c.seq_len * c.seq_len * c.head_dim, 0.0);
-  const long long N = (long long)c.micro_batch * c.seq_len;
   ++g_launches; attn_bwd_pre_kernel<act_t><<<grid_for(N * c.n_head * 32, 256), 256, 0, m->st>>>(
       o, dout, Dv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
   LAUNCH_CHECK();
   if (std::is_same<act_t, bf16>::value) {
     static bool attr = false;
     if (!attr) {
-      CUDA_TRY(cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::B_SMEM));
-      CUDA_TRY(cudaFuncSetAttribute(fa::fa_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::Q_SMEM));
+      CUDA_TRY(cudaFuncSetAttribute(fatcb::fa_tc_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fatcb::DKDV_SMEM));
+      CUDA_TRY(cudaFuncSetAttribute(fatcb::fa_tc_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fatcb::DQ_SMEM));
       attr = true;
     }
-    dim3 gk(cdiv(c.seq_len, fa::B_BK), c.micro_batch * c.n_head);
-    dim3 gq(cdiv(c.seq_len, fa::B_BQ), c.micro_batch * c.n_head);
-    const bf16* q16 = reinterpret_cast<const bf16*>(qkv);
-    const bf16* d16 = reinterpret_cast<const bf16*>(dout);
+    const long long a = (long long)c.n_head * c.head_dim;
+    CUtensorMap t128, t64, tdo;
+    TRY(make_tmap(&t128, qkv, 3 * a, N, 3 * a, 64, 128));
+    TRY(make_tmap(&t64, qkv, 3 * a, N, 3 * a, 64, 64));
+    TRY(make_tmap(&tdo, dout, a, N, a, 64, 64));
+    dim3 gk(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
+    dim3 gq(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
     bf16* g16 = reinterpret_cast<bf16*>(dqkv);
-    ++g_launches; fa::fa_bwd_dkdv_kernel<<<gk, fa::B_THREADS, fa::B_SMEM, m->st>>>(q16, d16, lse, Dv, g16, c.seq_len, c.n_head);
-    ++g_launches; fa::fa_bwd_dq_kernel<<<gq, fa::B_THREADS, fa::Q_SMEM, m->st>>>(q16, d16, lse, Dv, g16, c.seq_len, c.n_head);
+    ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<gk, fatcb::THREADS, fatcb::DKDV_SMEM, m->st>>>(
+        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
+    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<gq, fatcb::THREADS, fatcb::DQ_SMEM, m->st>>>(
+        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
   }
@@ -881,8 +892,18 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps););
       LAUNCH_CHECK();
     }
-    TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a), false, "gemm.qkv_fwd"));
-    {
+    if (b16) {
+      // QKV projection with RoPE + QK-norm (+ value-table row) in its epilogue
+      GemmEpilogue eq = epi(EPI_QKV, qkv, 3 * a);
+      eq.rope = m->at<float>(p.rope_cs);
+      eq.rstd_q = m->at<float>(L.rstd_q);
+      eq.rstd_k = m->at<float>(L.rstd_k);
+      eq.hv = c.v_rows ? (const void*)(m->base + p.hv) : nullptr;
+      eq.rv = m->at<int32_t>(p.rows_v);
+      eq.T = c.seq_len; eq.H = H; eq.qk_norm = c.qk_norm; eq.eps = c.norm_eps;
+      TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), eq, false, "gemm.qkv_fwd"));
+    } else {
+      TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a), false, "gemm.qkv_fwd"));
       ProfScope ps(pf, st, "rope_qknorm_fwd", 0.0, (double)N * a * es * (4 + (c.v_rows ? 3 : 0)));
       ++g_launches; rope_qknorm_fwd_kernel<act_t, act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
           qkv, m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
