@@ -97,8 +97,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 128);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&s_empty[s], 4);   // one arrival per softmax warp
+      mbar_init(&p_full[s], 4);
       mbar_init(&p_free[s], 1);
     }
     mbar_init(o_full, 1);
@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&s_empty[s]);  // the S buffer may be overwritten
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[s]);  // the S buffer may be overwritten
       const int k0 = j * BKV;
       if (k0 + BKV - 1 > qpos) {  // causal mask on the diagonal tile
 #pragma unroll
@@ -293,7 +294,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(&p_full[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
     }
     // ---------------------------------------------------------------- epilogue
     if (__all_sync(0xffffffffu, ok) && warp_wait(o_full, 0, abort_flag, err)) {
@@ -416,15 +418,67 @@ __device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* ds
 }
 
 // ---------------------------------------------------------------- dK, dV
+// 10 warps: 0 TMA, 1 MMA, 2..9 compute.  Compute warp w owns TMEM lane
+// quarter w % 4 (32 key rows) and half (w - 2) / 4 of the 64 query columns,
+// so two warps per scheduler share the elementwise work.
 // smem: K, V [128 x 128] (32 KB each); per stage Q_i, dO_i [64 x 128] (16 KB
-// each); per buffer P^T, dS^T [128 keys x 64 queries] (16 KB each).
+// each) and lse_i, D_i (64 floats each, by TMA); per buffer P^T, dS^T
+// [128 keys x 64 queries] (16 KB each).
+constexpr int THREADS_B = 320;
 constexpr int KV_T = 32768, QT64 = 16384, PT = 16384;
-constexpr int DKDV_SMEM = 2 * KV_T + 2 * 2 * QT64 + 2 * 2 * PT + 1024 + 256;
+constexpr int DKDV_SMEM = 2 * KV_T + 2 * 2 * QT64 + 2 * 2 * PT + 2 * 512 + 1024 + 256;
 
-__global__ void __launch_bounds__(THREADS, 1)
+__device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tc::tmem_ld32_nowait(taddr, r);
+  tc::tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 32 bf16 (64 bytes: chunks 4*half .. 4*half+3) of row r of a K-major
+// swizzled [rows x 64] tile
+__device__ __forceinline__ void st_half_row(uint8_t* tile, int r, int half, const float (&v)[32]) {
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    uint4 w;
+    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * jj], v[8 * jj + 1]);
+    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * jj + 2], v[8 * jj + 3]);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * jj + 4], v[8 * jj + 5]);
+    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * jj + 6], v[8 * jj + 7]);
+    w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
+    w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
+    const int j = half * 4 + jj;
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = w;
+  }
+}
+// 64 fp32 TMEM columns of a row, scaled, as bf16 to global (128 bytes)
+__device__ __forceinline__ void row64_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    uint32_t o[32];
+    tc::tmem_ld32_nowait(taddr + cc * 32, o);
+    tc::tmem_wait_ld();
+    if (valid) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        uint4 w;
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * scale, __uint_as_float(o[i + 1]) * scale);
+        __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * scale, __uint_as_float(o[i + 3]) * scale);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * scale, __uint_as_float(o[i + 5]) * scale);
+        __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * scale, __uint_as_float(o[i + 7]) * scale);
+        w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
+        w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
+        *reinterpret_cast<uint4*>(dst + cc * 32 + i) = w;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
-                          const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
-                          const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+                          const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmL,
+                          const __grid_constant__ CUtensorMap tmD, bf16* __restrict__ dqkv, int T, int H,
+                          unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -434,7 +488,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sO = sQ + 2 * QT64;       // dO [2 stages]
   uint8_t* sP = sO + 2 * QT64;       // P^T [2]
   uint8_t* sS = sP + 2 * PT;         // dS^T [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + 2 * PT);
+  float* sL = reinterpret_cast<float*>(sS + 2 * PT);   // lse [2 stages][64]
+  float* sD = sL + 2 * 64;                             // D [2 stages][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + 2 * 64);
   uint64_t* kv_full = bars;          // 1
   uint64_t* q_full = bars + 1;       // 2
   uint64_t* q_empty = bars + 3;      // 2
@@ -461,8 +517,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 128);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&s_empty[s], 8);   // one arrival per compute warp
+      mbar_init(&p_full[s], 8);
       mbar_init(&p_free[s], 1);
     }
     mbar_init(o_full, 1);
@@ -493,14 +549,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = 0; i < n_it && ok; ++i) {
         const int s = i & 1;
         if (!mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-        mbar_expect_tx(&q_full[s], 2 * QT64);
-        const int qr = row_base + (qi0 + i) * 64;
+        mbar_expect_tx(&q_full[s], 2 * QT64 + 2 * 256);
+        const int qs = (qi0 + i) * 64, qr = row_base + qs;
         uint8_t* q = sQ + s * QT64;
         uint8_t* o = sO + s * QT64;
         tma_load_2d(q, &tm64, &q_full[s], h * 128, qr);
         tma_load_2d(q + QT64 / 2, &tm64, &q_full[s], h * 128 + 64, qr);
         tma_load_2d(o, &tmDO, &q_full[s], h * 128, qr);
         tma_load_2d(o + QT64 / 2, &tmDO, &q_full[s], h * 128 + 64, qr);
+        tma_load_2d(sL + s * 64, &tmL, &q_full[s], qs, bh);
+        tma_load_2d(sD + s * 64, &tmD, &q_full[s], qs, bh);
         ++issued;
       }
       const uint64_t t0 = globaltimer_ns();
@@ -552,48 +610,60 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- P^T, dS^T
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
+    const int q4 = warp & 3, half = (warp - 2) >> 2;
+    const int r = q4 * 32 + lane;
     const int key = k0 + r;
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
-    const float* lse_bh = lse + (long long)bh * T;
-    const float* D_bh = Dv + (long long)bh * T;
     bool ok = true;
     for (int i = 0; i < n_it; ++i) {
       const int s = i & 1;
-      const int qbase = (qi0 + i) * 64;
+      const int qbase = (qi0 + i) * 64 + half * 32;
       if (!warp_wait(&s_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      float sv[64], dp[64];
-      ld64(tmem + lane_off + s * 64, sv);
-      ld64(tmem + lane_off + 128 + s * 64, dp);
-      tc_fence_before();
-      mbar_arrive(&s_empty[s]);
-      // P^T[key, q] = exp2(s c - lse_q log2e) for key <= q < T; dS^T = P^T (dP^T - D_q)
+      float sv[32], dp[32];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
+        tmem_ld32_nowait(tmem + lane_off + 128 + s * 64 + half * 32, r1);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const int qq = qbase + e;
-        const bool live = (key <= qq) && (qq < T);
-        const float L = live ? lse_bh[qq] * LOG2E : 0.f;
-        const float Dq = live ? D_bh[qq] : 0.f;
-        const float p = live ? exp2f(fmaf(sv[e], c, -L)) : 0.f;
-        sv[e] = p;
-        dp[e] = p * (dp[e] - Dq);
+        for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[s]);
+      // P^T[key, q] = exp2(s c - lse_q log2e) for key <= q < T; dS^T = P^T (dP^T - D_q)
+      const float* L = sL + s * 64 + half * 32;
+      const float* Dq = sD + s * 64 + half * 32;
+#pragma unroll
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(L + 4 * e4);
+        const float4 d4 = *reinterpret_cast<const float4*>(Dq + 4 * e4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 4 * e4 + u, qq = qbase + e;
+          const bool live = (key <= qq) && (qq < T);
+          const float p = live ? exp2f(fmaf(sv[e], c, -lv[u] * LOG2E)) : 0.f;
+          sv[e] = p;
+          dp[e] = p * (dp[e] - dv[u]);
+        }
       }
       if (i >= 2 && !warp_wait(&p_free[s], ((i - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      st_row64(sP + s * PT, r, sv);
-      st_row64(sS + s * PT, r, dp);
+      st_half_row(sP + s * PT, r, half, sv);
+      st_half_row(sS + s * PT, r, half, dp);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(&p_full[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
     }
     if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
       tc_fence_after();
       const bool valid = key < T;
-      bf16* krow = dqkv + ((long long)row_base + (valid ? key : 0)) * 3 * a + a + h * 128;
-      row128_out(tmem + lane_off + 256, 1.f, krow + a, valid);             // dV
-      row128_out(tmem + lane_off + 384, rsqrtf(128.f), krow, valid);       // dK
+      bf16* krow = dqkv + ((long long)row_base + (valid ? key : 0)) * 3 * a + a + h * 128 + half * 64;
+      row64_out(tmem + lane_off + 256 + half * 64, 1.f, krow + a, valid);          // dV
+      row64_out(tmem + lane_off + 384 + half * 64, rsqrtf(128.f), krow, valid);    // dK
     }
   }
   tc_fence_before();
@@ -605,12 +675,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------- dQ
+// 10 warps as above; compute warps split the 64 key columns in halves.
 // smem: Q, dO [128 x 128] (32 KB each); per stage K_j, V_j [64 x 128] (16 KB
 // each, 3 stages); per buffer dS [128 queries x 64 keys] (16 KB, 2 buffers).
 constexpr int DQ_STAGES = 3;
 constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 2 * PT + 1024 + 256;
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
                         const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
                         const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
@@ -647,8 +718,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 128);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&s_empty[s], 8);   // one arrival per compute warp
+      mbar_init(&p_full[s], 8);
       mbar_init(&p_free[s], 1);
     }
     mbar_init(o_full, 1);
@@ -737,11 +808,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- dS
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
+    const int q4 = warp & 3, half = (warp - 2) >> 2;
+    const int r = q4 * 32 + lane;
     const int qpos = q0 + r;
     const bool valid = qpos < T;
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
     const float L = valid ? lse[(long long)bh * T + qpos] * LOG2E : 0.f;
     const float Dq = valid ? Dv[(long long)bh * T + qpos] : 0.f;
@@ -750,28 +821,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int s = j & 1;
       if (!warp_wait(&s_full[s], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      float sv[64], dp[64];
-      ld64(tmem + lane_off + s * 64, sv);
-      ld64(tmem + lane_off + 128 + s * 64, dp);
-      tc_fence_before();
-      mbar_arrive(&s_empty[s]);
+      float sv[32], dp[32];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
+        tmem_ld32_nowait(tmem + lane_off + 128 + s * 64 + half * 32, r1);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const int kk = j * 64 + e;
-        const bool live = valid && (kk <= qpos);
+        for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[s]);
+      const int kbase = j * 64 + half * 32;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const bool live = valid && (kbase + e <= qpos);
         const float p = live ? exp2f(fmaf(sv[e], c, -L)) : 0.f;
         dp[e] = p * (dp[e] - Dq);
       }
       if (j >= 2 && !warp_wait(&p_free[s], ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      st_row64(sS + s * PT, r, dp);
+      st_half_row(sS + s * PT, r, half, dp);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(&p_full[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
     }
     if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
       tc_fence_after();
-      bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128;
-      row128_out(tmem + lane_off + 256, rsqrtf(128.f), qrow, valid);
+      bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128 + half * 64;
+      row64_out(tmem + lane_off + 256 + half * 64, rsqrtf(128.f), qrow, valid);
     }
   }
   tc_fence_before();

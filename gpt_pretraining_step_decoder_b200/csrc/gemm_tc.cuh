@@ -268,7 +268,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 128); }
+    // tempty: one arrival per epilogue warp
+    for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4); }
     for (int s = 0; s < 8; ++s) mbar_init(&auxbar[s], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -584,7 +585,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       if (KM == K_LOGITS && m < p.M) e.stats[m * p.n_tiles + (mn % p.n_tiles)] = make_float2(rmax, rsum);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
     if (lane == 0) bulk_wait0();  // all of this warp's stores are complete

@@ -104,7 +104,8 @@ static int get_encode() {
 // Tensor map of `rank` dims (innermost first) with byte strides for dims 1..,
 // 128-byte swizzle, zero fill outside the tensor.
 static int make_tmap_gen(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr,
-                         const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+                         const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                         CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   TRY(get_encode());
   if (reinterpret_cast<uintptr_t>(ptr) & 15) return fail(GPT_ERR_ARG, "TMA operand %p not 16-byte aligned", ptr);
   for (int i = 0; i + 1 < rank; ++i)
@@ -115,7 +116,7 @@ static int make_tmap_gen(CUtensorMap* m, CUtensorMapDataType dt, int rank, const
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
   CUresult r = g_encode(m, dt, rank, const_cast<void*>(ptr), d, s, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(GPT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return GPT_OK;
@@ -369,6 +370,7 @@ static int validate(const gpt_config* c) {
     if (c->head_dim != 128) return fail(GPT_ERR_CONFIG, "bf16 mode needs head_dim == 128");
     if (c->d_model % 64 || c->d_ff % 64 || c->vocab % 64)
       return fail(GPT_ERR_CONFIG, "bf16 mode needs d_model, d_ff, vocab multiples of 64");
+    if (c->seq_len % 4) return fail(GPT_ERR_CONFIG, "bf16 mode needs seq_len a multiple of 4");
   }
   if (c->x0_rows < 0 || c->v_rows < 0 || c->x0_rows > 0x7fffffffLL || c->v_rows > 0x7fffffffLL)
     return fail(GPT_ERR_CONFIG, "table rows out of range");
@@ -820,16 +822,24 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
       attr = true;
     }
     const long long a = (long long)c.n_head * c.head_dim;
-    CUtensorMap t128, t64, tdo;
+    CUtensorMap t128, t64, tdo, tl, td;
     TRY(make_tmap(&t128, qkv, 3 * a, N, 3 * a, 64, 128));
     TRY(make_tmap(&t64, qkv, 3 * a, N, 3 * a, 64, 64));
     TRY(make_tmap(&tdo, dout, a, N, a, 64, 64));
+    {
+      // lse and D [B*H, T] fp32, 64 positions per box, no swizzle
+      const uint64_t dims[2] = {(uint64_t)c.seq_len, (uint64_t)c.micro_batch * c.n_head};
+      const uint64_t str[1] = {(uint64_t)c.seq_len * 4};
+      const uint32_t box[2] = {64, 1};
+      TRY(make_tmap_gen(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, lse, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+      TRY(make_tmap_gen(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Dv, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    }
     dim3 gk(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
     dim3 gq(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
     bf16* g16 = reinterpret_cast<bf16*>(dqkv);
-    ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<gk, fatcb::THREADS, fatcb::DKDV_SMEM, m->st>>>(
-        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
-    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<gq, fatcb::THREADS, fatcb::DQ_SMEM, m->st>>>(
+    ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<gk, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st>>>(
+        t128, t64, tdo, tl, td, g16, c.seq_len, c.n_head, m->err());
+    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<gq, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
         t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;

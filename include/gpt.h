@@ -77,8 +77,9 @@ extern "C" {
  * PyTorch's default for F.rms_norm without eps), bigram hash constants
  * p1 = 2654435761, p2 = 2246822519, table beta 0.95 / eps 1e-10.
  * Constraints: d_model == n_head * head_dim, n_kv_head == n_head (or 0),
- * head_dim even; in bf16 mode head_dim == 128 and d_model, d_ff, vocab are
- * multiples of 64; x0_rows / v_rows are 0 (table absent) or >= 1.
+ * head_dim even; in bf16 mode head_dim == 128, d_model, d_ff, vocab are
+ * multiples of 64 and seq_len a multiple of 4; x0_rows / v_rows are 0
+ * (table absent) or >= 1.
  */
 typedef struct gpt_config {
   int n_layer, d_model, n_head, head_dim, n_kv_head, d_ff, vocab, seq_len, micro_batch;
