@@ -184,39 +184,29 @@ def run_ours(args, w, rank, world, dist):
     import gpt_pretraining_step_decoder_b200 as g
 
     dev = torch.device("cuda", torch.cuda.current_device())
+    from gpt_pretraining_step_decoder_b200 import dp
     cfg = g.make_config(**w)
-    model = g.Model(cfg, seed=w["seed"] + 17 * rank)
+    model = g.Model(cfg, seed=w["seed"])  # identical replicas on every rank
     A, B, T, V = w["grad_accum"], w["micro_batch"], w["seq_len"], w["vocab"]
     n_micro = A * (args.warmup + args.steps)
     host_tok, host_tgt = [], []
     for i in range(n_micro):
-        tok, tgt = tokens_and_targets(B, T, V, w["seed"] + 1000 * rank, w["zipf_s"], w["repeat_frac"], micro=i)
+        tok, tgt = tokens_and_targets(B, T, V, dp.rank_stream_seed(w["seed"], rank), w["zipf_s"], w["repeat_frac"],
+                                      micro=i)
         host_tok.append(torch.from_numpy(tok).pin_memory())
         host_tgt.append(torch.from_numpy(tgt).pin_memory())
     dev_tok = [t.to(dev) for t in host_tok]
     dev_tgt = [t.to(dev) for t in host_tgt]
     stream = model.stream
-    flat_grad = None
-    if world > 1:
-        p, _, shape = g.gpt_tensor(model.h, "*", g.KIND_GRAD)
-        off = p - model.arena.data_ptr()
-        flat_grad = model.arena[off:off + shape[0] * 4].view(torch.float32)
     lr = args.lr
 
-    def step(i, tok_src, tgt_src, loss_host=None):
-        for a in range(A):
-            j = i * A + a
-            model.forward_loss(tok_src[j], tgt_src[j])
-            if world > 1:
-                g.gpt_backward(model.h, lr)
-            else:
-                model.backward_step(lr)
-            if loss_host is not None:
-                loss_host.copy_(model.loss, non_blocking=True)
+    def step(i, tok_src, tgt_src):
         if world > 1:
-            dist.all_reduce(flat_grad)
-            flat_grad.mul_(1.0 / world)
-            g.gpt_optimizer_step(model.h, lr)
+            dp.train_step(model, [(tok_src[i * A + a], tgt_src[i * A + a]) for a in range(A)], lr)
+            return
+        for a in range(A):
+            model.forward_loss(tok_src[i * A + a], tgt_src[i * A + a])
+            model.backward_step(lr)
 
     def timed(fn_step, first, count):
         if dist is not None:
@@ -273,14 +263,13 @@ def run_ours(args, w, rank, world, dist):
             in_tgt.copy_(host_tgt[j], non_blocking=True)
             model.forward_loss(in_tok, in_tgt)
             if world > 1:
-                g.gpt_backward(model.h, lr)
+                model.backward(lr)
             else:
                 model.backward_step(lr)
             loss_host.copy_(model.loss, non_blocking=True)
         if world > 1:
-            dist.all_reduce(flat_grad)
-            flat_grad.mul_(1.0 / world)
-            g.gpt_optimizer_step(model.h, lr)
+            dp.average_gradients(model.flat_grad())
+            model.optimizer_step(lr)
 
     ms_e2e = timed(e2e_step, args.warmup, args.steps)
     st = model.sync_status()
@@ -344,6 +333,84 @@ def run_ours(args, w, rank, world, dist):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ table kernels
+def run_tables(args, w):
+    """Achieved HBM bandwidth of the standalone bigram-table calls on the
+    full-size tables (2,097,152 x d and 1,048,576 x d bf16), rows hashed from
+    the workload's token stream; one micro-batch (N = B*T) and a whole
+    accumulated step (N = A*B*T).  L2 is flushed (a 256 MB write) before every
+    timed call; each call is bracketed by CUDA events on the launching stream.
+    Algorithmic bytes: gather N*d*2 read + N*d*2 written + N*4 ids; update
+    N*d*4 gradient + U*(2*d*2 + 2*4) rows and states read and written + N*4
+    ids + 4*N*4 sorting, U = distinct rows."""
+    import torch
+    import gpt_pretraining_step_decoder_b200 as g
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream()
+    d = w["d_model"]
+    B, T, A, V = w["micro_batch"], w["seq_len"], w["grad_accum"], w["vocab"]
+    peaks, peak_src = measured_peaks()
+    toks = [torch.from_numpy(tokens_and_targets(B, T, V, w["seed"], w["zipf_s"], w["repeat_frac"], micro=i)[0]).to(dev)
+            for i in range(A)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    results = []
+    with ClockSampler(0) as clk:
+        for name, R in (("x0", w["x0_rows"]), ("v", w["v_rows"])):
+            if not R:
+                continue
+            table = (torch.randn((R, d), device=dev) * 0.02).to(torch.bfloat16)
+            state = torch.zeros(R, dtype=torch.float32, device=dev)
+            for n_micro in (1, A):
+                n = n_micro * B * T
+                rows = torch.empty(n, dtype=torch.int32, device=dev)
+                for i in range(n_micro):
+                    g.ngram_hash(toks[i], B, T, V, w["hash_p1"], w["hash_p2"], R, rows[i * B * T:(i + 1) * B * T])
+                out = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+                grad = torch.randn((n, d), dtype=torch.float32, device=dev)
+                ws_bytes = g.ngram_sparse_update_workspace_bytes(n, d)
+                ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+                nupd = torch.zeros(1, dtype=torch.int32, device=dev)
+                upd = torch.empty(n, dtype=torch.int32, device=dev)
+                g.ngram_sparse_update(table, state, R, d, g.DTYPE_BF16, rows, grad, n, 1e-4, 0.95, 1e-10,
+                                      upd, nupd, ws, ws_bytes)
+                torch.cuda.synchronize()
+                U = int(nupd.item())
+                calls = {
+                    "ngram_gather": (lambda: g.ngram_gather(rows, n, table, R, d, g.DTYPE_BF16, out, 0),
+                                     2.0 * n * d * 2 + 4.0 * n),
+                    "ngram_sparse_update": (lambda: g.ngram_sparse_update(table, state, R, d, g.DTYPE_BF16, rows, grad,
+                                                                          n, 1e-4, 0.95, 1e-10, None, None, ws,
+                                                                          ws_bytes),
+                                            4.0 * n * d + U * (2.0 * d * 2 + 8) + 4.0 * n + 16.0 * n),
+                }
+                for cname, (fn, nbytes) in calls.items():
+                    times = []
+                    for it in range(args.warmup + args.steps):
+                        flush.zero_()
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record(st)
+                        fn()
+                        e1.record(st)
+                        torch.cuda.synchronize()
+                        if it >= args.warmup:
+                            times.append(e0.elapsed_time(e1))
+                    if g.ngram_sync_status() != g.GPT_OK:
+                        raise RuntimeError(f"{cname}: device error {g.gpt_last_error()}")
+                    us = 1e3 * float(np.median(times))
+                    gbs = nbytes / (us * 1e-6) / 1e9
+                    results.append({"call": cname, "table": f"{name} {R}x{d} bf16", "n": n, "distinct_rows": U,
+                                    "u_over_n": U / n, "us": us, "algorithmic_bytes": nbytes, "gbs": gbs,
+                                    "frac_of_measured_hbm": gbs / peaks["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0})
+                del out, grad, ws, upd
+            del table, state
+            torch.cuda.empty_cache()
+    line = {"metric": "bigram table calls: achieved HBM bandwidth (algorithmic bytes / CUDA-event time)",
+            "unit": "GB/s", "workload": w["name"], "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy",
+            "steps": args.steps, "warmup": args.warmup, "l2": "flushed (256 MB write) before every timed call",
+            "results": results, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def parse_override(items):
     out = {}
     for it in items:
@@ -368,6 +435,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--lr", type=float, default=1e-4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--measure", default="step", choices=["step", "tables"],
+                    help="step: the training step (default); tables: bandwidth of the bigram-table calls")
     ap.add_argument("--override", nargs="*", default=[],
                     help="workload field overrides, e.g. n_layer=1 micro_batch=8 (profiling captures)")
     args = ap.parse_args()
@@ -378,6 +447,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         run_reference(args, w, rank, world)
+        return
+    if args.measure == "tables":
+        import torch
+        torch.cuda.set_device(0)
+        run_tables(args, workload(args.workload if args.workload != "gpt2s_bf16" else "gpt2s_tables_bf16",
+                                  **parse_override(args.override)))
         return
     import torch
     dist = None

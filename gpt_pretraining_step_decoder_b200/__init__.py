@@ -300,6 +300,20 @@ class Model:
     def backward_step(self, lr):
         gpt_backward_step(self.h, lr)
 
+    def backward(self, lr):
+        """Backward of the last forward without the dense optimizer step (the
+        table updates still run inline); pair with optimizer_step."""
+        gpt_backward(self.h, lr)
+
+    def optimizer_step(self, lr):
+        gpt_optimizer_step(self.h, lr)
+
+    def flat_grad(self):
+        """The whole fp32 dense gradient as one flat torch view (no copy)."""
+        p, _, shape = gpt_tensor(self.h, "*", KIND_GRAD)
+        off = p - self.arena.data_ptr()
+        return self.arena[off:off + shape[0] * 4].view(self.torch.float32)
+
     def sync_status(self):
         return gpt_sync_status(self.h)
 

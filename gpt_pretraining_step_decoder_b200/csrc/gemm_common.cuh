@@ -21,8 +21,10 @@ enum EpiMode {
   EPI_RELU2 = 3,      // C(act) = relu(acc)^2                        (ReLU^2 forward)
   EPI_DRELU2 = 4,     // C(act) = 2 * sqrt(aux(act)) * acc, aux = relu(a)^2  (ReLU^2 backward:
                       // d relu(a)^2 / da = 2 relu(a) = 2 sqrt(relu(a)^2))
-  EPI_LOGITS = 5,     // z = softcap(acc): C(f32) = z, and per (row, column tile) the
-                      // running max and sum of exp(z - max) into stats (tensor-core path)
+  EPI_LOGITS = 5,     // z = softcap(acc); per (row, column tile) m = max z and
+                      // s = sum exp(z - m) into stats; C(bf16) = exp(z - m) (the tile-local
+                      // softmax numerators); z at the row's target column into ztgt
+                      // (tensor-core path only)
   EPI_QKV = 6,        // fused q|k|v projection output (tensor-core path, 128-wide heads):
                       // q, k heads rotated (RoPE) and RMS-normalised per head, v heads plus
                       // the value-table row; C(act) = result
@@ -38,7 +40,9 @@ struct GemmEpilogue {
   int beta;
   float softcap;    // EPI_LOGITS: 0 = off, else z = softcap * tanh(acc / softcap)
   float2* stats;    // EPI_LOGITS: [M, n_tiles] (max, sum of exp(z - max))
-  // EPI_QKV: rope table [T, 64, (cos, sin)], per-(row, head) rstd outputs,
+  const int32_t* targets;  // EPI_LOGITS: target column per row (< 0: none), nullable
+  float* ztgt;             // EPI_LOGITS: z at the target column per row
+  // EPI_QKV: rope table frequency-major [64, T, (cos, sin)], per-(row, head) rstd outputs,
   // optional value table [rows, H*128] (bf16) and its row per position
   const float* rope;
   float* rstd_q;
@@ -72,8 +76,7 @@ __device__ __forceinline__ void epi_apply_one(const GemmEpilogue& e, long long m
       reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(2.f * sqrtf(g) * acc);
       break;
     }
-    case EPI_LOGITS:
-      reinterpret_cast<float*>(e.C)[off] = acc;
+    default:  // EPI_LOGITS and EPI_QKV exist only in the tensor-core kernel's epilogue
       break;
   }
 }

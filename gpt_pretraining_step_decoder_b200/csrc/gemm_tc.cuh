@@ -41,8 +41,15 @@ enum KMode {
   K_PARTIAL,      // split-K fp32 partials [splits, M, N]
   K_RELU2,        // bf16 relu(acc)^2
   K_DRELU2,       // bf16 2 sqrt(aux) acc
-  K_LOGITS,       // fp32 softcap(acc) + per-tile row statistics
+  K_LOGITS,       // bf16 exp(z - tile max), z = softcap(acc), + per-tile row statistics
   K_QKV,          // bf16 q|k|v with RoPE + QK-norm (+ value-table row) per 128-wide head
+};
+
+// The ReLU^2-backward epilogue streams activations through a ring of its
+// own, which costs a pipeline stage; every other epilogue uses the light
+// configuration.  Host and kernel both take the configuration from here.
+template <int KM> struct KmHeavy {
+  static constexpr int value = KM == K_DRELU2 ? 1 : 0;
 };
 
 // HEAVY = 1: the epilogue-heavy variant (logits, ReLU^2 backward) trades one
@@ -53,9 +60,9 @@ template <int BN, int HEAVY> struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators (power of two >= 32)
-  static constexpr int NSTG = HEAVY ? 2 : 1;          // staging buffers per epilogue warp
-  static constexpr int NAUX = HEAVY ? 2 : 1;          // activation blocks in flight per epilogue warp
-  static constexpr int AUX = NAUX * 32 * 128;         // activation bytes per epilogue warp
+  static constexpr int NSTG = 2;                      // staging buffers per epilogue warp
+  static constexpr int NAUX = 2;                      // activation blocks in flight (ReLU^2 backward)
+  static constexpr int AUX = HEAVY ? NAUX * 32 * 128 : 0;  // activation bytes per epilogue warp
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * NSTG * 32 * 128 + 4 * AUX + 1024 /*align*/ +
                                     256 /*barriers*/;
 };
@@ -64,6 +71,7 @@ struct Params {
   int M, N, K;
   int a_kmajor, b_kmajor;
   int m_tiles, n_tiles, splits, kb_per_split, kb_total;
+  int group_m;  // tile order: groups of group_m m-blocks, m fastest inside a group
   GemmEpilogue epi;
   float* partial;  // splits > 1: fp32 [splits, M, N]
   unsigned* err;
@@ -238,6 +246,32 @@ __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// z = cap * tanh(acc / cap) (nanochat's logit softcap) for a block of
+// values, with tanh(x) = 1 - 2 / (exp(2x) + 1).  Called only under a
+// warp-uniform `cap > 0` test around the whole block, so the default
+// (no softcap) path carries none of this arithmetic.
+template <int NVAL>
+__device__ __forceinline__ void softcap_block(float (&v)[NVAL], float cap) {
+  const float two_over_cap = 2.f / cap;
+#pragma unroll
+  for (int i = 0; i < NVAL; ++i) v[i] = cap * (1.f - __fdividef(2.f, __expf(v[i] * two_over_cap) + 1.f));
+}
+
+// Output tile (m-block, n-block) of linear tile index mn.  Tiles come in
+// groups of group_m m-blocks; inside a group the m-block varies fastest, so
+// the CTAs running at one time cover about group_m x (SMs / group_m) tiles
+// and read each A row-block and B column-block from HBM about once per group
+// (the rest of the reuse comes from L2).
+__device__ __forceinline__ void tile_coords(int mn, const Params& p, int& mt, int& nt) {
+  const int per_group = p.group_m * p.n_tiles;
+  const int g = mn / per_group;
+  const int first_m = g * p.group_m;
+  const int gsize = min(p.group_m, p.m_tiles - first_m);
+  const int r = mn - g * per_group;
+  mt = first_m + r % gsize;
+  nt = r / gsize;
+}
+
 // byte offset of 16-byte chunk j of row r in a 128-byte-swizzled block
 __device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
@@ -246,8 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmAux,
                    const Params p) {
-  constexpr int HEAVY = (KM == K_DRELU2 || KM == K_LOGITS) ? 1 : 0;
-  using C = Cfg<BN, HEAVY>;
+  using C = Cfg<BN, KmHeavy<KM>::value>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -298,7 +331,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int split = t % p.splits;
         const int mn = t / p.splits;
-        const int m0 = (mn / p.n_tiles) * BM, n0 = (mn % p.n_tiles) * BN;
+        int mt, nt;
+        tile_coords(mn, p, mt, nt);
+        const int m0 = mt * BM, n0 = nt * BN;
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -367,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t aux_phase = 0;             // bit b: parity of the next wait on abar[b]
     uint32_t aux_pending = 0;           // bit b: a load into buffer b is in flight
     const GemmEpilogue& e = p.epi;
-    constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL || KM == K_LOGITS;
+    constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL;
     constexpr bool has_aux = KM == K_DRELU2;
     constexpr int CW = f32out ? 32 : 64;  // columns per 128-byte staging row
     int acc = 0;
@@ -376,8 +411,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int split = t % p.splits;
       const int mn = t / p.splits;
-      const int m0 = (mn / p.n_tiles) * BM;
-      const int n0 = (mn % p.n_tiles) * BN;
+      int mt, nt;
+      tile_coords(mn, p, mt, nt);
+      const int m0 = mt * BM;
+      const int n0 = nt * BN;
       const int mrow0 = m0 + q * 32;
       const long long m = (long long)mrow0 + lane;
       const int nblk = min(BN / CW, (p.N - n0 + CW - 1) / CW);
@@ -394,6 +431,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       float rmax = -INFINITY, rsum = 0.f;
       const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      int ytgt = -1;
+      if constexpr (KM == K_LOGITS) {
+        // first pass over the accumulator: the tile's row maximum, so that
+        // the stored numerators exp(z - max) lie in (0, 1]
+        ytgt = (e.targets != nullptr && m < p.M) ? e.targets[m] : -1;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int nc = n0 + c * 32;
+          if (nc >= p.N) break;  // warp-uniform
+          uint32_t r[32];
+          tmem_ld32_nowait(trow + c * 32, r);
+          tmem_wait_ld();
+          const int nv = min(32, p.N - nc);
+          float z[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(r[i]) * e.alpha;
+          if (e.softcap > 0.f) softcap_block<32>(z, e.softcap);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nv) rmax = fmaxf(rmax, z[i]);
+        }
+      }
       if constexpr (KM == K_QKV) {
         // one 128-wide head per iteration; this lane owns row m of it
         const bool row_ok = m < p.M;
@@ -422,11 +481,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (sec < 2) {
             // RoPE ("$1000 tier nanochat run", apply_rotary_emb): y1 = x1 cos + x2 sin,
             // y2 = -x1 sin + x2 cos over the two halves of the head, then QK-norm
-            const float2* cs = reinterpret_cast<const float2*>(e.rope) + (long long)tpos * 64;
+            // frequency-major table: consecutive lanes (positions) read consecutive pairs
+            const float2* cs = reinterpret_cast<const float2*>(e.rope) + tpos;
             float ss = 0.f;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-              const float2 w = cs[i];
+              const float2 w = cs[(long long)i * e.T];
               const float x1 = v[i], x2 = v[i + 64];
               v[i] = x1 * w.x + x2 * w.y;
               v[i + 64] = -x1 * w.y + x2 * w.x;
@@ -499,22 +559,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         if constexpr (KM == K_LOGITS) {
-          const int nv = min(32, p.N - nc);
-          if (e.softcap > 0.f) {
+          const int nv = min(64, p.N - nc);
+          const int yo = ytgt - nc;  // target column within this block, if here
+          float zt = 0.f;
+          if (e.softcap > 0.f) softcap_block<64>(v, e.softcap);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = e.softcap * tanhf(v[i] / e.softcap);
+          for (int i = 0; i < 64; ++i) {
+            const float z = v[i];
+            zt = (i == yo) ? z : zt;
+            const float pr = (i < nv) ? __expf(z - rmax) : 0.f;
+            rsum += pr;
+            v[i] = pr;
           }
-          float cmax = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nv) cmax = fmaxf(cmax, v[i]);
-          const float nm = fmaxf(rmax, cmax);
-          float s = (rmax == -INFINITY) ? 0.f : rsum * __expf(rmax - nm);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nv) s += __expf(v[i] - nm);
-          rmax = nm;
-          rsum = s;
+          if (yo >= 0 && yo < 64) e.ztgt[m] = zt;
         } else if constexpr (KM == K_RELU2) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) { const float r = fmaxf(v[i], 0.f); v[i] = r * r; }
@@ -583,7 +640,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sbuf = (sbuf + 1) % C::NSTG;
       }
       if (!ok) break;
-      if (KM == K_LOGITS && m < p.M) e.stats[m * p.n_tiles + (mn % p.n_tiles)] = make_float2(rmax, rsum);
+      if (KM == K_LOGITS && m < p.M) e.stats[m * p.n_tiles + nt] = make_float2(rmax, rsum);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

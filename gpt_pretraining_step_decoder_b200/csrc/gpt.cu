@@ -134,7 +134,7 @@ static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t o
 template <int BN, int KM>
 static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tcm,
                             const CUtensorMap& taux, const tc::Params& p, cudaStream_t st) {
-  using C = tc::Cfg<BN, (KM == tc::K_DRELU2 || KM == tc::K_LOGITS) ? 1 : 0>;
+  using C = tc::Cfg<BN, tc::KmHeavy<KM>::value>;
   static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
   static bool attr_done = false;
   if (!attr_done) {
@@ -162,6 +162,9 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   p.a_kmajor = A.kmajor; p.b_kmajor = B.kmajor;
   p.m_tiles = cdiv(M, tc::BM);
   p.n_tiles = cdiv(N, BN);
+  // n-fastest order while the whole B operand stays in L2; grouped m-blocks
+  // when B is large (the LM head's vocab-sized operand)
+  p.group_m = (double)N * K * 2 > 32.0 * (1 << 20) ? (p.m_tiles < 16 ? p.m_tiles : 16) : 1;
   p.kb_total = cdiv(K, tc::BK);
   if (splits < 1) splits = 1;
   if (splits > p.kb_total) splits = p.kb_total;
@@ -177,7 +180,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
     const uint64_t str[2] = {(uint64_t)N * 4, (uint64_t)M * N * 4};
     const uint32_t box[3] = {32, 32, 1};
     TRY(make_tmap_gen(&tcm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, partial, dims, str, box));
-  } else if (e.mode == EPI_STORE_F32 || e.mode == EPI_ACCUM_F32 || e.mode == EPI_LOGITS) {
+  } else if (e.mode == EPI_STORE_F32 || e.mode == EPI_ACCUM_F32) {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M}, str[1] = {(uint64_t)e.ldc * 4};
     const uint32_t box[2] = {32, 32};
     TRY(make_tmap_gen(&tcm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, e.C, dims, str, box));
@@ -305,7 +308,7 @@ static GemmEpilogue epi(int mode, void* C, long long ldc, int beta = 0, void* C2
                         const void* aux = nullptr, float alpha = 1.f) {
   GemmEpilogue e;
   e.mode = mode; e.C = C; e.ldc = ldc; e.C2 = C2; e.aux = aux; e.alpha = alpha; e.beta = beta;
-  e.softcap = 0.f; e.stats = nullptr;
+  e.softcap = 0.f; e.stats = nullptr; e.targets = nullptr; e.ztgt = nullptr;
   e.rope = nullptr; e.rstd_q = e.rstd_k = nullptr; e.hv = nullptr; e.rv = nullptr;
   e.T = e.H = e.qk_norm = 0; e.eps = 0.f;
   return e;
@@ -341,11 +344,10 @@ struct Plan {
   size_t x, emb_rstd, xf, rstd_f, tok_copy, rows_x, rows_v;
   std::vector<LayerActs> layers;
   size_t dx, dx_lp, du, dqkv, da, dout, Dattn, gv, dxf, pending;
-  size_t logits, dz, ce_stats, tok_loss, ce_scale, ce_count, loss_scratch;
-  size_t sort_keys_a, sort_keys_b, sort_vals_a, sort_vals_b, sort_counts;
-  size_t seg_start, pstart, plen, pseg, pslot, lfirst, lnslots, lseg, counters, seg_partial;
+  size_t logits, dz, ce_stats, ce_ztgt, tok_loss, ce_scale, ce_count, loss_scratch;
+  size_t sort_keys_a, sort_keys_b, sort_vals_a, sort_vals_b, sort_counts, part_head, part_tail;
   size_t splitk; long long splitk_elems;
-  size_t norm_part, clip_coef, grad_norm, rope_cs, err;
+  size_t norm_part, clip_coef, grad_norm, rope_cs, rope_cs_t, err;
   int chunk;
   size_t total;
 };
@@ -449,31 +451,25 @@ static void make_plan(const gpt_config& c, Plan& p) {
   long long chunk = c.lm_chunk_rows > 0 ? c.lm_chunk_rows : 8192;
   if (chunk > N) chunk = N;
   p.chunk = (int)chunk;
-  p.logits = cv.take(chunk * V * 4);
+  // fp32 mode materialises fp32 logits; bf16 mode writes the tile-local
+  // softmax numerators straight into dz and rescales them in place
+  p.logits = b16 ? 0 : cv.take(chunk * V * 4);
   p.dz = cv.take(chunk * V * es);
   p.ce_stats = cv.take(chunk * ((V + 127) / 128) * 8);
+  p.ce_ztgt = cv.take(chunk * 4);
   p.tok_loss = cv.take(N * 4);
   p.ce_scale = cv.take(4);
   p.ce_count = cv.take(4);
   p.loss_scratch = cv.take(4);
   // ---- bucketing workspace (positions by row / by token)
-  const long long nblk = (N + RADIX_TILE - 1) / RADIX_TILE;
+  const long long nchunks = (N + CHUNK - 1) / CHUNK;
   p.sort_keys_a = cv.take(N * 4);
   p.sort_keys_b = cv.take(N * 4);
   p.sort_vals_a = cv.take(N * 4);
   p.sort_vals_b = cv.take(N * 4);
-  p.sort_counts = cv.take(256 * nblk * 4);
-  const long long maxp = N + N / PIECE + 2, maxl = N / PIECE + 2, maxslots = 2 * (N / PIECE) + 4;
-  p.seg_start = cv.take((N + 1) * 4);
-  p.pstart = cv.take(maxp * 4);
-  p.plen = cv.take(maxp * 4);
-  p.pseg = cv.take(maxp * 4);
-  p.pslot = cv.take(maxp * 4);
-  p.lfirst = cv.take(maxl * 4);
-  p.lnslots = cv.take(maxl * 4);
-  p.lseg = cv.take(maxl * 4);
-  p.counters = cv.take(16);
-  p.seg_partial = cv.take(maxslots * (d > a ? d : a) * 4);
+  p.sort_counts = cv.take(256 * radix_blocks(N) * 4);
+  p.part_head = cv.take(nchunks * (d > a ? d : a) * 4);
+  p.part_tail = cv.take(nchunks * (d > a ? d : a) * 4);
   // ---- split-K partials: the largest weight gradient x 8 splits
   long long mx = 3 * a * d;
   if (F * d > mx) mx = F * d;
@@ -483,6 +479,7 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.clip_coef = cv.take(4);
   p.grad_norm = cv.take(4);
   p.rope_cs = cv.take((long long)c.seq_len * c.head_dim * 4);
+  p.rope_cs_t = cv.take((long long)c.seq_len * c.head_dim * 4);
   p.err = cv.take(16);
   p.total = cv.take(0) + 256;
 }
@@ -599,7 +596,7 @@ extern "C" int gpt_create(const gpt_config* cfg, unsigned long long seed, void* 
     }
   }
   ++g_launches; rope_table_kernel<<<grid_for((long long)c.seq_len * c.head_dim / 2, 256), 256, 0, m->st>>>(
-      m->at<float>(p.rope_cs), c.seq_len, c.head_dim, (double)c.rope_base);
+      m->at<float>(p.rope_cs), m->at<float>(p.rope_cs_t), c.seq_len, c.head_dim, (double)c.rope_base);
   e = cudaGetLastError();
   if (e != cudaSuccess) { delete m; return fail(GPT_ERR_CUDA, "init launch: %s", cudaGetErrorString(e)); }
   int s = refresh_lp(m);
@@ -710,8 +707,7 @@ extern "C" int gpt_tensor(gpt_model* m, const char* name, int kind, void** ptr, 
 struct SortWs {
   uint32_t *ka, *kb, *counts;
   int32_t *va, *vb;
-  int32_t *seg_start, *pstart, *plen, *pseg, *pslot, *lfirst, *lnslots, *lseg, *counters;
-  float* partial;
+  float *part_head, *part_tail;  // [n / CHUNK, d] partial sums of runs that cross chunk edges
 };
 
 static SortWs sort_ws(const gpt_model* m) {
@@ -720,37 +716,43 @@ static SortWs sort_ws(const gpt_model* m) {
   w.ka = m->at<uint32_t>(p.sort_keys_a); w.kb = m->at<uint32_t>(p.sort_keys_b);
   w.va = m->at<int32_t>(p.sort_vals_a); w.vb = m->at<int32_t>(p.sort_vals_b);
   w.counts = m->at<uint32_t>(p.sort_counts);
-  w.seg_start = m->at<int32_t>(p.seg_start); w.pstart = m->at<int32_t>(p.pstart);
-  w.plen = m->at<int32_t>(p.plen); w.pseg = m->at<int32_t>(p.pseg); w.pslot = m->at<int32_t>(p.pslot);
-  w.lfirst = m->at<int32_t>(p.lfirst); w.lnslots = m->at<int32_t>(p.lnslots); w.lseg = m->at<int32_t>(p.lseg);
-  w.counters = m->at<int32_t>(p.counters); w.partial = m->at<float>(p.seg_partial);
+  w.part_head = m->at<float>(p.part_head); w.part_tail = m->at<float>(p.part_tail);
   return w;
 }
 
-// Stable sort of (key, position) by key, then segments and pieces.  Leaves
-// sorted keys in *keys_out and positions in *perm_out.
+// Stable sort of the positions 0..n-1 by key (row id in [0, key_range); an
+// invalid id sorts as key_range with position -1).  Leaves the sorted keys in
+// *keys_out and the positions in *perm_out; with uniq_out / n_uniq_out given,
+// also the distinct valid keys in ascending order and their number.
 static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long key_range,
                          const uint32_t** keys_out, const int32_t** perm_out, int32_t* uniq_out,
                          int* n_uniq_out, unsigned* err, cudaStream_t st) {
-  ++g_launches; iota_kernel<<<grid_for(n, 256), 256, 0, st>>>(keys, w.ka, w.va, n, key_range, err);
-  LAUNCH_CHECK();
   int bits = 1;
-  while (bits < 32 && (1LL << bits) < key_range) ++bits;
+  while (bits < 32 && (1LL << bits) <= key_range) ++bits;  // the value key_range must fit
   const int passes = (bits + 7) / 8;
-  const int nblk = (n + RADIX_TILE - 1) / RADIX_TILE;
-  uint32_t *kin = w.ka, *kout = w.kb;
-  int32_t *vin = w.va, *vout = w.vb;
+  const int items = radix_items(n);
+  const long long nblk = radix_blocks(n);
+  const int scanned = nblk > RADIX_FUSED_MAX_BLOCKS;
+  const uint32_t* kin = nullptr;
+  const int32_t* vin = nullptr;
+  uint32_t* kout = w.ka;
+  int32_t* vout = w.va;
   for (int ps = 0; ps < passes; ++ps) {
-    ++g_launches; radix_hist_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, n, 8 * ps, w.counts);
-    ++g_launches; exclusive_scan_kernel<<<1, 1024, 0, st>>>(w.counts, 256 * nblk);
-    ++g_launches; radix_scatter_kernel<<<nblk, RADIX_THREADS, 0, st>>>(kin, vin, n, 8 * ps, w.counts, kout, vout);
+    const int32_t* raw = ps == 0 ? keys : nullptr;
+    ++g_launches; radix_hist_kernel<<<(unsigned)nblk, RADIX_THREADS, 0, st>>>(kin, raw, n, key_range, items, 8 * ps, w.counts);
+    if (scanned) { ++g_launches; radix_offsets_kernel<<<1, 1024, 0, st>>>(w.counts, (int)nblk); }
+    ++g_launches; radix_scatter_kernel<<<(unsigned)nblk, RADIX_THREADS, 0, st>>>(kin, vin, raw, n, key_range, items, 8 * ps,
+                                                                  w.counts, scanned, kout, vout, err);
     LAUNCH_CHECK();
-    std::swap(kin, kout);
-    std::swap(vin, vout);
+    kin = kout;
+    vin = vout;
+    kout = (kout == w.ka) ? w.kb : w.ka;
+    vout = (vout == w.va) ? w.vb : w.va;
   }
-  ++g_launches; segments_kernel<<<1, 1024, 0, st>>>(kin, n, w.seg_start, w.pstart, w.plen, w.pseg, w.pslot, w.lfirst,
-                                      w.lnslots, w.lseg, w.counters, uniq_out, n_uniq_out);
-  LAUNCH_CHECK();
+  if (uniq_out || n_uniq_out) {
+    ++g_launches; unique_keys_kernel<<<1, 1024, 0, st>>>(kin, n, key_range, uniq_out, n_uniq_out);
+    LAUNCH_CHECK();
+  }
   *keys_out = kin;
   *perm_out = vin;
   return GPT_OK;
@@ -763,11 +765,11 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const uint32_t* skeys;
   const int32_t* perm;
   TRY(bucket_by_key(w, rows, n, n_rows, &skeys, &perm, uniq_out, n_uniq_out, err, st));
-  const long long maxp = (long long)n + n / PIECE + 2, maxl = n / PIECE + 2;
-  WITH_NV(d, ++g_launches; table_piece_kernel<NV, tab_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
-      table, state, d, grad, skeys, perm, w.pstart, w.plen, w.pslot, w.counters, w.partial, lr, beta, eps););
-  WITH_NV(d, ++g_launches; table_long_kernel<NV, tab_t><<<grid_for(maxl * 32, 256), 256, 0, st>>>(
-      table, state, d, skeys, w.seg_start, w.lfirst, w.lnslots, w.lseg, w.counters, w.partial, lr, beta, eps););
+  const long long nchunks = (n + CHUNK - 1) / CHUNK;
+  WITH_NV(d, ++g_launches; table_chunk_kernel<NV, tab_t><<<grid_for(nchunks * 32, 128), 128, 0, st>>>(
+      table, state, d, grad, skeys, perm, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
+  WITH_NV(d, ++g_launches; table_chain_kernel<NV, tab_t><<<grid_for(nchunks * 32, 256), 256, 0, st>>>(
+      table, state, d, skeys, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
   LAUNCH_CHECK();
   return GPT_OK;
 }
@@ -905,7 +907,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     if (b16) {
       // QKV projection with RoPE + QK-norm (+ value-table row) in its epilogue
       GemmEpilogue eq = epi(EPI_QKV, qkv, 3 * a);
-      eq.rope = m->at<float>(p.rope_cs);
+      eq.rope = m->at<float>(p.rope_cs_t);
       eq.rstd_q = m->at<float>(L.rstd_q);
       eq.rstd_k = m->at<float>(L.rstd_k);
       eq.hv = c.v_rows ? (const void*)(m->base + p.hv) : nullptr;
@@ -943,19 +945,22 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   // here while each logits chunk is live: dxf (fp32) and the pending head
   // weight gradient, which backward adds into the dense gradient.
   const act_t* Wlm = W(c.tie_embeddings ? "wte" : "lm_head");
-  float* logits = m->at<float>(p.logits);
+  float* logits = b16 ? nullptr : m->at<float>(p.logits);
   act_t* dz = m->at<act_t>(p.dz);
   for (int r0 = 0, ci = 0; r0 < N; r0 += p.chunk, ++ci) {
     const int rows = (N - r0 < p.chunk) ? (N - r0) : p.chunk;
     if (b16) {
-      GemmEpilogue el = epi(EPI_LOGITS, logits, V);
+      GemmEpilogue el = epi(EPI_LOGITS, dz, V);
       el.softcap = c.softcap;
       el.stats = m->at<float2>(p.ce_stats);
+      el.targets = targets + r0;
+      el.ztgt = m->at<float>(p.ce_ztgt);
       TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), el, false, "gemm.lm_fwd"));
-      ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * (4 + es));
-      ++g_launches; ce_stats_kernel<act_t><<<rows, 256, 0, st>>>(logits, m->at<float2>(p.ce_stats), cdiv(V, V >= 256 ? 256 : 128), dz,
-                                                   targets + r0, m->at<float>(p.tok_loss) + r0, V, c.softcap,
-                                                   m->at<float>(p.ce_scale), err);
+      ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * 4);
+      const int tcols = V >= 256 ? 256 : 128, ntl = cdiv(V, tcols);
+      ++g_launches; ce_prob_kernel<<<rows, 256, ntl * 4, st>>>(
+          reinterpret_cast<bf16*>(dz), m->at<float2>(p.ce_stats), ntl, tcols, targets + r0, m->at<float>(p.ce_ztgt),
+          m->at<float>(p.tok_loss) + r0, V, c.softcap, m->at<float>(p.ce_scale), err);
       LAUNCH_CHECK();
     } else {
       TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), epi(EPI_STORE_F32, logits, V), false,
@@ -1051,12 +1056,11 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const uint32_t* skeys;
     const int32_t* perm;
     TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
-    const long long maxp = (long long)N + N / PIECE + 2, maxl = N / PIECE + 2;
-    WITH_NV(d, ++g_launches; emb_piece_kernel<NV, act_t><<<grid_for(maxp * 32, 256), 256, 0, st>>>(
-        Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, w.pstart, w.plen, w.pslot,
-        w.counters, w.partial););
-    ++g_launches; emb_long_kernel<<<grid_for(maxl * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, w.seg_start, w.lfirst,
-                                                             w.lnslots, w.lseg, w.counters, w.partial);
+    const long long nchunks = (N + CHUNK - 1) / CHUNK;
+    WITH_NV(d, ++g_launches; emb_chunk_kernel<NV, act_t><<<grid_for(nchunks * 32, 256), 256, 0, st>>>(
+        Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, N, V, w.part_head, w.part_tail););
+    ++g_launches; emb_chain_kernel<<<grid_for(nchunks * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, N, V,
+                                                                               w.part_head, w.part_tail);
     LAUNCH_CHECK();
   }
   const float lr_t = lr * c.lr_mult_table;
@@ -1208,7 +1212,12 @@ extern "C" int ngram_gather(const int32_t* rows, int n, const void* table, long 
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
   const int grid = grid_for((long long)n * 32, 256);
-  if (dtype == GPT_DTYPE_BF16) {
+  const bool vec16 = d % 8 == 0 && (reinterpret_cast<uintptr_t>(table) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+  if (dtype == GPT_DTYPE_BF16 && vec16) {
+    ++g_launches; ngram_gather_bf16x8_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows,
+                                                                      d, (bf16*)out, accumulate, err);
+  } else if (dtype == GPT_DTYPE_BF16) {
     ++g_launches; ngram_gather_kernel<bf16><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows, d,
                                                                       (bf16*)out, accumulate, err);
   } else if (dtype == GPT_DTYPE_F32) {
@@ -1222,22 +1231,18 @@ extern "C" int ngram_gather(const int32_t* rows, int n, const void* table, long 
 }
 
 struct NgramWsPlan {
-  size_t ka, kb, va, vb, counts, seg_start, pstart, plen, pseg, pslot, lfirst, lnslots, lseg, counters, partial, total;
+  size_t ka, kb, va, vb, counts, part_head, part_tail, total;
 };
 
 static NgramWsPlan ngram_ws_plan(int n, int d) {
   NgramWsPlan w;
   Carver cv;
-  const long long nblk = (n + RADIX_TILE - 1) / RADIX_TILE;
-  const long long maxp = (long long)n + n / PIECE + 2, maxl = n / PIECE + 2, maxslots = 2 * (n / PIECE) + 4;
+  const long long nchunks = ((long long)n + CHUNK - 1) / CHUNK;
   w.ka = cv.take((size_t)n * 4); w.kb = cv.take((size_t)n * 4);
   w.va = cv.take((size_t)n * 4); w.vb = cv.take((size_t)n * 4);
-  w.counts = cv.take(256 * nblk * 4);
-  w.seg_start = cv.take(((size_t)n + 1) * 4);
-  w.pstart = cv.take(maxp * 4); w.plen = cv.take(maxp * 4); w.pseg = cv.take(maxp * 4); w.pslot = cv.take(maxp * 4);
-  w.lfirst = cv.take(maxl * 4); w.lnslots = cv.take(maxl * 4); w.lseg = cv.take(maxl * 4);
-  w.counters = cv.take(16);
-  w.partial = cv.take(maxslots * (size_t)d * 4);
+  w.counts = cv.take(256 * radix_blocks(n) * 4);
+  w.part_head = cv.take(nchunks * (size_t)d * 4);
+  w.part_tail = cv.take(nchunks * (size_t)d * 4);
   w.total = cv.take(0);
   return w;
 }
@@ -1269,10 +1274,7 @@ extern "C" int ngram_sparse_update(void* table, float* row_state, long long n_ro
   w.ka = (uint32_t*)(b + pl.ka); w.kb = (uint32_t*)(b + pl.kb);
   w.va = (int32_t*)(b + pl.va); w.vb = (int32_t*)(b + pl.vb);
   w.counts = (uint32_t*)(b + pl.counts);
-  w.seg_start = (int32_t*)(b + pl.seg_start); w.pstart = (int32_t*)(b + pl.pstart);
-  w.plen = (int32_t*)(b + pl.plen); w.pseg = (int32_t*)(b + pl.pseg); w.pslot = (int32_t*)(b + pl.pslot);
-  w.lfirst = (int32_t*)(b + pl.lfirst); w.lnslots = (int32_t*)(b + pl.lnslots); w.lseg = (int32_t*)(b + pl.lseg);
-  w.counters = (int32_t*)(b + pl.counters); w.partial = (float*)(b + pl.partial);
+  w.part_head = (float*)(b + pl.part_head); w.part_tail = (float*)(b + pl.part_tail);
   cudaStream_t st = (cudaStream_t)stream;
   // rows outside the table are rejected on the device before bucketing
   unsigned* err = nullptr;
@@ -1309,12 +1311,18 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
     return fail(GPT_ERR_ARG, "gptx_gemm_bf16: split-K only for fp32 outputs");
   if (splits > 1 && (!workspace || ws_bytes < (size_t)splits * M * N * 4))
     return fail(GPT_ERR_WORKSPACE, "gptx_gemm_bf16: split-K needs splits*M*N*4 bytes of workspace");
-  if (mode == EPI_LOGITS && (!workspace || ws_bytes < (size_t)M * cdiv(N, N >= 256 ? 256 : 128) * 8))
-    return fail(GPT_ERR_WORKSPACE, "gptx_gemm_bf16: logits need M*n_tiles*8 bytes of workspace for statistics");
+  const size_t stats_bytes = (size_t)M * cdiv(N, N >= 256 ? 256 : 128) * 8;
+  if (mode == EPI_LOGITS && (!workspace || ws_bytes < stats_bytes + (aux ? (size_t)M * 4 : 0)))
+    return fail(GPT_ERR_WORKSPACE,
+                "gptx_gemm_bf16: logits need M*n_tiles*8 bytes of workspace for statistics (+ M*4 with targets)");
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
-  GemmEpilogue e = epi(mode, C, ldc, beta, nullptr, aux);
-  if (mode == EPI_LOGITS) e.stats = (float2*)workspace;
+  GemmEpilogue e = epi(mode, C, ldc, beta, nullptr, mode == EPI_LOGITS ? nullptr : aux);
+  if (mode == EPI_LOGITS) {
+    e.stats = (float2*)workspace;
+    e.targets = (const int32_t*)aux;
+    e.ztgt = aux ? (float*)((uint8_t*)workspace + stats_bytes) : nullptr;
+  }
   GemmOperand a{A, lda, a_kmajor ? 1 : 0}, b{B, ldb, b_kmajor ? 1 : 0};
   GemmCtx g{true, (float*)workspace, (long long)(ws_bytes / 4), err, (cudaStream_t)stream, nullptr};
   if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);

@@ -131,7 +131,11 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __
 // RoPE cos/sin table: theta[t, i] = t * base^(-2i/hd) for i < hd/2
 // ("$1000 tier nanochat run", `_precompute_rotary_embeddings`), evaluated in
 // double precision and stored fp32 (the pages keep a bf16 table).
-__global__ void rope_table_kernel(float* __restrict__ cs, int T, int hd, double base) {
+// (cos, sin) of t * base^(-2j/hd) for every position t and frequency j < hd/2,
+// in two layouts: position-major cs[t][j] (one warp per position reads a
+// contiguous row) and frequency-major cs_t[j][t] (a warp over 32 consecutive
+// positions reads contiguous pairs, as the QKV GEMM epilogue does).
+__global__ void rope_table_kernel(float* __restrict__ cs, float* __restrict__ cs_t, int T, int hd, double base) {
   const int h = hd / 2;
   const long long total = (long long)T * h;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
@@ -139,8 +143,12 @@ __global__ void rope_table_kernel(float* __restrict__ cs, int T, int hd, double 
     const int t = (int)(i / h), j = (int)(i % h);
     const double inv_freq = 1.0 / pow(base, (2.0 * j) / hd);
     const double th = t * inv_freq;
-    cs[2 * i] = (float)cos(th);
-    cs[2 * i + 1] = (float)sin(th);
+    const float c = (float)cos(th), s = (float)sin(th);
+    cs[2 * i] = c;
+    cs[2 * i + 1] = s;
+    const long long it = (long long)j * T + t;
+    cs_t[2 * it] = c;
+    cs_t[2 * it + 1] = s;
   }
 }
 
@@ -297,21 +305,23 @@ __global__ void __launch_bounds__(512) ce_chunk_kernel(float* __restrict__ logit
   }
 }
 
-// The same loss and logit gradient for one row of a chunk whose GEMM epilogue
-// already folded each 256-column tile into (max, sum of exp(z - max)):
-// lse = M + log sum_j s_j exp(m_j - M) over the tiles, then one pass over the
-// row writes dz.  One block per row; V a multiple of 4.
-template <typename act_t>
-__global__ void __launch_bounds__(256) ce_stats_kernel(const float* __restrict__ logits,
-                                                       const float2* __restrict__ stats, int n_tiles,
-                                                       act_t* __restrict__ dz,
-                                                       const int32_t* __restrict__ targets,
-                                                       float* __restrict__ tok_loss, int V, float softcap,
-                                                       const float* __restrict__ scale_dev, unsigned* err) {
+// Cross-entropy from the logits GEMM's tile-local numerators (bf16 mode),
+// one block per row: lse = M + log sum_j s_j exp(m_j - M) over the row's
+// column tiles j (m_j tile max, s_j = sum exp(z - m_j), M = max m_j); loss =
+// lse - z[y]; and in place over the numerators e_c = exp(z_c - m_j):
+// dz_c = (e_c exp(m_j - lse) - [c == y]) * scale (* (1 - (z_c/cap)^2) with a
+// softcap, z_c recovered as m_j + log e_c).  ("$1000 tier nanochat run":
+// cross-entropy over softcapped logits; the chunking keeps logits bounded.)
+__global__ void __launch_bounds__(256) ce_prob_kernel(bf16* __restrict__ ez, const float2* __restrict__ stats,
+                                                      int n_tiles, int tile_cols,
+                                                      const int32_t* __restrict__ targets,
+                                                      const float* __restrict__ ztgt,
+                                                      float* __restrict__ tok_loss, int V, float softcap,
+                                                      const float* __restrict__ scale_dev, unsigned* err) {
+  extern __shared__ float fac[];  // exp(m_j - lse) per column tile
   __shared__ float sh[32];
   const long long row = blockIdx.x;
-  const float* z = logits + row * V;
-  act_t* g = dz + row * V;
+  bf16* g = ez + row * V;
   int y = targets[row];
   if (y < -1 || y >= V) {
     if (threadIdx.x == 0) set_error(err, GPT_EBIT_INPUT);
@@ -325,22 +335,53 @@ __global__ void __launch_bounds__(256) ce_stats_kernel(const float* __restrict__
   for (int j = threadIdx.x; j < n_tiles; j += blockDim.x) se += st[j].y * __expf(st[j].x - mx);
   se = block_sum(se, sh);
   const float lse = mx + logf(se);
+  for (int j = threadIdx.x; j < n_tiles; j += blockDim.x) fac[j] = __expf(st[j].x - lse);
   if (threadIdx.x == 0) {
-    const float l = (y >= 0) ? (lse - z[y]) : 0.f;
+    const float l = (y >= 0) ? (lse - ztgt[row]) : 0.f;
     tok_loss[row] = l;
     if (y >= 0 && !isfinite(l)) set_error(err, GPT_EBIT_NONFINITE);
   }
+  __syncthreads();
   const float sc = (y >= 0) ? *scale_dev : 0.f;
-  for (int i = threadIdx.x * 4; i < V; i += blockDim.x * 4) {
-    float v[4], o[4];
-    load4(z + i, v);
+  for (int i = threadIdx.x * 8; i < V; i += blockDim.x * 8) {
+    // 8 columns never straddle a tile (tile_cols is a multiple of 8)
+    const int j = i / tile_cols;
+    const float f = fac[j];
+    const int nv = min(8, V - i);
+    float e8[8];
+    if (nv == 8 && (V & 7) == 0) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(g + i);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float gi = (__expf(v[k] - lse) - (i + k == y ? 1.f : 0.f)) * sc;
-      if (softcap > 0.f) { const float tt = v[k] / softcap; gi *= (1.f - tt * tt); }
-      o[k] = gi;
+      for (int k = 0; k < 4; ++k) {
+        const float2 t = __bfloat1622float2(h[k]);
+        e8[2 * k] = t.x;
+        e8[2 * k + 1] = t.y;
+      }
+    } else {
+      for (int k = 0; k < 8; ++k) e8[k] = k < nv ? __bfloat162float(g[i + k]) : 0.f;
     }
-    store4(g + i, o);
+    float o[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o[k] = (e8[k] * f - (i + k == y ? 1.f : 0.f)) * sc;
+    if (softcap > 0.f) {  // block-uniform: the default path skips all of this
+      const float inv = 1.f / softcap;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        // z = m_j + log e (e = 0: p = 0 and dz = 0 off the target anyway)
+        const float tt = (i + k == y) ? ztgt[row] * inv : (e8[k] > 0.f ? (st[j].x + __logf(e8[k])) * inv : 1.f);
+        o[k] *= (1.f - tt * tt);
+      }
+    }
+    if (nv == 8 && (V & 7) == 0) {
+      uint4 raw;
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) h[k] = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
+      *reinterpret_cast<uint4*>(g + i) = raw;
+    } else {
+      for (int k = 0; k < nv; ++k) g[i + k] = __float2bfloat16_rn(o[k]);
+    }
   }
 }
 

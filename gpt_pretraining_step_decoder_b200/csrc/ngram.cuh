@@ -5,21 +5,38 @@
 // and only per-row magnitude").
 //
 // Bucketing: positions are sorted by row with a stable LSD radix sort (8-bit
-// digits; per-tile histograms, one exclusive scan, stable scatter ranked with
-// warp match masks) -- no atomics anywhere, so sums are formed in position
-// order and results are bit-reproducible.  Runs of equal rows (segments) are
-// cut into pieces of at most PIECE positions; one warp sums one piece.  A
-// segment that fits in one piece is finished by that warp (sum -> mean square
-// -> row state -> row update); longer segments write per-piece partial sums
-// that a second pass adds in piece order before updating the row.
+// digits, two launches a digit: per-tile histograms, then a stable scatter
+// whose blocks derive their own global offsets from the histograms and rank
+// equal digits with warp match masks).  The first pass reads the caller's
+// int32 rows directly.  No atomics anywhere, so sums are formed in position
+// order and results are bit-reproducible.
+//
+// Update: the sorted positions are cut into fixed chunks of 32; one warp owns
+// a chunk and finds the runs of equal rows in it with ballots.  A run that
+// lies inside the chunk is finished by that warp (sum -> mean square -> row
+// state -> row update).  A run that crosses chunk boundaries leaves one
+// partial sum per chunk it touches; a second launch adds those partials in
+// chunk order and finishes the row.  Every row is written by exactly one warp.
 #pragma once
 #include "common.cuh"
 #include "layers.cuh"
 
 constexpr int RADIX_THREADS = 256;
-constexpr int RADIX_ITEMS = 8;
-constexpr int RADIX_TILE = RADIX_THREADS * RADIX_ITEMS;  // 2048 keys per block
-constexpr int PIECE = 32;                                // positions per warp task
+constexpr int RADIX_MAX_ITEMS = 8;   // keys per thread per block, at most
+constexpr int RADIX_FUSED_MAX_BLOCKS = 256;  // above this, offsets come from a scan launch
+constexpr int CHUNK = 32;            // sorted positions per warp in the update
+
+// keys per thread so that a sort of n keys runs on about 96 blocks (or on
+// as many 2048-key tiles as it needs beyond that)
+static inline int radix_items(long long n) {
+  int it = 1;
+  while (it < RADIX_MAX_ITEMS && (n + (long long)RADIX_THREADS * it - 1) / ((long long)RADIX_THREADS * it) > 96) it <<= 1;
+  return it;
+}
+static inline long long radix_blocks(long long n) {
+  const long long tile = (long long)RADIX_THREADS * radix_items(n);
+  return (n + tile - 1) / tile;
+}
 
 // ---------------------------------------------------------------- hash
 // key = (a*p1 mod 2^64) XOR (c*p2 mod 2^64), a = tokens[t-1] (vocab at t = 0)
@@ -66,22 +83,74 @@ __global__ void ngram_gather_kernel(const int32_t* __restrict__ rows, int n,
   }
 }
 
+
+// bf16 rows with d % 8 == 0 and 16-byte aligned buffers: 16-byte accesses
+// (8 values per lane), the row copied as raw bits unless accumulating.
+__global__ void ngram_gather_bf16x8_kernel(const int32_t* __restrict__ rows, int n,
+                                           const bf16* __restrict__ table, long long n_rows, int d,
+                                           bf16* __restrict__ out, int accumulate, unsigned* err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= n) return;
+  const long long r = rows[warp];
+  if (r < 0 || r >= n_rows) {
+    if (lane == 0) set_error(err, GPT_EBIT_INPUT);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(table + r * d);
+  uint4* dst = reinterpret_cast<uint4*>(out + (long long)warp * d);
+#pragma unroll 4
+  for (int c = lane; c < d / 8; c += 32) {
+    uint4 v = __ldg(src + c);
+    if (accumulate) {
+      const uint4 o = dst[c];
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+      uint4 s;
+      __nv_bfloat162* s2 = reinterpret_cast<__nv_bfloat162*>(&s);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(a2[i]), y = __bfloat1622float2(o2[i]);
+        s2[i] = __floats2bfloat162_rn(x.x + y.x, x.y + y.y);
+      }
+      v = s;
+    }
+    dst[c] = v;
+  }
+}
+
 // ---------------------------------------------------------------- radix sort
-// counts layout: digit-major [256][nblocks] so one exclusive scan gives every
-// (digit, block) its stable global offset.
+// Keys are row ids in [0, key_range).  The first pass reads the caller's
+// int32 rows; an id outside the range sets the error word and is sorted as
+// key_range itself with position -1.  Those form one run past every real
+// row, which every consumer skips, so no out-of-range row is ever read or
+// written.  (The digit passes therefore cover the value key_range.)
+__device__ __forceinline__ uint32_t radix_key(const uint32_t* __restrict__ keys, const int32_t* __restrict__ raw,
+                                              long long idx, long long key_range, bool& ok) {
+  if (raw == nullptr) { ok = true; return keys[idx]; }
+  const int32_t k = raw[idx];
+  ok = k >= 0 && (long long)k < key_range;
+  return ok ? (uint32_t)k : (uint32_t)key_range;
+}
+
+// counts layout: block-major [nblocks][256]
 __global__ void __launch_bounds__(RADIX_THREADS) radix_hist_kernel(const uint32_t* __restrict__ keys,
-                                                                  int n, int shift,
+                                                                  const int32_t* __restrict__ raw, int n,
+                                                                  long long key_range, int items, int shift,
                                                                   uint32_t* __restrict__ counts) {
   constexpr int NW = RADIX_THREADS / 32;
   __shared__ uint32_t wh[NW][256];  // per-warp digit counts
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < NW * 256; i += RADIX_THREADS) (&wh[0][0])[i] = 0;
   __syncthreads();
-  const int base = blockIdx.x * RADIX_TILE;
+  const long long base = (long long)blockIdx.x * RADIX_THREADS * items;
   const uint32_t lt = (1u << lane) - 1u;
-  for (int round = 0; round < RADIX_ITEMS; ++round) {
-    const int idx = base + round * RADIX_THREADS + threadIdx.x;
-    const uint32_t dgt = (idx < n) ? ((keys[idx] >> shift) & 255u) : 256u;
+  for (int round = 0; round < items; ++round) {
+    const long long idx = base + (long long)round * RADIX_THREADS + threadIdx.x;
+    uint32_t dgt = 256u;
+    if (idx < n) {
+      bool ok;
+      dgt = (radix_key(keys, raw, idx, key_range, ok) >> shift) & 255u;
+    }
     const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
     // the lowest lane of each digit group adds the group's size: one writer
     // per (warp, digit), so no atomics are needed
@@ -91,60 +160,99 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_hist_kernel(const uint32_
   __syncthreads();
   uint32_t s = 0;
   for (int ww = 0; ww < NW; ++ww) s += wh[ww][threadIdx.x];
-  counts[(long long)threadIdx.x * gridDim.x + blockIdx.x] = s;
+  counts[(long long)blockIdx.x * 256 + threadIdx.x] = s;
 }
 
-// Exclusive scan of `n` counters in one block (sequential chunks + block scan).
-__global__ void __launch_bounds__(1024) exclusive_scan_kernel(uint32_t* __restrict__ data, int n) {
+// For many blocks: replace every count by its stable global offset (the
+// exclusive scan of the counts taken digit-major: all blocks of digit 0, then
+// digit 1, ...).  One block; each thread scans a contiguous stretch.
+__global__ void __launch_bounds__(1024) radix_offsets_kernel(uint32_t* __restrict__ counts, int nblk) {
   __shared__ uint32_t sh[1024];
-  const int per = (n + 1023) / 1024;
-  const int beg = threadIdx.x * per, end = min(beg + per, n);
+  const long long n = 256LL * nblk;
+  const long long per = (n + 1023) / 1024;
+  const long long beg = threadIdx.x * per, end = beg + per < n ? beg + per : n;
   uint32_t local = 0;
-  for (int i = beg; i < end; ++i) local += data[i];
+  for (long long i = beg; i < end; ++i) local += counts[(i % nblk) * 256 + i / nblk];
   sh[threadIdx.x] = local;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {
-    uint32_t v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
+    const uint32_t v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
     __syncthreads();
     sh[threadIdx.x] += v;
     __syncthreads();
   }
   uint32_t run = sh[threadIdx.x] - local;
-  for (int i = beg; i < end; ++i) {
-    const uint32_t v = data[i];
-    data[i] = run;
+  for (long long i = beg; i < end; ++i) {
+    uint32_t& c = counts[(i % nblk) * 256 + i / nblk];
+    const uint32_t v = c;
+    c = run;
     run += v;
   }
 }
 
-// Stable scatter: element order within a tile is idx = base + round*256 + tid;
-// ranks among equal digits follow that order (warp match masks inside a warp,
-// per-warp digit counts across warps, running totals across rounds).
+// Stable scatter.  Element order within a tile is idx = base + round*256 +
+// tid; ranks among equal digits follow that order (warp match masks inside a
+// warp, per-warp digit counts across warps, running totals across rounds).
+// With `scanned` == 0 each block first derives its global offsets from the
+// histograms: offset(digit, b) = sum of all blocks' counts of smaller digits
+// + sum of counts of this digit in blocks before b.
 __global__ void __launch_bounds__(RADIX_THREADS) radix_scatter_kernel(
-    const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, int n, int shift,
-    const uint32_t* __restrict__ offsets, uint32_t* __restrict__ keys_out,
-    int32_t* __restrict__ vals_out) {
+    const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, const int32_t* __restrict__ raw,
+    int n, long long key_range, int items, int shift, const uint32_t* __restrict__ counts, int scanned,
+    uint32_t* __restrict__ keys_out, int32_t* __restrict__ vals_out, unsigned* err) {
   constexpr int NW = RADIX_THREADS / 32;
   __shared__ uint32_t wcount[NW][256];
   __shared__ uint32_t running[256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  running[threadIdx.x] = offsets[(long long)threadIdx.x * gridDim.x + blockIdx.x];
-  const int base = blockIdx.x * RADIX_TILE;
-  for (int round = 0; round < RADIX_ITEMS; ++round) {
+  if (scanned) {
+    running[threadIdx.x] = counts[(long long)blockIdx.x * 256 + threadIdx.x];
+  } else {
+    uint32_t total = 0, before = 0;
+    for (int b = 0; b < (int)gridDim.x; ++b) {
+      const uint32_t c = counts[(long long)b * 256 + threadIdx.x];
+      total += c;
+      if (b < (int)blockIdx.x) before += c;
+    }
+    // exclusive scan of the per-digit totals over the 256 threads
+    uint32_t incl = total;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) wcount[0][w] = incl;
+    __syncthreads();
+    uint32_t wbase = 0;
+    for (int ww = 0; ww < w; ++ww) wbase += wcount[0][ww];
+    running[threadIdx.x] = wbase + incl - total + before;
+  }
+  const long long base = (long long)blockIdx.x * RADIX_THREADS * items;
+  for (int round = 0; round < items; ++round) {
+    __syncthreads();
     for (int i = threadIdx.x; i < NW * 256; i += RADIX_THREADS) (&wcount[0][0])[i] = 0;
     __syncthreads();
-    const int idx = base + round * RADIX_THREADS + threadIdx.x;
+    const long long idx = base + (long long)round * RADIX_THREADS + threadIdx.x;
     const bool valid = idx < n;
     uint32_t key = 0, dgt = 256;  // 256 = no digit (invalid lane)
     int32_t val = 0;
-    if (valid) { key = keys_in[idx]; val = vals_in[idx]; dgt = (key >> shift) & 255u; }
+    if (valid) {
+      bool ok;
+      key = radix_key(keys_in, raw, idx, key_range, ok);
+      if (raw != nullptr) {
+        val = ok ? (int32_t)idx : -1;
+        if (!ok) set_error(err, GPT_EBIT_INPUT);
+      } else {
+        val = vals_in[idx];
+      }
+      dgt = (key >> shift) & 255u;
+    }
     const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t rank_in_warp = __popc(peers & lt);
     if (valid && rank_in_warp == 0) wcount[w][dgt] = __popc(peers);
     __syncthreads();
-    uint32_t before = 0;
     if (valid) {
+      uint32_t before = 0;
       for (int ww = 0; ww < w; ++ww) before += wcount[ww][dgt];
       const uint32_t pos = running[dgt] + before + rank_in_warp;
       keys_out[pos] = key;
@@ -156,142 +264,134 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_scatter_kernel(
       for (int ww = 0; ww < NW; ++ww) tot += wcount[ww][threadIdx.x];
       running[threadIdx.x] += tot;
     }
-    __syncthreads();
   }
 }
 
-// Sort input: (key, position).  Keys outside [0, key_range) set the error
-// word; they are sorted as key_range - 1 with position -1, which every
-// consumer skips, so no out-of-range row is ever read or written.
-__global__ void iota_kernel(const int32_t* __restrict__ keys_in, uint32_t* __restrict__ keys,
-                            int32_t* __restrict__ vals, int n, long long key_range, unsigned* err) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int32_t k = keys_in[i];
-  if (k < 0 || (long long)k >= key_range) {
-    set_error(err, GPT_EBIT_INPUT);
-    keys[i] = (uint32_t)(key_range - 1);
-    vals[i] = -1;
-  } else {
-    keys[i] = (uint32_t)k;
-    vals[i] = i;
-  }
-}
-
-// ---------------------------------------------------------------- segments
-// From sorted keys, build (single block):
-//   pieces: pstart[p], plen[p], pseg[p], pslot[p] (-1: the piece is a whole
-//           segment; else its partial-sum slot)
-//   long segments: lseg_first_slot[s], lseg_nslots[s], lseg_key[s]
-//   counters[0] = #pieces, counters[1] = #long segments, counters[2] = #segments
-// and (optionally) the distinct keys in ascending order.
-__global__ void __launch_bounds__(1024) segments_kernel(
-    const uint32_t* __restrict__ skeys, int n, int32_t* __restrict__ seg_start /* [n+1] */,
-    int32_t* __restrict__ pstart, int32_t* __restrict__ plen, int32_t* __restrict__ pseg,
-    int32_t* __restrict__ pslot, int32_t* __restrict__ lseg_first_slot,
-    int32_t* __restrict__ lseg_nslots, int32_t* __restrict__ lseg_seg, int32_t* __restrict__ counters,
-    int32_t* __restrict__ uniq_out, int* __restrict__ n_uniq_out) {
+// Distinct sorted keys in ascending order and their number (one block; only
+// for callers that ask for the updated-row list).
+__global__ void __launch_bounds__(1024) unique_keys_kernel(const uint32_t* __restrict__ skeys, int n,
+                                                           long long key_range, int32_t* __restrict__ uniq_out,
+                                                           int* __restrict__ n_uniq_out) {
   __shared__ int sh[1024];
   const int per = (n + 1023) / 1024;
   const int beg = threadIdx.x * per, end = min(beg + per, n);
-  // pass 1: segment heads
   int heads = 0;
-  for (int i = beg; i < end; ++i) heads += (i == 0 || skeys[i] != skeys[i - 1]);
+  for (int i = beg; i < end; ++i) heads += ((i == 0 || skeys[i] != skeys[i - 1]) && skeys[i] < key_range);
   sh[threadIdx.x] = heads;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {
-    int v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
+    const int v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
     __syncthreads();
     sh[threadIdx.x] += v;
     __syncthreads();
   }
   int sid = sh[threadIdx.x] - heads;
-  const int U = sh[1023];
-  for (int i = beg; i < end; ++i) {
-    if (i == 0 || skeys[i] != skeys[i - 1]) {
-      seg_start[sid] = i;
-      if (uniq_out) uniq_out[sid] = (int32_t)skeys[i];
-      ++sid;
-    }
+  if (uniq_out)
+    for (int i = beg; i < end; ++i)
+      if ((i == 0 || skeys[i] != skeys[i - 1]) && skeys[i] < key_range) uniq_out[sid++] = (int32_t)skeys[i];
+  if (threadIdx.x == 1023 && n_uniq_out) *n_uniq_out = sh[1023];
+}
+
+// ---------------------------------------------------------------- runs in a chunk
+// One warp, chunk c = sorted positions [32c, 32c + len).  Lane l holds the
+// l-th key and position.  start_mask / end_mask mark the lanes where a run of
+// equal keys starts / ends inside the chunk (lane 0 always starts one, lane
+// len-1 always ends one); cont_in: the chunk's first run began in an earlier
+// chunk; cont_out: its last run goes on into the next chunk.
+struct ChunkRuns {
+  uint32_t key;
+  int32_t pos;
+  unsigned start_mask, end_mask;
+  int len;
+  bool cont_in, cont_out;
+};
+
+__device__ __forceinline__ ChunkRuns chunk_runs(const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm,
+                                                int n, int c) {
+  const int lane = threadIdx.x & 31;
+  const long long base = (long long)c * CHUNK;
+  ChunkRuns r;
+  r.len = (int)min((long long)CHUNK, n - base);
+  const bool valid = lane < r.len;
+  r.key = valid ? skeys[base + lane] : 0xffffffffu;
+  r.pos = valid ? perm[base + lane] : -1;
+  const uint32_t up = __shfl_up_sync(0xffffffffu, r.key, 1);
+  const uint32_t dn = __shfl_down_sync(0xffffffffu, r.key, 1);
+  r.start_mask = __ballot_sync(0xffffffffu, valid && (lane == 0 || up != r.key));
+  r.end_mask = __ballot_sync(0xffffffffu, valid && (lane == r.len - 1 || dn != r.key));
+  const uint32_t first = __shfl_sync(0xffffffffu, r.key, 0);
+  const uint32_t last = __shfl_sync(0xffffffffu, r.key, r.len - 1);
+  r.cont_in = c > 0 && skeys[base - 1] == first;
+  r.cont_out = base + CHUNK < n && skeys[base + CHUNK] == last;
+  return r;
+}
+
+// What the warp does with the run that ends at lane q.
+enum RunKind { RUN_WHOLE = 0, RUN_TAIL = 1, RUN_HEAD = 2 };
+__device__ __forceinline__ int run_kind(const ChunkRuns& r, int q) {
+  const unsigned upto = (q == 31) ? 0xffffffffu : ((2u << q) - 1u);
+  const int s = 31 - __clz(r.start_mask & upto);
+  if (s == 0 && r.cont_in) return RUN_TAIL;             // continues a run from before
+  if (q == r.len - 1 && r.cont_out) return RUN_HEAD;    // starts a run that goes on
+  return RUN_WHOLE;
+}
+
+// Chunk c starts a run that goes on into later chunks: returns its key and
+// the last chunk it reaches, else false.
+__device__ __forceinline__ bool chained_run(const uint32_t* __restrict__ skeys, int n, int c, uint32_t& key,
+                                            int& last_chunk) {
+  const long long base = (long long)c * CHUNK;
+  if (base + CHUNK >= n) return false;
+  key = skeys[base + CHUNK - 1];
+  if (skeys[base + CHUNK] != key) return false;
+  if (c > 0 && skeys[base - 1] == key) return false;
+  int cc = c + 1;
+  while ((long long)cc * CHUNK + CHUNK < n && skeys[(long long)cc * CHUNK + CHUNK] == key) ++cc;
+  last_chunk = cc;
+  return true;
+}
+
+// Four table values per lane in their storage type (8 bytes for bf16), so a
+// prefetched row costs half the registers of its fp32 copy.
+template <typename T> struct Raw4;
+template <> struct Raw4<float> {
+  using type = float4;
+  static __device__ __forceinline__ void unpack(const type& r, float v[4]) { v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w; }
+  static __device__ __forceinline__ type pack(const float v[4]) { return make_float4(v[0], v[1], v[2], v[3]); }
+};
+template <> struct Raw4<bf16> {
+  using type = uint2;
+  static __device__ __forceinline__ void unpack(const type& r, float v[4]) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) seg_start[U] = n;
-  __syncthreads();
-  // pass 2: pieces per segment, partial slots for long segments
-  const int sper = (U + 1023) / 1024;
-  const int sbeg = threadIdx.x * sper, send = min(sbeg + sper, U);
-  int np = 0, nslot = 0, nlong = 0;
-  for (int s = sbeg; s < send; ++s) {
-    const int len = seg_start[s + 1] - seg_start[s];
-    const int k = (len + PIECE - 1) / PIECE;
-    np += k;
-    if (k > 1) { nslot += k; ++nlong; }
+  static __device__ __forceinline__ type pack(const float v[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
   }
-  __syncthreads();
-  sh[threadIdx.x] = np;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    int v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
-    __syncthreads();
-    sh[threadIdx.x] += v;
-    __syncthreads();
-  }
-  int p = sh[threadIdx.x] - np;
-  const int NP = sh[1023];
-  __syncthreads();
-  sh[threadIdx.x] = (nslot << 0);
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    int v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
-    __syncthreads();
-    sh[threadIdx.x] += v;
-    __syncthreads();
-  }
-  int slot = sh[threadIdx.x] - nslot;
-  __syncthreads();
-  sh[threadIdx.x] = nlong;
-  __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
-    int v = (threadIdx.x >= off) ? sh[threadIdx.x - off] : 0;
-    __syncthreads();
-    sh[threadIdx.x] += v;
-    __syncthreads();
-  }
-  int ls = sh[threadIdx.x] - nlong;
-  const int NL = sh[1023];
-  for (int s = sbeg; s < send; ++s) {
-    const int st = seg_start[s], len = seg_start[s + 1] - st;
-    const int k = (len + PIECE - 1) / PIECE;
-    if (k > 1) {
-      lseg_first_slot[ls] = slot;
-      lseg_nslots[ls] = k;
-      lseg_seg[ls] = s;
-      ++ls;
-    }
-    for (int j = 0; j < k; ++j) {
-      pstart[p] = st + j * PIECE;
-      plen[p] = min(PIECE, len - j * PIECE);
-      pseg[p] = s;
-      pslot[p] = (k > 1) ? slot + j : -1;
-      ++p;
-    }
-    if (k > 1) slot += k;
-  }
-  if (threadIdx.x == 0) {
-    counters[0] = NP;
-    counters[1] = NL;
-    counters[2] = U;
-    if (n_uniq_out) *n_uniq_out = U;
+};
+
+template <int NV, typename T>
+__device__ __forceinline__ void load_raw_row(const T* __restrict__ src, int d, typename Raw4<T>::type (&v)[NV]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) v[j] = *reinterpret_cast<const typename Raw4<T>::type*>(src + c);
   }
 }
 
 // ---------------------------------------------------------------- row update
 // Apply the per-row-magnitude step to one row with its summed gradient G
-// (held by the warp, 4 values per lane per chunk).
+// (held by the warp, 4 values per lane per 128 columns): m = mean(G^2),
+// s <- beta*s + (1-beta)*m, W <- W - lr*G/(sqrt(s) + eps).  w holds the old
+// row, s_old the old state.
 template <int NV, typename tab_t>
-__device__ __forceinline__ void table_row_update(tab_t* __restrict__ table, float* __restrict__ state,
-                                                 long long r, int d, const float (&G)[NV][4],
-                                                 float lr, float beta, float eps) {
+__device__ __forceinline__ void table_row_apply(tab_t* __restrict__ table, float* __restrict__ state,
+                                                long long r, int d, const float (&G)[NV][4],
+                                                const typename Raw4<tab_t>::type (&w)[NV], float s_old,
+                                                float lr, float beta, float eps) {
   const int lane = threadIdx.x & 31;
   float ss = 0.f;
 #pragma unroll
@@ -300,97 +400,157 @@ __device__ __forceinline__ void table_row_update(tab_t* __restrict__ table, floa
     if (c < d) ss += G[j][0] * G[j][0] + G[j][1] * G[j][1] + G[j][2] * G[j][2] + G[j][3] * G[j][3];
   }
   ss = warp_sum(ss);
-  const float s_new = beta * state[r] + (1.f - beta) * (ss / d);
+  const float s_new = beta * s_old + (1.f - beta) * (ss / d);
   const float step = lr / (sqrtf(s_new) + eps);
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
-      float w[4];
-      load4(table + r * d + c, w);
+      float x[4];
+      Raw4<tab_t>::unpack(w[j], x);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] -= step * G[j][i];
-      store4(table + r * d + c, w);
+      for (int i = 0; i < 4; ++i) x[i] -= step * G[j][i];
+      *reinterpret_cast<typename Raw4<tab_t>::type*>(table + r * d + c) = Raw4<tab_t>::pack(x);
     }
   }
-  __syncwarp();
   if (lane == 0) state[r] = s_new;
 }
 
-// Sum the gradient rows of one piece (in sorted = position order).
-template <int NV>
-__device__ __forceinline__ void piece_sum(const float* __restrict__ grad, const int32_t* __restrict__ perm,
-                                          int st, int len, int d, float (&G)[NV][4]) {
+template <int NV, typename T>
+__device__ __forceinline__ void load_row(const T* __restrict__ src, int d, float (&v)[NV][4]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int j = 0; j < NV; ++j) G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
-  for (int q = 0; q < len; ++q) {
-    const long long pos = perm[st + q];
-    if (pos < 0) continue;
+  for (int j = 0; j < NV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) load4(src + c, v[j]);
+    else v[j][0] = v[j][1] = v[j][2] = v[j][3] = 0.f;
+  }
+}
+
+template <int NV>
+__device__ __forceinline__ void store_row(float* __restrict__ dst, int d, const float (&v)[NV][4]) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (j * 32 + lane) * 4;
-      if (c < d) {
-        float g[4];
-        load4(grad + pos * d + c, g);
-        G[j][0] += g[0]; G[j][1] += g[1]; G[j][2] += g[2]; G[j][3] += g[3];
+  for (int j = 0; j < NV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) store4(dst + c, v[j]);
+  }
+}
+
+template <int NV>
+__device__ __forceinline__ void zero_row(float (&v)[NV][4]) {
+#pragma unroll
+  for (int j = 0; j < NV; ++j) v[j][0] = v[j][1] = v[j][2] = v[j][3] = 0.f;
+}
+
+template <int NV>
+__device__ __forceinline__ void add_row(float (&a)[NV][4], const float (&b)[NV][4]) {
+#pragma unroll
+  for (int j = 0; j < NV; ++j)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[j][i] += b[j][i];
+}
+
+// Up to two sorted positions per step: their gradient rows, and (for runs
+// that end there and finish in this chunk) the table row and state, are
+// loaded before any of them is used, so each warp keeps several row loads in
+// flight.  Wide rows (more than 768 columns) take one position per step to
+// stay within registers.
+template <int NV>
+struct TabU {
+  static constexpr int value = NV <= 6 ? 2 : 1;
+};
+
+// One warp per chunk of sorted positions: runs inside the chunk are summed
+// and applied; a run's part that touches a chunk boundary goes to part_tail[c]
+// (the chunk's first run, begun earlier) or part_head[c] (its last run, going
+// on).
+template <int NV, typename tab_t>
+__global__ void __launch_bounds__(128, 3) table_chunk_kernel(
+    tab_t* __restrict__ table, float* __restrict__ state, int d, const float* __restrict__ grad,
+    const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n, long long n_rows,
+    float* __restrict__ part_head, float* __restrict__ part_tail, float lr, float beta, float eps) {
+  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if ((long long)c * CHUNK >= n) return;
+  constexpr int TAB_U = TabU<NV>::value;
+  const ChunkRuns r = chunk_runs(skeys, perm, n, c);
+  float G[NV][4];
+  zero_row<NV>(G);
+  for (int q0 = 0; q0 < r.len; q0 += TAB_U) {
+    float g[TAB_U][NV][4], s_old[TAB_U];
+    typename Raw4<tab_t>::type w[TAB_U][NV];
+    int kind[TAB_U];
+    bool ends[TAB_U];
+    uint32_t key[TAB_U];
+#pragma unroll
+    for (int u = 0; u < TAB_U; ++u) {
+      const int q = q0 + u;
+      const bool in = q < r.len;
+      const int qs = in ? q : r.len - 1;
+      const int p = __shfl_sync(0xffffffffu, r.pos, qs);
+      key[u] = __shfl_sync(0xffffffffu, r.key, qs);
+      ends[u] = in && ((r.end_mask >> q) & 1u);
+      kind[u] = ends[u] ? run_kind(r, q) : RUN_WHOLE;
+      if (in && p >= 0) load_row<NV>(grad + (long long)p * d, d, g[u]);
+      else zero_row<NV>(g[u]);
+      s_old[u] = 0.f;
+      if (ends[u] && kind[u] == RUN_WHOLE && key[u] < n_rows) {
+        load_raw_row<NV>(table + (long long)key[u] * d, d, w[u]);
+        s_old[u] = state[key[u]];
       }
+    }
+#pragma unroll
+    for (int u = 0; u < TAB_U; ++u) {
+      add_row<NV>(G, g[u]);
+      if (!ends[u]) continue;
+      if (kind[u] == RUN_WHOLE) {
+        // the run of invalid ids (key n_rows) touches nothing
+        if (key[u] < n_rows) table_row_apply<NV>(table, state, key[u], d, G, w[u], s_old[u], lr, beta, eps);
+      } else {
+        store_row<NV>((kind[u] == RUN_TAIL ? part_tail : part_head) + (long long)c * d, d, G);
+      }
+      zero_row<NV>(G);
     }
   }
 }
 
-// One warp per piece: whole segments are updated directly; pieces of long
-// segments store their partial sums.
-template <int NV, typename tab_t>
-__global__ void table_piece_kernel(tab_t* __restrict__ table, float* __restrict__ state, int d,
-                                   const float* __restrict__ grad, const uint32_t* __restrict__ skeys,
-                                   const int32_t* __restrict__ perm, const int32_t* __restrict__ pstart,
-                                   const int32_t* __restrict__ plen, const int32_t* __restrict__ pslot,
-                                   const int32_t* __restrict__ counters, float* __restrict__ partial,
-                                   float lr, float beta, float eps) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= counters[0]) return;
-  const int st = pstart[warp], len = plen[warp], slot = pslot[warp];
-  float G[NV][4];
-  piece_sum<NV>(grad, perm, st, len, d, G);
-  if (slot < 0) {
-    table_row_update<NV>(table, state, (long long)skeys[st], d, G, lr, beta, eps);
-  } else {
+// G += part_tail[first..last] in chunk order; several rows are loaded before
+// any is added, so a long run's partials stream instead of queueing one by one.
+template <int NV>
+__device__ __forceinline__ void chain_sum(const float* __restrict__ part_tail, int d, int first, int last,
+                                          float (&G)[NV][4]) {
+  constexpr int CHAIN_U = NV <= 6 ? 4 : (NV <= 8 ? 2 : 1);
+  for (int cc = first; cc <= last; cc += CHAIN_U) {
+    float t[CHAIN_U][NV][4];
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (j * 32 + lane) * 4;
-      if (c < d) store4(partial + (long long)slot * d + c, G[j]);
+    for (int u = 0; u < CHAIN_U; ++u) {
+      if (cc + u <= last) load_row<NV>(part_tail + (long long)(cc + u) * d, d, t[u]);
+      else zero_row<NV>(t[u]);
     }
+#pragma unroll
+    for (int u = 0; u < CHAIN_U; ++u)
+      if (cc + u <= last) add_row<NV>(G, t[u]);
   }
 }
 
-// One warp per long segment: add its partial sums in piece order, update.
+// One warp per chunk that starts a run going on into later chunks: its head
+// partial plus the tail partials of the chunks it reaches, in chunk order.
 template <int NV, typename tab_t>
-__global__ void table_long_kernel(tab_t* __restrict__ table, float* __restrict__ state, int d,
-                                  const uint32_t* __restrict__ skeys, const int32_t* __restrict__ seg_start,
-                                  const int32_t* __restrict__ lseg_first_slot,
-                                  const int32_t* __restrict__ lseg_nslots, const int32_t* __restrict__ lseg_seg,
-                                  const int32_t* __restrict__ counters, const float* __restrict__ partial,
-                                  float lr, float beta, float eps) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= counters[1]) return;
-  const int first = lseg_first_slot[warp], k = lseg_nslots[warp];
-  const long long r = skeys[seg_start[lseg_seg[warp]]];
+__global__ void __launch_bounds__(256) table_chain_kernel(
+    tab_t* __restrict__ table, float* __restrict__ state, int d, const uint32_t* __restrict__ skeys, int n,
+    long long n_rows, const float* __restrict__ part_head, const float* __restrict__ part_tail, float lr,
+    float beta, float eps) {
+  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if ((long long)c * CHUNK >= n) return;
+  uint32_t key;
+  int last;
+  if (!chained_run(skeys, n, c, key, last) || key >= n_rows) return;
   float G[NV][4];
-#pragma unroll
-  for (int j = 0; j < NV; ++j) G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
-  for (int q = 0; q < k; ++q) {
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (j * 32 + lane) * 4;
-      if (c < d) {
-        float g[4];
-        load4(partial + (long long)(first + q) * d + c, g);
-        G[j][0] += g[0]; G[j][1] += g[1]; G[j][2] += g[2]; G[j][3] += g[3];
-      }
-    }
-  }
-  table_row_update<NV>(table, state, r, d, G, lr, beta, eps);
+  load_row<NV>(part_head + (long long)c * d, d, G);
+  chain_sum<NV>(part_tail, d, c + 1, last, G);
+  typename Raw4<tab_t>::type w[NV];
+  load_raw_row<NV>(table + (long long)key * d, d, w);
+  table_row_apply<NV>(table, state, key, d, G, w, state[key], lr, beta, eps);
 }
 
 // ---------------------------------------------------------------- embedding grad
@@ -399,89 +559,110 @@ __global__ void table_long_kernel(tab_t* __restrict__ table, float* __restrict__
 // token id over its positions (same bucketing as the tables) and added to
 // the fp32 gradient dwte.
 template <int NV, typename w_t>
-__device__ __forceinline__ void emb_piece_sum(const float* __restrict__ dx0, const w_t* __restrict__ wte,
-                                              const float* __restrict__ rstd, const int32_t* __restrict__ perm,
-                                              long long row, int st, int len, int d, float (&G)[NV][4]) {
-  const int lane = threadIdx.x & 31;
-  float e[NV][4];
-#pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    G[j][0] = G[j][1] = G[j][2] = G[j][3] = 0.f;
-    const int c = (j * 32 + lane) * 4;
-    if (c < d) load4(wte + row * d + c, e[j]);
-  }
-  for (int q = 0; q < len; ++q) {
-    const long long pos = perm[st + q];
-    if (pos < 0) continue;
-    const float r = rstd[pos];
-    float g[NV][4];
-    float dot = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (j * 32 + lane) * 4;
-      if (c < d) {
-        load4(dx0 + pos * d + c, g[j]);
-        dot += g[j][0] * e[j][0] + g[j][1] * e[j][1] + g[j][2] * e[j][2] + g[j][3] * e[j][3];
-      }
-    }
-    dot = warp_sum(dot) * r / d;  // mean(dx0 * h)
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const int c = (j * 32 + lane) * 4;
-      if (c < d)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) G[j][i] += r * (g[j][i] - e[j][i] * r * dot);
-    }
-  }
-}
-
-template <int NV, typename w_t>
-__global__ void emb_piece_kernel(float* __restrict__ dwte, const w_t* __restrict__ wte, int d,
-                                 const float* __restrict__ dx0, const float* __restrict__ rstd,
-                                 const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm,
-                                 const int32_t* __restrict__ pstart, const int32_t* __restrict__ plen,
-                                 const int32_t* __restrict__ pslot, const int32_t* __restrict__ counters,
-                                 float* __restrict__ partial) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= counters[0]) return;
-  const int st = pstart[warp], len = plen[warp], slot = pslot[warp];
-  const long long row = skeys[st];
+__global__ void __launch_bounds__(256) emb_chunk_kernel(
+    float* __restrict__ dwte, const w_t* __restrict__ wte, int d, const float* __restrict__ dx0,
+    const float* __restrict__ rstd, const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n,
+    long long vocab, float* __restrict__ part_head, float* __restrict__ part_tail) {
+  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if ((long long)c * CHUNK >= n) return;
+  constexpr int TAB_U = TabU<NV>::value;
+  constexpr bool PREFETCH_OUT = TAB_U > 1;  // wide rows add into dwte when the run ends
+  const ChunkRuns r = chunk_runs(skeys, perm, n, c);
   float G[NV][4];
-  emb_piece_sum<NV>(dx0, wte, rstd, perm, row, st, len, d, G);
-  float* dst = (slot < 0) ? dwte + row * d : partial + (long long)slot * d;
+  zero_row<NV>(G);
+  for (int q0 = 0; q0 < r.len; q0 += TAB_U) {
+    float g[TAB_U][NV][4], e[TAB_U][NV][4], o[PREFETCH_OUT ? TAB_U : 1][NV][4], rs[TAB_U];
+    int kind[TAB_U];
+    bool ends[TAB_U];
+    uint32_t key[TAB_U];
 #pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    const int c = (j * 32 + lane) * 4;
-    if (c < d) {
-      float o[4];
-      if (slot < 0) {
-        load4(dst + c, o);
-        o[0] += G[j][0]; o[1] += G[j][1]; o[2] += G[j][2]; o[3] += G[j][3];
+    for (int u = 0; u < TAB_U; ++u) {
+      const int q = q0 + u;
+      const bool in = q < r.len;
+      const int qs = in ? q : r.len - 1;
+      const int p = __shfl_sync(0xffffffffu, r.pos, qs);
+      key[u] = __shfl_sync(0xffffffffu, r.key, qs);
+      ends[u] = in && ((r.end_mask >> q) & 1u);
+      kind[u] = ends[u] ? run_kind(r, q) : RUN_WHOLE;
+      rs[u] = 0.f;
+      if (in && p >= 0) {
+        load_row<NV>(dx0 + (long long)p * d, d, g[u]);
+        load_row<NV>(wte + (long long)key[u] * d, d, e[u]);
+        rs[u] = rstd[p];
       } else {
-        o[0] = G[j][0]; o[1] = G[j][1]; o[2] = G[j][2]; o[3] = G[j][3];
+        zero_row<NV>(g[u]);
+        zero_row<NV>(e[u]);
       }
-      store4(dst + c, o);
+      if constexpr (PREFETCH_OUT)
+        if (ends[u] && kind[u] == RUN_WHOLE && key[u] < vocab) load_row<NV>(dwte + (long long)key[u] * d, d, o[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < TAB_U; ++u) {
+      float dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        dot += g[u][j][0] * e[u][j][0] + g[u][j][1] * e[u][j][1] + g[u][j][2] * e[u][j][2] + g[u][j][3] * e[u][j][3];
+      dot = warp_sum(dot) * rs[u] / d;  // mean(dx0 * h)
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) G[j][i] += rs[u] * (g[u][j][i] - e[u][j][i] * rs[u] * dot);
+      if (!ends[u]) continue;
+      if (kind[u] == RUN_WHOLE) {
+        if (key[u] < vocab) {
+          if constexpr (PREFETCH_OUT) {
+            add_row<NV>(o[u], G);
+            store_row<NV>(dwte + (long long)key[u] * d, d, o[u]);
+          } else {
+            float* dst = dwte + (long long)key[u] * d;
+            const int lane = threadIdx.x & 31;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+              const int col = (j * 32 + lane) * 4;
+              if (col < d) {
+                float t[4];
+                load4(dst + col, t);
+                for (int i = 0; i < 4; ++i) t[i] += G[j][i];
+                store4(dst + col, t);
+              }
+            }
+          }
+        }
+      } else {
+        store_row<NV>((kind[u] == RUN_TAIL ? part_tail : part_head) + (long long)c * d, d, G);
+      }
+      zero_row<NV>(G);
     }
   }
 }
 
-__global__ void emb_long_kernel(float* __restrict__ dwte, int d, const uint32_t* __restrict__ skeys,
-                                const int32_t* __restrict__ seg_start,
-                                const int32_t* __restrict__ lseg_first_slot,
-                                const int32_t* __restrict__ lseg_nslots, const int32_t* __restrict__ lseg_seg,
-                                const int32_t* __restrict__ counters, const float* __restrict__ partial) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= counters[1]) return;
-  const int first = lseg_first_slot[warp], k = lseg_nslots[warp];
-  const long long row = skeys[seg_start[lseg_seg[warp]]];
-  for (int c = lane * 4; c < d; c += 128) {
+__global__ void __launch_bounds__(256) emb_chain_kernel(float* __restrict__ dwte, int d,
+                                                        const uint32_t* __restrict__ skeys, int n,
+                                                        long long vocab, const float* __restrict__ part_head,
+                                                        const float* __restrict__ part_tail) {
+  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+  if ((long long)c * CHUNK >= n) return;
+  uint32_t key;
+  int last;
+  if (!chained_run(skeys, n, c, key, last) || key >= vocab) return;
+  for (int col = lane * 4; col < d; col += 128) {
     float o[4];
-    load4(dwte + row * d + c, o);
-    for (int q = 0; q < k; ++q) {
-      float g[4];
-      load4(partial + (long long)(first + q) * d + c, g);
-      o[0] += g[0]; o[1] += g[1]; o[2] += g[2]; o[3] += g[3];
+    load4(part_head + (long long)c * d + col, o);
+    for (int cc = c + 1; cc <= last; cc += 8) {
+      float t[8][4];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (cc + u <= last) load4(part_tail + (long long)(cc + u) * d + col, t[u]);
+        else t[u][0] = t[u][1] = t[u][2] = t[u][3] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        o[0] += t[u][0]; o[1] += t[u][1]; o[2] += t[u][2]; o[3] += t[u][3];
+      }
     }
-    store4(dwte + row * d + c, o);
+    float w[4];
+    load4(dwte + (long long)key * d + col, w);
+    w[0] += o[0]; w[1] += o[1]; w[2] += o[2]; w[3] += o[3];
+    store4(dwte + (long long)key * d + col, w);
   }
 }

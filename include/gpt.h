@@ -302,9 +302,12 @@ int ngram_sparse_update_noalloc(void* table, float* row_state, long long n_rows,
  *   0 store      C (bf16) = acc                 3 ReLU^2     C (bf16) = relu(acc)^2
  *   1 store fp32 C (fp32) = acc                 4 ReLU^2 bwd C (bf16) = 2 sqrt(aux) acc
  *   2 accumulate C (fp32) = (beta ? C : 0) + acc   (aux: bf16 relu(a)^2, same ld as C)
- *   5 logits     C (fp32) = acc, and per (row, 256-column tile) the running max
- *                and sum of exp(acc - max) written as float pairs to `workspace`
- *                ([M, ceil(N/256)]; 128-column tiles when N < 256)
+ *   5 logits     per (row, 256-column tile; 128 when N < 256) the tile max m of
+ *                acc and s = sum exp(acc - m), written as float pairs (m, s) to
+ *                `workspace` ([M, n_tiles]); C (bf16) = exp(acc - m), the
+ *                tile-local softmax numerators.  With aux given it holds one
+ *                int32 target column per row (< 0: none) and acc at that
+ *                column goes to the M floats after the pairs in `workspace`
  * A is read K-major (a_kmajor = 1: element [m, k] at A[m*lda + k]) or M-major
  * (a_kmajor = 0: at A[k*lda + m]); B likewise with N.  splits > 1 (modes 1 and
  * 2 only) splits K and needs workspace of splits*M*N*4 bytes, the partials

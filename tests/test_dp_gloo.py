@@ -1,0 +1,113 @@
+"""Data-parallel host logic with two gloo ranks on the CPU.
+
+Each rank takes its own slice of the token stream (dp.rank_stream_seed),
+computes its gradient with the fp64 oracle, and averages it with
+dp.average_gradients -- the same call the GPU path makes on the flat fp32
+gradient.  The average must equal the gradient of the loss over both ranks'
+sequences taken together (every target valid, equal counts per rank), and the
+AdamW step that follows must leave bit-identical replicas.
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _cfg():
+    from synthetic import workload
+    return workload("tiny_fp32", x0_rows=0, n_layer=1, seq_len=16, micro_batch=2, vocab=96)
+
+
+def _batch(cfg, seed):
+    from synthetic import tokens_and_targets
+    return tokens_and_targets(cfg["micro_batch"], cfg["seq_len"], cfg["vocab"], seed, cfg["zipf_s"], 0.0)
+
+
+def _flat(G, keys):
+    return np.concatenate([np.asarray(G[k], dtype=np.float64).reshape(-1) for k in keys])
+
+
+def _rank_main(rank, world, port, out_dir):
+    import torch
+    import torch.distributed as dist
+    from gpt_pretraining_step_decoder_b200 import dp
+    from oracle import model, optim
+    from synthetic import init_params
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cfg = _cfg()
+        params = init_params(cfg, seed=3)
+        keys = sorted(params)
+        tok, tgt = _batch(cfg, dp.rank_stream_seed(cfg["seed"], rank))
+        _, _, cache = model.forward(cfg, params, tok, tgt, None, None)
+        G, _, _ = model.backward(cfg, params, cache, scale=1.0)
+        flat = torch.from_numpy(_flat(G, keys))
+        dp.average_gradients(flat)
+        avg = flat.numpy()
+
+        # the same step taken by every rank from the averaged gradient
+        new, off = {}, 0
+        for k in keys:
+            n = np.asarray(params[k]).size
+            g = avg[off:off + n].reshape(np.shape(params[k]))
+            off += n
+            z = np.zeros_like(g)
+            new[k], _, _ = optim.adamw(np.asarray(params[k], dtype=np.float64), g, z, z.copy(), 1, 1e-3,
+                                       cfg["adam_b1"], cfg["adam_b2"], cfg["adam_eps"], cfg["weight_decay"])
+        mine = torch.from_numpy(_flat(new, keys))
+        all_params = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(all_params, mine)
+        if rank == 0:
+            np.save(os.path.join(out_dir, "avg.npy"), avg)
+            np.save(os.path.join(out_dir, "params.npy"), torch.stack(all_params).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gradient_average_equals_joint_batch(tmp_path):
+    import torch.multiprocessing as mp
+    from gpt_pretraining_step_decoder_b200 import dp
+    from oracle import model, optim
+    from synthetic import init_params
+
+    world = 2
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    avg = np.load(tmp_path / "avg.npy")
+    reps = np.load(tmp_path / "params.npy")
+
+    cfg = _cfg()
+    params = init_params(cfg, seed=3)
+    keys = sorted(params)
+    toks, tgts = zip(*[_batch(cfg, dp.rank_stream_seed(cfg["seed"], r)) for r in range(world)])
+    joint = dict(cfg, micro_batch=cfg["micro_batch"] * world)
+    _, _, cache = model.forward(joint, params, np.concatenate(toks), np.concatenate(tgts), None, None)
+    G, _, _ = model.backward(joint, params, cache, scale=1.0)
+    ref = _flat(G, keys)
+    assert np.abs(avg - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+    # replicas identical bit for bit, and equal to one joint-batch AdamW step
+    np.testing.assert_array_equal(reps[0], reps[1])
+    new = {}
+    for k in keys:
+        g = np.asarray(G[k], dtype=np.float64)
+        z = np.zeros_like(g)
+        new[k], _, _ = optim.adamw(np.asarray(params[k], dtype=np.float64), g, z, z.copy(), 1, 1e-3,
+                                   cfg["adam_b1"], cfg["adam_b2"], cfg["adam_eps"], cfg["weight_decay"])
+    np.testing.assert_allclose(reps[0], _flat(new, keys), rtol=0, atol=1e-9)
+
+
+def test_rank_streams_differ():
+    from gpt_pretraining_step_decoder_b200 import dp
+    cfg = _cfg()
+    a, _ = _batch(cfg, dp.rank_stream_seed(cfg["seed"], 0))
+    b, _ = _batch(cfg, dp.rank_stream_seed(cfg["seed"], 1))
+    assert a.shape == b.shape and not np.array_equal(a, b)

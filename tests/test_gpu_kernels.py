@@ -166,6 +166,83 @@ def test_ngram_sparse_update_matches_oracle(g, dtype, R, n, d):
     assert int((T[mask] != 0).sum()) == 0 and int((S[mask] != 0).sum()) == 0
 
 
+def _run_update(g, rows, d, R, seed, dtype="bf16"):
+    """One ngram_sparse_update on a small table; returns host copies and the oracle's."""
+    import torch
+    rng = np.random.default_rng(seed)
+    n = len(rows)
+    grad = rng.standard_normal((n, d)).astype(np.float32)
+    tab0 = rng.standard_normal((R, d)).astype(np.float32) * 0.02
+    if dtype == "bf16":
+        tab0 = round_to_bf16(tab0)
+    s0 = (np.abs(rng.standard_normal(R)) * 0.1).astype(np.float32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    T = torch.from_numpy(tab0).to(tdt).cuda()
+    S = torch.from_numpy(s0).cuda()
+    ws_bytes = g.ngram_sparse_update_workspace_bytes(n, d)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    upd = torch.full((max(n, 1),), -7, dtype=torch.int32, device="cuda")
+    nupd = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    g.ngram_sparse_update(T, S, R, d, g.DTYPE_BF16 if dtype == "bf16" else g.DTYPE_F32,
+                          device_ints(np.asarray(rows, dtype=np.int32)), torch.from_numpy(grad).cuda(), n,
+                          0.01, 0.95, 1e-10, upd, nupd, ws, ws_bytes)
+    status = g.ngram_sync_status()
+    valid = (np.asarray(rows) >= 0) & (np.asarray(rows) < R)
+    W1, s1, touched = optim.table_update(tab0.astype(np.float64), s0.astype(np.float64),
+                                         np.asarray(rows)[valid], grad[valid].astype(np.float64),
+                                         0.01, 0.95, 1e-10)
+    k = int(nupd.item())
+    return status, T.float().cpu().numpy(), S.cpu().numpy(), upd[:k].cpu().numpy(), tab0, s0, W1, s1, touched
+
+
+@pytest.mark.parametrize("case", ["one", "33_same", "long_mid_chunk", "aligned_32_runs", "offset_32_runs",
+                                  "all_same_4096", "ragged_1001"])
+def test_ngram_sparse_update_run_shapes(g, case):
+    """Runs of equal rows against the chunk edges of the bucketed update: a run
+    inside one chunk, runs exactly one chunk long (aligned and straddling),
+    a run over many chunks, every position one row, a ragged tail."""
+    rng = np.random.default_rng(5)
+    R, d = 512, 768
+    if case == "one":
+        rows = [17]
+    elif case == "33_same":
+        rows = [3] * 33
+    elif case == "long_mid_chunk":
+        rows = list(rng.integers(0, R, 13)) + [R - 1] * 700 + list(rng.integers(0, R, 40))
+    elif case == "aligned_32_runs":
+        rows = [int(r) for r in rng.permutation(R)[:40] for _ in range(32)]
+    elif case == "offset_32_runs":
+        rows = [int(r) for r in rng.permutation(R)[:40] for _ in range(32)][16:] + [7] * 5
+    elif case == "all_same_4096":
+        rows = [R - 1] * 4096
+    else:
+        rows = list(rng.integers(0, R, 1001))
+    st, Wg, Sg, upd, tab0, s0, W1, s1, touched = _run_update(g, rows, d, R, seed=len(rows))
+    assert st == g.GPT_OK
+    np.testing.assert_array_equal(upd, np.unique(rows))
+    assert rel_l2(Wg - tab0, W1 - tab0) < 2e-2
+    assert rel_l2(Sg, s1) < 1e-5
+    untouched = np.setdiff1d(np.arange(R), touched)
+    np.testing.assert_array_equal(Wg[untouched], tab0[untouched])
+    np.testing.assert_array_equal(Sg[untouched], s0[untouched])
+
+
+def test_ngram_sparse_update_invalid_rows_touch_nothing(g):
+    """Ids outside [0, R) set the input error and are skipped; the valid
+    positions (including ones on the last row, R - 1) are still applied."""
+    rng = np.random.default_rng(9)
+    R, d = 256, 128
+    rows = np.concatenate([rng.integers(0, R, 300), [R - 1] * 40, [-1, R, R + 5, 1 << 30], [R - 1] * 3])
+    rows = rng.permutation(rows).astype(np.int64)
+    st, Wg, Sg, upd, tab0, s0, W1, s1, touched = _run_update(g, rows, d, R, seed=9, dtype="f32")
+    assert st == g.GPT_ERR_INPUT
+    np.testing.assert_array_equal(upd, touched)
+    assert rel_l2(Wg - tab0, W1 - tab0) < 1e-4
+    assert rel_l2(Sg, s1) < 1e-5
+    untouched = np.setdiff1d(np.arange(R), touched)
+    np.testing.assert_array_equal(Wg[untouched], tab0[untouched])
+
+
 @pytest.mark.parametrize("b_k", [1, 0])
 def test_gemm_epilogue_modes_match_fp64(g, b_k):
     """Every epilogue of the tensor-core GEMM against its definition on the fp64 product."""
@@ -179,18 +256,22 @@ def test_gemm_epilogue_modes_match_fp64(g, b_k):
     ldb = K if b_k else N
     aux = round_to_bf16(np.maximum(rng.standard_normal((M, N)), 0).astype(np.float32) ** 2)
     auxd = _bf16_dev(aux)
-    ws = torch.zeros(M * 3 * 8, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(M * 3 * 8 + M * 4, dtype=torch.uint8, device="cuda")
+    tgt = rng.integers(0, N, M).astype(np.int32)
+    tgt[::7] = -1
+    tgtd = torch.from_numpy(tgt).cuda()
+    tile_max = np.repeat(np.stack([acc[:, 256 * j:256 * (j + 1)].max(axis=1) for j in range(3)], 1), 256, 1)[:, :N]
     cases = {
         g.EPI_STORE: (torch.bfloat16, acc, 4e-3),
         g.EPI_STORE_F32: (torch.float32, acc, 1e-5),
         g.EPI_RELU2: (torch.bfloat16, np.maximum(acc, 0) ** 2, 4e-3),
         g.EPI_DRELU2: (torch.bfloat16, 2 * np.sqrt(aux.astype(np.float64)) * acc, 4e-3),
-        g.EPI_LOGITS: (torch.float32, acc, 1e-5),
+        g.EPI_LOGITS: (torch.bfloat16, np.exp(acc - tile_max), 4e-3),
     }
     for mode, (dt, ref, tol) in cases.items():
         C = torch.full((M, N), 3.0, dtype=dt, device="cuda")
         g.gptx_gemm_bf16(M, N, K, Ad, K, 1, Bd, ldb, b_k, C, N, 0, 1, ws, ws.numel(), mode=mode,
-                         aux=auxd if mode == g.EPI_DRELU2 else None)
+                         aux=auxd if mode == g.EPI_DRELU2 else (tgtd if mode == g.EPI_LOGITS else None))
         torch.cuda.synchronize()
         assert g.ngram_sync_status() == g.GPT_OK
         assert rel_l2(C.float().cpu().numpy(), ref) < tol, mode
@@ -201,6 +282,10 @@ def test_gemm_epilogue_modes_match_fp64(g, b_k):
         mx = z.max(axis=1)
         np.testing.assert_allclose(st[:, j, 0], mx, rtol=1e-5, atol=1e-4)
         np.testing.assert_allclose(st[:, j, 1], np.exp(z - mx[:, None]).sum(axis=1), rtol=1e-4)
+    # the logit at each row's target column (rows without a target are left alone)
+    zt = ws[M * 3 * 8:].view(torch.float32).cpu().numpy()
+    rows = np.nonzero(tgt >= 0)[0]
+    np.testing.assert_allclose(zt[rows], acc[rows, tgt[rows]], rtol=1e-5, atol=1e-4)
     # accumulate with beta = 1 adds into C (TMA reduce-add)
     C = torch.from_numpy(rng.standard_normal((M, N)).astype(np.float32)).cuda()
     C0 = C.cpu().numpy().astype(np.float64)

@@ -91,6 +91,14 @@ def test_bf16_gpt2_small_shape(g):
     check(g, w, model, orc, losses, 1e-2, 2e-2)
 
 
+def test_bf16_softcap_untied_clip(g):
+    """The tensor-core path with nanochat's logit softcap (z = 15 tanh(acc/15)),
+    an untied head and global-norm clipping."""
+    w = small_case("gpt2s_bf16", grad_accum=2, softcap=15.0, tie_embeddings=0, grad_clip=1.0)
+    model, orc, losses, _ = run_pair(g, w, steps=2)
+    check(g, w, model, orc, losses, 1e-2, 2e-2)
+
+
 def test_bf16_with_tables(g):
     # two micro-batches per AdamW step: both table updates happen (one per
     # backward call) and the accumulated dense gradient is compared before the
