@@ -9,10 +9,11 @@
 //   warp 1      allocates TMEM and one elected thread issues tcgen05.mma
 //               (M = 128, N = BN, K = 16 per instruction) into one of two
 //               TMEM accumulators, committing to mbarriers;
-//   warps 2..5  the epilogue: tcgen05.ld of the finished accumulator (one
-//               TMEM lane = one output row per thread), apply the epilogue,
-//               stage 128-byte rows in shared memory and write them with
-//               asynchronous TMA stores (TMA reduce-add for fp32
+//   warps 2..9  the epilogue: tcgen05.ld of the finished accumulator (one
+//               TMEM lane = one output row per thread; two warps share each
+//               32-lane quarter, one per half of the tile's columns), apply
+//               the epilogue, stage 128-byte rows in shared memory and write
+//               them with asynchronous TMA stores (TMA reduce-add for fp32
 //               accumulation), then release the accumulator.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i + 1.  K-major and MN-major operands are both read straight from their
@@ -30,7 +31,8 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // bf16 elements per 128-byte swizzle row
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 
 // Epilogue kind of one kernel instantiation (compile time, so each kernel
 // carries only its own epilogue code).
@@ -52,19 +54,20 @@ template <int KM> struct KmHeavy {
   static constexpr int value = KM == K_DRELU2 ? 1 : 0;
 };
 
-// HEAVY = 1: the epilogue-heavy variant (logits, ReLU^2 backward) trades one
-// pipeline stage for double-buffered staging and a whole-tile activation buffer.
+// HEAVY = 1 (ReLU^2 backward) trades one pipeline stage for each epilogue
+// warp's two activation blocks (its whole half tile), which also serve as its
+// output staging; the other epilogues stage through one block per warp.
 template <int BN, int HEAVY> struct Cfg {
   static constexpr int STAGES = (BN == 256) ? (HEAVY ? 3 : 4) : (HEAVY ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators (power of two >= 32)
-  static constexpr int NSTG = 2;                      // staging buffers per epilogue warp
-  static constexpr int NAUX = 2;                      // activation blocks in flight (ReLU^2 backward)
+  static constexpr int NSTG = HEAVY ? 0 : 1;           // staging blocks per epilogue warp
+  static constexpr int NAUX = 2;                       // activation blocks per epilogue warp (ReLU^2 bwd)
   static constexpr int AUX = HEAVY ? NAUX * 32 * 128 : 0;  // activation bytes per epilogue warp
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * NSTG * 32 * 128 + 4 * AUX + 1024 /*align*/ +
-                                    256 /*barriers*/;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * (NSTG * 32 * 128 + AUX) +
+                                    1024 /*align*/ + 512 /*barriers*/;
 };
 
 struct Params {
@@ -287,13 +290,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   uint8_t* stg_all = smem + C::STAGES * C::STAGE_BYTES;
-  uint8_t* aux_all = stg_all + 4 * C::NSTG * STG_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(aux_all + 4 * C::AUX);
+  uint8_t* aux_all = stg_all + EPI_WARPS * C::NSTG * STG_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(aux_all + EPI_WARPS * C::AUX);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* auxbar = tempty + 2;  // NAUX per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + EPI_WARPS * C::NAUX);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -302,8 +305,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     // tempty: one arrival per epilogue warp
-    for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], 4); }
-    for (int s = 0; s < 8; ++s) mbar_init(&auxbar[s], 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], EPI_WARPS); }
+    for (int s = 0; s < EPI_WARPS * C::NAUX; ++s) mbar_init(&auxbar[s], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -393,18 +396,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int ew = warp - 2;
+    constexpr int HALF = BN / 2;         // columns per epilogue warp
+    const int ew = warp - 2;             // 0 .. EPI_WARPS-1
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int ccol = (ew >> 2) * HALF;   // first tile column of this warp's half
     uint8_t* stg_base = stg_all + ew * C::NSTG * STG_BYTES;
     uint8_t* auxs = aux_all + ew * C::AUX;
-    int sbuf = 0;
-    uint64_t* abar = &auxbar[ew * 2];   // abar[b] guards activation buffer b
-    uint32_t aux_phase = 0;             // bit b: parity of the next wait on abar[b]
-    uint32_t aux_pending = 0;           // bit b: a load into buffer b is in flight
+    uint64_t* abar = &auxbar[ew * C::NAUX];  // abar[b] guards activation block b
+    uint32_t aux_phase = 0;                  // bit b: parity of the next wait on abar[b]
+    uint32_t aux_pending = 0;                // bit b: a load into block b is in flight
     const GemmEpilogue& e = p.epi;
     constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL;
     constexpr bool has_aux = KM == K_DRELU2;
     constexpr int CW = f32out ? 32 : 64;  // columns per 128-byte staging row
+    static_assert(!has_aux || HALF / CW <= C::NAUX, "one activation block per column block");
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -414,12 +419,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int mt, nt;
       tile_coords(mn, p, mt, nt);
       const int m0 = mt * BM;
-      const int n0 = nt * BN;
+      const int n0 = nt * BN + ccol;  // first output column of this warp
       const int mrow0 = m0 + q * 32;
       const long long m = (long long)mrow0 + lane;
-      const int nblk = min(BN / CW, (p.N - n0 + CW - 1) / CW);
-      if (has_aux) {  // the tile's first ReLU^2 activation blocks, ahead of the accumulator
-        for (int b = 0; b < C::NAUX && b < nblk; ++b) {
+      const int nblk = (p.N - n0 <= 0) ? 0 : min(HALF / CW, (p.N - n0 + CW - 1) / CW);
+      if (has_aux) {
+        // this half tile's ReLU^2 activations, ahead of the accumulator; the
+        // blocks double as output staging, so the previous tile's stores
+        // must have read them first
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+        for (int b = 0; b < nblk; ++b) {
           if (lane == 0) {
             mbar_expect_tx(&abar[b], AUX_BYTES);
             tma_load_2d(auxs + b * AUX_BYTES, &tmAux, &abar[b], n0 + b * 64, mrow0);
@@ -430,14 +440,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!warp_wait(&tfull[acc], acc_phase, abort_flag, p.err)) { ok = false; break; }
       tc_fence_after();
       float rmax = -INFINITY, rsum = 0.f;
-      const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ccol;
       int ytgt = -1;
       if constexpr (KM == K_LOGITS) {
-        // first pass over the accumulator: the tile's row maximum, so that
-        // the stored numerators exp(z - max) lie in (0, 1]
+        // first pass over the accumulator: the half tile's row maximum, so
+        // that the stored numerators exp(z - max) lie in (0, 1]
         ytgt = (e.targets != nullptr && m < p.M) ? e.targets[m] : -1;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HALF / 32; ++c) {
           const int nc = n0 + c * 32;
           if (nc >= p.N) break;  // warp-uniform
           uint32_t r[32];
@@ -453,22 +463,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (i < nv) rmax = fmaxf(rmax, z[i]);
         }
       }
-      if constexpr (KM == K_QKV) {
-        // one 128-wide head per iteration; this lane owns row m of it
+      if constexpr (KM == K_QKV && HALF == 128) {
+        // one 128-wide head (this warp's half tile); this lane owns row m of it
+        // (the host launches this epilogue with 256-column tiles only)
         const bool row_ok = m < p.M;
         const int tpos = row_ok ? (int)(m % e.T) : 0;
-#pragma unroll 1
-        for (int hh = 0; hh < BN / 128; ++hh) {
-          const int nc = n0 + hh * 128;
-          if (nc >= p.N) break;  // warp-uniform
-          const int head = nc / 128, sec = head / e.H, hi = head % e.H;
+        if (n0 < p.N) {  // warp-uniform
+          const int head = n0 / 128, sec = head / e.H, hi = head % e.H;
           float v[128];
           {
             uint32_t r0[32], r1[32], r2[32], r3[32];
-            tmem_ld32_nowait(trow + hh * 128, r0);
-            tmem_ld32_nowait(trow + hh * 128 + 32, r1);
-            tmem_ld32_nowait(trow + hh * 128 + 64, r2);
-            tmem_ld32_nowait(trow + hh * 128 + 96, r3);
+            tmem_ld32_nowait(trow, r0);
+            tmem_ld32_nowait(trow + 32, r1);
+            tmem_ld32_nowait(trow + 64, r2);
+            tmem_ld32_nowait(trow + 96, r3);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (sec < 2) {
             // RoPE ("$1000 tier nanochat run", apply_rotary_emb): y1 = x1 cos + x2 sin,
-            // y2 = -x1 sin + x2 cos over the two halves of the head, then QK-norm
+            // y2 = -x1 sin + x2 cos over the two halves of the head, then QK-norm;
             // frequency-major table: consecutive lanes (positions) read consecutive pairs
             const float2* cs = reinterpret_cast<const float2*>(e.rope) + tpos;
             float ss = 0.f;
@@ -516,11 +524,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            uint8_t* stg = stg_base + sbuf * STG_BYTES;
-            if (lane == 0) {
-              if (C::NSTG == 2) bulk_wait_read1();
-              else bulk_wait_read0();
-            }
+            uint8_t* stg = stg_base;
+            if (lane == 0) bulk_wait_read0();
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -535,10 +540,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmC, stg, nc + half * 64, mrow0);
+              tma_store_2d(&tmC, stg, n0 + half * 64, mrow0);
               bulk_commit();
             }
-            sbuf = (sbuf + 1) % C::NSTG;
           }
         }
       }
@@ -558,6 +562,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < 32; ++i) v[32 + i] = __uint_as_float(r1[i]) * e.alpha;
           }
         }
+        uint8_t* stg = stg_base;
         if constexpr (KM == K_LOGITS) {
           const int nv = min(64, p.N - nc);
           const int yo = ytgt - nc;  // target column within this block, if here
@@ -576,14 +581,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 64; ++i) { const float r = fmaxf(v[i], 0.f); v[i] = r * r; }
         } else if constexpr (KM == K_DRELU2) {
-          const int b = c % C::NAUX;
-          if (!warp_wait(&abar[b], (aux_phase >> b) & 1u, abort_flag, p.err)) { ok = false; break; }
-          aux_phase ^= 1u << b;
-          aux_pending &= ~(1u << b);
-          const uint8_t* ab = auxs + b * AUX_BYTES;
+          if (!warp_wait(&abar[c], (aux_phase >> c) & 1u, abort_flag, p.err)) { ok = false; break; }
+          aux_phase ^= 1u << c;
+          aux_pending &= ~(1u << c);
+          stg = auxs + c * AUX_BYTES;  // each lane rewrites only its own row below
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(ab + swz128(lane, j));
+            const uint4 raw = *reinterpret_cast<const uint4*>(stg + swz128(lane, j));
             const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -593,22 +597,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               v[j * 8 + 2 * h + 1] *= gg.y > 0.f ? 2.f * gg.y * rsqrtf(gg.y) : 0.f;
             }
           }
+        }
+        if constexpr (!has_aux) {
+          // the TMA store that last used the staging block must have read it
+          if (lane == 0) bulk_wait_read0();
           __syncwarp();
-          if (c + C::NAUX < nblk) {  // refill this buffer NAUX blocks ahead
-            if (lane == 0) {
-              mbar_expect_tx(&abar[b], AUX_BYTES);
-              tma_load_2d(auxs + b * AUX_BYTES, &tmAux, &abar[b], nc + C::NAUX * 64, mrow0);
-            }
-            aux_pending |= 1u << b;
-          }
         }
-        // the TMA store that last used this staging block must have read it
-        uint8_t* stg = stg_base + sbuf * STG_BYTES;
-        if (lane == 0) {
-          if (C::NSTG == 2) bulk_wait_read1();
-          else bulk_wait_read0();
-        }
-        __syncwarp();
         if (f32out) {
 #pragma unroll
           for (int j = 0; j < 8; ++j)
@@ -637,10 +631,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           else tma_store_2d(&tmC, stg, nc, mrow0);
           bulk_commit();
         }
-        sbuf = (sbuf + 1) % C::NSTG;
       }
       if (!ok) break;
-      if (KM == K_LOGITS && m < p.M) e.stats[m * p.n_tiles + nt] = make_float2(rmax, rsum);
+      // per (row, half tile) statistics of the logits
+      if (KM == K_LOGITS && nblk > 0 && m < p.M)
+        e.stats[m * ((p.N + HALF - 1) / HALF) + nt * 2 + (ew >> 2)] = make_float2(rmax, rsum);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

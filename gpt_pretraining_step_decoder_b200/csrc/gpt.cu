@@ -198,6 +198,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   else if (e.mode == EPI_DRELU2) km = tc::K_DRELU2;
   else if (e.mode == EPI_QKV) km = tc::K_QKV;
   else km = tc::K_LOGITS;
+  if (km == tc::K_QKV && BN != 256) return fail(GPT_ERR_ARG, "QKV epilogue needs 256-column tiles (N >= 256)");
   switch (km) {
     case tc::K_STORE: TRY((gemm_tc_launch_k<BN, tc::K_STORE>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32>(ta, tb, tcm, taux, p, st))); break;
@@ -455,7 +456,7 @@ static void make_plan(const gpt_config& c, Plan& p) {
   // softmax numerators straight into dz and rescales them in place
   p.logits = b16 ? 0 : cv.take(chunk * V * 4);
   p.dz = cv.take(chunk * V * es);
-  p.ce_stats = cv.take(chunk * ((V + 127) / 128) * 8);
+  p.ce_stats = cv.take(chunk * ((V + 63) / 64) * 8);  // (max, sum) per half tile
   p.ce_ztgt = cv.take(chunk * 4);
   p.tok_loss = cv.take(N * 4);
   p.ce_scale = cv.take(4);
@@ -768,7 +769,8 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const long long nchunks = (n + CHUNK - 1) / CHUNK;
   WITH_NV(d, ++g_launches; table_chunk_kernel<NV, tab_t><<<grid_for(nchunks * 32, 128), 128, 0, st>>>(
       table, state, d, grad, skeys, perm, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
-  WITH_NV(d, ++g_launches; table_chain_kernel<NV, tab_t><<<grid_for(nchunks * 32, 256), 256, 0, st>>>(
+  const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;  // <= 24 KB (d <= 2048)
+  WITH_NV(d, ++g_launches; table_chain_kernel<NV, tab_t><<<(unsigned)nchunks, CHAIN_WARPS * 32, chain_smem, st>>>(
       table, state, d, skeys, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
   LAUNCH_CHECK();
   return GPT_OK;
@@ -957,7 +959,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       el.ztgt = m->at<float>(p.ce_ztgt);
       TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), el, false, "gemm.lm_fwd"));
       ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * 4);
-      const int tcols = V >= 256 ? 256 : 128, ntl = cdiv(V, tcols);
+      const int tcols = V >= 256 ? 128 : 64, ntl = cdiv(V, tcols);  // half-tile statistics
       ++g_launches; ce_prob_kernel<<<rows, 256, ntl * 4, st>>>(
           reinterpret_cast<bf16*>(dz), m->at<float2>(p.ce_stats), ntl, tcols, targets + r0, m->at<float>(p.ce_ztgt),
           m->at<float>(p.tok_loss) + r0, V, c.softcap, m->at<float>(p.ce_scale), err);
@@ -1057,10 +1059,10 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const int32_t* perm;
     TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
     const long long nchunks = (N + CHUNK - 1) / CHUNK;
-    WITH_NV(d, ++g_launches; emb_chunk_kernel<NV, act_t><<<grid_for(nchunks * 32, 256), 256, 0, st>>>(
+    WITH_NV(d, ++g_launches; emb_chunk_kernel<NV, act_t><<<grid_for(nchunks * 32, 128), 128, 0, st>>>(
         Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, N, V, w.part_head, w.part_tail););
-    ++g_launches; emb_chain_kernel<<<grid_for(nchunks * 32, 256), 256, 0, st>>>(Gp("wte"), d, skeys, N, V,
-                                                                               w.part_head, w.part_tail);
+    WITH_NV(d, ++g_launches; emb_chain_kernel<NV><<<(unsigned)nchunks, CHAIN_WARPS * 32, (size_t)(CHAIN_WARPS - 1) * d * 4, st>>>(
+        Gp("wte"), d, skeys, N, V, w.part_head, w.part_tail););
     LAUNCH_CHECK();
   }
   const float lr_t = lr * c.lr_mult_table;
@@ -1311,10 +1313,10 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
     return fail(GPT_ERR_ARG, "gptx_gemm_bf16: split-K only for fp32 outputs");
   if (splits > 1 && (!workspace || ws_bytes < (size_t)splits * M * N * 4))
     return fail(GPT_ERR_WORKSPACE, "gptx_gemm_bf16: split-K needs splits*M*N*4 bytes of workspace");
-  const size_t stats_bytes = (size_t)M * cdiv(N, N >= 256 ? 256 : 128) * 8;
+  const size_t stats_bytes = (size_t)M * cdiv(N, N >= 256 ? 128 : 64) * 8;
   if (mode == EPI_LOGITS && (!workspace || ws_bytes < stats_bytes + (aux ? (size_t)M * 4 : 0)))
     return fail(GPT_ERR_WORKSPACE,
-                "gptx_gemm_bf16: logits need M*n_tiles*8 bytes of workspace for statistics (+ M*4 with targets)");
+                "gptx_gemm_bf16: logits need M*n_blocks*8 bytes of workspace for statistics (+ M*4 with targets)");
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
   GemmEpilogue e = epi(mode, C, ldc, beta, nullptr, mode == EPI_LOGITS ? nullptr : aux);

@@ -305,9 +305,9 @@ __global__ void __launch_bounds__(512) ce_chunk_kernel(float* __restrict__ logit
   }
 }
 
-// Cross-entropy from the logits GEMM's tile-local numerators (bf16 mode),
+// Cross-entropy from the logits GEMM's block-local numerators (bf16 mode),
 // one block per row: lse = M + log sum_j s_j exp(m_j - M) over the row's
-// column tiles j (m_j tile max, s_j = sum exp(z - m_j), M = max m_j); loss =
+// column blocks j (m_j block max, s_j = sum exp(z - m_j), M = max m_j); loss =
 // lse - z[y]; and in place over the numerators e_c = exp(z_c - m_j):
 // dz_c = (e_c exp(m_j - lse) - [c == y]) * scale (* (1 - (z_c/cap)^2) with a
 // softcap, z_c recovered as m_j + log e_c).  ("$1000 tier nanochat run":
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(256) ce_prob_kernel(bf16* __restrict__ ez, con
                                                       const float* __restrict__ ztgt,
                                                       float* __restrict__ tok_loss, int V, float softcap,
                                                       const float* __restrict__ scale_dev, unsigned* err) {
-  extern __shared__ float fac[];  // exp(m_j - lse) per column tile
+  extern __shared__ float fac[];  // exp(m_j - lse) per column block
   __shared__ float sh[32];
   const long long row = blockIdx.x;
   bf16* g = ez + row * V;
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(256) ce_prob_kernel(bf16* __restrict__ ez, con
   __syncthreads();
   const float sc = (y >= 0) ? *scale_dev : 0.f;
   for (int i = threadIdx.x * 8; i < V; i += blockDim.x * 8) {
-    // 8 columns never straddle a tile (tile_cols is a multiple of 8)
+    // 8 columns never straddle a block (tile_cols is a multiple of 8)
     const int j = i / tile_cols;
     const float f = fac[j];
     const int nv = min(8, V - i);

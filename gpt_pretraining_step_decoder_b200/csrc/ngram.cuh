@@ -11,7 +11,7 @@
 // int32 rows directly.  No atomics anywhere, so sums are formed in position
 // order and results are bit-reproducible.
 //
-// Update: the sorted positions are cut into fixed chunks of 32; one warp owns
+// Update: the sorted positions are cut into fixed chunks of 16; one warp owns
 // a chunk and finds the runs of equal rows in it with ballots.  A run that
 // lies inside the chunk is finished by that warp (sum -> mean square -> row
 // state -> row update).  A run that crosses chunk boundaries leaves one
@@ -24,7 +24,7 @@
 constexpr int RADIX_THREADS = 256;
 constexpr int RADIX_MAX_ITEMS = 8;   // keys per thread per block, at most
 constexpr int RADIX_FUSED_MAX_BLOCKS = 256;  // above this, offsets come from a scan launch
-constexpr int CHUNK = 32;            // sorted positions per warp in the update
+constexpr int CHUNK = 16;            // sorted positions per warp in the update (<= 32)
 
 // keys per thread so that a sort of n keys runs on about 96 blocks (or on
 // as many 2048-key tiles as it needs beyond that)
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(1024) unique_keys_kernel(const uint32_t* __res
 }
 
 // ---------------------------------------------------------------- runs in a chunk
-// One warp, chunk c = sorted positions [32c, 32c + len).  Lane l holds the
+// One warp, chunk c = sorted positions [CHUNK*c, CHUNK*c + len).  Lane l holds the
 // l-th key and position.  start_mask / end_mask mark the lanes where a run of
 // equal keys starts / ends inside the chunk (lane 0 always starts one, lane
 // len-1 always ends one); cont_in: the chunk's first run began in an earlier
@@ -451,14 +451,14 @@ __device__ __forceinline__ void add_row(float (&a)[NV][4], const float (&b)[NV][
     for (int i = 0; i < 4; ++i) a[j][i] += b[j][i];
 }
 
-// Up to two sorted positions per step: their gradient rows, and (for runs
-// that end there and finish in this chunk) the table row and state, are
-// loaded before any of them is used, so each warp keeps several row loads in
-// flight.  Wide rows (more than 768 columns) take one position per step to
-// stay within registers.
+// Sorted positions per step of a chunk warp: the position's gradient row and
+// (for a run that ends there and finishes in this chunk) the table row and
+// state are loaded together.  One position per step keeps the kernel near 80
+// registers so 24 warps fit on an SM; measured on the 2M x 768 table, that
+// beats two or four positions per step at 12 or 8 warps.
 template <int NV>
 struct TabU {
-  static constexpr int value = NV <= 6 ? 2 : 1;
+  static constexpr int value = 1;
 };
 
 // One warp per chunk of sorted positions: runs inside the chunk are summed
@@ -466,7 +466,7 @@ struct TabU {
 // (the chunk's first run, begun earlier) or part_head[c] (its last run, going
 // on).
 template <int NV, typename tab_t>
-__global__ void __launch_bounds__(128, 3) table_chunk_kernel(
+__global__ void __launch_bounds__(128, NV <= 6 ? 6 : (NV <= 8 ? 4 : 2)) table_chunk_kernel(
     tab_t* __restrict__ table, float* __restrict__ state, int d, const float* __restrict__ grad,
     const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n, long long n_rows,
     float* __restrict__ part_head, float* __restrict__ part_tail, float lr, float beta, float eps) {
@@ -533,21 +533,50 @@ __device__ __forceinline__ void chain_sum(const float* __restrict__ part_tail, i
   }
 }
 
-// One warp per chunk that starts a run going on into later chunks: its head
-// partial plus the tail partials of the chunks it reaches, in chunk order.
+// Sum of a chained run's partials: part_head[c] and part_tail[c+1..last].  The
+// block's CHAIN_WARPS warps each add a contiguous share of the tail partials in
+// chunk order; warp 0 then adds head + shares in warp order.  The grouping is
+// fixed by (c, last), so the result is reproducible.  Returns true in warp 0,
+// which then holds the sum in G.  sh: (CHAIN_WARPS - 1) * d floats.
+constexpr int CHAIN_WARPS = 4;
+template <int NV>
+__device__ __forceinline__ bool chain_block_sum(const float* __restrict__ part_head,
+                                                const float* __restrict__ part_tail, int d, int c, int last,
+                                                float* __restrict__ sh, float (&G)[NV][4]) {
+  const int w = threadIdx.x >> 5;
+  const int nparts = last - c;
+  const int per = (nparts + CHAIN_WARPS - 1) / CHAIN_WARPS;
+  const int b = c + 1 + w * per, e = min(last, b + per - 1);
+  float S[NV][4];
+  zero_row<NV>(S);
+  if (b <= e) chain_sum<NV>(part_tail, d, b, e, S);
+  if (w > 0) store_row<NV>(sh + (w - 1) * d, d, S);
+  __syncthreads();
+  if (w != 0) return false;
+  load_row<NV>(part_head + (long long)c * d, d, G);
+  add_row<NV>(G, S);
+  for (int ww = 1; ww < CHAIN_WARPS; ++ww) {
+    float t[NV][4];
+    load_row<NV>(sh + (ww - 1) * d, d, t);
+    add_row<NV>(G, t);
+  }
+  return true;
+}
+
+// One block per chunk; blocks whose chunk starts a run going on into later
+// chunks sum its partials and finish the row.
 template <int NV, typename tab_t>
-__global__ void __launch_bounds__(256) table_chain_kernel(
+__global__ void __launch_bounds__(CHAIN_WARPS * 32) table_chain_kernel(
     tab_t* __restrict__ table, float* __restrict__ state, int d, const uint32_t* __restrict__ skeys, int n,
     long long n_rows, const float* __restrict__ part_head, const float* __restrict__ part_tail, float lr,
     float beta, float eps) {
-  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  if ((long long)c * CHUNK >= n) return;
+  extern __shared__ float chain_sh[];
+  const int c = blockIdx.x;
   uint32_t key;
   int last;
-  if (!chained_run(skeys, n, c, key, last) || key >= n_rows) return;
+  if (!chained_run(skeys, n, c, key, last) || key >= n_rows) return;  // block-uniform
   float G[NV][4];
-  load_row<NV>(part_head + (long long)c * d, d, G);
-  chain_sum<NV>(part_tail, d, c + 1, last, G);
+  if (!chain_block_sum<NV>(part_head, part_tail, d, c, last, chain_sh, G)) return;
   typename Raw4<tab_t>::type w[NV];
   load_raw_row<NV>(table + (long long)key * d, d, w);
   table_row_apply<NV>(table, state, key, d, G, w, state[key], lr, beta, eps);
@@ -559,7 +588,7 @@ __global__ void __launch_bounds__(256) table_chain_kernel(
 // token id over its positions (same bucketing as the tables) and added to
 // the fp32 gradient dwte.
 template <int NV, typename w_t>
-__global__ void __launch_bounds__(256) emb_chunk_kernel(
+__global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chunk_kernel(
     float* __restrict__ dwte, const w_t* __restrict__ wte, int d, const float* __restrict__ dx0,
     const float* __restrict__ rstd, const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n,
     long long vocab, float* __restrict__ part_head, float* __restrict__ part_tail) {
@@ -636,33 +665,21 @@ __global__ void __launch_bounds__(256) emb_chunk_kernel(
   }
 }
 
-__global__ void __launch_bounds__(256) emb_chain_kernel(float* __restrict__ dwte, int d,
-                                                        const uint32_t* __restrict__ skeys, int n,
-                                                        long long vocab, const float* __restrict__ part_head,
-                                                        const float* __restrict__ part_tail) {
-  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
-  if ((long long)c * CHUNK >= n) return;
+template <int NV>
+__global__ void __launch_bounds__(CHAIN_WARPS * 32) emb_chain_kernel(float* __restrict__ dwte, int d,
+                                                                    const uint32_t* __restrict__ skeys, int n,
+                                                                    long long vocab,
+                                                                    const float* __restrict__ part_head,
+                                                                    const float* __restrict__ part_tail) {
+  extern __shared__ float chain_sh[];
+  const int c = blockIdx.x;
   uint32_t key;
   int last;
-  if (!chained_run(skeys, n, c, key, last) || key >= vocab) return;
-  for (int col = lane * 4; col < d; col += 128) {
-    float o[4];
-    load4(part_head + (long long)c * d + col, o);
-    for (int cc = c + 1; cc <= last; cc += 8) {
-      float t[8][4];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (cc + u <= last) load4(part_tail + (long long)(cc + u) * d + col, t[u]);
-        else t[u][0] = t[u][1] = t[u][2] = t[u][3] = 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        o[0] += t[u][0]; o[1] += t[u][1]; o[2] += t[u][2]; o[3] += t[u][3];
-      }
-    }
-    float w[4];
-    load4(dwte + (long long)key * d + col, w);
-    w[0] += o[0]; w[1] += o[1]; w[2] += o[2]; w[3] += o[3];
-    store4(dwte + (long long)key * d + col, w);
-  }
+  if (!chained_run(skeys, n, c, key, last) || key >= vocab) return;  // block-uniform
+  float G[NV][4];
+  if (!chain_block_sum<NV>(part_head, part_tail, d, c, last, chain_sh, G)) return;
+  float o[NV][4];
+  load_row<NV>(dwte + (long long)key * d, d, o);
+  add_row<NV>(o, G);
+  store_row<NV>(dwte + (long long)key * d, d, o);
 }

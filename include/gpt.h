@@ -247,11 +247,13 @@ int ngram_sparse_update_workspace_bytes(int n, int d, size_t* bytes);
  * Sparse per-row-magnitude table update, applied in place (decoder-rtx
  * posts: "sparse, no first moment, and only per-row magnitude", inlined
  * into backward).  For every distinct row r among rows[0..n):
- *   G = sum of grad[i, :] over i with rows[i] == r   (summed in order of i)
+ *   G = sum of grad[i, :] over i with rows[i] == r
  *   s_r = beta * s_r + (1 - beta) * mean_j G[j]^2
  *   table[r, :] -= lr * G / (sqrt(s_r) + eps)
  * Other rows and states are untouched.  Positions are bucketed by row with
- * a stable radix sort (no atomics), so the result is deterministic.
+ * a stable radix sort (no atomics); G is summed in a fixed order (positions
+ * in order within chunks of 16 sorted positions, then the chunks' partial
+ * sums in fixed groups), so the result is bit-reproducible.
  * table: device [n_rows, d] of `dtype` (bf16 rows are rounded to nearest
  * even); row_state: device fp32 [n_rows]; grad: device fp32 [n, d].
  * updated_rows_out (nullable): device int32 [n], receives the distinct
@@ -279,7 +281,8 @@ int ngram_sync_status(void* stream);
  * synchronisation.  The pages have no counterpart of this entry point.
  *
  * Limit: the scratch of ngram_sparse_update_workspace_bytes(n, d) must fit in
- * 16 MiB (e.g. n <= 32768 positions at d <= 1024, or n <= 65536 at d = 768);
+ * 16 MiB (about 16 + d/2 bytes per position: e.g. n <= 32768 positions at
+ * d <= 768, or n <= 8192 at d = 2048);
  * larger calls return GPT_ERR_WORKSPACE before any work is enqueued.
  * The first call on a device looks up the buffer's device address (with that
  * device current) and should come before any stream capture.  All calls share
@@ -302,10 +305,10 @@ int ngram_sparse_update_noalloc(void* table, float* row_state, long long n_rows,
  *   0 store      C (bf16) = acc                 3 ReLU^2     C (bf16) = relu(acc)^2
  *   1 store fp32 C (fp32) = acc                 4 ReLU^2 bwd C (bf16) = 2 sqrt(aux) acc
  *   2 accumulate C (fp32) = (beta ? C : 0) + acc   (aux: bf16 relu(a)^2, same ld as C)
- *   5 logits     per (row, 256-column tile; 128 when N < 256) the tile max m of
+ *   5 logits     per (row, 128-column block; 64 when N < 256) the block max m of
  *                acc and s = sum exp(acc - m), written as float pairs (m, s) to
- *                `workspace` ([M, n_tiles]); C (bf16) = exp(acc - m), the
- *                tile-local softmax numerators.  With aux given it holds one
+ *                `workspace` ([M, n_blocks]); C (bf16) = exp(acc - m), the
+ *                block-local softmax numerators.  With aux given it holds one
  *                int32 target column per row (< 0: none) and acc at that
  *                column goes to the M floats after the pairs in `workspace`
  * A is read K-major (a_kmajor = 1: element [m, k] at A[m*lda + k]) or M-major

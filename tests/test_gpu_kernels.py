@@ -256,11 +256,11 @@ def test_gemm_epilogue_modes_match_fp64(g, b_k):
     ldb = K if b_k else N
     aux = round_to_bf16(np.maximum(rng.standard_normal((M, N)), 0).astype(np.float32) ** 2)
     auxd = _bf16_dev(aux)
-    ws = torch.zeros(M * 3 * 8 + M * 4, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(M * 5 * 8 + M * 4, dtype=torch.uint8, device="cuda")
     tgt = rng.integers(0, N, M).astype(np.int32)
     tgt[::7] = -1
     tgtd = torch.from_numpy(tgt).cuda()
-    tile_max = np.repeat(np.stack([acc[:, 256 * j:256 * (j + 1)].max(axis=1) for j in range(3)], 1), 256, 1)[:, :N]
+    tile_max = np.repeat(np.stack([acc[:, 128 * j:128 * (j + 1)].max(axis=1) for j in range(5)], 1), 128, 1)[:, :N]
     cases = {
         g.EPI_STORE: (torch.bfloat16, acc, 4e-3),
         g.EPI_STORE_F32: (torch.float32, acc, 1e-5),
@@ -275,15 +275,15 @@ def test_gemm_epilogue_modes_match_fp64(g, b_k):
         torch.cuda.synchronize()
         assert g.ngram_sync_status() == g.GPT_OK
         assert rel_l2(C.float().cpu().numpy(), ref) < tol, mode
-    # logits statistics: per (row, 256-column tile) max and sum of exp(z - max)
-    st = ws[:M * 3 * 8].view(torch.float32).view(M, 3, 2).cpu().numpy().astype(np.float64)
-    for j in range(3):
-        z = acc[:, 256 * j:256 * (j + 1)]
+    # logits statistics: per (row, 128-column block) max and sum of exp(z - max)
+    st = ws[:M * 5 * 8].view(torch.float32).view(M, 5, 2).cpu().numpy().astype(np.float64)
+    for j in range(5):
+        z = acc[:, 128 * j:128 * (j + 1)]
         mx = z.max(axis=1)
         np.testing.assert_allclose(st[:, j, 0], mx, rtol=1e-5, atol=1e-4)
         np.testing.assert_allclose(st[:, j, 1], np.exp(z - mx[:, None]).sum(axis=1), rtol=1e-4)
     # the logit at each row's target column (rows without a target are left alone)
-    zt = ws[M * 3 * 8:].view(torch.float32).cpu().numpy()
+    zt = ws[M * 5 * 8:].view(torch.float32).cpu().numpy()
     rows = np.nonzero(tgt >= 0)[0]
     np.testing.assert_allclose(zt[rows], acc[rows, tgt[rows]], rtol=1e-5, atol=1e-4)
     # accumulate with beta = 1 adds into C (TMA reduce-add)
