@@ -1,10 +1,10 @@
 // attention_tc.cuh -- causal flash attention forward on the 5th-generation
 // tensor cores (tcgen05 + TMEM + TMA), bf16 in, fp32 accumulate, head_dim 128.
 //
-// Same operation as fa::fa_fwd_kernel (causal softmax attention with scale
-// 1/sqrt(hd), "$1000 tier nanochat run", `F.scaled_dot_product_attention(...,
-// is_causal=True)`): o = softmax(q k^T / sqrt(hd) + causal) v and the row
-// log-sum-exp for the backward pass.
+// Causal softmax attention with scale 1/sqrt(hd) ("$1000 tier nanochat run",
+// `F.scaled_dot_product_attention(..., is_causal=True)`): o = softmax(q k^T /
+// sqrt(hd) + causal) v, and the row log-sum-exp for the backward pass, kept
+// in log2 units (lse2 = lse / ln 2) since both backward kernels use exp2.
 //
 // One CTA per (128-query tile, sequence, head), heaviest tiles first:
 //   warp 0      TMA: Q once, then K_j and V_j (128 keys) into 2-deep rings
@@ -19,7 +19,7 @@
 //               O is rescaled in TMEM only when a row max grows by more than
 //               2^8 (log2 units) over the max in use, so most tiles skip it;
 //               the exponentials then stay below 2^8, safe in fp32 and bf16.
-// Epilogue: O / l to bf16 o, lse = (m + log2 l) ln 2.  Every wait is bounded.
+// Epilogue: O / l to bf16 o, lse2 = m + log2 l.  Every wait is bounded.
 #pragma once
 #include "gemm_tc.cuh"
 
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (qpos < T) lse_out[(long long)bh * T + qpos] = (m_use + log2f(l)) * 0.6931471805599453f;
+      if (qpos < T) lse_out[(long long)bh * T + qpos] = m_use + log2f(l);  // log2 units
     }
   }
   tc_fence_before();
@@ -336,9 +336,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace fatc
 
 // ============================================================================
-// Backward on tcgen05 (same operation as fa::fa_bwd_dkdv_kernel /
-// fa::fa_bwd_dq_kernel): with P = exp(s/sqrt(hd) - lse) recomputed from the
-// forward's log-sum-exp and D_q = rowsum(dO_q * O_q),
+// Backward on tcgen05: with P = exp(s/sqrt(hd) - lse) recomputed from the
+// forward's log-sum-exp (kept in log2 units) and D_q = rowsum(dO_q * O_q),
 //   dV = P^T dO,  dS = P (dP - D) with dP = dO V^T,  dK = dS^T Q / sqrt(hd),
 //   dQ = dS K / sqrt(hd).
 // Two kernels so every output element has one writer (no atomics): one CTA
@@ -354,6 +353,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 namespace fatcb {
 
 using fatc::LOG2E;
+// 2^x with the SFU's approximate exponential (PTX ex2.approx.ftz.f32; the
+// probabilities it feeds are rounded to bf16 right after)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns
@@ -422,11 +428,17 @@ __device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* ds
 // quarter w % 4 (32 key rows) and half (w - 2) / 4 of the 64 query columns,
 // so two warps per scheduler share the elementwise work.
 // smem: K, V [128 x 128] (32 KB each); per stage Q_i, dO_i [64 x 128] (16 KB
-// each) and lse_i, D_i (64 floats each, by TMA); per buffer P^T, dS^T
-// [128 keys x 64 queries] (16 KB each).
+// each); one P^T and one dS^T buffer [128 keys x 64 queries] (16 KB each).
+// The load of Q_{i+QS} waits for the dV/dK products of step i, and a Q/dO
+// load takes about as long as a whole step, so the ring is as deep as shared
+// memory allows (measured on B200: the step is otherwise one chain of S MMA,
+// elementwise work, dV/dK MMA and the next load).  A single P/dS buffer costs
+// nothing: the elementwise work of step i+1 outlasts the dV/dK MMAs of step
+// i that read the buffer.  lse and D come straight from global memory.
 constexpr int THREADS_B = 320;
 constexpr int KV_T = 32768, QT64 = 16384, PT = 16384;
-constexpr int DKDV_SMEM = 2 * KV_T + 2 * 2 * QT64 + 2 * 2 * PT + 2 * 512 + 1024 + 256;
+constexpr int DKDV_QS = 4;
+constexpr int DKDV_SMEM = 2 * KV_T + DKDV_QS * 2 * QT64 + 2 * PT + 1024 + 256;
 
 __device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -476,30 +488,27 @@ __device__ __forceinline__ void row64_out(uint32_t taddr, float scale, bf16* dst
 
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
-                          const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmL,
-                          const __grid_constant__ CUtensorMap tmD, bf16* __restrict__ dqkv, int T, int H,
-                          unsigned* err) {
+                          const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse2,
+                          const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + KV_T;
-  uint8_t* sQ = sV + KV_T;           // [2 stages]
-  uint8_t* sO = sQ + 2 * QT64;       // dO [2 stages]
-  uint8_t* sP = sO + 2 * QT64;       // P^T [2]
-  uint8_t* sS = sP + 2 * PT;         // dS^T [2]
-  float* sL = reinterpret_cast<float*>(sS + 2 * PT);   // lse [2 stages][64]
-  float* sD = sL + 2 * 64;                             // D [2 stages][64]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + 2 * 64);
-  uint64_t* kv_full = bars;          // 1
-  uint64_t* q_full = bars + 1;       // 2
-  uint64_t* q_empty = bars + 3;      // 2
-  uint64_t* s_full = bars + 5;       // 2
-  uint64_t* s_empty = bars + 7;      // 2
-  uint64_t* p_full = bars + 9;       // 2
-  uint64_t* p_free = bars + 11;      // 2
-  uint64_t* o_full = bars + 13;      // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint8_t* sQ = sV + KV_T;               // [DKDV_QS stages]
+  uint8_t* sO = sQ + DKDV_QS * QT64;     // dO [DKDV_QS stages]
+  uint8_t* sP = sO + DKDV_QS * QT64;     // P^T
+  uint8_t* sS = sP + PT;                 // dS^T
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + PT);
+  uint64_t* kv_full = bars;                  // 1
+  uint64_t* q_full = bars + 1;               // DKDV_QS
+  uint64_t* q_empty = q_full + DKDV_QS;      // DKDV_QS
+  uint64_t* s_full = q_empty + DKDV_QS;      // 2
+  uint64_t* s_empty = s_full + 2;            // 2
+  uint64_t* p_full = s_empty + 2;            // 2
+  uint64_t* p_free = p_full + 2;             // 2
+  uint64_t* o_full = p_free + 2;             // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -513,9 +522,11 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < DKDV_QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 8);   // one arrival per compute warp
       mbar_init(&p_full[s], 8);
@@ -547,9 +558,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       tma_load_2d(sV + KV_T / 2, &tm128, kv_full, 2 * a + h * 128 + 64, row_base + k0);
       int issued = 0;
       for (int i = 0; i < n_it && ok; ++i) {
-        const int s = i & 1;
-        if (!mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-        mbar_expect_tx(&q_full[s], 2 * QT64 + 2 * 256);
+        const int s = i % DKDV_QS;
+        if (!mbar_wait(&q_empty[s], ((i / DKDV_QS) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+        mbar_expect_tx(&q_full[s], 2 * QT64);
         const int qs = (qi0 + i) * 64, qr = row_base + qs;
         uint8_t* q = sQ + s * QT64;
         uint8_t* o = sO + s * QT64;
@@ -557,15 +568,14 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         tma_load_2d(q + QT64 / 2, &tm64, &q_full[s], h * 128 + 64, qr);
         tma_load_2d(o, &tmDO, &q_full[s], h * 128, qr);
         tma_load_2d(o + QT64 / 2, &tmDO, &q_full[s], h * 128 + 64, qr);
-        tma_load_2d(sL + s * 64, &tmL, &q_full[s], qs, bh);
-        tma_load_2d(sD + s * 64, &tmD, &q_full[s], qs, bh);
         ++issued;
       }
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(kv_full, 0)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
-      for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) {
+      for (int i = (issued > DKDV_QS ? issued - DKDV_QS : 0); i < issued; ++i) {
         const uint64_t t1 = globaltimer_ns();
-        while (!mbar_try_wait(&q_full[i & 1], (i >> 1) & 1)) if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
+        while (!mbar_try_wait(&q_full[i % DKDV_QS], (i / DKDV_QS) & 1))
+          if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
       }
     }
   } else if (warp == 1) {
@@ -577,11 +587,11 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       bool ok = mbar_wait(kv_full, 0, abort_flag, err);
       for (int i = 0; i <= n_it && ok; ++i) {
         if (i < n_it) {
-          const int s = i & 1;
-          if (!mbar_wait(&q_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          const int s = i & 1, st = i % DKDV_QS;
+          if (!mbar_wait(&q_full[st], (i / DKDV_QS) & 1, abort_flag, err)) { ok = false; break; }
           if (!mbar_wait(&s_empty[s], ((i >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aQ = smem_u32(sQ + s * QT64), aO = smem_u32(sO + s * QT64);
+          const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             tc_mma(tmem + s * 64, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
@@ -591,19 +601,19 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           tc_commit(&s_full[s]);
         }
         if (i >= 1) {
-          const int ip = i - 1, s = ip & 1;
-          if (!mbar_wait(&p_full[s], (ip >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          const int ip = i - 1, st = ip % DKDV_QS;
+          if (!mbar_wait(&p_full[0], ip & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aP = smem_u32(sP + s * PT), aS = smem_u32(sS + s * PT);
-          const uint32_t aQ = smem_u32(sQ + s * QT64), aO = smem_u32(sO + s * QT64);
+          const uint32_t aP = smem_u32(sP), aS = smem_u32(sS);
+          const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc_mma(tmem + 256, kdesc64(aP, k), mndesc(aO, QT64 / 2, k), id_g, (ip > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc_mma(tmem + 384, kdesc64(aS, k), mndesc(aQ, QT64 / 2, k), id_g, (ip > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&p_free[s]);
-          tc_commit(&q_empty[s]);
+          tc_commit(&p_free[0]);
+          tc_commit(&q_empty[st]);
           if (ip == n_it - 1) tc_commit(o_full);
         }
       }
@@ -613,12 +623,33 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     const int q4 = warp & 3, half = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
     const int key = k0 + r;
+    const int warp_key_max = k0 + q4 * 32 + 31;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
+    const float* lse_bh = lse2 + (long long)bh * T;
+    const float* D_bh = Dv + (long long)bh * T;
     bool ok = true;
     for (int i = 0; i < n_it; ++i) {
       const int s = i & 1;
       const int qbase = (qi0 + i) * 64 + half * 32;
+      // this half's 32 (lse2, D) pairs, fetched before the scores arrive
+      const bool full32 = qbase + 32 <= T;  // warp-uniform
+      float lv[32], dv[32];
+      if (full32) {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_bh + qbase + 4 * e4);
+          const float4 d4 = *reinterpret_cast<const float4*>(D_bh + qbase + 4 * e4);
+          lv[4 * e4] = l4.x; lv[4 * e4 + 1] = l4.y; lv[4 * e4 + 2] = l4.z; lv[4 * e4 + 3] = l4.w;
+          dv[4 * e4] = d4.x; dv[4 * e4 + 1] = d4.y; dv[4 * e4 + 2] = d4.z; dv[4 * e4 + 3] = d4.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          lv[e] = qbase + e < T ? lse_bh[qbase + e] : 0.f;
+          dv[e] = qbase + e < T ? D_bh[qbase + e] : 0.f;
+        }
+      }
       if (!warp_wait(&s_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       float sv[32], dp[32];
@@ -633,30 +664,33 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[s]);
-      // P^T[key, q] = exp2(s c - lse_q log2e) for key <= q < T; dS^T = P^T (dP^T - D_q)
-      const float* L = sL + s * 64 + half * 32;
-      const float* Dq = sD + s * 64 + half * 32;
+      // P^T[key, q] = exp2(s c - lse2_q) for key <= q < T; dS^T = P^T (dP^T - D_q).
+      // Off the diagonal every key of the warp is <= every query of the half
+      // (warp-uniform), so the causal test drops out.
+      if (full32 && warp_key_max <= qbase) {
 #pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(L + 4 * e4);
-        const float4 d4 = *reinterpret_cast<const float4*>(Dq + 4 * e4);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = 4 * e4 + u, qq = qbase + e;
-          const bool live = (key <= qq) && (qq < T);
-          const float p = live ? exp2f(fmaf(sv[e], c, -lv[u] * LOG2E)) : 0.f;
+        for (int e = 0; e < 32; ++e) {
+          const float p = fast_exp2(fmaf(sv[e], c, -lv[e]));
           sv[e] = p;
-          dp[e] = p * (dp[e] - dv[u]);
+          dp[e] = p * (dp[e] - dv[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int qq = qbase + e;
+          const float p = (key <= qq && qq < T) ? fast_exp2(fmaf(sv[e], c, -lv[e])) : 0.f;
+          sv[e] = p;
+          dp[e] = p * (dp[e] - dv[e]);
         }
       }
-      if (i >= 2 && !warp_wait(&p_free[s], ((i - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      st_half_row(sP + s * PT, r, half, sv);
-      st_half_row(sS + s * PT, r, half, dp);
+      // the single P/dS buffer: the dV/dK products of step i-1 must have read it
+      if (i >= 1 && !warp_wait(&p_free[0], (i - 1) & 1, abort_flag, err)) { ok = false; break; }
+      st_half_row(sP, r, half, sv);
+      st_half_row(sS, r, half, dp);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[s]);
+      if (lane == 0) mbar_arrive(&p_full[0]);
     }
     if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
       tc_fence_after();
@@ -677,13 +711,13 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 // ---------------------------------------------------------------- dQ
 // 10 warps as above; compute warps split the 64 key columns in halves.
 // smem: Q, dO [128 x 128] (32 KB each); per stage K_j, V_j [64 x 128] (16 KB
-// each, 3 stages); per buffer dS [128 queries x 64 keys] (16 KB, 2 buffers).
-constexpr int DQ_STAGES = 3;
+// each, 4 stages); per buffer dS [128 queries x 64 keys] (16 KB, 2 buffers).
+constexpr int DQ_STAGES = 4;
 constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 2 * PT + 1024 + 256;
 
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
-                        const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
+                        const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse2,
                         const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
@@ -694,15 +728,16 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint8_t* sV = sK + DQ_STAGES * QT64;       // [stages]
   uint8_t* sS = sV + DQ_STAGES * QT64;       // dS [2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sS + 2 * PT);
-  uint64_t* q_full = bars;                   // 1
-  uint64_t* kv_full = bars + 1;              // 3
-  uint64_t* kv_empty = bars + 4;             // 3
-  uint64_t* s_full = bars + 7;               // 2
-  uint64_t* s_empty = bars + 9;              // 2
-  uint64_t* p_full = bars + 11;              // 2
-  uint64_t* p_free = bars + 13;              // 2
-  uint64_t* o_full = bars + 15;              // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars;                      // 1
+  uint64_t* kv_full = q_full + 1;               // DQ_STAGES
+  uint64_t* kv_empty = kv_full + DQ_STAGES;     // DQ_STAGES
+  uint64_t* s_full = kv_empty + DQ_STAGES;      // 2
+  uint64_t* s_empty = s_full + 2;               // 2
+  uint64_t* p_full = s_empty + 2;               // 2
+  uint64_t* p_free = p_full + 2;                // 2
+  uint64_t* o_full = p_free + 2;                // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+  static_assert((2 + 2 * DQ_STAGES + 8) * 8 + 8 <= 256, "barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -814,7 +849,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     const bool valid = qpos < T;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
-    const float L = valid ? lse[(long long)bh * T + qpos] * LOG2E : 0.f;
+    const float L = valid ? lse2[(long long)bh * T + qpos] : 0.f;  // log2 units
     const float Dq = valid ? Dv[(long long)bh * T + qpos] : 0.f;
     bool ok = true;
     for (int j = 0; j < n_it; ++j) {
@@ -837,7 +872,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const bool live = valid && (kbase + e <= qpos);
-        const float p = live ? exp2f(fmaf(sv[e], c, -L)) : 0.f;
+        const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
         dp[e] = p * (dp[e] - Dq);
       }
       if (j >= 2 && !warp_wait(&p_free[s], ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }

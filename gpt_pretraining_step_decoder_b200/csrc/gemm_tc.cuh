@@ -57,17 +57,20 @@ template <int KM> struct KmHeavy {
 // HEAVY = 1 (ReLU^2 backward) trades one pipeline stage for each epilogue
 // warp's two activation blocks (its whole half tile), which also serve as its
 // output staging; the other epilogues stage through one block per warp.
+// BN = 128, 192 or 256 (192 only with fp32 outputs: 96 columns per epilogue
+// warp = three 32-column fp32 blocks); the ring takes what shared memory has
+// left after the epilogue's buffers, at most 6 stages.
 template <int BN, int HEAVY> struct Cfg {
-  static constexpr int STAGES = (BN == 256) ? (HEAVY ? 3 : 4) : (HEAVY ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators (power of two >= 32)
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;  // two accumulators, power of two
   static constexpr int NSTG = HEAVY ? 0 : 1;           // staging blocks per epilogue warp
   static constexpr int NAUX = 2;                       // activation blocks per epilogue warp (ReLU^2 bwd)
   static constexpr int AUX = HEAVY ? NAUX * 32 * 128 : 0;  // activation bytes per epilogue warp
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * (NSTG * 32 * 128 + AUX) +
-                                    1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int FIXED = EPI_WARPS * (NSTG * 32 * 128 + AUX) + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int STAGES = (232448 - FIXED) / STAGE_BYTES > 6 ? 6 : (232448 - FIXED) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
 };
 
 struct Params {

@@ -23,7 +23,6 @@
 #include "gemm_common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
-#include "attention_fa.cuh"
 #include "attention_tc.cuh"
 #include "layers.cuh"
 #include "ngram.cuh"
@@ -199,6 +198,14 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   else if (e.mode == EPI_QKV) km = tc::K_QKV;
   else km = tc::K_LOGITS;
   if (km == tc::K_QKV && BN != 256) return fail(GPT_ERR_ARG, "QKV epilogue needs 256-column tiles (N >= 256)");
+  if constexpr (BN == 192) {  // fp32 outputs only
+    switch (km) {
+      case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32>(ta, tb, tcm, taux, p, st))); break;
+      case tc::K_REDUCE_F32: TRY((gemm_tc_launch_k<BN, tc::K_REDUCE_F32>(ta, tb, tcm, taux, p, st))); break;
+      case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL>(ta, tb, tcm, taux, p, st))); break;
+      default: return fail(GPT_ERR_ARG, "192-column tiles take fp32-output epilogues only");
+    }
+  } else {
   switch (km) {
     case tc::K_STORE: TRY((gemm_tc_launch_k<BN, tc::K_STORE>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32>(ta, tb, tcm, taux, p, st))); break;
@@ -208,6 +215,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
     case tc::K_DRELU2: TRY((gemm_tc_launch_k<BN, tc::K_DRELU2>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_QKV: TRY((gemm_tc_launch_k<BN, tc::K_QKV>(ta, tb, tcm, taux, p, st))); break;
     default: TRY((gemm_tc_launch_k<BN, tc::K_LOGITS>(ta, tb, tcm, taux, p, st))); break;
+  }
   }
   if (p.splits > 1) {
     const long long total = (long long)M * N;
@@ -220,6 +228,15 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
 }
 
 // Choose split-K so a small-output, long-K product still fills the GPU.
+// Share of the SMs' tile slots doing useful columns: tiles over whole waves,
+// times the used fraction of the last column tile.
+static double tile_efficiency(int M, int N, int BN, int splits) {
+  const long long tiles = (long long)cdiv(M, 128) * cdiv(N, BN) * splits;
+  const long long sms = device_sms();
+  const double waves = (double)((tiles + sms - 1) / sms);
+  return ((double)tiles / (waves * sms)) * ((double)N / ((double)cdiv(N, BN) * BN));
+}
+
 static int pick_splits(int M, int N, int K, int BN) {
   const int tiles = cdiv(M, 128) * cdiv(N, BN);
   const int kb = cdiv(K, 64);
@@ -293,13 +310,24 @@ static int gemm(const GemmCtx& g, int M, int N, int K, GemmOperand A, GemmOperan
     LAUNCH_CHECK();
     return GPT_OK;
   }
-  const int BN = (N >= 256) ? 256 : 128;
-  int splits = 1;
-  if (allow_split && (e.mode == EPI_ACCUM_F32 || e.mode == EPI_STORE_F32)) {
-    splits = pick_splits(M, N, K, BN);
-    while (splits > 1 && (long long)splits * M * N > g.splitk_elems) --splits;
+  const bool f32out = e.mode == EPI_ACCUM_F32 || e.mode == EPI_STORE_F32;
+  const bool split_ok = allow_split && f32out;
+  auto splits_for = [&](int bn) {
+    if (!split_ok) return 1;
+    int s = pick_splits(M, N, K, bn);
+    while (s > 1 && (long long)s * M * N > g.splitk_elems) --s;
+    return s;
+  };
+  // tile width: 256 (128 below 256 columns); fp32 outputs may take 192 when
+  // that fills the last wave of SMs better (N = 768: 4 x 192 instead of 3 x 256)
+  int BN = (N >= 256) ? 256 : 128;
+  int splits = splits_for(BN);
+  if (f32out && N >= 256 && tile_efficiency(M, N, 192, splits_for(192)) > tile_efficiency(M, N, 256, splits) + 0.03) {
+    BN = 192;
+    splits = splits_for(192);
   }
   if (BN == 256) return gemm_tc_launch<256>(M, N, K, A, B, e, splits, g.splitk, g.err, g.st);
+  if (BN == 192) return gemm_tc_launch<192>(M, N, K, A, B, e, splits, g.splitk, g.err, g.st);
   return gemm_tc_launch<128>(M, N, K, A, B, e, splits, g.splitk, g.err, g.st);
 }
 
@@ -826,23 +854,15 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
       attr = true;
     }
     const long long a = (long long)c.n_head * c.head_dim;
-    CUtensorMap t128, t64, tdo, tl, td;
+    CUtensorMap t128, t64, tdo;
     TRY(make_tmap(&t128, qkv, 3 * a, N, 3 * a, 64, 128));
     TRY(make_tmap(&t64, qkv, 3 * a, N, 3 * a, 64, 64));
     TRY(make_tmap(&tdo, dout, a, N, a, 64, 64));
-    {
-      // lse and D [B*H, T] fp32, 64 positions per box, no swizzle
-      const uint64_t dims[2] = {(uint64_t)c.seq_len, (uint64_t)c.micro_batch * c.n_head};
-      const uint64_t str[1] = {(uint64_t)c.seq_len * 4};
-      const uint32_t box[2] = {64, 1};
-      TRY(make_tmap_gen(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, lse, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
-      TRY(make_tmap_gen(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Dv, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE));
-    }
     dim3 gk(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
     dim3 gq(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
     bf16* g16 = reinterpret_cast<bf16*>(dqkv);
     ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<gk, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st>>>(
-        t128, t64, tdo, tl, td, g16, c.seq_len, c.n_head, m->err());
+        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
     ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<gq, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
         t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
     LAUNCH_CHECK();
@@ -1327,6 +1347,10 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
   }
   GemmOperand a{A, lda, a_kmajor ? 1 : 0}, b{B, ldb, b_kmajor ? 1 : 0};
   GemmCtx g{true, (float*)workspace, (long long)(ws_bytes / 4), err, (cudaStream_t)stream, nullptr};
+  // the same tile width the step would take for this shape
+  const bool f32out = mode == EPI_ACCUM_F32 || mode == EPI_STORE_F32;
+  if (f32out && N >= 256 && tile_efficiency(M, N, 192, splits) > tile_efficiency(M, N, 256, splits) + 0.03)
+    return gemm_tc_launch<192>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
 }

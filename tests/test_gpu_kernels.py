@@ -25,7 +25,8 @@ def _bf16_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 384, 160), (776, 264, 520), (256, 768, 768)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 384, 160), (776, 264, 520), (256, 768, 768),
+                                   (2048, 768, 320)])  # the last one runs on 192-column tiles
 @pytest.mark.parametrize("a_k,b_k", [(1, 1), (1, 0), (0, 0), (0, 1)])
 def test_gemm_layouts_match_fp64(g, M, N, K, a_k, b_k):
     import torch
