@@ -39,6 +39,32 @@ METRIC = "training tokens/sec and MFU (% of B200 dense BF16 peak) at 1 GPU"
 L2_NOTE = "no L2 flush: a step's working set (weights, activations, logits chunk) is > 10 GB, far above the 126 MB L2"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic_gpt2s_bf16.json")
+GEMM_SOURCES = ["gemm_tc.cuh", "gemm_common.cuh", "gpt.cu"]
+
+
+def gemm_sources_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "gpt_pretraining_step_decoder_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on this workload with the current GEMM sources; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("workload") != workload_name or rec.get("sources_sha256") != gemm_sources_sha():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -294,7 +320,8 @@ def run_ours(args, w, rank, world, dist):
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": recorded_traffic(w["name"]) if dom_name == "gemm" else None,
                 "peak_source": f"{peak_src} bf16 sustained (cuBLAS loop under the power cap)"}
     else:
         achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
@@ -303,8 +330,9 @@ def run_ours(args, w, rank, world, dist):
                 "peak_source": f"{peak_src} HBM copy"}
     roof["launches_per_step"] = dom["launches"] / args.steps
     roof["share_of_step"] = dom["ms"] / total_ms if total_ms else None
-    roof["per_launch"] = ("gemm: algorithmic 2*M*N*K FLOPs of every contraction in the step, "
-                          "summed, over the summed CUDA-event time of those launches")
+    roof["per_launch"] = (f"{dom_name}: algorithmic FLOPs (2*M*N*K per contraction) or bytes of every launch in "
+                          "the step, summed, over the summed CUDA-event time of those launches; traffic = DRAM "
+                          "bytes per launch from the committed ncu summary (null unless taken with these sources)")
     breakdown = {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
                      "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["flops"] and v["ms"] else None,
                      "gbs": (v["bytes"] / (v["ms"] / 1e3) / 1e9) if v["bytes"] and v["ms"] else None}

@@ -33,6 +33,14 @@ constexpr int SMEM_BYTES = TILE_BYTES /*Q*/ + 2 * 2 * TILE_BYTES /*K,V x 2 stage
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;  // log2 units
 
+// 2^x with the SFU's approximate exponential (PTX ex2.approx.ftz.f32; the
+// probabilities it feeds are rounded to bf16 right after)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
@@ -282,7 +290,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 keys
         float p[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { p[e] = exp2f(fmaf(sv[ch * 8 + e], c, nm)); ps[e] += p[e]; }
+        for (int e = 0; e < 8; ++e) { p[e] = fast_exp2(fmaf(sv[ch * 8 + e], c, nm)); ps[e] += p[e]; }
         uint4 w;
         __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]), b1 = __floats2bfloat162_rn(p[2], p[3]);
         __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]), b3 = __floats2bfloat162_rn(p[6], p[7]);
@@ -353,13 +361,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 namespace fatcb {
 
 using fatc::LOG2E;
-// 2^x with the SFU's approximate exponential (PTX ex2.approx.ftz.f32; the
-// probabilities it feeds are rounded to bf16 right after)
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+using fatc::fast_exp2;
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns

@@ -1060,9 +1060,15 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
                              m->at<float>(p.Dattn), dqkv));
     {
       ProfScope ps(pf, st, "rope_qknorm_bwd", 0.0, (double)N * a * es * 6 + (c.v_rows ? (double)N * a * (es + 8) : 0.0));
-      ++g_launches; rope_qknorm_bwd_kernel<act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
-          dqkv, m->at<act_t>(L.qkv), m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
-          c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
+      if (b16)  // hd == 128 in bf16 mode
+        ++g_launches, rope_qknorm_bwd_hd128_kernel<<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+            reinterpret_cast<bf16*>(dqkv), reinterpret_cast<const bf16*>(m->at<act_t>(L.qkv)), m->at<float>(p.rope_cs),
+            m->at<float>(L.rstd_q), m->at<float>(L.rstd_k), c.v_rows ? m->at<float>(p.gv) : nullptr,
+            l != c.n_layer - 1, N, c.seq_len, H, c.qk_norm);
+      else
+        ++g_launches, rope_qknorm_bwd_kernel<act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+            dqkv, m->at<act_t>(L.qkv), m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
+            c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
       LAUNCH_CHECK();
     }
     TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true, "gemm.qkv_wgrad"));

@@ -257,6 +257,75 @@ __global__ void rope_qknorm_bwd_kernel(act_t* __restrict__ dqkv, const act_t* __
   }
 }
 
+// The same backward for bf16 activations and hd = 128, vectorised: lane l
+// owns elements 4j..4j+3 (j = l & 15) of half l >> 4 of the head, so each lane
+// moves 8-byte pieces of dq, dk, q and k at once; the rotation partner of
+// element i (i + 64 or i - 64) sits in lane l ^ 16.
+__global__ void __launch_bounds__(256) rope_qknorm_bwd_hd128_kernel(
+    bf16* __restrict__ dqkv, const bf16* __restrict__ qkv, const float* __restrict__ cs,
+    const float* __restrict__ rstd_q, const float* __restrict__ rstd_k, float* __restrict__ gv, int gv_accumulate,
+    int N, int T, int H, int qk_norm) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= N * H) return;  // whole warp
+  const int n = warp / H, h = warp % H, t = n % T;
+  const int a = H * 128;
+  const int j = lane & 15, hf = lane >> 4, i0 = hf * 64 + 4 * j;
+  const long long base = (long long)n * 3 * a + h * 128 + i0;
+  float g[2][4], y[2][4];
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const uint2 rg = *reinterpret_cast<const uint2*>(dqkv + base + w * a);
+    const uint2 ry = *reinterpret_cast<const uint2*>(qkv + base + w * a);
+    const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rg.x));
+    const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rg.y));
+    const float2 y01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ry.x));
+    const float2 y23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ry.y));
+    g[w][0] = g01.x; g[w][1] = g01.y; g[w][2] = g23.x; g[w][3] = g23.y;
+    y[w][0] = y01.x; y[w][1] = y01.y; y[w][2] = y23.x; y[w][3] = y23.y;
+  }
+  // QK-norm backward: d = r (g - y mean(g y)) per head
+  float d[2][4];
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    float dot = 0.f, r = 1.f;
+    if (qk_norm) {
+      dot = g[w][0] * y[w][0] + g[w][1] * y[w][1] + g[w][2] * y[w][2] + g[w][3] * y[w][3];
+      dot = warp_sum(dot) * (1.f / 128.f);
+      r = (w == 0 ? rstd_q : rstd_k)[(long long)n * H + h];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) d[w][e] = r * (g[w][e] - y[w][e] * dot);
+  }
+  // RoPE backward: dx1 = dy1 c - dy2 s, dx2 = dy1 s + dy2 c, frequencies 4j..4j+3
+  const float4* c4 = reinterpret_cast<const float4*>(cs + 2 * ((long long)t * 64 + 4 * j));
+  const float4 ca = c4[0], cb = c4[1];
+  const float cc[4] = {ca.x, ca.z, cb.x, cb.z}, ss[4] = {ca.y, ca.w, cb.y, cb.w};
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, d[w][e], 16);
+      const float d1 = hf == 0 ? d[w][e] : other, d2 = hf == 0 ? other : d[w][e];
+      o[e] = hf == 0 ? d1 * cc[e] - d2 * ss[e] : d1 * ss[e] + d2 * cc[e];
+    }
+    uint2 out;
+    __nv_bfloat162 b01 = __floats2bfloat162_rn(o[0], o[1]), b23 = __floats2bfloat162_rn(o[2], o[3]);
+    out.x = *reinterpret_cast<uint32_t*>(&b01);
+    out.y = *reinterpret_cast<uint32_t*>(&b23);
+    *reinterpret_cast<uint2*>(dqkv + base + w * a) = out;
+  }
+  if (gv) {  // value-table gradient: sum of dv over the layers, per position
+    const uint2 rv = *reinterpret_cast<const uint2*>(dqkv + base + 2 * a);
+    const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rv.x));
+    const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rv.y));
+    float4* dst = reinterpret_cast<float4*>(gv + (long long)n * a + h * 128 + i0);
+    float4 acc = gv_accumulate ? *dst : make_float4(0.f, 0.f, 0.f, 0.f);
+    acc.x += v01.x; acc.y += v01.y; acc.z += v23.x; acc.w += v23.y;
+    *dst = acc;
+  }
+}
+
 // --------------------------------------------------------------------------
 // Cross-entropy over one chunk of rows of fp32 logits [rows, V], fused
 // forward and backward ("$1000 tier nanochat run", `GPT.forward`: optional
