@@ -237,14 +237,18 @@ static double tile_efficiency(int M, int N, int BN, int splits) {
   return ((double)tiles / (waves * sms)) * ((double)N / ((double)cdiv(N, BN) * BN));
 }
 
+// Split-K factor for a product with few output tiles: the one that fills whole
+// waves of SMs best (tile_efficiency), keeping at least 8 k-blocks per split;
+// on a tie the smaller factor (fewer partial sums to add).
 static int pick_splits(int M, int N, int K, int BN) {
-  const int tiles = cdiv(M, 128) * cdiv(N, BN);
   const int kb = cdiv(K, 64);
-  const int sms = device_sms();
-  int s = 1;
-  while (tiles * s < sms && kb / (s * 2) >= 8) s *= 2;
-  while (tiles * (s + 1) <= sms + sms / 8 && kb / (s + 1) >= 8) ++s;
-  return s;
+  int best = 1;
+  double best_eff = tile_efficiency(M, N, BN, 1);
+  for (int s = 2; s <= 16 && kb / s >= 8; ++s) {
+    const double e = tile_efficiency(M, N, BN, s);
+    if (e > best_eff + 1e-9) { best = s; best_eff = e; }
+  }
+  return best;
 }
 
 // ======================================================================== live timing
@@ -992,7 +996,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
                                                    c.softcap, m->at<float>(p.ce_scale), err);
       LAUNCH_CHECK();
     }
-    TRY(gemm(g, rows, d, V, op_k(dz, V), op_mn(Wlm, d), epi(EPI_STORE_F32, m->at<float>(p.dxf) + (long long)r0 * d, d), false,
+    TRY(gemm(g, rows, d, V, op_k(dz, V), op_mn(Wlm, d), epi(EPI_STORE_F32, m->at<float>(p.dxf) + (long long)r0 * d, d), true,
              "gemm.lm_dgrad"));
     TRY(gemm(g, V, d, rows, op_mn(dz, V), op_mn(xf + (long long)r0 * d, d),
              epi(EPI_ACCUM_F32, m->at<float>(p.pending), d, ci > 0), true, "gemm.lm_wgrad"));
