@@ -562,8 +562,19 @@ __global__ void attn_bwd_pre_kernel(const act_t* __restrict__ o, const act_t* __
   const int n = warp / H, h = warp % H, b = n / T, t = n % T;
   const int a = H * hd;
   float s = 0.f;
-  for (int c = lane; c < hd; c += 32)
-    s += to_f(o[(long long)n * a + h * hd + c]) * to_f(dout[(long long)n * a + h * hd + c]);
+  if (sizeof(act_t) == 2 && hd == 128) {
+    // bf16 head of 128: 8 bytes (4 values) of each operand per lane
+    const uint2 ro = *reinterpret_cast<const uint2*>(o + (long long)n * a + h * 128 + 4 * lane);
+    const uint2 rd = *reinterpret_cast<const uint2*>(dout + (long long)n * a + h * 128 + 4 * lane);
+    const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ro.x));
+    const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ro.y));
+    const float2 d01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rd.x));
+    const float2 d23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rd.y));
+    s = o01.x * d01.x + o01.y * d01.y + o23.x * d23.x + o23.y * d23.y;
+  } else {
+    for (int c = lane; c < hd; c += 32)
+      s += to_f(o[(long long)n * a + h * hd + c]) * to_f(dout[(long long)n * a + h * hd + c]);
+  }
   s = warp_sum(s);
   if (lane == 0) Dout[((long long)b * H + h) * T + t] = s;
 }
