@@ -237,11 +237,14 @@ static double tile_efficiency(int M, int N, int BN, int splits) {
   return ((double)tiles / (waves * sms)) * ((double)N / ((double)cdiv(N, BN) * BN));
 }
 
-// Split-K factor for a product with few output tiles: the one that fills whole
-// waves of SMs best (tile_efficiency), keeping at least 8 k-blocks per split;
-// on a tie the smaller factor (fewer partial sums to add).
+// Split-K factor for a product with few output tiles (under 1.5 waves of SMs;
+// larger products pay more for the fp32 partials than a fuller last wave
+// returns): the one that fills whole waves best (tile_efficiency), keeping at
+// least 8 k-blocks per split; on a tie the smaller factor.
 static int pick_splits(int M, int N, int K, int BN) {
   const int kb = cdiv(K, 64);
+  const long long tiles = (long long)cdiv(M, 128) * cdiv(N, BN);
+  if (tiles >= device_sms() + device_sms() / 2) return 1;
   int best = 1;
   double best_eff = tile_efficiency(M, N, BN, 1);
   for (int s = 2; s <= 16 && kb / s >= 8; ++s) {

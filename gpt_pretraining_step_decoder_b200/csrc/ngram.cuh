@@ -337,7 +337,9 @@ __device__ __forceinline__ int run_kind(const ChunkRuns& r, int q) {
 }
 
 // Chunk c starts a run that goes on into later chunks: returns its key and
-// the last chunk it reaches, else false.
+// the last chunk it reaches, else false.  Called by whole warps: the end of
+// the run is found by a 32-way search over the sorted keys (a few rounds of
+// one load per lane instead of one dependent load per chunk of a long run).
 __device__ __forceinline__ bool chained_run(const uint32_t* __restrict__ skeys, int n, int c, uint32_t& key,
                                             int& last_chunk) {
   const long long base = (long long)c * CHUNK;
@@ -345,9 +347,20 @@ __device__ __forceinline__ bool chained_run(const uint32_t* __restrict__ skeys, 
   key = skeys[base + CHUNK - 1];
   if (skeys[base + CHUNK] != key) return false;
   if (c > 0 && skeys[base - 1] == key) return false;
-  int cc = c + 1;
-  while ((long long)cc * CHUNK + CHUNK < n && skeys[(long long)cc * CHUNK + CHUNK] == key) ++cc;
-  last_chunk = cc;
+  // first index with a different key lies in (lo, hi]; skeys[lo] == key
+  const int lane = threadIdx.x & 31;
+  long long lo = base + CHUNK, hi = n;
+  while (hi - lo > 1) {
+    const long long step = (hi - lo + 31) / 32;
+    const long long probe = lo + (long long)(lane + 1) * step;
+    const bool same = probe < hi && skeys[probe] == key;
+    const int cnt = __popc(__ballot_sync(0xffffffffu, same));  // keys sorted: a prefix of the lanes
+    const long long nlo = lo + (long long)cnt * step;
+    const long long nhi = lo + (long long)(cnt + 1) * step;
+    lo = nlo;
+    if (nhi < hi) hi = nhi;
+  }
+  last_chunk = (int)((hi - 1) / CHUNK);
   return true;
 }
 
