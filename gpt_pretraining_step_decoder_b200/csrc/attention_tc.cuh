@@ -6,7 +6,13 @@
 // sqrt(hd) + causal) v, and the row log-sum-exp for the backward pass, kept
 // in log2 units (lse2 = lse / ln 2) since both backward kernels use exp2.
 //
-// One CTA per (128-query tile, sequence, head), heaviest tiles first:
+// Persistent: one CTA per SM walks the (128-query tile, sequence, head)
+// items heaviest first (item i of CTA c is c + i * gridDim.x); the K/V rings,
+// S buffers and P buffers run on across items, the next item's Q loads as
+// soon as the previous item's last S has read Q, and O alternates between two
+// TMEM accumulators so an item's epilogue overlaps the next item's MMAs
+// (measured on B200: per-CTA set-up and epilogue took about as long as the
+// work of a short causal tile).  Roles:
 //   warp 0      TMA: Q once, then K_j and V_j (128 keys) into 2-deep rings
 //               with separate barriers, so K_{j+2} loads as soon as S_j
 //               has read K_j;
@@ -65,9 +71,15 @@ __device__ __forceinline__ uint64_t mnmaj_desc(uint32_t base, int k) {
   return tc::smem_desc(base + (k >> 2) * (TILE_BYTES / 2) + (k & 3) * 2048, 8192, 1024);
 }
 
+// Work item i of the grid (heaviest first): query tile and (sequence, head).
+__device__ __forceinline__ void fwd_item(int i, int n_qt, int BH, int& qt, int& bh) {
+  qt = n_qt - 1 - i / BH;
+  bh = i % BH;
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     fa_tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constant__ CUtensorMap tmV,
-                     bf16* __restrict__ out, float* __restrict__ lse_out, int T, int H, unsigned* err) {
+                     bf16* __restrict__ out, float* __restrict__ lse_out, int T, int H, int BH, unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -77,28 +89,30 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sP = sV + 2 * TILE_BYTES;        // [2 buffers]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * TILE_BYTES);
   uint64_t* q_full = bars;                  // 1
-  uint64_t* k_full = bars + 1;              // 2
-  uint64_t* k_empty = bars + 3;             // 2 (S_j done with K_j)
-  uint64_t* v_full = bars + 5;              // 2
-  uint64_t* v_empty = bars + 7;             // 2 (PV_j done with V_j)
-  uint64_t* s_full = bars + 9;              // 2
-  uint64_t* s_empty = bars + 11;            // 2
-  uint64_t* p_full = bars + 13;             // 2
-  uint64_t* p_free = bars + 15;             // 2 (PV_j done: P buffer and O are free)
-  uint64_t* o_full = bars + 17;             // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* q_empty = bars + 1;             // 1 (the item's last S has read Q)
+  uint64_t* k_full = bars + 2;              // 2
+  uint64_t* k_empty = bars + 4;             // 2 (S done with K)
+  uint64_t* v_full = bars + 6;              // 2
+  uint64_t* v_empty = bars + 8;             // 2 (PV done with V)
+  uint64_t* s_full = bars + 10;             // 2
+  uint64_t* s_empty = bars + 12;            // 2
+  uint64_t* p_full = bars + 14;             // 2
+  uint64_t* p_free = bars + 16;             // 2 (PV done: P buffer free, O updated)
+  uint64_t* o_full = bars + 18;             // 2 (per O buffer: the item's last PV is done)
+  uint64_t* o_empty = bars + 20;            // 2 (per O buffer: the softmax warps have read O)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;  // heaviest tiles first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int a = H * HD;
-  const int q0 = qt * BQ;
-  const int n_kv = min(qt + 1, (T + BKV - 1) / BKV);
-  const int row_base = b * T;  // token row of position 0 of this sequence
+  const int n_qt = (T + BQ - 1) / BQ;
+  const int total = n_qt * BH;
+  // this CTA's items: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int first = blockIdx.x, stride = gridDim.x;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -108,8 +122,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&s_empty[s], 4);   // one arrival per softmax warp
       mbar_init(&p_full[s], 4);
       mbar_init(&p_free[s], 1);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 4);
     }
-    mbar_init(o_full, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -122,47 +137,55 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S0: cols 0..127, S1: 128..255, O: 256..383
+  const uint32_t tmem = *tmem_slot;  // S0: cols 0..127, S1: 128..255, O0: 256..383, O1: 384..511
 
   if (warp == 0) {
     if (lane < 2) {
       // ---------------------------------------------------------------- TMA
-      // lane 0 streams Q and the K tiles, lane 1 the V tiles: a K buffer is
-      // refilled as soon as S_j has read it, independently of PV_j.
+      // lane 0 streams Q (once per item, after the previous item's last S
+      // has read it) and the K tiles, lane 1 the V tiles; the rings run on
+      // across items.
       const bool is_k = lane == 0;
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       bool ok = true;
-      if (is_k) {
-        mbar_expect_tx(q_full, TILE_BYTES);
-        tma_load_2d(sQ, &tmQK, q_full, h * HD, row_base + q0);
-        tma_load_2d(sQ + TILE_BYTES / 2, &tmQK, q_full, h * HD + 64, row_base + q0);
-      }
-      int issued = 0;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(&empty[s], ((j >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-        mbar_expect_tx(&full[s], TILE_BYTES);
-        const int kr = row_base + j * BKV;
+      int g = 0, nq = 0;  // tiles issued, Q tiles issued
+      for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+        int qt, bh;
+        fwd_item(i, n_qt, BH, qt, bh);
+        const int b = bh / H, h = bh % H, row_base = b * T, n_kv = qt + 1;
         if (is_k) {
-          uint8_t* k = sK + s * TILE_BYTES;
-          tma_load_2d(k, &tmQK, &full[s], a + h * HD, kr);
-          tma_load_2d(k + TILE_BYTES / 2, &tmQK, &full[s], a + h * HD + 64, kr);
-        } else {
-          // V as an MN-major operand: K-block kb (keys 64kb..), N chunk nc (hd 64nc..)
-          uint8_t* v = sV + s * TILE_BYTES;
-          for (int kb = 0; kb < 2; ++kb)
-            for (int nc = 0; nc < 2; ++nc)
-              tma_load_2d(v + kb * (TILE_BYTES / 2) + nc * 8192, &tmV, &full[s], 2 * a + h * HD + 64 * nc,
-                          kr + 64 * kb);
+          if (k > 0 && !mbar_wait(q_empty, (k - 1) & 1, abort_flag, err)) { ok = false; break; }
+          mbar_expect_tx(q_full, TILE_BYTES);
+          tma_load_2d(sQ, &tmQK, q_full, h * HD, row_base + qt * BQ);
+          tma_load_2d(sQ + TILE_BYTES / 2, &tmQK, q_full, h * HD + 64, row_base + qt * BQ);
+          ++nq;
         }
-        ++issued;
+        for (int j = 0; j < n_kv && ok; ++j, ++g) {
+          const int s = g & 1;
+          if (!mbar_wait(&empty[s], ((g >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          mbar_expect_tx(&full[s], TILE_BYTES);
+          const int kr = row_base + j * BKV;
+          if (is_k) {
+            uint8_t* kt = sK + s * TILE_BYTES;
+            tma_load_2d(kt, &tmQK, &full[s], a + h * HD, kr);
+            tma_load_2d(kt + TILE_BYTES / 2, &tmQK, &full[s], a + h * HD + 64, kr);
+          } else {
+            // V as an MN-major operand: K-block kb (keys 64kb..), N chunk nc (hd 64nc..)
+            uint8_t* v = sV + s * TILE_BYTES;
+            for (int kb = 0; kb < 2; ++kb)
+              for (int nc = 0; nc < 2; ++nc)
+                tma_load_2d(v + kb * (TILE_BYTES / 2) + nc * 8192, &tmV, &full[s], 2 * a + h * HD + 64 * nc,
+                            kr + 64 * kb);
+          }
+        }
       }
       // let every copy land before the CTA can exit
-      const uint64_t t0 = globaltimer_ns();
-      if (is_k)
-        while (!mbar_try_wait(q_full, 0)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j) {
+      if (is_k && nq > 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(q_full, (nq - 1) & 1)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
+      }
+      for (int j = (g > 2 ? g - 2 : 0); j < g; ++j) {
         const uint64_t t1 = globaltimer_ns();
         while (!mbar_try_wait(&full[j & 1], (j >> 1) & 1))
           if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
@@ -171,18 +194,28 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA
+      // One flattened sequence of steps over this CTA's items: iteration g
+      // issues S of step g, then PV of step g - 1 (which may belong to the
+      // previous item), so the next item's first S overlaps the last softmax.
       // S = Q K^T: A = Q (K-major), B = K (K-major), N = 128
       const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
                                ((uint32_t)(128 >> 4) << 24);
       // O += P V: A = P (K-major), B = V (MN-major), N = 128
       const uint32_t idesc_o = idesc_s | (1u << 16);
       const uint32_t aQ = smem_u32(sQ);
-      bool ok = mbar_wait(q_full, 0, abort_flag, err);
-      for (int j = 0; j <= n_kv && ok; ++j) {
-        if (j < n_kv) {
-          const int s = j & 1;
-          if (!mbar_wait(&k_full[s], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+      bool ok = true;
+      // S cursor (item index i_s, its k-th position k_s, step j_s) and PV cursor
+      int i_s = first, k_s = 0, j_s = 0, nkv_s = 0;
+      int i_p = first, k_p = 0, j_p = 0, nkv_p = 0;
+      if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = nkv_p = qt + 1; }
+      for (int g = 0; ok; ++g) {
+        const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
+        if (!s_left && !p_left) break;
+        if (s_left) {
+          const int s = g & 1;
+          if (j_s == 0 && !mbar_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&k_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aK = smem_u32(sK + s * TILE_BYTES);
 #pragma unroll
@@ -190,20 +223,40 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_mma(tmem + s * 128, kmaj_desc(aQ, k), kmaj_desc(aK, k), idesc_s, k > 0 ? 1u : 0u);
           tc_commit(&s_full[s]);
           tc_commit(&k_empty[s]);
+          if (++j_s == nkv_s) {  // the item's last S: Q may be replaced
+            tc_commit(q_empty);
+            j_s = 0;
+            ++k_s;
+            i_s += stride;
+            if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = qt + 1; }
+          }
         }
-        if (j >= 1) {
-          const int jp = j - 1, s = jp & 1;
-          if (!mbar_wait(&p_full[s], (jp >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&v_full[s], (jp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (p_left) {
+          const int gp = g - 1, s = gp & 1, ob = k_p & 1;
+          // the first PV of an item overwrites its O buffer: the softmax warps
+          // must have read that buffer for the item two positions back
+          if (j_p == 0 && k_p >= 2 && !mbar_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&v_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aP = smem_u32(sP + s * TILE_BYTES);
           const uint32_t aV = smem_u32(sV + s * TILE_BYTES);
 #pragma unroll
           for (int k = 0; k < BKV / 16; ++k)
-            tc_mma(tmem + 256, kmaj_desc(aP, k), mnmaj_desc(aV, k), idesc_o, (jp > 0 || k > 0) ? 1u : 0u);
+            tc_mma(tmem + 256 + ob * 128, kmaj_desc(aP, k), mnmaj_desc(aV, k), idesc_o,
+                   (j_p > 0 || k > 0) ? 1u : 0u);
           tc_commit(&p_free[s]);
           tc_commit(&v_empty[s]);
-          if (jp == n_kv - 1) tc_commit(o_full);
+          if (++j_p == nkv_p) {  // the item's last PV: O is complete
+            tc_commit(&o_full[ob]);
+            j_p = 0;
+            ++k_p;
+            i_p += stride;
+            if (i_p < total) { int qt, bh; fwd_item(i_p, n_qt, BH, qt, bh); nkv_p = qt + 1; }
+          }
         }
       }
     }
@@ -211,126 +264,136 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------------ softmax
     const int q = warp & 3;
     const int r = q * 32 + lane;               // row within the tile
-    const int qpos = q0 + r;                   // query position in the sequence
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float c = rsqrtf((float)HD) * LOG2E;
-    float m_use = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int s = j & 1;
-      if (!warp_wait(&s_full[s], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      tc_fence_after();
-      float sv[128];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t base = tmem + lane_off + s * 128;
-        tmem_ld32_nowait(base, r0);
-        tmem_ld32_nowait(base + 32, r1);
-        tmem_ld32_nowait(base + 64, r2);
-        tmem_ld32_nowait(base + 96, r3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = __uint_as_float(r0[i]);
-          sv[32 + i] = __uint_as_float(r1[i]);
-          sv[64 + i] = __uint_as_float(r2[i]);
-          sv[96 + i] = __uint_as_float(r3[i]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[s]);  // the S buffer may be overwritten
-      const int k0 = j * BKV;
-      if (k0 + BKV - 1 > qpos) {  // causal mask on the diagonal tile
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (k0 + i > qpos) sv[i] = -INFINITY;
-      }
-      // row max of the raw scores (the scale c > 0 commutes with max), as 8
-      // independent partial maxima so the reduction is not one long chain
-      float pm[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) pm[u] = sv[u];
-#pragma unroll
-      for (int i = 8; i < 128; ++i) pm[i & 7] = fmaxf(pm[i & 7], sv[i]);
-      const float mx = c * fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      if (j == 0) {
-        m_use = mx;
-      } else if (__any_sync(0xffffffffu, mx > m_use + RESCALE_THRESHOLD)) {
-        // grow the max in use: O_{<j} and l scale by 2^(m_old - m_new); the
-        // previous PV product must have landed in O first.  The decision is
-        // warp-wide (the TMEM accesses below are warp-collective); rows whose
-        // max did not grow rescale by exactly 1.
-        const float m_new = fmaxf(m_use, mx);
-        const float alpha = exp2f(m_use - m_new);
-        if (!warp_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+    int g = 0;  // global step
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int qt, bh;
+      fwd_item(i, n_qt, BH, qt, bh);
+      const int b = bh / H, h = bh % H, row_base = b * T, n_kv = qt + 1;
+      const int qpos = qt * BQ + r;              // query position in the sequence
+      const int ob = k & 1;
+      float m_use = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_kv; ++j, ++g) {
+        const int s = g & 1;
+        if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ob = tmem + lane_off + 256;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32_nowait(ob + cc * 32, o);
+        float sv[128];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          const uint32_t base = tmem + lane_off + s * 128;
+          tmem_ld32_nowait(base, r0);
+          tmem_ld32_nowait(base + 32, r1);
+          tmem_ld32_nowait(base + 64, r2);
+          tmem_ld32_nowait(base + 96, r3);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(ob + cc * 32, o);
+          for (int ii = 0; ii < 32; ++ii) {
+            sv[ii] = __uint_as_float(r0[ii]);
+            sv[32 + ii] = __uint_as_float(r1[ii]);
+            sv[64 + ii] = __uint_as_float(r2[ii]);
+            sv[96 + ii] = __uint_as_float(r3[ii]);
+          }
         }
-        tmem_wait_st();
-        l *= alpha;
-        m_use = m_new;
-      }
-      // P_j = exp2(s - m_use) as bf16 into the P buffer of this parity, once
-      // the PV product that read it two tiles ago is done
-      if (j >= 2 && !warp_wait(&p_free[s], ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      uint8_t* pb = sP + s * TILE_BYTES;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial sums
-      const float nm = -m_use;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[s]);  // the S buffer may be overwritten
+        const int k0 = j * BKV;
+        if (k0 + BKV - 1 > qpos) {  // causal mask on the diagonal tile
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 keys
-        float p[8];
+          for (int ii = 0; ii < 128; ++ii)
+            if (k0 + ii > qpos) sv[ii] = -INFINITY;
+        }
+        // row max of the raw scores (the scale c > 0 commutes with max), as 8
+        // independent partial maxima so the reduction is not one long chain
+        float pm[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { p[e] = fast_exp2(fmaf(sv[ch * 8 + e], c, nm)); ps[e] += p[e]; }
-        uint4 w;
-        __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]), b1 = __floats2bfloat162_rn(p[2], p[3]);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]), b3 = __floats2bfloat162_rn(p[6], p[7]);
-        w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-        w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-        const int sub = ch >> 3, jj = ch & 7;
-        *reinterpret_cast<uint4*>(pb + sub * (TILE_BYTES / 2) + r * 128 + ((jj ^ (r & 7)) << 4)) = w;
+        for (int u = 0; u < 8; ++u) pm[u] = sv[u];
+#pragma unroll
+        for (int ii = 8; ii < 128; ++ii) pm[ii & 7] = fmaxf(pm[ii & 7], sv[ii]);
+        const float mx = c * fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        if (j == 0) {
+          m_use = mx;
+        } else if (__any_sync(0xffffffffu, mx > m_use + RESCALE_THRESHOLD)) {
+          // grow the max in use: O_{<j} and l scale by 2^(m_old - m_new); the
+          // previous PV product must have landed in O first.  The decision is
+          // warp-wide (the TMEM accesses below are warp-collective); rows
+          // whose max did not grow rescale by exactly 1.
+          const float m_new = fmaxf(m_use, mx);
+          const float alpha = exp2f(m_use - m_new);
+          if (!warp_wait(&p_free[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t obase = tmem + lane_off + 256 + ob * 128;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32_nowait(obase + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ii = 0; ii < 32; ++ii) o[ii] = __float_as_uint(__uint_as_float(o[ii]) * alpha);
+            tmem_st32(obase + cc * 32, o);
+          }
+          tmem_wait_st();
+          l *= alpha;
+          m_use = m_new;
+        }
+        // P = exp2(s - m_use) as bf16 into the P buffer of this parity, once
+        // the PV product that read it two steps ago is done
+        if (g >= 2 && !warp_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        uint8_t* pb = sP + s * TILE_BYTES;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial sums
+        const float nm = -m_use;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 keys
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) { p[e] = fast_exp2(fmaf(sv[ch * 8 + e], c, nm)); ps[e] += p[e]; }
+          uint4 w;
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]), b1 = __floats2bfloat162_rn(p[2], p[3]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]), b3 = __floats2bfloat162_rn(p[6], p[7]);
+          w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
+          w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
+          const int sub = ch >> 3, jj = ch & 7;
+          *reinterpret_cast<uint4*>(pb + sub * (TILE_BYTES / 2) + r * 128 + ((jj ^ (r & 7)) << 4)) = w;
+        }
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[s]);
       }
-      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[s]);
-    }
-    // ---------------------------------------------------------------- epilogue
-    if (__all_sync(0xffffffffu, ok) && warp_wait(o_full, 0, abort_flag, err)) {
+      if (!ok) break;
+      // ------------------------------------------------------------ item epilogue
+      if (!warp_wait(&o_full[ob], (k >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.f / l;
-      const uint32_t ob = tmem + lane_off + 256;
+      const uint32_t obase = tmem + lane_off + 256 + ob * 128;
       bf16* orow = out + ((long long)row_base + qpos) * a + h * HD;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        tmem_ld32_nowait(ob + cc * 32, o);
+        tmem_ld32_nowait(obase + cc * 32, o);
         tmem_wait_ld();
         if (qpos < T) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
+          for (int ii = 0; ii < 32; ii += 8) {
             uint4 w;
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-            __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[ii]) * inv, __uint_as_float(o[ii + 1]) * inv);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[ii + 2]) * inv, __uint_as_float(o[ii + 3]) * inv);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[ii + 4]) * inv, __uint_as_float(o[ii + 5]) * inv);
+            __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[ii + 6]) * inv, __uint_as_float(o[ii + 7]) * inv);
             w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
             w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-            *reinterpret_cast<uint4*>(orow + cc * 32 + i) = w;
+            *reinterpret_cast<uint4*>(orow + cc * 32 + ii) = w;
           }
         }
       }
       if (qpos < T) lse_out[(long long)bh * T + qpos] = m_use + log2f(l);  // log2 units
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[ob]);  // this O buffer may be overwritten
     }
   }
   tc_fence_before();

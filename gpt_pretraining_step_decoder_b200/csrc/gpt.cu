@@ -828,9 +828,11 @@ static int attention_fwd(gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
     CUtensorMap tqk, tv;
     TRY(make_tmap(&tqk, qkv, 3 * a, ntok, 3 * a, 64, 128));
     TRY(make_tmap(&tv, qkv, 3 * a, ntok, 3 * a, 64, 64));
-    dim3 g(cdiv(c.seq_len, fatc::BQ), c.micro_batch * c.n_head);
-    ++g_launches; fatc::fa_tc_fwd_kernel<<<g, fatc::THREADS, fatc::SMEM_BYTES, m->st>>>(
-        tqk, tv, reinterpret_cast<bf16*>(o), lse, c.seq_len, c.n_head, m->err());
+    // persistent: one CTA per SM (or per item when there are fewer)
+    const long long items = (long long)cdiv(c.seq_len, fatc::BQ) * c.micro_batch * c.n_head;
+    const int grid = items < device_sms() ? (int)items : device_sms();
+    ++g_launches; fatc::fa_tc_fwd_kernel<<<grid, fatc::THREADS, fatc::SMEM_BYTES, m->st>>>(
+        tqk, tv, reinterpret_cast<bf16*>(o), lse, c.seq_len, c.n_head, c.micro_batch * c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
   }
