@@ -86,6 +86,30 @@ template <typename act_t>
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N,
                                      GemmEpilogue e) {
   const long long total = (long long)M * N;
+  const bool vec = (N % 4) == 0 && (e.ldc % 4) == 0 && (e.mode == EPI_ACCUM_F32 || e.mode == EPI_STORE_F32);
+  if (vec) {
+    // four consecutive columns of one row per thread (same sum order per element)
+    const long long total4 = total / 4;
+    for (long long i4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; i4 < total4;
+         i4 += (long long)gridDim.x * blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < S; ++s) {
+        const float4 v = reinterpret_cast<const float4*>(part + (long long)s * total)[i4];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const long long i = i4 * 4, m = i / N, n = i % N;
+      float4* c = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.C) + m * e.ldc + n);
+      if (e.mode == EPI_ACCUM_F32 && e.beta) {
+        const float4 o = *c;
+        acc.x = o.x + acc.x * e.alpha; acc.y = o.y + acc.y * e.alpha;
+        acc.z = o.z + acc.z * e.alpha; acc.w = o.w + acc.w * e.alpha;
+      } else {
+        acc.x *= e.alpha; acc.y *= e.alpha; acc.z *= e.alpha; acc.w *= e.alpha;
+      }
+      *c = acc;
+    }
+    return;
+  }
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     float acc = 0.f;
