@@ -775,6 +775,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 
 // ---------------------------------------------------------------- dQ
 // 10 warps as above; compute warps split the 64 key columns in halves.
+// Persistent like the forward: one CTA per SM over the (query tile,
+// sequence, head) items heaviest first; the K/V ring and the S/dP and dS
+// buffers run on across items, Q/dO for the next item load once the item's
+// last S/dP has read them, and dQ alternates between two TMEM accumulators.
 // smem: Q, dO [128 x 128] (32 KB each); per stage K_j, V_j [64 x 128] (16 KB
 // each, 4 stages); per buffer dS [128 queries x 64 keys] (16 KB, 2 buffers).
 constexpr int DQ_STAGES = 4;
@@ -783,7 +787,8 @@ constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 2 * PT + 1024 + 256;
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
                         const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse2,
-                        const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+                        const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, int BH,
+                        unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -794,35 +799,43 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint8_t* sS = sV + DQ_STAGES * QT64;       // dS [2]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sS + 2 * PT);
   uint64_t* q_full = bars;                      // 1
-  uint64_t* kv_full = q_full + 1;               // DQ_STAGES
+  uint64_t* q_empty = q_full + 1;               // 1 (the item's last S/dP have read Q and dO)
+  uint64_t* kv_full = q_empty + 1;              // DQ_STAGES
   uint64_t* kv_empty = kv_full + DQ_STAGES;     // DQ_STAGES
   uint64_t* s_full = kv_empty + DQ_STAGES;      // 2
   uint64_t* s_empty = s_full + 2;               // 2
   uint64_t* p_full = s_empty + 2;               // 2
   uint64_t* p_free = p_full + 2;                // 2
-  uint64_t* o_full = p_free + 2;                // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
-  static_assert((2 + 2 * DQ_STAGES + 8) * 8 + 8 <= 256, "barrier area");
+  uint64_t* o_full = p_free + 2;                // 2 (per dQ buffer: the item's last product is done)
+  uint64_t* o_empty = o_full + 2;               // 2 (per dQ buffer: the compute warps have read it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  static_assert((2 + 2 * DQ_STAGES + 12) * 8 + 8 <= 256, "barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;  // latest query tiles (most key tiles) first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int a = H * 128;
-  const int q0 = qt * 128;
-  const int row_base = b * T;
-  const int n_it = min((q0 + 128) / 64, (T + 63) / 64);  // key tiles of 64 up to the diagonal
+  const int n_qt = (T + 127) / 128;
+  const int total = n_qt * BH;
+  const int first = blockIdx.x, stride = gridDim.x;
+  // item i (heaviest first): query tile qt, (sequence, head) bh, key tiles of 64 up to the diagonal
+  auto item = [&](int i, int& qt, int& bh, int& n_it) {
+    qt = n_qt - 1 - i / BH;
+    bh = i % BH;
+    n_it = min((qt * 128 + 128) / 64, (T + 63) / 64);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 8);   // one arrival per compute warp
       mbar_init(&p_full[s], 8);
       mbar_init(&p_free[s], 1);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 8);
     }
-    mbar_init(o_full, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -835,36 +848,44 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S: 0, 64; dP: 128, 192; dQ: 256
+  const uint32_t tmem = *tmem_slot;  // S: 0, 64; dP: 128, 192; dQ: 256 and 384 (alternating per item)
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- TMA
       bool ok = true;
-      mbar_expect_tx(q_full, 2 * KV_T);
-      tma_load_2d(sQ, &tm128, q_full, h * 128, row_base + q0);
-      tma_load_2d(sQ + KV_T / 2, &tm128, q_full, h * 128 + 64, row_base + q0);
-      // dO [128 x 128] through the 64-row map: half hf (64 columns) x row block rb
-      for (int hf = 0; hf < 2; ++hf)
-        for (int rb = 0; rb < 2; ++rb)
-          tma_load_2d(sO + hf * (KV_T / 2) + rb * 8192, &tmDO, q_full, h * 128 + 64 * hf, row_base + q0 + 64 * rb);
-      int issued = 0;
-      for (int j = 0; j < n_it && ok; ++j) {
-        const int s = j % DQ_STAGES;
-        if (!mbar_wait(&kv_empty[s], ((j / DQ_STAGES) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-        mbar_expect_tx(&kv_full[s], 2 * QT64);
-        const int kr = row_base + j * 64;
-        uint8_t* k = sK + s * QT64;
-        uint8_t* v = sV + s * QT64;
-        tma_load_2d(k, &tm64, &kv_full[s], a + h * 128, kr);
-        tma_load_2d(k + QT64 / 2, &tm64, &kv_full[s], a + h * 128 + 64, kr);
-        tma_load_2d(v, &tm64, &kv_full[s], 2 * a + h * 128, kr);
-        tma_load_2d(v + QT64 / 2, &tm64, &kv_full[s], 2 * a + h * 128 + 64, kr);
-        ++issued;
+      int g = 0, nq = 0;
+      for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+        int qt, bh, n_it;
+        item(i, qt, bh, n_it);
+        const int b = bh / H, h = bh % H, row_base = b * T, q0 = qt * 128;
+        if (k > 0 && !mbar_wait(q_empty, (k - 1) & 1, abort_flag, err)) { ok = false; break; }
+        mbar_expect_tx(q_full, 2 * KV_T);
+        tma_load_2d(sQ, &tm128, q_full, h * 128, row_base + q0);
+        tma_load_2d(sQ + KV_T / 2, &tm128, q_full, h * 128 + 64, row_base + q0);
+        // dO [128 x 128] through the 64-row map: half hf (64 columns) x row block rb
+        for (int hf = 0; hf < 2; ++hf)
+          for (int rb = 0; rb < 2; ++rb)
+            tma_load_2d(sO + hf * (KV_T / 2) + rb * 8192, &tmDO, q_full, h * 128 + 64 * hf, row_base + q0 + 64 * rb);
+        ++nq;
+        for (int j = 0; j < n_it && ok; ++j, ++g) {
+          const int s = g % DQ_STAGES;
+          if (!mbar_wait(&kv_empty[s], ((g / DQ_STAGES) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          mbar_expect_tx(&kv_full[s], 2 * QT64);
+          const int kr = row_base + j * 64;
+          uint8_t* kt = sK + s * QT64;
+          uint8_t* v = sV + s * QT64;
+          tma_load_2d(kt, &tm64, &kv_full[s], a + h * 128, kr);
+          tma_load_2d(kt + QT64 / 2, &tm64, &kv_full[s], a + h * 128 + 64, kr);
+          tma_load_2d(v, &tm64, &kv_full[s], 2 * a + h * 128, kr);
+          tma_load_2d(v + QT64 / 2, &tm64, &kv_full[s], 2 * a + h * 128 + 64, kr);
+        }
       }
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(q_full, 0)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
-      for (int j = (issued > DQ_STAGES ? issued - DQ_STAGES : 0); j < issued; ++j) {
+      if (nq > 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(q_full, (nq - 1) & 1)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
+      }
+      for (int j = (g > DQ_STAGES ? g - DQ_STAGES : 0); j < g; ++j) {
         const uint64_t t1 = globaltimer_ns();
         while (!mbar_try_wait(&kv_full[j % DQ_STAGES], (j / DQ_STAGES) & 1))
           if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
@@ -873,15 +894,24 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA
+      // One flattened sequence over this CTA's items: iteration g issues S/dP
+      // of step g, then the dQ product of step g - 1 (possibly of the
+      // previous item).
       const uint32_t id_s = idesc(64, false);   // S = Q K^T, dP = dO V^T (N = 64 keys)
       const uint32_t id_g = idesc(128, true);   // dQ += dS K (N = 128, B MN-major)
       const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
-      bool ok = mbar_wait(q_full, 0, abort_flag, err);
-      for (int j = 0; j <= n_it && ok; ++j) {
-        if (j < n_it) {
-          const int st = j % DQ_STAGES, s = j & 1;
-          if (!mbar_wait(&kv_full[st], (j / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[s], ((j >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+      bool ok = true;
+      int i_s = first, k_s = 0, j_s = 0, n_s = 0;
+      int i_p = first, k_p = 0, j_p = 0, n_p = 0;
+      if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); n_p = n_s; }
+      for (int g = 0; ok; ++g) {
+        const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
+        if (!s_left && !p_left) break;
+        if (s_left) {
+          const int st = g % DQ_STAGES, s = g & 1;
+          if (j_s == 0 && !mbar_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&kv_full[st], (g / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(&s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
 #pragma unroll
@@ -891,18 +921,35 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           for (int k = 0; k < 8; ++k)
             tc_mma(tmem + 128 + s * 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
           tc_commit(&s_full[s]);
+          if (++j_s == n_s) {  // the item's last S/dP: Q and dO may be replaced
+            tc_commit(q_empty);
+            j_s = 0;
+            ++k_s;
+            i_s += stride;
+            if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); }
+          }
         }
-        if (j >= 1) {
-          const int jp = j - 1, s = jp & 1, st = jp % DQ_STAGES;
-          if (!mbar_wait(&p_full[s], (jp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (p_left) {
+          const int gp = g - 1, s = gp & 1, st = gp % DQ_STAGES, ob = k_p & 1;
+          if (j_p == 0 && k_p >= 2 && !mbar_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aS = smem_u32(sS + s * PT), aK = smem_u32(sK + st * QT64);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma(tmem + 256, kdesc64(aS, k), mndesc(aK, QT64 / 2, k), id_g, (jp > 0 || k > 0) ? 1u : 0u);
+            tc_mma(tmem + 256 + ob * 128, kdesc64(aS, k), mndesc(aK, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
           tc_commit(&p_free[s]);
           tc_commit(&kv_empty[st]);
-          if (jp == n_it - 1) tc_commit(o_full);
+          if (++j_p == n_p) {  // the item's last product: dQ is complete
+            tc_commit(&o_full[ob]);
+            j_p = 0;
+            ++k_p;
+            i_p += stride;
+            if (i_p < total) { int qt, bh; item(i_p, qt, bh, n_p); }
+          }
         }
       }
     }
@@ -910,47 +957,57 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     // ---------------------------------------------------------------- dS
     const int q4 = warp & 3, half = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
-    const int qpos = q0 + r;
-    const bool valid = qpos < T;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
-    const float L = valid ? lse2[(long long)bh * T + qpos] : 0.f;  // log2 units
-    const float Dq = valid ? Dv[(long long)bh * T + qpos] : 0.f;
     bool ok = true;
-    for (int j = 0; j < n_it; ++j) {
-      const int s = j & 1;
-      if (!warp_wait(&s_full[s], (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      tc_fence_after();
-      float sv[32], dp[32];
-      {
-        uint32_t r0[32], r1[32];
-        tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
-        tmem_ld32_nowait(tmem + lane_off + 128 + s * 64 + half * 32, r1);
-        tmem_wait_ld();
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int qt, bh, n_it;
+      item(i, qt, bh, n_it);
+      const int b = bh / H, h = bh % H, row_base = b * T;
+      const int qpos = qt * 128 + r;
+      const bool valid = qpos < T;
+      const float L = valid ? lse2[(long long)bh * T + qpos] : 0.f;  // log2 units
+      const float Dq = valid ? Dv[(long long)bh * T + qpos] : 0.f;
+      const int ob = k & 1;
+      for (int j = 0; j < n_it; ++j, ++g) {
+        const int s = g & 1;
+        if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        float sv[32], dp[32];
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
+          tmem_ld32_nowait(tmem + lane_off + 128 + s * 64 + half * 32, r1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[s]);
-      const int kbase = j * 64 + half * 32;
+          for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[s]);
+        const int kbase = j * 64 + half * 32;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const bool live = valid && (kbase + e <= qpos);
-        const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
-        dp[e] = p * (dp[e] - Dq);
+        for (int e = 0; e < 32; ++e) {
+          const bool live = valid && (kbase + e <= qpos);
+          const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
+          dp[e] = p * (dp[e] - Dq);
+        }
+        if (g >= 2 && !warp_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        st_half_row(sS + s * PT, r, half, dp);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[s]);
       }
-      if (j >= 2 && !warp_wait(&p_free[s], ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      st_half_row(sS + s * PT, r, half, dp);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[s]);
-    }
-    if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
+      if (!ok) break;
+      if (!warp_wait(&o_full[ob], (k >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128 + half * 64;
-      row64_out(tmem + lane_off + 256 + half * 64, rsqrtf(128.f), qrow, valid);
+      row64_out(tmem + lane_off + 256 + ob * 128 + half * 64, rsqrtf(128.f), qrow, valid);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[ob]);  // this dQ buffer may be overwritten
     }
   }
   tc_fence_before();

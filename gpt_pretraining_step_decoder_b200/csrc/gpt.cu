@@ -868,12 +868,13 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
     TRY(make_tmap(&t64, qkv, 3 * a, N, 3 * a, 64, 64));
     TRY(make_tmap(&tdo, dout, a, N, a, 64, 64));
     dim3 gk(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
-    dim3 gq(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
     bf16* g16 = reinterpret_cast<bf16*>(dqkv);
     ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<gk, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st>>>(
         t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
-    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<gq, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
-        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
+    const long long dq_items = (long long)cdiv(c.seq_len, 128) * c.micro_batch * c.n_head;
+    const int dq_grid = dq_items < device_sms() ? (int)dq_items : device_sms();  // persistent
+    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<dq_grid, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
+        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, c.micro_batch * c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
   }
