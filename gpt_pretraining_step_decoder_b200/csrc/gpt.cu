@@ -794,6 +794,33 @@ static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long 
   return GPT_OK;
 }
 
+// Dynamic shared memory above the default 48 KB needs the kernel's opt-in.
+template <typename K>
+static int allow_smem(K* kernel, size_t bytes) {
+  if (bytes > 48 * 1024)
+    CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  return GPT_OK;
+}
+
+template <typename tab_t, int MAXT, bool STAGE>
+static int launch_table_chunk(tab_t* table, float* state, int d, const float* grad, const uint32_t* skeys,
+                              const int32_t* perm, int n, long long n_rows, const SortWs& w, float lr, float beta,
+                              float eps, int nt, long long nchunks, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    CUDA_TRY(cudaFuncSetAttribute(table_chunk_kernel<tab_t, MAXT, STAGE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)table_chunk_smem<tab_t>(MAXT, STAGE)));
+    // all of the unified L1 / shared storage as shared memory: occupancy is set by it
+    CUDA_TRY(cudaFuncSetAttribute(table_chunk_kernel<tab_t, MAXT, STAGE>,
+                                  cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
+    attr = true;
+  }
+  ++g_launches;
+  table_chunk_kernel<tab_t, MAXT, STAGE><<<(unsigned)nchunks, nt, table_chunk_smem<tab_t>(nt, STAGE), st>>>(
+      table, state, d, grad, skeys, perm, n, n_rows, w.part_head, w.part_tail, lr, beta, eps);
+  return GPT_OK;
+}
+
 template <typename tab_t>
 static int table_update(const SortWs& w, tab_t* table, float* state, long long n_rows, int d,
                         const int32_t* rows, const float* grad, int n, float lr, float beta, float eps,
@@ -802,11 +829,21 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const int32_t* perm;
   TRY(bucket_by_key(w, rows, n, n_rows, &skeys, &perm, uniq_out, n_uniq_out, err, st));
   const long long nchunks = (n + CHUNK - 1) / CHUNK;
-  WITH_NV(d, ++g_launches; table_chunk_kernel<NV, tab_t><<<grid_for(nchunks * 32, 128), 128, 0, st>>>(
-      table, state, d, grad, skeys, perm, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
-  const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;  // <= 24 KB (d <= 2048)
-  WITH_NV(d, ++g_launches; table_chain_kernel<NV, tab_t><<<(unsigned)nchunks, CHAIN_WARPS * 32, chain_smem, st>>>(
-      table, state, d, skeys, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
+  const int chunk_threads = (d / 4 + 31) / 32 * 32;  // one float4 column group a thread (d <= 2048)
+  if (chunk_threads <= 256) {
+    TRY((launch_table_chunk<tab_t, 256, true>(table, state, d, grad, skeys, perm, n, n_rows, w, lr, beta, eps,
+                                              chunk_threads, nchunks, st)));
+  } else {
+    // rows wider than 1024: fp32 table values no longer fit beside the gradients
+    constexpr bool stage = sizeof(tab_t) == 2;
+    TRY((launch_table_chunk<tab_t, 512, stage>(table, state, d, grad, skeys, perm, n, n_rows, w, lr, beta, eps,
+                                               chunk_threads, nchunks, st)));
+  }
+  const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;  // <= 56 KB (d <= 2048)
+  const unsigned chain_grid = (unsigned)((nchunks + CHAIN_WARPS - 1) / CHAIN_WARPS);
+  WITH_NV(d, TRY(allow_smem(table_chain_kernel<NV, tab_t>, chain_smem)); ++g_launches;
+          table_chain_kernel<NV, tab_t><<<chain_grid, CHAIN_WARPS * 32, chain_smem, st>>>(
+              table, state, d, skeys, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
   LAUNCH_CHECK();
   return GPT_OK;
 }
@@ -1097,8 +1134,11 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const long long nchunks = (N + CHUNK - 1) / CHUNK;
     WITH_NV(d, ++g_launches; emb_chunk_kernel<NV, act_t><<<grid_for(nchunks * 32, 128), 128, 0, st>>>(
         Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, N, V, w.part_head, w.part_tail););
-    WITH_NV(d, ++g_launches; emb_chain_kernel<NV><<<(unsigned)nchunks, CHAIN_WARPS * 32, (size_t)(CHAIN_WARPS - 1) * d * 4, st>>>(
-        Gp("wte"), d, skeys, N, V, w.part_head, w.part_tail););
+    const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;
+    const unsigned chain_grid = (unsigned)((nchunks + CHAIN_WARPS - 1) / CHAIN_WARPS);
+    WITH_NV(d, TRY(allow_smem(emb_chain_kernel<NV>, chain_smem)); ++g_launches;
+            emb_chain_kernel<NV><<<chain_grid, CHAIN_WARPS * 32, chain_smem, st>>>(
+                Gp("wte"), d, skeys, N, V, w.part_head, w.part_tail););
     LAUNCH_CHECK();
   }
   const float lr_t = lr * c.lr_mult_table;

@@ -11,12 +11,14 @@
 // int32 rows directly.  No atomics anywhere, so sums are formed in position
 // order and results are bit-reproducible.
 //
-// Update: the sorted positions are cut into fixed chunks of 16; one warp owns
-// a chunk and finds the runs of equal rows in it with ballots.  A run that
-// lies inside the chunk is finished by that warp (sum -> mean square -> row
-// state -> row update).  A run that crosses chunk boundaries leaves one
-// partial sum per chunk it touches; a second launch adds those partials in
-// chunk order and finishes the row.  Every row is written by exactly one warp.
+// Update: the sorted positions are cut into fixed chunks of 16; one block owns
+// a chunk (each thread four columns of every row), its warps find the runs of
+// equal rows in it with ballots.  A run that lies inside the chunk is finished
+// by that block (sum -> mean square -> row state -> row update).  A run that
+// crosses chunk boundaries leaves one partial sum per chunk it touches; a
+// second launch adds those partials in chunk order and finishes the row.
+// Every row is written by exactly one block.  (The token-embedding gradient
+// uses the same bucketing with one warp per chunk.)
 #pragma once
 #include "common.cuh"
 #include "layers.cuh"
@@ -27,7 +29,8 @@ constexpr int RADIX_FUSED_MAX_BLOCKS = 256;  // above this, offsets come from a 
 constexpr int CHUNK = 16;            // sorted positions per warp in the update (<= 32)
 
 // keys per thread so that a sort of n keys runs on about 96 blocks (or on
-// as many 2048-key tiles as it needs beyond that)
+// as many 2048-key tiles as it needs beyond that; measured on B200, 192
+// blocks of fewer keys are no faster)
 static inline int radix_items(long long n) {
   int it = 1;
   while (it < RADIX_MAX_ITEMS && (n + (long long)RADIX_THREADS * it - 1) / ((long long)RADIX_THREADS * it) > 96) it <<= 1;
@@ -144,13 +147,21 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_hist_kernel(const uint32_
   __syncthreads();
   const long long base = (long long)blockIdx.x * RADIX_THREADS * items;
   const uint32_t lt = (1u << lane) - 1u;
-  for (int round = 0; round < items; ++round) {
+  // all of the tile's keys are requested before any is counted
+  uint32_t dg[RADIX_MAX_ITEMS];
+#pragma unroll
+  for (int round = 0; round < RADIX_MAX_ITEMS; ++round) {
     const long long idx = base + (long long)round * RADIX_THREADS + threadIdx.x;
-    uint32_t dgt = 256u;
-    if (idx < n) {
+    dg[round] = 256u;
+    if (round < items && idx < n) {
       bool ok;
-      dgt = (radix_key(keys, raw, idx, key_range, ok) >> shift) & 255u;
+      dg[round] = (radix_key(keys, raw, idx, key_range, ok) >> shift) & 255u;
     }
+  }
+#pragma unroll
+  for (int round = 0; round < RADIX_MAX_ITEMS; ++round) {
+    if (round >= items) break;
+    const uint32_t dgt = dg[round];
     const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
     // the lowest lane of each digit group adds the group's size: one writer
     // per (warp, digit), so no atomics are needed
@@ -227,25 +238,36 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_scatter_kernel(
     running[threadIdx.x] = wbase + incl - total + before;
   }
   const long long base = (long long)blockIdx.x * RADIX_THREADS * items;
-  for (int round = 0; round < items; ++round) {
+  // all of the tile's keys and values are requested before any is ranked
+  uint32_t kk[RADIX_MAX_ITEMS];
+  int32_t vv[RADIX_MAX_ITEMS];
+#pragma unroll
+  for (int round = 0; round < RADIX_MAX_ITEMS; ++round) {
+    const long long idx = base + (long long)round * RADIX_THREADS + threadIdx.x;
+    kk[round] = 0;
+    vv[round] = 0;
+    if (round < items && idx < n) {
+      bool ok;
+      kk[round] = radix_key(keys_in, raw, idx, key_range, ok);
+      if (raw != nullptr) {
+        vv[round] = ok ? (int32_t)idx : -1;
+        if (!ok) set_error(err, GPT_EBIT_INPUT);
+      } else {
+        vv[round] = vals_in[idx];
+      }
+    }
+  }
+#pragma unroll
+  for (int round = 0; round < RADIX_MAX_ITEMS; ++round) {
+    if (round >= items) break;
     __syncthreads();
     for (int i = threadIdx.x; i < NW * 256; i += RADIX_THREADS) (&wcount[0][0])[i] = 0;
     __syncthreads();
     const long long idx = base + (long long)round * RADIX_THREADS + threadIdx.x;
     const bool valid = idx < n;
-    uint32_t key = 0, dgt = 256;  // 256 = no digit (invalid lane)
-    int32_t val = 0;
-    if (valid) {
-      bool ok;
-      key = radix_key(keys_in, raw, idx, key_range, ok);
-      if (raw != nullptr) {
-        val = ok ? (int32_t)idx : -1;
-        if (!ok) set_error(err, GPT_EBIT_INPUT);
-      } else {
-        val = vals_in[idx];
-      }
-      dgt = (key >> shift) & 255u;
-    }
+    const uint32_t key = kk[round];
+    const int32_t val = vv[round];
+    const uint32_t dgt = valid ? (key >> shift) & 255u : 256u;  // 256 = no digit (invalid lane)
     const uint32_t peers = __match_any_sync(0xffffffffu, dgt);
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t rank_in_warp = __popc(peers & lt);
@@ -464,66 +486,140 @@ __device__ __forceinline__ void add_row(float (&a)[NV][4], const float (&b)[NV][
     for (int i = 0; i < 4; ++i) a[j][i] += b[j][i];
 }
 
-// Sorted positions per step of a chunk warp: the position's gradient row and
-// (for a run that ends there and finishes in this chunk) the table row and
-// state are loaded together.  One position per step keeps the kernel near 80
-// registers so 24 warps fit on an SM; measured on the 2M x 768 table, that
-// beats two or four positions per step at 12 or 8 warps.
-template <int NV>
-struct TabU {
-  static constexpr int value = 1;
-};
+// Sum of each of 16 values over the 32 lanes of a warp in 16 shuffles (a
+// butterfly that halves the list at every step instead of 16 separate
+// reductions).  On return lane l holds the total of value (l >> 1) & 15; the
+// grouping is fixed, so the result is reproducible.
+__device__ __forceinline__ float warp_sum16(float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int h = 8; h >= 1; h >>= 1) {
+    const bool hi = (lane >> 1) & h;  // bit of the lane that picks the kept half
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float keep = hi ? v[i + h] : v[i], give = hi ? v[i] : v[i + h];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, give, 2 * h);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
 
-// One warp per chunk of sorted positions: runs inside the chunk are summed
-// and applied; a run's part that touches a chunk boundary goes to part_tail[c]
-// (the chunk's first run, begun earlier) or part_head[c] (its last run, going
-// on).
-template <int NV, typename tab_t>
-__global__ void __launch_bounds__(128, NV <= 6 ? 6 : (NV <= 8 ? 4 : 2)) table_chunk_kernel(
+// Asynchronous global -> shared copies of one thread's own values (Ampere-style
+// cp.async): the data lands in shared memory without holding registers while
+// in flight, and after the wait the issuing thread reads it back itself.
+template <int BYTES>
+__device__ __forceinline__ void cp_async_own(void* dst, const void* src) {
+  static_assert(BYTES == 8 || BYTES == 16, "cp.async size");
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  if constexpr (BYTES == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_own() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Dynamic shared memory of table_chunk_kernel for a block of nt threads.
+template <typename tab_t>
+static inline size_t table_chunk_smem(int nt, bool stage_rows) {
+  return (size_t)CHUNK * nt * (sizeof(float4) + (stage_rows ? sizeof(typename Raw4<tab_t>::type) : 0));
+}
+
+// One block per chunk of CHUNK sorted positions; thread t owns columns
+// [4t, 4t + 4) of every row, so a block has d / 4 threads rounded up to whole
+// warps (at most MAXT).  Every gradient value of the chunk and (STAGE_ROWS)
+// the table values of the rows whose runs end inside it are requested into
+// shared memory before any is used: a chunk costs one memory round trip after
+// its keys, instead of one per position, and holds no registers meanwhile, so
+// the shared memory a block takes sets how many chunks an SM has in flight.
+// Runs inside the chunk are summed in position order and applied (their sums
+// of squares reduced across the block at once); a run's part that touches a
+// chunk boundary goes to part_tail[c] (the chunk's first run, begun earlier)
+// or part_head[c] (its last run, going on).  Without STAGE_ROWS (rows too
+// wide for the staging buffer) the table values are read when applied.
+template <typename tab_t, int MAXT, bool STAGE_ROWS>
+__global__ void __launch_bounds__(MAXT) table_chunk_kernel(
     tab_t* __restrict__ table, float* __restrict__ state, int d, const float* __restrict__ grad,
     const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n, long long n_rows,
     float* __restrict__ part_head, float* __restrict__ part_tail, float lr, float beta, float eps) {
-  const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  if ((long long)c * CHUNK >= n) return;
-  constexpr int TAB_U = TabU<NV>::value;
-  const ChunkRuns r = chunk_runs(skeys, perm, n, c);
-  float G[NV][4];
-  zero_row<NV>(G);
-  for (int q0 = 0; q0 < r.len; q0 += TAB_U) {
-    float g[TAB_U][NV][4], s_old[TAB_U];
-    typename Raw4<tab_t>::type w[TAB_U][NV];
-    int kind[TAB_U];
-    bool ends[TAB_U];
-    uint32_t key[TAB_U];
+  static_assert(CHUNK == 16, "warp_sum16 reduces one value per position of a chunk");
+  static_assert(MAXT <= 512, "ss_sh holds 16 warps");
+  using raw_t = typename Raw4<tab_t>::type;
+  extern __shared__ __align__(16) unsigned char chunk_sh[];
+  __shared__ float ss_sh[16][CHUNK];  // [warp][run-end position]: the warp's share of sum G^2
+  const int c = blockIdx.x, nt = blockDim.x, t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5, nwarps = nt >> 5;
+  float4* gs = reinterpret_cast<float4*>(chunk_sh);           // [CHUNK][nt]: gradients, then run sums
+  raw_t* ws = reinterpret_cast<raw_t*>(gs + (size_t)CHUNK * nt);  // [CHUNK][nt]: table values
+  const int col = 4 * t;
+  const bool own = col < d;
+  const ChunkRuns r = chunk_runs(skeys, perm, n, c);  // every warp finds the same runs
+  // positions with a gradient row (not past the chunk's end, not invalid ids)
+  const unsigned has = __ballot_sync(0xffffffffu, r.pos >= 0) & ((1u << CHUNK) - 1u);
+  // run ends whose row this block finishes (not the run of invalid ids)
+  unsigned whole = 0;
 #pragma unroll
-    for (int u = 0; u < TAB_U; ++u) {
-      const int q = q0 + u;
-      const bool in = q < r.len;
-      const int qs = in ? q : r.len - 1;
-      const int p = __shfl_sync(0xffffffffu, r.pos, qs);
-      key[u] = __shfl_sync(0xffffffffu, r.key, qs);
-      ends[u] = in && ((r.end_mask >> q) & 1u);
-      kind[u] = ends[u] ? run_kind(r, q) : RUN_WHOLE;
-      if (in && p >= 0) load_row<NV>(grad + (long long)p * d, d, g[u]);
-      else zero_row<NV>(g[u]);
-      s_old[u] = 0.f;
-      if (ends[u] && kind[u] == RUN_WHOLE && key[u] < n_rows) {
-        load_raw_row<NV>(table + (long long)key[u] * d, d, w[u]);
-        s_old[u] = state[key[u]];
-      }
-    }
+  for (int q = 0; q < CHUNK; ++q) {
+    const uint32_t kq = __shfl_sync(0xffffffffu, r.key, q);
+    if (((r.end_mask >> q) & 1u) && run_kind(r, q) == RUN_WHOLE && kq < n_rows) whole |= 1u << q;
+  }
 #pragma unroll
-    for (int u = 0; u < TAB_U; ++u) {
-      add_row<NV>(G, g[u]);
-      if (!ends[u]) continue;
-      if (kind[u] == RUN_WHOLE) {
-        // the run of invalid ids (key n_rows) touches nothing
-        if (key[u] < n_rows) table_row_apply<NV>(table, state, key[u], d, G, w[u], s_old[u], lr, beta, eps);
-      } else {
-        store_row<NV>((kind[u] == RUN_TAIL ? part_tail : part_head) + (long long)c * d, d, G);
-      }
-      zero_row<NV>(G);
+  for (int q = 0; q < CHUNK; ++q) {
+    const int p = __shfl_sync(0xffffffffu, r.pos, q);
+    const uint32_t kq = __shfl_sync(0xffffffffu, r.key, q);
+    if (own && ((has >> q) & 1u)) cp_async_own<16>(gs + q * nt + t, grad + (long long)p * d + col);
+    if constexpr (STAGE_ROWS)
+      if (own && ((whole >> q) & 1u)) cp_async_own<sizeof(raw_t)>(ws + q * nt + t, table + (long long)kq * d + col);
+  }
+  const float s_old = ((whole >> lane) & 1u) ? state[r.key] : 0.f;  // lane q: state of run end q
+  cp_async_wait_own();
+  // run sums in position order; gs[q] becomes the sum of the run ending at q
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float ss[CHUNK];
+#pragma unroll
+  for (int q = 0; q < CHUNK; ++q) {
+    if (own && ((has >> q) & 1u)) {
+      const float4 v = gs[q * nt + t];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+    ss[q] = 0.f;
+    if ((r.end_mask >> q) & 1u) {
+      ss[q] = ((acc.x * acc.x + acc.y * acc.y) + acc.z * acc.z) + acc.w * acc.w;
+      if (own) gs[q * nt + t] = acc;
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  const float wss = warp_sum16(ss);
+  if ((lane & 1) == 0) ss_sh[warp][lane >> 1] = wss;
+  // boundary runs: partial sums for the chain launch
+#pragma unroll
+  for (int q = 0; q < CHUNK; ++q) {
+    if (!own || !((r.end_mask >> q) & 1u) || ((whole >> q) & 1u)) continue;
+    const int kind = run_kind(r, q);
+    if (kind == RUN_WHOLE) continue;  // the run of invalid ids
+    *reinterpret_cast<float4*>((kind == RUN_TAIL ? part_tail : part_head) + (long long)c * d + col) = gs[q * nt + t];
+  }
+  __syncthreads();
+  // lane q: the block's sum G^2 of run end q in warp order, then its new state and step
+  float tot = 0.f;
+  if (lane < CHUNK)
+    for (int ww = 0; ww < nwarps; ++ww) tot += ss_sh[ww][lane];
+  const float s_new = beta * s_old + (1.f - beta) * (tot / d);
+  const float step = lr / (sqrtf(s_new) + eps);
+  if (warp == 0 && ((whole >> lane) & 1u)) state[r.key] = s_new;
+#pragma unroll
+  for (int q = 0; q < CHUNK; ++q) {
+    const float st = __shfl_sync(0xffffffffu, step, q);
+    const uint32_t kq = __shfl_sync(0xffffffffu, r.key, q);
+    if (!own || !((whole >> q) & 1u)) continue;
+    raw_t* dst = reinterpret_cast<raw_t*>(table + (long long)kq * d + col);
+    const raw_t wv = STAGE_ROWS ? ws[q * nt + t] : *dst;
+    const float4 G = gs[q * nt + t];
+    float x[4];
+    Raw4<tab_t>::unpack(wv, x);
+    x[0] -= st * G.x; x[1] -= st * G.y; x[2] -= st * G.z; x[3] -= st * G.w;
+    *dst = Raw4<tab_t>::pack(x);
   }
 }
 
@@ -532,7 +628,7 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 6 : (NV <= 8 ? 4 : 2)) table_ch
 template <int NV>
 __device__ __forceinline__ void chain_sum(const float* __restrict__ part_tail, int d, int first, int last,
                                           float (&G)[NV][4]) {
-  constexpr int CHAIN_U = NV <= 6 ? 4 : (NV <= 8 ? 2 : 1);
+  constexpr int CHAIN_U = NV <= 8 ? 2 : 1;  // rows in flight per warp within 128 registers
   for (int cc = first; cc <= last; cc += CHAIN_U) {
     float t[CHAIN_U][NV][4];
 #pragma unroll
@@ -550,8 +646,9 @@ __device__ __forceinline__ void chain_sum(const float* __restrict__ part_tail, i
 // block's CHAIN_WARPS warps each add a contiguous share of the tail partials in
 // chunk order; warp 0 then adds head + shares in warp order.  The grouping is
 // fixed by (c, last), so the result is reproducible.  Returns true in warp 0,
-// which then holds the sum in G.  sh: (CHAIN_WARPS - 1) * d floats.
-constexpr int CHAIN_WARPS = 4;
+// which then holds the sum in G.  sh: (CHAIN_WARPS - 1) * d floats; the caller
+// synchronises the block before sh is used again.
+constexpr int CHAIN_WARPS = 8;  // warps of a chain block, and chunks it scans for chain starts
 template <int NV>
 __device__ __forceinline__ bool chain_block_sum(const float* __restrict__ part_head,
                                                 const float* __restrict__ part_tail, int d, int c, int last,
@@ -576,23 +673,70 @@ __device__ __forceinline__ bool chain_block_sum(const float* __restrict__ part_h
   return true;
 }
 
-// One block per chunk; blocks whose chunk starts a run going on into later
-// chunks sum its partials and finish the row.
+// Chains are finished in two ways.  Warp w of a block checks chunk
+// blockIdx.x * CHAIN_WARPS + w; if it starts a run that goes on into at most
+// CHAIN_SHORT later chunks (nearly all of them), the warp alone adds
+// part_head[c] + part_tail[c+1] + ... + part_tail[last] in chunk order and
+// finishes the row, so a block's short chains proceed in parallel.  Longer
+// chains are listed in shared memory and summed by all warps of the block
+// (chain_block_sum) after a block barrier.  Which way a chain takes depends
+// only on its length, so every row's sum has one fixed grouping.
+constexpr int CHAIN_SHORT = 4;
+
+template <int NV>
+__device__ __forceinline__ void chain_warp_sum(const float* __restrict__ part_head,
+                                               const float* __restrict__ part_tail, int d, int c, int last,
+                                               float (&G)[NV][4]) {
+  load_row<NV>(part_head + (long long)c * d, d, G);
+  chain_sum<NV>(part_tail, d, c + 1, last, G);
+}
+
+// The scan of the block's chunks: returns true in a warp whose chunk starts a
+// short chain (key, last filled in); long chains go to the block's lists.
+// Ends with a block barrier.
+__device__ __forceinline__ bool chain_scan(const uint32_t* __restrict__ skeys, int n, long long key_limit,
+                                           uint32_t& key, int& last, int* flag, int* lastc, uint32_t* keyc) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * CHAIN_WARPS + w;
+  key = 0;
+  last = 0;
+  const bool ok = chained_run(skeys, n, c, key, last) && key < key_limit;  // warp-uniform
+  const bool longc = ok && last - c > CHAIN_SHORT;
+  if (lane == 0) { flag[w] = longc; lastc[w] = last; keyc[w] = key; }
+  __syncthreads();
+  return ok && !longc;
+}
+
 template <int NV, typename tab_t>
-__global__ void __launch_bounds__(CHAIN_WARPS * 32) table_chain_kernel(
+__global__ void __launch_bounds__(CHAIN_WARPS * 32, NV <= 6 ? 2 : 1) table_chain_kernel(
     tab_t* __restrict__ table, float* __restrict__ state, int d, const uint32_t* __restrict__ skeys, int n,
     long long n_rows, const float* __restrict__ part_head, const float* __restrict__ part_tail, float lr,
     float beta, float eps) {
   extern __shared__ float chain_sh[];
-  const int c = blockIdx.x;
+  __shared__ int flag[CHAIN_WARPS], lastc[CHAIN_WARPS];
+  __shared__ uint32_t keyc[CHAIN_WARPS];
   uint32_t key;
   int last;
-  if (!chained_run(skeys, n, c, key, last) || key >= n_rows) return;  // block-uniform
-  float G[NV][4];
-  if (!chain_block_sum<NV>(part_head, part_tail, d, c, last, chain_sh, G)) return;
-  typename Raw4<tab_t>::type w[NV];
-  load_raw_row<NV>(table + (long long)key * d, d, w);
-  table_row_apply<NV>(table, state, key, d, G, w, state[key], lr, beta, eps);
+  if (chain_scan(skeys, n, n_rows, key, last, flag, lastc, keyc)) {
+    const int c = blockIdx.x * CHAIN_WARPS + (threadIdx.x >> 5);
+    typename Raw4<tab_t>::type w[NV];
+    load_raw_row<NV>(table + (long long)key * d, d, w);
+    const float s_old = state[key];
+    float G[NV][4];
+    chain_warp_sum<NV>(part_head, part_tail, d, c, last, G);
+    table_row_apply<NV>(table, state, key, d, G, w, s_old, lr, beta, eps);
+  }
+  for (int i = 0; i < CHAIN_WARPS; ++i) {
+    if (!flag[i]) continue;  // block-uniform
+    const uint32_t k = keyc[i];
+    float G[NV][4];
+    if (chain_block_sum<NV>(part_head, part_tail, d, blockIdx.x * CHAIN_WARPS + i, lastc[i], chain_sh, G)) {
+      typename Raw4<tab_t>::type w[NV];
+      load_raw_row<NV>(table + (long long)k * d, d, w);
+      table_row_apply<NV>(table, state, k, d, G, w, state[k], lr, beta, eps);
+    }
+    __syncthreads();  // chain_sh is refilled for the next chain
+  }
 }
 
 // ---------------------------------------------------------------- embedding grad
@@ -607,7 +751,7 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chun
     long long vocab, float* __restrict__ part_head, float* __restrict__ part_tail) {
   const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if ((long long)c * CHUNK >= n) return;
-  constexpr int TAB_U = TabU<NV>::value;
+  constexpr int TAB_U = 1;  // positions a step: one keeps the kernel near 80 registers, 20 warps an SM
   constexpr bool PREFETCH_OUT = TAB_U > 1;  // wide rows add into dwte when the run ends
   const ChunkRuns r = chunk_runs(skeys, perm, n, c);
   float G[NV][4];
@@ -679,20 +823,34 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chun
 }
 
 template <int NV>
-__global__ void __launch_bounds__(CHAIN_WARPS * 32) emb_chain_kernel(float* __restrict__ dwte, int d,
-                                                                    const uint32_t* __restrict__ skeys, int n,
-                                                                    long long vocab,
-                                                                    const float* __restrict__ part_head,
-                                                                    const float* __restrict__ part_tail) {
+__global__ void __launch_bounds__(CHAIN_WARPS * 32, NV <= 6 ? 2 : 1) emb_chain_kernel(float* __restrict__ dwte, int d,
+                                                                       const uint32_t* __restrict__ skeys, int n,
+                                                                       long long vocab,
+                                                                       const float* __restrict__ part_head,
+                                                                       const float* __restrict__ part_tail) {
   extern __shared__ float chain_sh[];
-  const int c = blockIdx.x;
+  __shared__ int flag[CHAIN_WARPS], lastc[CHAIN_WARPS];
+  __shared__ uint32_t keyc[CHAIN_WARPS];
   uint32_t key;
   int last;
-  if (!chained_run(skeys, n, c, key, last) || key >= vocab) return;  // block-uniform
-  float G[NV][4];
-  if (!chain_block_sum<NV>(part_head, part_tail, d, c, last, chain_sh, G)) return;
-  float o[NV][4];
-  load_row<NV>(dwte + (long long)key * d, d, o);
-  add_row<NV>(o, G);
-  store_row<NV>(dwte + (long long)key * d, d, o);
+  if (chain_scan(skeys, n, vocab, key, last, flag, lastc, keyc)) {
+    const int c = blockIdx.x * CHAIN_WARPS + (threadIdx.x >> 5);
+    float o[NV][4], G[NV][4];
+    load_row<NV>(dwte + (long long)key * d, d, o);
+    chain_warp_sum<NV>(part_head, part_tail, d, c, last, G);
+    add_row<NV>(o, G);
+    store_row<NV>(dwte + (long long)key * d, d, o);
+  }
+  for (int i = 0; i < CHAIN_WARPS; ++i) {
+    if (!flag[i]) continue;  // block-uniform
+    const uint32_t k = keyc[i];
+    float G[NV][4];
+    if (chain_block_sum<NV>(part_head, part_tail, d, blockIdx.x * CHAIN_WARPS + i, lastc[i], chain_sh, G)) {
+      float o[NV][4];
+      load_row<NV>(dwte + (long long)k * d, d, o);
+      add_row<NV>(o, G);
+      store_row<NV>(dwte + (long long)k * d, d, o);
+    }
+    __syncthreads();  // chain_sh is refilled for the next chain
+  }
 }
