@@ -91,7 +91,9 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, act_t* __restric
 }
 
 // RMSNorm backward: dx (+)= rstd * (du - u * mean(du * u)); also writes the
-// activation-typed copy of dx that the next GEMMs read.
+// activation-typed copy of dx that the next GEMMs read.  One warp per row; the
+// row's du, u, rstd and (accumulating) old dx are all requested before the
+// reduction, so a row costs one memory round trip.
 template <int NV, typename act_t>
 __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __restrict__ u,
                                    const float* __restrict__ rstd, float* __restrict__ dx,
@@ -99,30 +101,33 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N) return;
   const long long base = (long long)warp * d;
-  float g[NV][4], y[NV][4];
-  float dot = 0.f;
+  float g[NV][4], y[NV][4], o[NV][4];
+  const float r = rstd[warp];
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
       load4(du + base + c, g[j]);
       load4(u + base + c, y[j]);
-      dot += g[j][0] * y[j][0] + g[j][1] * y[j][1] + g[j][2] * y[j][2] + g[j][3] * y[j][3];
+      if (accumulate) load4(dx + base + c, o[j]);
+      else o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     }
   }
+  float dot = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (j * 32 + lane) * 4;
+    if (c < d) dot += g[j][0] * y[j][0] + g[j][1] * y[j][1] + g[j][2] * y[j][2] + g[j][3] * y[j][3];
+  }
   dot = warp_sum(dot) / d;
-  const float r = rstd[warp];
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (j * 32 + lane) * 4;
     if (c < d) {
-      float o[4];
-      if (accumulate) load4(dx + base + c, o);
-      else o[0] = o[1] = o[2] = o[3] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] += r * (g[j][i] - y[j][i] * dot);
-      store4(dx + base + c, o);
-      store4(dx_lp + base + c, o);
+      for (int i = 0; i < 4; ++i) o[j][i] += r * (g[j][i] - y[j][i] * dot);
+      store4(dx + base + c, o[j]);
+      store4(dx_lp + base + c, o[j]);
     }
   }
 }
