@@ -17,7 +17,10 @@ Sources (each function names the passage it follows):
     ReLU^2 activation, RMSNorm without affine parameters;
   * Chris McCormick's decoder-rtx posts: hand-written backward, bigram hash
     tables added to x0 and to the attention values, "sparse, no first moment,
-    and only per-row magnitude" optimizer inlined into their backward.
+    and only per-row magnitude" optimizer inlined into their backward;
+  * modded-nanogpt README "Proposed optimizer" and the nanochat page's
+    ``zeropower_via_newtonschulz5`` / ``Muon.step``: Muon for the matrix
+    parameters (``muon``; no CUDA path yet).
 
 Parity status per function is listed in ``PINS`` below; every entry is pinned
 by a ``-m "not gpu"`` test in tests/test_oracle_*.py.
@@ -33,4 +36,8 @@ PINS = {
     "optim.adamw": "closed-form first step -lr*sign(g); torch.optim.AdamW",
     "optim.table_update": "closed-form first step; two-step recurrence by hand",
     "counts.num_params / flops_per_token": "nanochat d32 printed values",
+    "muon.newton_schulz": "singular values through the scalar quintic (known SVD); cubic coefficients "
+                          "converge to numpy's polar factor; the pages' (0.5, 1.5) spread",
+    "muon.muon_update": "closed-form Nesterov / plain momentum directions; sqrt(out/in) step scale "
+                        "through the step's singular values",
 }
