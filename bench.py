@@ -439,6 +439,54 @@ def run_tables(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_muon(args, w):
+    """One Muon step over every matrix parameter of the workload's blocks, in
+    the nanochat module's shapes ([out, in]): per layer c_q, c_k, c_v and the
+    attention projection (a x d, d x a) and the MLP's d_ff x d and d x d_ff.
+    Newton-Schulz FLOPs per matrix with R = min(out, in), C = max(out, in):
+    ns_steps * (2 R^2 C [X X^T] + 2 R^3 [A A] + 2 R^2 C [B X]).  The matrices'
+    W, M, G (fp32) exceed L2, so no flush is needed between steps."""
+    import torch
+    import gpt_pretraining_step_decoder_b200 as g
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream()
+    d, a, f, L = w["d_model"], w["n_head"] * w["head_dim"], w["d_ff"], w["n_layer"]
+    shapes = [(a, d), (a, d), (a, d), (d, a), (f, d), (d, f)] * L
+    peaks, peak_src = measured_peaks()
+    gen = torch.Generator(device=dev).manual_seed(w["seed"])
+    mats = []
+    for (o, i) in shapes:
+        W = 0.02 * torch.randn((o, i), device=dev, generator=gen)
+        G = 0.01 * torch.randn((o, i), device=dev, generator=gen)
+        mats.append((W, torch.zeros_like(W), G))
+    ws_bytes = max(g.muon_update_workspace_bytes(o, i) for (o, i) in shapes)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    steps = 5
+    flops = sum(steps * (4.0 * min(o, i) ** 2 * max(o, i) + 2.0 * min(o, i) ** 3) for (o, i) in shapes)
+    times = []
+    with ClockSampler(0) as clk:
+        for it in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for (W, M, G), (o, i) in zip(mats, shapes):
+                g.muon_update(W, M, G, o, i, 1, 0.02, 0.95, 1, steps, ws, ws_bytes)
+            e1.record(st)
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+    if g.ngram_sync_status() != g.GPT_OK:
+        raise RuntimeError(f"muon_update: device error {g.gpt_last_error()}")
+    ms = float(np.median(times))
+    tflops = flops / (ms * 1e-3) / 1e12
+    line = {"metric": "Muon optimizer step over the matrix parameters (CUDA-event time)", "unit": "ms",
+            "value": ms, "workload": w["name"], "matrices": len(shapes), "ns_steps": steps,
+            "ns_gemm_flops": flops, "tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+            "frac_of_peak": tflops / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16 burst",
+            "steps": args.steps, "warmup": args.warmup, "l2": "no flush: W, M, G of the matrices exceed L2",
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def parse_override(items):
     out = {}
     for it in items:
@@ -463,8 +511,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--lr", type=float, default=1e-4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--measure", default="step", choices=["step", "tables"],
-                    help="step: the training step (default); tables: bandwidth of the bigram-table calls")
+    ap.add_argument("--measure", default="step", choices=["step", "tables", "muon"],
+                    help="step: the training step (default); tables: bandwidth of the bigram-table calls; "
+                         "muon: one Muon step over the workload's matrix parameters")
     ap.add_argument("--override", nargs="*", default=[],
                     help="workload field overrides, e.g. n_layer=1 micro_batch=8 (profiling captures)")
     args = ap.parse_args()
@@ -475,6 +524,11 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         run_reference(args, w, rank, world)
+        return
+    if args.measure == "muon":
+        import torch
+        torch.cuda.set_device(0)
+        run_muon(args, workload(args.workload, **parse_override(args.override)))
         return
     if args.measure == "tables":
         import torch

@@ -76,6 +76,8 @@ _SIGS = {
     "ngram_sync_status": [_P],
     "ngram_sparse_update_noalloc": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P],
     "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
+    "muon_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
+    "muon_update": [_P, _P, _P, _I, _I, _I, _F, _F, _I, _I, _P, _SZ, _P],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -255,6 +257,19 @@ def ngram_sparse_update_noalloc(table, row_state, n_rows, d, dtype, rows, grad, 
 
 def ngram_sync_status(stream=None):
     return _lib.ngram_sync_status(_stream(stream))
+
+
+def muon_update_workspace_bytes(rows, cols):
+    b = ctypes.c_size_t(0)
+    _check(_lib.muon_update_workspace_bytes(rows, cols, ctypes.byref(b)), "muon_update_workspace_bytes")
+    return b.value
+
+
+def muon_update(W, M, G, rows, cols, out_rows, lr, momentum, nesterov, ns_steps, workspace, ws_bytes,
+                stream=None):
+    return _check(_lib.muon_update(_ptr(W), _ptr(M), _ptr(G), rows, cols, int(out_rows), float(lr),
+                                   float(momentum), int(nesterov), ns_steps, _ptr(workspace), ws_bytes,
+                                   _stream(stream)), "muon_update")
 
 
 EPI_STORE, EPI_STORE_F32, EPI_ACCUM_F32, EPI_RELU2, EPI_DRELU2, EPI_LOGITS = range(6)

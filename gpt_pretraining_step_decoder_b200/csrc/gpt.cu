@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdarg>
@@ -27,6 +28,7 @@
 #include "layers.cuh"
 #include "ngram.cuh"
 #include "optim.cuh"
+#include "muon.cuh"
 
 // Run the statements with NV = d / 128 (vec4 chunks per lane of a row kernel)
 // as a compile-time constant; rows that are not a multiple of 128 use MAXV.
@@ -1409,6 +1411,100 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
     return gemm_tc_launch<192>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
+}
+
+// ======================================================================== Muon
+// Byte offsets of muon_update's scratch inside the caller's workspace.
+struct MuonWs {
+  size_t x, xn, abf, bm, a, aa, p, partials, splitk, total;
+  long long splitk_elems;
+};
+
+static MuonWs muon_ws_plan(int rows, int cols) {
+  const long long n = (long long)rows * cols, R = rows < cols ? rows : cols;
+  Carver cv;
+  MuonWs w;
+  w.x = cv.take(n * 2);        // X (bf16), the iterate
+  w.xn = cv.take(n * 2);       // its successor
+  w.abf = cv.take(R * R * 2);  // A = X X^T (or X^T X) as the bf16 operand of A A
+  w.bm = cv.take(R * R * 2);   // B = b A + c A A (bf16)
+  w.a = cv.take(R * R * 4);    // A (fp32 GEMM output)
+  w.aa = cv.take(R * R * 4);   // A A (fp32)
+  w.p = cv.take(n * 4);        // B X (or X B) (fp32)
+  w.partials = cv.take((size_t)MUON_NORM_BLOCKS * 4);
+  w.splitk_elems = 4 * R * R;  // split-K partials of the two R x R products
+  w.splitk = cv.take((size_t)w.splitk_elems * 4);
+  w.total = cv.off + 256;      // + slack to align the caller's base to 256 bytes
+  return w;
+}
+
+extern "C" int muon_update_workspace_bytes(int rows, int cols, size_t* bytes) {
+  if (!bytes || rows < 8 || cols < 8 || rows % 8 || cols % 8)
+    return fail(GPT_ERR_ARG, "muon_update_workspace_bytes: rows and cols must be positive multiples of 8");
+  *bytes = muon_ws_plan(rows, cols).total;
+  return GPT_OK;
+}
+
+extern "C" int muon_update(float* W, float* M, const float* G, int rows, int cols, int out_rows, float lr,
+                           float momentum, int nesterov, int ns_steps, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  if (!W || !M || !G || rows < 8 || cols < 8 || rows % 8 || cols % 8 || ns_steps < 0 || ns_steps > 64 ||
+      !(momentum >= 0.f && momentum < 1.f))
+    return fail(GPT_ERR_ARG, "muon_update: bad argument (rows, cols multiples of 8; 0 <= momentum < 1; "
+                             "0 <= ns_steps <= 64)");
+  if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M) | reinterpret_cast<uintptr_t>(G)) & 15)
+    return fail(GPT_ERR_ARG, "muon_update: W, M and G must be 16-byte aligned");
+  const MuonWs p = muon_ws_plan(rows, cols);
+  if (!workspace || ws_bytes < p.total)
+    return fail(GPT_ERR_WORKSPACE, "muon_update: needs %zu bytes of workspace", p.total);
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~uintptr_t(255));
+  bf16* x = reinterpret_cast<bf16*>(base + p.x);
+  bf16* xn = reinterpret_cast<bf16*>(base + p.xn);
+  bf16* abf = reinterpret_cast<bf16*>(base + p.abf);
+  bf16* bm = reinterpret_cast<bf16*>(base + p.bm);
+  float* A = reinterpret_cast<float*>(base + p.a);
+  float* AA = reinterpret_cast<float*>(base + p.aa);
+  float* P = reinterpret_cast<float*>(base + p.p);
+  float* partials = reinterpret_cast<float*>(base + p.partials);
+  float* splitk = reinterpret_cast<float*>(base + p.splitk);
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  cudaStream_t st = (cudaStream_t)stream;
+  const long long n4 = (long long)rows * cols / 4;
+  const int R = rows < cols ? rows : cols;
+  const long long r4 = (long long)R * R / 4;
+  const bool tall = rows > cols;  // iterate as X^T X and X B: the small R x R products either way
+  auto grid = [](long long n) { const long long b = (n + MUON_THREADS - 1) / MUON_THREADS, cap = 4LL * device_sms();
+                                return (unsigned)(b < 1 ? 1 : (b > cap ? cap : b)); };
+  ++g_launches;
+  muon_momentum_kernel<<<MUON_NORM_BLOCKS, MUON_THREADS, 0, st>>>(G, M, n4, momentum, nesterov, partials);
+  ++g_launches;
+  muon_normalize_kernel<<<grid(n4), MUON_THREADS, 0, st>>>(G, M, n4, momentum, nesterov, partials,
+                                                            MUON_NORM_BLOCKS, 1e-7f, x);
+  LAUNCH_CHECK();
+  const GemmCtx g{true, splitk, p.splitk_elems, err, st, nullptr};
+  const float ca = 3.4445f, cb = -4.7750f, cc = 2.0315f;  // a x + b x^3 + c x^5
+  for (int it = 0; it < ns_steps; ++it) {
+    if (!tall) TRY(gemm(g, R, R, cols, op_k(x, cols), op_k(x, cols), epi(EPI_STORE_F32, A, R), true, "muon.gram"));
+    else TRY(gemm(g, R, R, rows, op_mn(x, cols), op_mn(x, cols), epi(EPI_STORE_F32, A, R), true, "muon.gram"));
+    ++g_launches;
+    muon_to_bf16_kernel<<<grid(r4), MUON_THREADS, 0, st>>>(A, r4, abf);
+    TRY(gemm(g, R, R, R, op_k(abf, R), op_mn(abf, R), epi(EPI_STORE_F32, AA, R), true, "muon.square"));
+    ++g_launches;
+    muon_combine_kernel<<<grid(r4), MUON_THREADS, 0, st>>>(abf, AA, r4, cb, cc, bm);
+    if (!tall) TRY(gemm(g, rows, cols, R, op_k(bm, R), op_mn(x, cols), epi(EPI_STORE_F32, P, cols), false, "muon.poly"));
+    else TRY(gemm(g, rows, cols, R, op_k(x, cols), op_mn(bm, R), epi(EPI_STORE_F32, P, cols), false, "muon.poly"));
+    ++g_launches;
+    muon_combine_kernel<<<grid(n4), MUON_THREADS, 0, st>>>(x, P, n4, ca, 1.f, xn);
+    LAUNCH_CHECK();
+    bf16* t = x; x = xn; xn = t;
+  }
+  const double out_dim = out_rows ? rows : cols, in_dim = out_rows ? cols : rows;
+  const float step = (float)(lr * std::sqrt(std::max(1.0, out_dim / in_dim)));
+  ++g_launches;
+  muon_apply_kernel<<<grid(n4), MUON_THREADS, 0, st>>>(W, x, n4, step);
+  LAUNCH_CHECK();
+  return GPT_OK;
 }
 
 // ======================================================================== allocation-free table update

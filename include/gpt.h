@@ -296,6 +296,37 @@ int ngram_sparse_update_noalloc(void* table, float* row_state, long long n_rows,
                                 float eps, int32_t* updated_rows_out, int* n_updated_out_dev,
                                 void* stream);
 
+/* ---- Muon (matrix-parameter optimizer) --------------------------------- */
+
+/* Device workspace bytes muon_update() needs for a rows x cols matrix
+ * (rows, cols: positive multiples of 8). */
+int muon_update_workspace_bytes(int rows, int cols, size_t* bytes);
+
+/*
+ * One Muon step of a matrix parameter, in place (modded-nanogpt README,
+ * "Proposed optimizer"; nanochat discussion #8, `zeropower_via_newtonschulz5`
+ * and `Muon.step`):
+ *   M <- momentum * M + (1 - momentum) * G
+ *   U  = (1 - momentum) * G + momentum * M        (nesterov != 0; else U = M)
+ *   X  = U / (||U||_F + 1e-7), then ns_steps times
+ *        X <- a X + (b A + c A A) X,  A = X X^T   (a, b, c = 3.4445, -4.7750, 2.0315;
+ *        a matrix with more rows than columns runs the same polynomial as
+ *        X <- a X + X (b A + c A A) with A = X^T X)
+ *   W <- W - lr * sqrt(max(1, out / in)) * X
+ * out / in = rows / cols when out_rows != 0 (the weight stored [out, in]),
+ * else cols / rows.  The iterate X, A and the polynomial are bf16 operands of
+ * the tcgen05 GEMM with fp32 accumulation, as the pages run it in bf16; the
+ * momentum and the weight stay fp32.  Sums are formed in a fixed order, so the
+ * result is bit-reproducible.
+ * W, M, G: device fp32 [rows, cols] row-major, 16-byte aligned; W and M are
+ * updated, G is read.  workspace: device, ws_bytes >=
+ * muon_update_workspace_bytes(rows, cols).  rows, cols: multiples of 8;
+ * 0 <= momentum < 1; 0 <= ns_steps <= 64.  Asynchronous on `stream`; a
+ * bounded wait that gives up is reported by ngram_sync_status().
+ */
+int muon_update(float* W, float* M, const float* G, int rows, int cols, int out_rows, float lr, float momentum,
+                int nesterov, int ns_steps, void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- kernel-level test entry point ------------------------------------- */
 
 /*
