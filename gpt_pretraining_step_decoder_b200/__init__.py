@@ -61,6 +61,7 @@ _SIGS = {
     "gpt_backward_step": [_P, _F],
     "gpt_backward": [_P, _F],
     "gpt_optimizer_step": [_P, _F],
+    "gpt_set_table_exchange": [_P, _I],
     "gpt_launch_count": [ctypes.POINTER(_LL)],
     "gpt_profile_enable": [_P, _I],
     "gpt_profile_read": [_P, ctypes.POINTER(GptProfEntry), _I, ctypes.POINTER(_I)],
@@ -317,11 +318,17 @@ class Model:
 
     def backward(self, lr):
         """Backward of the last forward without the dense optimizer step (the
-        table updates still run inline); pair with optimizer_step."""
+        table updates run inline unless set_table_exchange is on); pair with
+        optimizer_step."""
         gpt_backward(self.h, lr)
 
     def optimizer_step(self, lr):
         gpt_optimizer_step(self.h, lr)
+
+    def set_table_exchange(self, on):
+        """Leave the bigram-table gradients to the caller instead of applying
+        them inside backward (data-parallel replicas: see dp.exchange_tables)."""
+        _check(_lib.gpt_set_table_exchange(self.h, int(on)), "gpt_set_table_exchange")
 
     def flat_grad(self):
         """The whole fp32 dense gradient as one flat torch view (no copy)."""

@@ -532,6 +532,7 @@ struct gpt_model {
   int micro = 0;
   long long step_t = 0;
   bool have_fwd = false;
+  bool defer_tables = false;  // gpt_set_table_exchange: backward leaves the table gradients for the caller
   Prof prof;
   template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
   unsigned* err() const { return at<unsigned>(plan.err); }
@@ -700,8 +701,9 @@ extern "C" int gpt_tensor(gpt_model* m, const char* name, int kind, void** ptr, 
     else if (nm == "rows_x" && c.x0_rows) { ptr_out = m->at<int32_t>(p.rows_x); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
     else if (nm == "rows_v" && c.v_rows) { ptr_out = m->at<int32_t>(p.rows_v); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
     else if (nm == "grad_norm") { ptr_out = m->at<float>(p.grad_norm); }
+    else if (nm == "table_grad_x" && c.x0_rows) { ptr_out = m->at<float>(p.dx); sh[0] = N; sh[1] = c.d_model; }
+    else if (nm == "table_grad_v" && c.v_rows) { ptr_out = m->at<float>(p.gv); sh[0] = N; sh[1] = a; }
     else return fail(GPT_ERR_ARG, "unknown activation '%s'", name);
-    (void)N;
   } else if (nm == "*") {
     // the whole flat dense buffer of this kind (tensors padded to 64 elements)
     sh[0] = p.dense_n;
@@ -1144,13 +1146,13 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     LAUNCH_CHECK();
   }
   const float lr_t = lr * c.lr_mult_table;
-  if (c.v_rows) {
+  if (c.v_rows && !m->defer_tables) {
     ProfScope ps(pf, st, "table_update", 0.0, (double)N * a * 4);
     TRY(table_update<act_t>(w, reinterpret_cast<act_t*>(m->base + p.hv), m->at<float>(p.hv_state), c.v_rows, a,
                             m->at<int32_t>(p.rows_v), m->at<float>(p.gv), N, lr_t, c.table_beta, c.table_eps,
                             nullptr, nullptr, err, st));
   }
-  if (c.x0_rows) {
+  if (c.x0_rows && !m->defer_tables) {
     ProfScope ps(pf, st, "table_update", 0.0, (double)N * d * 4);
     TRY(table_update<act_t>(w, reinterpret_cast<act_t*>(m->base + p.hx), m->at<float>(p.hx_state), c.x0_rows, d,
                             m->at<int32_t>(p.rows_x), dx, N, lr_t, c.table_beta, c.table_eps, nullptr, nullptr, err, st));
@@ -1215,6 +1217,12 @@ extern "C" int gpt_backward(gpt_model* m, float lr) {
   if (!std::isfinite(lr)) return fail(GPT_ERR_ARG, "learning rate not finite");
   if (cfg_bf16(m->cfg)) return backward_impl<bf16>(m, lr, false);
   return backward_impl<float>(m, lr, false);
+}
+
+extern "C" int gpt_set_table_exchange(gpt_model* m, int on) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  m->defer_tables = on != 0;
+  return GPT_OK;
 }
 
 extern "C" int gpt_optimizer_step(gpt_model* m, float lr) {

@@ -162,6 +162,19 @@ int gpt_backward_step(gpt_model* m, float lr);
  * followed, on every grad_accum-th call, by gpt_optimizer_step(m, lr).
  */
 int gpt_backward(gpt_model* m, float lr);
+
+/*
+ * Table exchange mode (data-parallel training with replicated bigram tables).
+ * With on != 0, gpt_backward / gpt_backward_step no longer apply the sparse
+ * table updates; they leave each position's table gradient in the buffers
+ * gpt_tensor(..., GPT_KIND_ACT) names "table_grad_x" [B*T, d] and
+ * "table_grad_v" [B*T, H*hd] (fp32, the gradient the inline update would
+ * have applied), next to the rows "rows_x" / "rows_v".  The caller gathers
+ * them from every rank and applies one identical ngram_sparse_update (with
+ * lr * lr_mult_table, table_beta, table_eps) to its replica of "hx" / "hv";
+ * the buffers stay valid until the next gpt_forward_loss.  Off by default.
+ */
+int gpt_set_table_exchange(gpt_model* m, int on);
 int gpt_optimizer_step(gpt_model* m, float lr);
 
 /* Dense (matmul + embedding) and table parameter counts.  Host only. */
@@ -176,7 +189,8 @@ int gpt_flops_per_token(const gpt_config* cfg, long long* flops, long long* flop
  * "wte", "lm_head" (untied only), "h<l>.wqkv" [3*H*hd, d] (rows q|k|v),
  * "h<l>.wo" [d, H*hd], "h<l>.w1" [d_ff, d], "h<l>.w2" [d, d_ff], "hx", "hv";
  * kind GPT_KIND_ACT: "per_token_loss" [B, T] fp32, "rows_x" / "rows_v" [B, T]
- * int32, "grad_norm" (fp32 scalar, set when grad_clip > 0).  The name "*"
+ * int32, "grad_norm" (fp32 scalar, set when grad_clip > 0), "table_grad_x" /
+ * "table_grad_v" (see gpt_set_table_exchange).  The name "*"
  * with kind PARAM / GRAD / ADAM_M / ADAM_V is the whole flat fp32 dense
  * buffer [n] (each tensor padded to a multiple of 64 elements, pads zero),
  * e.g. for an all-reduce of the gradient between gpt_backward and

@@ -111,3 +111,82 @@ def test_rank_streams_differ():
     a, _ = _batch(cfg, dp.rank_stream_seed(cfg["seed"], 0))
     b, _ = _batch(cfg, dp.rank_stream_seed(cfg["seed"], 1))
     assert a.shape == b.shape and not np.array_equal(a, b)
+
+
+def _table_cfg():
+    from synthetic import workload
+    # few rows, so the two ranks' positions share rows and the exchange matters
+    return workload("tiny_fp32", n_layer=1, seq_len=16, micro_batch=2, vocab=96, x0_rows=64, v_rows=32)
+
+
+def _table_grads(cfg, params, tok, tgt, scale=1.0):
+    from oracle import hashing, model
+    rx = hashing.bigram_rows(tok, cfg["vocab"], cfg["hash_p1"], cfg["hash_p2"], cfg["x0_rows"])
+    rv = hashing.bigram_rows(tok, cfg["vocab"], cfg["hash_p1"], cfg["hash_p2"], cfg["v_rows"])
+    _, _, cache = model.forward(cfg, params, tok, tgt, rx, rv)
+    _, gx0, gv = model.backward(cfg, params, cache, scale=scale)
+    return rx.reshape(-1), gx0, rv.reshape(-1), gv
+
+
+def _apply_tables(cfg, params, rows_v, gv, rows_x, gx0, lr):
+    from oracle import optim
+    out = {}
+    for t, rows, g in (("hv", rows_v, gv), ("hx", rows_x, gx0)):
+        W = np.asarray(params[t], dtype=np.float64)
+        out[t], out[t + "_state"], _ = optim.table_update(W, np.zeros(W.shape[0]), rows, g, lr,
+                                                          cfg["table_beta"], cfg["table_eps"])
+    return out
+
+
+def _table_rank_main(rank, world, port, out_dir):
+    import torch
+    import torch.distributed as dist
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cfg = _table_cfg()
+        params = init_params(cfg, seed=3)
+        tok, tgt = _batch(cfg, dp.rank_stream_seed(cfg["seed"], rank))
+        rx, gx0, rv, gv = _table_grads(cfg, params, tok, tgt)
+        ex = {}
+        for name, rows, g in (("x", rx, gx0), ("v", rv, gv)):
+            r_all, g_all = dp.gather_table_grads(torch.from_numpy(rows.astype(np.int32)), torch.from_numpy(g))
+            ex[name] = (r_all.numpy(), g_all.numpy())
+        new = _apply_tables(cfg, params, ex["v"][0], ex["v"][1], ex["x"][0], ex["x"][1], 1e-2)
+        flat = torch.from_numpy(np.concatenate([new[k].reshape(-1) for k in ("hv", "hv_state", "hx", "hx_state")]))
+        reps = [torch.empty_like(flat) for _ in range(world)]
+        dist.all_gather(reps, flat)
+        if rank == 0:
+            np.save(os.path.join(out_dir, "tables.npy"), torch.stack(reps).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_table_exchange_equals_joint_batch_update(tmp_path):
+    """Replicated bigram tables: each rank's per-position table gradients are
+    gathered in rank order (scaled by 1/world) and every rank applies the same
+    sparse update.  The replicas must be bit-identical and equal the update a
+    single process makes from the joint batch's gradients."""
+    import torch.multiprocessing as mp
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    world = 2
+    mp.spawn(_table_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    reps = np.load(tmp_path / "tables.npy")
+    np.testing.assert_array_equal(reps[0], reps[1])
+
+    cfg = _table_cfg()
+    params = init_params(cfg, seed=3)
+    toks, tgts = zip(*[_batch(cfg, dp.rank_stream_seed(cfg["seed"], r)) for r in range(world)])
+    joint = dict(cfg, micro_batch=cfg["micro_batch"] * world)
+    rx, gx0, rv, gv = _table_grads(joint, params, np.concatenate(toks), np.concatenate(tgts))
+    ref = _apply_tables(cfg, params, rv, gv, rx, gx0, 1e-2)
+    flat = np.concatenate([ref[k].reshape(-1) for k in ("hv", "hv_state", "hx", "hx_state")])
+    np.testing.assert_allclose(reps[0], flat, rtol=1e-12, atol=1e-15)
+    # the exchange mattered: the ranks' positions share rows
+    rows0 = set(_table_grads(cfg, params, toks[0], tgts[0])[0])
+    rows1 = set(_table_grads(cfg, params, toks[1], tgts[1])[0])
+    assert rows0 & rows1
