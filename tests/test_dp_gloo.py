@@ -190,3 +190,130 @@ def test_two_rank_table_exchange_equals_joint_batch_update(tmp_path):
     rows0 = set(_table_grads(cfg, params, toks[0], tgts[0])[0])
     rows1 = set(_table_grads(cfg, params, toks[1], tgts[1])[0])
     assert rows0 & rows1
+
+
+class _OracleModel:
+    """The slice of `Model` that dp.train_step uses, backed by the fp64 oracle
+    on CPU tensors (table updates inline unless the exchange mode is on)."""
+
+    def __init__(self, cfg, params):
+        import types
+        import torch
+        self.torch, self.stream, self.w = torch, None, cfg
+        self.cfg = types.SimpleNamespace(x0_rows=cfg["x0_rows"], v_rows=cfg["v_rows"], dtype=0,
+                                         lr_mult_table=cfg["lr_mult_table"], table_beta=cfg["table_beta"],
+                                         table_eps=cfg["table_eps"])
+        self.P = {k: np.array(v, dtype=np.float64) for k, v in params.items()}
+        self.keys = sorted(k for k in self.P if k not in ("hx", "hv"))
+        self.S = {t: np.zeros(self.P[t].shape[0]) for t in ("hx", "hv")}
+        self.grad = torch.zeros(sum(self.P[k].size for k in self.keys), dtype=torch.float64)
+        self.exchange, self.calls = False, []
+
+    def set_table_exchange(self, on):
+        self.exchange = bool(on)
+        self.calls.append("exchange_on")
+
+    def forward_loss(self, tok, tgt):
+        from oracle import hashing, model
+        w = self.w
+        self.rx = hashing.bigram_rows(tok, w["vocab"], w["hash_p1"], w["hash_p2"], w["x0_rows"])
+        self.rv = hashing.bigram_rows(tok, w["vocab"], w["hash_p1"], w["hash_p2"], w["v_rows"])
+        self.loss, _, self.cache = model.forward(w, self.P, tok, tgt, self.rx, self.rv)
+        self.calls.append("forward")
+
+    def backward(self, lr):
+        from oracle import model, optim
+        G, self.gx0, self.gv = model.backward(self.w, self.P, self.cache, scale=1.0)
+        self.grad += self.torch.from_numpy(_flat(G, self.keys))
+        if not self.exchange:
+            lr_t = lr * self.cfg.lr_mult_table
+            for t, rows, g in (("hv", self.rv, self.gv), ("hx", self.rx, self.gx0)):
+                self.P[t], self.S[t], _ = optim.table_update(self.P[t], self.S[t], rows.reshape(-1), g, lr_t,
+                                                             self.cfg.table_beta, self.cfg.table_eps)
+        self.calls.append("backward")
+
+    def tensor(self, name, kind=0):
+        import gpt_pretraining_step_decoder_b200 as g
+        t = self.torch
+        if kind == g.KIND_ACT:
+            return {"rows_x": t.from_numpy(self.rx.astype(np.int32)), "rows_v": t.from_numpy(self.rv.astype(np.int32)),
+                    "table_grad_x": t.from_numpy(self.gx0), "table_grad_v": t.from_numpy(self.gv)}[name]
+        if kind == g.KIND_PARAM:
+            return t.from_numpy(self.P[name])  # shares memory: updated in place
+        if kind == g.KIND_ROW_STATE:
+            return t.from_numpy(self.S[name])
+        raise KeyError(name)
+
+    def flat_grad(self):
+        return self.grad
+
+    def optimizer_step(self, lr):
+        self.calls.append("optimizer")
+
+
+def _oracle_sparse_update(W, state, n_rows, d, dtype, rows, grad, n, lr, beta, eps, upd, nupd, ws, ws_bytes,
+                          stream=None):
+    """Stands in for the CUDA ngram_sparse_update inside the CPU ranks."""
+    from oracle import optim
+    assert rows.numel() == n and tuple(grad.shape) == (n, d) and W.shape == (n_rows, d) and dtype == 0
+    newW, newS, _ = optim.table_update(W.numpy(), state.numpy(), rows.numpy(), grad.numpy(), lr, beta, eps)
+    W.copy_(W.new_tensor(newW))
+    state.copy_(state.new_tensor(newS))
+
+
+def _train_rank_main(rank, world, port, out_dir):
+    import torch
+    import torch.distributed as dist
+    import gpt_pretraining_step_decoder_b200 as g
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    g.ngram_sparse_update = _oracle_sparse_update
+    g.ngram_sparse_update_workspace_bytes = lambda n, d: 1
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cfg = dict(_table_cfg(), lr_mult_table=0.5)
+        m = _OracleModel(cfg, init_params(cfg, seed=3))
+        batches = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], rank) + 7 * s) for s in range(2)]
+        dp.train_step(m, batches, 2e-2)
+        flat = torch.from_numpy(np.concatenate([m.P[t].reshape(-1) for t in ("hv", "hx")] +
+                                               [m.S[t] for t in ("hv", "hx")]))
+        reps = [torch.empty_like(flat) for _ in range(world)]
+        dist.all_gather(reps, flat)
+        if rank == 0:
+            np.save(os.path.join(out_dir, "tables.npy"), torch.stack(reps).numpy())
+            np.save(os.path.join(out_dir, "calls.npy"), np.array(m.calls))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_train_step_exchanges_tables_after_every_backward(tmp_path):
+    """dp.train_step with two ranks and tables: exchange mode on, the tables
+    exchanged after each micro-batch's backward (value table, then x0; the
+    table lr multiplier applied; gradients scaled 1/world), replicas equal,
+    and equal to one process updating per micro-batch over the joint batch."""
+    import torch.multiprocessing as mp
+    from gpt_pretraining_step_decoder_b200 import dp
+    from oracle import model, optim
+    from synthetic import init_params
+
+    world = 2
+    mp.spawn(_train_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    reps = np.load(tmp_path / "tables.npy")
+    calls = list(np.load(tmp_path / "calls.npy"))
+    assert calls == ["exchange_on", "forward", "backward", "forward", "backward", "optimizer"]
+    np.testing.assert_array_equal(reps[0], reps[1])
+
+    cfg = dict(_table_cfg(), lr_mult_table=0.5)
+    P = {k: np.array(v, dtype=np.float64) for k, v in init_params(cfg, seed=3).items()}
+    S = {t: np.zeros(P[t].shape[0]) for t in ("hx", "hv")}
+    joint = dict(cfg, micro_batch=cfg["micro_batch"] * world)
+    for s in range(2):
+        parts = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], r) + 7 * s) for r in range(world)]
+        tok = np.concatenate([p[0] for p in parts])
+        tgt = np.concatenate([p[1] for p in parts])
+        rx, gx0, rv, gv = _table_grads(joint, P, tok, tgt)
+        for t, rows, g in (("hv", rv, gv), ("hx", rx, gx0)):
+            P[t], S[t], _ = optim.table_update(P[t], S[t], rows, g, 2e-2 * 0.5, cfg["table_beta"], cfg["table_eps"])
+    ref = np.concatenate([P[t].reshape(-1) for t in ("hv", "hx")] + [S[t] for t in ("hv", "hx")])
+    np.testing.assert_allclose(reps[0], ref, rtol=1e-11, atol=1e-14)
