@@ -52,46 +52,84 @@ def gather_table_grads(rows, grad, group=None):
     return torch.cat(all_rows), torch.cat(all_grad).mul_(1.0 / world)
 
 
+# (table, rows buffer, per-position gradient buffer, row-count field), in the
+# order the inline update takes them: value table, then x0 table
+_TABLES = (("hv", "rows_v", "table_grad_v", "v_rows"), ("hx", "rows_x", "table_grad_x", "x0_rows"))
+
+
+def _apply_table_update(model, table, n_rows, rows, grad, lr):
+    """One ngram_sparse_update of the model's replica of `table` over the
+    (row, gradient) pairs given, with the table learning-rate multiplier."""
+    import gpt_pretraining_step_decoder_b200 as g
+    cfg = model.cfg
+    W = model.tensor(table, g.KIND_PARAM)
+    state = model.tensor(table, g.KIND_ROW_STATE)
+    n, d = grad.shape
+    ws_bytes = g.ngram_sparse_update_workspace_bytes(n, d)
+    ws = getattr(model, "_table_ws", None)
+    if ws is None or ws.numel() < ws_bytes:
+        ws = model.torch.empty(ws_bytes, dtype=model.torch.uint8, device=grad.device)
+        model._table_ws = ws
+    g.ngram_sparse_update(W, state, n_rows, d, cfg.dtype, rows, grad, n, lr * cfg.lr_mult_table, cfg.table_beta,
+                          cfg.table_eps, None, None, ws, ws.numel(), model.stream)
+
+
+def _table_grads(model, group):
+    """[(table, n_rows, rows, grad)] of every present table after a backward in
+    exchange mode, gathered over the ranks of `group`."""
+    import gpt_pretraining_step_decoder_b200 as g
+    out = []
+    for table, rows_name, grad_name, rows_field in _TABLES:
+        n_rows = getattr(model.cfg, rows_field)
+        if n_rows:
+            rows, grad = gather_table_grads(model.tensor(rows_name, g.KIND_ACT),
+                                            model.tensor(grad_name, g.KIND_ACT), group)
+            out.append((table, n_rows, rows, grad))
+    return out
+
+
 def exchange_tables(model, lr, group=None):
     """After a backward in table exchange mode: gather every rank's table
     gradients and apply the identical sparse update to this rank's replicas
     (value table, then x0 table, the order of the inline update)."""
-    import gpt_pretraining_step_decoder_b200 as g
-    cfg = model.cfg
-    lr_t = lr * cfg.lr_mult_table
-    for table, rows_name, grad_name, n_rows in (("hv", "rows_v", "table_grad_v", cfg.v_rows),
-                                                ("hx", "rows_x", "table_grad_x", cfg.x0_rows)):
-        if not n_rows:
-            continue
-        rows, grad = gather_table_grads(model.tensor(rows_name, g.KIND_ACT), model.tensor(grad_name, g.KIND_ACT),
-                                        group)
-        W = model.tensor(table, g.KIND_PARAM)
-        state = model.tensor(table, g.KIND_ROW_STATE)
-        n, d = grad.shape
-        ws_bytes = g.ngram_sparse_update_workspace_bytes(n, d)
-        ws = getattr(model, "_table_ws", None)
-        if ws is None or ws.numel() < ws_bytes:
-            ws = model.torch.empty(ws_bytes, dtype=model.torch.uint8, device=grad.device)
-            model._table_ws = ws
-        g.ngram_sparse_update(W, state, n_rows, d, cfg.dtype, rows, grad, n, lr_t, cfg.table_beta, cfg.table_eps,
-                              None, None, ws, ws.numel(), model.stream)
+    for table, n_rows, rows, grad in _table_grads(model, group):
+        _apply_table_update(model, table, n_rows, rows, grad, lr)
 
 
-def train_step(model, micro_batches, lr, group=None, loss_host=None):
+def train_step(model, micro_batches, lr, group=None, loss_host=None, tables="inline"):
     """One data-parallel optimizer step of a `Model`: forward + backward of
-    every (tokens, targets) pair on this rank (with the tables exchanged
-    after each backward when there are several ranks), gradient average,
-    AdamW."""
+    every (tokens, targets) pair on this rank, gradient average, AdamW.
+
+    tables="inline": the bigram tables are updated after every micro-batch
+    (inside backward on one rank; exchanged after each backward when there
+    are several).  tables="deferred": every micro-batch's (row, gradient)
+    pairs are collected (gathered over the ranks) and each table takes one
+    sparse update over all of them at the optimizer step, so every forward of
+    the step sees the same tables."""
+    if tables not in ("inline", "deferred"):
+        raise ValueError(f"tables must be 'inline' or 'deferred', not {tables!r}")
     world = dist.get_world_size(group) if dist.is_initialized() else 1
-    exchange = world > 1 and (model.cfg.x0_rows or model.cfg.v_rows)
+    has_tables = bool(model.cfg.x0_rows or model.cfg.v_rows)
+    deferred = has_tables and tables == "deferred"
+    exchange = has_tables and (world > 1 or deferred)
     if exchange:
         model.set_table_exchange(True)
+    pending = {}
     for tok, tgt in micro_batches:
         model.forward_loss(tok, tgt)
         model.backward(lr)
-        if exchange:
+        if deferred:
+            for table, n_rows, rows, grad in _table_grads(model, group):
+                # copies: the buffers are rewritten by the next forward
+                pending.setdefault(table, (n_rows, [], []))[1].append(rows.clone())
+                pending[table][2].append(grad.clone())
+        elif exchange:
             exchange_tables(model, lr, group)
         if loss_host is not None:
             loss_host.copy_(model.loss, non_blocking=True)
+    for table, *_ in _TABLES:
+        if table in pending:
+            n_rows, rows, grads = pending[table]
+            _apply_table_update(model, table, n_rows, model.torch.cat(rows), model.torch.cat(grads), lr)
     average_gradients(model.flat_grad(), group)
     model.optimizer_step(lr)

@@ -317,3 +317,80 @@ def test_train_step_exchanges_tables_after_every_backward(tmp_path):
             P[t], S[t], _ = optim.table_update(P[t], S[t], rows, g, 2e-2 * 0.5, cfg["table_beta"], cfg["table_eps"])
     ref = np.concatenate([P[t].reshape(-1) for t in ("hv", "hx")] + [S[t] for t in ("hv", "hx")])
     np.testing.assert_allclose(reps[0], ref, rtol=1e-11, atol=1e-14)
+
+
+def _deferred_rank_main(rank, world, port, out_dir):
+    import torch
+    import torch.distributed as dist
+    import gpt_pretraining_step_decoder_b200 as g
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    g.ngram_sparse_update = _oracle_sparse_update
+    g.ngram_sparse_update_workspace_bytes = lambda n, d: 1
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cfg = dict(_table_cfg(), lr_mult_table=0.5)
+        m = _OracleModel(cfg, init_params(cfg, seed=3))
+        batches = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], rank) + 7 * s) for s in range(2)]
+        dp.train_step(m, batches, 2e-2, tables="deferred")
+        flat = torch.from_numpy(np.concatenate([m.P[t].reshape(-1) for t in ("hv", "hx")] +
+                                               [m.S[t] for t in ("hv", "hx")]))
+        reps = [torch.empty_like(flat) for _ in range(world)]
+        dist.all_gather(reps, flat)
+        if rank == 0:
+            np.save(os.path.join(out_dir, "tables.npy"), torch.stack(reps).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_train_step_deferred_tables_take_one_update_per_step(tmp_path):
+    """tables="deferred": both micro-batches' (row, gradient) pairs of both
+    ranks are collected and each table takes one sparse update at the
+    optimizer step; the forwards of the step all see the initial tables."""
+    import torch.multiprocessing as mp
+    from gpt_pretraining_step_decoder_b200 import dp
+    from oracle import optim
+    from synthetic import init_params
+
+    world = 2
+    mp.spawn(_deferred_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    reps = np.load(tmp_path / "tables.npy")
+    np.testing.assert_array_equal(reps[0], reps[1])
+
+    cfg = dict(_table_cfg(), lr_mult_table=0.5)
+    P = {k: np.array(v, dtype=np.float64) for k, v in init_params(cfg, seed=3).items()}
+    joint = dict(cfg, micro_batch=cfg["micro_batch"] * world)
+    acc = {"hv": ([], []), "hx": ([], [])}
+    for s in range(2):
+        parts = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], r) + 7 * s) for r in range(world)]
+        rx, gx0, rv, gv = _table_grads(joint, P, np.concatenate([p[0] for p in parts]),
+                                       np.concatenate([p[1] for p in parts]))
+        for t, rows, g in (("hv", rv, gv), ("hx", rx, gx0)):
+            acc[t][0].append(rows)
+            acc[t][1].append(g)
+    out = []
+    for t in ("hv", "hx"):
+        W, S, _ = optim.table_update(P[t], np.zeros(P[t].shape[0]), np.concatenate(acc[t][0]),
+                                     np.concatenate(acc[t][1]), 2e-2 * 0.5, cfg["table_beta"], cfg["table_eps"])
+        out.append((W, S))
+    ref = np.concatenate([out[0][0].reshape(-1), out[1][0].reshape(-1), out[0][1], out[1][1]])
+    np.testing.assert_allclose(reps[0], ref, rtol=1e-11, atol=1e-14)
+    # and it is not the inline schedule, whose second micro-batch sees updated tables
+    Pi = {k: np.array(v, dtype=np.float64) for k, v in init_params(cfg, seed=3).items()}
+    Si = {t: np.zeros(Pi[t].shape[0]) for t in ("hx", "hv")}
+    for s in range(2):
+        parts = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], r) + 7 * s) for r in range(world)]
+        rx, gx0, rv, gv = _table_grads(joint, Pi, np.concatenate([p[0] for p in parts]),
+                                       np.concatenate([p[1] for p in parts]))
+        for t, rows, g in (("hv", rv, gv), ("hx", rx, gx0)):
+            Pi[t], Si[t], _ = optim.table_update(Pi[t], Si[t], rows, g, 2e-2 * 0.5, cfg["table_beta"],
+                                                 cfg["table_eps"])
+    inline = np.concatenate([Pi["hv"].reshape(-1), Pi["hx"].reshape(-1), Si["hv"], Si["hx"]])
+    assert np.abs(inline - ref).max() > 1e-6
+
+
+def test_train_step_rejects_unknown_table_mode():
+    from gpt_pretraining_step_decoder_b200 import dp
+    with pytest.raises(ValueError):
+        dp.train_step(None, [], 1e-3, tables="sharded")
