@@ -752,12 +752,11 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chun
   const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if ((long long)c * CHUNK >= n) return;
   constexpr int TAB_U = 1;  // positions a step: one keeps the kernel near 80 registers, 20 warps an SM
-  constexpr bool PREFETCH_OUT = TAB_U > 1;  // wide rows add into dwte when the run ends
   const ChunkRuns r = chunk_runs(skeys, perm, n, c);
   float G[NV][4];
   zero_row<NV>(G);
   for (int q0 = 0; q0 < r.len; q0 += TAB_U) {
-    float g[TAB_U][NV][4], e[TAB_U][NV][4], o[PREFETCH_OUT ? TAB_U : 1][NV][4], rs[TAB_U];
+    float g[TAB_U][NV][4], e[TAB_U][NV][4], rs[TAB_U];
     int kind[TAB_U];
     bool ends[TAB_U];
     uint32_t key[TAB_U];
@@ -779,8 +778,6 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chun
         zero_row<NV>(g[u]);
         zero_row<NV>(e[u]);
       }
-      if constexpr (PREFETCH_OUT)
-        if (ends[u] && kind[u] == RUN_WHOLE && key[u] < vocab) load_row<NV>(dwte + (long long)key[u] * d, d, o[u]);
     }
 #pragma unroll
     for (int u = 0; u < TAB_U; ++u) {
@@ -795,22 +792,17 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chun
         for (int i = 0; i < 4; ++i) G[j][i] += rs[u] * (g[u][j][i] - e[u][j][i] * rs[u] * dot);
       if (!ends[u]) continue;
       if (kind[u] == RUN_WHOLE) {
-        if (key[u] < vocab) {
-          if constexpr (PREFETCH_OUT) {
-            add_row<NV>(o[u], G);
-            store_row<NV>(dwte + (long long)key[u] * d, d, o[u]);
-          } else {
-            float* dst = dwte + (long long)key[u] * d;
-            const int lane = threadIdx.x & 31;
+        if (key[u] < vocab) {  // the run's sum added into dwte
+          float* dst = dwte + (long long)key[u] * d;
+          const int lane = threadIdx.x & 31;
 #pragma unroll
-            for (int j = 0; j < NV; ++j) {
-              const int col = (j * 32 + lane) * 4;
-              if (col < d) {
-                float t[4];
-                load4(dst + col, t);
-                for (int i = 0; i < 4; ++i) t[i] += G[j][i];
-                store4(dst + col, t);
-              }
+          for (int j = 0; j < NV; ++j) {
+            const int col = (j * 32 + lane) * 4;
+            if (col < d) {
+              float t[4];
+              load4(dst + col, t);
+              for (int i = 0; i < 4; ++i) t[i] += G[j][i];
+              store4(dst + col, t);
             }
           }
         }
