@@ -40,27 +40,46 @@ L2_NOTE = "no L2 flush: a step's working set (weights, activations, logits chunk
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic_gpt2s_bf16.json")
-GEMM_SOURCES = ["gemm_tc.cuh", "gemm_common.cuh", "gpt.cu"]
+GEMM_SOURCES = ["gemm_tc.cuh", "gemm_common.cuh"]
+# the GEMM host code inside gpt.cu: tensor maps, launch, tile width and split-K choice
+GEMM_DISPATCH = ("static int make_tmap_gen(", "// ======================================================================== arena plan")
 
 
 def gemm_sources_sha():
+    """sha256 of what decides a GEMM launch's DRAM traffic besides its shape:
+    the GEMM kernel sources and gpt.cu's GEMM dispatch code."""
     import hashlib
+    csrc = os.path.join(ROOT, "gpt_pretraining_step_decoder_b200", "csrc")
     h = hashlib.sha256()
     for f in GEMM_SOURCES:
-        with open(os.path.join(ROOT, "gpt_pretraining_step_decoder_b200", "csrc", f), "rb") as fh:
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
+    with open(os.path.join(csrc, "gpt.cu"), encoding="utf-8") as fh:
+        src = fh.read()
+    a, b = src.index(GEMM_DISPATCH[0]), src.index(GEMM_DISPATCH[1])
+    h.update(src[a:b].encode("utf-8"))
     return h.hexdigest()
 
 
-def recorded_traffic(workload_name):
+def gemm_launch_signature(prof, steps):
+    """The step's GEMM call plan: per GEMM scope label, launches and FLOPs
+    (2*M*N*K summed) per step."""
+    return {k: [round(v["launches"] / steps, 3), round(v["flops"] / steps)]
+            for k, v in sorted(prof.items()) if k.startswith("gemm")}
+
+
+def recorded_traffic(workload_name, signature):
     """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on this workload with the current GEMM sources; else None."""
+    taken on this workload with the current GEMM sources and the same GEMM
+    launches per step; else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
     if rec.get("workload") != workload_name or rec.get("sources_sha256") != gemm_sources_sha():
+        return None
+    if rec.get("gemm_launches") != signature:
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -321,7 +340,8 @@ def run_ours(args, w, rank, world, dist):
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops_sustained"],
-                "traffic": recorded_traffic(w["name"]) if dom_name == "gemm" else None,
+                "traffic": (recorded_traffic(w["name"], gemm_launch_signature(prof, args.steps))
+                            if dom_name == "gemm" else None),
                 "peak_source": f"{peak_src} bf16 sustained (cuBLAS loop under the power cap)"}
     else:
         achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
@@ -332,7 +352,8 @@ def run_ours(args, w, rank, world, dist):
     roof["share_of_step"] = dom["ms"] / total_ms if total_ms else None
     roof["per_launch"] = (f"{dom_name}: algorithmic FLOPs (2*M*N*K per contraction) or bytes of every launch in "
                           "the step, summed, over the summed CUDA-event time of those launches; traffic = DRAM "
-                          "bytes per launch from the committed ncu summary (null unless taken with these sources)")
+                          "bytes per launch from the committed ncu summary (null unless taken with the same GEMM "
+                          "kernel and dispatch sources and the same GEMM launches per step)")
     breakdown = {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
                      "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["flops"] and v["ms"] else None,
                      "gbs": (v["bytes"] / (v["ms"] / 1e3) / 1e9) if v["bytes"] and v["ms"] else None}
