@@ -286,6 +286,19 @@ def test_clip_coef_matches_torch():
         np.testing.assert_allclose(g * c, t.grad.numpy(), rtol=1e-12)
 
 
+def test_clip_coef_leaves_small_gradients_alone():
+    """Below max_norm torch's clip_grad_norm_ does not scale gradients up."""
+    gs = [RNG.standard_normal((3, 4)) * 1e-3, RNG.standard_normal(7) * 1e-3]
+    ts = [torch.zeros_like(torch.tensor(g), requires_grad=True) for g in gs]
+    for t, g in zip(ts, gs):
+        t.grad = torch.tensor(g)
+    torch.nn.utils.clip_grad_norm_(ts, max_norm=1.0)
+    c = optim.clip_coef(gs, 1.0)
+    assert c == 1.0
+    for t, g in zip(ts, gs):
+        np.testing.assert_array_equal(g * c, t.grad.numpy())
+
+
 def test_table_update_closed_form_and_two_step_recurrence():
     W = np.zeros((5, 4))
     s = np.zeros(5)
@@ -321,6 +334,37 @@ def test_accumulation_sums_scaled_micro_grads():
     one.backward_step(1e-3)
     for k in tr.dense:
         np.testing.assert_allclose(tr.accum_grads[k], one.accum_grads[k], rtol=1e-12, atol=1e-15)
+
+
+def _one_step(cfg, P, lr, batch):
+    tr = OracleTrainer(cfg, P)
+    tok, tgt = batch
+    tr.forward_loss(tok, tgt)
+    tr.backward_step(lr)
+    return tr
+
+
+def test_learning_rate_multipliers_scale_their_own_groups():
+    """A group's step uses lr * its multiplier: a zero multiplier leaves
+    exactly that group untouched, and (lr 1, multipliers 2) equals (lr 2,
+    multipliers 1) everywhere, tables included."""
+    base = tiny_cfg(grad_accum=1)
+    P = tiny_params(base)
+    batch = tiny_batch(base)
+    dense = [k for k in P if k not in ("hx", "hv")]
+    mats = [k for k in dense if k.startswith("h")]
+    for group, keys in (("lr_mult_matrix", mats), ("lr_mult_embed", ["wte"]), ("lr_mult_table", ["hx", "hv"])):
+        tr = _one_step(dict(base, **{group: 0.0}), P, 1e-2, batch)
+        for k in P:
+            if k in keys:
+                np.testing.assert_array_equal(tr.P[k], P[k])
+            else:
+                assert not np.array_equal(tr.P[k], P[k]), (group, k)
+    mults = {m: 2.0 for m in ("lr_mult_matrix", "lr_mult_embed", "lr_mult_head", "lr_mult_table")}
+    a = _one_step(dict(base, **mults), P, 1e-2, batch)
+    b = _one_step(base, P, 2e-2, batch)
+    for k in P:
+        np.testing.assert_allclose(a.P[k], b.P[k], rtol=1e-14, atol=1e-17)
 
 
 # ----------------------------------------------------------------------- counts
