@@ -69,3 +69,31 @@ def test_argument_errors_without_gpu():
     assert g._lib.gpt_backward_step(None, 1.0) == g.GPT_ERR_ARG
     with pytest.raises(g.GptError):
         g.ngram_sparse_update_workspace_bytes(-1, 768)
+
+
+def test_muon_and_table_exchange_argument_errors_without_gpu():
+    """The new entry points validate their arguments before any device work:
+    these calls return their error codes on a machine without a GPU."""
+    import gpt_pretraining_step_decoder_b200 as g
+    lib = g._lib
+    assert lib.gpt_set_table_exchange(None, 1) == g.GPT_ERR_ARG
+    for bad in ((100, 128), (128, 0), (8, 12)):
+        with pytest.raises(g.GptError) as e:
+            g.muon_update_workspace_bytes(*bad)
+        assert e.value.code == g.GPT_ERR_ARG
+    assert g.muon_update_workspace_bytes(768, 2304) > 0
+    W, M, G = 1 << 20, 2 << 20, 3 << 20  # aligned stand-in addresses, never dereferenced
+    args = dict(rows=64, cols=128, out_rows=1, lr=0.02, momentum=0.95, nesterov=1, ns_steps=5)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.muon_update(kw.get("W", W), M, G, a["rows"], a["cols"], a["out_rows"], a["lr"], a["momentum"],
+                               a["nesterov"], a["ns_steps"], kw.get("ws", 4 << 20), kw.get("ws_bytes", 16), None)
+
+    assert lib.muon_update(None, M, G, 64, 128, 1, 0.02, 0.95, 1, 5, None, 0, None) == g.GPT_ERR_ARG
+    assert call(rows=60) == g.GPT_ERR_ARG            # not a multiple of 8
+    assert call(momentum=1.0) == g.GPT_ERR_ARG       # momentum must be < 1
+    assert call(ns_steps=65) == g.GPT_ERR_ARG
+    assert call(W=W + 4) == g.GPT_ERR_ARG            # not 16-byte aligned
+    assert call() == g.GPT_ERR_WORKSPACE             # 16 bytes of workspace
+    assert "workspace" in g.gpt_last_error()
