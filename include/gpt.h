@@ -155,7 +155,8 @@ int gpt_backward_step(gpt_model* m, float lr);
 /*
  * The two halves of gpt_backward_step, for callers that exchange gradients
  * between them (data-parallel training): gpt_backward() runs the backward pass
- * and the table updates and accumulates the dense gradient without stepping;
+ * and the table updates (left to the caller in table exchange mode, see
+ * gpt_set_table_exchange) and accumulates the dense gradient without stepping;
  * gpt_optimizer_step() applies the clip and AdamW to whatever gradient has
  * accumulated (at least one gpt_backward since the last step), then starts a
  * new accumulation.  gpt_backward_step(m, lr) equals gpt_backward(m, lr)
