@@ -144,7 +144,8 @@ int gpt_forward_loss(gpt_model* m, const int32_t* tokens_dev, const int32_t* tar
  * fp32 (the first backward of a step overwrites).  Both bigram tables are
  * updated in place from this micro-batch's gradient before the call returns
  * (x0 table from dL/dx0 per position, value table from the sum over layers of
- * dL/dv), with learning rate lr * lr_mult_table.  On every grad_accum-th call
+ * dL/dv), with learning rate lr * lr_mult_table (unless the table exchange
+ * mode is on: see gpt_set_table_exchange).  On every grad_accum-th call
  * the optional global-norm clip and AdamW (learning rate lr * the group's
  * multiplier) are applied to the dense weights; the gradient buffers keep
  * that step's accumulated gradient until the next step starts.
