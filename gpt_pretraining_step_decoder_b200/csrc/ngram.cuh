@@ -16,8 +16,9 @@
 // equal rows in it with ballots.  A run that lies inside the chunk is finished
 // by that block (sum -> mean square -> row state -> row update).  A run that
 // crosses chunk boundaries leaves one partial sum per chunk it touches; a
-// second launch adds those partials in chunk order and finishes the row.
-// Every row is written by exactly one block.  (The token-embedding gradient
+// second launch adds those partials in a grouping fixed by the run's length
+// (chunk order for short runs, contiguous shares for long ones) and finishes
+// the row.  Every row has exactly one writer.  (The token-embedding gradient
 // uses the same bucketing with one warp per chunk.)
 #pragma once
 #include "common.cuh"
