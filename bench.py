@@ -297,24 +297,22 @@ def run_ours(args, w, rank, world, dist):
     g.gpt_profile_enable(model.h, 0)
 
     # end-to-end through the public calls with pinned host buffers
-    in_tok = torch.empty_like(dev_tok[0])
-    in_tgt = torch.empty_like(dev_tgt[0])
+    in_tok = [torch.empty_like(dev_tok[0]) for _ in range(A)]
+    in_tgt = [torch.empty_like(dev_tgt[0]) for _ in range(A)]
     loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
 
     def e2e_step(i):
         for a in range(A):
-            j = i * A + a
-            in_tok.copy_(host_tok[j], non_blocking=True)
-            in_tgt.copy_(host_tgt[j], non_blocking=True)
-            model.forward_loss(in_tok, in_tgt)
-            if world > 1:
-                model.backward(lr)
-            else:
+            in_tok[a].copy_(host_tok[i * A + a], non_blocking=True)
+            in_tgt[a].copy_(host_tgt[i * A + a], non_blocking=True)
+            if world == 1:
+                model.forward_loss(in_tok[a], in_tgt[a])
                 model.backward_step(lr)
-            loss_host.copy_(model.loss, non_blocking=True)
+                loss_host.copy_(model.loss, non_blocking=True)
         if world > 1:
-            dp.average_gradients(model.flat_grad())
-            model.optimizer_step(lr)
+            # the same data-parallel step as the device-resident pass (gradient
+            # average, table exchange after every backward, optimizer step)
+            dp.train_step(model, list(zip(in_tok, in_tgt)), lr, loss_host=loss_host)
 
     ms_e2e = timed(e2e_step, args.warmup, args.steps)
     st = model.sync_status()

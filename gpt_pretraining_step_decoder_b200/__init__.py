@@ -298,6 +298,7 @@ class Model:
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.h = gpt_create(cfg, seed, self.base, self.bytes, self.stream)
         self.loss = torch.zeros(1, dtype=torch.float32, device=device)
+        self.table_exchange = False
 
     def tensor(self, name, kind=KIND_PARAM):
         """torch view of a named tensor inside the arena (no copy)."""
@@ -329,6 +330,7 @@ class Model:
         """Leave the bigram-table gradients to the caller instead of applying
         them inside backward (data-parallel replicas: see dp.exchange_tables)."""
         _check(_lib.gpt_set_table_exchange(self.h, int(on)), "gpt_set_table_exchange")
+        self.table_exchange = bool(on)
 
     def flat_grad(self):
         """The whole fp32 dense gradient as one flat torch view (no copy)."""

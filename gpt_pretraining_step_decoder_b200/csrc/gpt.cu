@@ -1540,14 +1540,23 @@ extern "C" int ngram_sparse_update_noalloc(void* table, float* row_state, long l
                 "ngram_sparse_update_noalloc: n = %d positions of width d = %d need %zu bytes of scratch, "
                 "more than the %u-byte built-in buffer; use ngram_sparse_update with a workspace",
                 n, d, need, (unsigned)GPT_NOALLOC_SCRATCH_BYTES);
-  int dev = 0;
-  CUDA_TRY(cudaGetDevice(&dev));
+  // the scratch address and the launches belong to the device that owns the stream
+  int cur = 0, dev = 0;
+  CUDA_TRY(cudaGetDevice(&cur));
+  CUDA_TRY(cudaStreamGetDevice((cudaStream_t)stream, &dev));
   if (dev < 0 || dev >= 128) return fail(GPT_ERR_ARG, "ngram_sparse_update_noalloc: device index %d out of range", dev);
+  if (dev != cur) CUDA_TRY(cudaSetDevice(dev));
   void* scratch = g_noalloc_addr[dev].load();
+  cudaError_t e = cudaSuccess;
   if (!scratch) {
-    CUDA_TRY(cudaGetSymbolAddress(&scratch, g_noalloc_scratch));
-    g_noalloc_addr[dev].store(scratch);
+    e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+    if (e == cudaSuccess) g_noalloc_addr[dev].store(scratch);
   }
-  return ngram_sparse_update(table, row_state, n_rows, d, dtype, rows, grad, n, lr, beta, eps, updated_rows_out,
-                             n_updated_out_dev, scratch, GPT_NOALLOC_SCRATCH_BYTES, stream);
+  const int s = e != cudaSuccess
+                    ? fail(GPT_ERR_CUDA, "cudaGetSymbolAddress(g_noalloc_scratch): %s", cudaGetErrorString(e))
+                    : ngram_sparse_update(table, row_state, n_rows, d, dtype, rows, grad, n, lr, beta, eps,
+                                          updated_rows_out, n_updated_out_dev, scratch, GPT_NOALLOC_SCRATCH_BYTES,
+                                          stream);
+  if (dev != cur) CUDA_TRY(cudaSetDevice(cur));
+  return s;
 }

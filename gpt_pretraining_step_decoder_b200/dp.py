@@ -27,8 +27,9 @@ def rank_stream_seed(seed, rank):
 
 
 def average_gradients(flat_grad, group=None):
-    """In-place mean of a flat gradient tensor over the ranks of `group`."""
-    world = dist.get_world_size(group)
+    """In-place mean of a flat gradient tensor over the ranks of `group` (a
+    no-op in a process without a process group)."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
     if world > 1:
         dist.all_reduce(flat_grad, op=dist.ReduceOp.SUM, group=group)
         flat_grad.mul_(1.0 / world)
@@ -112,24 +113,30 @@ def train_step(model, micro_batches, lr, group=None, loss_host=None, tables="inl
     has_tables = bool(model.cfg.x0_rows or model.cfg.v_rows)
     deferred = has_tables and tables == "deferred"
     exchange = has_tables and (world > 1 or deferred)
+    was_exchange = model.table_exchange
     if exchange:
         model.set_table_exchange(True)
-    pending = {}
-    for tok, tgt in micro_batches:
-        model.forward_loss(tok, tgt)
-        model.backward(lr)
-        if deferred:
-            for table, n_rows, rows, grad in _table_grads(model, group):
-                # copies: the buffers are rewritten by the next forward
-                pending.setdefault(table, (n_rows, [], []))[1].append(rows.clone())
-                pending[table][2].append(grad.clone())
-        elif exchange:
-            exchange_tables(model, lr, group)
-        if loss_host is not None:
-            loss_host.copy_(model.loss, non_blocking=True)
-    for table, *_ in _TABLES:
-        if table in pending:
-            n_rows, rows, grads = pending[table]
-            _apply_table_update(model, table, n_rows, model.torch.cat(rows), model.torch.cat(grads), lr)
-    average_gradients(model.flat_grad(), group)
-    model.optimizer_step(lr)
+    try:
+        pending = {}
+        for tok, tgt in micro_batches:
+            model.forward_loss(tok, tgt)
+            model.backward(lr)
+            if deferred:
+                for table, n_rows, rows, grad in _table_grads(model, group):
+                    # copies: the buffers are rewritten by the next forward
+                    pending.setdefault(table, (n_rows, [], []))[1].append(rows.clone())
+                    pending[table][2].append(grad.clone())
+            elif exchange:
+                exchange_tables(model, lr, group)
+            if loss_host is not None:
+                loss_host.copy_(model.loss, non_blocking=True)
+        for table, *_ in _TABLES:
+            if table in pending:
+                n_rows, rows, grads = pending[table]
+                _apply_table_update(model, table, n_rows, model.torch.cat(rows), model.torch.cat(grads), lr)
+        average_gradients(model.flat_grad(), group)
+        model.optimizer_step(lr)
+    finally:
+        # a later plain backward_step must update the tables inline again
+        if exchange and not was_exchange:
+            model.set_table_exchange(False)

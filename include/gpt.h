@@ -282,7 +282,14 @@ int ngram_sparse_update(void* table, float* row_state, long long n_rows, int d, 
                         void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream` and read + clear the standalone operations' device
- * error word (GPT_ERR_INPUT for out-of-range ids). */
+ * error word (GPT_ERR_INPUT for out-of-range ids, GPT_ERR_TIMEOUT for a bounded
+ * wait that gave up).  The standalone calls (ngram_*, muon_update,
+ * gptx_gemm_bf16) share ONE such word per device, not one per stream: a status
+ * read here may report a fault raised by another stream's standalone call on
+ * the same device, and clearing it hides that fault from that stream's caller.
+ * Callers that run standalone calls on several streams at once should read the
+ * status once all of those streams are synchronised.  A model's own word
+ * (gpt_sync_status) is separate. */
 int ngram_sync_status(void* stream);
 
 /*
@@ -300,8 +307,10 @@ int ngram_sync_status(void* stream);
  * 16 MiB (about 16 + d/2 bytes per position: e.g. n <= 32768 positions at
  * d <= 768, or n <= 8192 at d = 2048);
  * larger calls return GPT_ERR_WORKSPACE before any work is enqueued.
- * The first call on a device looks up the buffer's device address (with that
- * device current) and should come before any stream capture.  All calls share
+ * The call runs on the device that owns `stream` (made current for the call
+ * and restored after).  The first call on a device looks up the buffer's
+ * device address (with that device current) and should come before any
+ * stream capture.  All calls share
  * the one buffer: calls whose execution overlaps on the GPU (different
  * streams, or the same buffer used from two host threads' streams) race on it
  * and must be ordered by the caller.  Every GPU that loads the library keeps

@@ -207,11 +207,11 @@ class _OracleModel:
         self.keys = sorted(k for k in self.P if k not in ("hx", "hv"))
         self.S = {t: np.zeros(self.P[t].shape[0]) for t in ("hx", "hv")}
         self.grad = torch.zeros(sum(self.P[k].size for k in self.keys), dtype=torch.float64)
-        self.exchange, self.calls = False, []
+        self.table_exchange, self.calls = False, []
 
     def set_table_exchange(self, on):
-        self.exchange = bool(on)
-        self.calls.append("exchange_on")
+        self.table_exchange = bool(on)
+        self.calls.append("exchange_on" if on else "exchange_off")
 
     def forward_loss(self, tok, tgt):
         from oracle import hashing, model
@@ -225,7 +225,7 @@ class _OracleModel:
         from oracle import model, optim
         G, self.gx0, self.gv = model.backward(self.w, self.P, self.cache, scale=1.0)
         self.grad += self.torch.from_numpy(_flat(G, self.keys))
-        if not self.exchange:
+        if not self.table_exchange:
             lr_t = lr * self.cfg.lr_mult_table
             for t, rows, g in (("hv", self.rv, self.gv), ("hx", self.rx, self.gx0)):
                 self.P[t], self.S[t], _ = optim.table_update(self.P[t], self.S[t], rows.reshape(-1), g, lr_t,
@@ -301,7 +301,7 @@ def test_train_step_exchanges_tables_after_every_backward(tmp_path):
     mp.spawn(_train_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
     reps = np.load(tmp_path / "tables.npy")
     calls = list(np.load(tmp_path / "calls.npy"))
-    assert calls == ["exchange_on", "forward", "backward", "forward", "backward", "optimizer"]
+    assert calls == ["exchange_on", "forward", "backward", "forward", "backward", "optimizer", "exchange_off"]
     np.testing.assert_array_equal(reps[0], reps[1])
 
     cfg = dict(_table_cfg(), lr_mult_table=0.5)
@@ -388,6 +388,44 @@ def test_train_step_deferred_tables_take_one_update_per_step(tmp_path):
                                                  cfg["table_eps"])
     inline = np.concatenate([Pi["hv"].reshape(-1), Pi["hx"].reshape(-1), Si["hv"], Si["hx"]])
     assert np.abs(inline - ref).max() > 1e-6
+
+
+def test_train_step_restores_inline_table_updates(monkeypatch):
+    """After a deferred train_step (one process, no process group) the model is
+    back in inline mode: a plain backward updates the tables again."""
+    import gpt_pretraining_step_decoder_b200 as g
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    monkeypatch.setattr(g, "ngram_sparse_update", _oracle_sparse_update)
+    monkeypatch.setattr(g, "ngram_sparse_update_workspace_bytes", lambda n, d: 1)
+
+    cfg = _table_cfg()
+    m = _OracleModel(cfg, init_params(cfg, seed=3))
+    dp.train_step(m, [_batch(cfg, 11)], 2e-2, tables="deferred")
+    assert m.calls[0] == "exchange_on" and m.calls[-1] == "exchange_off"
+    assert not m.table_exchange
+    hx0 = m.P["hx"].copy()
+    m.forward_loss(*_batch(cfg, 12))
+    m.backward(2e-2)
+    assert np.abs(m.P["hx"] - hx0).max() > 0
+
+
+def test_train_step_restores_exchange_mode_when_a_call_fails():
+    """An exception inside the step (here: a failing backward) still turns
+    the exchange mode back off."""
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    cfg = _table_cfg()
+    m = _OracleModel(cfg, init_params(cfg, seed=3))
+
+    def broken(lr):
+        raise RuntimeError("backward failed")
+    m.backward = broken
+    with pytest.raises(RuntimeError):
+        dp.train_step(m, [_batch(cfg, 11)], 2e-2, tables="deferred")
+    assert not m.table_exchange
 
 
 def test_train_step_rejects_unknown_table_mode():

@@ -163,3 +163,18 @@ def test_long_context_sampled_sequence_and_causal_prefix(g):
     assert rel_l2(per16[0, :4096], per4[0]) < 1e-3
     gm16.backward_step(1e-4)
     assert gm16.sync_status() == g.GPT_OK, g.gpt_last_error()
+
+
+@pytest.mark.parametrize("T", [2048, 8192])
+def test_long_context_full_batch_sampled_sequence(g, T):
+    """The long-context workloads at T = 2048 (32 sequences) and T = 8192
+    (8 sequences), full batch, one layer: the last sequence's per-token losses
+    against the oracle's forward of that sequence alone."""
+    import psutil
+    w = workload(f"long{T}_bf16", n_layer=1)
+    # the oracle's attention holds a few [heads, T, T] fp64 arrays (~13 GB at T = 8192)
+    need = 4 * w["n_head"] * T * T * 8
+    if psutil.virtual_memory().available < 2 * need:
+        pytest.skip(f"host memory below {2 * need / 2**30:.0f} GiB for the fp64 oracle at T = {T}")
+    params = init_params(w)
+    check_sequences(g, w, params, [w["micro_batch"] - 1])
