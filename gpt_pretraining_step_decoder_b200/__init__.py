@@ -77,6 +77,7 @@ _SIGS = {
     "ngram_sync_status": [_P],
     "ngram_sparse_update_noalloc": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P],
     "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
+    "gptx_set_gemm_cta_pairs": [_I],
     "muon_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
     "muon_update": [_P, _P, _P, _I, _I, _I, _F, _F, _I, _I, _P, _SZ, _P],
 }
@@ -281,6 +282,11 @@ def gptx_gemm_bf16(M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, C, ldc, beta=0, 
     return _check(_lib.gptx_gemm_bf16(M, N, K, _ptr(A), lda, a_kmajor, _ptr(B), ldb, b_kmajor, mode,
                                       _ptr(C), ldc, _ptr(aux), beta, splits, _ptr(workspace), ws_bytes,
                                       _stream(stream)), "gptx_gemm_bf16")
+
+
+def gptx_set_gemm_cta_pairs(on):
+    """Run later GEMMs with N >= 256 on SM pairs (True, the default) or one SM per tile."""
+    return _check(_lib.gptx_set_gemm_cta_pairs(int(bool(on))), "gptx_set_gemm_cta_pairs")
 
 
 # ------------------------------------------------------------------ convenience

@@ -16,7 +16,22 @@
 //               them with asynchronous TMA stores (TMA reduce-add for fp32
 //               accumulation), then release the accumulator.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
-// i + 1.  K-major and MN-major operands are both read straight from their
+// i + 1.
+//
+// CG = 2 runs the same roles on a cluster of two CTAs (a pair of SMs) that
+// share 256 x BN output tiles through tcgen05.mma.cta_group::2: each CTA loads
+// its own 128 rows of A and half of the tile's B rows (BN / 2), the MMA
+// thread of the even CTA issues M = 256 products that read both CTAs' shared
+// memory and write each CTA's 128 accumulator rows into its own TMEM, and
+// each CTA drains its own rows.  Per SM the tensor core then reads 8 KB of
+// operands per 128-cycle MMA instead of 12 KB, and TMA writes 32 KB instead
+// of 48 KB per k-block, which is what bounds the one-SM form: a k-block's
+// operand traffic through shared memory (TMA writes plus MMA reads) is about
+// 1.5x what shared memory moves in the k-block's MMA time.  The loads of both
+// CTAs complete on the even CTA's stage barrier; its MMA commits release the
+// stage and publish the accumulator in both CTAs (tcgen05.commit multicast);
+// the odd CTA's epilogue warps release the accumulator on the even CTA's
+// barrier.  No TMA load is multicast.  K-major and MN-major operands are both read straight from their
 // row-major buffers (the UMMA descriptor's major-ness bit), so forward,
 // data-gradient and weight-gradient products need no transposed copies.
 // Split-K writes fp32 partials that a second kernel sums in split order
@@ -60,9 +75,10 @@ template <int KM> struct KmHeavy {
 // BN = 128, 192 or 256 (192 only with fp32 outputs: 96 columns per epilogue
 // warp = three 32-column fp32 blocks); the ring takes what shared memory has
 // left after the epilogue's buffers, at most 6 stages.
-template <int BN, int HEAVY> struct Cfg {
+template <int BN, int HEAVY, int CG = 1> struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_ROWS = BN / CG;               // B rows this CTA loads per k-block
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;  // two accumulators, power of two
   static constexpr int NSTG = HEAVY ? 0 : 1;           // staging blocks per epilogue warp
@@ -74,7 +90,7 @@ template <int BN, int HEAVY> struct Cfg {
 };
 
 struct Params {
-  int M, N, K;
+  int M, N, K;   // m_tiles counts tiles of CG * BM rows
   int a_kmajor, b_kmajor;
   int m_tiles, n_tiles, splits, kb_per_split, kb_total;
   int group_m;  // tile order: groups of group_m m-blocks, m fastest inside a group
@@ -164,6 +180,52 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                    smem_u32(bar))
                : "memory");
 }
+// ---- CTA-pair (cta_group::2) forms
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the variable at shared::cta address `addr` in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on the
+// barrier at shared::cluster address `bar` (this CTA's or the pair peer's)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this offset in both CTAs of the pair once the
+// issuing thread's earlier tcgen05 operations are complete
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -193,6 +255,15 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
     tma_load_2d(dst, map, bar, kb * BK, r0);
   } else {
     for (int j = 0; j < rows / 64; ++j) tma_load_2d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+  }
+}
+// the same, counted on the pair's stage barrier at shared::cluster address `bar`
+__device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map, uint32_t bar,
+                                                  int kmajor, int rows, int r0, int kb) {
+  if (kmajor) {
+    tma_load_2d_pair(dst, map, bar, kb * BK, r0);
+  } else {
+    for (int j = 0; j < rows / 64; ++j) tma_load_2d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
   }
 }
 
@@ -281,12 +352,13 @@ __device__ __forceinline__ void tile_coords(int mn, const Params& p, int& mt, in
 // byte offset of 16-byte chunk j of row r in a 128-byte-swizzled block
 __device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
-template <int BN, int KM, typename act_t>
+template <int BN, int KM, typename act_t, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmAux,
                    const Params p) {
-  using C = Cfg<BN, KmHeavy<KM>::value>;
+  using C = Cfg<BN, KmHeavy<KM>::value, CG>;
+  static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -304,24 +376,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = p.m_tiles * p.n_tiles * p.splits;
+  // CTA pair: rank 0 issues the MMAs; tile t goes to pair blockIdx.x / CG
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int unit = blockIdx.x / CG, n_units = gridDim.x / CG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    // tempty: one arrival per epilogue warp
-    for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], EPI_WARPS); }
+    // tempty: one arrival per epilogue warp (of both CTAs of a pair)
+    for (int s = 0; s < 2; ++s) { mbar_init(&tfull[s], 1); mbar_init(&tempty[s], CG * EPI_WARPS); }
     for (int s = 0; s < EPI_WARPS * C::NAUX; ++s) mbar_init(&auxbar[s], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(C::TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    // a pair allocates together: the same columns in both CTAs' TMEM
+    if constexpr (CG == 2) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // the pair's barriers are initialised and its TMEM allocated before either
+  // CTA signals the other
+  if constexpr (CG == 2) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -334,27 +420,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool issued[C::STAGES];
       for (int s = 0; s < C::STAGES; ++s) issued[s] = false;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < tiles && ok; t += n_units) {
         const int split = t % p.splits;
         const int mn = t / p.splits;
         int mt, nt;
         tile_coords(mn, p, mt, nt);
-        const int m0 = mt * BM, n0 = nt * BN;
+        // this CTA's A rows and B rows of the tile
+        const int m0 = (mt * CG + (int)rank) * BM, n0 = nt * BN + (int)rank * C::B_ROWS;
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err)) { ok = false; break; }
-          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-          load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb);
-          load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb);
+          if constexpr (CG == 2) {
+            // both CTAs' bytes complete on the even CTA's stage barrier, which
+            // that CTA arms for the pair
+            const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+            if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
+            load_operand_pair(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb);
+            load_operand_pair(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb);
+          } else {
+            mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+            load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb);
+            load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb);
+          }
           issued[stage] = true;
           issued_phase[stage] = phase;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
-      // make sure no copy is still landing in this CTA's shared memory
+      // make sure no copy is still landing in this CTA's shared memory (the
+      // odd CTA of a pair cannot wait on the even CTA's barriers: every one
+      // of its copies is consumed by an MMA before the pair finishes, and an
+      // aborted pair waits out its copies before tearing down)
       for (int s = 0; s < C::STAGES; ++s) {
-        if (!issued[s]) continue;
+        if (!issued[s] || rank != 0) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&full[s], issued_phase[s])) {
           if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) { set_error(p.err, GPT_EBIT_TIMEOUT); break; }
@@ -362,17 +461,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(!p.a_kmajor) << 15) |
                              ((uint32_t)(!p.b_kmajor) << 16) | ((uint32_t)(BN >> 3) << 17) |
-                             ((uint32_t)(BM >> 4) << 24);
+                             ((uint32_t)((CG * BM) >> 4) << 24);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < tiles && ok; t += n_units) {
         const int split = t % p.splits;
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
@@ -386,14 +485,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            tc_mma(d_tmem, operand_desc(a_base, p.a_kmajor, k), operand_desc(b_base, p.b_kmajor, k),
-                   idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            if constexpr (CG == 2)
+              tc_mma_pair(d_tmem, operand_desc(a_base, p.a_kmajor, k), operand_desc(b_base, p.b_kmajor, k),
+                          idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            else
+              tc_mma(d_tmem, operand_desc(a_base, p.a_kmajor, k), operand_desc(b_base, p.b_kmajor, k),
+                     idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          if constexpr (CG == 2) tc_commit_pair(&empty[stage]);
+          else tc_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        if constexpr (CG == 2) tc_commit_pair(&tfull[acc]);
+        else tc_commit(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
     }
@@ -416,12 +521,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    // the accumulator-empty barrier lives in the even CTA of a pair
+    const uint32_t tempty0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
+    for (int t = unit; t < tiles && ok; t += n_units) {
       const int split = t % p.splits;
       const int mn = t / p.splits;
       int mt, nt;
       tile_coords(mn, p, mt, nt);
-      const int m0 = mt * BM;
+      const int m0 = (mt * CG + (int)rank) * BM;  // this CTA's 128 accumulator rows
       const int n0 = nt * BN + ccol;  // first output column of this warp
       const int mrow0 = m0 + q * 32;
       const long long m = (long long)mrow0 + lane;
@@ -641,7 +748,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         e.stats[m * ((p.N + HALF - 1) / HALF) + nt * 2 + (ew >> 2)] = make_float2(rmax, rsum);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if constexpr (CG == 2) mbar_arrive_cluster(tempty0 + acc * 8);
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
     if (lane == 0) bulk_wait0();  // all of this warp's stores are complete
@@ -658,10 +768,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) {
+    // an aborted pair may still have copies landing: let them finish (bounded)
+    if (*abort_flag) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 1000000ull) {}
+    }
+    // neither CTA frees TMEM or leaves while its peer may still read its
+    // shared memory, write its TMEM or arrive on its barriers
+    cluster_sync_all();
+  }
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(C::TMEM_COLS));
+    if constexpr (CG == 2)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS));
   }
 }
 

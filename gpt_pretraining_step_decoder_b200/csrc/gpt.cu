@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstring>
 #include <type_traits>
 #include <atomic>
@@ -132,36 +133,94 @@ static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t o
 }
 
 // ======================================================================== GEMM dispatch
-template <int BN, int KM>
+// CTA pairs (tcgen05 cta_group::2) for every GEMM with 256-column tiles,
+// unless GPT_GEMM_CTA_PAIR=0 in the environment or gptx_set_gemm_cta_pairs(0)
+// selects one-CTA tiles.
+static std::atomic<int> g_gemm_pairs{-1};
+static bool gemm_pairs_enabled() {
+  int v = g_gemm_pairs.load();
+  if (v < 0) {
+    const char* e = getenv("GPT_GEMM_CTA_PAIR");
+    v = (e && e[0] == '0') ? 0 : 1;
+    g_gemm_pairs.store(v);
+  }
+  return v == 1;
+}
+
+extern "C" int gptx_set_gemm_cta_pairs(int on) {
+  g_gemm_pairs.store(on ? 1 : 0);
+  return GPT_OK;
+}
+
+// Pairs of SMs that can hold one pair-mode GEMM cluster each at a time (the
+// persistent grid's size in units of tiles); computed once per kernel.
+template <typename K>
+static int resident_clusters(K* kernel, int smem, int cg) {
+  if (cg == 1) return device_sms();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cg; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(cg * (device_sms() / cg));
+  cfg.blockDim = dim3(tc::NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = device_sms() / cg;
+  }
+  return n;
+}
+
+template <int BN, int KM, int CG>
 static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tcm,
                             const CUtensorMap& taux, const tc::Params& p, cudaStream_t st) {
-  using C = tc::Cfg<BN, tc::KmHeavy<KM>::value>;
+  using C = tc::Cfg<BN, tc::KmHeavy<KM>::value, CG>;
   static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
-  static bool attr_done = false;
-  if (!attr_done) {
-    CUDA_TRY(cudaFuncSetAttribute(tc::gemm_tc_kernel<BN, KM, bf16>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    attr_done = true;
+  auto kernel = tc::gemm_tc_kernel<BN, KM, bf16, CG>;
+  static int units = 0;
+  if (!units) {
+    CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    units = resident_clusters(kernel, C::SMEM_BYTES, CG);
   }
   const int tiles = p.m_tiles * p.n_tiles * p.splits;
-  const int grid = tiles < device_sms() ? tiles : device_sms();
-  ++g_launches; tc::gemm_tc_kernel<BN, KM, bf16><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, tcm, taux, p);
+  const int grid = CG * (tiles < units ? tiles : units);
+  ++g_launches;
+  if constexpr (CG == 1) {
+    kernel<<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, tcm, taux, p);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CG; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(tc::NUM_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tcm, taux, p));
+  }
   LAUNCH_CHECK();
   return GPT_OK;
 }
 
-template <int BN>
+template <int BN, int CG = 1>
 static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
                           int splits, float* partial, unsigned* err, cudaStream_t st) {
+  static_assert(CG == 1 || BN == 256, "CTA pairs take 256-column tiles");
   CUtensorMap ta, tb, tcm, taux;
   if (A.kmajor) TRY(make_tmap(&ta, A.ptr, K, M, A.ld, tc::BK, tc::BM));
   else TRY(make_tmap(&ta, A.ptr, M, K, A.ld, 64, tc::BK));
-  if (B.kmajor) TRY(make_tmap(&tb, B.ptr, K, N, B.ld, tc::BK, BN));
+  // a CTA of a pair loads half of the tile's B rows
+  if (B.kmajor) TRY(make_tmap(&tb, B.ptr, K, N, B.ld, tc::BK, BN / CG));
   else TRY(make_tmap(&tb, B.ptr, N, K, B.ld, 64, tc::BK));
   tc::Params p;
   p.M = M; p.N = N; p.K = K;
   p.a_kmajor = A.kmajor; p.b_kmajor = B.kmajor;
-  p.m_tiles = cdiv(M, tc::BM);
+  p.m_tiles = cdiv(M, CG * tc::BM);
   p.n_tiles = cdiv(N, BN);
   // n-fastest order while the whole B operand stays in L2; grouped m-blocks
   // when B is large (the LM head's vocab-sized operand)
@@ -202,21 +261,21 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   if (km == tc::K_QKV && BN != 256) return fail(GPT_ERR_ARG, "QKV epilogue needs 256-column tiles (N >= 256)");
   if constexpr (BN == 192) {  // fp32 outputs only
     switch (km) {
-      case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32>(ta, tb, tcm, taux, p, st))); break;
-      case tc::K_REDUCE_F32: TRY((gemm_tc_launch_k<BN, tc::K_REDUCE_F32>(ta, tb, tcm, taux, p, st))); break;
-      case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL>(ta, tb, tcm, taux, p, st))); break;
+      case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32, CG>(ta, tb, tcm, taux, p, st))); break;
+      case tc::K_REDUCE_F32: TRY((gemm_tc_launch_k<BN, tc::K_REDUCE_F32, CG>(ta, tb, tcm, taux, p, st))); break;
+      case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL, CG>(ta, tb, tcm, taux, p, st))); break;
       default: return fail(GPT_ERR_ARG, "192-column tiles take fp32-output epilogues only");
     }
   } else {
   switch (km) {
-    case tc::K_STORE: TRY((gemm_tc_launch_k<BN, tc::K_STORE>(ta, tb, tcm, taux, p, st))); break;
-    case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32>(ta, tb, tcm, taux, p, st))); break;
-    case tc::K_REDUCE_F32: TRY((gemm_tc_launch_k<BN, tc::K_REDUCE_F32>(ta, tb, tcm, taux, p, st))); break;
-    case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL>(ta, tb, tcm, taux, p, st))); break;
-    case tc::K_RELU2: TRY((gemm_tc_launch_k<BN, tc::K_RELU2>(ta, tb, tcm, taux, p, st))); break;
-    case tc::K_DRELU2: TRY((gemm_tc_launch_k<BN, tc::K_DRELU2>(ta, tb, tcm, taux, p, st))); break;
-    case tc::K_QKV: TRY((gemm_tc_launch_k<BN, tc::K_QKV>(ta, tb, tcm, taux, p, st))); break;
-    default: TRY((gemm_tc_launch_k<BN, tc::K_LOGITS>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_STORE: TRY((gemm_tc_launch_k<BN, tc::K_STORE, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_REDUCE_F32: TRY((gemm_tc_launch_k<BN, tc::K_REDUCE_F32, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_PARTIAL: TRY((gemm_tc_launch_k<BN, tc::K_PARTIAL, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_RELU2: TRY((gemm_tc_launch_k<BN, tc::K_RELU2, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_DRELU2: TRY((gemm_tc_launch_k<BN, tc::K_DRELU2, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_QKV: TRY((gemm_tc_launch_k<BN, tc::K_QKV, CG>(ta, tb, tcm, taux, p, st))); break;
+    default: TRY((gemm_tc_launch_k<BN, tc::K_LOGITS, CG>(ta, tb, tcm, taux, p, st))); break;
   }
   }
   if (p.splits > 1) {
@@ -231,26 +290,28 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
 
 // Choose split-K so a small-output, long-K product still fills the GPU.
 // Share of the SMs' tile slots doing useful columns: tiles over whole waves,
-// times the used fraction of the last column tile.
-static double tile_efficiency(int M, int N, int BN, int splits) {
-  const long long tiles = (long long)cdiv(M, 128) * cdiv(N, BN) * splits;
-  const long long sms = device_sms();
-  const double waves = (double)((tiles + sms - 1) / sms);
-  return ((double)tiles / (waves * sms)) * ((double)N / ((double)cdiv(N, BN) * BN));
+// times the used fraction of the last column tile.  A tile of a CTA pair
+// covers 256 rows and takes two SMs.
+static double tile_efficiency(int M, int N, int BN, int splits, int cg = 1) {
+  const long long tiles = (long long)cdiv(M, 128 * cg) * cdiv(N, BN) * splits;
+  const long long units = device_sms() / cg;
+  const double waves = (double)((tiles + units - 1) / units);
+  return ((double)tiles / (waves * units)) * ((double)N / ((double)cdiv(N, BN) * BN));
 }
 
 // Split-K factor for a product with few output tiles (under 1.5 waves of SMs;
 // larger products pay more for the fp32 partials than a fuller last wave
 // returns): the one that fills whole waves best (tile_efficiency), keeping at
 // least 8 k-blocks per split; on a tie the smaller factor.
-static int pick_splits(int M, int N, int K, int BN) {
+static int pick_splits(int M, int N, int K, int BN, int cg = 1) {
   const int kb = cdiv(K, 64);
-  const long long tiles = (long long)cdiv(M, 128) * cdiv(N, BN);
-  if (tiles >= device_sms() + device_sms() / 2) return 1;
+  const long long tiles = (long long)cdiv(M, 128 * cg) * cdiv(N, BN);
+  const long long units = device_sms() / cg;
+  if (tiles >= units + units / 2) return 1;
   int best = 1;
-  double best_eff = tile_efficiency(M, N, BN, 1);
+  double best_eff = tile_efficiency(M, N, BN, 1, cg);
   for (int s = 2; s <= 16 && kb / s >= 8; ++s) {
-    const double e = tile_efficiency(M, N, BN, s);
+    const double e = tile_efficiency(M, N, BN, s, cg);
     if (e > best_eff + 1e-9) { best = s; best_eff = e; }
   }
   return best;
@@ -321,14 +382,17 @@ static int gemm(const GemmCtx& g, int M, int N, int K, GemmOperand A, GemmOperan
   }
   const bool f32out = e.mode == EPI_ACCUM_F32 || e.mode == EPI_STORE_F32;
   const bool split_ok = allow_split && f32out;
-  auto splits_for = [&](int bn) {
+  auto splits_for = [&](int bn, int cg = 1) {
     if (!split_ok) return 1;
-    int s = pick_splits(M, N, K, bn);
+    int s = pick_splits(M, N, K, bn, cg);
     while (s > 1 && (long long)s * M * N > g.splitk_elems) --s;
     return s;
   };
-  // tile width: 256 (128 below 256 columns); fp32 outputs may take 192 when
-  // that fills the last wave of SMs better (N = 768: 4 x 192 instead of 3 x 256)
+  // 256-column tiles on CTA pairs (256 x 256 output tiles) whenever N >= 256
+  if (N >= 256 && gemm_pairs_enabled())
+    return gemm_tc_launch<256, 2>(M, N, K, A, B, e, splits_for(256, 2), g.splitk, g.err, g.st);
+  // one-CTA tiles: 256 wide (128 below 256 columns); fp32 outputs may take 192
+  // when that fills the last wave of SMs better (N = 768: 4 x 192 instead of 3 x 256)
   int BN = (N >= 256) ? 256 : 128;
   int splits = splits_for(BN);
   if (f32out && N >= 256 && tile_efficiency(M, N, 192, splits_for(192)) > tile_efficiency(M, N, 256, splits) + 0.03) {
@@ -1413,8 +1477,10 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
   }
   GemmOperand a{A, lda, a_kmajor ? 1 : 0}, b{B, ldb, b_kmajor ? 1 : 0};
   GemmCtx g{true, (float*)workspace, (long long)(ws_bytes / 4), err, (cudaStream_t)stream, nullptr};
-  // the same tile width the step would take for this shape
+  // the same tile shape the step would take for this shape
   const bool f32out = mode == EPI_ACCUM_F32 || mode == EPI_STORE_F32;
+  if (N >= 256 && gemm_pairs_enabled())
+    return gemm_tc_launch<256, 2>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   if (f32out && N >= 256 && tile_efficiency(M, N, 192, splits) > tile_efficiency(M, N, 256, splits) + 0.03)
     return gemm_tc_launch<192>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);

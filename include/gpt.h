@@ -376,6 +376,18 @@ int muon_update(float* W, float* M, const float* G, int rows, int cols, int out_
 int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmajor, const void* B,
                    long long ldb, int b_kmajor, int mode, void* C, long long ldc, const void* aux,
                    int beta, int splits, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Tile shape of every later GEMM of this process (the step's and
+ * gptx_gemm_bf16's): on != 0 (the default) runs products with N >= 256 on
+ * pairs of SMs (tcgen05 cta_group::2, 256 x 256 output tiles, each SM loading
+ * half of the tile's B rows); 0 runs them on one SM per 128 x 256 (or 128 x 192)
+ * tile.  Both forms compute the same sums in the same order per output
+ * element.  The environment variable GPT_GEMM_CTA_PAIR=0 sets the initial
+ * value to 0.  A tuning and test switch; not thread-safe against GEMMs being
+ * enqueued at the same time.
+ */
+int gptx_set_gemm_cta_pairs(int on);
 #ifdef __cplusplus
 }
 #endif

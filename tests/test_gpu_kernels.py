@@ -25,10 +25,18 @@ def _bf16_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
 
 
+@pytest.fixture(params=[1, 0], ids=["sm_pairs", "one_sm"])
+def tiles(request, g):
+    """Both tile forms: CTA pairs (256 x 256 tiles over two SMs) and one SM per tile."""
+    g.gptx_set_gemm_cta_pairs(request.param)
+    yield request.param
+    g.gptx_set_gemm_cta_pairs(1)
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 384, 160), (776, 264, 520), (256, 768, 768),
-                                   (2048, 768, 320)])  # the last one runs on 192-column tiles
+                                   (2048, 768, 320)])  # one SM: the last one runs on 192-column tiles
 @pytest.mark.parametrize("a_k,b_k", [(1, 1), (1, 0), (0, 0), (0, 1)])
-def test_gemm_layouts_match_fp64(g, M, N, K, a_k, b_k):
+def test_gemm_layouts_match_fp64(g, tiles, M, N, K, a_k, b_k):
     import torch
     rng = np.random.default_rng(M * 7 + N * 3 + K + 11 * a_k + 5 * b_k)
     A = round_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
@@ -48,7 +56,7 @@ def test_gemm_layouts_match_fp64(g, M, N, K, a_k, b_k):
     assert rel_l2(C.cpu().numpy(), 2 * ref) < 1e-5
 
 
-def test_gemm_split_k_is_deterministic_and_exact(g):
+def test_gemm_split_k_is_deterministic_and_exact(g, tiles):
     import torch
     M, N, K = 768, 768, 4096
     rng = np.random.default_rng(5)
@@ -245,7 +253,7 @@ def test_ngram_sparse_update_invalid_rows_touch_nothing(g):
 
 
 @pytest.mark.parametrize("b_k", [1, 0])
-def test_gemm_epilogue_modes_match_fp64(g, b_k):
+def test_gemm_epilogue_modes_match_fp64(g, tiles, b_k):
     """Every epilogue of the tensor-core GEMM against its definition on the fp64 product."""
     import torch
     M, N, K = 200, 640, 192
@@ -293,3 +301,23 @@ def test_gemm_epilogue_modes_match_fp64(g, b_k):
     g.gptx_gemm_bf16(M, N, K, Ad, K, 1, Bd, ldb, b_k, C, N, 1, 1, None, 0, mode=g.EPI_ACCUM_F32)
     torch.cuda.synchronize()
     assert rel_l2(C.cpu().numpy(), C0 + acc) < 1e-5
+
+
+def test_gemm_tile_forms_agree_bitwise(g):
+    """SM pairs and single-SM tiles add the same products in the same order
+    per output element: identical fp32 results, several tiles and a ragged edge."""
+    import torch
+    M, N, K = 1000, 1280, 704
+    rng = np.random.default_rng(23)
+    Ad = _bf16_dev(round_to_bf16(rng.standard_normal((M, K)).astype(np.float32)))
+    Bd = _bf16_dev(round_to_bf16(rng.standard_normal((K, N)).astype(np.float32)))  # MN-major B
+    outs = []
+    for on in (1, 0):
+        g.gptx_set_gemm_cta_pairs(on)
+        C = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+        g.gptx_gemm_bf16(M, N, K, Ad, K, 1, Bd, N, 0, C, N, 0, 1, None, 0)
+        torch.cuda.synchronize()
+        outs.append(C.cpu().numpy())
+    g.gptx_set_gemm_cta_pairs(1)
+    assert g.ngram_sync_status() == g.GPT_OK
+    np.testing.assert_array_equal(outs[0], outs[1])
