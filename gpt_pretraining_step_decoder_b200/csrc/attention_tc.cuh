@@ -425,15 +425,12 @@ namespace fatcb {
 
 using fatc::LOG2E;
 using fatc::fast_exp2;
+using fatc::tmem_wait_st;
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns
 __device__ __forceinline__ uint64_t kdesc128(uint32_t base, int half_bytes, int k) {
   return tc::smem_desc(base + (k >> 2) * half_bytes + (k & 3) * 32, 16, 1024);
-}
-// K-major [rows x 64] tile (one swizzle atom wide), k-step k over the 64 columns
-__device__ __forceinline__ uint64_t kdesc64(uint32_t base, int k) {
-  return tc::smem_desc(base + k * 32, 16, 1024);
 }
 // the same [rows x 128] tile read MN-major as [N = 128 (two halves), K = rows]
 __device__ __forceinline__ uint64_t mndesc(uint32_t base, int half_bytes, int k) {
@@ -493,17 +490,18 @@ __device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* ds
 // quarter w % 4 (32 key rows) and half (w - 2) / 4 of the 64 query columns,
 // so two warps per scheduler share the elementwise work.
 // smem: K, V [128 x 128] (32 KB each); per stage Q_i, dO_i [64 x 128] (16 KB
-// each); one P^T and one dS^T buffer [128 keys x 64 queries] (16 KB each).
-// The load of Q_{i+QS} waits for the dV/dK products of step i, and a Q/dO
-// load takes about as long as a whole step, so the ring is as deep as shared
-// memory allows (measured on B200: the step is otherwise one chain of S MMA,
-// elementwise work, dV/dK MMA and the next load).  A single P/dS buffer costs
-// nothing: the elementwise work of step i+1 outlasts the dV/dK MMAs of step
-// i that read the buffer.  lse and D come straight from global memory.
+// each, DKDV_QS stages).  P^T and dS^T never touch shared memory: each
+// compute warp writes them as bf16 over the fp32 S^T / dP^T columns it has
+// just read (its own lanes and columns), and the dV / dK products take them
+// as their A operand straight from TMEM.  Per 64-query step the tensor core
+// then reads only K, V, Q and dO from shared memory, which is what bounds the
+// step (operand bytes through shared memory), and the S^T / dP^T buffers
+// alternate, so step i+1's S^T / dP^T products run while step i's
+// elementwise work does.  lse and D come straight from global memory.
 constexpr int THREADS_B = 320;
-constexpr int KV_T = 32768, QT64 = 16384, PT = 16384;
-constexpr int DKDV_QS = 4;
-constexpr int DKDV_SMEM = 2 * KV_T + DKDV_QS * 2 * QT64 + 2 * PT + 1024 + 256;
+constexpr int KV_T = 32768, QT64 = 16384;
+constexpr int DKDV_QS = 5;
+constexpr int DKDV_SMEM = 2 * KV_T + DKDV_QS * 2 * QT64 + 1024 + 256;
 
 __device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -511,22 +509,6 @@ __device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
   tc::tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-// 32 bf16 (64 bytes: chunks 4*half .. 4*half+3) of row r of a K-major
-// swizzled [rows x 64] tile
-__device__ __forceinline__ void st_half_row(uint8_t* tile, int r, int half, const float (&v)[32]) {
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) {
-    uint4 w;
-    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * jj], v[8 * jj + 1]);
-    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * jj + 2], v[8 * jj + 3]);
-    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * jj + 4], v[8 * jj + 5]);
-    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * jj + 6], v[8 * jj + 7]);
-    w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-    w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-    const int j = half * 4 + jj;
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = w;
-  }
 }
 // 64 fp32 TMEM columns of a row, scaled, as bf16 to global (128 bytes)
 __device__ __forceinline__ void row64_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
@@ -551,6 +533,37 @@ __device__ __forceinline__ void row64_out(uint32_t taddr, float scale, bf16* dst
   }
 }
 
+// 16 consecutive 32-bit TMEM columns of the warp's 32 lanes from registers
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+// D (TMEM) += A (TMEM, bf16 packed two per column along K) x B (shared memory)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// two floats as a bf16 pair (a in the low half), rounded half away from zero in
+// magnitude on the integer pipe: add half a bf16 unit in the last place to the
+// fp32 bit pattern, keep the upper 16 bits.  Equal to round-to-nearest-even
+// except on exact ties; it leaves the transcendental unit to the exponentials.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float a, float b) {
+  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
                           const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse2,
@@ -562,18 +575,16 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint8_t* sV = sK + KV_T;
   uint8_t* sQ = sV + KV_T;               // [DKDV_QS stages]
   uint8_t* sO = sQ + DKDV_QS * QT64;     // dO [DKDV_QS stages]
-  uint8_t* sP = sO + DKDV_QS * QT64;     // P^T
-  uint8_t* sS = sP + PT;                 // dS^T
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + PT);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sO + DKDV_QS * QT64);
   uint64_t* kv_full = bars;                  // 1
   uint64_t* q_full = bars + 1;               // DKDV_QS
   uint64_t* q_empty = q_full + DKDV_QS;      // DKDV_QS
-  uint64_t* s_full = q_empty + DKDV_QS;      // 2
-  uint64_t* s_empty = s_full + 2;            // 2
-  uint64_t* p_full = s_empty + 2;            // 2
-  uint64_t* p_free = p_full + 2;             // 2
-  uint64_t* o_full = p_free + 2;             // 1
+  uint64_t* s_full = q_empty + DKDV_QS;      // 2: S^T, dP^T of the buffer computed
+  uint64_t* p_full = s_full + 2;             // 2: P^T, dS^T of the buffer written (8 warps)
+  uint64_t* g_done = p_full + 2;             // 2: the dV/dK products have read the buffer
+  uint64_t* o_full = g_done + 2;             // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+  static_assert((1 + 2 * DKDV_QS + 7) * 8 + 8 <= 256, "barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -593,9 +604,8 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 8);   // one arrival per compute warp
-      mbar_init(&p_full[s], 8);
-      mbar_init(&p_free[s], 1);
+      mbar_init(&p_full[s], 8);    // one arrival per compute warp
+      mbar_init(&g_done[s], 1);
     }
     mbar_init(o_full, 1);
     *abort_flag = 0;
@@ -610,7 +620,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S^T: 0, 64; dP^T: 128, 192; dV: 256; dK: 384
+  // S^T buffers: cols 0, 64; dP^T buffers: 128, 192; dV: 256; dK: 384.  P^T / dS^T
+  // (bf16 pairs) overwrite the first 16 of each half's 32 S^T / dP^T columns.
+  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -646,6 +658,8 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA
+      // iteration i: S^T, dP^T of step i into buffer i & 1 (once the dV/dK
+      // products of step i - 2 have read that buffer), then dV, dK of step i - 1
       const uint32_t id_s = idesc(64, false);   // S^T = K Q^T, dP^T = V dO^T (N = 64 queries)
       const uint32_t id_g = idesc(128, true);   // dV += P^T dO, dK += dS^T Q (N = 128, B MN-major)
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
@@ -654,7 +668,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         if (i < n_it) {
           const int s = i & 1, st = i % DKDV_QS;
           if (!mbar_wait(&q_full[st], (i / DKDV_QS) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[s], ((i >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          if (i >= 2 && !mbar_wait(&g_done[s], ((i - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
 #pragma unroll
@@ -666,18 +680,20 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           tc_commit(&s_full[s]);
         }
         if (i >= 1) {
-          const int ip = i - 1, st = ip % DKDV_QS;
-          if (!mbar_wait(&p_full[0], ip & 1, abort_flag, err)) { ok = false; break; }
+          const int ip = i - 1, s = ip & 1, st = ip % DKDV_QS;
+          if (!mbar_wait(&p_full[s], (ip >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aP = smem_u32(sP), aS = smem_u32(sS);
           const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
+          // k-step k covers queries 16k..16k+15: half k / 2, packed columns (k % 2) * 8
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma(tmem + 256, kdesc64(aP, k), mndesc(aO, QT64 / 2, k), id_g, (ip > 0 || k > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + 256, tmem + s * 64 + (k >> 1) * 32 + (k & 1) * 8, mndesc(aO, QT64 / 2, k), id_g,
+                      (ip > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma(tmem + 384, kdesc64(aS, k), mndesc(aQ, QT64 / 2, k), id_g, (ip > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&p_free[0]);
+            tc_mma_ts(tmem + 384, tmem + 128 + s * 64 + (k >> 1) * 32 + (k & 1) * 8, mndesc(aQ, QT64 / 2, k), id_g,
+                      (ip > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&g_done[s]);
           tc_commit(&q_empty[st]);
           if (ip == n_it - 1) tc_commit(o_full);
         }
@@ -717,18 +733,17 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       }
       if (!warp_wait(&s_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t cs = tmem + lane_off + s * 64 + half * 32;   // this warp's S^T columns
+      const uint32_t cd = cs + 128;                                // and dP^T columns
       float sv[32], dp[32];
       {
         uint32_t r0[32], r1[32];
-        tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
-        tmem_ld32_nowait(tmem + lane_off + 128 + s * 64 + half * 32, r1);
+        tmem_ld32_nowait(cs, r0);
+        tmem_ld32_nowait(cd, r1);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[s]);
       // P^T[key, q] = exp2(s c - lse2_q) for key <= q < T; dS^T = P^T (dP^T - D_q).
       // Off the diagonal every key of the warp is <= every query of the half
       // (warp-uniform), so the causal test drops out.
@@ -748,14 +763,19 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           dp[e] = p * (dp[e] - dv[e]);
         }
       }
-      // the single P/dS buffer: the dV/dK products of step i-1 must have read it
-      if (i >= 1 && !warp_wait(&p_free[0], (i - 1) & 1, abort_flag, err)) { ok = false; break; }
-      st_half_row(sP, r, half, sv);
-      st_half_row(sS, r, half, dp);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // bf16 pairs over the columns just read (this warp's own lanes and columns)
+      uint32_t pw[16], dw[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        pw[j] = pack_bf16x2_rn(sv[2 * j], sv[2 * j + 1]);
+        dw[j] = pack_bf16x2_int(dp[2 * j], dp[2 * j + 1]);
+      }
+      tmem_st16(cs, pw);
+      tmem_st16(cd, dw);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[0]);
+      if (lane == 0) mbar_arrive(&p_full[s]);
     }
     if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
       tc_fence_after();
@@ -776,13 +796,15 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 // ---------------------------------------------------------------- dQ
 // 10 warps as above; compute warps split the 64 key columns in halves.
 // Persistent like the forward: one CTA per SM over the (query tile,
-// sequence, head) items heaviest first; the K/V ring and the S/dP and dS
-// buffers run on across items, Q/dO for the next item load once the item's
-// last S/dP has read them, and dQ alternates between two TMEM accumulators.
+// sequence, head) items heaviest first; the K/V ring and the S/dP buffers run
+// on across items, Q/dO for the next item load once the item's last S/dP has
+// read them, and dQ alternates between two TMEM accumulators.  dS is written
+// as bf16 over the dP columns each compute warp has just read and feeds the
+// dQ product from TMEM.
 // smem: Q, dO [128 x 128] (32 KB each); per stage K_j, V_j [64 x 128] (16 KB
-// each, 4 stages); per buffer dS [128 queries x 64 keys] (16 KB, 2 buffers).
-constexpr int DQ_STAGES = 4;
-constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 2 * PT + 1024 + 256;
+// each, DQ_STAGES stages).
+constexpr int DQ_STAGES = 5;
+constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 1024 + 256;
 
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
@@ -796,17 +818,15 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint8_t* sO = sQ + KV_T;
   uint8_t* sK = sO + KV_T;                   // [stages]
   uint8_t* sV = sK + DQ_STAGES * QT64;       // [stages]
-  uint8_t* sS = sV + DQ_STAGES * QT64;       // dS [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sS + 2 * PT);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + DQ_STAGES * QT64);
   uint64_t* q_full = bars;                      // 1
   uint64_t* q_empty = q_full + 1;               // 1 (the item's last S/dP have read Q and dO)
   uint64_t* kv_full = q_empty + 1;              // DQ_STAGES
   uint64_t* kv_empty = kv_full + DQ_STAGES;     // DQ_STAGES
-  uint64_t* s_full = kv_empty + DQ_STAGES;      // 2
-  uint64_t* s_empty = s_full + 2;               // 2
-  uint64_t* p_full = s_empty + 2;               // 2
-  uint64_t* p_free = p_full + 2;                // 2
-  uint64_t* o_full = p_free + 2;                // 2 (per dQ buffer: the item's last product is done)
+  uint64_t* s_full = kv_empty + DQ_STAGES;      // 2: S, dP of the buffer computed
+  uint64_t* p_full = s_full + 2;                // 2: dS of the buffer written (8 warps)
+  uint64_t* g_done = p_full + 2;                // 2: the dQ product has read the buffer
+  uint64_t* o_full = g_done + 2;                // 2 (per dQ buffer: the item's last product is done)
   uint64_t* o_empty = o_full + 2;               // 2 (per dQ buffer: the compute warps have read it)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
   static_assert((2 + 2 * DQ_STAGES + 12) * 8 + 8 <= 256, "barrier area");
@@ -830,9 +850,8 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 8);   // one arrival per compute warp
-      mbar_init(&p_full[s], 8);
-      mbar_init(&p_free[s], 1);
+      mbar_init(&p_full[s], 8);    // one arrival per compute warp
+      mbar_init(&g_done[s], 1);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_empty[s], 8);
     }
@@ -848,7 +867,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S: 0, 64; dP: 128, 192; dQ: 256 and 384 (alternating per item)
+  // S: 0, 64; dP: 128, 192 (dS as bf16 pairs over the first 16 of each half's
+  // 32 dP columns); dQ: 256 and 384 (alternating per item)
+  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -911,7 +932,8 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           const int st = g % DQ_STAGES, s = g & 1;
           if (j_s == 0 && !mbar_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
           if (!mbar_wait(&kv_full[st], (g / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          // the dQ product of step g - 2 has read dS from this buffer
+          if (g >= 2 && !mbar_wait(&g_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
 #pragma unroll
@@ -937,11 +959,13 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           }
           if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aS = smem_u32(sS + s * PT), aK = smem_u32(sK + st * QT64);
+          const uint32_t aK = smem_u32(sK + st * QT64);
+          // k-step k covers keys 16k..16k+15: half k / 2, packed columns (k % 2) * 8
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma(tmem + 256 + ob * 128, kdesc64(aS, k), mndesc(aK, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&p_free[s]);
+            tc_mma_ts(tmem + 256 + ob * 128, tmem + 128 + s * 64 + (k >> 1) * 32 + (k & 1) * 8,
+                      mndesc(aK, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&g_done[s]);
           tc_commit(&kv_empty[st]);
           if (++j_p == n_p) {  // the item's last product: dQ is complete
             tc_commit(&o_full[ob]);
@@ -974,18 +998,16 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         const int s = g & 1;
         if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t cd = tmem + lane_off + 128 + s * 64 + half * 32;  // this warp's dP columns
         float sv[32], dp[32];
         {
           uint32_t r0[32], r1[32];
           tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
-          tmem_ld32_nowait(tmem + lane_off + 128 + s * 64 + half * 32, r1);
+          tmem_ld32_nowait(cd, r1);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[s]);
         const int kbase = j * 64 + half * 32;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -993,9 +1015,12 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
           dp[e] = p * (dp[e] - Dq);
         }
-        if (g >= 2 && !warp_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        st_half_row(sS + s * PT, r, half, dp);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        // dS as bf16 pairs over the dP columns just read (this warp's own lanes and columns)
+        uint32_t dw[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) dw[jj] = pack_bf16x2_int(dp[2 * jj], dp[2 * jj + 1]);
+        tmem_st16(cd, dw);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[s]);

@@ -388,8 +388,12 @@ static int gemm(const GemmCtx& g, int M, int N, int K, GemmOperand A, GemmOperan
     while (s > 1 && (long long)s * M * N > g.splitk_elems) --s;
     return s;
   };
-  // 256-column tiles on CTA pairs (256 x 256 output tiles) whenever N >= 256
-  if (N >= 256 && gemm_pairs_enabled())
+  // 256-column tiles on CTA pairs (256 x 256 output tiles) whenever N >= 256,
+  // except for the two epilogues that bound their kernels (the logits'
+  // statistics and the ReLU^2 backward's activation stream), which measured
+  // faster on one-SM tiles (B200: LM-head logits 2.55 vs 2.79 ms, ReLU^2
+  // backward 2.04 vs 2.17 ms per GPT-2-small step)
+  if (N >= 256 && gemm_pairs_enabled() && e.mode != EPI_LOGITS && e.mode != EPI_DRELU2)
     return gemm_tc_launch<256, 2>(M, N, K, A, B, e, splits_for(256, 2), g.splitk, g.err, g.st);
   // one-CTA tiles: 256 wide (128 below 256 columns); fp32 outputs may take 192
   // when that fills the last wave of SMs better (N = 768: 4 x 192 instead of 3 x 256)
