@@ -20,8 +20,11 @@
 //               S_{j+1} is computed while row j's softmax runs) and
 //               O += P_j V_j into a TMEM accumulator;
 //   warps 2..5  softmax, one query row per thread: read S_j from TMEM, mask,
-//               running max, exp2, row sum, write P_j as bf16 into a swizzled
-//               shared-memory tile (the MMA's A operand, double-buffered).
+//               running max, exp2, row sum, write P_j as bf16 pairs (packed on
+//               the integer pipe) over the first half of S_j's own TMEM
+//               columns: the PV product takes P as its A operand from TMEM,
+//               so shared memory carries only Q, K and V.  S_{j+2} reuses the
+//               buffer once PV_j has read it.
 //               O is rescaled in TMEM only when a row max grows by more than
 //               2^8 (log2 units) over the max in use, so most tiles skip it;
 //               the exponentials then stay below 2^8, safe in fp32 and bf16.
@@ -34,8 +37,8 @@ namespace fatc {
 constexpr int BQ = 128, BKV = 128, HD = 128;
 constexpr int THREADS = 192;
 constexpr int TILE_BYTES = 128 * 128 * 2;          // one 128 x 128 bf16 tile
-constexpr int SMEM_BYTES = TILE_BYTES /*Q*/ + 2 * 2 * TILE_BYTES /*K,V x 2 stages*/ +
-                           2 * TILE_BYTES /*P x 2*/ + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int SMEM_BYTES = TILE_BYTES /*Q*/ + 2 * 2 * TILE_BYTES /*K,V x 2 stages*/ + 1024 /*align*/ +
+                           256 /*barriers*/;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float RESCALE_THRESHOLD = 8.f;  // log2 units
 
@@ -59,6 +62,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 16 consecutive 32-bit TMEM columns of the warp's 32 lanes from registers
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+// D (TMEM) += A (TMEM, bf16 packed two per column along K) x B (shared memory)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// two floats as a bf16 pair (a in the low half), rounded half away from zero in
+// magnitude on the integer pipe: add half a bf16 unit in the last place to the
+// fp32 bit pattern, keep the upper 16 bits.  Equal to round-to-nearest-even
+// except on exact ties; it leaves the transcendental unit to the exponentials.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float a, float b) {
+  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 
 // K-major 128 x 128 operand tile = two 128 x 64 sub-tiles (128-byte swizzle);
 // descriptor of MMA k-step k (16 elements along K).
@@ -86,8 +120,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + TILE_BYTES;            // [2 stages]
   uint8_t* sV = sK + 2 * TILE_BYTES;        // [2 stages]
-  uint8_t* sP = sV + 2 * TILE_BYTES;        // [2 buffers]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * TILE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * TILE_BYTES);
   uint64_t* q_full = bars;                  // 1
   uint64_t* q_empty = bars + 1;             // 1 (the item's last S has read Q)
   uint64_t* k_full = bars + 2;              // 2
@@ -95,9 +128,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* v_full = bars + 6;              // 2
   uint64_t* v_empty = bars + 8;             // 2 (PV done with V)
   uint64_t* s_full = bars + 10;             // 2
-  uint64_t* s_empty = bars + 12;            // 2
-  uint64_t* p_full = bars + 14;             // 2
-  uint64_t* p_free = bars + 16;             // 2 (PV done: P buffer free, O updated)
+  uint64_t* p_full = bars + 14;             // 2 (P written over the S buffer)
+  uint64_t* p_free = bars + 16;             // 2 (PV done: S/P buffer free, O updated)
   uint64_t* o_full = bars + 18;             // 2 (per O buffer: the item's last PV is done)
   uint64_t* o_empty = bars + 20;            // 2 (per O buffer: the softmax warps have read O)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
@@ -119,8 +151,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);   // one arrival per softmax warp
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[s], 4);    // one arrival per softmax warp
       mbar_init(&p_free[s], 1);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_empty[s], 4);
@@ -137,7 +168,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S0: cols 0..127, S1: 128..255, O0: 256..383, O1: 384..511
+  // S0: cols 0..127, S1: 128..255 (P as bf16 pairs over the first 64 columns
+  // of its S buffer), O0: 256..383, O1: 384..511
+  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane < 2) {
@@ -200,7 +233,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // S = Q K^T: A = Q (K-major), B = K (K-major), N = 128
       const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
                                ((uint32_t)(128 >> 4) << 24);
-      // O += P V: A = P (K-major), B = V (MN-major), N = 128
+      // O += P V: A = P (TMEM), B = V (MN-major), N = 128
       const uint32_t idesc_o = idesc_s | (1u << 16);
       const uint32_t aQ = smem_u32(sQ);
       bool ok = true;
@@ -215,7 +248,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int s = g & 1;
           if (j_s == 0 && !mbar_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
           if (!mbar_wait(&k_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          // the PV product of step g - 2 has read P from this buffer
+          if (g >= 2 && !mbar_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aK = smem_u32(sK + s * TILE_BYTES);
 #pragma unroll
@@ -242,12 +276,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
           if (!mbar_wait(&v_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aP = smem_u32(sP + s * TILE_BYTES);
           const uint32_t aV = smem_u32(sV + s * TILE_BYTES);
+          // k-step k covers keys 16k..16k+15: packed P columns 8k..8k+7
 #pragma unroll
           for (int k = 0; k < BKV / 16; ++k)
-            tc_mma(tmem + 256 + ob * 128, kmaj_desc(aP, k), mnmaj_desc(aV, k), idesc_o,
-                   (j_p > 0 || k > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + 256 + ob * 128, tmem + s * 128 + k * 8, mnmaj_desc(aV, k), idesc_o,
+                      (j_p > 0 || k > 0) ? 1u : 0u);
           tc_commit(&p_free[s]);
           tc_commit(&v_empty[s]);
           if (++j_p == nkv_p) {  // the item's last PV: O is complete
@@ -296,9 +330,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             sv[96 + ii] = __uint_as_float(r3[ii]);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[s]);  // the S buffer may be overwritten
         const int k0 = j * BKV;
         if (k0 + BKV - 1 > qpos) {  // causal mask on the diagonal tile
 #pragma unroll
@@ -339,27 +370,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           l *= alpha;
           m_use = m_new;
         }
-        // P = exp2(s - m_use) as bf16 into the P buffer of this parity, once
-        // the PV product that read it two steps ago is done
-        if (g >= 2 && !warp_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        uint8_t* pb = sP + s * TILE_BYTES;
+        // P = exp2(s - m_use) as bf16 pairs over the first 64 columns of this
+        // row's S buffer (read above), the A operand of the PV product
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial sums
         const float nm = -m_use;
+        const uint32_t sbase = tmem + lane_off + s * 128;
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 keys
-          float p[8];
+        for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 32 keys = 16 packed columns
+          uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) { p[e] = fast_exp2(fmaf(sv[ch * 8 + e], c, nm)); ps[e] += p[e]; }
-          uint4 w;
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]), b1 = __floats2bfloat162_rn(p[2], p[3]);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]), b3 = __floats2bfloat162_rn(p[6], p[7]);
-          w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-          w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-          const int sub = ch >> 3, jj = ch & 7;
-          *reinterpret_cast<uint4*>(pb + sub * (TILE_BYTES / 2) + r * 128 + ((jj ^ (r & 7)) << 4)) = w;
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(sv[ch * 32 + 2 * e], c, nm));
+            const float p1 = fast_exp2(fmaf(sv[ch * 32 + 2 * e + 1], c, nm));
+            ps[(2 * e) & 7] += p0;
+            ps[(2 * e + 1) & 7] += p1;
+            w[e] = pack_bf16x2_int(p0, p1);
+          }
+          tmem_st16(sbase + ch * 16, w);
         }
         l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[s]);
@@ -426,6 +456,10 @@ namespace fatcb {
 using fatc::LOG2E;
 using fatc::fast_exp2;
 using fatc::tmem_wait_st;
+using fatc::tmem_st16;
+using fatc::tc_mma_ts;
+using fatc::pack_bf16x2_int;
+using fatc::pack_bf16x2_rn;
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns
@@ -531,37 +565,6 @@ __device__ __forceinline__ void row64_out(uint32_t taddr, float scale, bf16* dst
       }
     }
   }
-}
-
-// 16 consecutive 32-bit TMEM columns of the warp's 32 lanes from registers
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-// D (TMEM) += A (TMEM, bf16 packed two per column along K) x B (shared memory)
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// two floats as a bf16 pair (a in the low half), rounded half away from zero in
-// magnitude on the integer pipe: add half a bf16 unit in the last place to the
-// fp32 bit pattern, keep the upper 16 bits.  Equal to round-to-nearest-even
-// except on exact ties; it leaves the transcendental unit to the exponentials.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float a, float b) {
-  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-}
-__device__ __forceinline__ uint32_t pack_bf16x2_rn(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __global__ void __launch_bounds__(THREADS_B, 1)
