@@ -7,12 +7,31 @@ backward every micro-batch, clip + optimizer step + zero_grad every
 ``grad_accum`` micro-batches).  The bigram tables are updated inside every
 backward call from that micro-batch's gradient (the decoder-rtx posts inline
 the table optimizer into backward, so no table gradient survives the call).
+
+With ``matrix_optimizer == "muon"`` the block matrices take Muon and only the
+embedding and the head take AdamW, as in the nanochat setup
+(``setup_optimizers``: Muon for the transformer matrices, AdamW for the rest;
+the pasted training loop clips the gradient norm of all parameters before
+either optimizer steps).  The fused q|k|v weight is three matrices to Muon
+(nanochat's separate ``c_q``, ``c_k``, ``c_v``), each orthogonalised on its
+own; the attention projection and the two MLP weights are one matrix each.
 """
 
 import numpy as np
 
-from . import model, optim
+from . import model, muon, optim
 from .hashing import bigram_rows
+
+
+def muon_blocks(cfg, name, shape):
+    """Row ranges of a dense parameter that Muon treats as separate matrices
+    ([] for parameters that AdamW steps)."""
+    if not name.startswith("h"):
+        return []
+    if name.endswith(".wqkv"):
+        a = cfg["n_head"] * cfg["head_dim"]
+        return [(0, a), (a, 2 * a), (2 * a, 3 * a)]
+    return [(0, shape[0])]
 
 
 class OracleTrainer:
@@ -76,10 +95,22 @@ class OracleTrainer:
             self.accum_grads = {k: self.acc[k].copy() for k in self.dense}
             coef = optim.clip_coef([self.acc[k] for k in self.dense], cfg["grad_clip"])
             self.t += 1
+            use_muon = cfg.get("matrix_optimizer", "adamw") == "muon"
             for k in self.dense:
                 mult = (cfg["lr_mult_embed"] if k == "wte" else
                         cfg["lr_mult_head"] if k == "lm_head" else
                         cfg["lr_mult_matrix"])
+                blocks = muon_blocks(cfg, k, self.P[k].shape) if use_muon else []
+                if blocks:
+                    # Muon on each block; the AdamW first moment buffer holds its momentum
+                    g = self.acc[k] * coef
+                    for r0, r1 in blocks:
+                        self.P[k][r0:r1], self.m[k][r0:r1] = muon.muon_update(
+                            self.P[k][r0:r1], g[r0:r1], self.m[k][r0:r1], lr * mult,
+                            cfg.get("muon_momentum", 0.95), nesterov=bool(cfg.get("muon_nesterov", 1)),
+                            steps=cfg.get("muon_ns_steps", 5))
+                    self.acc[k][...] = 0.0
+                    continue
                 self.P[k], self.m[k], self.v[k] = optim.adamw(
                     self.P[k], self.acc[k] * coef, self.m[k], self.v[k], self.t,
                     lr * mult, cfg["adam_b1"], cfg["adam_b2"], cfg["adam_eps"],

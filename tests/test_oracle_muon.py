@@ -117,3 +117,73 @@ def test_momentum_schedule_endpoints():
     assert abs(muon.muon_momentum(150) - 0.90) < 1e-15
     assert abs(muon.muon_momentum(300) - 0.95) < 1e-15
     assert muon.muon_momentum(5000) == 0.95
+
+
+# --------------------------------------------------------------------------- Muon in the training step
+def _muon_step_case(**kw):
+    from synthetic import init_params, tokens_and_targets, workload
+    w = workload("tiny_fp32", x0_rows=0, n_layer=1, seq_len=16, micro_batch=2, vocab=96, **kw)
+    params = init_params(w)
+    tok, tgt = tokens_and_targets(2, 16, 96, 5)
+    return w, params, tok, tgt
+
+
+def _one_step(w, params, tok, tgt, lr=0.02):
+    from oracle.step import OracleTrainer
+    orc = OracleTrainer(w, params)
+    orc.forward_loss(tok, tgt)
+    orc.backward_step(lr)
+    return orc
+
+
+def test_muon_step_leaves_embedding_and_head_to_adamw():
+    """matrix_optimizer = "muon": the token embedding and the untied head take
+    exactly the AdamW step they take with AdamW everywhere (same gradient,
+    same clip), while every block matrix moves differently."""
+    w_a, params, tok, tgt = _muon_step_case(tie_embeddings=0)
+    w_m = dict(w_a, matrix_optimizer="muon", muon_momentum=0.9)
+    oa, om_ = _one_step(w_a, params, tok, tgt), _one_step(w_m, params, tok, tgt)
+    for k in ("wte", "lm_head"):
+        np.testing.assert_array_equal(om_.P[k], oa.P[k])
+    for k in ("h0.wqkv", "h0.wo", "h0.w1", "h0.w2"):
+        assert np.abs(om_.P[k] - oa.P[k]).max() > 1e-4
+
+
+def test_muon_step_orthogonalises_q_k_v_separately():
+    """The fused q|k|v weight is three matrices to Muon: each block's step has
+    its non-zero singular values in (0.5, 1.5) (five quintic steps; the
+    gradient of 32 tokens has rank <= 32, and the iteration keeps zero
+    singular values at zero), and the q block's step is not the q rows of the
+    whole fused matrix's orthogonalised update."""
+    from oracle.step import muon_blocks
+    lr, mu = 0.02, 0.9
+    w, params, tok, tgt = _muon_step_case(matrix_optimizer="muon", muon_momentum=mu)
+    orc = _one_step(w, params, tok, tgt, lr)
+    W0 = np.asarray(params["h0.wqkv"], dtype=np.float64)
+    step = (W0 - orc.P["h0.wqkv"]) / lr
+    blocks = muon_blocks(w, "h0.wqkv", W0.shape)
+    assert len(blocks) == 3
+    for r0, r1 in blocks:
+        sv = np.linalg.svd(step[r0:r1], compute_uv=False)   # [a, d]: wide or square, scale 1
+        nz = sv[sv > 1e-8]
+        assert 0 < len(nz) <= 32
+        assert nz.min() > 0.5 and nz.max() < 1.5, (nz.min(), nz.max())
+    g = orc.accum_grads["h0.wqkv"]
+    u = (1 - mu) * g + mu * (1 - mu) * g      # Nesterov direction from a zero buffer
+    whole = np.sqrt(max(1.0, W0.shape[0] / W0.shape[1])) * muon.newton_schulz(u)
+    r0, r1 = blocks[0]
+    assert np.linalg.norm(step[r0:r1] - whole[r0:r1]) > 0.1 * np.linalg.norm(step[r0:r1])
+
+
+def test_muon_step_clips_before_the_momentum():
+    """The global-norm clip is taken over all dense gradients before Muon: the
+    momentum buffer after the first step is (1 - mu) * coef * g, with coef =
+    max_norm / (||g|| + 1e-6) when the norm is above max_norm."""
+    mu = 0.9
+    w, params, tok, tgt = _muon_step_case(matrix_optimizer="muon", muon_momentum=mu, grad_clip=1e-3)
+    orc = _one_step(w, params, tok, tgt)
+    norm = np.sqrt(sum(float(np.sum(orc.accum_grads[k] ** 2)) for k in orc.dense))
+    assert norm > 1e-3
+    coef = 1e-3 / (norm + 1e-6)
+    for k in ("h0.wo", "h0.w1"):
+        np.testing.assert_allclose(orc.m[k], (1 - mu) * coef * orc.accum_grads[k], rtol=1e-12)
