@@ -459,48 +459,63 @@ def run_tables(args, w):
 
 
 def run_muon(args, w):
-    """One Muon step over every matrix parameter of the workload's blocks, in
-    the nanochat module's shapes ([out, in]): per layer c_q, c_k, c_v and the
-    attention projection (a x d, d x a) and the MLP's d_ff x d and d x d_ff.
-    Newton-Schulz FLOPs per matrix with R = min(out, in), C = max(out, in):
-    ns_steps * (2 R^2 C [X X^T] + 2 R^3 [A A] + 2 R^2 C [B X]).  The matrices'
-    W, M, G (fp32) exceed L2, so no flush is needed between steps."""
+    """Muon inside the training step: the workload with matrix_optimizer =
+    muon (the q, k, v blocks, projection and MLP weights of every layer on
+    Muon, batched by shape; the embedding on AdamW).  Reports the Muon part of
+    the optimizer step from CUDA events bracketing its kernels (momentum and
+    normalisation, ns_steps x three batched Newton-Schulz GEMMs and two
+    elementwise kernels per shape group, the step), the whole training step's
+    time with Muon on, and the Newton-Schulz GEMM rate.  Newton-Schulz FLOPs per
+    matrix with R = min(out, in), C = max(out, in): ns_steps * (2 R^2 C [X X^T]
+    + 2 R^3 [A A] + 2 R^2 C [B X]).  Inputs exceed L2 (no flush)."""
     import torch
     import gpt_pretraining_step_decoder_b200 as g
     dev = torch.device("cuda", 0)
-    st = torch.cuda.current_stream()
-    d, a, f, L = w["d_model"], w["n_head"] * w["head_dim"], w["d_ff"], w["n_layer"]
-    shapes = [(a, d), (a, d), (a, d), (d, a), (f, d), (d, f)] * L
-    peaks, peak_src = measured_peaks()
-    gen = torch.Generator(device=dev).manual_seed(w["seed"])
-    mats = []
-    for (o, i) in shapes:
-        W = 0.02 * torch.randn((o, i), device=dev, generator=gen)
-        G = 0.01 * torch.randn((o, i), device=dev, generator=gen)
-        mats.append((W, torch.zeros_like(W), G))
-    ws_bytes = max(g.muon_update_workspace_bytes(o, i) for (o, i) in shapes)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    steps = 5
-    flops = sum(steps * (4.0 * min(o, i) ** 2 * max(o, i) + 2.0 * min(o, i) ** 3) for (o, i) in shapes)
-    times = []
+    w = dict(w, matrix_optimizer="muon")
+    model = g.Model(g.make_config(**w), seed=w["seed"])
+    A, B, T, V = w["grad_accum"], w["micro_batch"], w["seq_len"], w["vocab"]
+    toks = [tuple(torch.from_numpy(x).to(dev) for x in tokens_and_targets(B, T, V, w["seed"], w["zipf_s"],
+                                                                        w["repeat_frac"], micro=i))
+            for i in range(A)]
+    st = model.stream
+
+    def step():
+        for tok, tgt in toks:
+            model.forward_loss(tok, tgt)
+            model.backward_step(args.lr)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(0) as clk:
-        for it in range(args.warmup + args.steps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(st)
-            for (W, M, G), (o, i) in zip(mats, shapes):
-                g.muon_update(W, M, G, o, i, 1, 0.02, 0.95, 1, steps, ws, ws_bytes)
-            e1.record(st)
-            torch.cuda.synchronize()
-            if it >= args.warmup:
-                times.append(e0.elapsed_time(e1))
-    if g.ngram_sync_status() != g.GPT_OK:
-        raise RuntimeError(f"muon_update: device error {g.gpt_last_error()}")
-    ms = float(np.median(times))
-    tflops = flops / (ms * 1e-3) / 1e12
-    line = {"metric": "Muon optimizer step over the matrix parameters (CUDA-event time)", "unit": "ms",
-            "value": ms, "workload": w["name"], "matrices": len(shapes), "ns_steps": steps,
-            "ns_gemm_flops": flops, "tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
-            "frac_of_peak": tflops / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16 burst",
+        e0.record(st)
+        for _ in range(args.steps):
+            step()
+        e1.record(st)
+        torch.cuda.synchronize()
+    step_ms = e0.elapsed_time(e1) / args.steps
+    g.gpt_profile_enable(model.h, 1)
+    for _ in range(args.steps):
+        step()
+    prof = g.gpt_profile_read(model.h)
+    g.gpt_profile_enable(model.h, 0)
+    if model.sync_status() != g.GPT_OK:
+        raise RuntimeError(f"Muon step: device error {g.gpt_last_error()}")
+    mu = {k: v for k, v in prof.items() if k.startswith("muon")}
+    ms = sum(v["ms"] for v in mu.values()) / args.steps
+    ns_ms = sum(v["ms"] for k, v in mu.items() if k.startswith("muon.")) / args.steps
+    ns_flops = sum(v["flops"] for k, v in mu.items() if k.startswith("muon.")) / args.steps
+    peaks, peak_src = measured_peaks()
+    tflops = ns_flops / (ns_ms * 1e-3) / 1e12 if ns_ms else None
+    d, f, L = w["d_model"], w["d_ff"], w["n_layer"]
+    line = {"metric": "Muon optimizer step over the block matrices inside the training step (CUDA-event time)",
+            "unit": "ms", "value": ms, "workload": w["name"], "matrices": 6 * L, "ns_steps": w.get("muon_ns_steps", 5),
+            "training_step_ms": step_ms, "share_of_step": ms / step_ms,
+            "ns_gemm_ms": ns_ms, "ns_gemm_flops": ns_flops, "tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+            "frac_of_peak": (tflops / peaks["bf16_tflops"]) if tflops else None,
+            "peak_source": f"{peak_src} bf16 burst",
+            "launches_per_step": sum(v["launches"] for v in mu.values()) / args.steps,
             "steps": args.steps, "warmup": args.warmup, "l2": "no flush: W, M, G of the matrices exceed L2",
             "clocks": clk.summary()}
     print(json.dumps(line), flush=True)

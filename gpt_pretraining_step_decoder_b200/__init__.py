@@ -17,6 +17,7 @@ GPT_OK, GPT_ERR_ARG, GPT_ERR_CONFIG, GPT_ERR_WORKSPACE, GPT_ERR_STATE = 0, 1, 2,
 GPT_ERR_INPUT, GPT_ERR_NONFINITE, GPT_ERR_CUDA, GPT_ERR_TIMEOUT = 5, 6, 7, 8
 DTYPE_F32, DTYPE_BF16, DTYPE_I32 = 0, 1, 2
 KIND_PARAM, KIND_GRAD, KIND_ADAM_M, KIND_ADAM_V, KIND_ROW_STATE, KIND_PARAM_LP, KIND_ACT = range(7)
+MATRIX_ADAMW, MATRIX_MUON = 0, 1
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -40,6 +41,8 @@ class GptConfig(ctypes.Structure):
         ("v_rows", ctypes.c_longlong), ("table_beta", ctypes.c_float),
         ("table_eps", ctypes.c_float), ("hash_p1", ctypes.c_ulonglong),
         ("hash_p2", ctypes.c_ulonglong), ("lm_chunk_rows", ctypes.c_int),
+        ("matrix_optimizer", ctypes.c_int), ("muon_momentum", ctypes.c_float),
+        ("muon_ns_steps", ctypes.c_int), ("muon_nesterov", ctypes.c_int),
     ]
 
 
@@ -131,6 +134,8 @@ def make_config(**fields):
     for k, v in fields.items():
         if k == "dtype" and isinstance(v, str):
             v = DTYPE_BF16 if v == "bf16" else DTYPE_F32
+        if k == "matrix_optimizer" and isinstance(v, str):
+            v = {"adamw": MATRIX_ADAMW, "muon": MATRIX_MUON}[v]
         if any(k == f[0] for f in GptConfig._fields_):
             setattr(c, k, v)
     if c.n_kv_head == 0 or "n_kv_head" not in fields:

@@ -91,6 +91,8 @@ template <int BN, int HEAVY, int CG = 1> struct Cfg {
 
 struct Params {
   int M, N, K;   // m_tiles counts tiles of CG * BM rows
+  int batch;     // > 1: `batch` independent products of this shape, the third
+                 // coordinate of 3-D tensor maps (store epilogues only, no split-K)
   int a_kmajor, b_kmajor;
   int m_tiles, n_tiles, splits, kb_per_split, kb_total;
   int group_m;  // tile order: groups of group_m m-blocks, m fastest inside a group
@@ -180,6 +182,15 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                    smem_u32(bar))
                : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // ---- CTA-pair (cta_group::2) forms
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -202,6 +213,14 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
       "%4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                 int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -249,21 +268,30 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 
 // Load one operand tile (rows x BK) of the k-block `kb` into `dst`.
 // K-major: one box {BK, rows}.  MN-major: rows/64 boxes {64, BK}, each 8 KB.
+// z >= 0: product z of a batch (3-D tensor map); z < 0: a 2-D map.
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
-                                             int kmajor, int rows, int r0, int kb) {
+                                             int kmajor, int rows, int r0, int kb, int z) {
   if (kmajor) {
-    tma_load_2d(dst, map, bar, kb * BK, r0);
+    if (z >= 0) tma_load_3d(dst, map, bar, kb * BK, r0, z);
+    else tma_load_2d(dst, map, bar, kb * BK, r0);
   } else {
-    for (int j = 0; j < rows / 64; ++j) tma_load_2d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+    for (int j = 0; j < rows / 64; ++j) {
+      if (z >= 0) tma_load_3d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK, z);
+      else tma_load_2d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+    }
   }
 }
 // the same, counted on the pair's stage barrier at shared::cluster address `bar`
 __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map, uint32_t bar,
-                                                  int kmajor, int rows, int r0, int kb) {
+                                                  int kmajor, int rows, int r0, int kb, int z) {
   if (kmajor) {
-    tma_load_2d_pair(dst, map, bar, kb * BK, r0);
+    if (z >= 0) tma_load_3d_pair(dst, map, bar, kb * BK, r0, z);
+    else tma_load_2d_pair(dst, map, bar, kb * BK, r0);
   } else {
-    for (int j = 0; j < rows / 64; ++j) tma_load_2d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+    for (int j = 0; j < rows / 64; ++j) {
+      if (z >= 0) tma_load_3d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK, z);
+      else tma_load_2d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+    }
   }
 }
 
@@ -375,7 +403,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles = p.m_tiles * p.n_tiles * p.splits;
+  const int per_product = p.m_tiles * p.n_tiles * p.splits;
+  const int tiles = per_product * p.batch;
   // CTA pair: rank 0 issues the MMAs; tile t goes to pair blockIdx.x / CG
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
   const int unit = blockIdx.x / CG, n_units = gridDim.x / CG;
@@ -421,8 +450,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int s = 0; s < C::STAGES; ++s) issued[s] = false;
       bool ok = true;
       for (int t = unit; t < tiles && ok; t += n_units) {
-        const int split = t % p.splits;
-        const int mn = t / p.splits;
+        const int z = p.batch > 1 ? t / per_product : -1;
+        const int tt = t % per_product;
+        const int split = tt % p.splits;
+        const int mn = tt / p.splits;
         int mt, nt;
         tile_coords(mn, p, mt, nt);
         // this CTA's A rows and B rows of the tile
@@ -436,12 +467,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // that CTA arms for the pair
             const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
             if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
-            load_operand_pair(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb);
-            load_operand_pair(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb);
+            load_operand_pair(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb, z);
+            load_operand_pair(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb, z);
           } else {
             mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-            load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb);
-            load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb);
+            load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb, z);
+            load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb, z);
           }
           issued[stage] = true;
           issued_phase[stage] = phase;
@@ -472,7 +503,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = unit; t < tiles && ok; t += n_units) {
-        const int split = t % p.splits;
+        const int split = (t % per_product) % p.splits;
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -524,8 +555,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // the accumulator-empty barrier lives in the even CTA of a pair
     const uint32_t tempty0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
     for (int t = unit; t < tiles && ok; t += n_units) {
-      const int split = t % p.splits;
-      const int mn = t / p.splits;
+      const int z = p.batch > 1 ? t / per_product : -1;
+      const int tt = t % per_product;
+      const int split = tt % p.splits;
+      const int mn = tt / p.splits;
       int mt, nt;
       tile_coords(mn, p, mt, nt);
       const int m0 = (mt * CG + (int)rank) * BM;  // this CTA's 128 accumulator rows
@@ -738,6 +771,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
           if constexpr (KM == K_PARTIAL) tma_store_3d(&tmC, stg, nc, mrow0, split);
           else if constexpr (KM == K_REDUCE_F32) tma_reduce_add_2d(&tmC, stg, nc, mrow0);
+          else if (z >= 0) tma_store_3d(&tmC, stg, nc, mrow0, z);
           else tma_store_2d(&tmC, stg, nc, mrow0);
           bulk_commit();
         }

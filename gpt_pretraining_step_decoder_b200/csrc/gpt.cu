@@ -185,7 +185,7 @@ static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const 
     CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     units = resident_clusters(kernel, C::SMEM_BYTES, CG);
   }
-  const int tiles = p.m_tiles * p.n_tiles * p.splits;
+  const int tiles = p.m_tiles * p.n_tiles * p.splits * p.batch;
   const int grid = CG * (tiles < units ? tiles : units);
   ++g_launches;
   if constexpr (CG == 1) {
@@ -207,18 +207,45 @@ static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const 
   return GPT_OK;
 }
 
+// `n` independent products of one shape whose operands and outputs lie at
+// fixed element strides (n = 1: a single product).
+struct GemmBatch {
+  int n = 1;
+  long long sa = 0, sb = 0, sc = 0;
+};
+
+// 3-D bf16 map over `batch` row-major [outer, inner] matrices `stride` elements apart
+static int make_tmap3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld, int batch,
+                      long long stride, uint32_t box_inner, uint32_t box_outer) {
+  const uint64_t dims[3] = {inner, outer, (uint64_t)batch}, str[2] = {ld * 2, (uint64_t)stride * 2};
+  const uint32_t box[3] = {box_inner, box_outer, 1};
+  return make_tmap_gen(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, str, box);
+}
+
 template <int BN, int CG = 1>
 static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, GemmEpilogue e,
-                          int splits, float* partial, unsigned* err, cudaStream_t st) {
+                          int splits, float* partial, unsigned* err, cudaStream_t st,
+                          const GemmBatch& bt = GemmBatch()) {
   static_assert(CG == 1 || BN == 256, "CTA pairs take 256-column tiles");
+  const bool b3 = bt.n > 1;
+  if (b3 && (splits > 1 || (e.mode != EPI_STORE && e.mode != EPI_STORE_F32)))
+    return fail(GPT_ERR_ARG, "batched GEMMs take store epilogues without split-K");
   CUtensorMap ta, tb, tcm, taux;
-  if (A.kmajor) TRY(make_tmap(&ta, A.ptr, K, M, A.ld, tc::BK, tc::BM));
-  else TRY(make_tmap(&ta, A.ptr, M, K, A.ld, 64, tc::BK));
-  // a CTA of a pair loads half of the tile's B rows
-  if (B.kmajor) TRY(make_tmap(&tb, B.ptr, K, N, B.ld, tc::BK, BN / CG));
-  else TRY(make_tmap(&tb, B.ptr, N, K, B.ld, 64, tc::BK));
+  if (b3) {
+    if (A.kmajor) TRY(make_tmap3(&ta, A.ptr, K, M, A.ld, bt.n, bt.sa, tc::BK, tc::BM));
+    else TRY(make_tmap3(&ta, A.ptr, M, K, A.ld, bt.n, bt.sa, 64, tc::BK));
+    if (B.kmajor) TRY(make_tmap3(&tb, B.ptr, K, N, B.ld, bt.n, bt.sb, tc::BK, BN / CG));
+    else TRY(make_tmap3(&tb, B.ptr, N, K, B.ld, bt.n, bt.sb, 64, tc::BK));
+  } else {
+    if (A.kmajor) TRY(make_tmap(&ta, A.ptr, K, M, A.ld, tc::BK, tc::BM));
+    else TRY(make_tmap(&ta, A.ptr, M, K, A.ld, 64, tc::BK));
+    // a CTA of a pair loads half of the tile's B rows
+    if (B.kmajor) TRY(make_tmap(&tb, B.ptr, K, N, B.ld, tc::BK, BN / CG));
+    else TRY(make_tmap(&tb, B.ptr, N, K, B.ld, 64, tc::BK));
+  }
   tc::Params p;
   p.M = M; p.N = N; p.K = K;
+  p.batch = bt.n;
   p.a_kmajor = A.kmajor; p.b_kmajor = B.kmajor;
   p.m_tiles = cdiv(M, CG * tc::BM);
   p.n_tiles = cdiv(N, BN);
@@ -235,7 +262,14 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   p.err = err;
   // output map: split-K partials [splits, M, N] fp32 (3-D so each split clips at M),
   // fp32 outputs in 32-column boxes, bf16 outputs in 64-column boxes (128-byte rows)
-  if (p.splits > 1) {
+  if (b3) {
+    const bool f32 = e.mode == EPI_STORE_F32;
+    const uint64_t dims[3] = {(uint64_t)N, (uint64_t)M, (uint64_t)bt.n};
+    const uint64_t str[2] = {(uint64_t)e.ldc * (f32 ? 4 : 2), (uint64_t)bt.sc * (f32 ? 4 : 2)};
+    const uint32_t box[3] = {f32 ? 32u : 64u, 32, 1};
+    TRY(make_tmap_gen(&tcm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, e.C, dims,
+                      str, box));
+  } else if (p.splits > 1) {
     const uint64_t dims[3] = {(uint64_t)N, (uint64_t)M, (uint64_t)p.splits};
     const uint64_t str[2] = {(uint64_t)N * 4, (uint64_t)M * N * 4};
     const uint32_t box[3] = {32, 32, 1};
@@ -454,6 +488,11 @@ struct Plan {
   size_t sort_keys_a, sort_keys_b, sort_vals_a, sort_vals_b, sort_counts, part_head, part_tail;
   size_t splitk; long long splitk_elems;
   size_t norm_part, clip_coef, grad_norm, rope_cs, rope_cs_t, err;
+  // Muon (matrix_optimizer == GPT_MATRIX_MUON): the block matrices in three
+  // same-shape groups and one scratch sized for the largest group
+  MuonGroup muon_groups[3];
+  int n_muon_groups = 0;
+  size_t mu_x, mu_xn, mu_abf, mu_bm, mu_a, mu_aa, mu_p, mu_part;
   int chunk;
   size_t total;
 };
@@ -485,6 +524,13 @@ static int validate(const gpt_config* c) {
   const long long N = (long long)c->micro_batch * c->seq_len;
   if (N > (1LL << 24)) return fail(GPT_ERR_CONFIG, "too many tokens per micro-batch");
   if (c->norm_eps <= 0.f || c->rope_base <= 1.f) return fail(GPT_ERR_CONFIG, "bad norm_eps or rope_base");
+  if (c->matrix_optimizer != GPT_MATRIX_ADAMW && c->matrix_optimizer != GPT_MATRIX_MUON)
+    return fail(GPT_ERR_CONFIG, "matrix_optimizer must be GPT_MATRIX_ADAMW or GPT_MATRIX_MUON");
+  if (c->matrix_optimizer == GPT_MATRIX_MUON) {
+    if (!cfg_bf16(*c)) return fail(GPT_ERR_CONFIG, "Muon runs in bf16 mode only");
+    if (!(c->muon_momentum >= 0.f && c->muon_momentum < 1.f) || c->muon_ns_steps < 0 || c->muon_ns_steps > 64)
+      return fail(GPT_ERR_CONFIG, "Muon needs 0 <= muon_momentum < 1 and 0 <= muon_ns_steps <= 64");
+  }
   return GPT_OK;
 }
 
@@ -587,6 +633,28 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.rope_cs = cv.take((long long)c.seq_len * c.head_dim * 4);
   p.rope_cs_t = cv.take((long long)c.seq_len * c.head_dim * 4);
   p.err = cv.take(16);
+  if (c.matrix_optimizer == GPT_MATRIX_MUON) {
+    // groups: [q, k, v, proj] x layers ([a, d] each; a == d), w1 [F, d] x layers, w2 [d, F] x layers
+    const long long o0 = p.dense[p.h_end == p.e_end ? 1 : 2].off;  // h0.wqkv
+    const long long lstride = c.n_layer > 1 ? p.dense[(p.h_end == p.e_end ? 1 : 2) + 4].off - o0 : 0;
+    p.muon_groups[0] = MuonGroup{o0, lstride, a * d, 4, 4 * c.n_layer, (int)a, (int)d};
+    p.muon_groups[1] = MuonGroup{o0 + 4 * a * d, lstride, 0, 1, c.n_layer, (int)F, (int)d};
+    p.muon_groups[2] = MuonGroup{o0 + 4 * a * d + F * d, lstride, 0, 1, c.n_layer, (int)d, (int)F};
+    p.n_muon_groups = 3;
+    long long xn = 0, rr = 0, nm = 0;
+    for (int gi = 0; gi < 3; ++gi) {
+      const MuonGroup& g = p.muon_groups[gi];
+      const long long R = g.rows < g.cols ? g.rows : g.cols;
+      xn = std::max(xn, (long long)g.nmat * g.rows * g.cols);
+      rr = std::max(rr, (long long)g.nmat * R * R);
+      nm = std::max(nm, (long long)g.nmat);
+    }
+    p.mu_x = cv.take(xn * 2); p.mu_xn = cv.take(xn * 2);
+    p.mu_abf = cv.take(rr * 2); p.mu_bm = cv.take(rr * 2);
+    p.mu_a = cv.take(rr * 4); p.mu_aa = cv.take(rr * 4);
+    p.mu_p = cv.take(xn * 4);
+    p.mu_part = cv.take(nm * MUON_BATCH_BLOCKS * 4);
+  }
   p.total = cv.take(0) + 256;
 }
 
@@ -625,6 +693,7 @@ extern "C" int gpt_default_config(gpt_config* c) {
   c->x0_rows = 0; c->v_rows = 0; c->table_beta = 0.95f; c->table_eps = 1e-10f;
   c->hash_p1 = 2654435761ull; c->hash_p2 = 2246822519ull;
   c->lm_chunk_rows = 0;
+  c->matrix_optimizer = GPT_MATRIX_ADAMW; c->muon_momentum = 0.95f; c->muon_ns_steps = 5; c->muon_nesterov = 1;
   return GPT_OK;
 }
 
@@ -673,6 +742,21 @@ extern "C" int gpt_create(const gpt_config* cfg, unsigned long long seed, void* 
     size_t need = m->plan.total;
     delete m;
     return fail(GPT_ERR_WORKSPACE, "arena too small: %zu < %zu bytes", arena_bytes, need);
+  }
+  if (m->plan.n_muon_groups) {
+    // the block matrices must sit at the regular offsets the Muon groups assume
+    const Plan& pl = m->plan;
+    for (int l = 0; l < cfg->n_layer; ++l) {
+      const long long L = l * pl.muon_groups[0].layer_stride;
+      const std::string pre = "h" + std::to_string(l) + ".";
+      if (find_dense(m, pre + "wqkv")->off != pl.muon_groups[0].base + L ||
+          find_dense(m, pre + "wo")->off != pl.muon_groups[0].base + L + 3 * pl.muon_groups[0].inner_stride ||
+          find_dense(m, pre + "w1")->off != pl.muon_groups[1].base + L ||
+          find_dense(m, pre + "w2")->off != pl.muon_groups[2].base + L) {
+        delete m;
+        return fail(GPT_ERR_CONFIG, "Muon groups: unexpected parameter layout");
+      }
+    }
   }
   m->base = static_cast<uint8_t*>(arena);
   m->bytes = arena_bytes;
@@ -1231,18 +1315,121 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
   return GPT_OK;
 }
 
-// Global-norm clip (optional) and AdamW over the accumulated dense gradient.
+// `bt.n` same-shape products in one launch (store epilogues, no split-K)
+static int gemm_batched(const GemmCtx& g, const GemmBatch& bt, int M, int N, int K, GemmOperand A, GemmOperand B,
+                        GemmEpilogue e, const char* label) {
+  ProfScope ps(g.prof, g.st, label, 2.0 * M * N * K * bt.n, 0.0);
+  if (N >= 256 && gemm_pairs_enabled())
+    return gemm_tc_launch<256, 2>(M, N, K, A, B, e, 1, g.splitk, g.err, g.st, bt);
+  return gemm_tc_launch<128, 1>(M, N, K, A, B, e, 1, g.splitk, g.err, g.st, bt);
+}
+
+// Muon on every block matrix, one group of same-shape matrices at a time:
+// momentum (on the clipped gradient) with a per-matrix sum of squares, the
+// normalised bf16 iterate, muon_ns_steps Newton-Schulz steps as batched GEMMs
+// over the group (X X^T or X^T X, A A, then B X or X B), and the scaled step
+// into the fp32 master and its bf16 copy.  Same arithmetic as muon_update.
+static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
+  const gpt_config& c = m->cfg;
+  const Plan& p = m->plan;
+  cudaStream_t st = m->st;
+  float* P = m->at<float>(p.P);
+  float* G = m->at<float>(p.G);
+  float* M = m->at<float>(p.M);
+  bf16* Plp = m->at<bf16>(p.Plp);
+  bf16* x = m->at<bf16>(p.mu_x);
+  bf16* xn = m->at<bf16>(p.mu_xn);
+  bf16* abf = m->at<bf16>(p.mu_abf);
+  bf16* bm = m->at<bf16>(p.mu_bm);
+  float* A = m->at<float>(p.mu_a);
+  float* AA = m->at<float>(p.mu_aa);
+  float* Pp = m->at<float>(p.mu_p);
+  float* part = m->at<float>(p.mu_part);
+  const GemmCtx g{true, m->at<float>(p.splitk), p.splitk_elems, m->err(), st, &m->prof};
+  const float ca = 3.4445f, cb = -4.7750f, cc = 2.0315f;  // a x + b x^3 + c x^5
+  auto grid1 = [](long long n4) {
+    const long long b = (n4 + MUON_THREADS - 1) / MUON_THREADS, cap = 4LL * device_sms();
+    return (unsigned)(b < 1 ? 1 : (b > cap ? cap : b));
+  };
+  for (int gi = 0; gi < p.n_muon_groups; ++gi) {
+    const MuonGroup& grp = p.muon_groups[gi];
+    const int rows = grp.rows, cols = grp.cols, nmat = grp.nmat;
+    const int R = rows < cols ? rows : cols;
+    const bool tall = rows > cols;
+    const long long n = (long long)rows * cols, rr = (long long)R * R;
+    const unsigned per_mat = (unsigned)std::min<long long>((n / 4 + MUON_THREADS - 1) / MUON_THREADS, MUON_BATCH_BLOCKS);
+    {
+      // bytes: g, m read + m written; g, m read + bf16 iterate written
+      ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * (12 + 10));
+      ++g_launches;
+      muon_batch_momentum_kernel<<<dim3(MUON_BATCH_BLOCKS, nmat), MUON_THREADS, 0, st>>>(
+          G, M, grp, c.muon_momentum, c.muon_nesterov, clip, part);
+      ++g_launches;
+      muon_batch_normalize_kernel<<<dim3(per_mat, nmat), MUON_THREADS, 0, st>>>(
+          G, M, grp, c.muon_momentum, c.muon_nesterov, clip, part, 1e-7f, x);
+      LAUNCH_CHECK();
+    }
+    for (int it = 0; it < c.muon_ns_steps; ++it) {
+      if (!tall)
+        TRY(gemm_batched(g, GemmBatch{nmat, n, n, rr}, R, R, cols, op_k(x, cols), op_k(x, cols),
+                         epi(EPI_STORE_F32, A, R), "muon.gram"));
+      else
+        TRY(gemm_batched(g, GemmBatch{nmat, n, n, rr}, R, R, rows, op_mn(x, cols), op_mn(x, cols),
+                         epi(EPI_STORE_F32, A, R), "muon.gram"));
+      {
+        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * rr * 6);
+        ++g_launches;
+        muon_to_bf16_kernel<<<grid1(nmat * rr / 4), MUON_THREADS, 0, st>>>(A, nmat * rr / 4, abf);
+      }
+      TRY(gemm_batched(g, GemmBatch{nmat, rr, rr, rr}, R, R, R, op_k(abf, R), op_mn(abf, R),
+                       epi(EPI_STORE_F32, AA, R), "muon.square"));
+      {
+        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * rr * 8);
+        ++g_launches;
+        muon_combine_kernel<<<grid1(nmat * rr / 4), MUON_THREADS, 0, st>>>(abf, AA, nmat * rr / 4, cb, cc, bm);
+      }
+      if (!tall)
+        TRY(gemm_batched(g, GemmBatch{nmat, rr, n, n}, rows, cols, R, op_k(bm, R), op_mn(x, cols),
+                         epi(EPI_STORE_F32, Pp, cols), "muon.poly"));
+      else
+        TRY(gemm_batched(g, GemmBatch{nmat, n, rr, n}, rows, cols, R, op_k(x, cols), op_mn(bm, R),
+                         epi(EPI_STORE_F32, Pp, cols), "muon.poly"));
+      {
+        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 8);
+        ++g_launches;
+        muon_combine_kernel<<<grid1(nmat * n / 4), MUON_THREADS, 0, st>>>(x, Pp, nmat * n / 4, ca, 1.f, xn);
+      }
+      LAUNCH_CHECK();
+      std::swap(x, xn);
+    }
+    // weights are [out, in] = [rows, cols]
+    const float step = (float)(lr * c.lr_mult_matrix * std::sqrt(std::max(1.0, (double)rows / cols)));
+    {
+      ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 12);
+      ++g_launches;
+      muon_batch_apply_kernel<<<dim3(per_mat, nmat), MUON_THREADS, 0, st>>>(P, Plp, x, grp, step);
+    }
+    LAUNCH_CHECK();
+    // the next group starts from the scratch's first iterate buffer again
+    if (x != m->at<bf16>(p.mu_x)) std::swap(x, xn);
+  }
+  return GPT_OK;
+}
+
+// Global-norm clip (optional) and AdamW over the accumulated dense gradient
+// (with Muon: AdamW over the embedding and head, Muon over the block matrices).
 static int optimizer_step_impl(gpt_model* m, float lr) {
   const gpt_config& c = m->cfg;
   const Plan& p = m->plan;
   const bool b16 = cfg_bf16(c);
+  const bool muon = c.matrix_optimizer == GPT_MATRIX_MUON;
   cudaStream_t st = m->st;
   unsigned* err = m->err();
-  ProfScope ps(&m->prof, st, "adamw", 0.0, (double)p.dense_n * (b16 ? 30 : 28));
+  float* coef = nullptr;
   {
+    ProfScope ps(&m->prof, st, "adamw", 0.0, (double)(muon ? p.h_end : p.dense_n) * (b16 ? 30 : 28));
     m->micro = 0;
     m->step_t += 1;
-    float* coef = nullptr;
     if (c.grad_clip > 0.f) {
       ++g_launches; sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, st>>>(m->at<float>(p.G), p.dense_n, m->at<double>(p.norm_part));
       ++g_launches; clip_coef_kernel<<<1, 256, 0, st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, c.grad_clip,
@@ -1253,7 +1440,7 @@ static int optimizer_step_impl(gpt_model* m, float lr) {
     AdamArgs aa;
     aa.p = m->at<float>(p.P); aa.g = m->at<float>(p.G); aa.m = m->at<float>(p.M); aa.v = m->at<float>(p.V);
     aa.p_lp = b16 ? m->at<bf16>(p.Plp) : nullptr;
-    aa.n = p.dense_n; aa.e_end = p.e_end; aa.h_end = p.h_end;
+    aa.n = muon ? p.h_end : p.dense_n; aa.e_end = p.e_end; aa.h_end = p.h_end;
     aa.lr_e = lr * c.lr_mult_embed; aa.lr_h = lr * c.lr_mult_head; aa.lr_m = lr * c.lr_mult_matrix;
     aa.b1 = c.adam_b1; aa.b2 = c.adam_b2; aa.eps = c.adam_eps; aa.wd = c.weight_decay;
     aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
@@ -1262,6 +1449,7 @@ static int optimizer_step_impl(gpt_model* m, float lr) {
     ++g_launches; adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
     LAUNCH_CHECK();
   }
+  if (muon) TRY(muon_step_impl(m, lr, coef));
   return GPT_OK;
 }
 

@@ -99,7 +99,24 @@ typedef struct gpt_config {
   float table_beta, table_eps;
   unsigned long long hash_p1, hash_p2;
   int lm_chunk_rows;      /* rows per LM-head/cross-entropy chunk; 0 = default    */
+  /* Optimizer of the block matrices (q, k, v blocks of wqkv, wo, w1, w2):
+   * GPT_MATRIX_ADAMW (default) or GPT_MATRIX_MUON -- Muon (modded-nanogpt
+   * README, "Proposed optimizer"; nanochat discussion #8, `Muon.step`): each
+   * of the matrices (the q, k and v blocks of the fused wqkv separately, as
+   * nanochat's c_q / c_k / c_v) takes momentum, a Newton-Schulz
+   * orthogonalised update and the step lr * lr_mult_matrix * sqrt(max(1,
+   * out / in)); the embedding and the head keep AdamW.  The global clip
+   * (grad_clip) is taken over all dense gradients before either optimizer.
+   * The Muon momentum lives in the ADAM_M buffer of those matrices.  bf16
+   * mode only (the iteration runs on the bf16 tensor cores, as the pages run it). */
+  int matrix_optimizer;
+  float muon_momentum;    /* 0.95                                                 */
+  int muon_ns_steps;      /* Newton-Schulz steps, 5                               */
+  int muon_nesterov;      /* 1: Nesterov direction (1 - mu) g + mu m              */
 } gpt_config;
+
+#define GPT_MATRIX_ADAMW 0
+#define GPT_MATRIX_MUON  1
 
 typedef struct gpt_model gpt_model;
 

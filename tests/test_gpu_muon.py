@@ -4,8 +4,11 @@ Tolerance of the orthogonalised step: the kernels run the Newton-Schulz
 iteration with bf16 operands (X, A and the polynomial rounded to bf16 each
 step, fp32 accumulation), as the pages do.  Repeating exactly those roundings
 in NumPy puts the five-step result 1.0-1.2% (relative L2) from the fp64
-iteration on every shape tested here, so the bar is 3e-2.  The momentum
-buffer is plain fp32 arithmetic: 1e-6.
+iteration on every shape tested here, inside the 2e-2 bar the step uses for
+updated weights.  The momentum buffer is plain fp32 arithmetic: 1e-6.
+
+Muon inside the training step (matrix_optimizer = muon) is compared as a whole
+step against the oracle trainer's Muon path.
 """
 
 import numpy as np
@@ -53,7 +56,7 @@ def test_muon_update_matches_fp64_oracle(g, rows, cols, out_rows, nesterov):
     Wg, Mg = _run(g, W, M, G, out_rows, lr, mu, nesterov)
     assert rel_l2(Mg, Mo) < 1e-6
     err = rel_l2((W64 - Wg) / lr, (W64 - Wo) / lr)
-    assert err < 3e-2, err
+    assert err < 2e-2, err
 
 
 def test_muon_singular_values_and_reproducibility(g):
@@ -74,3 +77,15 @@ def test_muon_singular_values_and_reproducibility(g):
 def test_muon_rejects_bad_shapes(g):
     with pytest.raises(g.GptError):
         g.muon_update_workspace_bytes(100, 128)
+
+
+@pytest.mark.parametrize("grad_clip", [0.0, 0.5])
+def test_muon_in_the_training_step(g, grad_clip):
+    """Two optimizer steps (grad_accum 2) with Muon on the block matrices (q, k,
+    v blocks separately) and AdamW on the embedding: gradients, weight changes
+    and both optimizer buffers against the oracle trainer, clip taken first."""
+    from synthetic import small_case
+    from tests.stepcheck import check, run_pair
+    w = small_case("gpt2s_bf16", grad_accum=2, matrix_optimizer="muon", muon_momentum=0.9, grad_clip=grad_clip)
+    model, orc, losses, _, params = run_pair(g, w, steps=4, lr=2e-3)
+    check(g, w, model, orc, losses, params, 1e-2, 2e-2)
