@@ -92,31 +92,37 @@ class OracleTrainer:
         self.micro += 1
         stepped = False
         if self.micro == A:
-            self.accum_grads = {k: self.acc[k].copy() for k in self.dense}
-            coef = optim.clip_coef([self.acc[k] for k in self.dense], cfg["grad_clip"])
-            self.t += 1
-            use_muon = cfg.get("matrix_optimizer", "adamw") == "muon"
-            for k in self.dense:
-                mult = (cfg["lr_mult_embed"] if k == "wte" else
-                        cfg["lr_mult_head"] if k == "lm_head" else
-                        cfg["lr_mult_matrix"])
-                blocks = muon_blocks(cfg, k, self.P[k].shape) if use_muon else []
-                if blocks:
-                    # Muon on each block; the AdamW first moment buffer holds its momentum
-                    g = self.acc[k] * coef
-                    for r0, r1 in blocks:
-                        self.P[k][r0:r1], self.m[k][r0:r1] = muon.muon_update(
-                            self.P[k][r0:r1], g[r0:r1], self.m[k][r0:r1], lr * mult,
-                            cfg.get("muon_momentum", 0.95), nesterov=bool(cfg.get("muon_nesterov", 1)),
-                            steps=cfg.get("muon_ns_steps", 5))
-                    self.acc[k][...] = 0.0
-                    continue
-                self.P[k], self.m[k], self.v[k] = optim.adamw(
-                    self.P[k], self.acc[k] * coef, self.m[k], self.v[k], self.t,
-                    lr * mult, cfg["adam_b1"], cfg["adam_b2"], cfg["adam_eps"],
-                    cfg["weight_decay"])
-                self.acc[k][...] = 0.0
-            self.micro = 0
+            self.optimizer_step(lr)
             stepped = True
         self.cache = None
         return stepped
+
+    def optimizer_step(self, lr):
+        """Clip, then AdamW (and Muon on the block matrices when configured)
+        over the accumulated gradient ``self.acc``; zeroes it."""
+        cfg = self.cfg
+        self.accum_grads = {k: self.acc[k].copy() for k in self.dense}
+        coef = optim.clip_coef([self.acc[k] for k in self.dense], cfg["grad_clip"])
+        self.t += 1
+        use_muon = cfg.get("matrix_optimizer", "adamw") == "muon"
+        for k in self.dense:
+            mult = (cfg["lr_mult_embed"] if k == "wte" else
+                    cfg["lr_mult_head"] if k == "lm_head" else
+                    cfg["lr_mult_matrix"])
+            blocks = muon_blocks(cfg, k, self.P[k].shape) if use_muon else []
+            if blocks:
+                # Muon on each block; the AdamW first moment buffer holds its momentum
+                g = self.acc[k] * coef
+                for r0, r1 in blocks:
+                    self.P[k][r0:r1], self.m[k][r0:r1] = muon.muon_update(
+                        self.P[k][r0:r1], g[r0:r1], self.m[k][r0:r1], lr * mult,
+                        cfg.get("muon_momentum", 0.95), nesterov=bool(cfg.get("muon_nesterov", 1)),
+                        steps=cfg.get("muon_ns_steps", 5))
+                self.acc[k][...] = 0.0
+                continue
+            self.P[k], self.m[k], self.v[k] = optim.adamw(
+                self.P[k], self.acc[k] * coef, self.m[k], self.v[k], self.t,
+                lr * mult, cfg["adam_b1"], cfg["adam_b2"], cfg["adam_eps"],
+                cfg["weight_decay"])
+            self.acc[k][...] = 0.0
+        self.micro = 0

@@ -66,9 +66,11 @@ def run_pair(g, w, steps, lr=1e-3, ignore_frac=0.05, seed_moments=True):
     return model, orc, losses, batches[-1][0], params
 
 
-def check(g, w, model, orc, losses, params, tol_loss, tol, stepped=True):
+def check(g, w, model, orc, losses, params, tol_loss, tol, stepped=True, no_change=()):
     """Loss, accumulated gradient, and (after an AdamW step) the change of every
-    dense weight and both AdamW moments; table row states and updated-row sets."""
+    dense weight and both AdamW moments; table row states and updated-row sets.
+    Weights named in `no_change` skip the weight-change comparison (their
+    update is compared elsewhere)."""
     for lg, lo in losses:
         assert abs(lg - lo) / abs(lo) < tol_loss, (lg, lo)
     worst = []
@@ -82,7 +84,7 @@ def check(g, w, model, orc, losses, params, tol_loss, tol, stepped=True):
             ed = rel_l2(export(model, name, g.KIND_PARAM) - p0, orc.P[name] - p0)
             em = rel_l2(export(model, name, g.KIND_ADAM_M), orc.m[name])
             ev = rel_l2(export(model, name, g.KIND_ADAM_V), orc.v[name])
-            assert ed < tol, (name, "weight change", ed)
+            assert name in no_change or ed < tol, (name, "weight change", ed)
             assert em < tol, (name, "adam m", em)
             assert ev < tol, (name, "adam v", ev)
             row += [ed, em, ev]
