@@ -11,6 +11,8 @@ Model (nanochat discussion #8, user-pasted GPT module, ``GPT.forward`` and
     per layer:
         u = norm(x)
         q, k, v = split(u @ Wqkv.T);  v += Hv[rv_t]        (value table optional)
+                                      v += vproj S3[r3_t]  (frozen trigram statistics, optional;
+                                                            oracle/trigram.py)
         q, k = norm_head(rope(q)), norm_head(rope(k))      (QK-norm after RoPE)
         o = softmax(q k^T / sqrt(hd) + causal) v
         x = x + o @ Wo.T
@@ -109,12 +111,14 @@ def _unheads(x):
     return x.transpose(0, 2, 1, 3).reshape(B * T, H * hd)
 
 
-def forward(cfg, P, tokens, targets, rows_x=None, rows_v=None):
+def forward(cfg, P, tokens, targets, rows_x=None, rows_v=None, rows_3=None):
     """Forward pass; returns (loss, per_token_loss, cache).
 
-    P: dict of float64 parameters in the ``synthetic.param_shapes`` layout.
+    P: dict of float64 parameters in the ``synthetic.param_shapes`` layout
+    (plus the frozen trigram statistics "h3" when "vproj" is present).
     tokens/targets: int [B, T]; targets == -1 are ignored.  rows_x/rows_v are
-    the bigram table rows [B, T] when the tables are present.
+    the bigram table rows [B, T] when the tables are present, rows_3 the
+    trigram table rows.
     """
     B, T = tokens.shape
     d, H, hd, V = cfg["d_model"], cfg["n_head"], cfg["head_dim"], cfg["vocab"]
@@ -131,6 +135,10 @@ def forward(cfg, P, tokens, targets, rows_x=None, rows_v=None):
         x = x + P["hx"][rows_x.reshape(N)]
     cos, sin = rope_tables(T, hd, cfg["rope_base"])
     c["cos"], c["sin"] = cos, sin
+    vbias3 = None
+    if "vproj" in P:
+        c["s3g"] = P["h3"][rows_3.reshape(N)]      # [N, width] statistics of each position
+        vbias3 = c["s3g"] @ P["vproj"].T           # [N, a], the same in every layer
 
     layers = []
     for layer in range(cfg["n_layer"]):
@@ -142,6 +150,8 @@ def forward(cfg, P, tokens, targets, rows_x=None, rows_v=None):
         q, k, v = qkv[:, :a], qkv[:, a:2 * a], qkv[:, 2 * a:]
         if "hv" in P:
             v = v + P["hv"][rows_v.reshape(N)]
+        if vbias3 is not None:
+            v = v + vbias3
         qh, kh, vh = _heads(q, B, T, H, hd), _heads(k, B, T, H, hd), _heads(v, B, T, H, hd)
         qr, kr = rope(qh, cos, sin), rope(kh, cos, sin)
         if cfg["qk_norm"]:
@@ -243,6 +253,8 @@ def backward(cfg, P, c, scale=1.0):
         du = dqkv @ P[f"h{layer}.wqkv"]
         dx = dx + rmsnorm_bwd(du, L["u"], L["rstd1"])
     gx0 = dx
+    if "vproj" in P:
+        G["vproj"] = gv.T @ c["s3g"]
     # ---- embedding: h = norm(wte[tok])
     dh = rmsnorm_bwd(gx0, c["h"], c["emb_rstd"])
     dwte = np.zeros_like(P["wte"])

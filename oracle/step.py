@@ -21,6 +21,7 @@ import numpy as np
 
 from . import model, muon, optim
 from .hashing import bigram_rows
+from .trigram import P3, trigram_rows
 
 
 def muon_blocks(cfg, name, shape):
@@ -38,7 +39,7 @@ class OracleTrainer:
     def __init__(self, cfg, params, table_state=None):
         self.cfg = cfg
         self.P = {k: np.array(v, dtype=np.float64) for k, v in params.items()}
-        self.dense = [k for k in self.P if k not in ("hx", "hv")]
+        self.dense = [k for k in self.P if k not in ("hx", "hv", "h3")]
         self.m = {k: np.zeros_like(self.P[k]) for k in self.dense}
         self.v = {k: np.zeros_like(self.P[k]) for k in self.dense}
         self.acc = {k: np.zeros_like(self.P[k]) for k in self.dense}
@@ -65,9 +66,16 @@ class OracleTrainer:
                              cfg["v_rows"])
         return rx, rv
 
+    def rows3(self, tokens):
+        cfg = self.cfg
+        if not cfg.get("tri_rows", 0):
+            return None
+        return trigram_rows(tokens, cfg["vocab"], cfg["hash_p1"], cfg["hash_p2"], cfg["tri_rows"],
+                            cfg.get("hash_p3", P3))
+
     def forward_loss(self, tokens, targets):
         rx, rv = self.rows(tokens)
-        loss, per_tok, c = model.forward(self.cfg, self.P, tokens, targets, rx, rv)
+        loss, per_tok, c = model.forward(self.cfg, self.P, tokens, targets, rx, rv, self.rows3(tokens))
         c["rx"], c["rv"] = rx, rv
         self.cache = c
         return loss, per_tok

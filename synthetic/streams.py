@@ -92,6 +92,8 @@ def param_shapes(cfg):
     out = {"wte": (V, d)}
     if not cfg["tie_embeddings"]:
         out["lm_head"] = (V, d)
+    if cfg.get("tri_rows", 0):
+        out["vproj"] = (a, cfg["tri_width"])   # projection of the frozen trigram statistics
     for layer in range(cfg["n_layer"]):
         out[f"h{layer}.wqkv"] = (3 * a, d)
         out[f"h{layer}.wo"] = (d, a)

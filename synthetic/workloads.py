@@ -29,6 +29,7 @@ _BASE = dict(
     lr_mult_embed=1.0, lr_mult_head=1.0, lr_mult_matrix=1.0, lr_mult_table=1.0,
     x0_rows=0, v_rows=0, table_beta=0.95, table_eps=1e-10,
     hash_p1=2654435761, hash_p2=2246822519,
+    tri_rows=0, tri_width=64, hash_p3=3266489917,
     seed=0, zipf_s=1.1, repeat_frac=0.0, repeat_span=256,
 )
 
