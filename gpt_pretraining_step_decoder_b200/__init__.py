@@ -43,6 +43,7 @@ class GptConfig(ctypes.Structure):
         ("hash_p2", ctypes.c_ulonglong), ("lm_chunk_rows", ctypes.c_int),
         ("matrix_optimizer", ctypes.c_int), ("muon_momentum", ctypes.c_float),
         ("muon_ns_steps", ctypes.c_int), ("muon_nesterov", ctypes.c_int),
+        ("tri_rows", ctypes.c_longlong), ("tri_width", ctypes.c_int), ("hash_p3", ctypes.c_ulonglong),
     ]
 
 
@@ -81,6 +82,8 @@ _SIGS = {
     "ngram_sparse_update_noalloc": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P],
     "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
     "gptx_set_gemm_cta_pairs": [_I],
+    "trigram_tally_workspace_bytes": [_LL, _I, ctypes.POINTER(_SZ)],
+    "trigram_tally": [_P, _I, _I, _I, _ULL, _ULL, _ULL, _LL, _I, _I, _P, _P, _SZ, _P],
     "muon_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
     "muon_update": [_P, _P, _P, _I, _I, _I, _F, _F, _I, _I, _P, _SZ, _P],
 }
@@ -287,6 +290,18 @@ def gptx_gemm_bf16(M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, C, ldc, beta=0, 
     return _check(_lib.gptx_gemm_bf16(M, N, K, _ptr(A), lda, a_kmajor, _ptr(B), ldb, b_kmajor, mode,
                                       _ptr(C), ldc, _ptr(aux), beta, splits, _ptr(workspace), ws_bytes,
                                       _stream(stream)), "gptx_gemm_bf16")
+
+
+def trigram_tally_workspace_bytes(rows, width):
+    n = ctypes.c_size_t()
+    _check(_lib.trigram_tally_workspace_bytes(rows, width, ctypes.byref(n)), "trigram_tally_workspace_bytes")
+    return n.value
+
+
+def trigram_tally(streams, S, L, vocab, p1, p2, p3, rows, width, dtype, table, workspace, ws_bytes, stream=None):
+    """Fill the frozen trigram statistics table from token streams [S, L] (device int32)."""
+    return _check(_lib.trigram_tally(_ptr(streams), S, L, vocab, p1, p2, p3, rows, width, dtype, _ptr(table),
+                                     _ptr(workspace), ws_bytes, _stream(stream)), "trigram_tally")
 
 
 def gptx_set_gemm_cta_pairs(on):

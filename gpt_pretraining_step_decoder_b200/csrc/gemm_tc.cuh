@@ -651,8 +651,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           } else if (e.hv && row_ok) {
             // the value-table row of this position (decoder-rtx posts: table "added to values")
+            // row rv[m] of the value table, or (rv null) row m of a per-position bias
             const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const act_t*>(e.hv) +
-                                                              (long long)e.rv[m] * (e.H * 128) + hi * 128);
+                                                              (long long)(e.rv ? e.rv[m] : m) * (e.H * 128) +
+                                                              hi * 128);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const uint4 raw = src[j];

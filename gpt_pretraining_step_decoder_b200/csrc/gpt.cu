@@ -481,6 +481,8 @@ struct Plan {
   long long dense_n = 0, e_end = 0, h_end = 0;
   size_t P, G, M, V, Plp;
   size_t hx = 0, hv = 0, hx_state = 0, hv_state = 0;
+  size_t h3 = 0, rows_3 = 0, s3g = 0, p3 = 0, vb = 0, gv16 = 0;  // frozen trigram statistics
+  long long blocks_begin = 0;  // element offset of h0.wqkv: the block matrices start here
   size_t x, emb_rstd, xf, rstd_f, tok_copy, rows_x, rows_v;
   std::vector<LayerActs> layers;
   size_t dx, dx_lp, du, dqkv, da, dout, Dattn, gv, dxf, pending;
@@ -524,6 +526,9 @@ static int validate(const gpt_config* c) {
   const long long N = (long long)c->micro_batch * c->seq_len;
   if (N > (1LL << 24)) return fail(GPT_ERR_CONFIG, "too many tokens per micro-batch");
   if (c->norm_eps <= 0.f || c->rope_base <= 1.f) return fail(GPT_ERR_CONFIG, "bad norm_eps or rope_base");
+  if (c->tri_rows < 0 || c->tri_rows > 0x7fffffffLL) return fail(GPT_ERR_CONFIG, "tri_rows out of range");
+  if (c->tri_rows && (c->tri_width < 4 || c->tri_width > 1024 || c->tri_width % (cfg_bf16(*c) ? 64 : 4)))
+    return fail(GPT_ERR_CONFIG, "tri_width must be in [4, 1024], a multiple of 64 in bf16 mode (4 in fp32 mode)");
   if (c->matrix_optimizer != GPT_MATRIX_ADAMW && c->matrix_optimizer != GPT_MATRIX_MUON)
     return fail(GPT_ERR_CONFIG, "matrix_optimizer must be GPT_MATRIX_ADAMW or GPT_MATRIX_MUON");
   if (c->matrix_optimizer == GPT_MATRIX_MUON) {
@@ -550,6 +555,8 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.e_end = off;
   if (!c.tie_embeddings) add("lm_head", V, d);
   p.h_end = off;
+  if (c.tri_rows) add("vproj", a, c.tri_width);   // matrix learning rate (past h_end)
+  p.blocks_begin = off;
   for (int l = 0; l < c.n_layer; ++l) {
     add("h" + std::to_string(l) + ".wqkv", 3 * a, d);
     add("h" + std::to_string(l) + ".wo", d, a);
@@ -566,6 +573,14 @@ static void make_plan(const gpt_config& c, Plan& p) {
   const size_t tes = b16 ? 2 : 4;
   if (c.x0_rows) { p.hx = cv.take(c.x0_rows * d * tes); p.hx_state = cv.take(c.x0_rows * 4); }
   if (c.v_rows) { p.hv = cv.take(c.v_rows * a * tes); p.hv_state = cv.take(c.v_rows * 4); }
+  if (c.tri_rows) {
+    p.h3 = cv.take(c.tri_rows * c.tri_width * tes);
+    p.rows_3 = cv.take(N * 4);
+    p.s3g = cv.take(N * c.tri_width * es);
+    p.p3 = cv.take(N * a * 4);
+    p.vb = cv.take(N * a * es);
+    p.gv16 = b16 ? cv.take(N * a * 2) : 0;
+  }
   // ---- activations
   p.x = cv.take(N * d * 4);
   p.emb_rstd = cv.take(N * 4);
@@ -596,7 +611,7 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.da = cv.take(N * F * es);
   p.dout = cv.take(N * a * es);
   p.Dattn = cv.take(BH * c.seq_len * 4);
-  p.gv = c.v_rows ? cv.take(N * a * 4) : 0;
+  p.gv = (c.v_rows || c.tri_rows) ? cv.take(N * a * 4) : 0;
   p.dxf = cv.take(N * d * 4);
   p.pending = cv.take(V * d * 4);
   // ---- LM head chunk
@@ -635,8 +650,10 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.err = cv.take(16);
   if (c.matrix_optimizer == GPT_MATRIX_MUON) {
     // groups: [q, k, v, proj] x layers ([a, d] each; a == d), w1 [F, d] x layers, w2 [d, F] x layers
-    const long long o0 = p.dense[p.h_end == p.e_end ? 1 : 2].off;  // h0.wqkv
-    const long long lstride = c.n_layer > 1 ? p.dense[(p.h_end == p.e_end ? 1 : 2) + 4].off - o0 : 0;
+    int i0 = 0;
+    while (p.dense[i0].name != "h0.wqkv") ++i0;
+    const long long o0 = p.dense[i0].off;
+    const long long lstride = c.n_layer > 1 ? p.dense[i0 + 4].off - o0 : 0;
     p.muon_groups[0] = MuonGroup{o0, lstride, a * d, 4, 4 * c.n_layer, (int)a, (int)d};
     p.muon_groups[1] = MuonGroup{o0 + 4 * a * d, lstride, 0, 1, c.n_layer, (int)F, (int)d};
     p.muon_groups[2] = MuonGroup{o0 + 4 * a * d + F * d, lstride, 0, 1, c.n_layer, (int)d, (int)F};
@@ -694,6 +711,7 @@ extern "C" int gpt_default_config(gpt_config* c) {
   c->hash_p1 = 2654435761ull; c->hash_p2 = 2246822519ull;
   c->lm_chunk_rows = 0;
   c->matrix_optimizer = GPT_MATRIX_ADAMW; c->muon_momentum = 0.95f; c->muon_ns_steps = 5; c->muon_nesterov = 1;
+  c->tri_rows = 0; c->tri_width = 64; c->hash_p3 = 3266489917ull;
   return GPT_OK;
 }
 
@@ -852,6 +870,7 @@ extern "C" int gpt_tensor(gpt_model* m, const char* name, int kind, void** ptr, 
     if (nm == "per_token_loss") { ptr_out = m->at<float>(p.tok_loss); sh[0] = c.micro_batch; sh[1] = c.seq_len; }
     else if (nm == "rows_x" && c.x0_rows) { ptr_out = m->at<int32_t>(p.rows_x); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
     else if (nm == "rows_v" && c.v_rows) { ptr_out = m->at<int32_t>(p.rows_v); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
+    else if (nm == "rows_3" && c.tri_rows) { ptr_out = m->at<int32_t>(p.rows_3); dt = GPT_DTYPE_I32; sh[0] = c.micro_batch; sh[1] = c.seq_len; }
     else if (nm == "grad_norm") { ptr_out = m->at<float>(p.grad_norm); }
     else if (nm == "table_grad_x" && c.x0_rows) { ptr_out = m->at<float>(p.dx); sh[0] = N; sh[1] = c.d_model; }
     else if (nm == "table_grad_v" && c.v_rows) { ptr_out = m->at<float>(p.gv); sh[0] = N; sh[1] = a; }
@@ -866,6 +885,11 @@ extern "C" int gpt_tensor(gpt_model* m, const char* name, int kind, void** ptr, 
       case GPT_KIND_ADAM_V: ptr_out = m->at<float>(p.V); break;
       default: return fail(GPT_ERR_ARG, "flat buffer '*' has kinds PARAM, GRAD, ADAM_M, ADAM_V");
     }
+  } else if (nm == "h3") {
+    if (!c.tri_rows) return fail(GPT_ERR_ARG, "trigram table absent");
+    if (kind != GPT_KIND_PARAM) return fail(GPT_ERR_ARG, "the trigram table has kind PARAM only");
+    ptr_out = m->base + p.h3; dt = b16 ? GPT_DTYPE_BF16 : GPT_DTYPE_F32;
+    sh[0] = c.tri_rows; sh[1] = c.tri_width;
   } else if (nm == "hx" || nm == "hv") {
     const bool isx = nm == "hx";
     const long long rows = isx ? c.x0_rows : c.v_rows;
@@ -1107,6 +1131,40 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
         c.v_rows ? m->at<int32_t>(p.rows_v) : nullptr, err);
     LAUNCH_CHECK();
   }
+  // per-position value bias of the frozen trigram statistics: vb = S3[r3] vproj^T
+  // (+ the value-table row), added to v by every layer
+  const act_t* vbias = c.v_rows ? reinterpret_cast<const act_t*>(m->base + p.hv) : nullptr;
+  const int32_t* vrows = m->at<int32_t>(p.rows_v);
+  if (c.tri_rows) {
+    const int w3 = c.tri_width;
+    {
+      ProfScope ps(pf, st, "trigram_gather", 0.0, (double)N * (12 + 2.0 * w3 * es));
+      ++g_launches; trigram_hash_kernel<<<grid_for(N, 256), 256, 0, st>>>(
+          tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.hash_p3, c.tri_rows,
+          m->at<int32_t>(p.rows_3), err);
+      const act_t* h3 = reinterpret_cast<const act_t*>(m->base + p.h3);
+      act_t* s3g = m->at<act_t>(p.s3g);
+      if (b16) {
+        ++g_launches; ngram_gather_bf16x8_kernel<<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+            m->at<int32_t>(p.rows_3), N, reinterpret_cast<const bf16*>(h3), c.tri_rows, w3,
+            reinterpret_cast<bf16*>(s3g), 0, err);
+      } else {
+        ++g_launches; ngram_gather_kernel<act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+            m->at<int32_t>(p.rows_3), N, h3, c.tri_rows, w3, s3g, 0, err);
+      }
+      LAUNCH_CHECK();
+    }
+    TRY(gemm(g, N, a, w3, op_k(m->at<act_t>(p.s3g), w3), op_k(W("vproj"), w3),
+             epi(EPI_STORE_F32, m->at<float>(p.p3), a), false, "gemm.vproj_fwd"));
+    {
+      ProfScope ps(pf, st, "value_bias", 0.0, (double)N * a * (4 + es + (c.v_rows ? es : 0)));
+      ++g_launches; value_bias_kernel<act_t><<<4 * device_sms(), 256, 0, st>>>(
+          m->at<float>(p.p3), vbias, vrows, N, a, m->at<act_t>(p.vb));
+      LAUNCH_CHECK();
+    }
+    vbias = m->at<act_t>(p.vb);
+    vrows = nullptr;  // row n of the bias for position n
+  }
   float* x = m->at<float>(p.x);
   {
   ProfScope ps(pf, st, "embed", 0.0, (double)N * d * (es + 4 + (c.x0_rows ? es : 0)));
@@ -1135,16 +1193,15 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       eq.rope = m->at<float>(p.rope_cs_t);
       eq.rstd_q = m->at<float>(L.rstd_q);
       eq.rstd_k = m->at<float>(L.rstd_k);
-      eq.hv = c.v_rows ? (const void*)(m->base + p.hv) : nullptr;
-      eq.rv = m->at<int32_t>(p.rows_v);
+      eq.hv = vbias;
+      eq.rv = vrows;
       eq.T = c.seq_len; eq.H = H; eq.qk_norm = c.qk_norm; eq.eps = c.norm_eps;
       TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), eq, false, "gemm.qkv_fwd"));
     } else {
       TRY(gemm(g, N, 3 * a, d, op_k(u, d), op_k(W(pre + "wqkv"), d), epi(EPI_STORE, qkv, 3 * a), false, "gemm.qkv_fwd"));
       ProfScope ps(pf, st, "rope_qknorm_fwd", 0.0, (double)N * a * es * (4 + (c.v_rows ? 3 : 0)));
       ++g_launches; rope_qknorm_fwd_kernel<act_t, act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
-          qkv, m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
-          c.v_rows ? reinterpret_cast<const act_t*>(m->base + p.hv) : nullptr, m->at<int32_t>(p.rows_v), N,
+          qkv, m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k), vbias, vrows, N,
           c.seq_len, H, hd, c.qk_norm, c.norm_eps);
       LAUNCH_CHECK();
     }
@@ -1266,12 +1323,12 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
       if (b16)  // hd == 128 in bf16 mode
         ++g_launches, rope_qknorm_bwd_hd128_kernel<<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
             reinterpret_cast<bf16*>(dqkv), reinterpret_cast<const bf16*>(m->at<act_t>(L.qkv)), m->at<float>(p.rope_cs),
-            m->at<float>(L.rstd_q), m->at<float>(L.rstd_k), c.v_rows ? m->at<float>(p.gv) : nullptr,
+            m->at<float>(L.rstd_q), m->at<float>(L.rstd_k), p.gv ? m->at<float>(p.gv) : nullptr,
             l != c.n_layer - 1, N, c.seq_len, H, c.qk_norm);
       else
         ++g_launches, rope_qknorm_bwd_kernel<act_t><<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
             dqkv, m->at<act_t>(L.qkv), m->at<float>(p.rope_cs), m->at<float>(L.rstd_q), m->at<float>(L.rstd_k),
-            c.v_rows ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
+            p.gv ? m->at<float>(p.gv) : nullptr, l != c.n_layer - 1, N, c.seq_len, H, hd, c.qk_norm);
       LAUNCH_CHECK();
     }
     TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true, "gemm.qkv_wgrad"));
@@ -1280,6 +1337,23 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     LAUNCH_CHECK(); }
   }
   // dx now holds dL/dx0 per position.
+  if (c.tri_rows) {
+    // projection of the frozen trigram statistics: d vproj += gv^T S3[r3], gv the
+    // value gradient summed over layers (no gradient reaches the table)
+    const int w3 = c.tri_width;
+    const act_t* gva;
+    if (b16) {
+      ProfScope ps(pf, st, "value_grad_bf16", 0.0, (double)N * a * 6);
+      ++g_launches; to_bf16_kernel<<<4 * device_sms(), 256, 0, st>>>(m->at<float>(p.gv), m->at<bf16>(p.gv16),
+                                                                     (long long)N * a);
+      LAUNCH_CHECK();
+      gva = reinterpret_cast<const act_t*>(m->at<bf16>(p.gv16));
+    } else {
+      gva = reinterpret_cast<const act_t*>(m->at<float>(p.gv));
+    }
+    TRY(gemm(g, a, w3, N, op_mn(gva, a), op_mn(m->at<act_t>(p.s3g), w3),
+             epi(EPI_ACCUM_F32, Gp("vproj"), w3, beta), true, "gemm.vproj_wgrad"));
+  }
   const SortWs w = sort_ws(m);
   {
     // token embedding gradient, bucketed by token id
@@ -1427,7 +1501,7 @@ static int optimizer_step_impl(gpt_model* m, float lr) {
   unsigned* err = m->err();
   float* coef = nullptr;
   {
-    ProfScope ps(&m->prof, st, "adamw", 0.0, (double)(muon ? p.h_end : p.dense_n) * (b16 ? 30 : 28));
+    ProfScope ps(&m->prof, st, "adamw", 0.0, (double)(muon ? p.blocks_begin : p.dense_n) * (b16 ? 30 : 28));
     m->micro = 0;
     m->step_t += 1;
     if (c.grad_clip > 0.f) {
@@ -1440,7 +1514,7 @@ static int optimizer_step_impl(gpt_model* m, float lr) {
     AdamArgs aa;
     aa.p = m->at<float>(p.P); aa.g = m->at<float>(p.G); aa.m = m->at<float>(p.M); aa.v = m->at<float>(p.V);
     aa.p_lp = b16 ? m->at<bf16>(p.Plp) : nullptr;
-    aa.n = muon ? p.h_end : p.dense_n; aa.e_end = p.e_end; aa.h_end = p.h_end;
+    aa.n = muon ? p.blocks_begin : p.dense_n; aa.e_end = p.e_end; aa.h_end = p.h_end;
     aa.lr_e = lr * c.lr_mult_embed; aa.lr_h = lr * c.lr_mult_head; aa.lr_m = lr * c.lr_mult_matrix;
     aa.b1 = c.adam_b1; aa.b2 = c.adam_b2; aa.eps = c.adam_eps; aa.wd = c.weight_decay;
     aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
@@ -1677,6 +1751,44 @@ extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda,
     return gemm_tc_launch<192>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   if (N >= 256) return gemm_tc_launch<256>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
   return gemm_tc_launch<128>(M, N, K, a, b, e, splits, (float*)workspace, err, g.st);
+}
+
+// ======================================================================== trigram statistics
+extern "C" int trigram_tally_workspace_bytes(long long rows, int width, size_t* bytes) {
+  if (!bytes || rows < 1 || width < 1) return fail(GPT_ERR_ARG, "trigram_tally_workspace_bytes: bad argument");
+  *bytes = (size_t)rows * width * 4;
+  return GPT_OK;
+}
+
+extern "C" int trigram_tally(const int32_t* streams, int S, int L, int vocab, unsigned long long p1,
+                             unsigned long long p2, unsigned long long p3, long long rows, int width, int dtype,
+                             void* table, void* workspace, size_t ws_bytes, void* stream) {
+  if (!table || S < 0 || L < 0 || vocab < 1 || rows < 1 || rows > 0x7fffffffLL || width < 1 || width > 1024 ||
+      (S > 0 && L > 0 && !streams))
+    return fail(GPT_ERR_ARG, "trigram_tally: bad argument");
+  if (dtype != GPT_DTYPE_F32 && dtype != GPT_DTYPE_BF16) return fail(GPT_ERR_ARG, "trigram_tally: bad dtype");
+  const size_t need = (size_t)rows * width * 4;
+  if (!workspace || ws_bytes < need) return fail(GPT_ERR_WORKSPACE, "trigram_tally: needs %zu bytes of workspace", need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(GPT_ERR_ARG, "workspace not 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  unsigned* counts = static_cast<unsigned*>(workspace);
+  CUDA_TRY(cudaMemsetAsync(counts, 0, need, st));
+  const long long npos = L > 1 ? (long long)S * (L - 1) : 0;
+  if (npos > 0) {
+    ++g_launches; trigram_count_kernel<<<grid_for(npos, 256), 256, 0, st>>>(streams, S, L, vocab, p1, p2, p3, rows,
+                                                                           width, counts, err);
+  }
+  if (dtype == GPT_DTYPE_BF16) {
+    ++g_launches; trigram_normalize_kernel<bf16><<<grid_for(rows * 32, 256), 256, 0, st>>>(counts, rows, width,
+                                                                                           (bf16*)table);
+  } else {
+    ++g_launches; trigram_normalize_kernel<float><<<grid_for(rows * 32, 256), 256, 0, st>>>(counts, rows, width,
+                                                                                            (float*)table);
+  }
+  LAUNCH_CHECK();
+  return GPT_OK;
 }
 
 // ======================================================================== Muon

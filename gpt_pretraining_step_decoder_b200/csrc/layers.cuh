@@ -204,8 +204,9 @@ __global__ void rope_qknorm_fwd_kernel(act_t* __restrict__ qkv, const float* __r
     }
   }
   if (hv) {
+    // the value-table row of this position, or (rv null) row n of a per-position bias
     act_t* v = row + 2 * a + h * hd;
-    const tab_t* src = hv + (long long)rv[n] * a + h * hd;
+    const tab_t* src = hv + (long long)(rv ? rv[n] : n) * a + h * hd;
     for (int i = lane; i < hd; i += 32) v[i] = from_f<act_t>(to_f(v[i]) + to_f(src[i]));
   }
 }

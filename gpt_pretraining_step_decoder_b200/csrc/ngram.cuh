@@ -847,3 +847,92 @@ __global__ void __launch_bounds__(CHAIN_WARPS * 32, NV <= 6 ? 2 : 1) emb_chain_k
     __syncthreads();  // chain_sh is refilled for the next chain
   }
 }
+
+// ============================================================================
+// Frozen trigram statistics table (decoder-rtx posts: "a 2M row tri-gram stats
+// table (tallied from dataset, frozen), projected and added to values").  The
+// row of position t hashes the token triple (x_{t-2}, x_{t-1}, x_t) in the form
+// of the bigram key, key = a2*p1 XOR a1*p2 XOR c*p3 over uint64, the vocabulary
+// size standing for tokens before the start; row = key mod rows.  A row holds
+// the next-token statistics tallied over a token stream: the share of its
+// occurrences whose next token falls in bucket (next mod width).
+
+__device__ __forceinline__ unsigned long long trigram_key(int a2, int a1, int c, unsigned long long p1,
+                                                          unsigned long long p2, unsigned long long p3) {
+  return ((unsigned long long)a2 * p1) ^ ((unsigned long long)a1 * p2) ^ ((unsigned long long)c * p3);
+}
+
+// rows of every position of tokens [B, T]; out-of-range ids set the error word and give row 0
+__global__ void trigram_hash_kernel(const int32_t* __restrict__ tok, int B, int T, int V, unsigned long long p1,
+                                    unsigned long long p2, unsigned long long p3, long long rows,
+                                    int32_t* __restrict__ out, unsigned* err) {
+  const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= (long long)B * T) return;
+  const int t = (int)(n % T);
+  const int c = tok[n];
+  const int a1 = t > 0 ? tok[n - 1] : V;
+  const int a2 = t > 1 ? tok[n - 2] : V;
+  if (c < 0 || c >= V || a1 < 0 || a1 > V || a2 < 0 || a2 > V) {
+    set_error(err, GPT_EBIT_INPUT);
+    out[n] = 0;
+    return;
+  }
+  out[n] = (int32_t)(trigram_key(a2, a1, c, p1, p2, p3) % (unsigned long long)rows);
+}
+
+// counts[row, next mod width] += 1 for every position t < L - 1 of streams [S, L]
+// (integer adds: the counts do not depend on their order)
+__global__ void trigram_count_kernel(const int32_t* __restrict__ streams, int S, int L, int V,
+                                     unsigned long long p1, unsigned long long p2, unsigned long long p3,
+                                     long long rows, int width, unsigned* __restrict__ counts, unsigned* err) {
+  const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= (long long)S * (L - 1)) return;
+  const long long s = n / (L - 1);
+  const int t = (int)(n % (L - 1));
+  const int32_t* x = streams + s * L;
+  const int c = x[t], nx = x[t + 1];
+  const int a1 = t > 0 ? x[t - 1] : V;
+  const int a2 = t > 1 ? x[t - 2] : V;
+  if (c < 0 || c >= V || nx < 0 || nx >= V || a1 < 0 || a1 > V || a2 < 0 || a2 > V) {
+    set_error(err, GPT_EBIT_INPUT);
+    return;
+  }
+  const long long r = (long long)(trigram_key(a2, a1, c, p1, p2, p3) % (unsigned long long)rows);
+  atomicAdd(&counts[r * width + nx % width], 1u);
+}
+
+// table[row, :] = counts[row, :] / (sum of the row's counts); rows never seen stay 0.
+// One warp per row; the sum is exact (integers) and each entry one fp32 division.
+template <typename tab_t>
+__global__ void trigram_normalize_kernel(const unsigned* __restrict__ counts, long long rows, int width,
+                                         tab_t* __restrict__ table) {
+  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const unsigned* c = counts + r * width;
+  unsigned long long tot = 0;
+  for (int b = lane; b < width; b += 32) tot += c[b];
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  const float ft = (float)tot;
+  for (int b = lane; b < width; b += 32) table[r * width + b] = from_f<tab_t>(tot ? (float)c[b] / ft : 0.f);
+}
+
+// vb[t] = p3[t] (+ the value-table row hv[rv[t]]) in the activation type:
+// the per-position value bias every layer adds to v
+template <typename act_t>
+__global__ void value_bias_kernel(const float* __restrict__ p3, const act_t* __restrict__ hv,
+                                  const int32_t* __restrict__ rv, long long N, int a, act_t* __restrict__ vb) {
+  const long long total4 = N * a / 4;
+  for (long long i4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; i4 < total4;
+       i4 += (long long)gridDim.x * blockDim.x) {
+    const long long i = i4 * 4, n = i / a, j = i % a;
+    float v[4];
+    load4(p3 + i, v);
+    if (hv) {
+      float h[4];
+      load4(hv + (long long)rv[n] * a + j, h);
+      v[0] += h[0]; v[1] += h[1]; v[2] += h[2]; v[3] += h[3];
+    }
+    store4(vb + i, v);
+  }
+}

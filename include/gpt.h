@@ -113,6 +113,18 @@ typedef struct gpt_config {
   float muon_momentum;    /* 0.95                                                 */
   int muon_ns_steps;      /* Newton-Schulz steps, 5                               */
   int muon_nesterov;      /* 1: Nesterov direction (1 - mu) g + mu m              */
+  /* Frozen trigram statistics table (decoder-rtx posts: "a 2M row tri-gram
+   * stats table (tallied from dataset, frozen), projected and added to
+   * values"): tri_rows rows of tri_width statistics (0 rows = absent).  Row of
+   * position t: (x_{t-2} * hash_p1 XOR x_{t-1} * hash_p2 XOR x_t * hash_p3) mod
+   * tri_rows over uint64 (the vocabulary size for tokens before the start).
+   * Every layer adds vproj * S3[row] to the values, vproj [n_head * head_dim,
+   * tri_width] a dense weight (matrix learning rate, AdamW); the table gets no
+   * gradient.  It starts at zero: fill it with trigram_tally (gpt_tensor name
+   * "h3").  tri_width: a multiple of 64 in bf16 mode, of 4 in fp32 mode. */
+  long long tri_rows;
+  int tri_width;          /* 64                                                   */
+  unsigned long long hash_p3;  /* 3266489917                                      */
 } gpt_config;
 
 #define GPT_MATRIX_ADAMW 0
@@ -337,6 +349,29 @@ int ngram_sparse_update_noalloc(void* table, float* row_state, long long n_rows,
                                 const int32_t* rows, const float* grad, int n, float lr, float beta,
                                 float eps, int32_t* updated_rows_out, int* n_updated_out_dev,
                                 void* stream);
+
+/* ---- frozen trigram statistics ------------------------------------------ */
+
+/* Device workspace bytes trigram_tally() needs: rows * width * 4 (counts). */
+int trigram_tally_workspace_bytes(long long rows, int width, size_t* bytes);
+
+/*
+ * Tally the trigram statistics table from token streams (decoder-rtx posts:
+ * "tri-gram stats table (tallied from dataset, frozen)"): for every position
+ * t < L - 1 of each of the S streams (device int32 [S, L], row-major), the row
+ * of (x_{t-2}, x_{t-1}, x_t) -- the key of gpt_config's trigram fields,
+ * vocab standing for tokens before the start -- counts its next token in
+ * bucket x_{t+1} mod width; then table[r, b] = count[r, b] / (row r's total)
+ * in `dtype` (GPT_DTYPE_F32 or GPT_DTYPE_BF16), rows never seen 0.  The table
+ * (device [rows, width]) is overwritten; `workspace` holds the counts
+ * (trigram_tally_workspace_bytes, 256-byte aligned).  Counts are integers, so
+ * the result does not depend on the order of the adds.  Out-of-range token
+ * ids set the standalone error word (ngram_sync_status) and are not counted.
+ * Asynchronous on `stream`.
+ */
+int trigram_tally(const int32_t* streams, int S, int L, int vocab, unsigned long long p1, unsigned long long p2,
+                  unsigned long long p3, long long rows, int width, int dtype, void* table, void* workspace,
+                  size_t ws_bytes, void* stream);
 
 /* ---- Muon (matrix-parameter optimizer) --------------------------------- */
 

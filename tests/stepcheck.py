@@ -42,14 +42,18 @@ def seed_second_moments(g, model, orc, w, batches):
         model.tensor(k, g.KIND_ADAM_V).copy_(torch.from_numpy(v0))
 
 
-def run_pair(g, w, steps, lr=1e-3, ignore_frac=0.05, seed_moments=True):
+def run_pair(g, w, steps, lr=1e-3, ignore_frac=0.05, seed_moments=True, prepare=None):
     """Run `steps` micro-batches through gpt_forward_loss + gpt_backward_step on
     the GPU and through the oracle trainer; returns (model, oracle, losses,
-    last tokens, starting parameters)."""
+    last tokens, starting parameters).  `prepare(model, params)`, if given,
+    fills further model state before the run and adds the oracle's copy of it
+    to `params` (the frozen trigram statistics)."""
     cfg = to_cfg(w)
     params = init_params(w)
     model = g.Model(cfg, seed=w["seed"])
     import_params(model, params)
+    if prepare is not None:
+        prepare(model, params)
     orc = OracleTrainer(w, params)
     batches = micro_batches(w, steps, ignore_frac)
     if seed_moments:

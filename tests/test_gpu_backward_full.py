@@ -50,13 +50,13 @@ def masked_batch(w, keep, ignore_frac=0.02):
     return tok, tgt
 
 
-def oracle_two(w, params, tok, tgt, keep, rows=None):
+def oracle_two(w, params, tok, tgt, keep, rows=None, rows3=None):
     """Oracle loss and gradients of the loss over the sequences `keep` alone."""
     wk = dict(w, micro_batch=len(keep))
     rx = rv = None
     if rows is not None:
         rx, rv = rows
-    loss, _, cache = omodel.forward(wk, params, tok[list(keep)], tgt[list(keep)], rx, rv)
+    loss, _, cache = omodel.forward(wk, params, tok[list(keep)], tgt[list(keep)], rx, rv, rows3)
     G, gx0, gv = omodel.backward(wk, params, cache, scale=1.0)
     return loss, G, gx0, gv
 
@@ -168,3 +168,51 @@ def test_long_context_widths_full_step(g):
     w = workload("long2048_bf16", n_layer=1, micro_batch=1)
     model, orc, losses, _, params = run_pair(g, w, steps=1)
     check(g, w, model, orc, losses, params, 1e-2, 2e-2)
+
+
+def test_trigram_table_full_launch_backward(g):
+    """The frozen trigram statistics at full size (2,097,152 rows x 64, tallied
+    on the GPU from 64 x 2049 tokens) with both bigram tables, 16 x 2048
+    tokens, two layers: every dense gradient, the projection's included,
+    over the two kept sequences.  The oracle tallies the same streams and
+    keeps only the rows the kept sequences touch."""
+    import torch
+    from oracle import trigram
+    from synthetic import zipf_stream
+    w = workload("gpt2s_tables_bf16", n_layer=2, grad_accum=1, tri_rows=2097152, tri_width=64)
+    keep = (2, 13)
+    params = init_params(w, skip_tables=True)
+    tok, tgt = masked_batch(w, keep)
+    kt = tok[list(keep)]
+    gm = g.Model(to_cfg(w), seed=w["seed"])
+    import_params(gm, params)
+    for name in ("hx", "hv"):
+        gm.tensor(name).zero_()
+    streams = zipf_stream(64 * 2049, w["vocab"], 777).reshape(64, 2049)
+    ws_bytes = g.trigram_tally_workspace_bytes(w["tri_rows"], 64)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    g.trigram_tally(device_ints(streams), 64, 2049, w["vocab"], w["hash_p1"], w["hash_p2"], w["hash_p3"],
+                    w["tri_rows"], 64, g.DTYPE_BF16, gm.tensor("h3"), ws, ws_bytes)
+    loss = gm.forward_loss(device_ints(tok), device_ints(tgt))
+    gm.backward(1e-3)
+    assert gm.sync_status() == g.GPT_OK, g.gpt_last_error()
+    r3 = trigram.trigram_rows(kt, w["vocab"], w["hash_p1"], w["hash_p2"], w["tri_rows"], w["hash_p3"])
+    np.testing.assert_array_equal(gm.tensor("rows_3", g.KIND_ACT).cpu().numpy()[list(keep)], r3)
+    uniq, stats = trigram.tally_stats(streams, w["vocab"], w["hash_p1"], w["hash_p2"], w["tri_rows"], 64,
+                                      w["hash_p3"])
+    u3 = np.unique(r3)
+    s3 = np.zeros((len(u3), 64))
+    hit = np.isin(u3, uniq)
+    s3[hit] = stats[np.searchsorted(uniq, u3[hit])]
+    assert hit.sum() > 0
+    pc = dict(params)
+    pc["h3"] = s3
+    # the tables are zero here, so the oracle carries them as zero rows
+    rx = hashing.bigram_rows(kt, w["vocab"], w["hash_p1"], w["hash_p2"], w["x0_rows"])
+    rv = hashing.bigram_rows(kt, w["vocab"], w["hash_p1"], w["hash_p2"], w["v_rows"])
+    pc["hx"] = np.zeros((1, w["d_model"]))
+    pc["hv"] = np.zeros((1, w["d_model"]))
+    wc = dict(w, x0_rows=1, v_rows=1, tri_rows=len(u3))
+    lo, G, _, _ = oracle_two(wc, pc, tok, tgt, keep, rows=(0 * rx, 0 * rv), rows3=np.searchsorted(u3, r3))
+    assert abs(float(loss.item()) - lo) / lo < 1e-2
+    compare_dense(g, gm, G)
