@@ -377,11 +377,20 @@ def run_ours(args, w, rank, world, dist):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+    if world == 1 and not args.no_tables:
+        # the standalone table calls on the full-size x0 table (2,097,152 x 768 bf16) of the
+        # tables workload, one micro-batch (N = 32768) and one accumulated step (N = 196608);
+        # run after the timed region, on a fresh table
+        tb = table_bandwidth(workload("gpt2s_tables_bf16"), 5, 3, tables=("x0",))
+        line["tables"] = {"results": [{k: r[k] for k in ("call", "table", "n", "u_over_n", "us", "gbs",
+                                                         "frac_of_measured_hbm", "frac_of_8tbs")}
+                                      for r in tb["results"]],
+                          "peak_source": tb["peak_source"], "l2": tb["l2"], "target": "0.70 of 8 TB/s"}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ table kernels
-def run_tables(args, w):
+def table_bandwidth(w, steps, warmup, tables=("x0", "v")):
     """Achieved HBM bandwidth of the standalone bigram-table calls on the
     full-size tables (2,097,152 x d and 1,048,576 x d bf16), rows hashed from
     the workload's token stream; one micro-batch (N = B*T) and a whole
@@ -392,7 +401,7 @@ def run_tables(args, w):
     ids + 4*N*4 sorting, U = distinct rows."""
     import torch
     import gpt_pretraining_step_decoder_b200 as g
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
     st = torch.cuda.current_stream()
     d = w["d_model"]
     B, T, A, V = w["micro_batch"], w["seq_len"], w["grad_accum"], w["vocab"]
@@ -403,7 +412,7 @@ def run_tables(args, w):
     results = []
     with ClockSampler(0) as clk:
         for name, R in (("x0", w["x0_rows"]), ("v", w["v_rows"])):
-            if not R:
+            if not R or name not in tables:
                 continue
             table = (torch.randn((R, d), device=dev) * 0.02).to(torch.bfloat16)
             state = torch.zeros(R, dtype=torch.float32, device=dev)
@@ -432,14 +441,14 @@ def run_tables(args, w):
                 }
                 for cname, (fn, nbytes) in calls.items():
                     times = []
-                    for it in range(args.warmup + args.steps):
+                    for it in range(warmup + steps):
                         flush.zero_()
                         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                         e0.record(st)
                         fn()
                         e1.record(st)
                         torch.cuda.synchronize()
-                        if it >= args.warmup:
+                        if it >= warmup:
                             times.append(e0.elapsed_time(e1))
                     if g.ngram_sync_status() != g.GPT_OK:
                         raise RuntimeError(f"{cname}: device error {g.gpt_last_error()}")
@@ -451,11 +460,16 @@ def run_tables(args, w):
                 del out, grad, ws, upd
             del table, state
             torch.cuda.empty_cache()
-    line = {"metric": "bigram table calls: achieved HBM bandwidth (algorithmic bytes / CUDA-event time)",
+    del flush
+    torch.cuda.empty_cache()
+    return {"metric": "bigram table calls: achieved HBM bandwidth (algorithmic bytes / CUDA-event time)",
             "unit": "GB/s", "workload": w["name"], "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy",
-            "steps": args.steps, "warmup": args.warmup, "l2": "flushed (256 MB write) before every timed call",
+            "steps": steps, "warmup": warmup, "l2": "flushed (256 MB write) before every timed call",
             "results": results, "clocks": clk.summary()}
-    print(json.dumps(line), flush=True)
+
+
+def run_tables(args, w):
+    print(json.dumps(table_bandwidth(w, args.steps, args.warmup)), flush=True)
 
 
 def run_muon(args, w):
@@ -545,6 +559,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--lr", type=float, default=1e-4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tables", action="store_true",
+                    help="leave out the table-call bandwidth record of the default line")
     ap.add_argument("--measure", default="step", choices=["step", "tables", "muon"],
                     help="step: the training step (default); tables: bandwidth of the bigram-table calls; "
                          "muon: one Muon step over the workload's matrix parameters")

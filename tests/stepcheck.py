@@ -32,7 +32,7 @@ def seed_second_moments(g, model, orc, w, batches):
     import torch
     tok, tgt = batches[0]
     rx, rv = orc.rows(tok)
-    _, _, cache = omodel.forward(w, orc.P, tok, tgt, rx, rv)
+    _, _, cache = omodel.forward(w, orc.P, tok, tgt, rx, rv, orc.rows3(tok))
     G, _, _ = omodel.backward(w, orc.P, cache, scale=1.0 / w["grad_accum"])
     rng = np.random.default_rng(777)
     for k in orc.dense:
