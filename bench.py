@@ -535,6 +535,61 @@ def run_muon(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8(args, w):
+    """The FP8 GEMM path against the bf16 one on the same products: the
+    up-projection (N*d -> d_ff) and the LM-head logits chunk (8192 x vocab)
+    of the workload, e4m3 operands with per-tensor scales (fp32 output) vs
+    bf16 operands, CUDA events around each call; outputs exceed L2 (no flush).
+    FP8 peak: the measured bf16 peak times the nominal fp8/bf16 ratio (2)."""
+    import torch
+    import gpt_pretraining_step_decoder_b200 as g
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream()
+    peaks, peak_src = measured_peaks()
+    N_tok, d, F, V = w["micro_batch"] * w["seq_len"], w["d_model"], w["d_ff"], w["vocab"]
+    shapes = {"up_proj": (N_tok, F, d), "lm_head_chunk": (8192, V, d)}
+    ws = torch.empty(g.fp8_quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+    out = []
+    for name, (M, N, K) in shapes.items():
+        A = torch.randn((M, K), device=dev) * 0.05
+        B = torch.randn((N, K), device=dev) * 0.02
+        qa = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        qb = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        sa = torch.empty(1, device=dev)
+        sb = torch.empty(1, device=dev)
+        g.fp8_quantize(A, g.DTYPE_F32, M * K, qa, sa, ws, ws.numel())
+        g.fp8_quantize(B, g.DTYPE_F32, N * K, qb, sb, ws, ws.numel())
+        Ab, Bb = A.to(torch.bfloat16), B.to(torch.bfloat16)
+        C = torch.empty((M, N), dtype=torch.float32, device=dev)
+        calls = {"fp8": lambda: g.gptx_gemm_fp8(M, N, K, qa, K, qb, K, sa, sb, g.DTYPE_F32, C, N),
+                 "bf16": lambda: g.gptx_gemm_bf16(M, N, K, Ab, K, 1, Bb, K, 1, C, N, 0, 1, None, 0,
+                                                  mode=g.EPI_STORE_F32)}
+        rec = {"product": name, "M": M, "N": N, "K": K}
+        for cname, fn in calls.items():
+            times = []
+            for it in range(args.warmup + args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                fn()
+                e1.record(st)
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    times.append(e0.elapsed_time(e1))
+            us = 1e3 * float(np.median(times))
+            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            peak = peaks["bf16_tflops"] * (2.0 if cname == "fp8" else 1.0)
+            rec[cname] = {"us": us, "tflops": tf, "peak_tflops": peak, "frac": tf / peak}
+        rec["speedup"] = rec["bf16"]["us"] / rec["fp8"]["us"]
+        out.append(rec)
+        del A, B, qa, qb, Ab, Bb, C
+    if g.ngram_sync_status() != g.GPT_OK:
+        raise RuntimeError(f"fp8 measurement: device error {g.gpt_last_error()}")
+    print(json.dumps({"metric": "FP8 (e4m3, per-tensor scales) vs bf16 GEMM on the step's products (CUDA events)",
+                      "unit": "TFLOP/s", "workload": w["name"], "results": out,
+                      "peak_source": f"{peak_src} bf16 burst; fp8 = 2 x bf16 (nominal ratio)",
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+
+
 def parse_override(items):
     out = {}
     for it in items:
@@ -561,7 +616,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tables", action="store_true",
                     help="leave out the table-call bandwidth record of the default line")
-    ap.add_argument("--measure", default="step", choices=["step", "tables", "muon"],
+    ap.add_argument("--measure", default="step", choices=["step", "tables", "muon", "fp8"],
                     help="step: the training step (default); tables: bandwidth of the bigram-table calls; "
                          "muon: one Muon step over the workload's matrix parameters")
     ap.add_argument("--override", nargs="*", default=[],
@@ -579,6 +634,11 @@ def main():
         import torch
         torch.cuda.set_device(0)
         run_muon(args, workload(args.workload, **parse_override(args.override)))
+        return
+    if args.measure == "fp8":
+        import torch
+        torch.cuda.set_device(0)
+        run_fp8(args, w)
         return
     if args.measure == "tables":
         import torch

@@ -82,6 +82,9 @@ _SIGS = {
     "ngram_sparse_update_noalloc": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P],
     "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
     "gptx_set_gemm_cta_pairs": [_I],
+    "fp8_quantize_workspace_bytes": [ctypes.POINTER(_SZ)],
+    "fp8_quantize": [_P, _I, _LL, _P, _P, _P, _SZ, _P],
+    "gptx_gemm_fp8": [_I, _I, _I, _P, _LL, _P, _LL, _P, _P, _I, _P, _LL, _P],
     "trigram_tally_workspace_bytes": [_LL, _I, ctypes.POINTER(_SZ)],
     "trigram_tally": [_P, _I, _I, _I, _ULL, _ULL, _ULL, _LL, _I, _I, _P, _P, _SZ, _P],
     "muon_update_workspace_bytes": [_I, _I, ctypes.POINTER(_SZ)],
@@ -302,6 +305,23 @@ def trigram_tally(streams, S, L, vocab, p1, p2, p3, rows, width, dtype, table, w
     """Fill the frozen trigram statistics table from token streams [S, L] (device int32)."""
     return _check(_lib.trigram_tally(_ptr(streams), S, L, vocab, p1, p2, p3, rows, width, dtype, _ptr(table),
                                      _ptr(workspace), ws_bytes, _stream(stream)), "trigram_tally")
+
+
+def fp8_quantize_workspace_bytes():
+    n = ctypes.c_size_t()
+    _check(_lib.fp8_quantize_workspace_bytes(ctypes.byref(n)), "fp8_quantize_workspace_bytes")
+    return n.value
+
+
+def fp8_quantize(x, dtype, n, q, scale, workspace, ws_bytes, stream=None):
+    """Per-tensor e4m3 codes of x into q (uint8) and its scale (device float)."""
+    return _check(_lib.fp8_quantize(_ptr(x), dtype, n, _ptr(q), _ptr(scale), _ptr(workspace), ws_bytes,
+                                    _stream(stream)), "fp8_quantize")
+
+
+def gptx_gemm_fp8(M, N, K, A, lda, B, ldb, scale_a, scale_b, out_dtype, C, ldc, stream=None):
+    return _check(_lib.gptx_gemm_fp8(M, N, K, _ptr(A), lda, _ptr(B), ldb, _ptr(scale_a), _ptr(scale_b), out_dtype,
+                                     _ptr(C), ldc, _stream(stream)), "gptx_gemm_fp8")
 
 
 def gptx_set_gemm_cta_pairs(on):

@@ -51,6 +51,9 @@ struct GemmEpilogue {
   const int32_t* rv;
   int T, H, qk_norm;
   float eps;
+  // FP8 path: acc is further multiplied by *scale_a * *scale_b (device scalars; null = 1)
+  const float* scale_a;
+  const float* scale_b;
 };
 
 template <typename act_t>

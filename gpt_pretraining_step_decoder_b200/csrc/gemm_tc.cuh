@@ -31,7 +31,13 @@
 // CTAs complete on the even CTA's stage barrier; its MMA commits release the
 // stage and publish the accumulator in both CTAs (tcgen05.commit multicast);
 // the odd CTA's epilogue warps release the accumulator on the even CTA's
-// barrier.  No TMA load is multicast.  K-major and MN-major operands are both read straight from their
+// barrier.  No TMA load is multicast.
+//
+// F8 = 1 takes e4m3 operands (tcgen05.mma kind::f8f6f4, K = 32 per
+// instruction): a k-block is still one 128-byte swizzle row per operand row,
+// now 128 elements, so the stage layout, the descriptors and the epilogues are
+// those of the bf16 form; the epilogue multiplies by the two operands' scales
+// (device scalars).  K-major operands only.  K-major and MN-major operands are both read straight from their
 // row-major buffers (the UMMA descriptor's major-ness bit), so forward,
 // data-gradient and weight-gradient products need no transposed copies.
 // Split-K writes fp32 partials that a second kernel sums in split order
@@ -177,6 +183,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
@@ -234,6 +249,15 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
 }
 // arrive on the barrier at this offset in both CTAs of the pair once the
 // issuing thread's earlier tcgen05 operations are complete
+__device__ __forceinline__ void tc_mma_pair_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
@@ -268,29 +292,30 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 
 // Load one operand tile (rows x BK) of the k-block `kb` into `dst`.
 // K-major: one box {BK, rows}.  MN-major: rows/64 boxes {64, BK}, each 8 KB.
-// z >= 0: product z of a batch (3-D tensor map); z < 0: a 2-D map.
+// k-block starting at element kx; z >= 0: product z of a batch (3-D tensor
+// map); z < 0: a 2-D map.
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
-                                             int kmajor, int rows, int r0, int kb, int z) {
+                                             int kmajor, int rows, int r0, int kx, int z) {
   if (kmajor) {
-    if (z >= 0) tma_load_3d(dst, map, bar, kb * BK, r0, z);
-    else tma_load_2d(dst, map, bar, kb * BK, r0);
+    if (z >= 0) tma_load_3d(dst, map, bar, kx, r0, z);
+    else tma_load_2d(dst, map, bar, kx, r0);
   } else {
     for (int j = 0; j < rows / 64; ++j) {
-      if (z >= 0) tma_load_3d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK, z);
-      else tma_load_2d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+      if (z >= 0) tma_load_3d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx, z);
+      else tma_load_2d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx);
     }
   }
 }
 // the same, counted on the pair's stage barrier at shared::cluster address `bar`
 __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map, uint32_t bar,
-                                                  int kmajor, int rows, int r0, int kb, int z) {
+                                                  int kmajor, int rows, int r0, int kx, int z) {
   if (kmajor) {
-    if (z >= 0) tma_load_3d_pair(dst, map, bar, kb * BK, r0, z);
-    else tma_load_2d_pair(dst, map, bar, kb * BK, r0);
+    if (z >= 0) tma_load_3d_pair(dst, map, bar, kx, r0, z);
+    else tma_load_2d_pair(dst, map, bar, kx, r0);
   } else {
     for (int j = 0; j < rows / 64; ++j) {
-      if (z >= 0) tma_load_3d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK, z);
-      else tma_load_2d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kb * BK);
+      if (z >= 0) tma_load_3d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx, z);
+      else tma_load_2d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx);
     }
   }
 }
@@ -380,13 +405,14 @@ __device__ __forceinline__ void tile_coords(int mn, const Params& p, int& mt, in
 // byte offset of 16-byte chunk j of row r in a 128-byte-swizzled block
 __device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
-template <int BN, int KM, typename act_t, int CG>
+template <int BN, int KM, typename act_t, int CG, int F8 = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmAux,
                    const Params p) {
   using C = Cfg<BN, KmHeavy<KM>::value, CG>;
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
+  constexpr int KE = F8 ? 128 : BK;  // operand elements per 128-byte k-block row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -467,12 +493,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // that CTA arms for the pair
             const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
             if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
-            load_operand_pair(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb, z);
-            load_operand_pair(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb, z);
+            load_operand_pair(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb * KE, z);
+            load_operand_pair(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb * KE, z);
           } else {
             mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-            load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb, z);
-            load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb, z);
+            load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb * KE, z);
+            load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb * KE, z);
           }
           issued[stage] = true;
           issued_phase[stage] = phase;
@@ -494,7 +520,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(!p.a_kmajor) << 15) |
+      // D fp32; A, B bf16 (kind::f16) or e4m3 (kind::f8f6f4: format code 0)
+      const uint32_t idesc = (1u << 4) | (F8 ? 0u : (1u << 7) | (1u << 10)) | ((uint32_t)(!p.a_kmajor) << 15) |
                              ((uint32_t)(!p.b_kmajor) << 16) | ((uint32_t)(BN >> 3) << 17) |
                              ((uint32_t)((CG * BM) >> 4) << 24);
       int stage = 0;
@@ -515,13 +542,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            if constexpr (CG == 2)
-              tc_mma_pair(d_tmem, operand_desc(a_base, p.a_kmajor, k), operand_desc(b_base, p.b_kmajor, k),
-                          idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-            else
-              tc_mma(d_tmem, operand_desc(a_base, p.a_kmajor, k), operand_desc(b_base, p.b_kmajor, k),
-                     idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction: 16 bf16 or 32 e4m3
+            const uint64_t ad = operand_desc(a_base, p.a_kmajor, k), bd = operand_desc(b_base, p.b_kmajor, k);
+            const uint32_t acc_in = (kb > kb0 || k > 0) ? 1u : 0u;
+            if constexpr (CG == 2 && F8) tc_mma_pair_f8(d_tmem, ad, bd, idesc, acc_in);
+            else if constexpr (CG == 2) tc_mma_pair(d_tmem, ad, bd, idesc, acc_in);
+            else if constexpr (F8) tc_mma_f8(d_tmem, ad, bd, idesc, acc_in);
+            else tc_mma(d_tmem, ad, bd, idesc, acc_in);
           }
           if constexpr (CG == 2) tc_commit_pair(&empty[stage]);
           else tc_commit(&empty[stage]);
@@ -545,6 +572,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t aux_phase = 0;                  // bit b: parity of the next wait on abar[b]
     uint32_t aux_pending = 0;                // bit b: a load into block b is in flight
     const GemmEpilogue& e = p.epi;
+    // acc scale: alpha times the operands' device scales (the FP8 path), if any
+    const float ealpha = e.alpha * (e.scale_a ? *e.scale_a : 1.f) * (e.scale_b ? *e.scale_b : 1.f);
     constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL;
     constexpr bool has_aux = KM == K_DRELU2;
     constexpr int CW = f32out ? 32 : 64;  // columns per 128-byte staging row
@@ -599,7 +628,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int nv = min(32, p.N - nc);
           float z[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(r[i]) * e.alpha;
+          for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(r[i]) * ealpha;
           if (e.softcap > 0.f) softcap_block<32>(z, e.softcap);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -701,10 +730,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (CW == 64) tmem_ld32_nowait(trow + c * CW + 32, r1);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r0[i]) * e.alpha;
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r0[i]) * ealpha;
           if (CW == 64) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[32 + i] = __uint_as_float(r1[i]) * e.alpha;
+            for (int i = 0; i < 32; ++i) v[32 + i] = __uint_as_float(r1[i]) * ealpha;
           }
         }
         uint8_t* stg = stg_base;

@@ -30,6 +30,7 @@
 #include "ngram.cuh"
 #include "optim.cuh"
 #include "muon.cuh"
+#include "fp8.cuh"
 
 // Run the statements with NV = d / 128 (vec4 chunks per lane of a row kernel)
 // as a compile-time constant; rows that are not a multiple of 128 use MAXV.
@@ -174,12 +175,12 @@ static int resident_clusters(K* kernel, int smem, int cg) {
   return n;
 }
 
-template <int BN, int KM, int CG>
+template <int BN, int KM, int CG, int F8 = 0>
 static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tcm,
                             const CUtensorMap& taux, const tc::Params& p, cudaStream_t st) {
   using C = tc::Cfg<BN, tc::KmHeavy<KM>::value, CG>;
   static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
-  auto kernel = tc::gemm_tc_kernel<BN, KM, bf16, CG>;
+  auto kernel = tc::gemm_tc_kernel<BN, KM, bf16, CG, F8>;
   static int units = 0;
   if (!units) {
     CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
@@ -322,6 +323,40 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   return GPT_OK;
 }
 
+// FP8 product: C = (*sa * *sb) * A_q B_q^T with e4m3 operands A_q [M, K] and
+// B_q [N, K] (K-major, row pitches lda / ldb bytes), 256-column tiles, fp32 or
+// bf16 output; CTA pairs when enabled.
+template <int CG>
+static int gemm_f8_launch(int M, int N, int K, const uint8_t* A, long long lda, const uint8_t* B, long long ldb,
+                          GemmEpilogue e, unsigned* err, cudaStream_t st) {
+  CUtensorMap ta, tb, tcm;
+  {
+    const uint64_t da[2] = {(uint64_t)K, (uint64_t)M}, sa[1] = {(uint64_t)lda};
+    const uint32_t ba[2] = {128, tc::BM};
+    TRY(make_tmap_gen(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, A, da, sa, ba));
+    const uint64_t db[2] = {(uint64_t)K, (uint64_t)N}, sb[1] = {(uint64_t)ldb};
+    const uint32_t bb[2] = {128, (uint32_t)(256 / CG)};
+    TRY(make_tmap_gen(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, B, db, sb, bb));
+  }
+  tc::Params p;
+  p.M = M; p.N = N; p.K = K; p.batch = 1;
+  p.a_kmajor = 1; p.b_kmajor = 1;
+  p.m_tiles = cdiv(M, CG * tc::BM);
+  p.n_tiles = cdiv(N, 256);
+  p.group_m = 1;
+  p.kb_total = cdiv(K, 128);
+  p.splits = 1; p.kb_per_split = p.kb_total;
+  p.epi = e; p.partial = nullptr; p.err = err;
+  if (e.mode == EPI_STORE_F32) {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M}, str[1] = {(uint64_t)e.ldc * 4};
+    const uint32_t box[2] = {32, 32};
+    TRY(make_tmap_gen(&tcm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, e.C, dims, str, box));
+    return gemm_tc_launch_k<256, tc::K_STORE_F32, CG, 1>(ta, tb, tcm, tcm, p, st);
+  }
+  TRY(make_tmap(&tcm, e.C, N, M, e.ldc, 64, 32));
+  return gemm_tc_launch_k<256, tc::K_STORE, CG, 1>(ta, tb, tcm, tcm, p, st);
+}
+
 // Choose split-K so a small-output, long-K product still fills the GPU.
 // Share of the SMs' tile slots doing useful columns: tiles over whole waves,
 // times the used fraction of the last column tile.  A tile of a CTA pair
@@ -450,6 +485,7 @@ static GemmEpilogue epi(int mode, void* C, long long ldc, int beta = 0, void* C2
   e.mode = mode; e.C = C; e.ldc = ldc; e.C2 = C2; e.aux = aux; e.alpha = alpha; e.beta = beta;
   e.softcap = 0.f; e.stats = nullptr; e.targets = nullptr; e.ztgt = nullptr;
   e.rope = nullptr; e.rstd_q = e.rstd_k = nullptr; e.hv = nullptr; e.rv = nullptr;
+  e.scale_a = e.scale_b = nullptr;
   e.T = e.H = e.qk_norm = 0; e.eps = 0.f;
   return e;
 }
@@ -1789,6 +1825,49 @@ extern "C" int trigram_tally(const int32_t* streams, int S, int L, int vocab, un
   }
   LAUNCH_CHECK();
   return GPT_OK;
+}
+
+// ======================================================================== FP8 (e4m3) GEMM path
+extern "C" int fp8_quantize_workspace_bytes(size_t* bytes) {
+  if (!bytes) return fail(GPT_ERR_ARG, "fp8_quantize_workspace_bytes: null pointer");
+  *bytes = FP8_AMAX_BLOCKS * 4;
+  return GPT_OK;
+}
+
+extern "C" int fp8_quantize(const void* x, int dtype, long long n, uint8_t* q, float* scale, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  if (!x || !q || !scale || n < 0 || (n & 1)) return fail(GPT_ERR_ARG, "fp8_quantize: bad argument (n even)");
+  if (dtype != GPT_DTYPE_F32 && dtype != GPT_DTYPE_BF16) return fail(GPT_ERR_ARG, "fp8_quantize: bad dtype");
+  if (!workspace || ws_bytes < (size_t)FP8_AMAX_BLOCKS * 4)
+    return fail(GPT_ERR_WORKSPACE, "fp8_quantize: needs %d bytes of workspace", FP8_AMAX_BLOCKS * 4);
+  cudaStream_t st = (cudaStream_t)stream;
+  float* part = static_cast<float*>(workspace);
+  const unsigned qgrid = (unsigned)std::max<long long>(1, std::min<long long>((n / 2 + 255) / 256, 8LL * device_sms()));
+  if (dtype == GPT_DTYPE_BF16) {
+    ++g_launches; fp8_amax_kernel<bf16><<<FP8_AMAX_BLOCKS, 256, 0, st>>>((const bf16*)x, n, part);
+    ++g_launches; fp8_quantize_kernel<bf16><<<qgrid, 256, 0, st>>>((const bf16*)x, n, part, q, scale);
+  } else {
+    ++g_launches; fp8_amax_kernel<float><<<FP8_AMAX_BLOCKS, 256, 0, st>>>((const float*)x, n, part);
+    ++g_launches; fp8_quantize_kernel<float><<<qgrid, 256, 0, st>>>((const float*)x, n, part, q, scale);
+  }
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+extern "C" int gptx_gemm_fp8(int M, int N, int K, const uint8_t* A, long long lda, const uint8_t* B, long long ldb,
+                             const float* scale_a, const float* scale_b, int out_dtype, void* C, long long ldc,
+                             void* stream) {
+  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || !scale_a || !scale_b || ldc < N || lda < K || ldb < K)
+    return fail(GPT_ERR_ARG, "gptx_gemm_fp8: bad argument");
+  if ((lda | ldb) & 15) return fail(GPT_ERR_ARG, "gptx_gemm_fp8: row pitches must be multiples of 16 bytes");
+  if (out_dtype != GPT_DTYPE_F32 && out_dtype != GPT_DTYPE_BF16) return fail(GPT_ERR_ARG, "gptx_gemm_fp8: bad out_dtype");
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
+  GemmEpilogue e = epi(out_dtype == GPT_DTYPE_F32 ? EPI_STORE_F32 : EPI_STORE, C, ldc);
+  e.scale_a = scale_a;
+  e.scale_b = scale_b;
+  if (gemm_pairs_enabled()) return gemm_f8_launch<2>(M, N, K, A, lda, B, ldb, e, err, (cudaStream_t)stream);
+  return gemm_f8_launch<1>(M, N, K, A, lda, B, ldb, e, err, (cudaStream_t)stream);
 }
 
 // ======================================================================== Muon

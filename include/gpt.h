@@ -373,6 +373,34 @@ int trigram_tally(const int32_t* streams, int S, int L, int vocab, unsigned long
                   unsigned long long p3, long long rows, int width, int dtype, void* table, void* workspace,
                   size_t ws_bytes, void* stream);
 
+/* ---- FP8 (e4m3) GEMM path ----------------------------------------------- */
+
+/* Device workspace bytes fp8_quantize() needs (a fixed count of partial maxima). */
+int fp8_quantize_workspace_bytes(size_t* bytes);
+
+/*
+ * Per-tensor e4m3 quantization (Karpathy's llm.c post: FP8 training
+ * "imminent"; the pages give no recipe, this is the plainest per-tensor one):
+ * amax = max |x|, inv = 448 / amax, q[i] = e4m3(x[i] * inv) rounded to nearest
+ * even, saturated to +-448 (1 sign, 4 exponent bits, bias 7, 3 mantissa bits);
+ * *scale = amax / 448 (1 when amax is 0), the factor the product applies.
+ * x: device [n] of `dtype` (GPT_DTYPE_F32 or GPT_DTYPE_BF16), n even; q:
+ * device uint8 [n]; scale: device float.  Asynchronous on `stream`.
+ */
+int fp8_quantize(const void* x, int dtype, long long n, uint8_t* q, float* scale, void* workspace,
+                 size_t ws_bytes, void* stream);
+
+/*
+ * C[m, n] = (*scale_a) (*scale_b) sum_k A[m, k] B[n, k] with e4m3 codes A
+ * [M, K] and B [N, K] (device, row-major, row pitches lda / ldb bytes,
+ * multiples of 16) on the tcgen05 tensor cores (kind::f8f6f4, fp32
+ * accumulation; SM pairs when gptx_set_gemm_cta_pairs is on).  out_dtype:
+ * GPT_DTYPE_F32 or GPT_DTYPE_BF16 for C (device, row pitch ldc elements, 16-byte
+ * aligned).  Asynchronous on `stream`.
+ */
+int gptx_gemm_fp8(int M, int N, int K, const uint8_t* A, long long lda, const uint8_t* B, long long ldb,
+                  const float* scale_a, const float* scale_b, int out_dtype, void* C, long long ldc, void* stream);
+
 /* ---- Muon (matrix-parameter optimizer) --------------------------------- */
 
 /* Device workspace bytes muon_update() needs for a rows x cols matrix
