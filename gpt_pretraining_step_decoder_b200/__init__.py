@@ -66,6 +66,8 @@ _SIGS = {
     "gpt_backward": [_P, _F],
     "gpt_optimizer_step": [_P, _F],
     "gpt_set_table_exchange": [_P, _I],
+    "gpt_grad_sumsq": [_P, _LL, _LL, _P],
+    "gpt_optimizer_step_range": [_P, _F, _LL, _LL, _P],
     "gpt_launch_count": [ctypes.POINTER(_LL)],
     "gpt_profile_enable": [_P, _I],
     "gpt_profile_read": [_P, ctypes.POINTER(GptProfEntry), _I, ctypes.POINTER(_I)],
@@ -377,6 +379,23 @@ class Model:
         them inside backward (data-parallel replicas: see dp.exchange_tables)."""
         _check(_lib.gpt_set_table_exchange(self.h, int(on)), "gpt_set_table_exchange")
         self.table_exchange = bool(on)
+
+    def grad_sumsq(self, lo, hi, out):
+        """Sum of squares of the flat gradient over [lo, hi) into `out` (device float64 [1])."""
+        _check(_lib.gpt_grad_sumsq(self.h, lo, hi, _ptr(out)), "gpt_grad_sumsq")
+
+    def optimizer_step_range(self, lr, lo, hi, grad_sumsq=None):
+        """AdamW on the flat elements [lo, hi) only (a sharded optimizer step)."""
+        _check(_lib.gpt_optimizer_step_range(self.h, lr, lo, hi, _ptr(grad_sumsq)), "gpt_optimizer_step_range")
+
+    def flat_param(self):
+        """The whole fp32 dense master buffer as one flat torch view (no copy)."""
+        p, _, shape = gpt_tensor(self.h, "*", KIND_PARAM)
+        off = p - self.arena.data_ptr()
+        return self.arena[off:off + shape[0] * 4].view(self.torch.float32)
+
+    def params_changed(self):
+        gpt_params_changed(self.h)
 
     def flat_grad(self):
         """The whole fp32 dense gradient as one flat torch view (no copy)."""

@@ -1598,6 +1598,57 @@ extern "C" int gpt_optimizer_step(gpt_model* m, float lr) {
   return optimizer_step_impl(m, lr);
 }
 
+// ---- sharded optimizer step (data parallelism with a reduce-scattered gradient)
+extern "C" int gpt_grad_sumsq(gpt_model* m, long long lo, long long hi, double* out_dev) {
+  if (!m || !out_dev || lo < 0 || hi < lo || hi > m->plan.dense_n)
+    return fail(GPT_ERR_ARG, "gpt_grad_sumsq: bad range");
+  const Plan& p = m->plan;
+  ++g_launches; sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, m->st>>>(m->at<float>(p.G) + lo, hi - lo,
+                                                                      m->at<double>(p.norm_part));
+  ++g_launches; sum_partials_kernel<<<1, 256, 0, m->st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, out_dev);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
+extern "C" int gpt_optimizer_step_range(gpt_model* m, float lr, long long lo, long long hi,
+                                        const double* grad_sumsq_dev) {
+  if (!m) return fail(GPT_ERR_ARG, "null model");
+  const gpt_config& c = m->cfg;
+  const Plan& p = m->plan;
+  if (m->micro == 0) return fail(GPT_ERR_STATE, "gpt_optimizer_step_range needs at least one gpt_backward");
+  if (!std::isfinite(lr)) return fail(GPT_ERR_ARG, "learning rate not finite");
+  if (lo < 0 || hi < lo || hi > p.dense_n || (lo & 3) || (hi & 3))
+    return fail(GPT_ERR_ARG, "gpt_optimizer_step_range: range must lie in the flat buffer, ends multiples of 4");
+  if (c.matrix_optimizer == GPT_MATRIX_MUON)
+    return fail(GPT_ERR_CONFIG, "a sharded optimizer step needs whole matrices for Muon: use gpt_optimizer_step");
+  if (c.grad_clip > 0.f && !grad_sumsq_dev)
+    return fail(GPT_ERR_ARG, "grad_clip > 0 needs the global gradient sum of squares");
+  const bool b16 = cfg_bf16(c);
+  cudaStream_t st = m->st;
+  ProfScope ps(&m->prof, st, "adamw", 0.0, (double)(hi - lo) * (b16 ? 30 : 28));
+  m->micro = 0;
+  m->step_t += 1;
+  float* coef = nullptr;
+  if (c.grad_clip > 0.f) {
+    ++g_launches; clip_coef_kernel<<<1, 256, 0, st>>>(grad_sumsq_dev, 1, c.grad_clip, m->at<float>(p.clip_coef),
+                                                       m->at<float>(p.grad_norm), m->err());
+    coef = m->at<float>(p.clip_coef);
+  }
+  AdamArgs aa;
+  aa.p = m->at<float>(p.P) + lo; aa.g = m->at<float>(p.G) + lo; aa.m = m->at<float>(p.M) + lo;
+  aa.v = m->at<float>(p.V) + lo;
+  aa.p_lp = b16 ? m->at<bf16>(p.Plp) + lo : nullptr;
+  aa.n = hi - lo; aa.e_end = std::max(0LL, p.e_end - lo); aa.h_end = std::max(0LL, p.h_end - lo);
+  aa.lr_e = lr * c.lr_mult_embed; aa.lr_h = lr * c.lr_mult_head; aa.lr_m = lr * c.lr_mult_matrix;
+  aa.b1 = c.adam_b1; aa.b2 = c.adam_b2; aa.eps = c.adam_eps; aa.wd = c.weight_decay;
+  aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
+  aa.bc2 = (float)(1.0 - pow((double)c.adam_b2, (double)m->step_t));
+  aa.clip = coef;
+  ++g_launches; adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
 extern "C" int gpt_launch_count(long long* n) {
   if (!n) return fail(GPT_ERR_ARG, "null pointer");
   *n = g_launches.load();

@@ -77,6 +77,22 @@ __global__ void clip_coef_kernel(const double* __restrict__ part, int nparts, fl
   }
 }
 
+// *out = sum of the partials in order (one block)
+__global__ void sum_partials_kernel(const double* __restrict__ part, int nparts, double* __restrict__ out) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
+  s = warp_sum_d(s);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) sh[wid] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh[w];
+    *out = t;
+  }
+}
+
 // fp32 master -> bf16 copy (round to nearest even).
 __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long long n) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;

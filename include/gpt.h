@@ -208,6 +208,26 @@ int gpt_backward(gpt_model* m, float lr);
 int gpt_set_table_exchange(gpt_model* m, int on);
 int gpt_optimizer_step(gpt_model* m, float lr);
 
+/*
+ * Data parallelism with a sharded optimizer step (the dense weights'
+ * reduce-scatter -> sharded AdamW -> all-gather form of ZeRO-style sharding;
+ * the caller runs the collectives, see dp.py):
+ *   gpt_grad_sumsq writes sum_{i in [lo, hi)} G[i]^2 (the accumulated dense
+ *     gradient of the flat buffer, gpt_tensor "*" GRAD) to *out_dev (device
+ *     double), summed in a fixed order;
+ *   gpt_optimizer_step_range runs the AdamW step of gpt_optimizer_step on the
+ *     elements [lo, hi) of the flat buffers only (the group learning rates
+ *     by position as usual; the bf16 copy of the range refreshed), after the
+ *     caller has put the rank-averaged gradient of that range into G; with
+ *     grad_clip > 0 the clip coefficient comes from *grad_sumsq_dev, the
+ *     global sum of squares (all ranks' gpt_grad_sumsq over their ranges,
+ *     all-reduced).  lo, hi: multiples of 4 within [0, flat size].  Advances
+ *     the step counter like gpt_optimizer_step.  Not with Muon (it needs
+ *     whole matrices).  Both asynchronous on the model's stream.
+ */
+int gpt_grad_sumsq(gpt_model* m, long long lo, long long hi, double* out_dev);
+int gpt_optimizer_step_range(gpt_model* m, float lr, long long lo, long long hi, const double* grad_sumsq_dev);
+
 /* Dense (matmul + embedding) and table parameter counts.  Host only. */
 int gpt_num_params(const gpt_model* m, long long* dense, long long* table);
 

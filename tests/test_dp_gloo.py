@@ -256,9 +256,13 @@ def _oracle_sparse_update(W, state, n_rows, d, dtype, rows, grad, n, lr, beta, e
     """Stands in for the CUDA ngram_sparse_update inside the CPU ranks."""
     from oracle import optim
     assert rows.numel() == n and tuple(grad.shape) == (n, d) and W.shape == (n_rows, d) and dtype == 0
-    newW, newS, _ = optim.table_update(W.numpy(), state.numpy(), rows.numpy(), grad.numpy(), lr, beta, eps)
+    newW, newS, uniq = optim.table_update(W.numpy(), state.numpy(), rows.numpy(), grad.numpy(), lr, beta, eps)
     W.copy_(W.new_tensor(newW))
     state.copy_(state.new_tensor(newS))
+    if upd is not None:
+        upd[:len(uniq)] = upd.new_tensor(uniq)
+    if nupd is not None:
+        nupd[0] = len(uniq)
 
 
 def _train_rank_main(rank, world, port, out_dir):
@@ -428,7 +432,183 @@ def test_train_step_restores_exchange_mode_when_a_call_fails():
     assert not m.table_exchange
 
 
-def test_train_step_rejects_unknown_table_mode():
+def test_train_step_rejects_unknown_modes():
     from gpt_pretraining_step_decoder_b200 import dp
     with pytest.raises(ValueError):
-        dp.train_step(None, [], 1e-3, tables="sharded")
+        dp.train_step(None, [], 1e-3, tables="striped")
+    with pytest.raises(ValueError):
+        dp.train_step(None, [], 1e-3, dense="zero3")
+
+
+# --------------------------------------------------------------------------- row-sharded table exchange
+def _sharded_rank_main(rank, world, port, out_dir):
+    import torch
+    import torch.distributed as dist
+    import gpt_pretraining_step_decoder_b200 as g
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+
+    g.ngram_sparse_update = _oracle_sparse_update
+    g.ngram_sparse_update_workspace_bytes = lambda n, d: 1
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cfg = dict(_table_cfg(), lr_mult_table=0.5)
+        m = _OracleModel(cfg, init_params(cfg, seed=3))
+        batches = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], rank) + 7 * s) for s in range(2)]
+        dp.train_step(m, batches, 2e-2, tables="sharded")
+        flat = torch.from_numpy(np.concatenate([m.P[t].reshape(-1) for t in ("hv", "hx")] +
+                                               [m.S[t] for t in ("hv", "hx")]))
+        reps = [torch.empty_like(flat) for _ in range(world)]
+        dist.all_gather(reps, flat)
+        if rank == 0:
+            np.save(os.path.join(out_dir, "tables.npy"), torch.stack(reps).numpy())
+            np.save(os.path.join(out_dir, "calls.npy"), np.array(m.calls))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_row_sharded_table_exchange_equals_joint_batch_update(tmp_path, world):
+    """tables="sharded": every row's gradient goes to its owner (row mod
+    world), the owner updates its rows over the pairs in rank order, the
+    updated rows are gathered back: replicas bit-identical and equal, bit
+    for bit, to one process updating per micro-batch over the joint batch."""
+    import torch.multiprocessing as mp
+    from gpt_pretraining_step_decoder_b200 import dp
+    from oracle import optim
+    from synthetic import init_params
+
+    mp.spawn(_sharded_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    reps = np.load(tmp_path / "tables.npy")
+    for r in range(1, world):
+        np.testing.assert_array_equal(reps[0], reps[r])
+    cfg = dict(_table_cfg(), lr_mult_table=0.5)
+    P = {k: np.array(v, dtype=np.float64) for k, v in init_params(cfg, seed=3).items()}
+    S = {t: np.zeros(P[t].shape[0]) for t in ("hx", "hv")}
+    joint = dict(cfg, micro_batch=cfg["micro_batch"] * world)
+    for s in range(2):
+        parts = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], r) + 7 * s) for r in range(world)]
+        rx, gx0, rv, gv = _table_grads(joint, P, np.concatenate([p[0] for p in parts]),
+                                       np.concatenate([p[1] for p in parts]))
+        for t, rows, g in (("hv", rv, gv), ("hx", rx, gx0)):
+            P[t], S[t], _ = optim.table_update(P[t], S[t], rows, g, 2e-2 * 0.5, cfg["table_beta"],
+                                               cfg["table_eps"])
+    ref = np.concatenate([P[t].reshape(-1) for t in ("hv", "hx")] + [S[t] for t in ("hv", "hx")])
+    np.testing.assert_allclose(reps[0], ref, rtol=1e-12, atol=1e-15)
+
+
+# --------------------------------------------------------------------------- sharded dense optimizer step
+class _FlatOracleModel:
+    """The slice of `Model` the dense paths of dp.train_step use, over flat
+    fp64 buffers with the oracle's forward/backward and AdamW (group learning
+    rates by position: embedding, then head, then matrices)."""
+
+    def __init__(self, cfg, params):
+        import types
+        import torch
+        from synthetic import param_shapes
+        self.torch, self.w, self.stream = torch, cfg, None
+        self.cfg = types.SimpleNamespace(x0_rows=0, v_rows=0)
+        self.table_exchange = False
+        self.names = [k for k in param_shapes(cfg) if k not in ("hx", "hv")]
+        self.shapes = {k: np.asarray(params[k]).shape for k in self.names}
+        sizes = [int(np.prod(self.shapes[k])) for k in self.names]
+        self.offs = np.concatenate([[0], np.cumsum(sizes)])
+        self.P = torch.from_numpy(np.concatenate([np.asarray(params[k], np.float64).reshape(-1) for k in self.names]))
+        self.G, self.M, self.V = (torch.zeros_like(self.P) for _ in range(3))
+        self.e_end = int(self.offs[1])
+        self.h_end = int(self.offs[2]) if "lm_head" in self.names else self.e_end
+        self.t = 0
+
+    def _dict(self):
+        return {k: self.P[self.offs[i]:self.offs[i + 1]].numpy().reshape(self.shapes[k])
+                for i, k in enumerate(self.names)}
+
+    def forward_loss(self, tok, tgt):
+        from oracle import model
+        self.cache = model.forward(self.w, self._dict(), tok, tgt)[2]
+
+    def backward(self, lr):
+        from oracle import model
+        G, _, _ = model.backward(self.w, self._dict(), self.cache)
+        self.G += self.torch.from_numpy(np.concatenate([G[k].reshape(-1) for k in self.names]))
+
+    def flat_grad(self):
+        return self.G
+
+    def flat_param(self):
+        return self.P
+
+    def params_changed(self):
+        pass
+
+    def grad_sumsq(self, lo, hi, out):
+        out[0] = float((self.G[lo:hi] ** 2).sum())
+
+    def _adamw(self, lr, lo, hi, coef):
+        from oracle import optim
+        w = self.w
+        bounds = sorted({lo, hi, min(max(self.e_end, lo), hi), min(max(self.h_end, lo), hi)})
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            mult = w["lr_mult_embed"] if a < self.e_end else (w["lr_mult_head"] if a < self.h_end
+                                                               else w["lr_mult_matrix"])
+            p, m, v = optim.adamw(self.P[a:b].numpy(), self.G[a:b].numpy() * coef, self.M[a:b].numpy(),
+                                  self.V[a:b].numpy(), self.t, lr * mult, w["adam_b1"], w["adam_b2"],
+                                  w["adam_eps"], w["weight_decay"])
+            self.P[a:b], self.M[a:b], self.V[a:b] = (self.torch.from_numpy(np.asarray(z)) for z in (p, m, v))
+
+    def optimizer_step(self, lr):
+        from oracle import optim
+        self.t += 1
+        self._adamw(lr, 0, self.P.numel(), optim.clip_coef([self.G.numpy()], self.w["grad_clip"]))
+        self.G.zero_()
+
+    def optimizer_step_range(self, lr, lo, hi, sumsq):
+        self.t += 1
+        coef = 1.0
+        if self.w["grad_clip"] > 0:
+            coef = min(1.0, self.w["grad_clip"] / (float(np.sqrt(float(sumsq[0]))) + 1e-6))
+        self._adamw(lr, lo, hi, coef)
+        self.G.zero_()
+
+
+def _dense_cfg():
+    from synthetic import workload
+    return workload("tiny_fp32", x0_rows=0, n_layer=1, seq_len=16, micro_batch=2, vocab=96, tie_embeddings=0,
+                    grad_clip=0.05, lr_mult_head=0.5, lr_mult_embed=2.0)
+
+
+def _dense_rank_main(rank, world, port, out_dir, dense):
+    import torch
+    import torch.distributed as dist
+    from gpt_pretraining_step_decoder_b200 import dp
+    from synthetic import init_params
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cfg = _dense_cfg()
+        m = _FlatOracleModel(cfg, init_params(cfg, seed=5))
+        for step in range(2):
+            batches = [_batch(cfg, dp.rank_stream_seed(cfg["seed"], rank) + 11 * step + s) for s in range(2)]
+            dp.train_step(m, batches, 1e-2, dense=dense)
+        reps = [torch.empty_like(m.P) for _ in range(world)]
+        dist.all_gather(reps, m.P)
+        if rank == 0:
+            np.save(os.path.join(out_dir, f"params_{dense}.npy"), torch.stack(reps).numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_dense_step_equals_replicated_step(tmp_path, world):
+    """dense="sharded" (reduce-scatter, AdamW on each rank's slice with the
+    all-reduced clip norm, all-gather) gives the replicated all-reduce +
+    AdamW result on every rank: two optimizer steps with clipping active and
+    three learning-rate groups, a slice boundary inside a tensor."""
+    import torch.multiprocessing as mp
+    for dense in ("replicated", "sharded"):
+        mp.spawn(_dense_rank_main, args=(world, _free_port(), str(tmp_path), dense), nprocs=world, join=True)
+    rep = np.load(tmp_path / "params_replicated.npy")
+    sh = np.load(tmp_path / "params_sharded.npy")
+    for r in range(world):
+        np.testing.assert_array_equal(sh[r], sh[0])
+    np.testing.assert_allclose(sh[0], rep[0], rtol=1e-10, atol=1e-13)
