@@ -530,7 +530,7 @@ struct Plan {
   // same-shape groups and one scratch sized for the largest group
   MuonGroup muon_groups[3];
   int n_muon_groups = 0;
-  size_t mu_x, mu_xn, mu_abf, mu_bm, mu_a, mu_aa, mu_p, mu_part;
+  size_t mu_x, mu_xn, mu_abf, mu_bm, mu_aa, mu_p, mu_part;
   int chunk;
   size_t total;
 };
@@ -704,8 +704,8 @@ static void make_plan(const gpt_config& c, Plan& p) {
     }
     p.mu_x = cv.take(xn * 2); p.mu_xn = cv.take(xn * 2);
     p.mu_abf = cv.take(rr * 2); p.mu_bm = cv.take(rr * 2);
-    p.mu_a = cv.take(rr * 4); p.mu_aa = cv.take(rr * 4);
-    p.mu_p = cv.take(xn * 4);
+    p.mu_aa = cv.take(rr * 2);   // A A (bf16)
+    p.mu_p = cv.take(xn * 2);    // B X (bf16)
     p.mu_part = cv.take(nm * MUON_BATCH_BLOCKS * 4);
   }
   p.total = cv.take(0) + 256;
@@ -1438,7 +1438,10 @@ static int gemm_batched(const GemmCtx& g, const GemmBatch& bt, int M, int N, int
 // momentum (on the clipped gradient) with a per-matrix sum of squares, the
 // normalised bf16 iterate, muon_ns_steps Newton-Schulz steps as batched GEMMs
 // over the group (X X^T or X^T X, A A, then B X or X B), and the scaled step
-// into the fp32 master and its bf16 copy.  Same arithmetic as muon_update.
+// into the fp32 master and its bf16 copy.  Every product leaves its GEMM
+// rounded to bf16, as in the pages' bf16 iteration (A, A A, B X each a bf16
+// matmul output; B = b A + c A A and X <- a X + B X formed from bf16 values,
+// rounded once), which halves the iteration's elementwise traffic.
 static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
   const gpt_config& c = m->cfg;
   const Plan& p = m->plan;
@@ -1451,9 +1454,8 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
   bf16* xn = m->at<bf16>(p.mu_xn);
   bf16* abf = m->at<bf16>(p.mu_abf);
   bf16* bm = m->at<bf16>(p.mu_bm);
-  float* A = m->at<float>(p.mu_a);
-  float* AA = m->at<float>(p.mu_aa);
-  float* Pp = m->at<float>(p.mu_p);
+  bf16* aa16 = m->at<bf16>(p.mu_aa);  // A A
+  bf16* p16 = m->at<bf16>(p.mu_p);    // B X (X B)
   float* part = m->at<float>(p.mu_part);
   const GemmCtx g{true, m->at<float>(p.splitk), p.splitk_elems, m->err(), st, &m->prof};
   const float ca = 3.4445f, cb = -4.7750f, cc = 2.0315f;  // a x + b x^3 + c x^5
@@ -1482,32 +1484,28 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
     for (int it = 0; it < c.muon_ns_steps; ++it) {
       if (!tall)
         TRY(gemm_batched(g, GemmBatch{nmat, n, n, rr}, R, R, cols, op_k(x, cols), op_k(x, cols),
-                         epi(EPI_STORE_F32, A, R), "muon.gram"));
+                         epi(EPI_STORE, abf, R), "muon.gram"));
       else
         TRY(gemm_batched(g, GemmBatch{nmat, n, n, rr}, R, R, rows, op_mn(x, cols), op_mn(x, cols),
-                         epi(EPI_STORE_F32, A, R), "muon.gram"));
+                         epi(EPI_STORE, abf, R), "muon.gram"));
+      TRY(gemm_batched(g, GemmBatch{nmat, rr, rr, rr}, R, R, R, op_k(abf, R), op_mn(abf, R),
+                       epi(EPI_STORE, aa16, R), "muon.square"));
       {
         ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * rr * 6);
         ++g_launches;
-        muon_to_bf16_kernel<<<grid1(nmat * rr / 4), MUON_THREADS, 0, st>>>(A, nmat * rr / 4, abf);
-      }
-      TRY(gemm_batched(g, GemmBatch{nmat, rr, rr, rr}, R, R, R, op_k(abf, R), op_mn(abf, R),
-                       epi(EPI_STORE_F32, AA, R), "muon.square"));
-      {
-        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * rr * 8);
-        ++g_launches;
-        muon_combine_kernel<<<grid1(nmat * rr / 4), MUON_THREADS, 0, st>>>(abf, AA, nmat * rr / 4, cb, cc, bm);
+        muon_combine_bf16_kernel<<<grid1(nmat * rr / 4), MUON_THREADS, 0, st>>>(abf, aa16, nmat * rr / 4, cb, cc,
+                                                                                 bm);
       }
       if (!tall)
         TRY(gemm_batched(g, GemmBatch{nmat, rr, n, n}, rows, cols, R, op_k(bm, R), op_mn(x, cols),
-                         epi(EPI_STORE_F32, Pp, cols), "muon.poly"));
+                         epi(EPI_STORE, p16, cols), "muon.poly"));
       else
         TRY(gemm_batched(g, GemmBatch{nmat, n, rr, n}, rows, cols, R, op_k(x, cols), op_mn(bm, R),
-                         epi(EPI_STORE_F32, Pp, cols), "muon.poly"));
+                         epi(EPI_STORE, p16, cols), "muon.poly"));
       {
-        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 8);
+        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 6);
         ++g_launches;
-        muon_combine_kernel<<<grid1(nmat * n / 4), MUON_THREADS, 0, st>>>(x, Pp, nmat * n / 4, ca, 1.f, xn);
+        muon_combine_bf16_kernel<<<grid1(nmat * n / 4), MUON_THREADS, 0, st>>>(x, p16, nmat * n / 4, ca, 1.f, xn);
       }
       LAUNCH_CHECK();
       std::swap(x, xn);
