@@ -292,29 +292,30 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 
 // Load one operand tile (rows x BK) of the k-block `kb` into `dst`.
 // K-major: one box {BK, rows}.  MN-major: rows/64 boxes {64, BK}, each 8 KB.
-// k-block starting at element kx; z >= 0: product z of a batch (3-D tensor
-// map); z < 0: a 2-D map.
+// k-block starting at element kx; B3: product z of a batch (3-D tensor map).
+template <bool B3>
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
                                              int kmajor, int rows, int r0, int kx, int z) {
   if (kmajor) {
-    if (z >= 0) tma_load_3d(dst, map, bar, kx, r0, z);
+    if constexpr (B3) tma_load_3d(dst, map, bar, kx, r0, z);
     else tma_load_2d(dst, map, bar, kx, r0);
   } else {
     for (int j = 0; j < rows / 64; ++j) {
-      if (z >= 0) tma_load_3d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx, z);
+      if constexpr (B3) tma_load_3d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx, z);
       else tma_load_2d(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx);
     }
   }
 }
 // the same, counted on the pair's stage barrier at shared::cluster address `bar`
+template <bool B3>
 __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map, uint32_t bar,
                                                   int kmajor, int rows, int r0, int kx, int z) {
   if (kmajor) {
-    if (z >= 0) tma_load_3d_pair(dst, map, bar, kx, r0, z);
+    if constexpr (B3) tma_load_3d_pair(dst, map, bar, kx, r0, z);
     else tma_load_2d_pair(dst, map, bar, kx, r0);
   } else {
     for (int j = 0; j < rows / 64; ++j) {
-      if (z >= 0) tma_load_3d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx, z);
+      if constexpr (B3) tma_load_3d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx, z);
       else tma_load_2d_pair(dst + j * 64 * BK * 2, map, bar, r0 + 64 * j, kx);
     }
   }
@@ -405,7 +406,7 @@ __device__ __forceinline__ void tile_coords(int mn, const Params& p, int& mt, in
 // byte offset of 16-byte chunk j of row r in a 128-byte-swizzled block
 __device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
-template <int BN, int KM, typename act_t, int CG, int F8 = 0>
+template <int BN, int KM, typename act_t, int CG, int F8 = 0, bool B3 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmAux,
@@ -430,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_product = p.m_tiles * p.n_tiles * p.splits;
-  const int tiles = per_product * p.batch;
+  const int tiles = B3 ? per_product * p.batch : per_product;
   // CTA pair: rank 0 issues the MMAs; tile t goes to pair blockIdx.x / CG
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
   const int unit = blockIdx.x / CG, n_units = gridDim.x / CG;
@@ -467,8 +468,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
+    if (lane < 2) {
+      // ------------------------------------------------------------ producers
+      // lane 0 issues the A tiles (and arms the stage barrier for the whole
+      // stage), lane 1 the B tiles, so the two operands' copies are requested
+      // in parallel: a single issuing thread is on the critical path when an
+      // MN-major operand takes several boxes per k-block
+      const bool is_a = lane == 0;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_phase[C::STAGES];
@@ -476,8 +482,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int s = 0; s < C::STAGES; ++s) issued[s] = false;
       bool ok = true;
       for (int t = unit; t < tiles && ok; t += n_units) {
-        const int z = p.batch > 1 ? t / per_product : -1;
-        const int tt = t % per_product;
+        const int z = B3 ? t / per_product : 0;
+        const int tt = B3 ? t % per_product : t;
         const int split = tt % p.splits;
         const int mn = tt / p.splits;
         int mt, nt;
@@ -492,13 +498,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // both CTAs' bytes complete on the even CTA's stage barrier, which
             // that CTA arms for the pair
             const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-            if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
-            load_operand_pair(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb * KE, z);
-            load_operand_pair(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb * KE, z);
+            if (is_a) {
+              if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
+              load_operand_pair<B3>(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb * KE, z);
+            } else {
+              load_operand_pair<B3>(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb * KE, z);
+            }
           } else {
-            mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-            load_operand(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb * KE, z);
-            load_operand(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb * KE, z);
+            if (is_a) {
+              mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+              load_operand<B3>(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb * KE, z);
+            } else {
+              load_operand<B3>(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb * KE, z);
+            }
           }
           issued[stage] = true;
           issued_phase[stage] = phase;
@@ -510,7 +522,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // of its copies is consumed by an MMA before the pair finishes, and an
       // aborted pair waits out its copies before tearing down)
       for (int s = 0; s < C::STAGES; ++s) {
-        if (!issued[s] || rank != 0) continue;
+        if (!issued[s] || rank != 0 || !is_a) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&full[s], issued_phase[s])) {
           if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) { set_error(p.err, GPT_EBIT_TIMEOUT); break; }
@@ -530,7 +542,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = unit; t < tiles && ok; t += n_units) {
-        const int split = (t % per_product) % p.splits;
+        const int split = (B3 ? t % per_product : t) % p.splits;
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err)) { ok = false; break; }
@@ -573,7 +585,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t aux_pending = 0;                // bit b: a load into block b is in flight
     const GemmEpilogue& e = p.epi;
     // acc scale: alpha times the operands' device scales (the FP8 path), if any
-    const float ealpha = e.alpha * (e.scale_a ? *e.scale_a : 1.f) * (e.scale_b ? *e.scale_b : 1.f);
+    float ealpha = e.alpha;
+    if constexpr (F8) ealpha *= (e.scale_a ? *e.scale_a : 1.f) * (e.scale_b ? *e.scale_b : 1.f);
     constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL;
     constexpr bool has_aux = KM == K_DRELU2;
     constexpr int CW = f32out ? 32 : 64;  // columns per 128-byte staging row
@@ -584,8 +597,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // the accumulator-empty barrier lives in the even CTA of a pair
     const uint32_t tempty0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
     for (int t = unit; t < tiles && ok; t += n_units) {
-      const int z = p.batch > 1 ? t / per_product : -1;
-      const int tt = t % per_product;
+      const int z = B3 ? t / per_product : 0;
+      const int tt = B3 ? t % per_product : t;
       const int split = tt % p.splits;
       const int mn = tt / p.splits;
       int mt, nt;
@@ -802,7 +815,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
           if constexpr (KM == K_PARTIAL) tma_store_3d(&tmC, stg, nc, mrow0, split);
           else if constexpr (KM == K_REDUCE_F32) tma_reduce_add_2d(&tmC, stg, nc, mrow0);
-          else if (z >= 0) tma_store_3d(&tmC, stg, nc, mrow0, z);
+          else if constexpr (B3) tma_store_3d(&tmC, stg, nc, mrow0, z);
           else tma_store_2d(&tmC, stg, nc, mrow0);
           bulk_commit();
         }
@@ -833,12 +846,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // an aborted CTA (or pair) may still have copies landing: let them finish (bounded)
+  if (*abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 1000000ull) {}
+  }
   if constexpr (CG == 2) {
-    // an aborted pair may still have copies landing: let them finish (bounded)
-    if (*abort_flag) {
-      const uint64_t t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < 1000000ull) {}
-    }
     // neither CTA frees TMEM or leaves while its peer may still read its
     // shared memory, write its TMEM or arrive on its barriers
     cluster_sync_all();

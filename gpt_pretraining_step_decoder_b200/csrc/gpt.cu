@@ -175,12 +175,12 @@ static int resident_clusters(K* kernel, int smem, int cg) {
   return n;
 }
 
-template <int BN, int KM, int CG, int F8 = 0>
+template <int BN, int KM, int CG, int F8 = 0, bool B3 = false>
 static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tcm,
                             const CUtensorMap& taux, const tc::Params& p, cudaStream_t st) {
   using C = tc::Cfg<BN, tc::KmHeavy<KM>::value, CG>;
   static_assert(C::SMEM_BYTES <= 232448, "shared memory budget");
-  auto kernel = tc::gemm_tc_kernel<BN, KM, bf16, CG, F8>;
+  auto kernel = tc::gemm_tc_kernel<BN, KM, bf16, CG, F8, B3>;
   static int units = 0;
   if (!units) {
     CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
@@ -294,6 +294,12 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   else if (e.mode == EPI_QKV) km = tc::K_QKV;
   else km = tc::K_LOGITS;
   if (km == tc::K_QKV && BN != 256) return fail(GPT_ERR_ARG, "QKV epilogue needs 256-column tiles (N >= 256)");
+  if (b3) {
+    // batched products: their own kernel instances (the third tensor-map coordinate)
+    if (km == tc::K_STORE_F32) TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32, CG, 0, true>(ta, tb, tcm, taux, p, st)));
+    else TRY((gemm_tc_launch_k<BN, tc::K_STORE, CG, 0, true>(ta, tb, tcm, taux, p, st)));
+    return GPT_OK;
+  }
   if constexpr (BN == 192) {  // fp32 outputs only
     switch (km) {
       case tc::K_STORE_F32: TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32, CG>(ta, tb, tcm, taux, p, st))); break;
