@@ -468,13 +468,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    if (lane < 2) {
-      // ------------------------------------------------------------ producers
-      // lane 0 issues the A tiles (and arms the stage barrier for the whole
-      // stage), lane 1 the B tiles, so the two operands' copies are requested
-      // in parallel: a single issuing thread is on the critical path when an
-      // MN-major operand takes several boxes per k-block
-      const bool is_a = lane == 0;
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_phase[C::STAGES];
@@ -498,19 +493,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // both CTAs' bytes complete on the even CTA's stage barrier, which
             // that CTA arms for the pair
             const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-            if (is_a) {
-              if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
-              load_operand_pair<B3>(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb * KE, z);
-            } else {
-              load_operand_pair<B3>(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb * KE, z);
-            }
+            if (rank == 0) mbar_expect_tx(&full[stage], CG * C::STAGE_BYTES);
+            load_operand_pair<B3>(sA + stage * C::A_BYTES, &tmA, bar0, p.a_kmajor, BM, m0, kb * KE, z);
+            load_operand_pair<B3>(sB + stage * C::B_BYTES, &tmB, bar0, p.b_kmajor, C::B_ROWS, n0, kb * KE, z);
           } else {
-            if (is_a) {
-              mbar_expect_tx(&full[stage], C::STAGE_BYTES);
-              load_operand<B3>(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb * KE, z);
-            } else {
-              load_operand<B3>(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb * KE, z);
-            }
+            mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+            load_operand<B3>(sA + stage * C::A_BYTES, &tmA, &full[stage], p.a_kmajor, BM, m0, kb * KE, z);
+            load_operand<B3>(sB + stage * C::B_BYTES, &tmB, &full[stage], p.b_kmajor, BN, n0, kb * KE, z);
           }
           issued[stage] = true;
           issued_phase[stage] = phase;
@@ -522,7 +511,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // of its copies is consumed by an MMA before the pair finishes, and an
       // aborted pair waits out its copies before tearing down)
       for (int s = 0; s < C::STAGES; ++s) {
-        if (!issued[s] || rank != 0 || !is_a) continue;
+        if (!issued[s] || rank != 0) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&full[s], issued_phase[s])) {
           if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) { set_error(p.err, GPT_EBIT_TIMEOUT); break; }
