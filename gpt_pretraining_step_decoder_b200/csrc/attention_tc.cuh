@@ -71,6 +71,37 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+// W (8, 16 or 32) consecutive 32-bit TMEM columns of the warp's 32 lanes
+template <int W>
+__device__ __forceinline__ void tmem_ldw(uint32_t taddr, uint32_t (&r)[W]) {
+  static_assert(W == 8 || W == 16 || W == 32, "tcgen05.ld width");
+  if constexpr (W == 32) {
+    tc::tmem_ld32_nowait(taddr, r);
+  } else if constexpr (W == 16) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  } else {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  }
+}
+template <int W>
+__device__ __forceinline__ void tmem_stw(uint32_t taddr, const uint32_t (&r)[W]) {
+  static_assert(W == 8 || W == 16, "tcgen05.st width");
+  if constexpr (W == 16) {
+    tmem_st16(taddr, r);
+  } else {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+  }
+}
+
 // D (TMEM) += A (TMEM, bf16 packed two per column along K) x B (shared memory)
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -460,6 +491,8 @@ using fatc::tmem_st16;
 using fatc::tc_mma_ts;
 using fatc::pack_bf16x2_int;
 using fatc::pack_bf16x2_rn;
+using fatc::tmem_ldw;
+using fatc::tmem_stw;
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns
@@ -520,9 +553,9 @@ __device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* ds
 }
 
 // ---------------------------------------------------------------- dK, dV
-// 10 warps: 0 TMA, 1 MMA, 2..9 compute.  Compute warp w owns TMEM lane
-// quarter w % 4 (32 key rows) and half (w - 2) / 4 of the 64 query columns,
-// so two warps per scheduler share the elementwise work.
+// 2 + 4 * NCG warps: 0 TMA, 1 MMA, the rest compute.  Compute warp w owns
+// TMEM lane quarter w % 4 (32 key rows) and column group (w - 2) / 4 of the
+// 64 query columns, so NCG warps per scheduler share the elementwise work.
 // smem: K, V [128 x 128] (32 KB each); per stage Q_i, dO_i [64 x 128] (16 KB
 // each, DKDV_QS stages).  P^T and dS^T never touch shared memory: each
 // compute warp writes them as bf16 over the fp32 S^T / dP^T columns it has
@@ -532,8 +565,16 @@ __device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* ds
 // step (operand bytes through shared memory), and the S^T / dP^T buffers
 // alternate, so step i+1's S^T / dP^T products run while step i's
 // elementwise work does.  lse and D come straight from global memory.
-constexpr int THREADS_B = 320;
+// NCG warps share each 32-row TMEM lane quarter, one group of CSP = 64 / NCG
+// of a step's 64 columns each: 4 * NCG compute warps, so every scheduler has
+// NCG of them to interleave (the elementwise work has no cross-warp step).
+constexpr int NCG = 2;
+constexpr int CSP = 64 / NCG;
+constexpr int THREADS_B = 64 + 32 * 4 * NCG;
 constexpr int KV_T = 32768, QT64 = 16384;
+// TMEM column of the packed bf16 A operand for MMA k-step k (16 of the 64 step
+// columns): column group 16k / CSP, packed column (16k mod CSP) / 2 inside it
+__device__ __forceinline__ uint32_t packed_col(int k) { return (16 * k / CSP) * CSP + ((16 * k) % CSP) / 2; }
 constexpr int DKDV_QS = 5;
 constexpr int DKDV_SMEM = 2 * KV_T + DKDV_QS * 2 * QT64 + 1024 + 256;
 
@@ -544,10 +585,11 @@ __device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-// 64 fp32 TMEM columns of a row, scaled, as bf16 to global (128 bytes)
-__device__ __forceinline__ void row64_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
+// NC (a multiple of 32) fp32 TMEM columns of a row, scaled, as bf16 to global
+template <int NC>
+__device__ __forceinline__ void row_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
 #pragma unroll
-  for (int cc = 0; cc < 2; ++cc) {
+  for (int cc = 0; cc < NC / 32; ++cc) {
     uint32_t o[32];
     tc::tmem_ld32_nowait(taddr + cc * 32, o);
     tc::tmem_wait_ld();
@@ -607,7 +649,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 8);    // one arrival per compute warp
+      mbar_init(&p_full[s], 4 * NCG);  // one arrival per compute warp
       mbar_init(&g_done[s], 1);
     }
     mbar_init(o_full, 1);
@@ -624,7 +666,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   __syncthreads();
   tc_fence_after();
   // S^T buffers: cols 0, 64; dP^T buffers: 128, 192; dV: 256; dK: 384.  P^T / dS^T
-  // (bf16 pairs) overwrite the first 16 of each half's 32 S^T / dP^T columns.
+  // (bf16 pairs) overwrite the first CSP / 2 of each group's CSP S^T / dP^T columns.
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -687,14 +729,14 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           if (!mbar_wait(&p_full[s], (ip >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
-          // k-step k covers queries 16k..16k+15: half k / 2, packed columns (k % 2) * 8
+          // k-step k covers queries 16k..16k+15 (packed_col)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem + 256, tmem + s * 64 + (k >> 1) * 32 + (k & 1) * 8, mndesc(aO, QT64 / 2, k), id_g,
+            tc_mma_ts(tmem + 256, tmem + s * 64 + packed_col(k), mndesc(aO, QT64 / 2, k), id_g,
                       (ip > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem + 384, tmem + 128 + s * 64 + (k >> 1) * 32 + (k & 1) * 8, mndesc(aQ, QT64 / 2, k), id_g,
+            tc_mma_ts(tmem + 384, tmem + 128 + s * 64 + packed_col(k), mndesc(aQ, QT64 / 2, k), id_g,
                       (ip > 0 || k > 0) ? 1u : 0u);
           tc_commit(&g_done[s]);
           tc_commit(&q_empty[st]);
@@ -704,7 +746,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     }
   } else {
     // ---------------------------------------------------------------- P^T, dS^T
-    const int q4 = warp & 3, half = (warp - 2) >> 2;
+    const int q4 = warp & 3, grp = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
     const int key = k0 + r;
     const int warp_key_max = k0 + q4 * 32 + 31;
@@ -715,13 +757,13 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     bool ok = true;
     for (int i = 0; i < n_it; ++i) {
       const int s = i & 1;
-      const int qbase = (qi0 + i) * 64 + half * 32;
-      // this half's 32 (lse2, D) pairs, fetched before the scores arrive
-      const bool full32 = qbase + 32 <= T;  // warp-uniform
-      float lv[32], dv[32];
-      if (full32) {
+      const int qbase = (qi0 + i) * 64 + grp * CSP;
+      // this group's CSP (lse2, D) pairs, fetched before the scores arrive
+      const bool fullc = qbase + CSP <= T;  // warp-uniform
+      float lv[CSP], dv[CSP];
+      if (fullc) {
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
+        for (int e4 = 0; e4 < CSP / 4; ++e4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_bh + qbase + 4 * e4);
           const float4 d4 = *reinterpret_cast<const float4*>(D_bh + qbase + 4 * e4);
           lv[4 * e4] = l4.x; lv[4 * e4 + 1] = l4.y; lv[4 * e4 + 2] = l4.z; lv[4 * e4 + 3] = l4.w;
@@ -729,37 +771,37 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < CSP; ++e) {
           lv[e] = qbase + e < T ? lse_bh[qbase + e] : 0.f;
           dv[e] = qbase + e < T ? D_bh[qbase + e] : 0.f;
         }
       }
       if (!warp_wait(&s_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t cs = tmem + lane_off + s * 64 + half * 32;   // this warp's S^T columns
+      const uint32_t cs = tmem + lane_off + s * 64 + grp * CSP;   // this warp's S^T columns
       const uint32_t cd = cs + 128;                                // and dP^T columns
-      float sv[32], dp[32];
+      float sv[CSP], dp[CSP];
       {
-        uint32_t r0[32], r1[32];
-        tmem_ld32_nowait(cs, r0);
-        tmem_ld32_nowait(cd, r1);
+        uint32_t r0[CSP], r1[CSP];
+        tmem_ldw<CSP>(cs, r0);
+        tmem_ldw<CSP>(cd, r1);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
+        for (int e = 0; e < CSP; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
       }
       // P^T[key, q] = exp2(s c - lse2_q) for key <= q < T; dS^T = P^T (dP^T - D_q).
-      // Off the diagonal every key of the warp is <= every query of the half
+      // Off the diagonal every key of the warp is <= every query of the group
       // (warp-uniform), so the causal test drops out.
-      if (full32 && warp_key_max <= qbase) {
+      if (fullc && warp_key_max <= qbase) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < CSP; ++e) {
           const float p = fast_exp2(fmaf(sv[e], c, -lv[e]));
           sv[e] = p;
           dp[e] = p * (dp[e] - dv[e]);
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < CSP; ++e) {
           const int qq = qbase + e;
           const float p = (key <= qq && qq < T) ? fast_exp2(fmaf(sv[e], c, -lv[e])) : 0.f;
           sv[e] = p;
@@ -767,14 +809,14 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         }
       }
       // bf16 pairs over the columns just read (this warp's own lanes and columns)
-      uint32_t pw[16], dw[16];
+      uint32_t pw[CSP / 2], dw[CSP / 2];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < CSP / 2; ++j) {
         pw[j] = pack_bf16x2_rn(sv[2 * j], sv[2 * j + 1]);
         dw[j] = pack_bf16x2_int(dp[2 * j], dp[2 * j + 1]);
       }
-      tmem_st16(cs, pw);
-      tmem_st16(cd, dw);
+      tmem_stw<CSP / 2>(cs, pw);
+      tmem_stw<CSP / 2>(cd, dw);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -783,9 +825,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
       tc_fence_after();
       const bool valid = key < T;
-      bf16* krow = dqkv + ((long long)row_base + (valid ? key : 0)) * 3 * a + a + h * 128 + half * 64;
-      row64_out(tmem + lane_off + 256 + half * 64, 1.f, krow + a, valid);          // dV
-      row64_out(tmem + lane_off + 384 + half * 64, rsqrtf(128.f), krow, valid);    // dK
+      constexpr int OC = 128 / NCG;  // output columns of dV and dK per warp
+      bf16* krow = dqkv + ((long long)row_base + (valid ? key : 0)) * 3 * a + a + h * 128 + grp * OC;
+      row_out<OC>(tmem + lane_off + 256 + grp * OC, 1.f, krow + a, valid);          // dV
+      row_out<OC>(tmem + lane_off + 384 + grp * OC, rsqrtf(128.f), krow, valid);    // dK
     }
   }
   tc_fence_before();
@@ -797,7 +840,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 }
 
 // ---------------------------------------------------------------- dQ
-// 10 warps as above; compute warps split the 64 key columns in halves.
+// Warps as above; the compute warps' column groups split the 64 key columns.
 // Persistent like the forward: one CTA per SM over the (query tile,
 // sequence, head) items heaviest first; the K/V ring and the S/dP buffers run
 // on across items, Q/dO for the next item load once the item's last S/dP has
@@ -853,10 +896,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 8);    // one arrival per compute warp
+      mbar_init(&p_full[s], 4 * NCG);  // one arrival per compute warp
       mbar_init(&g_done[s], 1);
       mbar_init(&o_full[s], 1);
-      mbar_init(&o_empty[s], 8);
+      mbar_init(&o_empty[s], 4 * NCG);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -870,8 +913,8 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // S: 0, 64; dP: 128, 192 (dS as bf16 pairs over the first 16 of each half's
-  // 32 dP columns); dQ: 256 and 384 (alternating per item)
+  // S: 0, 64; dP: 128, 192 (dS as bf16 pairs over the first CSP / 2 of each
+  // group's CSP dP columns); dQ: 256 and 384 (alternating per item)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -963,10 +1006,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aK = smem_u32(sK + st * QT64);
-          // k-step k covers keys 16k..16k+15: half k / 2, packed columns (k % 2) * 8
+          // k-step k covers keys 16k..16k+15 (packed_col)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem + 256 + ob * 128, tmem + 128 + s * 64 + (k >> 1) * 32 + (k & 1) * 8,
+            tc_mma_ts(tmem + 256 + ob * 128, tmem + 128 + s * 64 + packed_col(k),
                       mndesc(aK, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
           tc_commit(&g_done[s]);
           tc_commit(&kv_empty[st]);
@@ -982,7 +1025,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     }
   } else {
     // ---------------------------------------------------------------- dS
-    const int q4 = warp & 3, half = (warp - 2) >> 2;
+    const int q4 = warp & 3, grp = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
@@ -1001,28 +1044,28 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         const int s = g & 1;
         if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t cd = tmem + lane_off + 128 + s * 64 + half * 32;  // this warp's dP columns
-        float sv[32], dp[32];
+        const uint32_t cd = tmem + lane_off + 128 + s * 64 + grp * CSP;  // this warp's dP columns
+        float sv[CSP], dp[CSP];
         {
-          uint32_t r0[32], r1[32];
-          tmem_ld32_nowait(tmem + lane_off + s * 64 + half * 32, r0);
-          tmem_ld32_nowait(cd, r1);
+          uint32_t r0[CSP], r1[CSP];
+          tmem_ldw<CSP>(tmem + lane_off + s * 64 + grp * CSP, r0);
+          tmem_ldw<CSP>(cd, r1);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
+          for (int e = 0; e < CSP; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
         }
-        const int kbase = j * 64 + half * 32;
+        const int kbase = j * 64 + grp * CSP;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < CSP; ++e) {
           const bool live = valid && (kbase + e <= qpos);
           const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
           dp[e] = p * (dp[e] - Dq);
         }
         // dS as bf16 pairs over the dP columns just read (this warp's own lanes and columns)
-        uint32_t dw[16];
+        uint32_t dw[CSP / 2];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) dw[jj] = pack_bf16x2_int(dp[2 * jj], dp[2 * jj + 1]);
-        tmem_st16(cd, dw);
+        for (int jj = 0; jj < CSP / 2; ++jj) dw[jj] = pack_bf16x2_int(dp[2 * jj], dp[2 * jj + 1]);
+        tmem_stw<CSP / 2>(cd, dw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -1031,8 +1074,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       if (!ok) break;
       if (!warp_wait(&o_full[ob], (k >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128 + half * 64;
-      row64_out(tmem + lane_off + 256 + ob * 128 + half * 64, rsqrtf(128.f), qrow, valid);
+      constexpr int OC = 128 / NCG;  // dQ output columns per warp
+      bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128 + grp * OC;
+      row_out<OC>(tmem + lane_off + 256 + ob * 128 + grp * OC, rsqrtf(128.f), qrow, valid);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[ob]);  // this dQ buffer may be overwritten
