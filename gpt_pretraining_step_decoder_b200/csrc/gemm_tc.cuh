@@ -265,6 +265,62 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
       "h"((uint16_t)3)
       : "memory");
 }
+// ---- warp-issued forms: the whole (converged) warp executes the call and
+// elect.sync picks the one lane that issues.  Measured on B200: issuing from a
+// converged warp keeps the operand descriptors on the warp-uniform path, which
+// takes about a fifth off the issue time of short products, and a commit
+// between products then costs nothing (from a lone lane each commit stalled
+// the issuing thread for about 100 cycles).  The election depends only on the
+// active mask, so a full warp elects the same lane at every call, and that
+// lane's commits track the products it issued.
+#define TC_ELECT_ISSUE(instr) \
+  "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t@e " instr ";\n\t}"
+__device__ __forceinline__ void tc_mma_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(TC_ELECT_ISSUE("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p") ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_f8_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(TC_ELECT_ISSUE("tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p") ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(TC_ELECT_ISSUE("tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p") ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair_f8_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(TC_ELECT_ISSUE("tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p") ::"r"(d_tmem),
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+// A from tensor memory (the `ts` form), warp-issued
+__device__ __forceinline__ void tc_mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(TC_ELECT_ISSUE("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p") ::"r"(d_tmem),
+               "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+               : "memory");
+}
+#undef TC_ELECT_ISSUE
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -519,8 +575,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (rank == 0) {
       // ------------------------------------------------------------ MMA issuer
+      // the whole warp runs the loop; one elected lane issues (tc_*_w)
       // D fp32; A, B bf16 (kind::f16) or e4m3 (kind::f8f6f4: format code 0)
       const uint32_t idesc = (1u << 4) | (F8 ? 0u : (1u << 7) | (1u << 10)) | ((uint32_t)(!p.a_kmajor) << 15) |
                              ((uint32_t)(!p.b_kmajor) << 16) | ((uint32_t)(BN >> 3) << 17) |
@@ -534,11 +591,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int split = (B3 ? t % per_product : t) % p.splits;
         const int kb0 = split * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err)) { ok = false; break; }
+        if (!warp_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+          if (!warp_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
@@ -546,18 +603,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction: 16 bf16 or 32 e4m3
             const uint64_t ad = operand_desc(a_base, p.a_kmajor, k), bd = operand_desc(b_base, p.b_kmajor, k);
             const uint32_t acc_in = (kb > kb0 || k > 0) ? 1u : 0u;
-            if constexpr (CG == 2 && F8) tc_mma_pair_f8(d_tmem, ad, bd, idesc, acc_in);
-            else if constexpr (CG == 2) tc_mma_pair(d_tmem, ad, bd, idesc, acc_in);
-            else if constexpr (F8) tc_mma_f8(d_tmem, ad, bd, idesc, acc_in);
-            else tc_mma(d_tmem, ad, bd, idesc, acc_in);
+            if constexpr (CG == 2 && F8) tc_mma_pair_f8_w(d_tmem, ad, bd, idesc, acc_in);
+            else if constexpr (CG == 2) tc_mma_pair_w(d_tmem, ad, bd, idesc, acc_in);
+            else if constexpr (F8) tc_mma_f8_w(d_tmem, ad, bd, idesc, acc_in);
+            else tc_mma_w(d_tmem, ad, bd, idesc, acc_in);
           }
-          if constexpr (CG == 2) tc_commit_pair(&empty[stage]);
-          else tc_commit(&empty[stage]);
+          if constexpr (CG == 2) tc_commit_pair_w(&empty[stage]);
+          else tc_commit_w(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        if constexpr (CG == 2) tc_commit_pair(&tfull[acc]);
-        else tc_commit(&tfull[acc]);
+        if constexpr (CG == 2) tc_commit_pair_w(&tfull[acc]);
+        else tc_commit_w(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
     }
