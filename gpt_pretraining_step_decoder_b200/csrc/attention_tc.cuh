@@ -507,67 +507,32 @@ __device__ __forceinline__ uint32_t idesc(int n, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(128 >> 4) << 24);
 }
-__device__ __forceinline__ void ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r0[32], r1[32];
-  tc::tmem_ld32_nowait(taddr, r0);
-  tc::tmem_ld32_nowait(taddr + 32, r1);
-  tc::tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) { v[i] = __uint_as_float(r0[i]); v[32 + i] = __uint_as_float(r1[i]); }
-}
-// one row of 64 bf16 (128 bytes) into a K-major swizzled [rows x 64] tile
-__device__ __forceinline__ void st_row64(uint8_t* tile, int r, const float (&v)[64]) {
-#pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    uint4 w;
-    __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * jj], v[8 * jj + 1]);
-    __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * jj + 2], v[8 * jj + 3]);
-    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * jj + 4], v[8 * jj + 5]);
-    __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * jj + 6], v[8 * jj + 7]);
-    w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-    w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-    *reinterpret_cast<uint4*>(tile + r * 128 + ((jj ^ (r & 7)) << 4)) = w;
-  }
-}
-// one 128-column fp32 TMEM row, scaled, as bf16 to global (256 bytes)
-__device__ __forceinline__ void row128_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
-#pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
-    uint32_t o[32];
-    tc::tmem_ld32_nowait(taddr + cc * 32, o);
-    tc::tmem_wait_ld();
-    if (valid) {
-#pragma unroll
-      for (int i = 0; i < 32; i += 8) {
-        uint4 w;
-        __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * scale, __uint_as_float(o[i + 1]) * scale);
-        __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * scale, __uint_as_float(o[i + 3]) * scale);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * scale, __uint_as_float(o[i + 5]) * scale);
-        __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * scale, __uint_as_float(o[i + 7]) * scale);
-        w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-        w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-        *reinterpret_cast<uint4*>(dst + cc * 32 + i) = w;
-      }
-    }
-  }
-}
-
 // ---------------------------------------------------------------- dK, dV
-// 2 + 4 * NCG warps: 0 TMA, 1 MMA, the rest compute.  Compute warp w owns
-// TMEM lane quarter w % 4 (32 key rows) and column group (w - 2) / 4 of the
-// 64 query columns, so NCG warps per scheduler share the elementwise work.
-// smem: K, V [128 x 128] (32 KB each); per stage Q_i, dO_i [64 x 128] (16 KB
-// each, DKDV_QS stages).  P^T and dS^T never touch shared memory: each
-// compute warp writes them as bf16 over the fp32 S^T / dP^T columns it has
-// just read (its own lanes and columns), and the dV / dK products take them
-// as their A operand straight from TMEM.  Per 64-query step the tensor core
-// then reads only K, V, Q and dO from shared memory, which is what bounds the
-// step (operand bytes through shared memory), and the S^T / dP^T buffers
-// alternate, so step i+1's S^T / dP^T products run while step i's
-// elementwise work does.  lse and D come straight from global memory.
-// NCG warps share each 32-row TMEM lane quarter, one group of CSP = 64 / NCG
-// of a step's 64 columns each: 4 * NCG compute warps, so every scheduler has
-// NCG of them to interleave (the elementwise work has no cross-warp step).
+// 2 + 4 * NCG warps: 0 TMA (lane 0 the Q/dO ring, lane 1 the K/V tiles), 1
+// MMA, the rest compute.  Compute warp w owns TMEM lane quarter w % 4 (32 key
+// rows) and column group (w - 2) / 4 of the 64 query columns, so NCG warps
+// per scheduler share the elementwise work.
+// Persistent: one CTA per SM over the (key tile, sequence, head) items,
+// heaviest first.  smem: two K/V buffers [128 x 128] x 2 (64 KB each, item k
+// in buffer k & 1, so the next item's keys load while this item runs) and
+// the Q_i, dO_i [64 x 128] ring (16 KB each, DKDV_QS stages).  P^T and dS^T
+// never touch shared memory: each compute warp writes them as bf16 over the
+// fp32 S^T / dP^T columns it has just read (its own lanes and columns), and
+// the dV / dK products take them as their A operand straight from TMEM.  The
+// S^T / dP^T buffers alternate, so step i+1's S^T / dP^T products run while
+// step i's elementwise work does.  lse and D come straight from global
+// memory.
+// The MMA warp issues as a whole warp (one elected lane), and the dV and dK
+// products commit separately: step i + 2's S^T product waits only for step
+// i's dV product (which read P^T from that buffer) and its dP^T product for
+// step i's dK product, each of which the tensor pipe has finished or is
+// finishing while the other runs, so the pipe never drains between steps.
+// An item's dK and dV leave through shared memory: the item's K/V buffer is
+// free once its last S^T / dP^T products are done, and each compute warp
+// writes its 32 rows x 64 columns of dK and of dV there as bf16 in the
+// 128-byte swizzle and stores them with TMA copies (rows past the sequence
+// end clipped by the map's T extent).  The buffer returns to the K/V loader
+// once those copies have read it.
 constexpr int NCG = 2;
 constexpr int CSP = 64 / NCG;
 constexpr int THREADS_B = 64 + 32 * 4 * NCG;
@@ -575,84 +540,65 @@ constexpr int KV_T = 32768, QT64 = 16384;
 // TMEM column of the packed bf16 A operand for MMA k-step k (16 of the 64 step
 // columns): column group 16k / CSP, packed column (16k mod CSP) / 2 inside it
 __device__ __forceinline__ uint32_t packed_col(int k) { return (16 * k / CSP) * CSP + ((16 * k) % CSP) / 2; }
-constexpr int DKDV_QS = 5;
-constexpr int DKDV_SMEM = 2 * KV_T + DKDV_QS * 2 * QT64 + 1024 + 256;
 
-__device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  tc::tmem_ld32_nowait(taddr, r);
-  tc::tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-// NC (a multiple of 32) fp32 TMEM columns of a row, scaled, as bf16 to global
-template <int NC>
-__device__ __forceinline__ void row_out(uint32_t taddr, float scale, bf16* dst, bool valid) {
-#pragma unroll
-  for (int cc = 0; cc < NC / 32; ++cc) {
-    uint32_t o[32];
-    tc::tmem_ld32_nowait(taddr + cc * 32, o);
-    tc::tmem_wait_ld();
-    if (valid) {
-#pragma unroll
-      for (int i = 0; i < 32; i += 8) {
-        uint4 w;
-        __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[i]) * scale, __uint_as_float(o[i + 1]) * scale);
-        __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[i + 2]) * scale, __uint_as_float(o[i + 3]) * scale);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[i + 4]) * scale, __uint_as_float(o[i + 5]) * scale);
-        __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[i + 6]) * scale, __uint_as_float(o[i + 7]) * scale);
-        w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-        w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-        *reinterpret_cast<uint4*>(dst + cc * 32 + i) = w;
-      }
-    }
-  }
-}
+constexpr int STG_WARP = 32 * 128;   // one compute warp's 32 x 64 bf16 block (128-byte rows)
+constexpr int DKDV_QS = 3;
+constexpr int KV_BUF = 2 * KV_T;   // K and V of one item
+constexpr int DKDV_SMEM = 2 * KV_BUF + DKDV_QS * 2 * QT64 + 1024 + 256;
 
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
-                          const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse2,
-                          const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, unsigned* err) {
+                          const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmG,
+                          const float* __restrict__ lse2, const float* __restrict__ Dv, int T, int H, int BH,
+                          unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = smem;
-  uint8_t* sV = sK + KV_T;
-  uint8_t* sQ = sV + KV_T;               // [DKDV_QS stages]
-  uint8_t* sO = sQ + DKDV_QS * QT64;     // dO [DKDV_QS stages]
+  uint8_t* sKV = smem;                        // [2 buffers]: K then V
+  uint8_t* sQ = sKV + 2 * KV_BUF;             // [DKDV_QS stages]
+  uint8_t* sO = sQ + DKDV_QS * QT64;          // dO [DKDV_QS stages]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sO + DKDV_QS * QT64);
-  uint64_t* kv_full = bars;                  // 1
-  uint64_t* q_full = bars + 1;               // DKDV_QS
-  uint64_t* q_empty = q_full + DKDV_QS;      // DKDV_QS
-  uint64_t* s_full = q_empty + DKDV_QS;      // 2: S^T, dP^T of the buffer computed
-  uint64_t* p_full = s_full + 2;             // 2: P^T, dS^T of the buffer written (8 warps)
-  uint64_t* g_done = p_full + 2;             // 2: the dV/dK products have read the buffer
-  uint64_t* o_full = g_done + 2;             // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
-  static_assert((1 + 2 * DKDV_QS + 7) * 8 + 8 <= 256, "barrier area");
+  uint64_t* kv_full = bars;                   // 2 (per K/V buffer)
+  uint64_t* kv_free = kv_full + 2;            // 2 (per K/V buffer: the item's dK/dV copies have read it)
+  uint64_t* q_full = kv_free + 2;             // DKDV_QS
+  uint64_t* q_empty = q_full + DKDV_QS;       // DKDV_QS
+  uint64_t* s_full = q_empty + DKDV_QS;       // 2: S^T, dP^T of the buffer computed
+  uint64_t* p_full = s_full + 2;              // 2: P^T, dS^T of the buffer written (all compute warps)
+  uint64_t* dv_done = p_full + 2;             // 2: the dV product has read P^T of the buffer
+  uint64_t* dk_done = dv_done + 2;            // 2: the dK product has read dS^T of the buffer
+  uint64_t* acc_full = dk_done + 2;           // 1: the item's last dV/dK products are done
+  uint64_t* acc_empty = acc_full + 1;         // 1: the compute warps have read dV/dK
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  static_assert((14 + 2 * DKDV_QS) * 8 + 8 <= 256, "barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;  // key tiles near the start have the most query tiles: launched first
-  const int bh = blockIdx.y, b = bh / H, h = bh % H;
   const int a = H * 128;
-  const int k0 = kt * 128;
-  const int row_base = b * T;
-  const int qi0 = k0 / 64, nq = (T + 63) / 64;
-  const int n_it = nq - qi0;
+  const int n_kt = (T + 127) / 128, nq = (T + 63) / 64;
+  const int total = n_kt * BH;
+  const int first = blockIdx.x, stride = gridDim.x;
+  // item i (heaviest first): key tile kt, (sequence, head) bh, query steps of 64 from the diagonal on
+  auto item = [&](int i, int& kt, int& bh, int& n_it) {
+    kt = i / BH;
+    bh = i % BH;
+    n_it = nq - 2 * kt;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_free[s], 4 * NCG);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 4 * NCG);  // one arrival per compute warp
+      mbar_init(&dv_done[s], 1);
+      mbar_init(&dk_done[s], 1);
+    }
     for (int s = 0; s < DKDV_QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4 * NCG);  // one arrival per compute warp
-      mbar_init(&g_done[s], 1);
-    }
-    mbar_init(o_full, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4 * NCG);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -670,77 +616,120 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- TMA
+    if (lane == 1) {
+      // ---------------------------------------------------------------- TMA: K, V
       bool ok = true;
-      mbar_expect_tx(kv_full, 2 * KV_T);
-      tma_load_2d(sK, &tm128, kv_full, a + h * 128, row_base + k0);
-      tma_load_2d(sK + KV_T / 2, &tm128, kv_full, a + h * 128 + 64, row_base + k0);
-      tma_load_2d(sV, &tm128, kv_full, 2 * a + h * 128, row_base + k0);
-      tma_load_2d(sV + KV_T / 2, &tm128, kv_full, 2 * a + h * 128 + 64, row_base + k0);
-      int issued = 0;
-      for (int i = 0; i < n_it && ok; ++i) {
-        const int s = i % DKDV_QS;
-        if (!mbar_wait(&q_empty[s], ((i / DKDV_QS) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
-        mbar_expect_tx(&q_full[s], 2 * QT64);
-        const int qs = (qi0 + i) * 64, qr = row_base + qs;
-        uint8_t* q = sQ + s * QT64;
-        uint8_t* o = sO + s * QT64;
-        tma_load_2d(q, &tm64, &q_full[s], h * 128, qr);
-        tma_load_2d(q + QT64 / 2, &tm64, &q_full[s], h * 128 + 64, qr);
-        tma_load_2d(o, &tmDO, &q_full[s], h * 128, qr);
-        tma_load_2d(o + QT64 / 2, &tmDO, &q_full[s], h * 128 + 64, qr);
-        ++issued;
+      int nkv = 0;
+      for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+        int kt, bh, n_it;
+        item(i, kt, bh, n_it);
+        const int b = bh / H, h = bh % H, kr = b * T + kt * 128, kb = k & 1;
+        // the dK/dV copies of item k - 2 have read this buffer
+        if (k >= 2 && !mbar_wait(&kv_free[kb], ((k - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        uint8_t* kv = sKV + kb * KV_BUF;
+        mbar_expect_tx(&kv_full[kb], KV_BUF);
+        tma_load_2d(kv, &tm128, &kv_full[kb], a + h * 128, kr);
+        tma_load_2d(kv + KV_T / 2, &tm128, &kv_full[kb], a + h * 128 + 64, kr);
+        tma_load_2d(kv + KV_T, &tm128, &kv_full[kb], 2 * a + h * 128, kr);
+        tma_load_2d(kv + KV_T + KV_T / 2, &tm128, &kv_full[kb], 2 * a + h * 128 + 64, kr);
+        ++nkv;
       }
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(kv_full, 0)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
-      for (int i = (issued > DKDV_QS ? issued - DKDV_QS : 0); i < issued; ++i) {
+      for (int k = (nkv > 2 ? nkv - 2 : 0); k < nkv; ++k) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&kv_full[k & 1], (k >> 1) & 1)) if (globaltimer_ns() - t0 > GPT_WAIT_LIMIT_NS) break;
+      }
+    } else if (lane == 0) {
+      // ---------------------------------------------------------------- TMA: Q, dO ring
+      bool ok = true;
+      int g = 0;
+      for (int i = first; i < total && ok; i += stride) {
+        int kt, bh, n_it;
+        item(i, kt, bh, n_it);
+        const int b = bh / H, h = bh % H, row_base = b * T;
+        for (int j = 0; j < n_it && ok; ++j, ++g) {
+          const int s = g % DKDV_QS;
+          if (!mbar_wait(&q_empty[s], ((g / DKDV_QS) & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          mbar_expect_tx(&q_full[s], 2 * QT64);
+          const int qr = row_base + (2 * kt + j) * 64;
+          uint8_t* q = sQ + s * QT64;
+          uint8_t* o = sO + s * QT64;
+          tma_load_2d(q, &tm64, &q_full[s], h * 128, qr);
+          tma_load_2d(q + QT64 / 2, &tm64, &q_full[s], h * 128 + 64, qr);
+          tma_load_2d(o, &tmDO, &q_full[s], h * 128, qr);
+          tma_load_2d(o + QT64 / 2, &tmDO, &q_full[s], h * 128 + 64, qr);
+        }
+      }
+      for (int j = (g > DKDV_QS ? g - DKDV_QS : 0); j < g; ++j) {
         const uint64_t t1 = globaltimer_ns();
-        while (!mbar_try_wait(&q_full[i % DKDV_QS], (i / DKDV_QS) & 1))
+        while (!mbar_try_wait(&q_full[j % DKDV_QS], (j / DKDV_QS) & 1))
           if (globaltimer_ns() - t1 > GPT_WAIT_LIMIT_NS) break;
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA
-      // iteration i: S^T, dP^T of step i into buffer i & 1 (once the dV/dK
-      // products of step i - 2 have read that buffer), then dV, dK of step i - 1
-      const uint32_t id_s = idesc(64, false);   // S^T = K Q^T, dP^T = V dO^T (N = 64 queries)
-      const uint32_t id_g = idesc(128, true);   // dV += P^T dO, dK += dS^T Q (N = 128, B MN-major)
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(kv_full, 0, abort_flag, err);
-      for (int i = 0; i <= n_it && ok; ++i) {
-        if (i < n_it) {
-          const int s = i & 1, st = i % DKDV_QS;
-          if (!mbar_wait(&q_full[st], (i / DKDV_QS) & 1, abort_flag, err)) { ok = false; break; }
-          if (i >= 2 && !mbar_wait(&g_done[s], ((i - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
+    // ---------------------------------------------------------------- MMA
+    // One flattened sequence over this CTA's items: iteration g issues S^T,
+    // dP^T of step g, then dV, dK of step g - 1 (possibly of the previous
+    // item).  The whole warp runs it; one elected lane issues.
+    const uint32_t id_s = idesc(64, false);   // S^T = K Q^T, dP^T = V dO^T (N = 64 queries)
+    const uint32_t id_g = idesc(128, true);   // dV += P^T dO, dK += dS^T Q (N = 128, B MN-major)
+    bool ok = true;
+    int i_s = first, k_s = 0, j_s = 0, n_s = 0;
+    int i_p = first, k_p = 0, j_p = 0, n_p = 0;
+    if (i_s < total) { int kt, bh; item(i_s, kt, bh, n_s); n_p = n_s; }
+    for (int g = 0; ok; ++g) {
+      const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
+      if (!s_left && !p_left) break;
+      if (s_left) {
+        const int s = g & 1, st = g % DKDV_QS, kb = k_s & 1;
+        if (j_s == 0 && !warp_wait(&kv_full[kb], (k_s >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(&q_full[st], (g / DKDV_QS) & 1, abort_flag, err)) { ok = false; break; }
+        // S^T goes over P^T of step g - 2: the dV product of step g - 2 has read it
+        if (g >= 2 && !warp_wait(&dv_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sKV + kb * KV_BUF), aV = aK + KV_T;
+        const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            tc_mma(tmem + s * 64, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 8; ++k)
+          tc_mma_w(tmem + s * 64, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        // dP^T goes over dS^T of step g - 2: the dK product of step g - 2 has read it
+        if (g >= 2 && !warp_wait(&dk_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            tc_mma(tmem + 128 + s * 64, kdesc128(aV, KV_T / 2, k), kdesc128(aO, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
-          tc_commit(&s_full[s]);
+        for (int k = 0; k < 8; ++k)
+          tc_mma_w(tmem + 128 + s * 64, kdesc128(aV, KV_T / 2, k), kdesc128(aO, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        tc_commit_w(&s_full[s]);
+        if (++j_s == n_s) {
+          j_s = 0;
+          ++k_s;
+          i_s += stride;
+          if (i_s < total) { int kt, bh; item(i_s, kt, bh, n_s); }
         }
-        if (i >= 1) {
-          const int ip = i - 1, s = ip & 1, st = ip % DKDV_QS;
-          if (!mbar_wait(&p_full[s], (ip >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
-          // k-step k covers queries 16k..16k+15 (packed_col)
+      }
+      if (p_left) {
+        const int gp = g - 1, s = gp & 1, st = gp % DKDV_QS;
+        // the item's first products overwrite dV, dK: the previous item's have been read
+        if (j_p == 0 && k_p >= 1 && !warp_wait(acc_empty, (k_p - 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
+        // k-step k covers queries 16k..16k+15 (packed_col)
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem + 256, tmem + s * 64 + packed_col(k), mndesc(aO, QT64 / 2, k), id_g,
-                      (ip > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < 4; ++k)
+          tc_mma_ts_w(tmem + 256, tmem + s * 64 + packed_col(k), mndesc(aO, QT64 / 2, k), id_g,
+                      (j_p > 0 || k > 0) ? 1u : 0u);
+        tc_commit_w(&dv_done[s]);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem + 384, tmem + 128 + s * 64 + packed_col(k), mndesc(aQ, QT64 / 2, k), id_g,
-                      (ip > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&g_done[s]);
-          tc_commit(&q_empty[st]);
-          if (ip == n_it - 1) tc_commit(o_full);
+        for (int k = 0; k < 4; ++k)
+          tc_mma_ts_w(tmem + 384, tmem + 128 + s * 64 + packed_col(k), mndesc(aQ, QT64 / 2, k), id_g,
+                      (j_p > 0 || k > 0) ? 1u : 0u);
+        tc_commit_w(&dk_done[s]);
+        tc_commit_w(&q_empty[st]);
+        if (++j_p == n_p) {  // the item's last products: dV, dK are complete
+          tc_commit_w(acc_full);
+          j_p = 0;
+          ++k_p;
+          i_p += stride;
+          if (i_p < total) { int kt, bh; item(i_p, kt, bh, n_p); }
         }
       }
     }
@@ -748,88 +737,143 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     // ---------------------------------------------------------------- P^T, dS^T
     const int q4 = warp & 3, grp = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
-    const int key = k0 + r;
-    const int warp_key_max = k0 + q4 * 32 + 31;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
-    const float* lse_bh = lse2 + (long long)bh * T;
-    const float* D_bh = Dv + (long long)bh * T;
+    const int blk = (grp * 4 + q4) * STG_WARP;   // this warp's 32 x 64 block inside the K (dK) / V (dV) halves
     bool ok = true;
-    for (int i = 0; i < n_it; ++i) {
-      const int s = i & 1;
-      const int qbase = (qi0 + i) * 64 + grp * CSP;
-      // this group's CSP (lse2, D) pairs, fetched before the scores arrive
-      const bool fullc = qbase + CSP <= T;  // warp-uniform
-      float lv[CSP], dv[CSP];
-      if (fullc) {
+    bool store_pending = false;   // the previous item's dK/dV copies may still be reading its buffer
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int kt, bh, n_it;
+      item(i, kt, bh, n_it);
+      const int b = bh / H, h = bh % H;
+      const int k0 = kt * 128, qi0 = 2 * kt;
+      const int key = k0 + r;
+      const int warp_key_max = k0 + q4 * 32 + 31;
+      const float* lse_bh = lse2 + (long long)bh * T;
+      const float* D_bh = Dv + (long long)bh * T;
+      for (int j = 0; j < n_it; ++j, ++g) {
+        const int s = g & 1;
+        const int qbase = (qi0 + j) * 64 + grp * CSP;
+        // this group's CSP (lse2, D) pairs, fetched before the scores arrive
+        const bool fullc = qbase + CSP <= T;  // warp-uniform
+        float lv[CSP], dv[CSP];
+        if (fullc) {
 #pragma unroll
-        for (int e4 = 0; e4 < CSP / 4; ++e4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_bh + qbase + 4 * e4);
-          const float4 d4 = *reinterpret_cast<const float4*>(D_bh + qbase + 4 * e4);
-          lv[4 * e4] = l4.x; lv[4 * e4 + 1] = l4.y; lv[4 * e4 + 2] = l4.z; lv[4 * e4 + 3] = l4.w;
-          dv[4 * e4] = d4.x; dv[4 * e4 + 1] = d4.y; dv[4 * e4 + 2] = d4.z; dv[4 * e4 + 3] = d4.w;
+          for (int e4 = 0; e4 < CSP / 4; ++e4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse_bh + qbase + 4 * e4);
+            const float4 d4 = *reinterpret_cast<const float4*>(D_bh + qbase + 4 * e4);
+            lv[4 * e4] = l4.x; lv[4 * e4 + 1] = l4.y; lv[4 * e4 + 2] = l4.z; lv[4 * e4 + 3] = l4.w;
+            dv[4 * e4] = d4.x; dv[4 * e4 + 1] = d4.y; dv[4 * e4 + 2] = d4.z; dv[4 * e4 + 3] = d4.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < CSP; ++e) {
+            lv[e] = qbase + e < T ? lse_bh[qbase + e] : 0.f;
+            dv[e] = qbase + e < T ? D_bh[qbase + e] : 0.f;
+          }
         }
-      } else {
+        if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t cs = tmem + lane_off + s * 64 + grp * CSP;   // this warp's S^T columns
+        const uint32_t cd = cs + 128;                                // and dP^T columns
+        float sv[CSP], dp[CSP];
+        {
+          uint32_t r0[CSP], r1[CSP];
+          tmem_ldw<CSP>(cs, r0);
+          tmem_ldw<CSP>(cd, r1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < CSP; ++e) {
-          lv[e] = qbase + e < T ? lse_bh[qbase + e] : 0.f;
-          dv[e] = qbase + e < T ? D_bh[qbase + e] : 0.f;
+          for (int e = 0; e < CSP; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
+        }
+        // P^T[key, q] = exp2(s c - lse2_q) for key <= q < T; dS^T = P^T (dP^T - D_q).
+        // Off the diagonal every key of the warp is <= every query of the group
+        // (warp-uniform), so the causal test drops out.
+        if (fullc && warp_key_max <= qbase) {
+#pragma unroll
+          for (int e = 0; e < CSP; ++e) {
+            const float p = fast_exp2(fmaf(sv[e], c, -lv[e]));
+            sv[e] = p;
+            dp[e] = p * (dp[e] - dv[e]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < CSP; ++e) {
+            const int qq = qbase + e;
+            const float p = (key <= qq && qq < T) ? fast_exp2(fmaf(sv[e], c, -lv[e])) : 0.f;
+            sv[e] = p;
+            dp[e] = p * (dp[e] - dv[e]);
+          }
+        }
+        // bf16 pairs over the columns just read (this warp's own lanes and columns)
+        uint32_t pw[CSP / 2], dw[CSP / 2];
+#pragma unroll
+        for (int jj = 0; jj < CSP / 2; ++jj) {
+          pw[jj] = pack_bf16x2_rn(sv[2 * jj], sv[2 * jj + 1]);
+          dw[jj] = pack_bf16x2_int(dp[2 * jj], dp[2 * jj + 1]);
+        }
+        tmem_stw<CSP / 2>(cs, pw);
+        tmem_stw<CSP / 2>(cd, dw);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[s]);
+        if (j == 0 && store_pending) {
+          // the previous item's dK/dV copies have had a step to read its K/V
+          // buffer: hand the buffer back to the K/V loader
+          if (lane == 0) {
+            bulk_wait_read0();
+            mbar_arrive(&kv_free[(k - 1) & 1]);
+          }
+          store_pending = false;
         }
       }
-      if (!warp_wait(&s_full[s], (i >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (!ok) break;
+      // ------------------------------------------------------------ item epilogue
+      if (!warp_wait(acc_full, k & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t cs = tmem + lane_off + s * 64 + grp * CSP;   // this warp's S^T columns
-      const uint32_t cd = cs + 128;                                // and dP^T columns
-      float sv[CSP], dp[CSP];
-      {
-        uint32_t r0[CSP], r1[CSP];
-        tmem_ldw<CSP>(cs, r0);
-        tmem_ldw<CSP>(cd, r1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < CSP; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
-      }
-      // P^T[key, q] = exp2(s c - lse2_q) for key <= q < T; dS^T = P^T (dP^T - D_q).
-      // Off the diagonal every key of the warp is <= every query of the group
-      // (warp-uniform), so the causal test drops out.
-      if (fullc && warp_key_max <= qbase) {
-#pragma unroll
-        for (int e = 0; e < CSP; ++e) {
-          const float p = fast_exp2(fmaf(sv[e], c, -lv[e]));
-          sv[e] = p;
-          dp[e] = p * (dp[e] - dv[e]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < CSP; ++e) {
-          const int qq = qbase + e;
-          const float p = (key <= qq && qq < T) ? fast_exp2(fmaf(sv[e], c, -lv[e])) : 0.f;
-          sv[e] = p;
-          dp[e] = p * (dp[e] - dv[e]);
-        }
-      }
-      // bf16 pairs over the columns just read (this warp's own lanes and columns)
-      uint32_t pw[CSP / 2], dw[CSP / 2];
-#pragma unroll
-      for (int j = 0; j < CSP / 2; ++j) {
-        pw[j] = pack_bf16x2_rn(sv[2 * j], sv[2 * j + 1]);
-        dw[j] = pack_bf16x2_int(dp[2 * j], dp[2 * j + 1]);
-      }
-      tmem_stw<CSP / 2>(cs, pw);
-      tmem_stw<CSP / 2>(cd, dw);
-      tmem_wait_st();
+      static_assert(NCG == 2, "two 64-column groups of dK and dV");
+      uint32_t v0[32], v1[32], k0r[32], k1r[32];
+      tmem_ld32_nowait(tmem + lane_off + 256 + grp * 64, v0);
+      tmem_ld32_nowait(tmem + lane_off + 256 + grp * 64 + 32, v1);
+      tmem_ld32_nowait(tmem + lane_off + 384 + grp * 64, k0r);
+      tmem_ld32_nowait(tmem + lane_off + 384 + grp * 64 + 32, k1r);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[s]);
+      if (lane == 0) mbar_arrive(acc_empty);  // the next item's products may overwrite dV, dK
+      // staging: this item's K/V buffer (its last S^T / dP^T products are done)
+      uint8_t* stK = sKV + (k & 1) * KV_BUF + blk;
+      uint8_t* stV = stK + KV_T;
+      const float sc = rsqrtf(128.f);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t* sv_ = jj < 4 ? v0 + 8 * jj : v1 + 8 * (jj - 4);
+        const uint32_t* sk_ = jj < 4 ? k0r + 8 * jj : k1r + 8 * (jj - 4);
+        uint4 wv, wk;
+        wv.x = pack_bf16x2_rn(__uint_as_float(sv_[0]), __uint_as_float(sv_[1]));
+        wv.y = pack_bf16x2_rn(__uint_as_float(sv_[2]), __uint_as_float(sv_[3]));
+        wv.z = pack_bf16x2_rn(__uint_as_float(sv_[4]), __uint_as_float(sv_[5]));
+        wv.w = pack_bf16x2_rn(__uint_as_float(sv_[6]), __uint_as_float(sv_[7]));
+        wk.x = pack_bf16x2_rn(__uint_as_float(sk_[0]) * sc, __uint_as_float(sk_[1]) * sc);
+        wk.y = pack_bf16x2_rn(__uint_as_float(sk_[2]) * sc, __uint_as_float(sk_[3]) * sc);
+        wk.z = pack_bf16x2_rn(__uint_as_float(sk_[4]) * sc, __uint_as_float(sk_[5]) * sc);
+        wk.w = pack_bf16x2_rn(__uint_as_float(sk_[6]) * sc, __uint_as_float(sk_[7]) * sc);
+        *reinterpret_cast<uint4*>(stV + swz128(lane, jj)) = wv;
+        *reinterpret_cast<uint4*>(stK + swz128(lane, jj)) = wk;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (k0 + q4 * 32 < T) {  // rows past T are clipped; a block wholly past it is skipped
+          tma_store_3d(&tmG, stK, a + h * 128 + grp * 64, k0 + q4 * 32, b);
+          tma_store_3d(&tmG, stV, 2 * a + h * 128 + grp * 64, k0 + q4 * 32, b);
+        }
+        bulk_commit();
+      }
+      store_pending = true;
     }
-    if (__all_sync(0xffffffffu, ok) && n_it > 0 && warp_wait(o_full, 0, abort_flag, err)) {
-      tc_fence_after();
-      const bool valid = key < T;
-      constexpr int OC = 128 / NCG;  // output columns of dV and dK per warp
-      bf16* krow = dqkv + ((long long)row_base + (valid ? key : 0)) * 3 * a + a + h * 128 + grp * OC;
-      row_out<OC>(tmem + lane_off + 256 + grp * OC, 1.f, krow + a, valid);          // dV
-      row_out<OC>(tmem + lane_off + 384 + grp * OC, rsqrtf(128.f), krow, valid);    // dK
-    }
+    if (lane == 0) bulk_wait0();  // this warp's stores are complete
   }
   tc_fence_before();
   __syncthreads();
@@ -847,15 +891,23 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 // read them, and dQ alternates between two TMEM accumulators.  dS is written
 // as bf16 over the dP columns each compute warp has just read and feeds the
 // dQ product from TMEM.
+// The MMA warp issues as a whole warp (one elected lane).  Step g's score
+// product needs only that the compute warps have read buffer g & 1 (they
+// released step g - 2 before the dQ product of step g - 2 was issued); its dP
+// product waits for that dQ product, which the score product separates from
+// it in the tensor pipe, so the pipe never drains between steps.
+// The item's dQ leaves through shared memory: each compute warp writes its 32
+// rows x 64 columns as bf16 in the 128-byte swizzle and stores them with one
+// TMA copy (rows past the sequence end are clipped by the map's T extent).
 // smem: Q, dO [128 x 128] (32 KB each); per stage K_j, V_j [64 x 128] (16 KB
-// each, DQ_STAGES stages).
-constexpr int DQ_STAGES = 5;
-constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 1024 + 256;
+// each, DQ_STAGES stages); 8 staging blocks of 4 KB.
+constexpr int DQ_STAGES = 4;
+constexpr int DQ_SMEM = 2 * KV_T + DQ_STAGES * 2 * QT64 + 4 * NCG * STG_WARP + 1024 + 256;
 
 __global__ void __launch_bounds__(THREADS_B, 1)
     fa_tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm128, const __grid_constant__ CUtensorMap tm64,
-                        const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse2,
-                        const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, int BH,
+                        const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmG,
+                        const float* __restrict__ lse2, const float* __restrict__ Dv, int T, int H, int BH,
                         unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
@@ -864,18 +916,19 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint8_t* sO = sQ + KV_T;
   uint8_t* sK = sO + KV_T;                   // [stages]
   uint8_t* sV = sK + DQ_STAGES * QT64;       // [stages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + DQ_STAGES * QT64);
+  uint8_t* sStg = sV + DQ_STAGES * QT64;     // [compute warps]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + 4 * NCG * STG_WARP);
   uint64_t* q_full = bars;                      // 1
   uint64_t* q_empty = q_full + 1;               // 1 (the item's last S/dP have read Q and dO)
   uint64_t* kv_full = q_empty + 1;              // DQ_STAGES
   uint64_t* kv_empty = kv_full + DQ_STAGES;     // DQ_STAGES
   uint64_t* s_full = kv_empty + DQ_STAGES;      // 2: S, dP of the buffer computed
-  uint64_t* p_full = s_full + 2;                // 2: dS of the buffer written (8 warps)
+  uint64_t* p_full = s_full + 2;                // 2: dS of the buffer written (all compute warps)
   uint64_t* g_done = p_full + 2;                // 2: the dQ product has read the buffer
   uint64_t* o_full = g_done + 2;                // 2 (per dQ buffer: the item's last product is done)
   uint64_t* o_empty = o_full + 2;               // 2 (per dQ buffer: the compute warps have read it)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
-  static_assert((2 + 2 * DQ_STAGES + 12) * 8 + 8 <= 256, "barrier area");
+  static_assert((2 + 2 * DQ_STAGES + 10) * 8 + 8 <= 256, "barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -959,67 +1012,66 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA
-      // One flattened sequence over this CTA's items: iteration g issues S/dP
-      // of step g, then the dQ product of step g - 1 (possibly of the
-      // previous item).
-      const uint32_t id_s = idesc(64, false);   // S = Q K^T, dP = dO V^T (N = 64 keys)
-      const uint32_t id_g = idesc(128, true);   // dQ += dS K (N = 128, B MN-major)
-      const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
-      bool ok = true;
-      int i_s = first, k_s = 0, j_s = 0, n_s = 0;
-      int i_p = first, k_p = 0, j_p = 0, n_p = 0;
-      if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); n_p = n_s; }
-      for (int g = 0; ok; ++g) {
-        const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
-        if (!s_left && !p_left) break;
-        if (s_left) {
-          const int st = g % DQ_STAGES, s = g & 1;
-          if (j_s == 0 && !mbar_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&kv_full[st], (g / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
-          // the dQ product of step g - 2 has read dS from this buffer
-          if (g >= 2 && !mbar_wait(&g_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
+    // ---------------------------------------------------------------- MMA
+    // One flattened sequence over this CTA's items: iteration g issues S/dP
+    // of step g, then the dQ product of step g - 1 (possibly of the previous
+    // item).  The whole warp runs it; one elected lane issues.
+    const uint32_t id_s = idesc(64, false);   // S = Q K^T, dP = dO V^T (N = 64 keys)
+    const uint32_t id_g = idesc(128, true);   // dQ += dS K (N = 128, B MN-major)
+    const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
+    bool ok = true;
+    int i_s = first, k_s = 0, j_s = 0, n_s = 0;
+    int i_p = first, k_p = 0, j_p = 0, n_p = 0;
+    if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); n_p = n_s; }
+    for (int g = 0; ok; ++g) {
+      const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
+      if (!s_left && !p_left) break;
+      if (s_left) {
+        const int st = g % DQ_STAGES, s = g & 1;
+        if (j_s == 0 && !warp_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(&kv_full[st], (g / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            tc_mma(tmem + s * 64, kdesc128(aQ, KV_T / 2, k), kdesc128(aK, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        for (int k = 0; k < 8; ++k)
+          tc_mma_w(tmem + s * 64, kdesc128(aQ, KV_T / 2, k), kdesc128(aK, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        // dP goes over the dS of step g - 2: the dQ product of step g - 2 has read it
+        if (g >= 2 && !warp_wait(&g_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            tc_mma(tmem + 128 + s * 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
-          tc_commit(&s_full[s]);
-          if (++j_s == n_s) {  // the item's last S/dP: Q and dO may be replaced
-            tc_commit(q_empty);
-            j_s = 0;
-            ++k_s;
-            i_s += stride;
-            if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); }
-          }
+        for (int k = 0; k < 8; ++k)
+          tc_mma_w(tmem + 128 + s * 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        tc_commit_w(&s_full[s]);
+        if (++j_s == n_s) {  // the item's last S/dP: Q and dO may be replaced
+          tc_commit_w(q_empty);
+          j_s = 0;
+          ++k_s;
+          i_s += stride;
+          if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); }
         }
-        if (p_left) {
-          const int gp = g - 1, s = gp & 1, st = gp % DQ_STAGES, ob = k_p & 1;
-          if (j_p == 0 && k_p >= 2 && !mbar_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t aK = smem_u32(sK + st * QT64);
-          // k-step k covers keys 16k..16k+15 (packed_col)
+      }
+      if (p_left) {
+        const int gp = g - 1, s = gp & 1, st = gp % DQ_STAGES, ob = k_p & 1;
+        if (j_p == 0 && k_p >= 2 && !warp_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sK + st * QT64);
+        // k-step k covers keys 16k..16k+15 (packed_col)
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_ts(tmem + 256 + ob * 128, tmem + 128 + s * 64 + packed_col(k),
-                      mndesc(aK, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&g_done[s]);
-          tc_commit(&kv_empty[st]);
-          if (++j_p == n_p) {  // the item's last product: dQ is complete
-            tc_commit(&o_full[ob]);
-            j_p = 0;
-            ++k_p;
-            i_p += stride;
-            if (i_p < total) { int qt, bh; item(i_p, qt, bh, n_p); }
-          }
+        for (int k = 0; k < 4; ++k)
+          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 64 + packed_col(k), mndesc(aK, QT64 / 2, k), id_g,
+                      (j_p > 0 || k > 0) ? 1u : 0u);
+        tc_commit_w(&g_done[s]);
+        tc_commit_w(&kv_empty[st]);
+        if (++j_p == n_p) {  // the item's last product: dQ is complete
+          tc_commit_w(&o_full[ob]);
+          j_p = 0;
+          ++k_p;
+          i_p += stride;
+          if (i_p < total) { int qt, bh; item(i_p, qt, bh, n_p); }
         }
       }
     }
@@ -1029,12 +1081,13 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float c = rsqrtf(128.f) * LOG2E;
+    uint8_t* stg = sStg + (warp - 2) * STG_WARP;
     bool ok = true;
     int g = 0;
     for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
       int qt, bh, n_it;
       item(i, qt, bh, n_it);
-      const int b = bh / H, h = bh % H, row_base = b * T;
+      const int b = bh / H, h = bh % H;
       const int qpos = qt * 128 + r;
       const bool valid = qpos < T;
       const float L = valid ? lse2[(long long)bh * T + qpos] : 0.f;  // log2 units
@@ -1074,13 +1127,37 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       if (!ok) break;
       if (!warp_wait(&o_full[ob], (k >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      constexpr int OC = 128 / NCG;  // dQ output columns per warp
-      bf16* qrow = dqkv + ((long long)row_base + (valid ? qpos : 0)) * 3 * a + h * 128 + grp * OC;
-      row_out<OC>(tmem + lane_off + 256 + ob * 128 + grp * OC, rsqrtf(128.f), qrow, valid);
+      // this warp's 32 rows x 64 columns of dQ (column group grp)
+      static_assert(NCG == 2, "two 64-column groups of dQ");
+      uint32_t o0[32], o1[32];
+      tmem_ld32_nowait(tmem + lane_off + 256 + ob * 128 + grp * 64, o0);
+      tmem_ld32_nowait(tmem + lane_off + 256 + ob * 128 + grp * 64 + 32, o1);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[ob]);  // this dQ buffer may be overwritten
+      // the previous item's store has read the staging block
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();
+      const float sc = rsqrtf(128.f);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t* src = jj < 4 ? o0 + 8 * jj : o1 + 8 * (jj - 4);
+        uint4 w;
+        w.x = pack_bf16x2_rn(__uint_as_float(src[0]) * sc, __uint_as_float(src[1]) * sc);
+        w.y = pack_bf16x2_rn(__uint_as_float(src[2]) * sc, __uint_as_float(src[3]) * sc);
+        w.z = pack_bf16x2_rn(__uint_as_float(src[4]) * sc, __uint_as_float(src[5]) * sc);
+        w.w = pack_bf16x2_rn(__uint_as_float(src[6]) * sc, __uint_as_float(src[7]) * sc);
+        *reinterpret_cast<uint4*>(stg + swz128(lane, jj)) = w;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0 && qt * 128 + q4 * 32 < T) {  // rows past T are clipped; a block wholly past it is skipped
+        tma_store_3d(&tmG, stg, h * 128 + grp * 64, qt * 128 + q4 * 32, b);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait0();  // this warp's stores are complete
   }
   tc_fence_before();
   __syncthreads();

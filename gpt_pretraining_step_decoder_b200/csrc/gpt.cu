@@ -1126,14 +1126,17 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
     TRY(make_tmap(&t128, qkv, 3 * a, N, 3 * a, 64, 128));
     TRY(make_tmap(&t64, qkv, 3 * a, N, 3 * a, 64, 64));
     TRY(make_tmap(&tdo, dout, a, N, a, 64, 64));
-    dim3 gk(cdiv(c.seq_len, 128), c.micro_batch * c.n_head);
-    bf16* g16 = reinterpret_cast<bf16*>(dqkv);
-    ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<gk, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st>>>(
-        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, m->err());
-    const long long dq_items = (long long)cdiv(c.seq_len, 128) * c.micro_batch * c.n_head;
-    const int dq_grid = dq_items < device_sms() ? (int)dq_items : device_sms();  // persistent
-    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<dq_grid, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
-        t128, t64, tdo, lse, Dv, g16, c.seq_len, c.n_head, c.micro_batch * c.n_head, m->err());
+    // dqkv as [B][T][3a] for the TMA stores of dQ, dK, dV: 32-row x 64-column
+    // blocks, rows past a sequence's end clipped
+    CUtensorMap tg;
+    TRY(make_tmap3(&tg, dqkv, 3 * a, c.seq_len, 3 * a, c.micro_batch, (long long)c.seq_len * 3 * a, 64, 32));
+    const int BH = c.micro_batch * c.n_head;
+    const long long items = (long long)cdiv(c.seq_len, 128) * BH;  // key tiles (dK, dV) = query tiles (dQ)
+    const int grid = items < device_sms() ? (int)items : device_sms();  // persistent
+    ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<grid, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st>>>(
+        t128, t64, tdo, tg, lse, Dv, c.seq_len, c.n_head, BH, m->err());
+    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<grid, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
+        t128, t64, tdo, tg, lse, Dv, c.seq_len, c.n_head, BH, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
   }
