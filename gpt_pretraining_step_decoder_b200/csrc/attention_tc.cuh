@@ -537,9 +537,6 @@ constexpr int NCG = 2;
 constexpr int CSP = 64 / NCG;
 constexpr int THREADS_B = 64 + 32 * 4 * NCG;
 constexpr int KV_T = 32768, QT64 = 16384;
-// TMEM column of the packed bf16 A operand for MMA k-step k (16 of the 64 step
-// columns): column group 16k / CSP, packed column (16k mod CSP) / 2 inside it
-__device__ __forceinline__ uint32_t packed_col(int k) { return (16 * k / CSP) * CSP + ((16 * k) % CSP) / 2; }
 
 constexpr int STG_WARP = 32 * 128;   // one compute warp's 32 x 64 bf16 block (128-byte rows)
 constexpr int DKDV_QS = 3;
@@ -562,14 +559,14 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint64_t* kv_free = kv_full + 2;            // 2 (per K/V buffer: the item's dK/dV copies have read it)
   uint64_t* q_full = kv_free + 2;             // DKDV_QS
   uint64_t* q_empty = q_full + DKDV_QS;       // DKDV_QS
-  uint64_t* s_full = q_empty + DKDV_QS;       // 2: S^T, dP^T of the buffer computed
-  uint64_t* p_full = s_full + 2;              // 2: P^T, dS^T of the buffer written (all compute warps)
-  uint64_t* dv_done = p_full + 2;             // 2: the dV product has read P^T of the buffer
-  uint64_t* dk_done = dv_done + 2;            // 2: the dK product has read dS^T of the buffer
-  uint64_t* acc_full = dk_done + 2;           // 1: the item's last dV/dK products are done
+  uint64_t* s_full = q_empty + DKDV_QS;       // 1: S^T, dP^T of the step computed
+  uint64_t* s_read = s_full + 1;              // 1: the compute warps have loaded them
+  uint64_t* p_full = s_read + 1;              // 2: P^T, dS^T of the packed buffer written
+  uint64_t* g_done = p_full + 2;              // 2: the dV, dK products have read the packed buffer
+  uint64_t* acc_full = g_done + 2;            // 1: the item's last dV/dK products are done
   uint64_t* acc_empty = acc_full + 1;         // 1: the compute warps have read dV/dK
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
-  static_assert((14 + 2 * DKDV_QS) * 8 + 8 <= 256, "barrier area");
+  static_assert((12 + 2 * DKDV_QS) * 8 + 8 <= 256, "barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -588,11 +585,11 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_free[s], 4 * NCG);
-      mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4 * NCG);  // one arrival per compute warp
-      mbar_init(&dv_done[s], 1);
-      mbar_init(&dk_done[s], 1);
+      mbar_init(&g_done[s], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 4 * NCG);
     for (int s = 0; s < DKDV_QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
@@ -611,8 +608,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // S^T buffers: cols 0, 64; dP^T buffers: 128, 192; dV: 256; dK: 384.  P^T / dS^T
-  // (bf16 pairs) overwrite the first CSP / 2 of each group's CSP S^T / dP^T columns.
+  // S^T: cols 0..63, dP^T: 64..127 (fp32, one step at a time); packed buffer b
+  // at 128 + 64 b: P^T in its first 32 columns, dS^T in the next 32 (bf16
+  // pairs, column group grp at 16 grp); dV: 256; dK: 384.
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -680,24 +678,21 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
       if (!s_left && !p_left) break;
       if (s_left) {
-        const int s = g & 1, st = g % DKDV_QS, kb = k_s & 1;
+        const int st = g % DKDV_QS, kb = k_s & 1;
         if (j_s == 0 && !warp_wait(&kv_full[kb], (k_s >> 1) & 1, abort_flag, err)) { ok = false; break; }
         if (!warp_wait(&q_full[st], (g / DKDV_QS) & 1, abort_flag, err)) { ok = false; break; }
-        // S^T goes over P^T of step g - 2: the dV product of step g - 2 has read it
-        if (g >= 2 && !warp_wait(&dv_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        // S^T, dP^T of step g overwrite step g - 1's: the compute warps have loaded those
+        if (g >= 1 && !warp_wait(s_read, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aK = smem_u32(sKV + kb * KV_BUF), aV = aK + KV_T;
         const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem + s * 64, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
-        // dP^T goes over dS^T of step g - 2: the dK product of step g - 2 has read it
-        if (g >= 2 && !warp_wait(&dk_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        tc_fence_after();
+          tc_mma_w(tmem, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem + 128 + s * 64, kdesc128(aV, KV_T / 2, k), kdesc128(aO, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
-        tc_commit_w(&s_full[s]);
+          tc_mma_w(tmem + 64, kdesc128(aV, KV_T / 2, k), kdesc128(aO, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        tc_commit_w(s_full);
         if (++j_s == n_s) {
           j_s = 0;
           ++k_s;
@@ -712,17 +707,15 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
-        // k-step k covers queries 16k..16k+15 (packed_col)
+        // k-step k covers queries 16k..16k+15: packed columns 8k..8k+7
+        const uint32_t pb = tmem + 128 + s * 64;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          tc_mma_ts_w(tmem + 256, tmem + s * 64 + packed_col(k), mndesc(aO, QT64 / 2, k), id_g,
-                      (j_p > 0 || k > 0) ? 1u : 0u);
-        tc_commit_w(&dv_done[s]);
+          tc_mma_ts_w(tmem + 256, pb + 8 * k, mndesc(aO, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          tc_mma_ts_w(tmem + 384, tmem + 128 + s * 64 + packed_col(k), mndesc(aQ, QT64 / 2, k), id_g,
-                      (j_p > 0 || k > 0) ? 1u : 0u);
-        tc_commit_w(&dk_done[s]);
+          tc_mma_ts_w(tmem + 384, pb + 32 + 8 * k, mndesc(aQ, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
+        tc_commit_w(&g_done[s]);
         tc_commit_w(&q_empty[st]);
         if (++j_p == n_p) {  // the item's last products: dV, dK are complete
           tc_commit_w(acc_full);
@@ -773,10 +766,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
             dv[e] = qbase + e < T ? D_bh[qbase + e] : 0.f;
           }
         }
-        if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(s_full, g & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t cs = tmem + lane_off + s * 64 + grp * CSP;   // this warp's S^T columns
-        const uint32_t cd = cs + 128;                                // and dP^T columns
+        const uint32_t cs = tmem + lane_off + grp * CSP;   // this warp's S^T columns
+        const uint32_t cd = cs + 64;                       // and dP^T columns
         float sv[CSP], dp[CSP];
         {
           uint32_t r0[CSP], r1[CSP];
@@ -786,6 +779,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
 #pragma unroll
           for (int e = 0; e < CSP; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
         }
+        // loaded: the next step's S^T, dP^T may overwrite these columns
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_read);
         // P^T[key, q] = exp2(s c - lse2_q) for key <= q < T; dS^T = P^T (dP^T - D_q).
         // Off the diagonal every key of the warp is <= every query of the group
         // (warp-uniform), so the causal test drops out.
@@ -805,15 +802,19 @@ __global__ void __launch_bounds__(THREADS_B, 1)
             dp[e] = p * (dp[e] - dv[e]);
           }
         }
-        // bf16 pairs over the columns just read (this warp's own lanes and columns)
+        // bf16 pairs into packed buffer s (this warp's own lanes and columns),
+        // once the dV, dK products of step g - 2 have read it
         uint32_t pw[CSP / 2], dw[CSP / 2];
 #pragma unroll
         for (int jj = 0; jj < CSP / 2; ++jj) {
           pw[jj] = pack_bf16x2_rn(sv[2 * jj], sv[2 * jj + 1]);
           dw[jj] = pack_bf16x2_int(dp[2 * jj], dp[2 * jj + 1]);
         }
-        tmem_stw<CSP / 2>(cs, pw);
-        tmem_stw<CSP / 2>(cd, dw);
+        if (g >= 2 && !warp_wait(&g_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t pbw = tmem + lane_off + 128 + s * 64 + grp * (CSP / 2);
+        tmem_stw<CSP / 2>(pbw, pw);
+        tmem_stw<CSP / 2>(pbw + 32, dw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -922,9 +923,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   uint64_t* q_empty = q_full + 1;               // 1 (the item's last S/dP have read Q and dO)
   uint64_t* kv_full = q_empty + 1;              // DQ_STAGES
   uint64_t* kv_empty = kv_full + DQ_STAGES;     // DQ_STAGES
-  uint64_t* s_full = kv_empty + DQ_STAGES;      // 2: S, dP of the buffer computed
-  uint64_t* p_full = s_full + 2;                // 2: dS of the buffer written (all compute warps)
-  uint64_t* g_done = p_full + 2;                // 2: the dQ product has read the buffer
+  uint64_t* s_full = kv_empty + DQ_STAGES;      // 1: S, dP of the step computed
+  uint64_t* s_read = s_full + 1;                // 1: the compute warps have loaded them
+  uint64_t* p_full = s_read + 1;                // 2: dS of the packed buffer written (all compute warps)
+  uint64_t* g_done = p_full + 2;                // 2: the dQ product has read the packed buffer
   uint64_t* o_full = g_done + 2;                // 2 (per dQ buffer: the item's last product is done)
   uint64_t* o_empty = o_full + 2;               // 2 (per dQ buffer: the compute warps have read it)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
@@ -947,8 +949,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 4 * NCG);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4 * NCG);  // one arrival per compute warp
       mbar_init(&g_done[s], 1);
       mbar_init(&o_full[s], 1);
@@ -966,8 +969,9 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // S: 0, 64; dP: 128, 192 (dS as bf16 pairs over the first CSP / 2 of each
-  // group's CSP dP columns); dQ: 256 and 384 (alternating per item)
+  // S: cols 0..63, dP: 64..127 (fp32, one step at a time); packed dS buffer b
+  // at 128 + 32 b (bf16 pairs, column group grp at 16 grp); dQ: 256 and 384
+  // (alternating per item)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -1027,21 +1031,20 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
       if (!s_left && !p_left) break;
       if (s_left) {
-        const int st = g % DQ_STAGES, s = g & 1;
+        const int st = g % DQ_STAGES;
         if (j_s == 0 && !warp_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
         if (!warp_wait(&kv_full[st], (g / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
+        // S, dP of step g overwrite step g - 1's: the compute warps have loaded those
+        if (g >= 1 && !warp_wait(s_read, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem + s * 64, kdesc128(aQ, KV_T / 2, k), kdesc128(aK, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
-        // dP goes over the dS of step g - 2: the dQ product of step g - 2 has read it
-        if (g >= 2 && !warp_wait(&g_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        tc_fence_after();
+          tc_mma_w(tmem, kdesc128(aQ, KV_T / 2, k), kdesc128(aK, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem + 128 + s * 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
-        tc_commit_w(&s_full[s]);
+          tc_mma_w(tmem + 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        tc_commit_w(s_full);
         if (++j_s == n_s) {  // the item's last S/dP: Q and dO may be replaced
           tc_commit_w(q_empty);
           j_s = 0;
@@ -1059,10 +1062,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aK = smem_u32(sK + st * QT64);
-        // k-step k covers keys 16k..16k+15 (packed_col)
+        // k-step k covers keys 16k..16k+15: packed columns 8k..8k+7
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 64 + packed_col(k), mndesc(aK, QT64 / 2, k), id_g,
+          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 32 + 8 * k, mndesc(aK, QT64 / 2, k), id_g,
                       (j_p > 0 || k > 0) ? 1u : 0u);
         tc_commit_w(&g_done[s]);
         tc_commit_w(&kv_empty[st]);
@@ -1095,18 +1098,21 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       const int ob = k & 1;
       for (int j = 0; j < n_it; ++j, ++g) {
         const int s = g & 1;
-        if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(s_full, g & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t cd = tmem + lane_off + 128 + s * 64 + grp * CSP;  // this warp's dP columns
         float sv[CSP], dp[CSP];
         {
           uint32_t r0[CSP], r1[CSP];
-          tmem_ldw<CSP>(tmem + lane_off + s * 64 + grp * CSP, r0);
-          tmem_ldw<CSP>(cd, r1);
+          tmem_ldw<CSP>(tmem + lane_off + grp * CSP, r0);        // this warp's S columns
+          tmem_ldw<CSP>(tmem + lane_off + 64 + grp * CSP, r1);   // and dP columns
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < CSP; ++e) { sv[e] = __uint_as_float(r0[e]); dp[e] = __uint_as_float(r1[e]); }
         }
+        // loaded: the next step's S, dP may overwrite these columns
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_read);
         const int kbase = j * 64 + grp * CSP;
 #pragma unroll
         for (int e = 0; e < CSP; ++e) {
@@ -1114,11 +1120,14 @@ __global__ void __launch_bounds__(THREADS_B, 1)
           const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
           dp[e] = p * (dp[e] - Dq);
         }
-        // dS as bf16 pairs over the dP columns just read (this warp's own lanes and columns)
+        // dS as bf16 pairs into packed buffer s (this warp's own lanes and
+        // columns), once the dQ product of step g - 2 has read it
         uint32_t dw[CSP / 2];
 #pragma unroll
         for (int jj = 0; jj < CSP / 2; ++jj) dw[jj] = pack_bf16x2_int(dp[2 * jj], dp[2 * jj + 1]);
-        tmem_stw<CSP / 2>(cd, dw);
+        if (g >= 2 && !warp_wait(&g_done[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        tmem_stw<CSP / 2>(tmem + lane_off + 128 + s * 32 + grp * (CSP / 2), dw);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
