@@ -142,28 +142,48 @@ __device__ __forceinline__ void fwd_item(int i, int n_qt, int BH, int& qt, int& 
   bh = i % BH;
 }
 
+// The forward on tcgen05, persistent: one CTA per SM over the (query tile,
+// sequence, head) items heaviest first.  Warp 0: TMA (lane 0 Q and the K
+// ring, lane 1 the V ring); warp 1: MMA, issued as a whole warp (one elected
+// lane); warps 2..5: softmax, one per TMEM lane quarter (32 query rows x 128
+// keys each).
+// TMEM: S (fp32, one step at a time) in columns 0..127; the probabilities P
+// as bf16 pairs in packed buffer b at 128 + 64 b (the A operand of the PV
+// product); O in 256 + 128 ob, alternating per item.  Step g + 1's scores wait
+// only until the softmax warps have loaded step g's, and the PV product of
+// step g only for step g's probabilities, so the score product of one step
+// and the PV product of the previous one keep the tensor pipe busy together.
+// The item's O leaves through shared memory: each softmax warp writes its 32
+// rows as bf16 (two 64-column blocks in the 128-byte swizzle) and stores them
+// with TMA copies (rows past the sequence end clipped by the map's T extent).
+constexpr int STG_BYTES_FWD = 4 * 2 * 32 * 128;   // 4 softmax warps x two 32 x 64 bf16 blocks
+constexpr int SMEM_BYTES_TC = SMEM_BYTES + STG_BYTES_FWD;
+
 __global__ void __launch_bounds__(THREADS, 1)
     fa_tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constant__ CUtensorMap tmV,
-                     bf16* __restrict__ out, float* __restrict__ lse_out, int T, int H, int BH, unsigned* err) {
+                     const __grid_constant__ CUtensorMap tmO, float* __restrict__ lse_out, int T, int H, int BH,
+                     unsigned* err) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + TILE_BYTES;            // [2 stages]
   uint8_t* sV = sK + 2 * TILE_BYTES;        // [2 stages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * TILE_BYTES);
+  uint8_t* sStg = sV + 2 * TILE_BYTES;      // [4 softmax warps][2 blocks]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + STG_BYTES_FWD);
   uint64_t* q_full = bars;                  // 1
   uint64_t* q_empty = bars + 1;             // 1 (the item's last S has read Q)
   uint64_t* k_full = bars + 2;              // 2
   uint64_t* k_empty = bars + 4;             // 2 (S done with K)
   uint64_t* v_full = bars + 6;              // 2
   uint64_t* v_empty = bars + 8;             // 2 (PV done with V)
-  uint64_t* s_full = bars + 10;             // 2
-  uint64_t* p_full = bars + 14;             // 2 (P written over the S buffer)
-  uint64_t* p_free = bars + 16;             // 2 (PV done: S/P buffer free, O updated)
-  uint64_t* o_full = bars + 18;             // 2 (per O buffer: the item's last PV is done)
-  uint64_t* o_empty = bars + 20;            // 2 (per O buffer: the softmax warps have read O)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* s_full = bars + 10;             // 1: S of the step computed
+  uint64_t* s_read = bars + 11;             // 1: the softmax warps have loaded it
+  uint64_t* p_full = bars + 12;             // 2 (per packed buffer: P written)
+  uint64_t* p_free = bars + 14;             // 2 (per packed buffer: PV done with it, O updated)
+  uint64_t* o_full = bars + 16;             // 2 (per O buffer: the item's last PV is done)
+  uint64_t* o_empty = bars + 18;            // 2 (per O buffer: the softmax warps have read it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,13 +196,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 4);      // one arrival per softmax warp
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);    // one arrival per softmax warp
+      mbar_init(&p_full[s], 4);
       mbar_init(&p_free[s], 1);
       mbar_init(&o_full[s], 1);
       mbar_init(&o_empty[s], 4);
@@ -199,8 +220,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // S0: cols 0..127, S1: 128..255 (P as bf16 pairs over the first 64 columns
-  // of its S buffer), O0: 256..383, O1: 384..511
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -256,72 +275,70 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA
-      // One flattened sequence of steps over this CTA's items: iteration g
-      // issues S of step g, then PV of step g - 1 (which may belong to the
-      // previous item), so the next item's first S overlaps the last softmax.
-      // S = Q K^T: A = Q (K-major), B = K (K-major), N = 128
-      const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
-                               ((uint32_t)(128 >> 4) << 24);
-      // O += P V: A = P (TMEM), B = V (MN-major), N = 128
-      const uint32_t idesc_o = idesc_s | (1u << 16);
-      const uint32_t aQ = smem_u32(sQ);
-      bool ok = true;
-      // S cursor (item index i_s, its k-th position k_s, step j_s) and PV cursor
-      int i_s = first, k_s = 0, j_s = 0, nkv_s = 0;
-      int i_p = first, k_p = 0, j_p = 0, nkv_p = 0;
-      if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = nkv_p = qt + 1; }
-      for (int g = 0; ok; ++g) {
-        const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
-        if (!s_left && !p_left) break;
-        if (s_left) {
-          const int s = g & 1;
-          if (j_s == 0 && !mbar_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&k_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          // the PV product of step g - 2 has read P from this buffer
-          if (g >= 2 && !mbar_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t aK = smem_u32(sK + s * TILE_BYTES);
+    // ---------------------------------------------------------------- MMA
+    // One flattened sequence of steps over this CTA's items: iteration g
+    // issues S of step g, then PV of step g - 1 (which may belong to the
+    // previous item), so the next item's first S overlaps the last softmax.
+    // S = Q K^T: A = Q (K-major), B = K (K-major), N = 128
+    const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);
+    // O += P V: A = P (TMEM), B = V (MN-major), N = 128
+    const uint32_t idesc_o = idesc_s | (1u << 16);
+    const uint32_t aQ = smem_u32(sQ);
+    bool ok = true;
+    // S cursor (item index i_s, its k-th position k_s, step j_s) and PV cursor
+    int i_s = first, k_s = 0, j_s = 0, nkv_s = 0;
+    int i_p = first, k_p = 0, j_p = 0, nkv_p = 0;
+    if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = nkv_p = qt + 1; }
+    for (int g = 0; ok; ++g) {
+      const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
+      if (!s_left && !p_left) break;
+      if (s_left) {
+        const int s = g & 1;
+        if (j_s == 0 && !warp_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(&k_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        // S of step g overwrites step g - 1's: the softmax warps have loaded it
+        if (g >= 1 && !warp_wait(s_read, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aK = smem_u32(sK + s * TILE_BYTES);
 #pragma unroll
-          for (int k = 0; k < HD / 16; ++k)
-            tc_mma(tmem + s * 128, kmaj_desc(aQ, k), kmaj_desc(aK, k), idesc_s, k > 0 ? 1u : 0u);
-          tc_commit(&s_full[s]);
-          tc_commit(&k_empty[s]);
-          if (++j_s == nkv_s) {  // the item's last S: Q may be replaced
-            tc_commit(q_empty);
-            j_s = 0;
-            ++k_s;
-            i_s += stride;
-            if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = qt + 1; }
-          }
+        for (int k = 0; k < HD / 16; ++k)
+          tc_mma_w(tmem, kmaj_desc(aQ, k), kmaj_desc(aK, k), idesc_s, k > 0 ? 1u : 0u);
+        tc_commit_w(s_full);
+        tc_commit_w(&k_empty[s]);
+        if (++j_s == nkv_s) {  // the item's last S: Q may be replaced
+          tc_commit_w(q_empty);
+          j_s = 0;
+          ++k_s;
+          i_s += stride;
+          if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = qt + 1; }
         }
-        if (p_left) {
-          const int gp = g - 1, s = gp & 1, ob = k_p & 1;
-          // the first PV of an item overwrites its O buffer: the softmax warps
-          // must have read that buffer for the item two positions back
-          if (j_p == 0 && k_p >= 2 && !mbar_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          if (!mbar_wait(&v_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t aV = smem_u32(sV + s * TILE_BYTES);
-          // k-step k covers keys 16k..16k+15: packed P columns 8k..8k+7
+      }
+      if (p_left) {
+        const int gp = g - 1, s = gp & 1, ob = k_p & 1;
+        // the first PV of an item overwrites its O buffer: the softmax warps
+        // must have read that buffer for the item two positions back
+        if (j_p == 0 && k_p >= 2 && !warp_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(&v_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aV = smem_u32(sV + s * TILE_BYTES);
+        // k-step k covers keys 16k..16k+15: packed P columns 8k..8k+7
 #pragma unroll
-          for (int k = 0; k < BKV / 16; ++k)
-            tc_mma_ts(tmem + 256 + ob * 128, tmem + s * 128 + k * 8, mnmaj_desc(aV, k), idesc_o,
+        for (int k = 0; k < BKV / 16; ++k)
+          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 64 + k * 8, mnmaj_desc(aV, k), idesc_o,
                       (j_p > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&p_free[s]);
-          tc_commit(&v_empty[s]);
-          if (++j_p == nkv_p) {  // the item's last PV: O is complete
-            tc_commit(&o_full[ob]);
-            j_p = 0;
-            ++k_p;
-            i_p += stride;
-            if (i_p < total) { int qt, bh; fwd_item(i_p, n_qt, BH, qt, bh); nkv_p = qt + 1; }
-          }
+        tc_commit_w(&p_free[s]);
+        tc_commit_w(&v_empty[s]);
+        if (++j_p == nkv_p) {  // the item's last PV: O is complete
+          tc_commit_w(&o_full[ob]);
+          j_p = 0;
+          ++k_p;
+          i_p += stride;
+          if (i_p < total) { int qt, bh; fwd_item(i_p, n_qt, BH, qt, bh); nkv_p = qt + 1; }
         }
       }
     }
@@ -331,23 +348,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int r = q * 32 + lane;               // row within the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float c = rsqrtf((float)HD) * LOG2E;
+    uint8_t* stg = sStg + (warp - 2) * (2 * 32 * 128);
     bool ok = true;
     int g = 0;  // global step
     for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
       int qt, bh;
       fwd_item(i, n_qt, BH, qt, bh);
-      const int b = bh / H, h = bh % H, row_base = b * T, n_kv = qt + 1;
+      const int b = bh / H, h = bh % H, n_kv = qt + 1;
       const int qpos = qt * BQ + r;              // query position in the sequence
       const int ob = k & 1;
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n_kv; ++j, ++g) {
         const int s = g & 1;
-        if (!warp_wait(&s_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(s_full, g & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         float sv[128];
         {
           uint32_t r0[32], r1[32], r2[32], r3[32];
-          const uint32_t base = tmem + lane_off + s * 128;
+          const uint32_t base = tmem + lane_off;
           tmem_ld32_nowait(base, r0);
           tmem_ld32_nowait(base + 32, r1);
           tmem_ld32_nowait(base + 64, r2);
@@ -361,6 +379,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             sv[96 + ii] = __uint_as_float(r3[ii]);
           }
         }
+        // loaded: the next step's S may overwrite these columns
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_read);
         const int k0 = j * BKV;
         if (k0 + BKV - 1 > qpos) {  // causal mask on the diagonal tile
 #pragma unroll
@@ -401,11 +423,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           l *= alpha;
           m_use = m_new;
         }
-        // P = exp2(s - m_use) as bf16 pairs over the first 64 columns of this
-        // row's S buffer (read above), the A operand of the PV product
+        // packed buffer s was last read by the PV product of step g - 2
+        if (g >= 2 && !warp_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        // P = exp2(s - m_use) as bf16 pairs in packed buffer s, the A operand
+        // of the PV product
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial sums
         const float nm = -m_use;
-        const uint32_t sbase = tmem + lane_off + s * 128;
+        const uint32_t pbase = tmem + lane_off + 128 + s * 64;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 32 keys = 16 packed columns
           uint32_t w[16];
@@ -417,7 +442,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             ps[(2 * e + 1) & 7] += p1;
             w[e] = pack_bf16x2_int(p0, p1);
           }
-          tmem_st16(sbase + ch * 16, w);
+          tmem_st16(pbase + ch * 16, w);
         }
         l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         tmem_wait_st();
@@ -429,33 +454,43 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------------------ item epilogue
       if (!warp_wait(&o_full[ob], (k >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
+      if (qpos < T) lse_out[(long long)bh * T + qpos] = m_use + log2f(l);  // log2 units
+      // the previous item's stores have read the staging blocks
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();
       const float inv = 1.f / l;
       const uint32_t obase = tmem + lane_off + 256 + ob * 128;
-      bf16* orow = out + ((long long)row_base + qpos) * a + h * HD;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t o[32];
-        tmem_ld32_nowait(obase + cc * 32, o);
+      for (int hb = 0; hb < 2; ++hb) {   // two 64-column halves, one staging block each
+        uint32_t o0[32], o1[32];
+        tmem_ld32_nowait(obase + hb * 64, o0);
+        tmem_ld32_nowait(obase + hb * 64 + 32, o1);
         tmem_wait_ld();
-        if (qpos < T) {
+        if (hb == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty[ob]);  // this O buffer may be overwritten
+        }
 #pragma unroll
-          for (int ii = 0; ii < 32; ii += 8) {
-            uint4 w;
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(__uint_as_float(o[ii]) * inv, __uint_as_float(o[ii + 1]) * inv);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(__uint_as_float(o[ii + 2]) * inv, __uint_as_float(o[ii + 3]) * inv);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[ii + 4]) * inv, __uint_as_float(o[ii + 5]) * inv);
-            __nv_bfloat162 b3 = __floats2bfloat162_rn(__uint_as_float(o[ii + 6]) * inv, __uint_as_float(o[ii + 7]) * inv);
-            w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
-            w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
-            *reinterpret_cast<uint4*>(orow + cc * 32 + ii) = w;
-          }
+        for (int jj = 0; jj < 8; ++jj) {   // 16-byte chunk jj of the block: columns 8jj..8jj+7
+          const uint32_t* src = jj < 4 ? o0 + 8 * jj : o1 + 8 * (jj - 4);
+          uint4 wv;
+          wv.x = pack_bf16x2_rn(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+          wv.y = pack_bf16x2_rn(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+          wv.z = pack_bf16x2_rn(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+          wv.w = pack_bf16x2_rn(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+          *reinterpret_cast<uint4*>(stg + hb * 4096 + swz128(lane, jj)) = wv;
         }
       }
-      if (qpos < T) lse_out[(long long)bh * T + qpos] = m_use + log2f(l);  // log2 units
-      tc_fence_before();
+      fence_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[ob]);  // this O buffer may be overwritten
+      if (lane == 0 && qt * BQ + q * 32 < T) {  // rows past T are clipped; a block wholly past it is skipped
+        tma_store_3d(&tmO, stg, h * HD, qt * BQ + q * 32, b);
+        tma_store_3d(&tmO, stg + 4096, h * HD + 64, qt * BQ + q * 32, b);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait0();  // this warp's stores are complete
   }
   tc_fence_before();
   __syncthreads();

@@ -1080,7 +1080,7 @@ static int attention_fwd(gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
     static bool attr = false;
     if (!attr) {
       CUDA_TRY(cudaFuncSetAttribute(fatc::fa_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fatc::SMEM_BYTES));
+                                    fatc::SMEM_BYTES_TC));
       attr = true;
     }
     const long long a = (long long)c.n_head * c.head_dim, ntok = (long long)c.micro_batch * c.seq_len;
@@ -1090,8 +1090,12 @@ static int attention_fwd(gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
     // persistent: one CTA per SM (or per item when there are fewer)
     const long long items = (long long)cdiv(c.seq_len, fatc::BQ) * c.micro_batch * c.n_head;
     const int grid = items < device_sms() ? (int)items : device_sms();
-    ++g_launches; fatc::fa_tc_fwd_kernel<<<grid, fatc::THREADS, fatc::SMEM_BYTES, m->st>>>(
-        tqk, tv, reinterpret_cast<bf16*>(o), lse, c.seq_len, c.n_head, c.micro_batch * c.n_head, m->err());
+    // the output as [B][T][a] for the TMA stores of O: 32-row x 64-column
+    // blocks, rows past a sequence's end clipped
+    CUtensorMap to;
+    TRY(make_tmap3(&to, o, a, c.seq_len, a, c.micro_batch, (long long)c.seq_len * a, 64, 32));
+    ++g_launches; fatc::fa_tc_fwd_kernel<<<grid, fatc::THREADS, fatc::SMEM_BYTES_TC, m->st>>>(
+        tqk, tv, to, lse, c.seq_len, c.n_head, c.micro_batch * c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
   }
