@@ -50,6 +50,43 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// two fp32 lanes per instruction (sm_100 packed f32x2 arithmetic):
+// (y0, y1) = (x0, x1) * c + d
+__device__ __forceinline__ void fma2(float& y0, float& y1, float x0, float x1, float c, float d) {
+  asm("{\n\t.reg .b64 a, b, e, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 e, {%5, %5};\n\t"
+      "fma.rn.f32x2 r, a, b, e;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(c), "f"(d));
+}
+// (y0, y1) += (x0, x1)
+__device__ __forceinline__ void add2(float& y0, float& y1, float x0, float x1) {
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 a, a, b;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(y0), "+f"(y1)
+      : "f"(x0), "f"(x1));
+}
+// (y0, y1) = (x0, x1) * c + (d0, d1)
+__device__ __forceinline__ void fma2v(float& y0, float& y1, float x0, float x1, float c, float d0, float d1) {
+  asm("{\n\t.reg .b64 a, b, e, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 e, {%5, %6};\n\t"
+      "fma.rn.f32x2 r, a, b, e;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(c), "f"(d0), "f"(d1));
+}
+// (y0, y1) = (p0, p1) * ((x0, x1) - (d0, d1))
+__device__ __forceinline__ void mulsub2(float& y0, float& y1, float p0, float p1, float x0, float x1, float d0,
+                                        float d1) {
+  asm("{\n\t.reg .b64 a, b, q;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 q, {%6, %7};\n\t"
+      "sub.rn.f32x2 a, a, b;\n\tmul.rn.f32x2 a, a, q;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(d0), "f"(d1), "f"(p0), "f"(p1));
+}
+// max of three (one sm_100 instruction)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
@@ -393,9 +430,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         // independent partial maxima so the reduction is not one long chain
         float pm[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) pm[u] = sv[u];
+        for (int u = 0; u < 8; ++u) pm[u] = fmaxf(sv[u], sv[8 + u]);
 #pragma unroll
-        for (int ii = 8; ii < 128; ++ii) pm[ii & 7] = fmaxf(pm[ii & 7], sv[ii]);
+        for (int ii = 16; ii < 128; ii += 16)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) pm[u] = fmax3(pm[u], sv[ii + u], sv[ii + 8 + u]);
         const float mx = c * fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                                    fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         if (j == 0) {
@@ -427,7 +466,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (g >= 2 && !warp_wait(&p_free[s], ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         // P = exp2(s - m_use) as bf16 pairs in packed buffer s, the A operand
-        // of the PV product
+        // of the PV product (arguments and partial sums two lanes at a time)
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial sums
         const float nm = -m_use;
         const uint32_t pbase = tmem + lane_off + 128 + s * 64;
@@ -436,10 +475,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(sv[ch * 32 + 2 * e], c, nm));
-            const float p1 = fast_exp2(fmaf(sv[ch * 32 + 2 * e + 1], c, nm));
-            ps[(2 * e) & 7] += p0;
-            ps[(2 * e + 1) & 7] += p1;
+            float x0, x1;
+            fma2(x0, x1, sv[ch * 32 + 2 * e], sv[ch * 32 + 2 * e + 1], c, nm);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            add2(ps[2 * (e & 3)], ps[2 * (e & 3) + 1], p0, p1);
             w[e] = pack_bf16x2_int(p0, p1);
           }
           tmem_st16(pbase + ch * 16, w);
@@ -528,6 +567,9 @@ using fatc::pack_bf16x2_int;
 using fatc::pack_bf16x2_rn;
 using fatc::tmem_ldw;
 using fatc::tmem_stw;
+using fatc::fma2;
+using fatc::fma2v;
+using fatc::mulsub2;
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns
@@ -823,10 +865,13 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         // (warp-uniform), so the causal test drops out.
         if (fullc && warp_key_max <= qbase) {
 #pragma unroll
-          for (int e = 0; e < CSP; ++e) {
-            const float p = fast_exp2(fmaf(sv[e], c, -lv[e]));
-            sv[e] = p;
-            dp[e] = p * (dp[e] - dv[e]);
+          for (int e = 0; e < CSP; e += 2) {   // two lanes of fp32 per instruction
+            float x0, x1;
+            fma2v(x0, x1, sv[e], sv[e + 1], c, -lv[e], -lv[e + 1]);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            sv[e] = p0;
+            sv[e + 1] = p1;
+            mulsub2(dp[e], dp[e + 1], p0, p1, dp[e], dp[e + 1], dv[e], dv[e + 1]);
           }
         } else {
 #pragma unroll
@@ -1150,10 +1195,12 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         if (lane == 0) mbar_arrive(s_read);
         const int kbase = j * 64 + grp * CSP;
 #pragma unroll
-        for (int e = 0; e < CSP; ++e) {
-          const bool live = valid && (kbase + e <= qpos);
-          const float p = live ? fast_exp2(fmaf(sv[e], c, -L)) : 0.f;
-          dp[e] = p * (dp[e] - Dq);
+        for (int e = 0; e < CSP; e += 2) {   // two lanes of fp32 per instruction
+          float x0, x1;
+          fma2(x0, x1, sv[e], sv[e + 1], c, -L);
+          const float p0 = (valid && kbase + e <= qpos) ? fast_exp2(x0) : 0.f;
+          const float p1 = (valid && kbase + e + 1 <= qpos) ? fast_exp2(x1) : 0.f;
+          mulsub2(dp[e], dp[e + 1], p0, p1, dp[e], dp[e + 1], Dq, Dq);
         }
         // dS as bf16 pairs into packed buffer s (this warp's own lanes and
         // columns), once the dQ product of step g - 2 has read it
