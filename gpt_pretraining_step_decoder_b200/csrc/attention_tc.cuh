@@ -50,36 +50,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// two fp32 lanes per instruction (sm_100 packed f32x2 arithmetic):
-// (y0, y1) = (x0, x1) * c + d
-__device__ __forceinline__ void fma2(float& y0, float& y1, float x0, float x1, float c, float d) {
-  asm("{\n\t.reg .b64 a, b, e, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 e, {%5, %5};\n\t"
-      "fma.rn.f32x2 r, a, b, e;\n\tmov.b64 {%0, %1}, r;\n\t}"
-      : "=f"(y0), "=f"(y1)
-      : "f"(x0), "f"(x1), "f"(c), "f"(d));
-}
-// (y0, y1) += (x0, x1)
-__device__ __forceinline__ void add2(float& y0, float& y1, float x0, float x1) {
-  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
-      "add.rn.f32x2 a, a, b;\n\tmov.b64 {%0, %1}, a;\n\t}"
-      : "+f"(y0), "+f"(y1)
-      : "f"(x0), "f"(x1));
-}
-// (y0, y1) = (x0, x1) * c + (d0, d1)
-__device__ __forceinline__ void fma2v(float& y0, float& y1, float x0, float x1, float c, float d0, float d1) {
-  asm("{\n\t.reg .b64 a, b, e, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 e, {%5, %6};\n\t"
-      "fma.rn.f32x2 r, a, b, e;\n\tmov.b64 {%0, %1}, r;\n\t}"
-      : "=f"(y0), "=f"(y1)
-      : "f"(x0), "f"(x1), "f"(c), "f"(d0), "f"(d1));
-}
-// (y0, y1) = (p0, p1) * ((x0, x1) - (d0, d1))
-__device__ __forceinline__ void mulsub2(float& y0, float& y1, float p0, float p1, float x0, float x1, float d0,
-                                        float d1) {
-  asm("{\n\t.reg .b64 a, b, q;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 q, {%6, %7};\n\t"
-      "sub.rn.f32x2 a, a, b;\n\tmul.rn.f32x2 a, a, q;\n\tmov.b64 {%0, %1}, a;\n\t}"
-      : "=f"(y0), "=f"(y1)
-      : "f"(x0), "f"(x1), "f"(d0), "f"(d1), "f"(p0), "f"(p1));
-}
 // max of three (one sm_100 instruction)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -567,9 +537,6 @@ using fatc::pack_bf16x2_int;
 using fatc::pack_bf16x2_rn;
 using fatc::tmem_ldw;
 using fatc::tmem_stw;
-using fatc::fma2;
-using fatc::fma2v;
-using fatc::mulsub2;
 constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns

@@ -464,6 +464,36 @@ __device__ __forceinline__ void tile_coords(int mn, const Params& p, int& mt, in
 }
 
 // byte offset of 16-byte chunk j of row r in a 128-byte-swizzled block
+// two fp32 lanes per instruction (sm_100 packed f32x2 arithmetic):
+// (y0, y1) = (x0, x1) * c + d
+__device__ __forceinline__ void fma2(float& y0, float& y1, float x0, float x1, float c, float d) {
+  asm("{\n\t.reg .b64 a, b, e, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 e, {%5, %5};\n\t"
+      "fma.rn.f32x2 r, a, b, e;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(c), "f"(d));
+}
+// (y0, y1) += (x0, x1)
+__device__ __forceinline__ void add2(float& y0, float& y1, float x0, float x1) {
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 a, a, b;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(y0), "+f"(y1)
+      : "f"(x0), "f"(x1));
+}
+// (y0, y1) = (x0, x1) * c + (d0, d1)
+__device__ __forceinline__ void fma2v(float& y0, float& y1, float x0, float x1, float c, float d0, float d1) {
+  asm("{\n\t.reg .b64 a, b, e, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 e, {%5, %6};\n\t"
+      "fma.rn.f32x2 r, a, b, e;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(c), "f"(d0), "f"(d1));
+}
+// (y0, y1) = (p0, p1) * ((x0, x1) - (d0, d1))
+__device__ __forceinline__ void mulsub2(float& y0, float& y1, float p0, float p1, float x0, float x1, float d0,
+                                        float d1) {
+  asm("{\n\t.reg .b64 a, b, q;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 q, {%6, %7};\n\t"
+      "sub.rn.f32x2 a, a, b;\n\tmul.rn.f32x2 a, a, q;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(x0), "f"(x1), "f"(d0), "f"(d1), "f"(p0), "f"(p1));
+}
 __device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
 template <int BN, int KM, typename act_t, int CG, int F8 = 0, bool B3 = false>
@@ -815,16 +845,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if constexpr (KM == K_LOGITS) {
           const int nv = min(64, p.N - nc);
           const int yo = ytgt - nc;  // target column within this block, if here
-          float zt = 0.f;
+          if (yo >= 0 && yo < 64) {  // rare: this row's target logit
+            float zt = 0.f;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float z = v[i];
-            zt = (i == yo) ? z : zt;
-            const float pr = (i < nv) ? __expf(z - rmax) : 0.f;
-            rsum += pr;
-            v[i] = pr;
+            for (int i = 0; i < 64; ++i) zt = (i == yo) ? v[i] : zt;
+            e.ztgt[m] = zt;
           }
-          if (yo >= 0 && yo < 64) e.ztgt[m] = zt;
+          // numerators exp(z - max) = 2^(z log2 e - max log2 e), the arguments
+          // and the row sum (8 independent partial sums) two lanes at a time
+          constexpr float L2E = 1.4426950408889634f;
+          const float nb = -rmax * L2E;
+          float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          if (nv == 64) {  // warp-uniform: all but the vocabulary's last block
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              float x0, x1;
+              fma2(x0, x1, v[i], v[i + 1], L2E, nb);
+              float p0, p1;
+              asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p0) : "f"(x0));
+              asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p1) : "f"(x1));
+              add2(ps[(i >> 1) & 7], ps[((i >> 1) + 4) & 7], p0, p1);
+              v[i] = p0;
+              v[i + 1] = p1;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              const float pr = (i < nv) ? __expf(v[i] - rmax) : 0.f;
+              ps[i & 7] += pr;
+              v[i] = pr;
+            }
+          }
+          rsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         } else if constexpr (KM == K_RELU2) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) { const float r = fmaxf(v[i], 0.f); v[i] = r * r; }
