@@ -579,7 +579,8 @@ __device__ __forceinline__ uint32_t idesc(int n, bool b_mn) {
 // once those copies have read it.
 constexpr int NCG = 2;
 constexpr int CSP = 64 / NCG;
-constexpr int THREADS_B = 64 + 32 * 4 * NCG;
+constexpr int MMA_G_WARP = 2 + 4 * NCG;          // the warp that issues the gradient products
+constexpr int THREADS_B = 64 + 32 * 4 * NCG + 32;
 constexpr int KV_T = 32768, QT64 = 16384;
 
 constexpr int STG_WARP = 32 * 128;   // one compute warp's 32 x 64 bf16 block (128-byte rows)
@@ -636,7 +637,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
     mbar_init(s_read, 4 * NCG);
     for (int s = 0; s < DKDV_QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&q_empty[s], 2);   // released by both MMA warps
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 4 * NCG);
@@ -708,22 +709,21 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA
-    // One flattened sequence over this CTA's items: iteration g issues S^T,
-    // dP^T of step g, then dV, dK of step g - 1 (possibly of the previous
-    // item).  The whole warp runs it; one elected lane issues.
+    // ---------------------------------------------------------------- MMA: scores
+    // Two MMA warps, each running as a whole warp with one elected lane
+    // issuing: this one issues S^T, dP^T of every step of this CTA's items in
+    // order, warp MMA_G_WARP the dV, dK products, so neither waits behind
+    // the other's barriers; the tensor pipe interleaves the two streams.
     const uint32_t id_s = idesc(64, false);   // S^T = K Q^T, dP^T = V dO^T (N = 64 queries)
-    const uint32_t id_g = idesc(128, true);   // dV += P^T dO, dK += dS^T Q (N = 128, B MN-major)
     bool ok = true;
-    int i_s = first, k_s = 0, j_s = 0, n_s = 0;
-    int i_p = first, k_p = 0, j_p = 0, n_p = 0;
-    if (i_s < total) { int kt, bh; item(i_s, kt, bh, n_s); n_p = n_s; }
-    for (int g = 0; ok; ++g) {
-      const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
-      if (!s_left && !p_left) break;
-      if (s_left) {
-        const int st = g % DKDV_QS, kb = k_s & 1;
-        if (j_s == 0 && !warp_wait(&kv_full[kb], (k_s >> 1) & 1, abort_flag, err)) { ok = false; break; }
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int kt, bh, n_it;
+      item(i, kt, bh, n_it);
+      const int kb = k & 1;
+      if (!warp_wait(&kv_full[kb], (k >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      for (int j = 0; j < n_it; ++j, ++g) {
+        const int st = g % DKDV_QS;
         if (!warp_wait(&q_full[st], (g / DKDV_QS) & 1, abort_flag, err)) { ok = false; break; }
         // S^T, dP^T of step g overwrite step g - 1's: the compute warps have loaded those
         if (g >= 1 && !warp_wait(s_read, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
@@ -731,46 +731,44 @@ __global__ void __launch_bounds__(THREADS_B, 1)
         const uint32_t aK = smem_u32(sKV + kb * KV_BUF), aV = aK + KV_T;
         const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem, kdesc128(aK, KV_T / 2, k), kdesc128(aQ, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_w(tmem, kdesc128(aK, KV_T / 2, kk), kdesc128(aQ, QT64 / 2, kk), id_s, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem + 64, kdesc128(aV, KV_T / 2, k), kdesc128(aO, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_w(tmem + 64, kdesc128(aV, KV_T / 2, kk), kdesc128(aO, QT64 / 2, kk), id_s, kk > 0 ? 1u : 0u);
         tc_commit_w(s_full);
-        if (++j_s == n_s) {
-          j_s = 0;
-          ++k_s;
-          i_s += stride;
-          if (i_s < total) { int kt, bh; item(i_s, kt, bh, n_s); }
-        }
-      }
-      if (p_left) {
-        const int gp = g - 1, s = gp & 1, st = gp % DKDV_QS;
-        // the item's first products overwrite dV, dK: the previous item's have been read
-        if (j_p == 0 && k_p >= 1 && !warp_wait(acc_empty, (k_p - 1) & 1, abort_flag, err)) { ok = false; break; }
-        if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
-        // k-step k covers queries 16k..16k+15: packed columns 8k..8k+7
-        const uint32_t pb = tmem + 128 + s * 64;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_ts_w(tmem + 256, pb + 8 * k, mndesc(aO, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_ts_w(tmem + 384, pb + 32 + 8 * k, mndesc(aQ, QT64 / 2, k), id_g, (j_p > 0 || k > 0) ? 1u : 0u);
-        tc_commit_w(&g_done[s]);
-        tc_commit_w(&q_empty[st]);
-        if (++j_p == n_p) {  // the item's last products: dV, dK are complete
-          tc_commit_w(acc_full);
-          j_p = 0;
-          ++k_p;
-          i_p += stride;
-          if (i_p < total) { int kt, bh; item(i_p, kt, bh, n_p); }
-        }
+        tc_commit_w(&q_empty[st]);   // one of the stage's two releases
       }
     }
-  } else {
+  } else if (warp == MMA_G_WARP) {
+    // ---------------------------------------------------------------- MMA: gradients
+    const uint32_t id_g = idesc(128, true);   // dV += P^T dO, dK += dS^T Q (N = 128, B MN-major)
+    bool ok = true;
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int kt, bh, n_it;
+      item(i, kt, bh, n_it);
+      // the item's first products overwrite dV, dK: the previous item's have been read
+      if (k >= 1 && !warp_wait(acc_empty, (k - 1) & 1, abort_flag, err)) { ok = false; break; }
+      for (int j = 0; j < n_it; ++j, ++g) {
+        const int s = g & 1, st = g % DKDV_QS;
+        if (!warp_wait(&p_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ + st * QT64), aO = smem_u32(sO + st * QT64);
+        // k-step kk covers queries 16kk..16kk+15: packed columns 8kk..8kk+7
+        const uint32_t pb = tmem + 128 + s * 64;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts_w(tmem + 256, pb + 8 * kk, mndesc(aO, QT64 / 2, kk), id_g, (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts_w(tmem + 384, pb + 32 + 8 * kk, mndesc(aQ, QT64 / 2, kk), id_g, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit_w(&g_done[s]);
+        tc_commit_w(&q_empty[st]);   // the stage's other release
+      }
+      if (ok) tc_commit_w(acc_full);   // the item's dV, dK are complete
+    }
+  } else if (warp < MMA_G_WARP) {
     // ---------------------------------------------------------------- P^T, dS^T
     const int q4 = warp & 3, grp = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
@@ -995,7 +993,10 @@ __global__ void __launch_bounds__(THREADS_B, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < DQ_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < DQ_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 2);   // released by both MMA warps
+    }
     mbar_init(s_full, 1);
     mbar_init(s_read, 4 * NCG);
     for (int s = 0; s < 2; ++s) {
@@ -1063,69 +1064,63 @@ __global__ void __launch_bounds__(THREADS_B, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA
-    // One flattened sequence over this CTA's items: iteration g issues S/dP
-    // of step g, then the dQ product of step g - 1 (possibly of the previous
-    // item).  The whole warp runs it; one elected lane issues.
+    // ---------------------------------------------------------------- MMA: scores
+    // Two MMA warps as in the dK/dV kernel: this one issues S and dP of every
+    // step, warp MMA_G_WARP the dQ products.
     const uint32_t id_s = idesc(64, false);   // S = Q K^T, dP = dO V^T (N = 64 keys)
-    const uint32_t id_g = idesc(128, true);   // dQ += dS K (N = 128, B MN-major)
     const uint32_t aQ = smem_u32(sQ), aO = smem_u32(sO);
     bool ok = true;
-    int i_s = first, k_s = 0, j_s = 0, n_s = 0;
-    int i_p = first, k_p = 0, j_p = 0, n_p = 0;
-    if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); n_p = n_s; }
-    for (int g = 0; ok; ++g) {
-      const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
-      if (!s_left && !p_left) break;
-      if (s_left) {
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int qt, bh, n_it;
+      item(i, qt, bh, n_it);
+      if (!warp_wait(q_full, k & 1, abort_flag, err)) { ok = false; break; }
+      for (int j = 0; j < n_it; ++j, ++g) {
         const int st = g % DQ_STAGES;
-        if (j_s == 0 && !warp_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
         if (!warp_wait(&kv_full[st], (g / DQ_STAGES) & 1, abort_flag, err)) { ok = false; break; }
         // S, dP of step g overwrite step g - 1's: the compute warps have loaded those
         if (g >= 1 && !warp_wait(s_read, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aK = smem_u32(sK + st * QT64), aV = smem_u32(sV + st * QT64);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem, kdesc128(aQ, KV_T / 2, k), kdesc128(aK, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_w(tmem, kdesc128(aQ, KV_T / 2, kk), kdesc128(aK, QT64 / 2, kk), id_s, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc_mma_w(tmem + 64, kdesc128(aO, KV_T / 2, k), kdesc128(aV, QT64 / 2, k), id_s, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_w(tmem + 64, kdesc128(aO, KV_T / 2, kk), kdesc128(aV, QT64 / 2, kk), id_s, kk > 0 ? 1u : 0u);
         tc_commit_w(s_full);
-        if (++j_s == n_s) {  // the item's last S/dP: Q and dO may be replaced
-          tc_commit_w(q_empty);
-          j_s = 0;
-          ++k_s;
-          i_s += stride;
-          if (i_s < total) { int qt, bh; item(i_s, qt, bh, n_s); }
-        }
+        tc_commit_w(&kv_empty[st]);   // one of the stage's two releases
       }
-      if (p_left) {
-        const int gp = g - 1, s = gp & 1, st = gp % DQ_STAGES, ob = k_p & 1;
-        if (j_p == 0 && k_p >= 2 && !warp_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (ok) tc_commit_w(q_empty);   // the item's last S/dP: Q and dO may be replaced
+    }
+  } else if (warp == MMA_G_WARP) {
+    // ---------------------------------------------------------------- MMA: dQ
+    const uint32_t id_g = idesc(128, true);   // dQ += dS K (N = 128, B MN-major)
+    bool ok = true;
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int qt, bh, n_it;
+      item(i, qt, bh, n_it);
+      const int ob = k & 1;
+      // the item's first product overwrites its dQ buffer: the compute warps
+      // have read that buffer for the item two positions back
+      if (k >= 2 && !warp_wait(&o_empty[ob], ((k - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      for (int j = 0; j < n_it; ++j, ++g) {
+        const int s = g & 1, st = g % DQ_STAGES;
+        if (!warp_wait(&p_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aK = smem_u32(sK + st * QT64);
-        // k-step k covers keys 16k..16k+15: packed columns 8k..8k+7
+        // k-step kk covers keys 16kk..16kk+15: packed columns 8kk..8kk+7
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 32 + 8 * k, mndesc(aK, QT64 / 2, k), id_g,
-                      (j_p > 0 || k > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 32 + 8 * kk, mndesc(aK, QT64 / 2, kk), id_g,
+                      (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit_w(&g_done[s]);
-        tc_commit_w(&kv_empty[st]);
-        if (++j_p == n_p) {  // the item's last product: dQ is complete
-          tc_commit_w(&o_full[ob]);
-          j_p = 0;
-          ++k_p;
-          i_p += stride;
-          if (i_p < total) { int qt, bh; item(i_p, qt, bh, n_p); }
-        }
+        tc_commit_w(&kv_empty[st]);   // the stage's other release
       }
+      if (ok) tc_commit_w(&o_full[ob]);   // the item's dQ is complete
     }
-  } else {
+  } else if (warp < MMA_G_WARP) {
     // ---------------------------------------------------------------- dS
     const int q4 = warp & 3, grp = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
