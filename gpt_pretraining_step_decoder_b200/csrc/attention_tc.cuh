@@ -35,7 +35,8 @@
 namespace fatc {
 
 constexpr int BQ = 128, BKV = 128, HD = 128;
-constexpr int THREADS = 192;
+constexpr int PV_WARP = 6;        // warps 2..5 are the softmax warps
+constexpr int THREADS = 224;
 constexpr int TILE_BYTES = 128 * 128 * 2;          // one 128 x 128 bf16 tile
 constexpr int SMEM_BYTES = TILE_BYTES /*Q*/ + 2 * 2 * TILE_BYTES /*K,V x 2 stages*/ + 1024 /*align*/ +
                            256 /*barriers*/;
@@ -282,74 +283,67 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA
-    // One flattened sequence of steps over this CTA's items: iteration g
-    // issues S of step g, then PV of step g - 1 (which may belong to the
-    // previous item), so the next item's first S overlaps the last softmax.
-    // S = Q K^T: A = Q (K-major), B = K (K-major), N = 128
+    // ---------------------------------------------------------------- MMA: scores
+    // Two MMA warps, each running as a whole warp with one elected lane
+    // issuing: this one issues S of every step of this CTA's items in order,
+    // warp PV_WARP the PV products, so neither waits behind the other's
+    // barriers.  S = Q K^T: A = Q (K-major), B = K (K-major), N = 128
     const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
                              ((uint32_t)(128 >> 4) << 24);
-    // O += P V: A = P (TMEM), B = V (MN-major), N = 128
-    const uint32_t idesc_o = idesc_s | (1u << 16);
     const uint32_t aQ = smem_u32(sQ);
     bool ok = true;
-    // S cursor (item index i_s, its k-th position k_s, step j_s) and PV cursor
-    int i_s = first, k_s = 0, j_s = 0, nkv_s = 0;
-    int i_p = first, k_p = 0, j_p = 0, nkv_p = 0;
-    if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = nkv_p = qt + 1; }
-    for (int g = 0; ok; ++g) {
-      const bool s_left = i_s < total, p_left = g >= 1 && i_p < total;
-      if (!s_left && !p_left) break;
-      if (s_left) {
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int qt, bh;
+      fwd_item(i, n_qt, BH, qt, bh);
+      const int n_kv = qt + 1;
+      if (!warp_wait(q_full, k & 1, abort_flag, err)) { ok = false; break; }
+      for (int j = 0; j < n_kv; ++j, ++g) {
         const int s = g & 1;
-        if (j_s == 0 && !warp_wait(q_full, k_s & 1, abort_flag, err)) { ok = false; break; }
         if (!warp_wait(&k_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         // S of step g overwrites step g - 1's: the softmax warps have loaded it
         if (g >= 1 && !warp_wait(s_read, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aK = smem_u32(sK + s * TILE_BYTES);
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k)
-          tc_mma_w(tmem, kmaj_desc(aQ, k), kmaj_desc(aK, k), idesc_s, k > 0 ? 1u : 0u);
+        for (int kk = 0; kk < HD / 16; ++kk)
+          tc_mma_w(tmem, kmaj_desc(aQ, kk), kmaj_desc(aK, kk), idesc_s, kk > 0 ? 1u : 0u);
         tc_commit_w(s_full);
         tc_commit_w(&k_empty[s]);
-        if (++j_s == nkv_s) {  // the item's last S: Q may be replaced
-          tc_commit_w(q_empty);
-          j_s = 0;
-          ++k_s;
-          i_s += stride;
-          if (i_s < total) { int qt, bh; fwd_item(i_s, n_qt, BH, qt, bh); nkv_s = qt + 1; }
-        }
       }
-      if (p_left) {
-        const int gp = g - 1, s = gp & 1, ob = k_p & 1;
-        // the first PV of an item overwrites its O buffer: the softmax warps
-        // must have read that buffer for the item two positions back
-        if (j_p == 0 && k_p >= 2 && !warp_wait(&o_empty[ob], ((k_p - 2) >> 1) & 1, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        if (!warp_wait(&p_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        if (!warp_wait(&v_full[s], (gp >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (ok) tc_commit_w(q_empty);   // the item's last S: Q may be replaced
+    }
+  } else if (warp == PV_WARP) {
+    // ---------------------------------------------------------------- MMA: PV
+    // O += P V: A = P (TMEM), B = V (MN-major), N = 128
+    const uint32_t idesc_o = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(128 >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);
+    bool ok = true;
+    int g = 0;
+    for (int i = first, k = 0; i < total && ok; i += stride, ++k) {
+      int qt, bh;
+      fwd_item(i, n_qt, BH, qt, bh);
+      const int n_kv = qt + 1, ob = k & 1;
+      // the first PV of an item overwrites its O buffer: the softmax warps
+      // must have read that buffer for the item two positions back
+      if (k >= 2 && !warp_wait(&o_empty[ob], ((k - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      for (int j = 0; j < n_kv; ++j, ++g) {
+        const int s = g & 1;
+        if (!warp_wait(&p_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (!warp_wait(&v_full[s], (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t aV = smem_u32(sV + s * TILE_BYTES);
-        // k-step k covers keys 16k..16k+15: packed P columns 8k..8k+7
+        // k-step kk covers keys 16kk..16kk+15: packed P columns 8kk..8kk+7
 #pragma unroll
-        for (int k = 0; k < BKV / 16; ++k)
-          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 64 + k * 8, mnmaj_desc(aV, k), idesc_o,
-                      (j_p > 0 || k > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc_mma_ts_w(tmem + 256 + ob * 128, tmem + 128 + s * 64 + kk * 8, mnmaj_desc(aV, kk), idesc_o,
+                      (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit_w(&p_free[s]);
         tc_commit_w(&v_empty[s]);
-        if (++j_p == nkv_p) {  // the item's last PV: O is complete
-          tc_commit_w(&o_full[ob]);
-          j_p = 0;
-          ++k_p;
-          i_p += stride;
-          if (i_p < total) { int qt, bh; fwd_item(i_p, n_qt, BH, qt, bh); nkv_p = qt + 1; }
-        }
       }
+      if (ok) tc_commit_w(&o_full[ob]);   // the item's last PV: O is complete
     }
-  } else {
+  } else if (warp < PV_WARP) {
     // ------------------------------------------------------------------ softmax
     const int q = warp & 3;
     const int r = q * 32 + lane;               // row within the tile
@@ -537,7 +531,6 @@ using fatc::pack_bf16x2_int;
 using fatc::pack_bf16x2_rn;
 using fatc::tmem_ldw;
 using fatc::tmem_stw;
-constexpr int THREADS = 192;
 
 // K-major [rows x 128] tile, MMA k-step k over the 128 columns
 __device__ __forceinline__ uint64_t kdesc128(uint32_t base, int half_bytes, int k) {
