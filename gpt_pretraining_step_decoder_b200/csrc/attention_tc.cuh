@@ -171,6 +171,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fa_tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmO, float* __restrict__ lse_out, int T, int H, int BH,
                      unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -586,6 +587,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
                           const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmG,
                           const float* __restrict__ lse2, const float* __restrict__ Dv, int T, int H, int BH,
                           unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -948,6 +950,7 @@ __global__ void __launch_bounds__(THREADS_B, 1)
                         const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmG,
                         const float* __restrict__ lse2, const float* __restrict__ Dv, int T, int H, int BH,
                         unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

@@ -33,6 +33,15 @@ template <typename T> __device__ __forceinline__ T from_f(float x);
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation is set up while
+// the kernel before it in the stream runs; pdl_wait() blocks until that
+// kernel has completed and its memory is visible (a no-op for a kernel
+// launched without the attribute).  Every such kernel calls it before
+// touching global memory.  (None triggers its dependents early: CTAs of the
+// next kernel waiting on SMs the current one still uses measured slower.)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -88,6 +88,7 @@ __device__ __forceinline__ void epi_apply_one(const GemmEpilogue& e, long long m
 template <typename act_t>
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N,
                                      GemmEpilogue e) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const long long total = (long long)M * N;
   const bool vec = (N % 4) == 0 && (e.ldc % 4) == 0 && (e.mode == EPI_ACCUM_F32 || e.mode == EPI_STORE_F32);
   if (vec) {

@@ -501,6 +501,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmAux,
                    const Params p) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   using C = Cfg<BN, KmHeavy<KM>::value, CG>;
   static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair per tile");
   constexpr int KE = F8 ? 128 : BK;  // operand elements per 128-byte k-block row

@@ -153,6 +153,39 @@ extern "C" int gptx_set_gemm_cta_pairs(int on) {
   return GPT_OK;
 }
 
+// Programmatic dependent launch for the step's frequent kernels (GEMM,
+// split-K reduce, attention, norms, RoPE backward, cross-entropy, AdamW):
+// each is set up while the kernel before it in the stream finishes, and calls
+// pdl_wait() before touching global memory.  Measured on B200: 33.97 -> 33.25
+// ms per GPT-2-small step, about the time the step spent between kernels.
+// GPT_PDL=0 in the environment launches them plainly.
+static bool pdl_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("GPT_PDL");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+static void pdl_attr(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+}
+template <typename... KArgs, typename... Args>
+static void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  pdl_attr(at[0]);
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Pairs of SMs that can hold one pair-mode GEMM cluster each at a time (the
 // persistent grid's size in units of tiles); computed once per kernel.
 template <typename K>
@@ -189,19 +222,22 @@ static int gemm_tc_launch_k(const CUtensorMap& ta, const CUtensorMap& tb, const 
   const int tiles = p.m_tiles * p.n_tiles * p.splits * p.batch;
   const int grid = CG * (tiles < units ? tiles : units);
   ++g_launches;
-  if constexpr (CG == 1) {
-    kernel<<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, tcm, taux, p);
-  } else {
+  {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = CG; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    if constexpr (CG == 2) {
+      at[na].id = cudaLaunchAttributeClusterDimension;
+      at[na].val.clusterDim.x = CG; at[na].val.clusterDim.y = 1; at[na].val.clusterDim.z = 1;
+      ++na;
+    }
+    if (pdl_enabled()) pdl_attr(at[na++]);
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(tc::NUM_THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = st;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, ta, tb, tcm, taux, p));
   }
   LAUNCH_CHECK();
@@ -323,7 +359,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
     const long long total = (long long)M * N;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 4 * device_sms()) blocks = 4 * device_sms();
-    ++g_launches; splitk_reduce_kernel<bf16><<<blocks, 256, 0, st>>>(partial, p.splits, M, N, e);
+    ++g_launches; launch_pdl(splitk_reduce_kernel<bf16>, blocks, 256, 0, st, partial, p.splits, M, N, e);
     LAUNCH_CHECK();
   }
   return GPT_OK;
@@ -1094,7 +1130,7 @@ static int attention_fwd(gpt_model* m, const act_t* qkv, act_t* o, float* lse) {
     // blocks, rows past a sequence's end clipped
     CUtensorMap to;
     TRY(make_tmap3(&to, o, a, c.seq_len, a, c.micro_batch, (long long)c.seq_len * a, 64, 32));
-    ++g_launches; fatc::fa_tc_fwd_kernel<<<grid, fatc::THREADS, fatc::SMEM_BYTES_TC, m->st>>>(
+    ++g_launches; launch_pdl(fatc::fa_tc_fwd_kernel, grid, fatc::THREADS, fatc::SMEM_BYTES_TC, m->st,
         tqk, tv, to, lse, c.seq_len, c.n_head, c.micro_batch * c.n_head, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
@@ -1113,7 +1149,7 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
   const long long N = (long long)c.micro_batch * c.seq_len;
   ProfScope ps(&m->prof, m->st, "attention_bwd",
                5.0 * c.micro_batch * c.n_head * (double)c.seq_len * c.seq_len * c.head_dim, 0.0);
-  ++g_launches; attn_bwd_pre_kernel<act_t><<<grid_for(N * c.n_head * 32, 256), 256, 0, m->st>>>(
+  ++g_launches; launch_pdl(attn_bwd_pre_kernel<act_t>, grid_for(N * c.n_head * 32, 256), 256, 0, m->st,
       o, dout, Dv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
   LAUNCH_CHECK();
   if (std::is_same<act_t, bf16>::value) {
@@ -1137,9 +1173,9 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
     const int BH = c.micro_batch * c.n_head;
     const long long items = (long long)cdiv(c.seq_len, 128) * BH;  // key tiles (dK, dV) = query tiles (dQ)
     const int grid = items < device_sms() ? (int)items : device_sms();  // persistent
-    ++g_launches; fatcb::fa_tc_bwd_dkdv_kernel<<<grid, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st>>>(
+    ++g_launches; launch_pdl(fatcb::fa_tc_bwd_dkdv_kernel, grid, fatcb::THREADS_B, fatcb::DKDV_SMEM, m->st,
         t128, t64, tdo, tg, lse, Dv, c.seq_len, c.n_head, BH, m->err());
-    ++g_launches; fatcb::fa_tc_bwd_dq_kernel<<<grid, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st>>>(
+    ++g_launches; launch_pdl(fatcb::fa_tc_bwd_dq_kernel, grid, fatcb::THREADS_B, fatcb::DQ_SMEM, m->st,
         t128, t64, tdo, tg, lse, Dv, c.seq_len, c.n_head, BH, m->err());
     LAUNCH_CHECK();
     return GPT_OK;
@@ -1217,7 +1253,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   float* x = m->at<float>(p.x);
   {
   ProfScope ps(pf, st, "embed", 0.0, (double)N * d * (es + 4 + (c.x0_rows ? es : 0)));
-  WITH_NV(d, ++g_launches; embed_fwd_kernel<NV, act_t, act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+  WITH_NV(d, ++g_launches; launch_pdl(embed_fwd_kernel<NV, act_t, act_t>, grid_for((long long)N * 32, 256), 256, 0, st,
       tokens, W("wte"), c.x0_rows ? reinterpret_cast<const act_t*>(m->base + p.hx) : nullptr,
       m->at<int32_t>(p.rows_x), x, m->at<float>(p.emb_rstd), N, d, V, c.norm_eps, err););
   LAUNCH_CHECK();
@@ -1233,7 +1269,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     act_t* u2 = m->at<act_t>(L.u2);
     {
       ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
-      WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, u, m->at<float>(L.rstd1), N, d, c.norm_eps););
+      WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_fwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, x, u, m->at<float>(L.rstd1), N, d, c.norm_eps););
       LAUNCH_CHECK();
     }
     if (b16) {
@@ -1258,7 +1294,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     TRY(gemm(g, N, d, a, op_k(o, a), op_k(W(pre + "wo"), a), epi(EPI_ACCUM_F32, x, d, 1), false, "gemm.o_fwd"));
     {
       ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
-      WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps););
+      WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_fwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, x, u2, m->at<float>(L.rstd2), N, d, c.norm_eps););
       LAUNCH_CHECK();
     }
     TRY(gemm(g, N, F, d, op_k(u2, d), op_k(W(pre + "w1"), d),
@@ -1268,7 +1304,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   act_t* xf = m->at<act_t>(p.xf);
   {
     ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
-    WITH_NV(d, ++g_launches; rmsnorm_fwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps););
+    WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_fwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps););
   }
   ++g_launches; ce_prepare_kernel<<<1, 1024, 0, st>>>(targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
   LAUNCH_CHECK();
@@ -1289,7 +1325,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       TRY(gemm(g, rows, V, d, op_k(xf + (long long)r0 * d, d), op_k(Wlm, d), el, false, "gemm.lm_fwd"));
       ProfScope ps(pf, st, "cross_entropy", 0.0, (double)rows * V * 4);
       const int tcols = V >= 256 ? 128 : 64, ntl = cdiv(V, tcols);  // half-tile statistics
-      ++g_launches; ce_prob_kernel<<<rows, 256, ntl * 4, st>>>(
+      ++g_launches; launch_pdl(ce_prob_kernel, rows, 256, ntl * 4, st,
           reinterpret_cast<bf16*>(dz), m->at<float2>(p.ce_stats), ntl, tcols, targets + r0, m->at<float>(p.ce_ztgt),
           m->at<float>(p.tok_loss) + r0, V, c.softcap, m->at<float>(p.ce_scale), err);
       LAUNCH_CHECK();
@@ -1340,7 +1376,7 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
   float* g_head = Gp(c.tie_embeddings ? "wte" : "lm_head");
   {
     ProfScope ps(pf, st, "head_grad_accumulate", 0.0, (double)V * d * 12);
-    ++g_launches; accumulate_kernel<<<4 * device_sms(), 256, 0, st>>>(g_head, m->at<float>(p.pending), (long long)V * d, beta);
+    ++g_launches; launch_pdl(accumulate_kernel, 4 * device_sms(), 256, 0, st, g_head, m->at<float>(p.pending), (long long)V * d, beta);
     if (!c.tie_embeddings && !beta) CUDA_TRY(cudaMemsetAsync(Gp("wte"), 0, (size_t)V * d * 4, st));
   }
   float* dx = m->at<float>(p.dx);
@@ -1349,7 +1385,7 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
   act_t* dqkv = m->at<act_t>(p.dqkv);
   act_t* da = m->at<act_t>(p.da);
   act_t* dout = m->at<act_t>(p.dout);
-  { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; rmsnorm_bwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(m->at<float>(p.dxf), m->at<act_t>(p.xf),
+  { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_bwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, m->at<float>(p.dxf), m->at<act_t>(p.xf),
                                                         m->at<float>(p.rstd_f), dx, dx_lp, N, d, 0););
   LAUNCH_CHECK(); }
   for (int l = c.n_layer - 1; l >= 0; --l) {
@@ -1360,7 +1396,7 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     TRY(gemm(g, N, F, d, op_k(dx_lp, d), op_mn(W(pre + "w2"), F), epi(EPI_DRELU2, da, F, 0, nullptr, m->at<act_t>(L.g)), false, "gemm.down_dgrad"));
     TRY(gemm(g, F, d, N, op_mn(da, F), op_mn(m->at<act_t>(L.u2), d), epi(EPI_ACCUM_F32, Gp(pre + "w1"), d, beta), true, "gemm.up_wgrad"));
     TRY(gemm(g, N, d, F, op_k(da, F), op_mn(W(pre + "w1"), d), epi(EPI_STORE_F32, du, d), false, "gemm.up_dgrad"));
-    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; rmsnorm_bwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1););
+    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_bwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, du, m->at<act_t>(L.u2), m->at<float>(L.rstd2), dx, dx_lp, N, d, 1););
     LAUNCH_CHECK(); }
     // ---- attention: x += o Wo^T
     TRY(gemm(g, d, a, N, op_mn(dx_lp, d), op_mn(m->at<act_t>(L.o), a), epi(EPI_ACCUM_F32, Gp(pre + "wo"), a, beta), true, "gemm.o_wgrad"));
@@ -1370,7 +1406,7 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     {
       ProfScope ps(pf, st, "rope_qknorm_bwd", 0.0, (double)N * a * es * 6 + (c.v_rows ? (double)N * a * (es + 8) : 0.0));
       if (b16)  // hd == 128 in bf16 mode
-        ++g_launches, rope_qknorm_bwd_hd128_kernel<<<grid_for((long long)N * H * 32, 256), 256, 0, st>>>(
+        ++g_launches, launch_pdl(rope_qknorm_bwd_hd128_kernel, grid_for((long long)N * H * 32, 256), 256, 0, st,
             reinterpret_cast<bf16*>(dqkv), reinterpret_cast<const bf16*>(m->at<act_t>(L.qkv)), m->at<float>(p.rope_cs),
             m->at<float>(L.rstd_q), m->at<float>(L.rstd_k), p.gv ? m->at<float>(p.gv) : nullptr,
             l != c.n_layer - 1, N, c.seq_len, H, c.qk_norm);
@@ -1382,7 +1418,7 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     }
     TRY(gemm(g, 3 * a, d, N, op_mn(dqkv, 3 * a), op_mn(m->at<act_t>(L.u), d), epi(EPI_ACCUM_F32, Gp(pre + "wqkv"), d, beta), true, "gemm.qkv_wgrad"));
     TRY(gemm(g, N, d, 3 * a, op_k(dqkv, 3 * a), op_mn(W(pre + "wqkv"), d), epi(EPI_STORE_F32, du, d), false, "gemm.qkv_dgrad"));
-    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; rmsnorm_bwd_kernel<NV, act_t><<<rows_blocks, 256, 0, st>>>(du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1););
+    { ProfScope psn(pf, st, "rmsnorm_bwd", 0.0, nb_bytes); WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_bwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, du, m->at<act_t>(L.u), m->at<float>(L.rstd1), dx, dx_lp, N, d, 1););
     LAUNCH_CHECK(); }
   }
   // dx now holds dL/dx0 per position.
@@ -1567,7 +1603,7 @@ static int optimizer_step_impl(gpt_model* m, float lr) {
     aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
     aa.bc2 = (float)(1.0 - pow((double)c.adam_b2, (double)m->step_t));
     aa.clip = coef;
-    ++g_launches; adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
+    ++g_launches; launch_pdl(adamw_kernel, 8 * device_sms(), 256, 0, st, aa);
     LAUNCH_CHECK();
   }
   if (muon) TRY(muon_step_impl(m, lr, coef));
@@ -1655,7 +1691,7 @@ extern "C" int gpt_optimizer_step_range(gpt_model* m, float lr, long long lo, lo
   aa.bc1 = (float)(1.0 - pow((double)c.adam_b1, (double)m->step_t));
   aa.bc2 = (float)(1.0 - pow((double)c.adam_b2, (double)m->step_t));
   aa.clip = coef;
-  ++g_launches; adamw_kernel<<<8 * device_sms(), 256, 0, st>>>(aa);
+  ++g_launches; launch_pdl(adamw_kernel, 8 * device_sms(), 256, 0, st, aa);
   LAUNCH_CHECK();
   return GPT_OK;
 }

@@ -22,6 +22,7 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __r
                                  const tab_t* __restrict__ hx, const int32_t* __restrict__ rx,
                                  float* __restrict__ x, float* __restrict__ rstd_out, int N, int d,
                                  int V, float eps, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N) return;
   int id = tok[warp];
@@ -64,6 +65,7 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const w_t* __r
 template <int NV, typename act_t>
 __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, act_t* __restrict__ u,
                                    float* __restrict__ rstd_out, int N, int d, float eps) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N) return;
   const float* xr = x + (long long)warp * d;
@@ -98,6 +100,7 @@ template <int NV, typename act_t>
 __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __restrict__ u,
                                    const float* __restrict__ rstd, float* __restrict__ dx,
                                    act_t* __restrict__ dx_lp, int N, int d, int accumulate) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N) return;
   const long long base = (long long)warp * d;
@@ -271,6 +274,7 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_hd128_kernel(
     bf16* __restrict__ dqkv, const bf16* __restrict__ qkv, const float* __restrict__ cs,
     const float* __restrict__ rstd_q, const float* __restrict__ rstd_k, float* __restrict__ gv, int gv_accumulate,
     int N, int T, int H, int qk_norm) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= N * H) return;  // whole warp
   const int n = warp / H, h = warp % H, t = n % T;
@@ -393,6 +397,7 @@ __global__ void __launch_bounds__(256) ce_prob_kernel(bf16* __restrict__ ez, con
                                                       const float* __restrict__ ztgt,
                                                       float* __restrict__ tok_loss, int V, float softcap,
                                                       const float* __restrict__ scale_dev, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   extern __shared__ float fac[];  // exp(m_j - lse) per column block
   __shared__ float sh[32];
   const long long row = blockIdx.x;
@@ -563,6 +568,7 @@ __global__ void attn_fwd_simt_kernel(const act_t* __restrict__ qkv, act_t* __res
 template <typename act_t>
 __global__ void attn_bwd_pre_kernel(const act_t* __restrict__ o, const act_t* __restrict__ dout,
                                     float* __restrict__ Dout, int B, int T, int H, int hd) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= B * T * H) return;
   const int n = warp / H, h = warp % H, b = n / T, t = n % T;

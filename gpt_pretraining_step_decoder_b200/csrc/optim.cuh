@@ -16,6 +16,7 @@ struct AdamArgs {
 };
 
 __global__ void adamw_kernel(AdamArgs a) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const float coef = a.clip ? *a.clip : 1.f;
   const long long n4 = a.n / 4;
   for (long long i4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
@@ -103,6 +104,7 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__
 // out[i] = (beta ? out[i] : 0) + add[i]
 __global__ void accumulate_kernel(float* __restrict__ out, const float* __restrict__ add, long long n,
                                   int beta) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x)
     out[i] = (beta ? out[i] : 0.f) + add[i];
