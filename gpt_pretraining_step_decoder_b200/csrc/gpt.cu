@@ -820,7 +820,7 @@ static int grid_for(long long n, int per_block) {
 static int refresh_lp(gpt_model* m) {
   if (!cfg_bf16(m->cfg)) return GPT_OK;
   const Plan& p = m->plan;
-  ++g_launches; to_bf16_kernel<<<4 * device_sms(), 256, 0, m->st>>>(m->at<float>(p.P), m->at<bf16>(p.Plp), p.dense_n);
+  ++g_launches; launch_pdl(to_bf16_kernel, 4 * device_sms(), 256, 0, m->st, m->at<float>(p.P), m->at<bf16>(p.Plp), p.dense_n);
   LAUNCH_CHECK();
   return GPT_OK;
 }
@@ -1033,9 +1033,9 @@ static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long 
   int32_t* vout = w.va;
   for (int ps = 0; ps < passes; ++ps) {
     const int32_t* raw = ps == 0 ? keys : nullptr;
-    ++g_launches; radix_hist_kernel<<<(unsigned)nblk, RADIX_THREADS, 0, st>>>(kin, raw, n, key_range, items, 8 * ps, w.counts);
-    if (scanned) { ++g_launches; radix_offsets_kernel<<<1, 1024, 0, st>>>(w.counts, (int)nblk); }
-    ++g_launches; radix_scatter_kernel<<<(unsigned)nblk, RADIX_THREADS, 0, st>>>(kin, vin, raw, n, key_range, items, 8 * ps,
+    ++g_launches; launch_pdl(radix_hist_kernel, (unsigned)nblk, RADIX_THREADS, 0, st, kin, raw, n, key_range, items, 8 * ps, w.counts);
+    if (scanned) { ++g_launches; launch_pdl(radix_offsets_kernel, 1, 1024, 0, st, w.counts, (int)nblk); }
+    ++g_launches; launch_pdl(radix_scatter_kernel, (unsigned)nblk, RADIX_THREADS, 0, st, kin, vin, raw, n, key_range, items, 8 * ps,
                                                                   w.counts, scanned, kout, vout, err);
     LAUNCH_CHECK();
     kin = kout;
@@ -1044,7 +1044,7 @@ static int bucket_by_key(const SortWs& w, const int32_t* keys, int n, long long 
     vout = (vout == w.va) ? w.vb : w.va;
   }
   if (uniq_out || n_uniq_out) {
-    ++g_launches; unique_keys_kernel<<<1, 1024, 0, st>>>(kin, n, key_range, uniq_out, n_uniq_out);
+    ++g_launches; launch_pdl(unique_keys_kernel, 1, 1024, 0, st, kin, n, key_range, uniq_out, n_uniq_out);
     LAUNCH_CHECK();
   }
   *keys_out = kin;
@@ -1074,7 +1074,7 @@ static int launch_table_chunk(tab_t* table, float* state, int d, const float* gr
     attr = true;
   }
   ++g_launches;
-  table_chunk_kernel<tab_t, MAXT, STAGE><<<(unsigned)nchunks, nt, table_chunk_smem<tab_t>(nt, STAGE), st>>>(
+  launch_pdl(table_chunk_kernel<tab_t, MAXT, STAGE>, (unsigned)nchunks, nt, table_chunk_smem<tab_t>(nt, STAGE), st, 
       table, state, d, grad, skeys, perm, n, n_rows, w.part_head, w.part_tail, lr, beta, eps);
   return GPT_OK;
 }
@@ -1100,7 +1100,7 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;  // <= 56 KB (d <= 2048)
   const unsigned chain_grid = (unsigned)((nchunks + CHAIN_WARPS - 1) / CHAIN_WARPS);
   WITH_NV(d, TRY(allow_smem(table_chain_kernel<NV, tab_t>, chain_smem)); ++g_launches;
-          table_chain_kernel<NV, tab_t><<<chain_grid, CHAIN_WARPS * 32, chain_smem, st>>>(
+          launch_pdl(table_chain_kernel<NV, tab_t>, chain_grid, CHAIN_WARPS * 32, chain_smem, st, 
               table, state, d, skeys, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
   LAUNCH_CHECK();
   return GPT_OK;
@@ -1210,7 +1210,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   CUDA_TRY(cudaMemcpyAsync(m->at<int32_t>(p.tok_copy), tokens, (size_t)N * 4, cudaMemcpyDeviceToDevice, st));
   if (c.x0_rows || c.v_rows) {
     ProfScope ps(pf, st, "ngram_hash", 0.0, (double)N * 12);
-    ++g_launches; ngram_hash_kernel<<<grid_for(N, 256), 256, 0, st>>>(
+    ++g_launches; launch_pdl(ngram_hash_kernel, grid_for(N, 256), 256, 0, st, 
         tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.x0_rows ? c.x0_rows : 1,
         c.x0_rows ? m->at<int32_t>(p.rows_x) : nullptr, c.v_rows ? c.v_rows : 1,
         c.v_rows ? m->at<int32_t>(p.rows_v) : nullptr, err);
@@ -1224,17 +1224,17 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     const int w3 = c.tri_width;
     {
       ProfScope ps(pf, st, "trigram_gather", 0.0, (double)N * (12 + 2.0 * w3 * es));
-      ++g_launches; trigram_hash_kernel<<<grid_for(N, 256), 256, 0, st>>>(
+      ++g_launches; launch_pdl(trigram_hash_kernel, grid_for(N, 256), 256, 0, st, 
           tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.hash_p3, c.tri_rows,
           m->at<int32_t>(p.rows_3), err);
       const act_t* h3 = reinterpret_cast<const act_t*>(m->base + p.h3);
       act_t* s3g = m->at<act_t>(p.s3g);
       if (b16) {
-        ++g_launches; ngram_gather_bf16x8_kernel<<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+        ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid_for((long long)N * 32, 256), 256, 0, st, 
             m->at<int32_t>(p.rows_3), N, reinterpret_cast<const bf16*>(h3), c.tri_rows, w3,
             reinterpret_cast<bf16*>(s3g), 0, err);
       } else {
-        ++g_launches; ngram_gather_kernel<act_t><<<grid_for((long long)N * 32, 256), 256, 0, st>>>(
+        ++g_launches; launch_pdl(ngram_gather_kernel<act_t>, grid_for((long long)N * 32, 256), 256, 0, st, 
             m->at<int32_t>(p.rows_3), N, h3, c.tri_rows, w3, s3g, 0, err);
       }
       LAUNCH_CHECK();
@@ -1243,7 +1243,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
              epi(EPI_STORE_F32, m->at<float>(p.p3), a), false, "gemm.vproj_fwd"));
     {
       ProfScope ps(pf, st, "value_bias", 0.0, (double)N * a * (4 + es + (c.v_rows ? es : 0)));
-      ++g_launches; value_bias_kernel<act_t><<<4 * device_sms(), 256, 0, st>>>(
+      ++g_launches; launch_pdl(value_bias_kernel<act_t>, 4 * device_sms(), 256, 0, st, 
           m->at<float>(p.p3), vbias, vrows, N, a, m->at<act_t>(p.vb));
       LAUNCH_CHECK();
     }
@@ -1306,7 +1306,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     ProfScope ps(pf, st, "rmsnorm_fwd", 0.0, norm_bytes);
     WITH_NV(d, ++g_launches; launch_pdl(rmsnorm_fwd_kernel<NV, act_t>, rows_blocks, 256, 0, st, x, xf, m->at<float>(p.rstd_f), N, d, c.norm_eps););
   }
-  ++g_launches; ce_prepare_kernel<<<1, 1024, 0, st>>>(targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
+  ++g_launches; launch_pdl(ce_prepare_kernel, 1, 1024, 0, st, targets, N, c.grad_accum, m->at<float>(p.ce_scale), m->at<int>(p.ce_count));
   LAUNCH_CHECK();
   // chunked LM head + cross-entropy; the head's gradient pieces are formed
   // here while each logits chunk is live: dxf (fp32) and the pending head
@@ -1342,7 +1342,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     TRY(gemm(g, V, d, rows, op_mn(dz, V), op_mn(xf + (long long)r0 * d, d),
              epi(EPI_ACCUM_F32, m->at<float>(p.pending), d, ci > 0), true, "gemm.lm_wgrad"));
   }
-  ++g_launches; loss_reduce_kernel<<<1, 1024, 0, st>>>(m->at<float>(p.tok_loss), N, m->at<int>(p.ce_count), loss_dev, err);
+  ++g_launches; launch_pdl(loss_reduce_kernel, 1, 1024, 0, st, m->at<float>(p.tok_loss), N, m->at<int>(p.ce_count), loss_dev, err);
   LAUNCH_CHECK();
   m->have_fwd = true;
   return GPT_OK;
@@ -1429,7 +1429,7 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const act_t* gva;
     if (b16) {
       ProfScope ps(pf, st, "value_grad_bf16", 0.0, (double)N * a * 6);
-      ++g_launches; to_bf16_kernel<<<4 * device_sms(), 256, 0, st>>>(m->at<float>(p.gv), m->at<bf16>(p.gv16),
+      ++g_launches; launch_pdl(to_bf16_kernel, 4 * device_sms(), 256, 0, st, m->at<float>(p.gv), m->at<bf16>(p.gv16),
                                                                      (long long)N * a);
       LAUNCH_CHECK();
       gva = reinterpret_cast<const act_t*>(m->at<bf16>(p.gv16));
@@ -1447,12 +1447,12 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const int32_t* perm;
     TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
     const long long nchunks = (N + CHUNK - 1) / CHUNK;
-    WITH_NV(d, ++g_launches; emb_chunk_kernel<NV, act_t><<<grid_for(nchunks * 32, 128), 128, 0, st>>>(
+    WITH_NV(d, ++g_launches; launch_pdl(emb_chunk_kernel<NV, act_t>, grid_for(nchunks * 32, 128), 128, 0, st, 
         Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, N, V, w.part_head, w.part_tail););
     const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;
     const unsigned chain_grid = (unsigned)((nchunks + CHAIN_WARPS - 1) / CHAIN_WARPS);
     WITH_NV(d, TRY(allow_smem(emb_chain_kernel<NV>, chain_smem)); ++g_launches;
-            emb_chain_kernel<NV><<<chain_grid, CHAIN_WARPS * 32, chain_smem, st>>>(
+            launch_pdl(emb_chain_kernel<NV>, chain_grid, CHAIN_WARPS * 32, chain_smem, st, 
                 Gp("wte"), d, skeys, N, V, w.part_head, w.part_tail););
     LAUNCH_CHECK();
   }
@@ -1523,10 +1523,10 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
       // bytes: g, m read + m written; g, m read + bf16 iterate written
       ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * (12 + 10));
       ++g_launches;
-      muon_batch_momentum_kernel<<<dim3(MUON_BATCH_BLOCKS, nmat), MUON_THREADS, 0, st>>>(
+      launch_pdl(muon_batch_momentum_kernel, dim3(MUON_BATCH_BLOCKS, nmat), MUON_THREADS, 0, st, 
           G, M, grp, c.muon_momentum, c.muon_nesterov, clip, part);
       ++g_launches;
-      muon_batch_normalize_kernel<<<dim3(per_mat, nmat), MUON_THREADS, 0, st>>>(
+      launch_pdl(muon_batch_normalize_kernel, dim3(per_mat, nmat), MUON_THREADS, 0, st, 
           G, M, grp, c.muon_momentum, c.muon_nesterov, clip, part, 1e-7f, x);
       LAUNCH_CHECK();
     }
@@ -1542,7 +1542,7 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
       {
         ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * rr * 6);
         ++g_launches;
-        muon_combine_bf16_kernel<<<grid1(nmat * rr / 4), MUON_THREADS, 0, st>>>(abf, aa16, nmat * rr / 4, cb, cc,
+        launch_pdl(muon_combine_bf16_kernel, grid1(nmat * rr / 4), MUON_THREADS, 0, st, abf, aa16, nmat * rr / 4, cb, cc,
                                                                                  bm);
       }
       if (!tall)
@@ -1554,7 +1554,7 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
       {
         ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 6);
         ++g_launches;
-        muon_combine_bf16_kernel<<<grid1(nmat * n / 4), MUON_THREADS, 0, st>>>(x, p16, nmat * n / 4, ca, 1.f, xn);
+        launch_pdl(muon_combine_bf16_kernel, grid1(nmat * n / 4), MUON_THREADS, 0, st, x, p16, nmat * n / 4, ca, 1.f, xn);
       }
       LAUNCH_CHECK();
       std::swap(x, xn);
@@ -1564,7 +1564,7 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
     {
       ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 12);
       ++g_launches;
-      muon_batch_apply_kernel<<<dim3(per_mat, nmat), MUON_THREADS, 0, st>>>(P, Plp, x, grp, step);
+      launch_pdl(muon_batch_apply_kernel, dim3(per_mat, nmat), MUON_THREADS, 0, st, P, Plp, x, grp, step);
     }
     LAUNCH_CHECK();
     // the next group starts from the scratch's first iterate buffer again
@@ -1588,8 +1588,8 @@ static int optimizer_step_impl(gpt_model* m, float lr) {
     m->micro = 0;
     m->step_t += 1;
     if (c.grad_clip > 0.f) {
-      ++g_launches; sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, st>>>(m->at<float>(p.G), p.dense_n, m->at<double>(p.norm_part));
-      ++g_launches; clip_coef_kernel<<<1, 256, 0, st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, c.grad_clip,
+      ++g_launches; launch_pdl(sumsq_partial_kernel, NORM_BLOCKS, 256, 0, st, m->at<float>(p.G), p.dense_n, m->at<double>(p.norm_part));
+      ++g_launches; launch_pdl(clip_coef_kernel, 1, 256, 0, st, m->at<double>(p.norm_part), NORM_BLOCKS, c.grad_clip,
                                          m->at<float>(p.clip_coef), m->at<float>(p.grad_norm), err);
       LAUNCH_CHECK();
       coef = m->at<float>(p.clip_coef);
@@ -1650,9 +1650,9 @@ extern "C" int gpt_grad_sumsq(gpt_model* m, long long lo, long long hi, double* 
   if (!m || !out_dev || lo < 0 || hi < lo || hi > m->plan.dense_n)
     return fail(GPT_ERR_ARG, "gpt_grad_sumsq: bad range");
   const Plan& p = m->plan;
-  ++g_launches; sumsq_partial_kernel<<<NORM_BLOCKS, 256, 0, m->st>>>(m->at<float>(p.G) + lo, hi - lo,
+  ++g_launches; launch_pdl(sumsq_partial_kernel, NORM_BLOCKS, 256, 0, m->st, m->at<float>(p.G) + lo, hi - lo,
                                                                       m->at<double>(p.norm_part));
-  ++g_launches; sum_partials_kernel<<<1, 256, 0, m->st>>>(m->at<double>(p.norm_part), NORM_BLOCKS, out_dev);
+  ++g_launches; launch_pdl(sum_partials_kernel, 1, 256, 0, m->st, m->at<double>(p.norm_part), NORM_BLOCKS, out_dev);
   LAUNCH_CHECK();
   return GPT_OK;
 }
@@ -1677,7 +1677,7 @@ extern "C" int gpt_optimizer_step_range(gpt_model* m, float lr, long long lo, lo
   m->step_t += 1;
   float* coef = nullptr;
   if (c.grad_clip > 0.f) {
-    ++g_launches; clip_coef_kernel<<<1, 256, 0, st>>>(grad_sumsq_dev, 1, c.grad_clip, m->at<float>(p.clip_coef),
+    ++g_launches; launch_pdl(clip_coef_kernel, 1, 256, 0, st, grad_sumsq_dev, 1, c.grad_clip, m->at<float>(p.clip_coef),
                                                        m->at<float>(p.grad_norm), m->err());
     coef = m->at<float>(p.clip_coef);
   }
@@ -1750,7 +1750,7 @@ extern "C" int ngram_hash(const int32_t* tokens, int B, int T, int vocab, unsign
   if ((long long)B * T == 0) return GPT_OK;
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
-  ++g_launches; ngram_hash_kernel<<<grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream>>>(
+  ++g_launches; launch_pdl(ngram_hash_kernel, grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream, 
       tokens, B, T, vocab, p1, p2, rows, rows_out, 1, nullptr, err);
   LAUNCH_CHECK();
   return GPT_OK;
@@ -1767,13 +1767,13 @@ extern "C" int ngram_gather(const int32_t* rows, int n, const void* table, long 
   const bool vec16 = d % 8 == 0 && (reinterpret_cast<uintptr_t>(table) & 15) == 0 &&
                      (reinterpret_cast<uintptr_t>(out) & 15) == 0;
   if (dtype == GPT_DTYPE_BF16 && vec16) {
-    ++g_launches; ngram_gather_bf16x8_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows,
+    ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid, 256, 0, (cudaStream_t)stream, rows, n, (const bf16*)table, n_rows,
                                                                       d, (bf16*)out, accumulate, err);
   } else if (dtype == GPT_DTYPE_BF16) {
-    ++g_launches; ngram_gather_kernel<bf16><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const bf16*)table, n_rows, d,
+    ++g_launches; launch_pdl(ngram_gather_kernel<bf16>, grid, 256, 0, (cudaStream_t)stream, rows, n, (const bf16*)table, n_rows, d,
                                                                       (bf16*)out, accumulate, err);
   } else if (dtype == GPT_DTYPE_F32) {
-    ++g_launches; ngram_gather_kernel<float><<<grid, 256, 0, (cudaStream_t)stream>>>(rows, n, (const float*)table, n_rows, d,
+    ++g_launches; launch_pdl(ngram_gather_kernel<float>, grid, 256, 0, (cudaStream_t)stream, rows, n, (const float*)table, n_rows, d,
                                                                        (float*)out, accumulate, err);
   } else {
     return fail(GPT_ERR_ARG, "ngram_gather: dtype must be F32 or BF16");

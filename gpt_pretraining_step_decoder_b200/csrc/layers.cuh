@@ -468,6 +468,7 @@ __global__ void __launch_bounds__(256) ce_prob_kernel(bf16* __restrict__ ez, con
 // Counts non-ignored targets and sets scale = 1/(count * A) (single block).
 __global__ void ce_prepare_kernel(const int32_t* __restrict__ targets, int N, int A,
                                   float* __restrict__ scale_out, int* __restrict__ count_out) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ float sh[32];
   float c = 0.f;
   for (int i = threadIdx.x; i < N; i += blockDim.x) c += (targets[i] >= 0) ? 1.f : 0.f;
@@ -483,6 +484,7 @@ __global__ void ce_prepare_kernel(const int32_t* __restrict__ targets, int N, in
 __global__ void loss_reduce_kernel(const float* __restrict__ tok_loss, int N,
                                    const int* __restrict__ count, float* __restrict__ loss_out,
                                    unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ double sh[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < N; i += blockDim.x) s += tok_loss[i];

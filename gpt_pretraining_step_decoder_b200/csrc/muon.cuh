@@ -137,6 +137,7 @@ __device__ __forceinline__ long long muon_off(const MuonGroup& g, int j) {
 __global__ void __launch_bounds__(MUON_THREADS) muon_batch_momentum_kernel(
     const float* __restrict__ Gall, float* __restrict__ Mall, MuonGroup grp, float mu, int nesterov,
     const float* __restrict__ clip, float* __restrict__ partials) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ float wsum[MUON_THREADS / 32];
   const int j = blockIdx.y;
   const long long off = muon_off(grp, j);
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(MUON_THREADS) muon_batch_momentum_kernel(
 __global__ void __launch_bounds__(MUON_THREADS) muon_batch_normalize_kernel(
     const float* __restrict__ Gall, const float* __restrict__ Mall, MuonGroup grp, float mu, int nesterov,
     const float* __restrict__ clip, const float* __restrict__ partials, float eps, bf16* __restrict__ Xall) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ float inv_norm;
   const int j = blockIdx.y;
   if (threadIdx.x < 32) {
@@ -204,6 +206,7 @@ __global__ void __launch_bounds__(MUON_THREADS) muon_batch_apply_kernel(float* _
                                                                         bf16* __restrict__ Wlp_all,
                                                                         const bf16* __restrict__ Xall,
                                                                         MuonGroup grp, float step) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int j = blockIdx.y;
   const long long off = muon_off(grp, j);
   float* W = Wall + off;
@@ -231,6 +234,7 @@ __global__ void __launch_bounds__(MUON_THREADS) muon_batch_apply_kernel(float* _
 __global__ void __launch_bounds__(MUON_THREADS) muon_combine_bf16_kernel(const bf16* __restrict__ x,
                                                                          const bf16* __restrict__ y, long long n4,
                                                                          float a, float c, bf16* __restrict__ out) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     float xv[4], yv[4];
     load4(x + 4 * i, xv);

@@ -48,6 +48,7 @@ __global__ void ngram_hash_kernel(const int32_t* __restrict__ tok, int B, int T,
                                   unsigned long long p1, unsigned long long p2, long long rows_a,
                                   int32_t* __restrict__ out_a, long long rows_b,
                                   int32_t* __restrict__ out_b, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= (long long)B * T) return;
   const int t = (int)(n % T);
@@ -69,6 +70,7 @@ template <typename tab_t>
 __global__ void ngram_gather_kernel(const int32_t* __restrict__ rows, int n,
                                     const tab_t* __restrict__ table, long long n_rows, int d,
                                     tab_t* __restrict__ out, int accumulate, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= n) return;
   const long long r = rows[warp];
@@ -93,6 +95,7 @@ __global__ void ngram_gather_kernel(const int32_t* __restrict__ rows, int n,
 __global__ void ngram_gather_bf16x8_kernel(const int32_t* __restrict__ rows, int n,
                                            const bf16* __restrict__ table, long long n_rows, int d,
                                            bf16* __restrict__ out, int accumulate, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= n) return;
   const long long r = rows[warp];
@@ -141,6 +144,7 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_hist_kernel(const uint32_
                                                                   const int32_t* __restrict__ raw, int n,
                                                                   long long key_range, int items, int shift,
                                                                   uint32_t* __restrict__ counts) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   constexpr int NW = RADIX_THREADS / 32;
   __shared__ uint32_t wh[NW][256];  // per-warp digit counts
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -179,6 +183,7 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_hist_kernel(const uint32_
 // exclusive scan of the counts taken digit-major: all blocks of digit 0, then
 // digit 1, ...).  One block; each thread scans a contiguous stretch.
 __global__ void __launch_bounds__(1024) radix_offsets_kernel(uint32_t* __restrict__ counts, int nblk) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ uint32_t sh[1024];
   const long long n = 256LL * nblk;
   const long long per = (n + 1023) / 1024;
@@ -212,6 +217,7 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_scatter_kernel(
     const uint32_t* __restrict__ keys_in, const int32_t* __restrict__ vals_in, const int32_t* __restrict__ raw,
     int n, long long key_range, int items, int shift, const uint32_t* __restrict__ counts, int scanned,
     uint32_t* __restrict__ keys_out, int32_t* __restrict__ vals_out, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   constexpr int NW = RADIX_THREADS / 32;
   __shared__ uint32_t wcount[NW][256];
   __shared__ uint32_t running[256];
@@ -295,6 +301,7 @@ __global__ void __launch_bounds__(RADIX_THREADS) radix_scatter_kernel(
 __global__ void __launch_bounds__(1024) unique_keys_kernel(const uint32_t* __restrict__ skeys, int n,
                                                            long long key_range, int32_t* __restrict__ uniq_out,
                                                            int* __restrict__ n_uniq_out) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ int sh[1024];
   const int per = (n + 1023) / 1024;
   const int beg = threadIdx.x * per, end = min(beg + per, n);
@@ -544,6 +551,7 @@ __global__ void __launch_bounds__(MAXT) table_chunk_kernel(
     tab_t* __restrict__ table, float* __restrict__ state, int d, const float* __restrict__ grad,
     const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n, long long n_rows,
     float* __restrict__ part_head, float* __restrict__ part_tail, float lr, float beta, float eps) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   static_assert(CHUNK == 16, "warp_sum16 reduces one value per position of a chunk");
   static_assert(MAXT <= 512, "ss_sh holds 16 warps");
   using raw_t = typename Raw4<tab_t>::type;
@@ -713,6 +721,7 @@ __global__ void __launch_bounds__(CHAIN_WARPS * 32, NV <= 6 ? 2 : 1) table_chain
     tab_t* __restrict__ table, float* __restrict__ state, int d, const uint32_t* __restrict__ skeys, int n,
     long long n_rows, const float* __restrict__ part_head, const float* __restrict__ part_tail, float lr,
     float beta, float eps) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   extern __shared__ float chain_sh[];
   __shared__ int flag[CHAIN_WARPS], lastc[CHAIN_WARPS];
   __shared__ uint32_t keyc[CHAIN_WARPS];
@@ -750,6 +759,7 @@ __global__ void __launch_bounds__(128, NV <= 6 ? 5 : (NV <= 8 ? 4 : 2)) emb_chun
     float* __restrict__ dwte, const w_t* __restrict__ wte, int d, const float* __restrict__ dx0,
     const float* __restrict__ rstd, const uint32_t* __restrict__ skeys, const int32_t* __restrict__ perm, int n,
     long long vocab, float* __restrict__ part_head, float* __restrict__ part_tail) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const int c = (int)(((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if ((long long)c * CHUNK >= n) return;
   constexpr int TAB_U = 1;  // positions a step: one keeps the kernel near 80 registers, 20 warps an SM
@@ -821,6 +831,7 @@ __global__ void __launch_bounds__(CHAIN_WARPS * 32, NV <= 6 ? 2 : 1) emb_chain_k
                                                                        long long vocab,
                                                                        const float* __restrict__ part_head,
                                                                        const float* __restrict__ part_tail) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   extern __shared__ float chain_sh[];
   __shared__ int flag[CHAIN_WARPS], lastc[CHAIN_WARPS];
   __shared__ uint32_t keyc[CHAIN_WARPS];
@@ -866,6 +877,7 @@ __device__ __forceinline__ unsigned long long trigram_key(int a2, int a1, int c,
 __global__ void trigram_hash_kernel(const int32_t* __restrict__ tok, int B, int T, int V, unsigned long long p1,
                                     unsigned long long p2, unsigned long long p3, long long rows,
                                     int32_t* __restrict__ out, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= (long long)B * T) return;
   const int t = (int)(n % T);
@@ -922,6 +934,7 @@ __global__ void trigram_normalize_kernel(const unsigned* __restrict__ counts, lo
 template <typename act_t>
 __global__ void value_bias_kernel(const float* __restrict__ p3, const act_t* __restrict__ hv,
                                   const int32_t* __restrict__ rv, long long N, int a, act_t* __restrict__ vb) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   const long long total4 = N * a / 4;
   for (long long i4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; i4 < total4;
        i4 += (long long)gridDim.x * blockDim.x) {

@@ -42,6 +42,7 @@ __global__ void adamw_kernel(AdamArgs a) {
 // block sums the partials in order and forms min(1, clip / (norm + 1e-6)).
 constexpr int NORM_BLOCKS = 1024;
 __global__ void sumsq_partial_kernel(const float* __restrict__ g, long long n, double* __restrict__ part) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ double sh[32];
   double s = 0.0;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -61,6 +62,7 @@ __global__ void sumsq_partial_kernel(const float* __restrict__ g, long long n, d
 }
 __global__ void clip_coef_kernel(const double* __restrict__ part, int nparts, float max_norm,
                                  float* __restrict__ coef, float* __restrict__ norm_out, unsigned* err) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ double sh[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
@@ -80,6 +82,7 @@ __global__ void clip_coef_kernel(const double* __restrict__ part, int nparts, fl
 
 // *out = sum of the partials in order (one block)
 __global__ void sum_partials_kernel(const double* __restrict__ part, int nparts, double* __restrict__ out) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   __shared__ double sh[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
@@ -96,6 +99,7 @@ __global__ void sum_partials_kernel(const double* __restrict__ part, int nparts,
 
 // fp32 master -> bf16 copy (round to nearest even).
 __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long long n) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x)
     dst[i] = __float2bfloat16_rn(src[i]);
