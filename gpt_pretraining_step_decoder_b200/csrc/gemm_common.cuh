@@ -28,6 +28,8 @@ enum EpiMode {
   EPI_QKV = 6,        // fused q|k|v projection output (tensor-core path, 128-wide heads):
                       // q, k heads rotated (RoPE) and RMS-normalised per head, v heads plus
                       // the value-table row; C(act) = result
+  EPI_AXPBY = 7,      // C(act) = alpha * acc + aux_scale * aux(act), aux of C's shape and ld
+                      // (the Newton-Schulz polynomial's combinations; tensor-core path)
 };
 
 struct GemmEpilogue {
@@ -35,7 +37,7 @@ struct GemmEpilogue {
   void* C;          // output [M, ldc]
   long long ldc;
   void* C2;         // unused second output
-  const void* aux;  // EPI_DRELU2 input relu(a)^2, same ld as C
+  const void* aux;  // EPI_DRELU2 input relu(a)^2, EPI_AXPBY input; same ld as C
   float alpha;
   int beta;
   float softcap;    // EPI_LOGITS: 0 = off, else z = softcap * tanh(acc / softcap)
@@ -54,6 +56,7 @@ struct GemmEpilogue {
   // FP8 path: acc is further multiplied by *scale_a * *scale_b (device scalars; null = 1)
   const float* scale_a;
   const float* scale_b;
+  float aux_scale;  // EPI_AXPBY
 };
 
 template <typename act_t>
@@ -77,6 +80,11 @@ __device__ __forceinline__ void epi_apply_one(const GemmEpilogue& e, long long m
     case EPI_DRELU2: {
       const float g = to_f(reinterpret_cast<const act_t*>(e.aux)[off]);
       reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(2.f * sqrtf(g) * acc);
+      break;
+    }
+    case EPI_AXPBY: {
+      const float g = to_f(reinterpret_cast<const act_t*>(e.aux)[off]);
+      reinterpret_cast<act_t*>(e.C)[off] = from_f<act_t>(acc + e.aux_scale * g);
       break;
     }
     default:  // EPI_LOGITS and EPI_QKV exist only in the tensor-core kernel's epilogue

@@ -66,17 +66,19 @@ enum KMode {
   K_DRELU2,       // bf16 2 sqrt(aux) acc
   K_LOGITS,       // bf16 exp(z - tile max), z = softcap(acc), + per-tile row statistics
   K_QKV,          // bf16 q|k|v with RoPE + QK-norm (+ value-table row) per 128-wide head
+  K_AXPBY,        // bf16 acc + aux_scale * aux (aux streamed like the ReLU^2 backward's)
 };
 
 // The ReLU^2-backward epilogue streams activations through a ring of its
 // own, which costs a pipeline stage; every other epilogue uses the light
 // configuration.  Host and kernel both take the configuration from here.
 template <int KM> struct KmHeavy {
-  static constexpr int value = KM == K_DRELU2 ? 1 : 0;
+  static constexpr int value = (KM == K_DRELU2 || KM == K_AXPBY) ? 1 : 0;
 };
 
-// HEAVY = 1 (ReLU^2 backward) trades one pipeline stage for each epilogue
-// warp's two activation blocks (its whole half tile), which also serve as its
+// HEAVY = 1 (ReLU^2 backward, the Newton-Schulz combinations) trades one
+// pipeline stage for each epilogue warp's two input blocks (its whole half
+// tile of the second input), which also serve as its
 // output staging; the other epilogues stage through one block per warp.
 // BN = 128, 192 or 256 (192 only with fp32 outputs: 96 columns per epilogue
 // warp = three 32-column fp32 blocks); the ring takes what shared memory has
@@ -669,7 +671,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float ealpha = e.alpha;
     if constexpr (F8) ealpha *= (e.scale_a ? *e.scale_a : 1.f) * (e.scale_b ? *e.scale_b : 1.f);
     constexpr bool f32out = KM == K_STORE_F32 || KM == K_REDUCE_F32 || KM == K_PARTIAL;
-    constexpr bool has_aux = KM == K_DRELU2;
+    constexpr bool has_aux = KM == K_DRELU2 || KM == K_AXPBY;
     constexpr int CW = f32out ? 32 : 64;  // columns per 128-byte staging row
     static_assert(!has_aux || HALF / CW <= C::NAUX, "one activation block per column block");
     int acc = 0;
@@ -698,7 +700,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int b = 0; b < nblk; ++b) {
           if (lane == 0) {
             mbar_expect_tx(&abar[b], AUX_BYTES);
-            tma_load_2d(auxs + b * AUX_BYTES, &tmAux, &abar[b], n0 + b * 64, mrow0);
+            if constexpr (B3) tma_load_3d(auxs + b * AUX_BYTES, &tmAux, &abar[b], n0 + b * 64, mrow0, z);
+            else tma_load_2d(auxs + b * AUX_BYTES, &tmAux, &abar[b], n0 + b * 64, mrow0);
           }
           aux_pending |= 1u << b;
         }
@@ -715,7 +718,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // The logits and ReLU^2-backward epilogues hold fewer registers: they
       // read a block at a time and release the accumulator at the tile's end
       // (holding the whole half tile spilled and measured slower there).
-      constexpr bool PRE = KM != K_QKV && KM != K_LOGITS && KM != K_DRELU2;
+      constexpr bool PRE = KM != K_QKV && KM != K_LOGITS && KM != K_DRELU2 && KM != K_AXPBY;
       float accr[PRE ? HALF : 1];
       if constexpr (PRE) {
         uint32_t r[HALF / 32][32];
@@ -896,6 +899,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const float2 gg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
               v[j * 8 + 2 * h] *= gg.x > 0.f ? 2.f * gg.x * rsqrtf(gg.x) : 0.f;
               v[j * 8 + 2 * h + 1] *= gg.y > 0.f ? 2.f * gg.y * rsqrtf(gg.y) : 0.f;
+            }
+          }
+        } else if constexpr (KM == K_AXPBY) {
+          if (!warp_wait(&abar[c], (aux_phase >> c) & 1u, abort_flag, p.err)) return false;
+          aux_phase ^= 1u << c;
+          aux_pending &= ~(1u << c);
+          stg = auxs + c * AUX_BYTES;  // each lane rewrites only its own row below
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(stg + swz128(lane, j));
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 gg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+              v[j * 8 + 2 * h] = fmaf(e.aux_scale, gg.x, v[j * 8 + 2 * h]);
+              v[j * 8 + 2 * h + 1] = fmaf(e.aux_scale, gg.y, v[j * 8 + 2 * h + 1]);
             }
           }
         }

@@ -265,8 +265,8 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
                           const GemmBatch& bt = GemmBatch()) {
   static_assert(CG == 1 || BN == 256, "CTA pairs take 256-column tiles");
   const bool b3 = bt.n > 1;
-  if (b3 && (splits > 1 || (e.mode != EPI_STORE && e.mode != EPI_STORE_F32)))
-    return fail(GPT_ERR_ARG, "batched GEMMs take store epilogues without split-K");
+  if (b3 && (splits > 1 || (e.mode != EPI_STORE && e.mode != EPI_STORE_F32 && e.mode != EPI_AXPBY)))
+    return fail(GPT_ERR_ARG, "batched GEMMs take store or AXPBY epilogues without split-K");
   CUtensorMap ta, tb, tcm, taux;
   if (b3) {
     if (A.kmajor) TRY(make_tmap3(&ta, A.ptr, K, M, A.ld, bt.n, bt.sa, tc::BK, tc::BM));
@@ -318,8 +318,13 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   } else {
     TRY(make_tmap(&tcm, e.C, N, M, e.ldc, 64, 32));
   }
-  if (p.splits == 1 && e.mode == EPI_DRELU2) TRY(make_tmap(&taux, e.aux, N, M, e.ldc, 64, 32));
-  else taux = tcm;
+  if (p.splits == 1 && (e.mode == EPI_DRELU2 || e.mode == EPI_AXPBY)) {
+    if (!e.aux) return fail(GPT_ERR_ARG, "this epilogue needs its second input");
+    if (b3) TRY(make_tmap3(&taux, e.aux, N, M, e.ldc, bt.n, bt.sc, 64, 32));
+    else TRY(make_tmap(&taux, e.aux, N, M, e.ldc, 64, 32));
+  } else {
+    taux = tcm;
+  }
   int km;
   if (p.splits > 1) km = tc::K_PARTIAL;
   else if (e.mode == EPI_STORE) km = tc::K_STORE;
@@ -328,11 +333,13 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   else if (e.mode == EPI_RELU2) km = tc::K_RELU2;
   else if (e.mode == EPI_DRELU2) km = tc::K_DRELU2;
   else if (e.mode == EPI_QKV) km = tc::K_QKV;
+  else if (e.mode == EPI_AXPBY) km = tc::K_AXPBY;
   else km = tc::K_LOGITS;
   if (km == tc::K_QKV && BN != 256) return fail(GPT_ERR_ARG, "QKV epilogue needs 256-column tiles (N >= 256)");
   if (b3) {
     // batched products: their own kernel instances (the third tensor-map coordinate)
     if (km == tc::K_STORE_F32) TRY((gemm_tc_launch_k<BN, tc::K_STORE_F32, CG, 0, true>(ta, tb, tcm, taux, p, st)));
+    else if (km == tc::K_AXPBY) TRY((gemm_tc_launch_k<BN, tc::K_AXPBY, CG, 0, true>(ta, tb, tcm, taux, p, st)));
     else TRY((gemm_tc_launch_k<BN, tc::K_STORE, CG, 0, true>(ta, tb, tcm, taux, p, st)));
     return GPT_OK;
   }
@@ -352,6 +359,7 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
     case tc::K_RELU2: TRY((gemm_tc_launch_k<BN, tc::K_RELU2, CG>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_DRELU2: TRY((gemm_tc_launch_k<BN, tc::K_DRELU2, CG>(ta, tb, tcm, taux, p, st))); break;
     case tc::K_QKV: TRY((gemm_tc_launch_k<BN, tc::K_QKV, CG>(ta, tb, tcm, taux, p, st))); break;
+    case tc::K_AXPBY: TRY((gemm_tc_launch_k<BN, tc::K_AXPBY, CG>(ta, tb, tcm, taux, p, st))); break;
     default: TRY((gemm_tc_launch_k<BN, tc::K_LOGITS, CG>(ta, tb, tcm, taux, p, st))); break;
   }
   }
@@ -528,6 +536,7 @@ static GemmEpilogue epi(int mode, void* C, long long ldc, int beta = 0, void* C2
   e.softcap = 0.f; e.stats = nullptr; e.targets = nullptr; e.ztgt = nullptr;
   e.rope = nullptr; e.rstd_q = e.rstd_k = nullptr; e.hv = nullptr; e.rv = nullptr;
   e.scale_a = e.scale_b = nullptr;
+  e.aux_scale = 0.f;
   e.T = e.H = e.qk_norm = 0; e.eps = 0.f;
   return e;
 }
@@ -572,7 +581,7 @@ struct Plan {
   // same-shape groups and one scratch sized for the largest group
   MuonGroup muon_groups[3];
   int n_muon_groups = 0;
-  size_t mu_x, mu_xn, mu_abf, mu_bm, mu_aa, mu_p, mu_part;
+  size_t mu_x, mu_xn, mu_abf, mu_bm, mu_part;
   int chunk;
   size_t total;
 };
@@ -746,8 +755,6 @@ static void make_plan(const gpt_config& c, Plan& p) {
     }
     p.mu_x = cv.take(xn * 2); p.mu_xn = cv.take(xn * 2);
     p.mu_abf = cv.take(rr * 2); p.mu_bm = cv.take(rr * 2);
-    p.mu_aa = cv.take(rr * 2);   // A A (bf16)
-    p.mu_p = cv.take(xn * 2);    // B X (bf16)
     p.mu_part = cv.take(nm * MUON_BATCH_BLOCKS * 4);
   }
   p.total = cv.take(0) + 256;
@@ -1074,7 +1081,7 @@ static int launch_table_chunk(tab_t* table, float* state, int d, const float* gr
     attr = true;
   }
   ++g_launches;
-  launch_pdl(table_chunk_kernel<tab_t, MAXT, STAGE>, (unsigned)nchunks, nt, table_chunk_smem<tab_t>(nt, STAGE), st, 
+  launch_pdl(table_chunk_kernel<tab_t, MAXT, STAGE>, (unsigned)nchunks, nt, table_chunk_smem<tab_t>(nt, STAGE), st,
       table, state, d, grad, skeys, perm, n, n_rows, w.part_head, w.part_tail, lr, beta, eps);
   return GPT_OK;
 }
@@ -1100,7 +1107,7 @@ static int table_update(const SortWs& w, tab_t* table, float* state, long long n
   const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;  // <= 56 KB (d <= 2048)
   const unsigned chain_grid = (unsigned)((nchunks + CHAIN_WARPS - 1) / CHAIN_WARPS);
   WITH_NV(d, TRY(allow_smem(table_chain_kernel<NV, tab_t>, chain_smem)); ++g_launches;
-          launch_pdl(table_chain_kernel<NV, tab_t>, chain_grid, CHAIN_WARPS * 32, chain_smem, st, 
+          launch_pdl(table_chain_kernel<NV, tab_t>, chain_grid, CHAIN_WARPS * 32, chain_smem, st,
               table, state, d, skeys, n, n_rows, w.part_head, w.part_tail, lr, beta, eps););
   LAUNCH_CHECK();
   return GPT_OK;
@@ -1210,7 +1217,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
   CUDA_TRY(cudaMemcpyAsync(m->at<int32_t>(p.tok_copy), tokens, (size_t)N * 4, cudaMemcpyDeviceToDevice, st));
   if (c.x0_rows || c.v_rows) {
     ProfScope ps(pf, st, "ngram_hash", 0.0, (double)N * 12);
-    ++g_launches; launch_pdl(ngram_hash_kernel, grid_for(N, 256), 256, 0, st, 
+    ++g_launches; launch_pdl(ngram_hash_kernel, grid_for(N, 256), 256, 0, st,
         tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.x0_rows ? c.x0_rows : 1,
         c.x0_rows ? m->at<int32_t>(p.rows_x) : nullptr, c.v_rows ? c.v_rows : 1,
         c.v_rows ? m->at<int32_t>(p.rows_v) : nullptr, err);
@@ -1224,17 +1231,17 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     const int w3 = c.tri_width;
     {
       ProfScope ps(pf, st, "trigram_gather", 0.0, (double)N * (12 + 2.0 * w3 * es));
-      ++g_launches; launch_pdl(trigram_hash_kernel, grid_for(N, 256), 256, 0, st, 
+      ++g_launches; launch_pdl(trigram_hash_kernel, grid_for(N, 256), 256, 0, st,
           tokens, c.micro_batch, c.seq_len, V, c.hash_p1, c.hash_p2, c.hash_p3, c.tri_rows,
           m->at<int32_t>(p.rows_3), err);
       const act_t* h3 = reinterpret_cast<const act_t*>(m->base + p.h3);
       act_t* s3g = m->at<act_t>(p.s3g);
       if (b16) {
-        ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid_for((long long)N * 32, 256), 256, 0, st, 
+        ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid_for((long long)N * 32, 256), 256, 0, st,
             m->at<int32_t>(p.rows_3), N, reinterpret_cast<const bf16*>(h3), c.tri_rows, w3,
             reinterpret_cast<bf16*>(s3g), 0, err);
       } else {
-        ++g_launches; launch_pdl(ngram_gather_kernel<act_t>, grid_for((long long)N * 32, 256), 256, 0, st, 
+        ++g_launches; launch_pdl(ngram_gather_kernel<act_t>, grid_for((long long)N * 32, 256), 256, 0, st,
             m->at<int32_t>(p.rows_3), N, h3, c.tri_rows, w3, s3g, 0, err);
       }
       LAUNCH_CHECK();
@@ -1243,7 +1250,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
              epi(EPI_STORE_F32, m->at<float>(p.p3), a), false, "gemm.vproj_fwd"));
     {
       ProfScope ps(pf, st, "value_bias", 0.0, (double)N * a * (4 + es + (c.v_rows ? es : 0)));
-      ++g_launches; launch_pdl(value_bias_kernel<act_t>, 4 * device_sms(), 256, 0, st, 
+      ++g_launches; launch_pdl(value_bias_kernel<act_t>, 4 * device_sms(), 256, 0, st,
           m->at<float>(p.p3), vbias, vrows, N, a, m->at<act_t>(p.vb));
       LAUNCH_CHECK();
     }
@@ -1447,12 +1454,12 @@ static int backward_impl(gpt_model* m, float lr, bool do_step) {
     const int32_t* perm;
     TRY(bucket_by_key(w, m->at<int32_t>(p.tok_copy), N, V, &skeys, &perm, nullptr, nullptr, err, st));
     const long long nchunks = (N + CHUNK - 1) / CHUNK;
-    WITH_NV(d, ++g_launches; launch_pdl(emb_chunk_kernel<NV, act_t>, grid_for(nchunks * 32, 128), 128, 0, st, 
+    WITH_NV(d, ++g_launches; launch_pdl(emb_chunk_kernel<NV, act_t>, grid_for(nchunks * 32, 128), 128, 0, st,
         Gp("wte"), W("wte"), d, dx, m->at<float>(p.emb_rstd), skeys, perm, N, V, w.part_head, w.part_tail););
     const size_t chain_smem = (size_t)(CHAIN_WARPS - 1) * d * 4;
     const unsigned chain_grid = (unsigned)((nchunks + CHAIN_WARPS - 1) / CHAIN_WARPS);
     WITH_NV(d, TRY(allow_smem(emb_chain_kernel<NV>, chain_smem)); ++g_launches;
-            launch_pdl(emb_chain_kernel<NV>, chain_grid, CHAIN_WARPS * 32, chain_smem, st, 
+            launch_pdl(emb_chain_kernel<NV>, chain_grid, CHAIN_WARPS * 32, chain_smem, st,
                 Gp("wte"), d, skeys, N, V, w.part_head, w.part_tail););
     LAUNCH_CHECK();
   }
@@ -1503,8 +1510,6 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
   bf16* xn = m->at<bf16>(p.mu_xn);
   bf16* abf = m->at<bf16>(p.mu_abf);
   bf16* bm = m->at<bf16>(p.mu_bm);
-  bf16* aa16 = m->at<bf16>(p.mu_aa);  // A A
-  bf16* p16 = m->at<bf16>(p.mu_p);    // B X (X B)
   float* part = m->at<float>(p.mu_part);
   const GemmCtx g{true, m->at<float>(p.splitk), p.splitk_elems, m->err(), st, &m->prof};
   const float ca = 3.4445f, cb = -4.7750f, cc = 2.0315f;  // a x + b x^3 + c x^5
@@ -1523,10 +1528,10 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
       // bytes: g, m read + m written; g, m read + bf16 iterate written
       ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * (12 + 10));
       ++g_launches;
-      launch_pdl(muon_batch_momentum_kernel, dim3(MUON_BATCH_BLOCKS, nmat), MUON_THREADS, 0, st, 
+      launch_pdl(muon_batch_momentum_kernel, dim3(MUON_BATCH_BLOCKS, nmat), MUON_THREADS, 0, st,
           G, M, grp, c.muon_momentum, c.muon_nesterov, clip, part);
       ++g_launches;
-      launch_pdl(muon_batch_normalize_kernel, dim3(per_mat, nmat), MUON_THREADS, 0, st, 
+      launch_pdl(muon_batch_normalize_kernel, dim3(per_mat, nmat), MUON_THREADS, 0, st,
           G, M, grp, c.muon_momentum, c.muon_nesterov, clip, part, 1e-7f, x);
       LAUNCH_CHECK();
     }
@@ -1537,25 +1542,19 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
       else
         TRY(gemm_batched(g, GemmBatch{nmat, n, n, rr}, R, R, rows, op_mn(x, cols), op_mn(x, cols),
                          epi(EPI_STORE, abf, R), "muon.gram"));
-      TRY(gemm_batched(g, GemmBatch{nmat, rr, rr, rr}, R, R, R, op_k(abf, R), op_mn(abf, R),
-                       epi(EPI_STORE, aa16, R), "muon.square"));
-      {
-        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * rr * 6);
-        ++g_launches;
-        launch_pdl(muon_combine_bf16_kernel, grid1(nmat * rr / 4), MUON_THREADS, 0, st, abf, aa16, nmat * rr / 4, cb, cc,
-                                                                                 bm);
-      }
+      // B = b A + c A A, the combination taken in the square product's epilogue
+      GemmEpilogue esq = epi(EPI_AXPBY, bm, R, 0, nullptr, abf, cc);
+      esq.aux_scale = cb;
+      TRY(gemm_batched(g, GemmBatch{nmat, rr, rr, rr}, R, R, R, op_k(abf, R), op_mn(abf, R), esq, "muon.square"));
+      // X' = a X + B X (X B when tall), the combination in the product's epilogue
+      GemmEpilogue epo = epi(EPI_AXPBY, xn, cols, 0, nullptr, x, 1.f);
+      epo.aux_scale = ca;
       if (!tall)
-        TRY(gemm_batched(g, GemmBatch{nmat, rr, n, n}, rows, cols, R, op_k(bm, R), op_mn(x, cols),
-                         epi(EPI_STORE, p16, cols), "muon.poly"));
+        TRY(gemm_batched(g, GemmBatch{nmat, rr, n, n}, rows, cols, R, op_k(bm, R), op_mn(x, cols), epo,
+                         "muon.poly"));
       else
-        TRY(gemm_batched(g, GemmBatch{nmat, n, rr, n}, rows, cols, R, op_k(x, cols), op_mn(bm, R),
-                         epi(EPI_STORE, p16, cols), "muon.poly"));
-      {
-        ProfScope ps(&m->prof, st, "muon_elementwise", 0.0, (double)nmat * n * 6);
-        ++g_launches;
-        launch_pdl(muon_combine_bf16_kernel, grid1(nmat * n / 4), MUON_THREADS, 0, st, x, p16, nmat * n / 4, ca, 1.f, xn);
-      }
+        TRY(gemm_batched(g, GemmBatch{nmat, n, rr, n}, rows, cols, R, op_k(x, cols), op_mn(bm, R), epo,
+                         "muon.poly"));
       LAUNCH_CHECK();
       std::swap(x, xn);
     }
@@ -1750,7 +1749,7 @@ extern "C" int ngram_hash(const int32_t* tokens, int B, int T, int vocab, unsign
   if ((long long)B * T == 0) return GPT_OK;
   unsigned* err = nullptr;
   CUDA_TRY(cudaGetSymbolAddress((void**)&err, g_ngram_err));
-  ++g_launches; launch_pdl(ngram_hash_kernel, grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream, 
+  ++g_launches; launch_pdl(ngram_hash_kernel, grid_for((long long)B * T, 256), 256, 0, (cudaStream_t)stream,
       tokens, B, T, vocab, p1, p2, rows, rows_out, 1, nullptr, err);
   LAUNCH_CHECK();
   return GPT_OK;

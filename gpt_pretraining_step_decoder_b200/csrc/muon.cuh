@@ -229,17 +229,3 @@ __global__ void __launch_bounds__(MUON_THREADS) muon_batch_apply_kernel(float* _
   }
 }
 
-// out = bf16(a * x + c * y) with both inputs bf16 (the batched iteration keeps
-// every product in bf16, as the pages' bf16 iteration does)
-__global__ void __launch_bounds__(MUON_THREADS) muon_combine_bf16_kernel(const bf16* __restrict__ x,
-                                                                         const bf16* __restrict__ y, long long n4,
-                                                                         float a, float c, bf16* __restrict__ out) {
-  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
-    float xv[4], yv[4];
-    load4(x + 4 * i, xv);
-    load4(y + 4 * i, yv);
-    const float v[4] = {a * xv[0] + c * yv[0], a * xv[1] + c * yv[1], a * xv[2] + c * yv[2], a * xv[3] + c * yv[3]};
-    store4(out + 4 * i, v);
-  }
-}
