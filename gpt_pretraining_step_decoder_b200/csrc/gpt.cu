@@ -1237,7 +1237,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
       const act_t* h3 = reinterpret_cast<const act_t*>(m->base + p.h3);
       act_t* s3g = m->at<act_t>(p.s3g);
       if (b16) {
-        ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid_for((long long)N * 32, 256), 256, 0, st,
+        ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid_for((long long)(N + 1) / 2 * 32, 256), 256, 0, st,
             m->at<int32_t>(p.rows_3), N, reinterpret_cast<const bf16*>(h3), c.tri_rows, w3,
             reinterpret_cast<bf16*>(s3g), 0, err);
       } else {
@@ -1766,7 +1766,8 @@ extern "C" int ngram_gather(const int32_t* rows, int n, const void* table, long 
   const bool vec16 = d % 8 == 0 && (reinterpret_cast<uintptr_t>(table) & 15) == 0 &&
                      (reinterpret_cast<uintptr_t>(out) & 15) == 0;
   if (dtype == GPT_DTYPE_BF16 && vec16) {
-    ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid, 256, 0, (cudaStream_t)stream, rows, n, (const bf16*)table, n_rows,
+    // two rows a warp
+    ++g_launches; launch_pdl(ngram_gather_bf16x8_kernel, grid_for((long long)(n + 1) / 2 * 32, 256), 256, 0, (cudaStream_t)stream, rows, n, (const bf16*)table, n_rows,
                                                                       d, (bf16*)out, accumulate, err);
   } else if (dtype == GPT_DTYPE_BF16) {
     ++g_launches; launch_pdl(ngram_gather_kernel<bf16>, grid, 256, 0, (cudaStream_t)stream, rows, n, (const bf16*)table, n_rows, d,

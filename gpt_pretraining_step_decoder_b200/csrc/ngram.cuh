@@ -96,32 +96,57 @@ __global__ void ngram_gather_bf16x8_kernel(const int32_t* __restrict__ rows, int
                                            const bf16* __restrict__ table, long long n_rows, int d,
                                            bf16* __restrict__ out, int accumulate, unsigned* err) {
   pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
+  // two rows a warp, both rows' loads in flight before any store (a short
+  // call is bound by how much a warp has in flight, not by its instructions)
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= n) return;
-  const long long r = rows[warp];
-  if (r < 0 || r >= n_rows) {
-    if (lane == 0) set_error(err, GPT_EBIT_INPUT);
-    return;
-  }
-  const uint4* src = reinterpret_cast<const uint4*>(table + r * d);
-  uint4* dst = reinterpret_cast<uint4*>(out + (long long)warp * d);
-#pragma unroll 4
-  for (int c = lane; c < d / 8; c += 32) {
-    uint4 v = __ldg(src + c);
-    if (accumulate) {
-      const uint4 o = dst[c];
-      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
-      uint4 s;
-      __nv_bfloat162* s2 = reinterpret_cast<__nv_bfloat162*>(&s);
+  const int i0 = 2 * warp;
+  if (i0 >= n) return;
+  const int nr = min(2, n - i0);
+  long long r[2] = {0, 0};
+  bool ok[2] = {false, false};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 x = __bfloat1622float2(a2[i]), y = __bfloat1622float2(o2[i]);
-        s2[i] = __floats2bfloat162_rn(x.x + y.x, x.y + y.y);
-      }
-      v = s;
+  for (int u = 0; u < 2; ++u) {
+    if (u < nr) {
+      r[u] = rows[i0 + u];
+      ok[u] = r[u] >= 0 && r[u] < n_rows;
+      if (!ok[u] && lane == 0) set_error(err, GPT_EBIT_INPUT);
     }
-    dst[c] = v;
+  }
+  const int nc = d / 8;
+  for (int c0 = 0; c0 < nc; c0 += 32 * 4) {
+    uint4 v[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = c0 + lane + 32 * k;
+        if (ok[u] && c < nc) v[u][k] = __ldg(reinterpret_cast<const uint4*>(table + r[u] * d) + c);
+      }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!ok[u]) continue;
+      uint4* dst = reinterpret_cast<uint4*>(out + (long long)(i0 + u) * d);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = c0 + lane + 32 * k;
+        if (c >= nc) continue;
+        uint4 x = v[u][k];
+        if (accumulate) {
+          const uint4 o = dst[c];
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+          const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+          uint4 sum;
+          __nv_bfloat162* s2 = reinterpret_cast<__nv_bfloat162*>(&sum);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 xa = __bfloat1622float2(a2[i]), ya = __bfloat1622float2(o2[i]);
+            s2[i] = __floats2bfloat162_rn(xa.x + ya.x, xa.y + ya.y);
+          }
+          x = sum;
+        }
+        dst[c] = x;
+      }
+    }
   }
 }
 

@@ -97,10 +97,12 @@ def test_ngram_hash_rejects_bad_tokens(g):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_ngram_gather(g, dtype):
+@pytest.mark.parametrize("R,d,n", [(5000, 768, 1000), (3000, 136, 999), (300, 2048, 33)])
+def test_ngram_gather(g, dtype, R, d, n):
+    """Rows of any width (whole and partial 16-byte passes, two passes of a
+    warp), an odd number of rows (the bf16 kernel takes two a warp)."""
     import torch
     rng = np.random.default_rng(2)
-    R, d, n = 5000, 768, 1000
     tab = rng.standard_normal((R, d)).astype(np.float32)
     if dtype == "bf16":
         tab = round_to_bf16(tab)
