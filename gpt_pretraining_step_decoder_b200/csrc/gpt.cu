@@ -1513,10 +1513,6 @@ static int muon_step_impl(gpt_model* m, float lr, const float* clip) {
   float* part = m->at<float>(p.mu_part);
   const GemmCtx g{true, m->at<float>(p.splitk), p.splitk_elems, m->err(), st, &m->prof};
   const float ca = 3.4445f, cb = -4.7750f, cc = 2.0315f;  // a x + b x^3 + c x^5
-  auto grid1 = [](long long n4) {
-    const long long b = (n4 + MUON_THREADS - 1) / MUON_THREADS, cap = 4LL * device_sms();
-    return (unsigned)(b < 1 ? 1 : (b > cap ? cap : b));
-  };
   for (int gi = 0; gi < p.n_muon_groups; ++gi) {
     const MuonGroup& grp = p.muon_groups[gi];
     const int rows = grp.rows, cols = grp.cols, nmat = grp.nmat;
