@@ -44,9 +44,10 @@ struct GemmEpilogue {
   float2* stats;    // EPI_LOGITS: [M, n_tiles] (max, sum of exp(z - max))
   const int32_t* targets;  // EPI_LOGITS: target column per row (< 0: none), nullable
   float* ztgt;             // EPI_LOGITS: z at the target column per row
-  // EPI_QKV: rope table frequency-major [64, T, (cos, sin)], per-(row, head) rstd outputs,
-  // optional value table [rows, H*128] (bf16) and its row per position
-  const float* rope;
+  // EPI_QKV: RoPE turns per position of the 64 frequencies ([64] float2, an
+  // fp32 hi + lo pair each), per-(row, head) rstd outputs, optional value
+  // table [rows, H*128] (bf16) and its row per position
+  const float2* rope;
   float* rstd_q;
   float* rstd_k;
   const void* hv;

@@ -92,7 +92,8 @@ template <int BN, int HEAVY, int CG = 1> struct Cfg {
   static constexpr int NSTG = HEAVY ? 0 : 1;           // staging blocks per epilogue warp
   static constexpr int NAUX = 2;                       // activation blocks per epilogue warp (ReLU^2 bwd)
   static constexpr int AUX = HEAVY ? NAUX * 32 * 128 : 0;  // activation bytes per epilogue warp
-  static constexpr int FIXED = EPI_WARPS * (NSTG * 32 * 128 + AUX) + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int FIXED = EPI_WARPS * (NSTG * 32 * 128 + AUX) + 1024 /*align*/ + 512 /*barriers*/ +
+                               512 /*RoPE turns*/;
   static constexpr int STAGES = (232448 - FIXED) / STAGE_BYTES > 6 ? 6 : (232448 - FIXED) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED;
 };
@@ -498,6 +499,19 @@ __device__ __forceinline__ void mulsub2(float& y0, float& y1, float p0, float p1
 }
 __device__ __forceinline__ uint32_t swz128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
+// cos and sin of the RoPE angle t theta_f from the frequency's turns per
+// position u = hi + lo (an fp32 pair): t hi = p + e exactly (e = fma(t, hi,
+// -p)), the whole turns k = rint(p) drop out exactly, and the remaining
+// fraction of a turn, in [-1/2, 1/2], goes to the special-function unit's
+// sin / cos.  Absolute error ~1e-6 for positions below 2^16.
+__device__ __forceinline__ void rope_cos_sin(float tf, float2 u, float& c, float& s) {
+  const float p = tf * u.x;
+  const float e = fmaf(tf, u.x, -p);
+  const float k = rintf(p);
+  const float fr = (p - k) + fmaf(tf, u.y, e);
+  __sincosf(6.28318530717958648f * fr, &s, &c);
+}
+
 template <int BN, int KM, typename act_t, int CG, int F8 = 0, bool B3 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -521,8 +535,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* auxbar = tempty + 2;  // NAUX per epilogue warp
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(auxbar + EPI_WARPS * C::NAUX);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* sturns = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(full) + 512);  // [64]
+  static_assert((2 * C::STAGES + 4 + EPI_WARPS * C::NAUX) * 8 + 8 <= 512, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if constexpr (KM == K_QKV)
+    if (threadIdx.x < 64 && p.epi.rope != nullptr) sturns[threadIdx.x] = p.epi.rope[threadIdx.x];
   const int per_product = p.m_tiles * p.n_tiles * p.splits;
   const int tiles = B3 ? per_product * p.batch : per_product;
   // CTA pair: rank 0 issues the MMAs; tile t goes to pair blockIdx.x / CG
@@ -783,15 +801,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (sec < 2) {
             // RoPE ("$1000 tier nanochat run", apply_rotary_emb): y1 = x1 cos + x2 sin,
             // y2 = -x1 sin + x2 cos over the two halves of the head, then QK-norm;
-            // frequency-major table: consecutive lanes (positions) read consecutive pairs
-            const float2* cs = reinterpret_cast<const float2*>(e.rope) + tpos;
+            // cos / sin of frequency i at this row's position from its turns table
+            const float tf = (float)tpos;
             float ss = 0.f;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-              const float2 w = cs[(long long)i * e.T];
+              float wc, ws;
+              rope_cos_sin(tf, sturns[i], wc, ws);
               const float x1 = v[i], x2 = v[i + 64];
-              v[i] = x1 * w.x + x2 * w.y;
-              v[i + 64] = -x1 * w.y + x2 * w.x;
+              v[i] = x1 * wc + x2 * ws;
+              v[i + 64] = -x1 * ws + x2 * wc;
               ss += v[i] * v[i] + v[i + 64] * v[i + 64];
             }
             if (e.qk_norm) {

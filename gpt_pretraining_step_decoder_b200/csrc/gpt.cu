@@ -576,7 +576,7 @@ struct Plan {
   size_t logits, dz, ce_stats, ce_ztgt, tok_loss, ce_scale, ce_count, loss_scratch;
   size_t sort_keys_a, sort_keys_b, sort_vals_a, sort_vals_b, sort_counts, part_head, part_tail;
   size_t splitk; long long splitk_elems;
-  size_t norm_part, clip_coef, grad_norm, rope_cs, rope_cs_t, err;
+  size_t norm_part, clip_coef, grad_norm, rope_cs, rope_turns, err;
   // Muon (matrix_optimizer == GPT_MATRIX_MUON): the block matrices in three
   // same-shape groups and one scratch sized for the largest group
   MuonGroup muon_groups[3];
@@ -733,7 +733,7 @@ static void make_plan(const gpt_config& c, Plan& p) {
   p.clip_coef = cv.take(4);
   p.grad_norm = cv.take(4);
   p.rope_cs = cv.take((long long)c.seq_len * c.head_dim * 4);
-  p.rope_cs_t = cv.take((long long)c.seq_len * c.head_dim * 4);
+  p.rope_turns = cv.take((long long)c.head_dim / 2 * 8);
   p.err = cv.take(16);
   if (c.matrix_optimizer == GPT_MATRIX_MUON) {
     // groups: [q, k, v, proj] x layers ([a, d] each; a == d), w1 [F, d] x layers, w2 [d, F] x layers
@@ -890,7 +890,7 @@ extern "C" int gpt_create(const gpt_config* cfg, unsigned long long seed, void* 
     }
   }
   ++g_launches; rope_table_kernel<<<grid_for((long long)c.seq_len * c.head_dim / 2, 256), 256, 0, m->st>>>(
-      m->at<float>(p.rope_cs), m->at<float>(p.rope_cs_t), c.seq_len, c.head_dim, (double)c.rope_base);
+      m->at<float>(p.rope_cs), m->at<float2>(p.rope_turns), c.seq_len, c.head_dim, (double)c.rope_base);
   e = cudaGetLastError();
   if (e != cudaSuccess) { delete m; return fail(GPT_ERR_CUDA, "init launch: %s", cudaGetErrorString(e)); }
   int s = refresh_lp(m);
@@ -1282,7 +1282,7 @@ static int forward_impl(gpt_model* m, const int32_t* tokens, const int32_t* targ
     if (b16) {
       // QKV projection with RoPE + QK-norm (+ value-table row) in its epilogue
       GemmEpilogue eq = epi(EPI_QKV, qkv, 3 * a);
-      eq.rope = m->at<float>(p.rope_cs_t);
+      eq.rope = m->at<float2>(p.rope_turns);
       eq.rstd_q = m->at<float>(L.rstd_q);
       eq.rstd_k = m->at<float>(L.rstd_k);
       eq.hv = vbias;

@@ -143,20 +143,22 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __
 // in two layouts: position-major cs[t][j] (one warp per position reads a
 // contiguous row) and frequency-major cs_t[j][t] (a warp over 32 consecutive
 // positions reads contiguous pairs, as the QKV GEMM epilogue does).
-__global__ void rope_table_kernel(float* __restrict__ cs, float* __restrict__ cs_t, int T, int hd, double base) {
+__global__ void rope_table_kernel(float* __restrict__ cs, float2* __restrict__ turns, int T, int hd, double base) {
   const int h = hd / 2;
   const long long total = (long long)T * h;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int t = (int)(i / h), j = (int)(i % h);
     const double inv_freq = 1.0 / pow(base, (2.0 * j) / hd);
+    if (t == 0) {
+      // turns per position of frequency j, as an unevaluated fp32 sum hi + lo
+      const double u = inv_freq / 6.283185307179586476925287;
+      const float hi = (float)u;
+      turns[j] = make_float2(hi, (float)(u - (double)hi));
+    }
     const double th = t * inv_freq;
-    const float c = (float)cos(th), s = (float)sin(th);
-    cs[2 * i] = c;
-    cs[2 * i + 1] = s;
-    const long long it = (long long)j * T + t;
-    cs_t[2 * it] = c;
-    cs_t[2 * it + 1] = s;
+    cs[2 * i] = (float)cos(th);
+    cs[2 * i + 1] = (float)sin(th);
   }
 }
 
