@@ -1156,8 +1156,15 @@ static int attention_bwd(gpt_model* m, const act_t* qkv, const act_t* o, const a
   const long long N = (long long)c.micro_batch * c.seq_len;
   ProfScope ps(&m->prof, m->st, "attention_bwd",
                5.0 * c.micro_batch * c.n_head * (double)c.seq_len * c.seq_len * c.head_dim, 0.0);
-  ++g_launches; launch_pdl(attn_bwd_pre_kernel<act_t>, grid_for(N * c.n_head * 32, 256), 256, 0, m->st,
-      o, dout, Dv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
+  if (std::is_same<act_t, bf16>::value && c.head_dim == 128) {
+    const long long warps = cdiv_ll(N * c.n_head, ATTN_PRE_ROWS);
+    ++g_launches; launch_pdl(attn_bwd_pre_hd128_kernel, grid_for(warps * 32, 256), 256, 0, m->st,
+        reinterpret_cast<const bf16*>(o), reinterpret_cast<const bf16*>(dout), Dv, c.micro_batch, c.seq_len,
+        c.n_head);
+  } else {
+    ++g_launches; launch_pdl(attn_bwd_pre_kernel<act_t>, grid_for(N * c.n_head * 32, 256), 256, 0, m->st,
+        o, dout, Dv, c.micro_batch, c.seq_len, c.n_head, c.head_dim);
+  }
   LAUNCH_CHECK();
   if (std::is_same<act_t, bf16>::value) {
     static bool attr = false;

@@ -568,6 +568,50 @@ __global__ void attn_fwd_simt_kernel(const act_t* __restrict__ qkv, act_t* __res
   if (lane == 0) lse_out[(long long)bh * T + i] = lse;
 }
 
+// D[bh, i] = sum_c dO[i, c] * O[i, c] for bf16 heads of 128: a warp takes
+// ROWS (position, head) rows, two at a time (16 lanes a row, 16 bytes of each
+// operand a lane), with all of its loads requested before any is used.
+constexpr int ATTN_PRE_ROWS = 8;
+__global__ void __launch_bounds__(256) attn_bwd_pre_hd128_kernel(const bf16* __restrict__ o,
+                                                                 const bf16* __restrict__ dout,
+                                                                 float* __restrict__ Dout, int B, int T, int H) {
+  pdl_wait();     // the previous kernel in the stream has completed (programmatic launch)
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31, half = lane >> 4, ch = lane & 15;
+  const long long rows = (long long)B * T * H, r0 = warp * ATTN_PRE_ROWS;
+  if (r0 >= rows) return;  // whole warp
+  uint4 ro[ATTN_PRE_ROWS / 2], rd[ATTN_PRE_ROWS / 2];
+#pragma unroll
+  for (int k = 0; k < ATTN_PRE_ROWS / 2; ++k) {
+    const long long r = r0 + 2 * k + half;   // row = n * H + h, 128 contiguous values
+    ro[k] = make_uint4(0u, 0u, 0u, 0u);
+    rd[k] = ro[k];
+    if (r < rows) {
+      ro[k] = *reinterpret_cast<const uint4*>(o + r * 128 + 8 * ch);
+      rd[k] = *reinterpret_cast<const uint4*>(dout + r * 128 + 8 * ch);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < ATTN_PRE_ROWS / 2; ++k) {
+    const uint32_t wo[4] = {ro[k].x, ro[k].y, ro[k].z, ro[k].w}, wd[4] = {rd[k].x, rd[k].y, rd[k].z, rd[k].w};
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wo[q]));
+      const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[q]));
+      s = fmaf(a.x, d.x, fmaf(a.y, d.y, s));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    const long long r = r0 + 2 * k + half;
+    if (ch == 0 && r < rows) {
+      const long long n = r / H;
+      const int h = (int)(r % H), b = (int)(n / T), t = (int)(n % T);
+      Dout[((long long)b * H + h) * T + t] = s;
+    }
+  }
+}
+
 // D[bh, i] = sum_c dO[i, c] * O[i, c]  (softmax-backward row term)
 template <typename act_t>
 __global__ void attn_bwd_pre_kernel(const act_t* __restrict__ o, const act_t* __restrict__ dout,
