@@ -287,8 +287,11 @@ static int gemm_tc_launch(int M, int N, int K, GemmOperand A, GemmOperand B, Gem
   p.m_tiles = cdiv(M, CG * tc::BM);
   p.n_tiles = cdiv(N, BN);
   // n-fastest order while the whole B operand stays in L2; grouped m-blocks
-  // when B is large (the LM head's vocab-sized operand)
-  p.group_m = (double)N * K * 2 > 32.0 * (1 << 20) ? (p.m_tiles < 16 ? p.m_tiles : 16) : 1;
+  // when B is large (the LM head's vocab-sized operand): all of them when A
+  // itself fits in L2 (the logits of a row chunk: each vocab tile is read
+  // from HBM once, A from L2), else groups of 16
+  const bool big_b = (double)N * K * 2 > 32.0 * (1 << 20), small_a = (double)M * K * 2 <= 32.0 * (1 << 20);
+  p.group_m = big_b ? (small_a || p.m_tiles < 16 ? p.m_tiles : 16) : 1;
   p.kb_total = cdiv(K, tc::BK);
   if (splits < 1) splits = 1;
   if (splits > p.kb_total) splits = p.kb_total;
