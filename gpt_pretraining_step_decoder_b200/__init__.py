@@ -84,6 +84,7 @@ _SIGS = {
     "ngram_sparse_update_noalloc": [_P, _P, _LL, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P],
     "gptx_gemm_bf16": [_I, _I, _I, _P, _LL, _I, _P, _LL, _I, _I, _P, _LL, _P, _I, _I, _P, _SZ, _P],
     "gptx_set_gemm_cta_pairs": [_I],
+    "gptx_wait_probe": [_I, _P],
     "fp8_quantize_workspace_bytes": [ctypes.POINTER(_SZ)],
     "fp8_quantize": [_P, _I, _LL, _P, _P, _P, _SZ, _P],
     "gptx_gemm_fp8": [_I, _I, _I, _P, _LL, _P, _LL, _P, _P, _I, _P, _LL, _P],
@@ -329,6 +330,12 @@ def gptx_gemm_fp8(M, N, K, A, lda, B, ldb, scale_a, scale_b, out_dtype, C, ldc, 
 def gptx_set_gemm_cta_pairs(on):
     """Run later GEMMs with N >= 256 on SM pairs (True, the default) or one SM per tile."""
     return _check(_lib.gptx_set_gemm_cta_pairs(int(bool(on))), "gptx_set_gemm_cta_pairs")
+
+
+def gptx_wait_probe(limit_us, stream=None):
+    """Enqueue one bounded wait that nothing satisfies; it gives up after
+    limit_us and the next ngram_sync_status(stream) reports GPT_ERR_TIMEOUT."""
+    return _check(_lib.gptx_wait_probe(int(limit_us), _stream(stream)), "gptx_wait_probe")
 
 
 # ------------------------------------------------------------------ convenience

@@ -1858,6 +1858,35 @@ extern "C" int ngram_sync_status(void* stream) {
 }
 
 // ======================================================================== kernel-level test entry
+// One thread waits, with the kernels' bounded-wait loop, on an mbarrier that
+// nothing arrives on; when the limit passes it records a timeout and returns.
+__global__ void wait_probe_kernel(unsigned long long limit_ns, unsigned* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!tc::mbar_try_wait(&bar, 0)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_error(err, GPT_EBIT_TIMEOUT);
+      return;
+    }
+  }
+}
+
+extern "C" int gptx_wait_probe(int limit_us, void* stream) {
+  const long long us = limit_us < 1 ? 1 : (limit_us > 2000000 ? 2000000 : limit_us);
+  unsigned* err = nullptr;
+  CUDA_TRY(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_ngram_err));
+  ++g_launches;
+  wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)us * 1000ull, err);
+  LAUNCH_CHECK();
+  return GPT_OK;
+}
+
 extern "C" int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmajor, const void* B,
                               long long ldb, int b_kmajor, int mode, void* C, long long ldc, const void* aux,
                               int beta, int splits, void* workspace, size_t ws_bytes, void* stream) {

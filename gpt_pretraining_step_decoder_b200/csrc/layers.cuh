@@ -425,7 +425,34 @@ __global__ void __launch_bounds__(256) ce_prob_kernel(bf16* __restrict__ ez, con
   }
   __syncthreads();
   const float sc = (y >= 0) ? *scale_dev : 0.f;
-  for (int i = threadIdx.x * 8; i < V; i += blockDim.x * 8) {
+  const int stride = blockDim.x * 8;
+  int i0 = threadIdx.x * 8;
+  if (softcap <= 0.f && (V & 7) == 0) {
+    // four 16-byte pieces per thread in flight: every load of the group is
+    // requested before any of its stores (the buffer is rewritten in place)
+    for (; i0 + 3 * stride + 8 <= V; i0 += 4 * stride) {
+      uint4 raw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) raw[u] = *reinterpret_cast<const uint4*>(g + i0 + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * stride;
+        const float f = fac[i / tile_cols];
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+        uint4 out;
+        __nv_bfloat162* ho = reinterpret_cast<__nv_bfloat162*>(&out);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 t = __bfloat1622float2(h[k]);
+          const float o0 = (t.x * f - (i + 2 * k == y ? 1.f : 0.f)) * sc;
+          const float o1 = (t.y * f - (i + 2 * k + 1 == y ? 1.f : 0.f)) * sc;
+          ho[k] = __floats2bfloat162_rn(o0, o1);
+        }
+        *reinterpret_cast<uint4*>(g + i) = out;
+      }
+    }
+  }
+  for (int i = i0; i < V; i += stride) {
     // 8 columns never straddle a block (tile_cols is a multiple of 8)
     const int j = i / tile_cols;
     const float f = fac[j];

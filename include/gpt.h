@@ -488,6 +488,17 @@ int gptx_gemm_bf16(int M, int N, int K, const void* A, long long lda, int a_kmaj
  * enqueued at the same time.
  */
 int gptx_set_gemm_cta_pairs(int on);
+
+/*
+ * Check of the bounded-wait path (diagnostic): enqueues on `stream` one
+ * thread that waits on a shared-memory mbarrier nothing ever arrives on,
+ * exactly as the kernels' bounded waits do, gives up after limit_us
+ * microseconds (clamped to [1, 2,000,000]), sets the timeout bit of the
+ * standalone error word and returns.  The next ngram_sync_status(stream)
+ * reports GPT_ERR_TIMEOUT; the context stays usable.  GPT_ERR_CUDA if the
+ * launch fails.
+ */
+int gptx_wait_probe(int limit_us, void* stream);
 #ifdef __cplusplus
 }
 #endif
