@@ -140,9 +140,9 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ du, const act_t* __
 // ("$1000 tier nanochat run", `_precompute_rotary_embeddings`), evaluated in
 // double precision and stored fp32 (the pages keep a bf16 table).
 // (cos, sin) of t * base^(-2j/hd) for every position t and frequency j < hd/2,
-// in two layouts: position-major cs[t][j] (one warp per position reads a
-// contiguous row) and frequency-major cs_t[j][t] (a warp over 32 consecutive
-// positions reads contiguous pairs, as the QKV GEMM epilogue does).
+// position-major cs[t][j] (one warp per position reads a contiguous row), and
+// for the QKV GEMM epilogue, which computes each row's cos / sin itself, the
+// frequencies' turns per position base^(-2j/hd) / (2 pi) as fp32 hi + lo.
 __global__ void rope_table_kernel(float* __restrict__ cs, float2* __restrict__ turns, int T, int hd, double base) {
   const int h = hd / 2;
   const long long total = (long long)T * h;
